@@ -1,0 +1,170 @@
+"""fp64 CPU oracle of the Muir gated delta rule -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` leg of
+``bench.py`` may import this package.  The CUDA library never calls it, and
+nothing here imports the CUDA library: the two share no code.
+
+Two independent C sources are wrapped:
+
+* ``muir_ref.c`` -- the token-by-token recurrence of "Muir: Linear Attention
+  with Sensitivity-Allocated Gating and Matched-Filter Readout" (arXiv
+  2611.08376; wolonglab.org page, "Methodology", eq:gdn2 and eq:ours), its
+  back-propagation through time, and the single-token decode step.
+* ``muir_chunk_ref.c`` -- the chunked (WY / UT) form of the same recurrence,
+  derived by unrolling it over a chunk (same page, "Methodology": each chunk is
+  a triangular system), with exact exponent differences.
+
+Every function takes numpy-convertible arrays, computes in float64 and returns
+float64 numpy arrays.  Per-token tensors are ``[B, T, H, d]``; states are
+``[B, H, dk, dv]``.
+
+Pins (what fixes these functions other than themselves) live in
+``tests/test_oracle_pins.py``: linear-attention and gated-linear-attention
+closed forms, the delta rule (Widrow-Hoff), an exact-retrieval invariant,
+pure decay, chunk-size invariance, linearity, column equivariance, state
+passing, decode/recurrence equivalence, a hand-computed example in
+``tests/golden/``, central finite differences and torch autograd for the
+gradients.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "liboracle.so")
+_SOURCES = ["muir_ref.c", "muir_chunk_ref.c"]
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile the C oracle into ``oracle/liboracle.so`` (gcc, -O2, no fast-math)."""
+    srcs = [os.path.join(_HERE, s) for s in _SOURCES]
+    if not force and os.path.exists(_LIB_PATH):
+        newest = max(os.path.getmtime(s) for s in srcs)
+        if os.path.getmtime(_LIB_PATH) >= newest:
+            return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-fno-fast-math", "-ffp-contract=off", "-fPIC", "-shared",
+           "-pthread", "-o", tmp] + srcs + ["-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        build()
+        lib = ctypes.CDLL(_LIB_PATH)
+        P = ctypes.c_void_p
+        I = ctypes.c_int
+        lib.muir_ref_fwd.argtypes = [I] * 5 + [P] * 10 + [I]
+        lib.muir_ref_bwd.argtypes = [I] * 5 + [P] * 18 + [I, I]
+        lib.muir_ref_step.argtypes = [I] * 4 + [P] * 7 + [I, P, P]
+        lib.muir_chunk_ref_fwd.argtypes = [I] * 6 + [P] * 11 + [I]
+        for f in (lib.muir_ref_fwd, lib.muir_ref_bwd, lib.muir_ref_step,
+                  lib.muir_chunk_ref_fwd):
+            f.restype = I
+        _lib = lib
+    return _lib
+
+
+def default_threads() -> int:
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+def _f64(x):
+    if x is None:
+        return None
+    if hasattr(x, "detach"):  # torch tensor
+        x = x.detach().cpu().double().numpy()
+    return np.ascontiguousarray(np.asarray(x, dtype=np.float64))
+
+
+def _p(x):
+    return None if x is None else x.ctypes.data_as(ctypes.c_void_p)
+
+
+def _dims(q, v):
+    B, T, H, dk = q.shape
+    dv = v.shape[3]
+    return B, T, H, dk, dv
+
+
+def fwd(q, k, v, g, e, w, gamma=None, S0=None, threads=None):
+    """Token-by-token forward.  Returns ``(o [B,T,H,dv], S_T [B,H,dk,dv])``."""
+    lib = _load()
+    q, k, v, g, e, w, gamma, S0 = map(_f64, (q, k, v, g, e, w, gamma, S0))
+    B, T, H, dk, dv = _dims(q, v)
+    o = np.zeros((B, T, H, dv))
+    S = np.zeros((B, H, dk, dv))
+    rc = lib.muir_ref_fwd(B, T, H, dk, dv, _p(q), _p(k), _p(v), _p(g), _p(e), _p(w),
+                          _p(gamma), _p(S0), _p(o), _p(S), threads or default_threads())
+    if rc:
+        raise ValueError("muir_ref_fwd: bad shape")
+    return o, S
+
+
+def bwd(q, k, v, g, e, w, gamma=None, S0=None, dO=None, dS_final=None, ckpt=64,
+        threads=None):
+    """Back-propagation through time of ``sum(o*dO) + sum(S_T*dS_final)``.
+
+    Returns a dict with ``dq, dk, dv, dg, de, dw, dgamma`` ([B,T,H,d]) and
+    ``dS0`` ([B,H,dk,dv]).
+    """
+    lib = _load()
+    q, k, v, g, e, w, gamma, S0, dO, dS_final = map(
+        _f64, (q, k, v, g, e, w, gamma, S0, dO, dS_final))
+    B, T, H, dk, dv = _dims(q, v)
+    if dO is None:
+        dO = np.zeros((B, T, H, dv))
+    out = {n: np.zeros((B, T, H, dk)) for n in ("dq", "dk", "dg", "de", "dgamma")}
+    out.update({n: np.zeros((B, T, H, dv)) for n in ("dv", "dw")})
+    out["dS0"] = np.zeros((B, H, dk, dv))
+    rc = lib.muir_ref_bwd(B, T, H, dk, dv, _p(q), _p(k), _p(v), _p(g), _p(e), _p(w),
+                          _p(gamma), _p(S0), _p(dO), _p(dS_final), _p(out["dq"]),
+                          _p(out["dk"]), _p(out["dv"]), _p(out["dg"]), _p(out["de"]),
+                          _p(out["dw"]), _p(out["dgamma"]), _p(out["dS0"]), int(ckpt),
+                          threads or default_threads())
+    if rc:
+        raise ValueError("muir_ref_bwd: bad shape")
+    return out
+
+
+def chunk_fwd(q, k, v, g, e, w, gamma=None, S0=None, chunk=64, threads=None):
+    """Chunked (WY form) forward.  Returns ``(o, S_T, S_chunks)`` where
+    ``S_chunks[b, h, n]`` is the state at the start of chunk ``n``."""
+    lib = _load()
+    q, k, v, g, e, w, gamma, S0 = map(_f64, (q, k, v, g, e, w, gamma, S0))
+    B, T, H, dk, dv = _dims(q, v)
+    n = (T + chunk - 1) // chunk
+    o = np.zeros((B, T, H, dv))
+    S = np.zeros((B, H, dk, dv))
+    Sc = np.zeros((B, H, n, dk, dv))
+    rc = lib.muir_chunk_ref_fwd(B, T, H, dk, dv, int(chunk), _p(q), _p(k), _p(v), _p(g),
+                                _p(e), _p(w), _p(gamma), _p(S0), _p(o), _p(S), _p(Sc),
+                                threads or default_threads())
+    if rc:
+        raise ValueError("muir_chunk_ref_fwd: bad shape")
+    return o, S, Sc
+
+
+def step(q, k, v, g, e, w, gamma, S, gamma_static=False):
+    """One decode token for every (b, h).  Per-token inputs are ``[B, H, d]``;
+    ``gamma`` is ``[B, H, dk]``, or ``[H, dk]`` with ``gamma_static=True``, or
+    None.  Returns ``(o [B,H,dv], S_new)``; the input ``S`` is not modified."""
+    lib = _load()
+    q, k, v, g, e, w, gamma = map(_f64, (q, k, v, g, e, w, gamma))
+    S = _f64(S).copy()
+    B, H, dk = q.shape
+    dv = v.shape[2]
+    o = np.zeros((B, H, dv))
+    rc = lib.muir_ref_step(B, H, dk, dv, _p(q), _p(k), _p(v), _p(g), _p(e), _p(w),
+                           _p(gamma), int(bool(gamma_static)), _p(S), _p(o))
+    if rc:
+        raise ValueError("muir_ref_step: bad shape")
+    return o, S
