@@ -1,0 +1,211 @@
+"""Python binding of libmuir, the Muir gated delta rule on one NVIDIA B200.
+
+Argument marshalling only: every step of the computation runs in the CUDA
+kernels of ``libmuir.so`` (built in-tree by ``gated_delta_rule_115_b200.build``)
+behind the C ABI declared in ``include/muir.h``.  PyTorch supplies device
+memory and the current CUDA stream.  There is no CPU fallback: if the library
+is missing or a call fails, an exception is raised.
+
+Recurrence (arXiv 2611.08376, wolonglab.org page, "Methodology", eq:gdn2 and
+eq:ours), per batch and head, state S in R^{dk x dv} with rows = key channels:
+
+    S_t = diag(exp g_t) S_{t-1} - (e_t*k_t)(k_t^T diag(exp g_t) S_{t-1}) + k_t (w_t*v_t)^T
+    o_t = S_t^T (gamma_t * q_t)
+
+Per-token tensors are ``[B, T, H, d]``; states ``[B, H, dk, dv]`` float32.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "MuirError", "lib", "chunk_fwd", "chunk_bwd", "recurrent_step", "fwd_workspace_bytes",
+    "bwd_workspace_bytes", "MuirChunkFunction", "LIB_PATH",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmuir.so")
+
+MUIR_BF16, MUIR_FP32 = 0, 1
+_STATUS = {0: "MUIR_OK", 1: "MUIR_ERR_INVALID_ARG", 2: "MUIR_ERR_UNSUPPORTED",
+           3: "MUIR_ERR_WORKSPACE", 4: "MUIR_ERR_CUDA", 5: "MUIR_ERR_DEVICE_TIMEOUT"}
+
+
+class MuirError(RuntimeError):
+    def __init__(self, fn: str, code: int):
+        self.code = code
+        msg = _lib.muir_status_string(code).decode() if _lib is not None else _STATUS.get(code)
+        super().__init__(f"{fn} failed: {msg}")
+
+
+class MuirShape(ctypes.Structure):
+    _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
+                ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("chunk", ctypes.c_int),
+                ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int)]
+
+
+_lib = None
+
+
+def lib():
+    """The loaded ``libmuir.so`` (ctypes).  Raises if it has not been built."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise ImportError(f"{LIB_PATH} is missing: run `python -m gated_delta_rule_115_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
+        SP = ctypes.POINTER(MuirShape)
+        L.muir_status_string.argtypes = [I]
+        L.muir_status_string.restype = ctypes.c_char_p
+        L.muir_chunk_fwd_workspace.argtypes = [SP]
+        L.muir_chunk_fwd_workspace.restype = S
+        L.muir_chunk_bwd_workspace.argtypes = [SP]
+        L.muir_chunk_bwd_workspace.restype = S
+        L.muir_chunk_fwd.argtypes = [SP] + [P] * 12 + [S, P]
+        L.muir_chunk_fwd.restype = I
+        L.muir_chunk_bwd.argtypes = [SP] + [P] * 20 + [S, P]
+        L.muir_chunk_bwd.restype = I
+        L.muir_recurrent_step.argtypes = [I, I, I, I, I, I] + [P] * 7 + [I, P, P, P]
+        L.muir_recurrent_step.restype = I
+        _lib = L
+    return _lib
+
+
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.bfloat16:
+        return MUIR_BF16
+    if t.dtype == torch.float32:
+        return MUIR_FP32
+    raise TypeError(f"unsupported dtype {t.dtype} (bfloat16 or float32)")
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("libmuir takes CUDA tensors only")
+    if not t.is_contiguous():
+        raise ValueError("libmuir takes contiguous tensors")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(dev):
+    return ctypes.c_void_p(torch.cuda.current_stream(dev).cuda_stream)
+
+
+def _check(fn, rc):
+    if rc != 0:
+        raise MuirError(fn, rc)
+
+
+def _shape(q, v, chunk, out_dtype):
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    od = _dt(q) if out_dtype is None else (MUIR_BF16 if out_dtype == torch.bfloat16 else MUIR_FP32)
+    return MuirShape(B, T, H, dk, dv, chunk, _dt(q), od)
+
+
+def fwd_workspace_bytes(B, T, H, d, chunk, dtype=torch.bfloat16) -> int:
+    s = MuirShape(B, T, H, d, d, chunk, MUIR_BF16 if dtype == torch.bfloat16 else MUIR_FP32, 0)
+    return int(lib().muir_chunk_fwd_workspace(ctypes.byref(s)))
+
+
+def bwd_workspace_bytes(B, T, H, d, chunk, dtype=torch.bfloat16) -> int:
+    s = MuirShape(B, T, H, d, d, chunk, MUIR_BF16 if dtype == torch.bfloat16 else MUIR_FP32, 0)
+    return int(lib().muir_chunk_bwd_workspace(ctypes.byref(s)))
+
+
+def _workspace(nbytes, dev, ws):
+    if nbytes == 0:
+        return None
+    if ws is not None and ws.numel() >= nbytes:
+        return ws
+    return torch.empty(nbytes, dtype=torch.uint8, device=dev)
+
+
+def chunk_fwd(q, k, v, g, e, w, gamma, S0=None, chunk=64, out_dtype=None,
+              return_chunk_states=False, ws=None):
+    """Chunkwise forward.  Returns ``(o, S_final)`` or, with
+    ``return_chunk_states``, ``(o, S_final, S_chunks)`` where ``S_chunks[b,h,n]``
+    is the state at the start of chunk ``n`` (reusable by :func:`chunk_bwd`)."""
+    L = lib()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    shp = _shape(q, v, chunk, out_dtype)
+    od = torch.bfloat16 if shp.out_dtype == MUIR_BF16 else torch.float32
+    o = torch.empty(B, T, H, dv, dtype=od, device=q.device)
+    S_final = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    Sc = (torch.empty(B, H, T // chunk, dk, dv, dtype=torch.float32, device=q.device)
+          if return_chunk_states else None)
+    need = int(L.muir_chunk_fwd_workspace(ctypes.byref(shp)))
+    wsb = _workspace(need, q.device, ws)
+    rc = L.muir_chunk_fwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(e),
+                          _ptr(w), _ptr(gamma), _ptr(S0), _ptr(o), _ptr(S_final), _ptr(Sc),
+                          _ptr(wsb), ctypes.c_size_t(0 if wsb is None else wsb.numel()),
+                          _stream(q.device))
+    _check("muir_chunk_fwd", rc)
+    return (o, S_final, Sc) if return_chunk_states else (o, S_final)
+
+
+def chunk_bwd(q, k, v, g, e, w, gamma, S0, dO, dS_final=None, chunk=64, S_chunks=None,
+              ws=None):
+    """Gradients of ``sum(o*dO) + sum(S_final*dS_final)``.  Returns a dict with
+    ``dq, dk, dv, dg, de, dw, dgamma`` (input dtype) and ``dS0`` (float32)."""
+    L = lib()
+    shp = _shape(q, v, chunk, None)
+    grads = {n: torch.empty_like(x) for n, x in
+             dict(dq=q, dk=k, dv=v, dg=g, de=e, dw=w, dgamma=gamma).items()}
+    B, T, H, dk = q.shape
+    grads["dS0"] = torch.empty(B, H, dk, v.shape[-1], dtype=torch.float32, device=q.device)
+    need = int(L.muir_chunk_bwd_workspace(ctypes.byref(shp)))
+    wsb = _workspace(need, q.device, ws)
+    rc = L.muir_chunk_bwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(e),
+                          _ptr(w), _ptr(gamma), _ptr(S0), _ptr(S_chunks), _ptr(dO),
+                          _ptr(dS_final), _ptr(grads["dq"]), _ptr(grads["dk"]),
+                          _ptr(grads["dv"]), _ptr(grads["dg"]), _ptr(grads["de"]),
+                          _ptr(grads["dw"]), _ptr(grads["dgamma"]), _ptr(grads["dS0"]),
+                          _ptr(wsb), ctypes.c_size_t(0 if wsb is None else wsb.numel()),
+                          _stream(q.device))
+    _check("muir_chunk_bwd", rc)
+    return grads
+
+
+def recurrent_step(q, k, v, g, e, w, gamma, S, gamma_static=False, out_dtype=None, o=None):
+    """One decode token for every (b, h); ``S`` ([B,H,dk,dv] float32) is
+    updated in place.  ``gamma`` is ``[B,H,dk]``, ``[H,dk]`` with
+    ``gamma_static=True``, or None.  Returns ``o`` ([B,H,dv])."""
+    L = lib()
+    B, H, dk = q.shape
+    dv = v.shape[-1]
+    od = q.dtype if out_dtype is None else out_dtype
+    if o is None:
+        o = torch.empty(B, H, dv, dtype=od, device=q.device)
+    rc = L.muir_recurrent_step(B, H, dk, dv, _dt(q), _dt(o), _ptr(q), _ptr(k), _ptr(v),
+                               _ptr(g), _ptr(e), _ptr(w), _ptr(gamma), int(bool(gamma_static)),
+                               _ptr(S), _ptr(o), _stream(q.device))
+    _check("muir_recurrent_step", rc)
+    return o
+
+
+class MuirChunkFunction(torch.autograd.Function):
+    """Autograd wrapper: forward saves the chunk states, backward reuses them."""
+
+    @staticmethod
+    def forward(ctx, q, k, v, g, e, w, gamma, S0, chunk):
+        o, S_final, Sc = chunk_fwd(q, k, v, g, e, w, gamma, S0, chunk=chunk,
+                                   return_chunk_states=True)
+        ctx.save_for_backward(q, k, v, g, e, w, gamma, S0, Sc)
+        ctx.chunk = chunk
+        return o, S_final
+
+    @staticmethod
+    def backward(ctx, dO, dS_final):
+        q, k, v, g, e, w, gamma, S0, Sc = ctx.saved_tensors
+        gr = chunk_bwd(q, k, v, g, e, w, gamma, S0, dO.contiguous().to(q.dtype),
+                       None if dS_final is None else dS_final.contiguous().float(),
+                       chunk=ctx.chunk, S_chunks=Sc)
+        return (gr["dq"], gr["dk"], gr["dv"], gr["dg"], gr["de"], gr["dw"], gr["dgamma"],
+                gr["dS0"] if S0 is not None else None, None)

@@ -1,0 +1,145 @@
+// api.cu -- the extern "C" entry points of libmuir: host-side argument checks,
+// workspace sizing and dispatch to the CUDA kernels.  Nothing here computes.
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/muir.h"
+#include "kernels.h"
+
+namespace {
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
+bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
+bool ok_dtype(muir_dtype d) { return d == MUIR_BF16 || d == MUIR_FP32; }
+
+// The kernels use sm_100a instructions: require compute capability 10.x.
+muir_status check_device() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return MUIR_ERR_CUDA;
+    int major = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return MUIR_ERR_CUDA;
+    return major == 10 ? MUIR_OK : MUIR_ERR_UNSUPPORTED;
+}
+
+// Shape checks shared by the chunk entry points (no CUDA calls).
+muir_status check_shape(const muir_shape* s) {
+    if (!s) return MUIR_ERR_INVALID_ARG;
+    if (s->B <= 0 || s->T <= 0 || s->H <= 0 || s->dk <= 0 || s->dv <= 0 || s->chunk <= 0)
+        return MUIR_ERR_INVALID_ARG;
+    if (!ok_dtype(s->in_dtype) || !ok_dtype(s->out_dtype)) return MUIR_ERR_INVALID_ARG;
+    if (s->dk != s->dv || (s->dk != 64 && s->dk != 128)) return MUIR_ERR_UNSUPPORTED;
+    const int C = s->chunk;
+    if (C != 16 && C != 32 && C != 64 && C != 128 && C != 256) return MUIR_ERR_UNSUPPORTED;
+    if (s->T % C != 0) return MUIR_ERR_UNSUPPORTED;
+    // index arithmetic inside the kernels is 64-bit for tensors; keep counts in int range
+    if ((long long)s->B * s->H * (s->T / C) > (1LL << 30)) return MUIR_ERR_UNSUPPORTED;
+    return MUIR_OK;
+}
+
+muir::ChunkProblem make_problem(const muir_shape* s, const void* q, const void* k,
+                                const void* v, const void* g, const void* e, const void* w,
+                                const void* gamma) {
+    muir::ChunkProblem P;
+    P.B = s->B; P.T = s->T; P.H = s->H; P.D = s->dk; P.C = s->chunk; P.N = s->T / s->chunk;
+    P.in_bf16 = s->in_dtype == MUIR_BF16;
+    P.out_bf16 = s->out_dtype == MUIR_BF16;
+    P.q = q; P.k = k; P.v = v; P.g = g; P.e = e; P.w = w; P.gamma = gamma;
+    return P;
+}
+
+muir_status from_cuda(cudaError_t err) {
+    if (err == cudaSuccess) return MUIR_OK;
+    if (err == cudaErrorNotSupported) return MUIR_ERR_UNSUPPORTED;
+    return MUIR_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* muir_status_string(muir_status s) {
+    switch (s) {
+        case MUIR_OK: return "MUIR_OK";
+        case MUIR_ERR_INVALID_ARG: return "MUIR_ERR_INVALID_ARG: null, misaligned or out-of-range argument";
+        case MUIR_ERR_UNSUPPORTED: return "MUIR_ERR_UNSUPPORTED: shape, chunk, tail or device not supported";
+        case MUIR_ERR_WORKSPACE: return "MUIR_ERR_WORKSPACE: workspace missing or too small";
+        case MUIR_ERR_CUDA: return "MUIR_ERR_CUDA: a CUDA runtime call or kernel launch failed";
+        case MUIR_ERR_DEVICE_TIMEOUT: return "MUIR_ERR_DEVICE_TIMEOUT: a bounded device wait expired";
+    }
+    return "MUIR_ERR_UNKNOWN";
+}
+
+size_t muir_chunk_fwd_workspace(const muir_shape* s) {
+    if (check_shape(s) != MUIR_OK) return 0;
+    return muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false);
+}
+
+size_t muir_chunk_bwd_workspace(const muir_shape* s) {
+    if (check_shape(s) != MUIR_OK) return 0;
+    return muir::chunk_bwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false);
+}
+
+muir_status muir_chunk_fwd(const muir_shape* s, const void* q, const void* k, const void* v,
+                           const void* g, const void* e, const void* w, const void* gamma,
+                           const float* S0, void* o, float* S_final, float* S_chunks, void* ws,
+                           size_t ws_bytes, void* stream) {
+    muir_status st = check_shape(s);
+    if (st != MUIR_OK) return st;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
+        !ok_ptr(gamma) || !ok_ptr(o) || !ok_opt(S0) || !ok_opt(S_final) || !ok_opt(S_chunks))
+        return MUIR_ERR_INVALID_ARG;
+    const size_t need = muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk,
+                                                 S_chunks != nullptr);
+    if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
+    if ((st = check_device()) != MUIR_OK) return st;
+    muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);
+    return from_cuda(muir::run_chunk_fwd(P, S0, o, S_final, S_chunks, ws, ws_bytes,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+muir_status muir_chunk_bwd(const muir_shape* s, const void* q, const void* k, const void* v,
+                           const void* g, const void* e, const void* w, const void* gamma,
+                           const float* S0, const float* S_chunks, const void* dO,
+                           const float* dS_final, void* dq, void* dk, void* dv, void* dg,
+                           void* de, void* dw, void* dgamma, float* dS0, void* ws,
+                           size_t ws_bytes, void* stream) {
+    muir_status st = check_shape(s);
+    if (st != MUIR_OK) return st;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
+        !ok_ptr(gamma) || !ok_ptr(dO) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) ||
+        !ok_ptr(dg) || !ok_ptr(de) || !ok_ptr(dw) || !ok_ptr(dgamma) || !ok_opt(S0) ||
+        !ok_opt(S_chunks) || !ok_opt(dS_final) || !ok_opt(dS0))
+        return MUIR_ERR_INVALID_ARG;
+    const size_t need = muir::chunk_bwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk,
+                                                 S_chunks != nullptr);
+    if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
+    if ((st = check_device()) != MUIR_OK) return st;
+    muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);
+    return from_cuda(muir::run_chunk_bwd(P, S0, S_chunks, dO, dS_final, dq, dk, dv, dg, de, dw,
+                                         dgamma, dS0, ws, ws_bytes,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+muir_status muir_recurrent_step(int B, int H, int dk, int dv, muir_dtype dtype,
+                                muir_dtype out_dtype, const void* q, const void* k,
+                                const void* v, const void* g, const void* e, const void* w,
+                                const void* gamma, int gamma_static, float* S, void* o,
+                                void* stream) {
+    if (B <= 0 || H <= 0 || dk <= 0 || dv <= 0) return MUIR_ERR_INVALID_ARG;
+    if (!ok_dtype(dtype) || !ok_dtype(out_dtype)) return MUIR_ERR_INVALID_ARG;
+    if (gamma_static != 0 && gamma_static != 1) return MUIR_ERR_INVALID_ARG;
+    if (dk != dv || (dk != 64 && dk != 128)) return MUIR_ERR_UNSUPPORTED;
+    if ((long long)B * H > (1LL << 30)) return MUIR_ERR_UNSUPPORTED;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
+        !ok_opt(gamma) || !ok_ptr(S) || !ok_ptr(o))
+        return MUIR_ERR_INVALID_ARG;
+    muir_status st = check_device();
+    if (st != MUIR_OK) return st;
+    return from_cuda(muir::launch_decode(B, H, dk, dtype == MUIR_BF16, out_dtype == MUIR_BF16,
+                                         q, k, v, g, e, w, gamma, gamma_static, S, o,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+}  // extern "C"

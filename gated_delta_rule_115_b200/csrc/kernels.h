@@ -1,0 +1,33 @@
+// kernels.h -- internal launchers of libmuir (not part of the C ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace muir {
+
+cudaError_t launch_decode(int B, int H, int D, bool in_bf16, bool out_bf16, const void* q,
+                          const void* k, const void* v, const void* g, const void* e,
+                          const void* w, const void* gamma, int gamma_static, float* S,
+                          void* o, cudaStream_t st);
+
+// Problem description shared by the chunk kernels.
+struct ChunkProblem {
+    int B, T, H, D, C;     // D = dk = dv
+    int N;                 // chunks per sequence, T / C
+    bool in_bf16, out_bf16;
+    const void *q, *k, *v, *g, *e, *w, *gamma;
+};
+
+// Workspace carving (bytes) for the chunk forward / backward.
+size_t chunk_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states);
+size_t chunk_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states);
+
+cudaError_t run_chunk_fwd(const ChunkProblem& P, const float* S0, void* o, float* S_final,
+                          float* S_chunks, void* ws, size_t ws_bytes, cudaStream_t st);
+cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S_chunks,
+                          const void* dO, const float* dS_final, void* dq, void* dk, void* dv,
+                          void* dg, void* de, void* dw, void* dgamma, float* dS0, void* ws,
+                          size_t ws_bytes, cudaStream_t st);
+
+}  // namespace muir

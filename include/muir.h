@@ -1,0 +1,136 @@
+/*
+ * muir.h -- C ABI of libmuir: the Muir gated delta rule on one NVIDIA B200.
+ *
+ * The operation (per batch b and head h, state S in R^{dk x dv}, rows = key
+ * channels) is the recurrence of "Muir: Linear Attention with
+ * Sensitivity-Allocated Gating and Matched-Filter Readout" (arXiv 2611.08376),
+ * wolonglab.org page, section "Methodology", eq:gdn2 and eq:ours:
+ *
+ *     S_t = D_t S_{t-1} - (e_t * k_t) (k_t^T D_t S_{t-1}) + k_t (w_t * v_t)^T
+ *     o_t = S_t^T (gamma_t * q_t),                  D_t = diag(exp(g_t))
+ *
+ * g is the log decay (caller applies any -softplus; precondition g <= 0), e the
+ * erase gate, w the write gate, gamma the readout (matched-filter) gate; q and k
+ * are expected to be unit-normalised by the caller.  No 1/sqrt(dk) scale and no
+ * output gate are applied here.
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Pointers named q, k, v, g, e, w, gamma, o, dO and the gradient outputs are
+ *   DEVICE pointers.  Per-token tensors are token-major [B][T][H][d]
+ *   (contiguous, d fastest); decode tensors are [B][H][d].  States are float32
+ *   [B][H][dk][dv], row-major.  The caller owns all memory; the library never
+ *   allocates or frees device memory: scratch comes from the caller's
+ *   workspace (ws, ws_bytes), whose size the *_workspace() queries return.
+ * - Every pointer must be 16-byte aligned.
+ * - stream is a cudaStream_t (NULL = legacy default stream).  All work is
+ *   enqueued asynchronously on it; no call synchronises the host.
+ * - Argument checks run on the host before anything is enqueued; a failed
+ *   check returns MUIR_ERR_INVALID_ARG or MUIR_ERR_UNSUPPORTED and enqueues
+ *   nothing.  A launch failure returns MUIR_ERR_CUDA.
+ * - Supported: dk == dv in {64, 128}; chunk in {16, 32, 64, 128, 256};
+ *   T % chunk == 0 (a ragged tail returns MUIR_ERR_UNSUPPORTED); a device of
+ *   compute capability 10.x.  Inside the kernels g is clamped at -20 per
+ *   token (exp(-20) ~ 2e-9; a row decayed that hard is already erased).
+ * - dtype MUIR_BF16 means bfloat16 inputs; MUIR_FP32 means float32 inputs.
+ *   Internal arithmetic is float32 with tensor-core TF32 products (three TF32
+ *   passes for float32 inputs).  out_dtype selects o's storage.
+ */
+#ifndef MUIR_H_
+#define MUIR_H_
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    MUIR_OK = 0,
+    MUIR_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size */
+    MUIR_ERR_UNSUPPORTED = 2,   /* valid but not implemented (head dim, chunk, tail, device) */
+    MUIR_ERR_WORKSPACE = 3,     /* ws too small or NULL with ws_bytes > 0 */
+    MUIR_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
+    MUIR_ERR_DEVICE_TIMEOUT = 5 /* a bounded device-side wait expired */
+} muir_status;
+
+typedef enum { MUIR_BF16 = 0, MUIR_FP32 = 1 } muir_dtype;
+
+typedef struct {
+    int B, T, H;           /* batch, tokens, heads */
+    int dk, dv;            /* key / value head dims (must be equal) */
+    int chunk;             /* chunk size C of the chunkwise algorithm */
+    muir_dtype in_dtype;   /* dtype of q, k, v, g, e, w, gamma, dO and of the input grads */
+    muir_dtype out_dtype;  /* dtype of o */
+} muir_shape;
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* muir_status_string(muir_status s);
+
+/* Bytes of device workspace muir_chunk_fwd / muir_chunk_bwd need for this
+ * shape (0 for an invalid shape).  Host-only; enqueues nothing. */
+size_t muir_chunk_fwd_workspace(const muir_shape* shape);
+size_t muir_chunk_bwd_workspace(const muir_shape* shape);
+
+/*
+ * Chunkwise-parallel forward.  Same page, "Methodology": each chunk of C
+ * tokens is written as a unit-lower-triangular system (WY/UT form); the
+ * cumulative log decay is split at block boundaries so every exponential
+ * applied to an operand is <= 1 ("boundary-pivoted", fig:kernel); chunk
+ * states are propagated by a sequential pass with the float32 state on chip.
+ *
+ *   q, k, g, e, gamma : [B][T][H][dk]   in_dtype
+ *   v, w              : [B][T][H][dv]   in_dtype
+ *   S0                : [B][H][dk][dv]  float32, NULL = zero initial state
+ *   o                 : [B][T][H][dv]   out_dtype (written)
+ *   S_final           : [B][H][dk][dv]  float32, may be NULL (written)
+ *   S_chunks          : [B][H][T/C][dk][dv] float32, may be NULL; receives the
+ *                       state at the start of every chunk, which
+ *                       muir_chunk_bwd can reuse instead of recomputing it.
+ */
+muir_status muir_chunk_fwd(const muir_shape* shape, const void* q, const void* k,
+                           const void* v, const void* g, const void* e, const void* w,
+                           const void* gamma, const float* S0, void* o, float* S_final,
+                           float* S_chunks, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * Backward of muir_chunk_fwd ("custom backward pass", same page,
+ * "Methodology"): gradients of L = sum(o * dO) + sum(S_final * dS_final).
+ *
+ *   inputs as for muir_chunk_fwd; dO [B][T][H][dv] in_dtype;
+ *   dS_final [B][H][dk][dv] float32 or NULL (= 0);
+ *   S_chunks: NULL (recompute the chunk states) or the array a previous
+ *             muir_chunk_fwd with the same inputs wrote;
+ *   dq, dk, dg, de, dgamma [B][T][H][dk] and dv, dw [B][T][H][dv] are written
+ *   in in_dtype; dS0 [B][H][dk][dv] float32 may be NULL.
+ */
+muir_status muir_chunk_bwd(const muir_shape* shape, const void* q, const void* k,
+                           const void* v, const void* g, const void* e, const void* w,
+                           const void* gamma, const float* S0, const float* S_chunks,
+                           const void* dO, const float* dS_final, void* dq, void* dk,
+                           void* dv, void* dg, void* de, void* dw, void* dgamma,
+                           float* dS0, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * One decode token for every (b, h) against a resident float32 state (same
+ * page, "Experiments": streaming inference with a constant-size float32 state;
+ * fig:longctx_niah: static or dynamic readout gain).
+ *
+ *   q, k, g, e : [B][H][dk]   dtype;    v, w : [B][H][dv]   dtype
+ *   gamma      : [B][H][dk] (gamma_static == 0), [H][dk] shared by every b
+ *                (gamma_static == 1), or NULL (gamma = 1)
+ *   S          : [B][H][dk][dv] float32, updated in place
+ *   o          : [B][H][dv] out_dtype
+ * Bandwidth bound: S is read and written once.  No workspace.
+ */
+muir_status muir_recurrent_step(int B, int H, int dk, int dv, muir_dtype dtype,
+                                muir_dtype out_dtype, const void* q, const void* k,
+                                const void* v, const void* g, const void* e, const void* w,
+                                const void* gamma, int gamma_static, float* S, void* o,
+                                void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MUIR_H_ */

@@ -1,0 +1,111 @@
+"""Host-side checks of the C ABI (no GPU needed).
+
+The library must load, export every function ``include/muir.h`` declares, and
+reject bad arguments with the documented status codes before touching CUDA.
+"""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from gated_delta_rule_115_b200 import build
+    build.build()
+    import gated_delta_rule_115_b200 as m
+    return m.lib()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "muir.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(muir_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = header_functions()
+    assert {"muir_chunk_fwd", "muir_chunk_bwd", "muir_recurrent_step"} <= set(names)
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_status_strings(L):
+    for code in range(6):
+        s = L.muir_status_string(code).decode()
+        assert s.startswith("MUIR_")
+    assert L.muir_status_string(99).decode() == "MUIR_ERR_UNKNOWN"
+
+
+def _shape(m, **kw):
+    d = dict(B=1, T=256, H=2, dk=64, dv=64, chunk=64, in_dtype=0, out_dtype=1)
+    d.update(kw)
+    return m.MuirShape(**d)
+
+
+FAKE = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced: checks fail first
+
+
+def _fwd(L, shp, **over):
+    args = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, e=FAKE, w=FAKE, gamma=FAKE, S0=None, o=FAKE,
+                S_final=None, S_chunks=None, ws=None, ws_bytes=0)
+    args.update(over)
+    return L.muir_chunk_fwd(ctypes.byref(shp), args["q"], args["k"], args["v"], args["g"],
+                            args["e"], args["w"], args["gamma"], args["S0"], args["o"],
+                            args["S_final"], args["S_chunks"], args["ws"],
+                            ctypes.c_size_t(args["ws_bytes"]), None)
+
+
+def test_chunk_fwd_rejects_bad_arguments(L):
+    import gated_delta_rule_115_b200 as m
+    assert _fwd(L, _shape(m, dk=96, dv=96)) == 2            # head dim
+    assert _fwd(L, _shape(m, dk=64, dv=128)) == 2           # dk != dv
+    assert _fwd(L, _shape(m, chunk=48)) == 2                # chunk size
+    assert _fwd(L, _shape(m, T=250)) == 2                   # ragged tail
+    assert _fwd(L, _shape(m, B=0)) == 1
+    assert _fwd(L, _shape(m, in_dtype=7)) == 1
+    assert _fwd(L, _shape(m), q=None) == 1                  # null input
+    assert _fwd(L, _shape(m), o=ctypes.c_void_p(0x10004)) == 1  # misaligned output
+    assert L.muir_chunk_fwd(None, *([FAKE] * 12), ctypes.c_size_t(0), None) == 1
+
+
+def test_chunk_workspace_query(L):
+    import gated_delta_rule_115_b200 as m
+    assert L.muir_chunk_fwd_workspace(ctypes.byref(_shape(m, chunk=48))) == 0
+    assert L.muir_chunk_bwd_workspace(ctypes.byref(_shape(m, T=100))) == 0
+    need = L.muir_chunk_fwd_workspace(ctypes.byref(_shape(m)))
+    if need > 0:
+        assert _fwd(L, _shape(m), ws=FAKE, ws_bytes=need - 1) == 3
+        assert _fwd(L, _shape(m), ws=None, ws_bytes=need) == 3
+
+
+def test_chunk_bwd_rejects_bad_arguments(L):
+    import gated_delta_rule_115_b200 as m
+    shp = _shape(m, dk=32, dv=32)
+    args = [FAKE] * 7 + [None, None, FAKE, None] + [FAKE] * 7 + [None, None]
+    assert L.muir_chunk_bwd(ctypes.byref(shp), *args, ctypes.c_size_t(0), None) == 2
+    shp = _shape(m)
+    args2 = list(args)
+    args2[10] = ctypes.c_void_p(0x10008)  # misaligned dS_final
+    assert L.muir_chunk_bwd(ctypes.byref(shp), *args2, ctypes.c_size_t(0), None) == 1
+
+
+def test_recurrent_step_rejects_bad_arguments(L):
+    P = [FAKE] * 6
+    assert L.muir_recurrent_step(0, 16, 128, 128, 0, 1, *P, None, 0, FAKE, FAKE, None) == 1
+    assert L.muir_recurrent_step(2, 16, 96, 96, 0, 1, *P, None, 0, FAKE, FAKE, None) == 2
+    assert L.muir_recurrent_step(2, 16, 128, 128, 0, 1, *P, None, 2, FAKE, FAKE, None) == 1
+    assert L.muir_recurrent_step(2, 16, 128, 128, 0, 1, *P, None, 0, None, FAKE, None) == 1
+    assert L.muir_recurrent_step(2, 16, 128, 128, 3, 1, *P, None, 0, FAKE, FAKE, None) == 1
+
+
+def test_binding_refuses_cpu_tensors(L):
+    import torch
+    import gated_delta_rule_115_b200 as m
+    x = torch.zeros(1, 2, 64)
+    with pytest.raises(ValueError):
+        m.recurrent_step(x, x, x, x, x, x, None, torch.zeros(1, 2, 64, 64), out_dtype=torch.float32,
+                         o=torch.zeros(1, 2, 64))
