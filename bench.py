@@ -1,0 +1,509 @@
+#!/usr/bin/env python
+"""Benchmark of the Muir chunkwise gated delta rule on B200 GPUs.
+
+One step = the whole hot path over one batch of the long-context workload
+(B=1, H=16, T=32768, dk=dv=128, chunk 128, bf16 inputs): ``muir_chunk_fwd``
+(saving chunk states) followed by ``muir_chunk_bwd`` with a random upstream
+gradient.  The streaming-decode step (B=64, H=16, d=128, float32 state) is
+measured in the same run and reported under ``"decode"``.
+
+Usage::
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl muir|reference]
+
+N > 1 runs one process per GPU (launched by torch.distributed.run); every rank
+processes its own batch (weak scaling, no data-path collective); the time is
+the max over ranks.  ``--impl reference`` times the fp64 CPU oracle on a
+bounded sample of the same workload (rank 0 only).  Prints ONE JSON line.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+WID = 2
+METRIC = "Muir chunk fwd+bwd tokens/s & % bf16 TC peak (H=16,d=128,T=32K); decode GB/s"
+NAMES = ["q", "k", "v", "g", "e", "w", "gamma"]
+
+# Nominal dense tensor-core ratios (TF32 : BF16 = 1.1 : 2.25 PFLOP/s per GPU).
+TF32_OVER_BF16 = 1.1 / 2.25
+
+
+def flops_fwd_per_token_head(C: int, d: int) -> float:
+    """Algorithmic forward FLOPs per token and head (2 per multiply-add,
+    triangular products counted at half size): 9Cd + C^2/3 + 8d^2."""
+    return 9 * C * d + C * C / 3 + 8 * d * d
+
+
+# Algorithmic HBM bytes per token and head (bf16 I/O, one pass, nothing saved):
+BYTES_FWD = 7 * 256 + 256            # 7 inputs read, o written
+BYTES_BWD = 8 * 256 + 7 * 256        # 7 inputs + dO read, 7 gradients written
+DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 6 * 128 * 2 + 128 * 2  # S read+write, tokens, o
+
+# DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
+# keyed by kernel; valid only while the kernel source hash matches.
+NCU_TRAFFIC = {
+    # profiles/k_bwd_B1_H16_T8192_d128_C128.md: 8.492 GB for 131,072 token-heads
+    "k_bwd": {"bytes_per_token_head": 8.492118e9 / 131072, "source": "db35a5a6a35fddcb"},
+}
+
+
+def source_hash() -> str:
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(os.path.join(ROOT, "gated_delta_rule_115_b200", "csrc"))):
+        with open(os.path.join(ROOT, "gated_delta_rule_115_b200", "csrc", f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def parse_args(argv=None):
+    p = argparse.ArgumentParser(description=__doc__.split("\n")[0])
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=20)
+    p.add_argument("--warmup", type=int, default=3)
+    p.add_argument("--impl", choices=["muir", "reference"], default="muir")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0,
+                   help="target CPU time of the oracle sample")
+    p.add_argument("--T", type=int, default=None,
+                   help="shorter sequence for profiling captures (not a bench number)")
+    a = p.parse_args(argv)
+    if a.warmup < 3:
+        p.error("--warmup must be >= 3")
+    if a.steps < 1:
+        p.error("--steps must be >= 1")
+    return a
+
+
+def dist_env():
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", str(rank)))
+    return rank, world, local
+
+
+def max_over_ranks(value: float, world: int, device=None) -> float:
+    """Max of a float over all ranks (identity when world == 1)."""
+    if world == 1:
+        return value
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def rank_seed(rank: int) -> int:
+    """Seed of this rank's batch: rank 0 draws the canonical workload."""
+    return 1000 + WID + 7919 * rank
+
+
+# ------------------------------------------------------------------ clocks
+
+CLOCK_FIELDS = ["clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+                "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+                "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+
+class ClockSampler:
+    """nvidia-smi sampling every 200 ms while the timed region runs."""
+
+    def __init__(self, gpu_id: str):
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        cmd = ["nvidia-smi", "--query-gpu=" + ",".join(CLOCK_FIELDS), "--format=csv,noheader,nounits",
+               "-lms", "200"]
+        if gpu_id:
+            cmd += ["-i", gpu_id]
+        try:
+            self.p = subprocess.Popen(cmd, stdout=self.f, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.p = None
+
+    def stop(self) -> dict:
+        if self.p is not None:
+            self.p.terminate()
+            try:
+                self.p.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.p.kill()
+        self.f.flush()
+        self.f.seek(0)
+        rows = [r.strip().split(",") for r in self.f.read().strip().splitlines() if r.strip()]
+        self.f.close()
+        os.unlink(self.f.name)
+        return summarize_clocks(rows)
+
+
+def summarize_clocks(rows) -> dict:
+    sm, mx, reasons = [], [], set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for r in rows:
+        r = [x.strip() for x in r]
+        if len(r) < 8:
+            continue
+        try:
+            sm.append(float(r[0]))
+            mx.append(float(r[1]))
+        except ValueError:
+            continue
+        for n, v in zip(names, r[4:8]):
+            if v.lower() == "active":
+                reasons.add(n)
+    if not sm:
+        return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+    return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(mx), "reasons": sorted(reasons),
+            "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle arm
+
+def oracle_tokens(T_s: int, threads: int) -> float:
+    """Seconds the fp64 oracle (token-loop forward + BPTT backward) takes on
+    all 16 heads of the first T_s tokens of the workload."""
+    import oracle
+    from gated_delta_rule_115_b200 import inputs as I
+    oracle.build()
+    x = I.chunk_inputs(WID, T=T_s)
+    t0 = time.perf_counter()
+    oracle.fwd(*[x[n] for n in NAMES], S0=x["S0"], threads=threads)
+    oracle.bwd(*[x[n] for n in NAMES], S0=x["S0"], dO=x["dO"], ckpt=128, threads=threads)
+    return time.perf_counter() - t0
+
+
+def oracle_sample_size(seconds: float, threads: int) -> int:
+    """Tokens T_s (multiple of 128, <= 32768) whose oracle run takes about `seconds`."""
+    t_cal = oracle_tokens(128, threads)
+    return int(max(128, min(32768, 128 * seconds / max(t_cal, 1e-3))) // 128 * 128)
+
+
+def sample_desc(T_s: int) -> str:
+    return f"fwd+bwd of B=1, all H=16 heads, first T={T_s} tokens of the workload (tokens/s = T_s / seconds)"
+
+
+def oracle_sample(seconds: float, threads: int):
+    T_s = oracle_sample_size(seconds, threads)
+    dt = oracle_tokens(T_s, threads)
+    return T_s / dt, sample_desc(T_s), dt
+
+
+def reference_arm(args, rank, world):
+    """The oracle as the reference arm: each step is one bounded sample of the
+    workload, sized so that warm-up plus timed steps take about two minutes."""
+    if rank != 0:
+        return None
+    threads = len(os.sched_getaffinity(0))
+    per = max(0.5, 120.0 / (args.steps + args.warmup))
+    T_s = oracle_sample_size(per, threads)
+    times = []
+    for i in range(args.warmup + args.steps):
+        dt = oracle_tokens(T_s, threads)
+        if i >= args.warmup:
+            times.append(dt)
+    dt = statistics.median(times)
+    value = T_s / dt
+    return {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup, "ms_per_step": dt * 1e3,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic", "config": workload_config(),
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": sample_desc(T_s)},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def workload_config(T=32768):
+    return {"workload": f"long-context chunkwise fwd+bwd, B=1 H=16 T={T} dk=dv=128 chunk=128",
+            "B": 1, "H": 16, "T": T, "d": 128, "chunk": 128, "io_dtype": "bf16",
+            "l2": "per-step inputs (0.94 GB) and outputs exceed the 126 MB L2; no extra flush"}
+
+
+# ------------------------------------------------------------------ GPU arm
+
+def gpu_arm(args, rank, world, local):
+    import torch
+    import gated_delta_rule_115_b200 as muir
+    from gated_delta_rule_115_b200 import inputs as I
+    from gated_delta_rule_115_b200 import build as B
+    B.build()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    L = muir.lib()
+    W = I.WORKLOADS[WID]
+    if args.T is not None:
+        import dataclasses
+        W = dataclasses.replace(W, T=args.T)
+    x = I.chunk_inputs(WID, seed=rank_seed(rank), T=W.T)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in x.items()}
+    C = W.chunk
+    args_in = [d[n] for n in NAMES]
+
+    def step():
+        o, S, Sc = muir.chunk_fwd(*args_in, d["S0"], chunk=C, return_chunk_states=True, ws=ws_f)
+        gr = muir.chunk_bwd(*args_in, d["S0"], d["dO"], chunk=C, S_chunks=Sc, ws=ws_b)
+        return o, gr
+
+    ws_f = torch.empty(muir.fwd_workspace_bytes(W.B, W.T, W.H, W.dk, C), dtype=torch.uint8, device=dev)
+    ws_b = torch.empty(muir.bwd_workspace_bytes(W.B, W.T, W.H, W.dk, C), dtype=torch.uint8, device=dev)
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    gpu_id = ""
+    try:
+        gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
+    except Exception:
+        pass
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(gpu_id)
+    L.muir_profile_reset()
+    L.muir_profile_enable(1)
+    st = torch.cuda.current_stream(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(args.steps):
+        step()
+    e1.record(st)
+    torch.cuda.synchronize()
+    L.muir_profile_enable(0)
+    L.muir_profile_collect()
+    clocks = sampler.stop()
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
+    ms = ms_total / args.steps
+    prof = {L.muir_profile_name(i).decode(): (L.muir_profile_total_ms(i), L.muir_profile_launches(i))
+            for i in range(L.muir_profile_count())}
+    launches = sum(n for _, n in prof.values())
+    tokens = W.B * W.T * world
+    value = tokens / (ms / 1e3)
+    token_heads = W.B * W.T * W.H
+    fl = 3 * flops_fwd_per_token_head(C, W.dk) * token_heads * world
+    tflops = fl / (ms / 1e3) / 1e12
+
+    peaks = load_peaks()
+    # dominant kernel
+    dom = max(prof.items(), key=lambda kv: kv[1][0])
+    dom_name, (dom_ms, dom_n) = dom
+    dom_avg = dom_ms / max(dom_n, 1)
+    roof = kernel_roofline(dom_name, dom_avg, token_heads, C, W.dk, peaks)
+
+    out = {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "tf32",
+        "data": "synthetic", "config": workload_config(W.T),
+        "tflops": tflops, "tc_peak_frac": tflops / peaks["bf16_tflops"],
+        "hbm_gbs_algorithmic": (BYTES_FWD + BYTES_BWD) * token_heads * world / (ms / 1e3) / 1e9,
+        "roofline": roof,
+        "kernels_ms_per_step": {k: v[0] / args.steps for k, v in sorted(prof.items())},
+        "gpu_launches": launches,
+        "clocks": clocks,
+        "source": source_hash(),
+    }
+    if not args.no_e2e:
+        out["e2e"] = e2e_measure(muir, x, W, C, dev, ws_f, ws_b, max(1, min(args.steps, 3)), world)
+    if not args.no_decode:
+        out["decode"] = decode_measure(muir, I, dev, peaks)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        threads = len(os.sched_getaffinity(0))
+        v, desc, dt = oracle_sample(args.cpu_seconds, threads)
+        out["cpu_baseline"] = {"value": v, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                               "sample": desc, "seconds": dt}
+    return out
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return {"hbm_gbs": j["hbm_gbs"], "bf16_tflops": j["bf16_tflops"],
+                "bf16_tflops_sustained": j.get("bf16_tflops_sustained", j["bf16_tflops"]),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+def kernel_roofline(name, avg_ms, token_heads, C, d, peaks):
+    """Roofline of one launch of the dominant kernel from its algorithmic work."""
+    F = flops_fwd_per_token_head(C, d)
+    work = {  # (algorithmic bytes, algorithmic flops) per token-head
+        "k_bwd": (BYTES_BWD, 2 * F),
+        "k_out": (BYTES_FWD, F),
+        "k_intra": (5 * 256, F),
+        "k_bprep": (6 * 256, F),
+        "k_chain": (2 * d * d * 4 / C, 2 * d * d * d / C),
+        "k_chain_rev": (2 * d * d * 4 / C, 2 * d * d * d / C),
+    }.get(name, (BYTES_FWD, F))
+    byts = work[0] * token_heads
+    fl = work[1] * token_heads
+    gbs = byts / (avg_ms / 1e3) / 1e9
+    tfl = fl / (avg_ms / 1e3) / 1e12
+    tf32_peak = peaks["bf16_tflops_sustained"] * TF32_OVER_BF16
+    f_hbm, f_tc = gbs / peaks["hbm_gbs"], tfl / tf32_peak
+    traffic = None
+    t = NCU_TRAFFIC.get(name)
+    if t and t.get("source") == source_hash():
+        traffic = t["bytes_per_token_head"] * token_heads
+    if f_hbm >= f_tc:
+        r = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": f_hbm}
+    else:
+        r = {"bound": "tensor", "achieved": tfl, "peak": tf32_peak, "unit": "TFLOP/s", "frac": f_tc}
+    r.update({"traffic": traffic, "kernel": name, "avg_launch_ms": avg_ms,
+              "peak_source": peaks["source"] + (" (tf32 = sustained bf16 x 1.1/2.25)" if r["bound"] == "tensor" else ""),
+              "other_bound_frac": f_tc if r["bound"] == "hbm" else f_hbm})
+    return r
+
+
+def e2e_measure(muir, x, W, C, dev, ws_f, ws_b, steps, world):
+    """The same step through the public API with host buffers: per step, copy
+    the inputs from pinned host memory, run forward + backward, copy o and all
+    gradients back to pinned host memory."""
+    import torch
+    host = {k: v.pin_memory() for k, v in x.items() if v is not None}
+    dev_in = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    outs_host = None
+    st = torch.cuda.current_stream(dev)
+    h2d = sum(v.numel() * v.element_size() for v in host.values())
+    d2h = 0
+
+    def one():
+        nonlocal outs_host, d2h
+        for k, v in host.items():
+            dev_in[k].copy_(v, non_blocking=True)
+        a = [dev_in[n] for n in NAMES]
+        o, S, Sc = muir.chunk_fwd(*a, dev_in.get("S0"), chunk=C, return_chunk_states=True, ws=ws_f)
+        gr = muir.chunk_bwd(*a, dev_in.get("S0"), dev_in["dO"], chunk=C, S_chunks=Sc, ws=ws_b)
+        res = [o, S] + [gr[k] for k in sorted(gr)]
+        if outs_host is None:
+            outs_host = [torch.empty_like(r, device="cpu").pin_memory() for r in res]
+            d2h = sum(r.numel() * r.element_size() for r in res)
+        for hbuf, r in zip(outs_host, res):
+            hbuf.copy_(r, non_blocking=True)
+
+    one()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(st)
+    for _ in range(steps):
+        one()
+    e1.record(st)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(e0.elapsed_time(e1) / steps, world, dev)
+    return {"value": W.B * W.T * world / (ms / 1e3), "unit": "tokens/s", "ms_per_step": ms,
+            "steps": steps, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+
+
+def decode_measure(muir, I, dev, peaks, steps=50):
+    """Decode step (B=64, H=16, d=128, float32 state, static gamma): each timed
+    step is bracketed by CUDA events with a 256 MB L2 flush in between, so the
+    state really comes from HBM.  Also reports CUDA-graph replay of 1,000
+    back-to-back steps (state resident in L2)."""
+    import torch
+    W = I.WORKLOADS[4]
+    S0, gstat = I.decode_state()
+    S = S0.to(dev)
+    tok = {k: v.to(dev) for k, v in I.decode_tokens(0).items()}
+    gam = gstat.to(dev)
+    o = torch.empty(W.B, W.H, W.dv, dtype=torch.bfloat16, device=dev)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream(dev)
+
+    def one():
+        muir.recurrent_step(tok["q"], tok["k"], tok["v"], tok["g"], tok["e"], tok["w"], gam, S,
+                            gamma_static=True, o=o)
+
+    for _ in range(5):
+        one()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        one()
+        b.record(st)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    ms = statistics.median(times)
+    byts = DECODE_BYTES_PER_HEAD * W.B * W.H
+    gbs = byts / (ms / 1e3) / 1e9
+    # graph replay, L2 resident
+    g = torch.cuda.CUDAGraph()
+    s2 = torch.cuda.Stream(dev)
+    s2.wait_stream(st)
+    with torch.cuda.stream(s2):
+        one()
+        torch.cuda.synchronize()
+        with torch.cuda.graph(g, stream=s2):
+            for _ in range(100):
+                one()
+    st.wait_stream(s2)
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(10):
+        g.replay()
+    b.record(st)
+    torch.cuda.synchronize()
+    ms_g = a.elapsed_time(b) / 1000
+    return {
+        "workload": "decode step B=64 H=16 d=128, fp32 state, bf16 tokens, static gamma",
+        "ms_per_step_l2_flushed": ms, "gbs_l2_flushed": gbs,
+        "hbm_frac": gbs / peaks["hbm_gbs"], "tokens_per_s": W.B / (ms / 1e3),
+        "bytes_per_step": byts,
+        "graph_replay_ms_per_step": ms_g, "graph_replay_gbs_l2_resident": byts / (ms_g / 1e3) / 1e9,
+        "note": "graph replay keeps the 64 MiB state in L2; the flushed number is the HBM one",
+    }
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    rank, world, local = dist_env()
+    if world != args.gpus:
+        print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
+    if args.impl == "reference":
+        out = reference_arm(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                device_id=torch.device("cuda", local))
+    try:
+        out = gpu_arm(args, rank, world, local)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -70,6 +70,20 @@ def lib():
         L.muir_chunk_bwd.restype = I
         L.muir_recurrent_step.argtypes = [I, I, I, I, I, I] + [P] * 7 + [I, P, P, P]
         L.muir_recurrent_step.restype = I
+        L.muir_profile_enable.argtypes = [I]
+        L.muir_profile_enable.restype = None
+        L.muir_profile_reset.argtypes = []
+        L.muir_profile_reset.restype = None
+        L.muir_profile_collect.argtypes = []
+        L.muir_profile_collect.restype = I
+        L.muir_profile_count.argtypes = []
+        L.muir_profile_count.restype = I
+        L.muir_profile_name.argtypes = [I]
+        L.muir_profile_name.restype = ctypes.c_char_p
+        L.muir_profile_total_ms.argtypes = [I]
+        L.muir_profile_total_ms.restype = ctypes.c_double
+        L.muir_profile_launches.argtypes = [I]
+        L.muir_profile_launches.restype = ctypes.c_longlong
         _lib = L
     return _lib
 

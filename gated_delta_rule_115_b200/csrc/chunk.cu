@@ -42,6 +42,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "mma.cuh"
+#include "profile.h"
 
 namespace muir {
 
@@ -855,10 +856,10 @@ static cudaError_t launch_chain(int BH, int N, const float* M, const float* Bn, 
     // column slabs: enough CTAs to cover the GPU when B*H is small
     if (BH >= 64) {
         constexpr int SL = 32;
-        k_chain<D, SL, PASSES, REV><<<BH * (D / SL), kThreads, 0, st>>>(M, Bn, S_in, S_rec, S_out, N);
+        MUIR_TIMED(REV ? "k_chain_rev" : "k_chain", st, k_chain<D, SL, PASSES, REV><<<BH * (D / SL), kThreads, 0, st>>>(M, Bn, S_in, S_rec, S_out, N));
     } else {
         constexpr int SL = 16;
-        k_chain<D, SL, PASSES, REV><<<BH * (D / SL), kThreads, 0, st>>>(M, Bn, S_in, S_rec, S_out, N);
+        MUIR_TIMED(REV ? "k_chain_rev" : "k_chain", st, k_chain<D, SL, PASSES, REV><<<BH * (D / SL), kThreads, 0, st>>>(M, Bn, S_in, S_rec, S_out, N));
     }
     return cudaGetLastError();
 }
@@ -881,15 +882,15 @@ static cudaError_t fwd_impl(const ChunkProblem& P, const float* S0, void* o, flo
     kp.S_chunks = Sc;
     kp.o = o;
     const int grid = num_slots(nch);
-    k_intra<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp);
+    MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, S_final, st);
     if (err != cudaSuccess) return err;
     if (P.out_bf16)
-        k_out<Tin, __nv_bfloat16, D, PASSES><<<grid, kThreads, 0, st>>>(kp);
+        MUIR_TIMED("k_out", st, k_out<Tin, __nv_bfloat16, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
     else
-        k_out<Tin, float, D, PASSES><<<grid, kThreads, 0, st>>>(kp);
+        MUIR_TIMED("k_out", st, k_out<Tin, float, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
     return cudaGetLastError();
 }
 
@@ -917,18 +918,18 @@ static cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float*
     kp.dS_chunks = dSc;
     kp.dq = dq; kp.dk = dk; kp.dv = dv; kp.dg = dg; kp.de = de; kp.dw = dw; kp.dgamma = dgamma;
     const int grid = num_slots(nch);
-    k_intra<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp);
+    MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
     cudaError_t err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (recompute) {
         err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, nullptr, st);
         if (err != cudaSuccess) return err;
     }
-    k_bprep<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp);
+    MUIR_TIMED("k_bprep", st, k_bprep<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     err = launch_chain<D, PASSES, true>(BH, P.N, kp.M, kp.Bn, dS_final, dSc, dS0, st);
     if (err != cudaSuccess) return err;
-    k_bwd<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp);
+    MUIR_TIMED("k_bwd", st, k_bwd<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
     return cudaGetLastError();
 }
 

@@ -16,6 +16,7 @@
 // go through a small shared-memory table.
 #include "common.cuh"
 #include "kernels.h"
+#include "profile.h"
 
 namespace muir {
 
@@ -107,9 +108,9 @@ static cudaError_t launch_decode_t(int B, int H, int D, const void* q, const voi
     (const Tin*)q, (const Tin*)k, (const Tin*)v, (const Tin*)g, (const Tin*)e,          \
         (const Tin*)w, (const Tin*)gamma, gamma_static, S, (Tout*)o, H
     if (D == 128)
-        decode_step_kernel<Tin, Tout, 128><<<grid, block, 0, st>>>(MUIR_DEC_ARGS);
+        MUIR_TIMED("k_decode", st, decode_step_kernel<Tin, Tout, 128><<<grid, block, 0, st>>>(MUIR_DEC_ARGS));
     else
-        decode_step_kernel<Tin, Tout, 64><<<grid, block, 0, st>>>(MUIR_DEC_ARGS);
+        MUIR_TIMED("k_decode", st, decode_step_kernel<Tin, Tout, 64><<<grid, block, 0, st>>>(MUIR_DEC_ARGS));
 #undef MUIR_DEC_ARGS
     return cudaGetLastError();
 }

@@ -21,9 +21,13 @@ def L():
 
 
 def header_functions():
-    src = open(os.path.join(ROOT, "include", "muir.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(muir_[a-z_0-9]+)\s*\(", src)))
+    names = set()
+    inc = os.path.join(ROOT, "include")
+    for f in sorted(os.listdir(inc)):
+        if f.endswith(".h"):
+            src = re.sub(r"/\*.*?\*/", "", open(os.path.join(inc, f)).read(), flags=re.S)
+            names |= set(re.findall(r"\b(muir_[a-z_0-9]+)\s*\(", src))
+    return sorted(names)
 
 
 def test_exports_every_declared_symbol(L):
@@ -31,6 +35,16 @@ def test_exports_every_declared_symbol(L):
     assert {"muir_chunk_fwd", "muir_chunk_bwd", "muir_recurrent_step"} <= set(names)
     for n in names:
         assert hasattr(L, n), n
+    assert "muir_profile_collect" in names
+
+
+def test_profile_hook_without_launches(L):
+    L.muir_profile_reset()
+    L.muir_profile_enable(1)
+    L.muir_profile_enable(0)
+    assert L.muir_profile_collect() == 0
+    assert L.muir_profile_count() == 0
+    assert L.muir_profile_name(0) is None
 
 
 def test_status_strings(L):
