@@ -70,6 +70,8 @@ def lib():
         L.muir_chunk_bwd.restype = I
         L.muir_recurrent_step.argtypes = [I, I, I, I, I, I] + [P] * 7 + [I, P, P, P]
         L.muir_recurrent_step.restype = I
+        L.muir_chunk_fwd_noalloc.argtypes = [SP] + [P] * 10 + [P]
+        L.muir_chunk_fwd_noalloc.restype = I
         L.muir_profile_enable.argtypes = [I]
         L.muir_profile_enable.restype = None
         L.muir_profile_reset.argtypes = []

@@ -112,6 +112,28 @@ muir_status muir_chunk_bwd(const muir_shape* shape, const void* q, const void* k
                            float* dS0, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * muir_chunk_fwd for callers that cannot allocate device memory.  The paper
+ * has no counterpart; this is a deployment convenience.  Some hosts hand a
+ * library only input and output pointers (plugin interfaces of runtimes that
+ * own all device memory; hot paths where cudaMalloc is forbidden because it
+ * can synchronise the device or break a fixed memory budget).  This call runs
+ * the same forward as muir_chunk_fwd with its workspace in a 16 MiB array that
+ * is part of the library's device image (held on every GPU that loads the
+ * library until exit) and allocates nothing.
+ *   - Arguments as muir_chunk_fwd, without S_chunks and workspace.
+ *   - Returns MUIR_ERR_WORKSPACE when muir_chunk_fwd_workspace(shape) exceeds
+ *     16 MiB (e.g. B=1, H=2, T=1024, d=64, chunk 64 fits).
+ *   - All calls share the array: calls that overlap on the GPU race; order
+ *     them (one stream).  No state carries over between calls.
+ *   - The first call on each device looks up the array's device address with
+ *     that device current; make it before any stream capture.
+ */
+muir_status muir_chunk_fwd_noalloc(const muir_shape* shape, const void* q, const void* k,
+                                   const void* v, const void* g, const void* e, const void* w,
+                                   const void* gamma, const float* S0, void* o, float* S_final,
+                                   void* stream);
+
+/*
  * One decode token for every (b, h) against a resident float32 state (same
  * page, "Experiments": streaming inference with a constant-size float32 state;
  * fig:longctx_niah: static or dynamic readout gain).
