@@ -42,6 +42,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "mma.cuh"
+#include "tc.cuh"
 #include "profile.h"
 
 namespace muir {
@@ -53,18 +54,17 @@ constexpr int kMaxSlots = 296;  // 2 CTAs per SM on a 148-SM B200
 
 struct Lay {
     int C, D, nb8, nb16;
-    size_t G, EG, EGB, X8F, XOF, Z8F, ZOF, F, LA, LK, MQK, MQA, TII, W[8], total;
+    size_t LC, RC, BT, PRE, SUF, GBAR, LA, LK, MQK, MQA, TII, W[8], total;
 };
 
 __host__ __device__ inline Lay make_lay(int C, int D) {
     Lay L;
     L.C = C; L.D = D; L.nb8 = C / 8; L.nb16 = C / 16;
-    const size_t cd = (size_t)C * D, cc = (size_t)C * C;
+    const size_t cd = (size_t)C * D, cc = (size_t)C * C, bd = (size_t)(C / 8) * D;
     size_t o = 0;
 #define MUIR_TAKE(field, n) L.field = o; o += ((size_t)(n) + 63) & ~(size_t)63;
-    MUIR_TAKE(G, cd) MUIR_TAKE(EG, cd) MUIR_TAKE(EGB, cd)
-    MUIR_TAKE(X8F, cd) MUIR_TAKE(XOF, cd) MUIR_TAKE(Z8F, cd) MUIR_TAKE(ZOF, cd)
-    MUIR_TAKE(F, (size_t)(C / 8) * (C / 8) * D)
+    MUIR_TAKE(LC, cd) MUIR_TAKE(RC, cd) MUIR_TAKE(BT, bd) MUIR_TAKE(PRE, bd) MUIR_TAKE(SUF, bd)
+    MUIR_TAKE(GBAR, D)
     MUIR_TAKE(LA, cc) MUIR_TAKE(LK, cc) MUIR_TAKE(MQK, cc) MUIR_TAKE(MQA, cc)
     MUIR_TAKE(TII, (size_t)C * 16)
     for (int i = 0; i < 8; ++i) { MUIR_TAKE(W[i], cd) }
@@ -124,59 +124,6 @@ __device__ Chunk<Tin, D> make_chunk(const KParams& p, int chunk, float* slot) {
     return c;
 }
 
-// ------------------------------------------------------------------ prologue
-
-// Gam (clamped cumulative log decay), e^Gam, e^{gbar-Gam}, pivot factor tables.
-// The cumulative sum runs as a warp-level scan: each channel's C tokens are
-// split into 256/D segments held by lanes of one warp; segment totals are
-// combined with shuffles.
-template <typename Tin, int D>
-__device__ void prologue(const Chunk<Tin, D>& c) {
-    const Lay& L = c.L;
-    const int C = L.C, tid = threadIdx.x;
-    constexpr int S = kThreads / D;  // segments per channel
-    constexpr int CPW = 32 / S;      // channels per warp
-    const int warp = tid >> 5, lane = tid & 31;
-    const int j = warp * CPW + (lane % CPW), seg = lane / CPW, len = C / S;
-    float* G = c.s + L.G;
-    float run = 0.f;
-    for (int i = 0; i < len; ++i) {
-        const int t = seg * len + i;
-        run += fmaxf(ldf(c.g + c.base + t * c.rs + j), kLogDecayMin);
-        G[(size_t)t * D + j] = run;
-    }
-    float incl = run;
-#pragma unroll
-    for (int off = CPW; off < 32; off <<= 1) {
-        const float y = __shfl_up_sync(0xffffffffu, incl, off);
-        if (lane >= off) incl += y;
-    }
-    const float excl = incl - run;
-    for (int i = 0; i < len; ++i) G[(size_t)(seg * len + i) * D + j] += excl;
-    __syncthreads();
-    for (int idx = tid; idx < C * D; idx += kThreads) {
-        const int t = idx / D, jj = idx % D;
-        const float Gt = G[idx], gb = G[(size_t)(C - 1) * D + jj];
-        const int st = t & ~7;
-        const float Gbef = st > 0 ? G[(size_t)(st - 1) * D + jj] : 0.f;
-        const float Gm = G[(size_t)(st + 3) * D + jj], Ge = G[(size_t)(st + 7) * D + jj];
-        c.s[L.EG + idx] = expf(Gt);
-        c.s[L.EGB + idx] = expf(gb - Gt);
-        c.s[L.X8F + idx] = expf(Gt - Gbef);
-        c.s[L.XOF + idx] = expf(Gt - Gm);
-        c.s[L.Z8F + idx] = expf(Ge - Gt);
-        c.s[L.ZOF + idx] = expf(Gm - Gt);
-    }
-    const int nb8 = L.nb8;
-    for (int idx = tid; idx < nb8 * nb8 * D; idx += kThreads) {
-        const int I8 = idx / (nb8 * D), J8 = (idx / D) % nb8, jj = idx % D;
-        float f = 0.f;
-        if (J8 < I8) f = expf(G[(size_t)(8 * I8 - 1) * D + jj] - G[(size_t)(8 * J8 + 7) * D + jj]);
-        c.s[L.F + idx] = f;
-    }
-    __syncthreads();
-}
-
 // ------------------------------------------------------------------ masked products
 
 // Operand kinds for the masked products.
@@ -187,75 +134,7 @@ __device__ __forceinline__ float opval(const Chunk<Tin, D>& c, int kind, int t, 
     return kind == OP_K ? c.K(t, j) : (kind == OP_Q ? c.Qh(t, j) : c.A(t, j));
 }
 
-// Two decay-masked products sharing X: out_p[t][s] = [X (*) Z_p]_{ts}, masked
-// to s < t (strict) or s <= t, for all (t, s) of the chunk.  Work is split in
-// (16-row, 8-column) tiles over the warps.
-template <typename Tin, int D, int PASSES>
-__device__ void masked_pair(const Chunk<Tin, D>& c, int X, int Z0, int Z1, size_t out0,
-                            size_t out1, bool incl0, bool incl1) {
-    const Lay& L = c.L;
-    const int C = L.C, nb8 = L.nb8, nb16 = L.nb16;
-    const int warp = threadIdx.x >> 5, nwarps = kThreads / 32;
-    const int ntiles = nb16 * (nb16 + 1);  // sum over I16 of (2*I16 + 2)
-    const float* s = c.s;
-    for (int tile = warp; tile < ntiles; tile += nwarps) {
-        // tile -> (I16, J8) with J8 in [0, 2*I16+1]
-        int I16 = 0, rem = tile;
-        while (rem >= 2 * I16 + 2) { rem -= 2 * I16 + 2; ++I16; }
-        const int J8 = rem, t0 = 16 * I16, s0 = 8 * J8;
-        const int rb0 = 2 * I16, rb1 = 2 * I16 + 1;
-        float acc0[1][1][4], acc1[1][1][4];
-        zero_acc(acc0);
-        zero_acc(acc1);
-        if (rb1 > J8) {  // rows strictly after column block J8: pivot at J8's end
-            auto fa = [&](int r, int k) -> float {
-                const int rb = r < 8 ? rb0 : rb1;
-                if (rb <= J8) return 0.f;
-                const int t = t0 + r;
-                return opval(c, X, t, k) * s[L.X8F + (size_t)t * D + k] *
-                       s[L.F + ((size_t)rb * nb8 + J8) * D + k];
-            };
-            warp_gemm<PASSES, 1, 1>(acc0, D, fa, [&](int k, int n) {
-                return opval(c, Z0, s0 + n, k) * s[L.Z8F + (size_t)(s0 + n) * D + k];
-            });
-            warp_gemm<PASSES, 1, 1>(acc1, D, fa, [&](int k, int n) {
-                return opval(c, Z1, s0 + n, k) * s[L.Z8F + (size_t)(s0 + n) * D + k];
-            });
-        }
-        if (rb0 == J8 || rb1 == J8) {  // rows inside block J8: mid-block pivot
-            auto fa = [&](int r, int k) -> float {
-                const int rb = r < 8 ? rb0 : rb1;
-                if (rb != J8) return 0.f;
-                const int t = t0 + r;
-                return opval(c, X, t, k) * s[L.XOF + (size_t)t * D + k];
-            };
-            warp_gemm<PASSES, 1, 1>(acc0, D, fa, [&](int k, int n) {
-                return opval(c, Z0, s0 + n, k) * s[L.ZOF + (size_t)(s0 + n) * D + k];
-            });
-            warp_gemm<PASSES, 1, 1>(acc1, D, fa, [&](int k, int n) {
-                return opval(c, Z1, s0 + n, k) * s[L.ZOF + (size_t)(s0 + n) * D + k];
-            });
-        }
-        float* o0 = c.s + out0;
-        float* o1 = c.s + out1;
-        for_acc(acc0, [&](int r, int cc, float& v) {
-            const int t = t0 + r, ss = s0 + cc;
-            o0[(size_t)t * C + ss] = (incl0 ? ss <= t : ss < t) ? v : 0.f;
-        });
-        for_acc(acc1, [&](int r, int cc, float& v) {
-            const int t = t0 + r, ss = s0 + cc;
-            o1[(size_t)t * C + ss] = (incl1 ? ss <= t : ss < t) ? v : 0.f;
-        });
-    }
-    // the strict upper part (tiles never visited) must read as zero
-    for (int idx = threadIdx.x; idx < C * C; idx += kThreads) {
-        const int t = idx / C, ss = idx % C;
-        if ((ss >> 3) > 2 * (t >> 4) + 1) {
-            c.s[out0 + idx] = 0.f;
-            c.s[out1 + idx] = 0.f;
-        }
-    }
-}
+#include "staged.cuh"
 
 // ------------------------------------------------------------------ triangular solves
 
@@ -281,64 +160,43 @@ __device__ void compute_tii(float* s, const Lay& L, size_t Loff) {
     }
 }
 
-// Solve (I + L) X = R in place (X holds R on entry), L strictly lower C x C.
-// Each warp owns D/8 columns; the 16-row blocks are handled in order.
-template <int D, int PASSES>
-__device__ void fwd_solve(float* s, const Lay& L, size_t Loff, size_t Xoff) {
-    constexpr int NT = D / 64;  // n8 tiles per warp: D/8 columns / 8
-    const int C = L.C, c0 = (threadIdx.x >> 5) * (D / 8);
-    float* X = s + Xoff;
-    for (int I = 0; I < L.nb16; ++I) {
-        float acc[1][NT][4];
-        zero_acc(acc);
-        if (I > 0)
-            warp_gemm<PASSES, 1, NT>(
-                acc, 16 * I, [&](int r, int k) { return s[Loff + (size_t)(16 * I + r) * C + k]; },
-                [&](int k, int n) { return X[(size_t)k * D + c0 + n]; });
-        for_acc(acc, [&](int r, int cc, float& v) {
-            float& x = X[(size_t)(16 * I + r) * D + c0 + cc];
-            x = x - v;
-        });
-        __syncwarp();
-        float acc2[1][NT][4];
-        zero_acc(acc2);
-        warp_gemm<PASSES, 1, NT>(
-            acc2, 16, [&](int r, int k) { return s[L.TII + ((size_t)I * 16 + r) * 16 + k]; },
-            [&](int k, int n) { return X[(size_t)(16 * I + k) * D + c0 + n]; });
-        __syncwarp();
-        for_acc(acc2, [&](int r, int cc, float& v) { X[(size_t)(16 * I + r) * D + c0 + cc] = v; });
-        __syncwarp();
-    }
+// ------------------------------------------------------------------ tensor-core helpers
+
+// Four consecutive float32 scratch elements (16-byte aligned).
+__device__ __forceinline__ void ld4(const float* p, float* v) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+// Four consecutive input elements (8- or 16-byte aligned).
+__device__ __forceinline__ void ld4in(const float* p, float* v) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+__device__ __forceinline__ void ld4in(const __nv_bfloat16* p, float* v) {
+    const uint2 x = __ldg(reinterpret_cast<const uint2*>(p));
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&x.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&x.y);
+    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    v[0] = fa.x; v[1] = fa.y; v[2] = fb.x; v[3] = fb.y;
 }
 
-// Solve (I + L)^T X = R in place.
-template <int D, int PASSES>
-__device__ void bwd_solve(float* s, const Lay& L, size_t Loff, size_t Xoff) {
-    constexpr int NT = D / 64;
-    const int C = L.C, c0 = (threadIdx.x >> 5) * (D / 8);
-    float* X = s + Xoff;
-    for (int I = L.nb16 - 1; I >= 0; --I) {
-        const int r1 = 16 * (I + 1);
-        float acc[1][NT][4];
-        zero_acc(acc);
-        if (r1 < C)
-            warp_gemm<PASSES, 1, NT>(
-                acc, C - r1,
-                [&](int r, int k) { return s[Loff + (size_t)(r1 + k) * C + 16 * I + r]; },
-                [&](int k, int n) { return X[(size_t)(r1 + k) * D + c0 + n]; });
-        for_acc(acc, [&](int r, int cc, float& v) {
-            float& x = X[(size_t)(16 * I + r) * D + c0 + cc];
-            x = x - v;
-        });
-        __syncwarp();
-        float acc2[1][NT][4];
-        zero_acc(acc2);
-        warp_gemm<PASSES, 1, NT>(
-            acc2, 16, [&](int r, int k) { return s[L.TII + ((size_t)I * 16 + k) * 16 + r]; },
-            [&](int k, int n) { return X[(size_t)(16 * I + k) * D + c0 + n]; });
-        __syncwarp();
-        for_acc(acc2, [&](int r, int cc, float& v) { X[(size_t)(16 * I + r) * D + c0 + cc] = v; });
-        __syncwarp();
+// Tensor-core state shared by one CTA's products (TMEM columns, mbarrier).
+struct TcCta {
+    tc::State st;
+    unsigned char* sbuf;
+};
+
+constexpr int kTmemCols = 128;
+
+// Product over M rows (looped in 128-row tiles) and N = NT columns.
+template <int PASSES, int N, bool AR, bool BR, class FA4, class FB4, class EPI>
+__device__ __forceinline__ void tc_rows(TcCta& t, int M, int K, const FA4& fa4, const FB4& fb4,
+                                        const EPI& epi) {
+    for (int m0 = 0; m0 < M; m0 += 128) {
+        const int Mt = M - m0 < 128 ? M - m0 : 128;
+        tc::gemm<PASSES, N, AR, BR>(
+            t.st, t.sbuf, Mt, K, [&](int m, int k, float* v) { fa4(m0 + m, k, v); }, fb4,
+            [&](int m, int n, float x) { epi(m0 + m, n, x); });
     }
 }
 
@@ -346,7 +204,14 @@ __device__ void bwd_solve(float* s, const Lay& L, size_t Loff, size_t Xoff) {
 
 template <typename Tin, int D, int PASSES>
 __global__ void __launch_bounds__(kThreads) k_intra(KParams p) {
-    constexpr int NT = 2;
+    __shared__ uint32_t tmem_slot;
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ int tc_status;
+    extern __shared__ __align__(128) unsigned char dsm[];
+    TcCta tcx;
+    tcx.sbuf = dsm;
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
@@ -354,49 +219,42 @@ __global__ void __launch_bounds__(kThreads) k_intra(KParams p) {
         const Lay& L = c.L;
         const int C = L.C;
         float* s = c.s;
-        prologue(c);
-        masked_pair<Tin, D, PASSES>(c, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
+        prologue2(c);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
         __syncthreads();
         compute_tii(s, L, L.LA);
         for (int idx = threadIdx.x; idx < C * D; idx += kThreads)
-            s[L.W[0] + idx] = c.A(idx / D, idx % D) * s[L.EGB + idx];  // Ab
+            s[L.W[0] + idx] = c.A(idx / D, idx % D) * facs(c).egb(idx / D, idx % D);  // Ab
         __syncthreads();
-        bwd_solve<D, PASSES>(s, L, L.LA, L.W[0]);  // Psi = T^T Ab
+        solve_s<D, PASSES, true>(s, sm, L, L.LA, L.W[0]);  // Psi = T^T Ab
         __syncthreads();
         float* M = p.M + c.sbase;
-        // M = diag(e^gbar) - Psi^T Kt
-        cta_tiles<NT>(D, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, C,
-                    [&](int r, int k) { return s[L.W[0] + (size_t)k * D + m0 + r]; },
-                    [&](int k, int n) { return c.K(k, n0 + n) * s[L.EG + (size_t)k * D + n0 + n]; });
+        const float* Psi = s + L.W[0];
+        const Fac<Tin, D> f = facs(c);
+        // M = diag(e^gbar) - Psi^T Kt      (rows i, contraction over tokens)
+        tc_rows<PASSES, D, true, true>(tcx, D, C,
+            [&](int i, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = Psi[(size_t)(t + u) * D + i]; },
+            [&](int j, int t, float* v) {
+                for (int u = 0; u < 4; ++u) v[u] = c.K(t + u, j) * f.eg(t + u, j);
             },
-            [&](int i, int j, float v) {
-                const float d = (i == j) ? expf(s[L.G + (size_t)(C - 1) * D + i]) : 0.f;
-                M[(size_t)i * D + j] = d - v;
+            [&](int i, int j, float x) {
+                const float d = (i == j) ? expf(f.gbar(i)) : 0.f;
+                M[(size_t)i * D + j] = d - x;
             });
-        // Phi = Kb - L_K^T Psi
-        cta_tiles<NT>(C, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, C,
-                    [&](int r, int k) { return s[L.LK + (size_t)k * C + m0 + r]; },
-                    [&](int k, int n) { return s[L.W[0] + (size_t)k * D + n0 + n]; });
-            },
-            [&](int t, int j, float v) {
-                s[L.W[1] + (size_t)t * D + j] = c.K(t, j) * s[L.EGB + (size_t)t * D + j] - v;
-            });
-        __syncthreads();
-        float* Bn = p.Bn + c.sbase;
+        // Phi = Kb - L_K^T Psi              (rows t, contraction over tokens s)
+        float* Phi = s + L.W[1];
+        tc_rows<PASSES, D, true, true>(tcx, C, C,
+            [&](int t, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = s[L.LK + (size_t)(k + u) * C + t]; },
+            [&](int j, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = Psi[(size_t)(k + u) * D + j]; },
+            [&](int t, int j, float x) { Phi[(size_t)t * D + j] = c.K(t, j) * f.egb(t, j) - x; });
         // Bn = Phi^T U
-        cta_tiles<NT>(D, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, C,
-                    [&](int r, int k) { return s[L.W[1] + (size_t)k * D + m0 + r]; },
-                    [&](int k, int n) { return c.U(k, n0 + n); });
-            },
-            [&](int i, int j, float v) { Bn[(size_t)i * D + j] = v; });
-        __syncthreads();
+        float* Bn = p.Bn + c.sbase;
+        tc_rows<PASSES, D, true, true>(tcx, D, C,
+            [&](int i, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = Phi[(size_t)(t + u) * D + i]; },
+            [&](int cc, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = c.U(t + u, cc); },
+            [&](int i, int j, float x) { Bn[(size_t)i * D + j] = x; });
     }
+    tc::release(tcx.st, kTmemCols);
 }
 
 // ------------------------------------------------------------------ k_chain
@@ -451,31 +309,41 @@ __global__ void __launch_bounds__(kThreads) k_chain(const float* __restrict__ M,
 
 // ------------------------------------------------------------------ k_out
 
-// Y = T (Kt S + L_K U) into scratch W[0] (needs LA, LK, TII).
+// Y = T (Kt S + L_K U) into scratch at Yoff (needs LA, LK, TII).
 template <typename Tin, int D, int PASSES>
-__device__ void compute_Y(const Chunk<Tin, D>& c, const float* S, size_t Yoff) {
-    constexpr int NT = 2;
+__device__ void compute_Y(TcCta& tcx, const Chunk<Tin, D>& c, const float* S, size_t Yoff) {
     const Lay& L = c.L;
     const int C = L.C;
     float* s = c.s;
-    cta_tiles<NT>(C, D,
-        [&](float (&acc)[1][NT][4], int m0, int n0) {
-            warp_gemm<PASSES, 1, NT>(acc, D,
-                [&](int r, int k) { return c.K(m0 + r, k) * s[L.EG + (size_t)(m0 + r) * D + k]; },
-                [&](int k, int n) { return __ldg(S + (size_t)k * D + n0 + n); });
-            warp_gemm<PASSES, 1, NT>(acc, m0 + 16,
-                [&](int r, int k) { return s[L.LK + (size_t)(m0 + r) * C + k]; },
-                [&](int k, int n) { return c.U(k, n0 + n); });
+    const Fac<Tin, D> f = facs(c);
+    tc_rows<PASSES, D, false, true>(tcx, C, D + C,
+        [&](int t, int k, float* v) {
+            if (k < D) {
+                ld4in(c.k + c.base + t * c.rs + k, v);
+                for (int u = 0; u < 4; ++u) v[u] *= f.eg(t, k + u);
+            } else {
+                ld4(s + L.LK + (size_t)t * C + (k - D), v);
+            }
         },
-        [&](int t, int j, float v) { s[Yoff + (size_t)t * D + j] = v; });
-    __syncthreads();
-    fwd_solve<D, PASSES>(s, L, L.LA, Yoff);
+        [&](int cc, int k, float* v) {
+            if (k < D) for (int u = 0; u < 4; ++u) v[u] = __ldg(S + (size_t)(k + u) * D + cc);
+            else for (int u = 0; u < 4; ++u) v[u] = c.U(k - D + u, cc);
+        },
+        [&](int t, int j, float x) { s[Yoff + (size_t)t * D + j] = x; });
+    solve_s<D, PASSES, false>(s, reinterpret_cast<float*>(tcx.sbuf), L, L.LA, Yoff);
     __syncthreads();
 }
 
 template <typename Tin, typename Tout, int D, int PASSES>
 __global__ void __launch_bounds__(kThreads) k_out(KParams p) {
-    constexpr int NT = 2;
+    __shared__ uint32_t tmem_slot;
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ int tc_status;
+    extern __shared__ __align__(128) unsigned char dsm[];
+    TcCta tcx;
+    tcx.sbuf = dsm;
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
@@ -483,37 +351,54 @@ __global__ void __launch_bounds__(kThreads) k_out(KParams p) {
         const Lay& L = c.L;
         const int C = L.C;
         float* s = c.s;
-        prologue(c);
-        masked_pair<Tin, D, PASSES>(c, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
-        masked_pair<Tin, D, PASSES>(c, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
+        prologue2(c);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
         __syncthreads();
         compute_tii(s, L, L.LA);
         __syncthreads();
         const float* S = p.S_chunks + c.sbase;
-        compute_Y<Tin, D, PASSES>(c, S, L.W[0]);
+        compute_Y<Tin, D, PASSES>(tcx, c, S, L.W[0]);
         Tout* o = (Tout*)p.o;
-        cta_tiles<NT>(C, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, D,
-                    [&](int r, int k) { return c.Qh(m0 + r, k) * s[L.EG + (size_t)(m0 + r) * D + k]; },
-                    [&](int k, int n) { return __ldg(S + (size_t)k * D + n0 + n); });
-                warp_gemm<PASSES, 1, NT>(acc, m0 + 16,
-                    [&](int r, int k) { return s[L.MQK + (size_t)(m0 + r) * C + k]; },
-                    [&](int k, int n) { return c.U(k, n0 + n); });
-                warp_gemm<PASSES, 1, NT>(acc, m0 + 16,
-                    [&](int r, int k) { return -s[L.MQA + (size_t)(m0 + r) * C + k]; },
-                    [&](int k, int n) { return s[L.W[0] + (size_t)k * D + n0 + n]; });
+        const Fac<Tin, D> f = facs(c);
+        const float* Y = s + L.W[0];
+        // O = Qt S + M_QK U - M_QA Y
+        tc_rows<PASSES, D, false, true>(tcx, C, D + 2 * C,
+            [&](int t, int k, float* v) {
+                if (k < D) {
+                    float g4[4];
+                    ld4in(c.q + c.base + t * c.rs + k, v);
+                    ld4in(c.gm + c.base + t * c.rs + k, g4);
+                    for (int u = 0; u < 4; ++u) v[u] *= g4[u] * f.eg(t, k + u);
+                } else if (k < D + C) {
+                    ld4(s + L.MQK + (size_t)t * C + (k - D), v);
+                } else {
+                    ld4(s + L.MQA + (size_t)t * C + (k - D - C), v);
+                    for (int u = 0; u < 4; ++u) v[u] = -v[u];
+                }
             },
-            [&](int t, int j, float v) { stf(o + c.base + t * c.rs + j, v); });
-        __syncthreads();
+            [&](int cc, int k, float* v) {
+                if (k < D) for (int u = 0; u < 4; ++u) v[u] = __ldg(S + (size_t)(k + u) * D + cc);
+                else if (k < D + C) for (int u = 0; u < 4; ++u) v[u] = c.U(k - D + u, cc);
+                else for (int u = 0; u < 4; ++u) v[u] = Y[(size_t)(k - D - C + u) * D + cc];
+            },
+            [&](int t, int j, float x) { stf(o + c.base + t * c.rs + j, x); });
     }
+    tc::release(tcx.st, kTmemCols);
 }
 
 // ------------------------------------------------------------------ k_bprep
 
 template <typename Tin, int D, int PASSES>
 __global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
-    constexpr int NT = 2;
+    __shared__ uint32_t tmem_slot;
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ int tc_status;
+    extern __shared__ __align__(128) unsigned char dsm[];
+    TcCta tcx;
+    tcx.sbuf = dsm;
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
@@ -521,132 +406,49 @@ __global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
         const Lay& L = c.L;
         const int C = L.C;
         float* s = c.s;
-        prologue(c);
-        masked_pair<Tin, D, PASSES>(c, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
-        masked_pair<Tin, D, PASSES>(c, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
+        prologue2(c);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
         __syncthreads();
         compute_tii(s, L, L.LA);
-        // Z0 = M_QA^T dO
-        cta_tiles<NT>(C, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, C - m0,
-                    [&](int r, int k) { return s[L.MQA + (size_t)(m0 + k) * C + m0 + r]; },
-                    [&](int k, int n) { return c.dOv(m0 + k, n0 + n); });
-            },
-            [&](int t, int j, float v) { s[L.W[0] + (size_t)t * D + j] = v; });
         __syncthreads();
-        bwd_solve<D, PASSES>(s, L, L.LA, L.W[0]);  // Xi = T^T Z0
+        float* Xi = s + L.W[0];
+        // Z0 = M_QA^T dO
+        tc_rows<PASSES, D, true, true>(tcx, C, C,
+            [&](int t, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = s[L.MQA + (size_t)(k + u) * C + t]; },
+            [&](int cc, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc); },
+            [&](int t, int j, float x) { Xi[(size_t)t * D + j] = x; });
+        solve_s<D, PASSES, true>(s, sm, L, L.LA, L.W[0]);  // Xi = T^T Z0
         __syncthreads();
         float* Bp = p.Bn + c.sbase;
+        const Fac<Tin, D> f = facs(c);
         // B' = Qt^T dO - Kt^T Xi
-        cta_tiles<NT>(D, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, C,
-                    [&](int r, int k) { return c.Qh(k, m0 + r) * s[L.EG + (size_t)k * D + m0 + r]; },
-                    [&](int k, int n) { return c.dOv(k, n0 + n); });
-                warp_gemm<PASSES, 1, NT>(acc, C,
-                    [&](int r, int k) { return -c.K(k, m0 + r) * s[L.EG + (size_t)k * D + m0 + r]; },
-                    [&](int k, int n) { return s[L.W[0] + (size_t)k * D + n0 + n]; });
+        tc_rows<PASSES, D, true, true>(tcx, D, 2 * C,
+            [&](int i, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.Qh(k + u, i) * f.eg(k + u, i);
+                else for (int u = 0; u < 4; ++u) v[u] = -c.K(k - C + u, i) * f.eg(k - C + u, i);
             },
-            [&](int i, int j, float v) { Bp[(size_t)i * D + j] = v; });
-        __syncthreads();
+            [&](int cc, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc);
+                else for (int u = 0; u < 4; ++u) v[u] = Xi[(size_t)(k - C + u) * D + cc];
+            },
+            [&](int i, int j, float x) { Bp[(size_t)i * D + j] = x; });
     }
+    tc::release(tcx.st, kTmemCols);
 }
 
 // ------------------------------------------------------------------ k_bwd
 
-// Gradient through a decay-masked product, X side:
-//   out[t][j] = sum_{s} Gm[t][s] Z_sj exp(Gam_tj - Gam_sj)   (Gm already masked)
-// Z side:
-//   out[s][j] = sum_{t} Gm[t][s] X_tj exp(Gam_tj - Gam_sj)
-// Each 16-row output tile walks the 8-token blocks of the contraction index;
-// every block is one k8 MMA step whose result is scaled by the block-pair factor.
-template <typename Tin, int D, int PASSES, bool XSIDE, class EPI>
-__device__ void decayed_grad(const Chunk<Tin, D>& c, size_t G0, int op0, size_t G1, int op1,
-                             const EPI& epi) {
-    constexpr int NT = 2;
-    const Lay& L = c.L;
-    const int C = L.C, nb8 = L.nb8;
-    const float* s = c.s;
-    const int lane = threadIdx.x & 31, gq = lane >> 2, cq = lane & 3;
-    const int warp = threadIdx.x >> 5, nwarps = kThreads / 32;
-    const int tn = D / (8 * NT), tiles = L.nb16 * tn;
-    for (int tile = warp; tile < tiles; tile += nwarps) {
-        const int m0 = (tile / tn) * 16, n0 = (tile % tn) * 8 * NT;
-        const int rb0 = m0 / 8, rb1 = rb0 + 1;  // 8-blocks of the two row halves
-        float off[1][NT][4], dia[1][NT][4];
-        zero_acc(off);
-        zero_acc(dia);
-        for (int B8 = 0; B8 < nb8; ++B8) {
-            // relation of each row half to block B8: 1 = off-diagonal, 2 = diagonal, 0 = none
-            int rel0, rel1;
-            if (XSIDE) {
-                rel0 = B8 < rb0 ? 1 : (B8 == rb0 ? 2 : 0);
-                rel1 = B8 < rb1 ? 1 : (B8 == rb1 ? 2 : 0);
-            } else {
-                rel0 = B8 > rb0 ? 1 : (B8 == rb0 ? 2 : 0);
-                rel1 = B8 > rb1 ? 1 : (B8 == rb1 ? 2 : 0);
-            }
-            if (rel0 == 0 && rel1 == 0) continue;
-            const int k0 = 8 * B8;
-            for (int kind = 1; kind <= 2; ++kind) {
-                if (rel0 != kind && rel1 != kind) continue;
-                // A(r, k): gradient matrix entry; rows of the other kind are zero
-                auto gm = [&](size_t Goff, int r, int k) -> float {
-                    const int rel = r < 8 ? rel0 : rel1;
-                    if (rel != kind) return 0.f;
-                    return XSIDE ? s[Goff + (size_t)(m0 + r) * C + k0 + k]
-                                 : s[Goff + (size_t)(k0 + k) * C + m0 + r];
-                };
-                // B(k, n): operand row (k0 + k), scaled by its pivot factor
-                const size_t fac = XSIDE ? (kind == 1 ? L.Z8F : L.ZOF) : (kind == 1 ? L.X8F : L.XOF);
-                float tmp[1][NT][4];
-                zero_acc(tmp);
-                warp_gemm<PASSES, 1, NT>(tmp, 8, [&](int r, int k) { return gm(G0, r, k); },
-                    [&](int k, int n) {
-                        return opval(c, op0, k0 + k, n0 + n) * s[fac + (size_t)(k0 + k) * D + n0 + n];
-                    });
-                warp_gemm<PASSES, 1, NT>(tmp, 8, [&](int r, int k) { return gm(G1, r, k); },
-                    [&](int k, int n) {
-                        return opval(c, op1, k0 + k, n0 + n) * s[fac + (size_t)(k0 + k) * D + n0 + n];
-                    });
-                if (kind == 2) {
-#pragma unroll
-                    for (int n = 0; n < NT; ++n)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) dia[0][n][i] += tmp[0][n][i];
-                } else {
-                    // off-diagonal block pair factor F[row block][B8] (X side) or F[B8][row block]
-#pragma unroll
-                    for (int n = 0; n < NT; ++n)
-#pragma unroll
-                        for (int i = 0; i < 4; ++i) {
-                            const int rb = i < 2 ? rb0 : rb1;
-                            const int col = n0 + 8 * n + 2 * cq + (i & 1);
-                            const size_t fi = XSIDE ? ((size_t)rb * nb8 + B8) : ((size_t)B8 * nb8 + rb);
-                            const float f = (i < 2 ? rel0 : rel1) == 1 ? s[L.F + fi * D + col] : 0.f;
-                            off[0][n][i] += f * tmp[0][n][i];
-                        }
-                }
-            }
-        }
-        // output-side pivot factors
-        const size_t fo = XSIDE ? L.X8F : L.Z8F, fd = XSIDE ? L.XOF : L.ZOF;
-#pragma unroll
-        for (int n = 0; n < NT; ++n)
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                const int row = m0 + gq + (i < 2 ? 0 : 8);
-                const int col = n0 + 8 * n + 2 * cq + (i & 1);
-                const size_t x = (size_t)row * D + col;
-                epi(row, col, s[fo + x] * off[0][n][i] + s[fd + x] * dia[0][n][i]);
-            }
-    }
-}
-
 template <typename Tin, int D, int PASSES>
 __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
-    constexpr int NT = 2;
+    __shared__ uint32_t tmem_slot;
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ int tc_status;
+    extern __shared__ __align__(128) unsigned char dsm[];
+    TcCta tcx;
+    tcx.sbuf = dsm;
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
@@ -658,138 +460,151 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         const float* dS = p.dS_chunks + c.sbase;
         const size_t Y = L.W[0], dR = L.W[1], dK = L.W[2], dQh = L.W[3], dA = L.W[4],
                      dU = L.W[5], dGam = L.W[6], XB = L.W[7];
-        prologue(c);
-        masked_pair<Tin, D, PASSES>(c, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
-        masked_pair<Tin, D, PASSES>(c, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
+        prologue2(c);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
         __syncthreads();
         compute_tii(s, L, L.LA);
         __syncthreads();
-        compute_Y<Tin, D, PASSES>(c, S, Y);
-        // dY = -M_QA^T dO - Ab dS'
-        cta_tiles<NT>(C, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, C - m0,
-                    [&](int r, int k) { return s[L.MQA + (size_t)(m0 + k) * C + m0 + r]; },
-                    [&](int k, int n) { return c.dOv(m0 + k, n0 + n); });
-                warp_gemm<PASSES, 1, NT>(acc, D,
-                    [&](int r, int k) { return c.A(m0 + r, k) * s[L.EGB + (size_t)(m0 + r) * D + k]; },
-                    [&](int k, int n) { return __ldg(dS + (size_t)k * D + n0 + n); });
+        compute_Y<Tin, D, PASSES>(tcx, c, S, Y);
+        const Fac<Tin, D> f = facs(c);
+        // dY = -M_QA^T dO - Ab dS'   (stored in dR, then dR = T^T dY)
+        tc_rows<PASSES, D, true, true>(tcx, C, C + D,
+            [&](int t, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = s[L.MQA + (size_t)(k + u) * C + t];
+                else {
+                    float k4[4];
+                    ld4in(c.e + c.base + t * c.rs + (k - C), v);
+                    ld4in(c.k + c.base + t * c.rs + (k - C), k4);
+                    for (int u = 0; u < 4; ++u) v[u] *= k4[u] * f.egb(t, k - C + u);
+                }
             },
-            [&](int t, int j, float v) { s[dR + (size_t)t * D + j] = -v; });
+            [&](int cc, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc);
+                else for (int u = 0; u < 4; ++u) v[u] = __ldg(dS + (size_t)(k - C + u) * D + cc);
+            },
+            [&](int t, int j, float x) { s[dR + (size_t)t * D + j] = -x; });
+        solve_s<D, PASSES, true>(s, sm, L, L.LA, dR);  // dR = T^T dY
         __syncthreads();
-        bwd_solve<D, PASSES>(s, L, L.LA, dR);  // dR = T^T dY
-        __syncthreads();
+        // B(k = c, n = j) = S[j][c] or dS'[j][c]: rows of the staged B are rows of S
+        auto rowsS = [&](int j, int k, float* v) { ld4in(S + (size_t)j * D + k, v); };
+        auto rowsdS = [&](int j, int k, float* v) { ld4in(dS + (size_t)j * D + k, v); };
         // dQt = dO S^T  -> dQh = dQt e^Gam ; dGam = dQt * Qt
-        cta_tiles<NT>(C, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, D, [&](int r, int k) { return c.dOv(m0 + r, k); },
-                    [&](int k, int n) { return __ldg(S + (size_t)(n0 + n) * D + k); });
-            },
-            [&](int t, int j, float v) {
-                const size_t x = (size_t)t * D + j;
-                s[dQh + x] = v * s[L.EG + x];
-                s[dGam + x] = v * c.Qh(t, j) * s[L.EG + x];
+        tc_rows<PASSES, D, false, false>(tcx, C, D,
+            [&](int t, int k, float* v) { ld4in(c.dO + c.base + t * c.rs + k, v); }, rowsS,
+            [&](int t, int j, float x) {
+                const size_t i = (size_t)t * D + j;
+                const float eg = f.eg(t, j);
+                s[dQh + i] = x * eg;
+                s[dGam + i] = x * c.Qh(t, j) * eg;
             });
-        __syncthreads();
         // dKt = dR S^T -> dK = dKt e^Gam ; dGam += dKt * Kt
-        cta_tiles<NT>(C, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, D, [&](int r, int k) { return s[dR + (size_t)(m0 + r) * D + k]; },
-                    [&](int k, int n) { return __ldg(S + (size_t)(n0 + n) * D + k); });
-            },
-            [&](int t, int j, float v) {
-                const size_t x = (size_t)t * D + j;
-                s[dK + x] = v * s[L.EG + x];
-                s[dGam + x] += v * c.K(t, j) * s[L.EG + x];
+        tc_rows<PASSES, D, false, false>(tcx, C, D,
+            [&](int t, int k, float* v) { ld4(s + dR + (size_t)t * D + k, v); }, rowsS,
+            [&](int t, int j, float x) {
+                const size_t i = (size_t)t * D + j;
+                const float eg = f.eg(t, j);
+                s[dK + i] = x * eg;
+                s[dGam + i] += x * c.K(t, j) * eg;
             });
-        __syncthreads();
         // dKb = U dS'^T -> dK += dKb e^{gbar-Gam} ; dGam -= dKb*Kb ; XB = dKb*Kb
-        cta_tiles<NT>(C, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, D, [&](int r, int k) { return c.U(m0 + r, k); },
-                    [&](int k, int n) { return __ldg(dS + (size_t)(n0 + n) * D + k); });
+        tc_rows<PASSES, D, false, false>(tcx, C, D,
+            [&](int t, int k, float* v) {
+                float w4[4];
+                ld4in(c.v + c.base + t * c.rs + k, v);
+                ld4in(c.w + c.base + t * c.rs + k, w4);
+                for (int u = 0; u < 4; ++u) v[u] *= w4[u];
             },
-            [&](int t, int j, float v) {
-                const size_t x = (size_t)t * D + j;
-                const float kb = c.K(t, j) * s[L.EGB + x];
-                s[dK + x] += v * s[L.EGB + x];
-                s[dGam + x] -= v * kb;
-                s[XB + x] = v * kb;
+            rowsdS,
+            [&](int t, int j, float x) {
+                const size_t i = (size_t)t * D + j;
+                const float egb = f.egb(t, j), kb = c.K(t, j) * egb;
+                s[dK + i] += x * egb;
+                s[dGam + i] -= x * kb;
+                s[XB + i] = x * kb;
             });
-        __syncthreads();
         // dAb = -Y dS'^T -> dA = dAb e^{gbar-Gam} ; dGam -= dAb*Ab ; XB += dAb*Ab
-        cta_tiles<NT>(C, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, D, [&](int r, int k) { return -s[Y + (size_t)(m0 + r) * D + k]; },
-                    [&](int k, int n) { return __ldg(dS + (size_t)(n0 + n) * D + k); });
+        tc_rows<PASSES, D, false, false>(tcx, C, D,
+            [&](int t, int k, float* v) {
+                ld4(s + Y + (size_t)t * D + k, v);
+                for (int u = 0; u < 4; ++u) v[u] = -v[u];
             },
-            [&](int t, int j, float v) {
-                const size_t x = (size_t)t * D + j;
-                const float ab = c.A(t, j) * s[L.EGB + x];
-                s[dA + x] = v * s[L.EGB + x];
-                s[dGam + x] -= v * ab;
-                s[XB + x] += v * ab;
+            rowsdS,
+            [&](int t, int j, float x) {
+                const size_t i = (size_t)t * D + j;
+                const float egb = f.egb(t, j), ab = c.A(t, j) * egb;
+                s[dA + i] = x * egb;
+                s[dGam + i] -= x * ab;
+                s[XB + i] += x * ab;
             });
-        __syncthreads();
         // dU = M_QK^T dO + L_K^T dR + Kb dS'
-        cta_tiles<NT>(C, D,
-            [&](float (&acc)[1][NT][4], int m0, int n0) {
-                warp_gemm<PASSES, 1, NT>(acc, C - m0,
-                    [&](int r, int k) { return s[L.MQK + (size_t)(m0 + k) * C + m0 + r]; },
-                    [&](int k, int n) { return c.dOv(m0 + k, n0 + n); });
-                warp_gemm<PASSES, 1, NT>(acc, C - m0,
-                    [&](int r, int k) { return s[L.LK + (size_t)(m0 + k) * C + m0 + r]; },
-                    [&](int k, int n) { return s[dR + (size_t)(m0 + k) * D + n0 + n]; });
-                warp_gemm<PASSES, 1, NT>(acc, D,
-                    [&](int r, int k) { return c.K(m0 + r, k) * s[L.EGB + (size_t)(m0 + r) * D + k]; },
-                    [&](int k, int n) { return __ldg(dS + (size_t)k * D + n0 + n); });
+        tc_rows<PASSES, D, true, true>(tcx, C, 2 * C + D,
+            [&](int t, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = s[L.MQK + (size_t)(k + u) * C + t];
+                else if (k < 2 * C) for (int u = 0; u < 4; ++u) v[u] = s[L.LK + (size_t)(k - C + u) * C + t];
+                else {
+                    ld4in(c.k + c.base + t * c.rs + (k - 2 * C), v);
+                    for (int u = 0; u < 4; ++u) v[u] *= f.egb(t, k - 2 * C + u);
+                }
             },
-            [&](int t, int j, float v) { s[dU + (size_t)t * D + j] = v; });
-        __syncthreads();
+            [&](int cc, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc);
+                else if (k < 2 * C) for (int u = 0; u < 4; ++u) v[u] = s[dR + (size_t)(k - C + u) * D + cc];
+                else for (int u = 0; u < 4; ++u) v[u] = __ldg(dS + (size_t)(k - 2 * C + u) * D + cc);
+            },
+            [&](int t, int j, float x) { s[dU + (size_t)t * D + j] = x; });
         // gradients of the masked products (overwrite them): dL_A = -strict(dR Y^T),
         // dL_K = strict(dR U^T), dM_QK = incl(dO U^T), dM_QA = -incl(dO Y^T)
         for (int which = 0; which < 4; ++which) {
             const size_t out = which == 0 ? L.LA : which == 1 ? L.LK : which == 2 ? L.MQK : L.MQA;
             const bool incl = which >= 2;
             const float sg = (which == 0 || which == 3) ? -1.f : 1.f;
-            cta_tiles<NT>(C, C,
-                [&](float (&acc)[1][NT][4], int m0, int n0) {
-                    if (n0 > m0 + 15) return;
-                    warp_gemm<PASSES, 1, NT>(acc, D,
-                        [&](int r, int k) {
-                            return which < 2 ? s[dR + (size_t)(m0 + r) * D + k] : c.dOv(m0 + r, k);
-                        },
-                        [&](int k, int n) {
-                            return (which == 0 || which == 3) ? s[Y + (size_t)(n0 + n) * D + k]
-                                                              : c.U(n0 + n, k);
-                        });
-                },
-                [&](int t, int ss, float v) {
-                    const bool keep = incl ? ss <= t : ss < t;
-                    s[out + (size_t)t * C + ss] = keep ? sg * v : 0.f;
-                });
+            for (int n0 = 0; n0 < C; n0 += 128) {
+                tc_rows<PASSES, 128, false, false>(tcx, C, D,
+                    [&](int t, int k, float* v) {
+                        if (which < 2) ld4(s + dR + (size_t)t * D + k, v);
+                        else ld4in(c.dO + c.base + t * c.rs + k, v);
+                    },
+                    [&](int n, int k, float* v) {
+                        const int ss = n0 + n;
+                        if (ss >= C) { v[0] = v[1] = v[2] = v[3] = 0.f; return; }
+                        if (which == 0 || which == 3) ld4(s + Y + (size_t)ss * D + k, v);
+                        else {
+                            float w4[4];
+                            ld4in(c.v + c.base + ss * c.rs + k, v);
+                            ld4in(c.w + c.base + ss * c.rs + k, w4);
+                            for (int u = 0; u < 4; ++u) v[u] *= w4[u];
+                        }
+                    },
+                    [&](int t, int n, float x) {
+                        const int ss = n0 + n;
+                        if (ss >= C) return;
+                        const bool keep = incl ? ss <= t : ss < t;
+                        s[out + (size_t)t * C + ss] = keep ? sg * x : 0.f;
+                    });
+            }
         }
         __syncthreads();
         // X side: dK += dL_A (*) A + dL_K (*) K ; dQh += dM_QK (*) K + dM_QA (*) A ; dGam += X * dX
-        decayed_grad<Tin, D, PASSES, true>(c, L.LA, OP_A, L.LK, OP_K, [&](int t, int j, float v) {
+        decayed_grad_any<Tin, D, PASSES, true>(c, sm, L.LA, OP_A, L.LK, OP_K, [&](int t, int j, float v) {
             const size_t x = (size_t)t * D + j;
             s[dK + x] += v;
             s[dGam + x] += c.K(t, j) * v;
         });
-        decayed_grad<Tin, D, PASSES, true>(c, L.MQK, OP_K, L.MQA, OP_A, [&](int t, int j, float v) {
+        decayed_grad_any<Tin, D, PASSES, true>(c, sm, L.MQK, OP_K, L.MQA, OP_A, [&](int t, int j, float v) {
             const size_t x = (size_t)t * D + j;
             s[dQh + x] += v;
             s[dGam + x] += c.Qh(t, j) * v;
         });
         __syncthreads();
         // Z side: dA += dL_A^T (*) K + dM_QA^T (*) Qh ; dK += dL_K^T (*) K + dM_QK^T (*) Qh ; dGam -= Z * dZ
-        decayed_grad<Tin, D, PASSES, false>(c, L.LA, OP_K, L.MQA, OP_Q, [&](int t, int j, float v) {
+        decayed_grad_any<Tin, D, PASSES, false>(c, sm, L.LA, OP_K, L.MQA, OP_Q, [&](int t, int j, float v) {
             const size_t x = (size_t)t * D + j;
             s[dA + x] += v;
             s[dGam + x] -= c.A(t, j) * v;
         });
         __syncthreads();
-        decayed_grad<Tin, D, PASSES, false>(c, L.LK, OP_K, L.MQK, OP_Q, [&](int t, int j, float v) {
+        decayed_grad_any<Tin, D, PASSES, false>(c, sm, L.LK, OP_K, L.MQK, OP_Q, [&](int t, int j, float v) {
             const size_t x = (size_t)t * D + j;
             s[dK + x] += v;
             s[dGam + x] -= c.K(t, j) * v;
@@ -802,7 +617,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
             const int j = threadIdx.x;
             float acc = 0.f;
             for (int cc = 0; cc < D; ++cc) acc += __ldg(S + (size_t)j * D + cc) * __ldg(dS + (size_t)j * D + cc);
-            float dgb = acc * expf(s[L.G + (size_t)(C - 1) * D + j]);
+            float dgb = acc * expf(facs(c).gbar(j));
             for (int t = 0; t < C; ++t) dgb += s[XB + (size_t)t * D + j];
             float run = dgb;
             for (int t = C - 1; t >= 0; --t) {
@@ -826,9 +641,35 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         }
         __syncthreads();
     }
+    tc::release(tcx.st, kTmemCols);
 }
 
 // ------------------------------------------------------------------ host side
+
+// Dynamic shared memory of the per-chunk kernels: the largest staging area of
+// their phases (tensor-core slabs, masked products, gradient products, solves).
+template <int D, int PASSES>
+static int dyn_bytes(int C) {
+    int f = tc::stage_bytes<PASSES, 128>() / 4;
+    const int m = masked_smem_floats(C, D), g = decayed_smem_floats(C), s = solve_smem_floats(C, D);
+    f = f > m ? f : m;
+    f = f > g ? f : g;
+    f = f > s ? f : s;
+    return f * 4;
+}
+
+// CTAs that fit on one SM next to each other with this much shared memory.
+static int ctas_per_sm(int dyn) { return dyn <= 100 * 1024 ? 2 : 1; }
+
+template <typename Tin, int D, int PASSES>
+static cudaError_t set_smem_attrs(int bytes) {
+    cudaError_t e = cudaFuncSetAttribute(k_intra<Tin, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_out<Tin, float, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_out<Tin, __nv_bfloat16, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_bprep<Tin, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_bwd<Tin, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    return e;
+}
 
 static int num_slots(int nch) { return nch < kMaxSlots ? nch : kMaxSlots; }
 
@@ -881,16 +722,21 @@ static cudaError_t fwd_impl(const ChunkProblem& P, const float* S0, void* o, flo
     kp.slot = slot_floats(P.C, D);
     kp.S_chunks = Sc;
     kp.o = o;
-    const int grid = num_slots(nch);
-    MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
-    cudaError_t err = cudaGetLastError();
+    const int dyn = dyn_bytes<D, PASSES>(P.C);
+    int grid = num_slots(nch);
+    const int resident = 148 * ctas_per_sm(dyn);
+    if (grid > resident) grid = resident;
+    cudaError_t err = set_smem_attrs<Tin, D, PASSES>(dyn);
+    if (err != cudaSuccess) return err;
+    MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+    err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, S_final, st);
     if (err != cudaSuccess) return err;
     if (P.out_bf16)
-        MUIR_TIMED("k_out", st, k_out<Tin, __nv_bfloat16, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
+        MUIR_TIMED("k_out", st, k_out<Tin, __nv_bfloat16, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
     else
-        MUIR_TIMED("k_out", st, k_out<Tin, float, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
+        MUIR_TIMED("k_out", st, k_out<Tin, float, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
     return cudaGetLastError();
 }
 
@@ -917,19 +763,24 @@ static cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float*
     kp.S_chunks = Sc;
     kp.dS_chunks = dSc;
     kp.dq = dq; kp.dk = dk; kp.dv = dv; kp.dg = dg; kp.de = de; kp.dw = dw; kp.dgamma = dgamma;
-    const int grid = num_slots(nch);
-    MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
-    cudaError_t err = cudaGetLastError();
+    const int dyn = dyn_bytes<D, PASSES>(P.C);
+    int grid = num_slots(nch);
+    const int resident = 148 * ctas_per_sm(dyn);
+    if (grid > resident) grid = resident;
+    cudaError_t err = set_smem_attrs<Tin, D, PASSES>(dyn);
+    if (err != cudaSuccess) return err;
+    MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+    err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     if (recompute) {
         err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, nullptr, st);
         if (err != cudaSuccess) return err;
     }
-    MUIR_TIMED("k_bprep", st, k_bprep<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
+    MUIR_TIMED("k_bprep", st, k_bprep<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     err = launch_chain<D, PASSES, true>(BH, P.N, kp.M, kp.Bn, dS_final, dSc, dS0, st);
     if (err != cudaSuccess) return err;
-    MUIR_TIMED("k_bwd", st, k_bwd<Tin, D, PASSES><<<grid, kThreads, 0, st>>>(kp));
+    MUIR_TIMED("k_bwd", st, k_bwd<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
     return cudaGetLastError();
 }
 

@@ -1,0 +1,220 @@
+// tc.cuh -- dense products on the 5th-generation tensor cores (tcgen05).
+//
+// D[m][n] = sum_k A(m, k) B(k, n) for m < 128, n < N (N % 16 == 0, N <= 256),
+// with A and B produced by element functors, staged through shared memory in
+// K slabs of KS = 32 in the K-major, no-swizzle canonical layout (core matrix =
+// 8 rows x 16 bytes; LBO = 128 B between the 4-element K groups, SBO = KS/4 *
+// 128 B between 8-row groups), accumulated in TMEM (row m = TMEM lane m,
+// column n = TMEM column n) by kind::tf32 MMAs (M = 128, K = 8) that one thread
+// issues, completion tracked by tcgen05.commit on an mbarrier, read back with
+// tcgen05.ld (32 lanes x 32 bit) for an element epilogue.
+//
+// PASSES = 1: operands rounded to TF32 (round to nearest) when staged.
+// PASSES = 3: split TF32, hi = tf32(x), lo = tf32(x - hi); hi*hi + hi*lo + lo*hi.
+//
+// Every wait is bounded: after kSpinLimit polls a wait gives up, records an
+// error code in the CTA's status word and returns (results are then garbage,
+// nothing hangs).
+#pragma once
+
+#include <stdint.h>
+
+namespace muir {
+namespace tc {
+
+constexpr int KS = 32;                       // K slab staged per round
+constexpr uint32_t kSpinLimit = 1u << 26;    // mbarrier polls before giving up
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFF);
+    d |= (uint64_t)((lbo >> 4) & 0x3FFF) << 16;
+    d |= (uint64_t)((sbo >> 4) & 0x3FFF) << 32;
+    d |= (uint64_t)1 << 46;  // descriptor version for sm_100
+    return d;                // base offset 0, legacy LBO mode, no swizzle
+}
+
+// Instruction descriptor: kind::tf32, D = f32, A = B = tf32, both K-major.
+__host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
+    return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
+           ((uint32_t)(M >> 4) << 24);
+}
+
+__device__ __forceinline__ float tf32_rn(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
+// Byte offset of element (row, k) in a K-major canonical slab with KS columns.
+__device__ __forceinline__ uint32_t kmaj_off(int row, int k) {
+    return (uint32_t)((row >> 3) * (KS / 4 * 128) + (k >> 2) * 128 + (row & 7) * 16 + (k & 3) * 4);
+}
+
+struct State {
+    uint32_t tmem;     // TMEM base address (lane 0, first allocated column)
+    uint64_t* mbar;    // completion barrier in shared memory
+    uint32_t phase;    // parity of the next phase to wait for
+    int* status;       // CTA status word in shared memory (0 = ok)
+};
+
+// Allocate ncols TMEM columns (power of two >= 32); all threads call it.
+__device__ __forceinline__ void init(State& s, uint32_t* tmem_slot, uint64_t* mbar, int* status,
+                                     int ncols) {
+    if (threadIdx.x == 0) {
+        asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(mbar)));
+        *status = 0;
+    }
+    if (threadIdx.x < 32) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_addr(tmem_slot)), "r"(ncols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+    asm volatile("tcgen05.fence::after_thread_sync;");
+    s.tmem = *tmem_slot;
+    s.mbar = mbar;
+    s.phase = 0;
+    s.status = status;
+}
+
+__device__ __forceinline__ void release(const State& s, int ncols) {
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+    if (threadIdx.x < 32)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(s.tmem),
+                     "r"(ncols));
+}
+
+// Wait (bounded) for the mbarrier phase s.phase, then flip it.  All threads call.
+__device__ __forceinline__ void wait_mma(State& s) {
+    uint32_t done = 0;
+    for (uint32_t it = 0; it < kSpinLimit && !done; ++it) {
+        asm volatile(
+            "{\n.reg .pred p;\nmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+            "selp.u32 %0, 1, 0, p;\n}"
+            : "=r"(done)
+            : "r"(smem_addr(s.mbar)), "r"(s.phase));
+    }
+    if (!done) *s.status = 1;
+    s.phase ^= 1u;
+    asm volatile("tcgen05.fence::after_thread_sync;");
+}
+
+__device__ __forceinline__ void issue_mma(uint32_t tmem, uint64_t da, uint64_t db, uint32_t idesc,
+                                          uint32_t accumulate) {
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], %1, %2, %3, p;\n}" ::"r"(tmem),
+        "l"(da), "l"(db), "r"(idesc), "r"(accumulate));
+}
+
+__device__ __forceinline__ void commit(const State& s) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(smem_addr(s.mbar)));
+}
+
+// Shared-memory bytes a gemm<PASSES, N> needs for its staging buffers.
+template <int PASSES, int N>
+__host__ __device__ constexpr int stage_bytes() {
+    return (PASSES == 3 ? 2 : 1) * (128 + N) * KS * 4;
+}
+
+// Stage one operand slab: rows [0, R) x K columns [k0, k0 + KS) into `dst`
+// (and `dst_lo` for PASSES == 3).  f4(row, k, out[4]) produces elements
+// (row, k..k+3) with k a multiple of 4 (zeros past kmax).  ROWMAJ_LANES: lanes
+// walk rows (source contiguous along rows) instead of K groups.
+template <int PASSES, bool ROW_LANES, class F4>
+__device__ __forceinline__ void stage(unsigned char* dst, unsigned char* dst_lo, int R, int k0,
+                                      int kmax, const F4& f4) {
+    constexpr int KG = KS / 4;
+    const int total = R * KG;
+    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+        int row, kg;
+        if (ROW_LANES) { row = idx % R; kg = idx / R; }
+        else { kg = idx % KG; row = idx / KG; }
+        const int k = k0 + 4 * kg;
+        float v[4] = {0.f, 0.f, 0.f, 0.f};
+        if (k < kmax) f4(row, k, v);
+        float4 hi, lo;
+        hi.x = tf32_rn(v[0]); hi.y = tf32_rn(v[1]); hi.z = tf32_rn(v[2]); hi.w = tf32_rn(v[3]);
+        *reinterpret_cast<float4*>(dst + kmaj_off(row, 4 * kg)) = hi;
+        if (PASSES == 3) {
+            lo.x = tf32_rn(v[0] - hi.x); lo.y = tf32_rn(v[1] - hi.y);
+            lo.z = tf32_rn(v[2] - hi.z); lo.w = tf32_rn(v[3] - hi.w);
+            *reinterpret_cast<float4*>(dst_lo + kmaj_off(row, 4 * kg)) = lo;
+        }
+    }
+}
+
+// D (128 x N, TMEM) = sum over K of A(m, k) B(k, n).  fa4(m, k, v[4]) gives
+// A(m, k..k+3); fb4(n, k, v[4]) gives B(k..k+3, n).  Rows m >= M are zero.
+// Then epi(m, n, value) for m < M, n < N.  All threads of the CTA call it.
+template <int PASSES, int N, bool A_ROW_LANES, bool B_ROW_LANES, class FA4, class FB4, class EPI>
+__device__ void gemm(State& s, unsigned char* sbuf, int M, int K, const FA4& fa4, const FB4& fb4,
+                     const EPI& epi) {
+    static_assert(N % 16 == 0 && N <= 256, "N");
+    constexpr int ABYTES = 128 * KS * 4, BBYTES = N * KS * 4;
+    unsigned char* sA = sbuf;
+    unsigned char* sB = sbuf + ABYTES;
+    unsigned char* sAl = sbuf + ABYTES + BBYTES;
+    unsigned char* sBl = sAl + ABYTES;
+    constexpr uint32_t idesc = idesc_tf32(128, N);
+    constexpr uint32_t SBO = KS / 4 * 128;
+    const int nslab = (K + KS - 1) / KS;
+    for (int sl = 0; sl < nslab; ++sl) {
+        const int k0 = sl * KS;
+        stage<PASSES, A_ROW_LANES>(sA, sAl, 128, k0, K, [&](int m, int k, float* v) {
+            if (m < M) fa4(m, k, v);
+        });
+        stage<PASSES, B_ROW_LANES>(sB, sBl, N, k0, K, fb4);
+        asm volatile("fence.proxy.async.shared::cta;");
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            asm volatile("tcgen05.fence::after_thread_sync;");
+#pragma unroll
+            for (int ks = 0; ks < KS / 8; ++ks) {
+                const uint32_t acc = (sl > 0 || ks > 0) ? 1u : 0u;
+                const uint64_t da = make_desc(smem_addr(sA) + ks * 256, 128, SBO);
+                const uint64_t db = make_desc(smem_addr(sB) + ks * 256, 128, SBO);
+                issue_mma(s.tmem, da, db, idesc, acc);
+                if (PASSES == 3) {
+                    const uint64_t dal = make_desc(smem_addr(sAl) + ks * 256, 128, SBO);
+                    const uint64_t dbl = make_desc(smem_addr(sBl) + ks * 256, 128, SBO);
+                    issue_mma(s.tmem, da, dbl, idesc, 1u);
+                    issue_mma(s.tmem, dal, db, idesc, 1u);
+                }
+            }
+            commit(s);
+        }
+        wait_mma(s);  // the slab buffers are free again and, after the last slab, D is final
+    }
+    // epilogue: warp w reads TMEM lanes [32 (w % 4), +32) and half of the columns
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = 32 * quarter + lane;
+    constexpr int NH = N / 2;
+    for (int c0 = half * NH; c0 < (half + 1) * NH; c0 += 8) {
+        uint32_t r[8];
+        const uint32_t taddr = s.tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0;
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                       "=r"(r[6]), "=r"(r[7])
+                     : "r"(taddr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;");
+        if (row < M) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) epi(row, c0 + j, __uint_as_float(r[j]));
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+}
+
+}  // namespace tc
+}  // namespace muir
