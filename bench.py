@@ -55,8 +55,8 @@ DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 6 * 128 * 2 + 128 * 2  # S read+writ
 # DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel; valid only while the kernel source hash matches.
 NCU_TRAFFIC = {
-    # profiles/k_bwd_B1_H16_T8192_d128_C128.md: 8.492 GB for 131,072 token-heads
-    "k_bwd": {"bytes_per_token_head": 8.492118e9 / 131072, "source": "db35a5a6a35fddcb"},
+    # profiles/k_bwd_B1_H16_T8192_d128_C128.md: 4.889 GB for 131,072 token-heads
+    "k_bwd": {"bytes_per_token_head": 4.889042e9 / 131072, "source": "e35e4f419180ed8f"},
 }
 
 
@@ -254,8 +254,8 @@ def gpu_arm(args, rank, world, local):
     args_in = [d[n] for n in NAMES]
 
     def step():
-        o, S, Sc = muir.chunk_fwd(*args_in, d["S0"], chunk=C, return_chunk_states=True, ws=ws_f)
-        gr = muir.chunk_bwd(*args_in, d["S0"], d["dO"], chunk=C, S_chunks=Sc, ws=ws_b)
+        o, S, Sc, Mc = muir.chunk_fwd(*args_in, d["S0"], chunk=C, return_saved=True, ws=ws_f)
+        gr = muir.chunk_bwd(*args_in, d["S0"], d["dO"], chunk=C, S_chunks=Sc, M_chunks=Mc, ws=ws_b)
         return o, gr
 
     ws_f = torch.empty(muir.fwd_workspace_bytes(W.B, W.T, W.H, W.dk, C), dtype=torch.uint8, device=dev)
@@ -392,8 +392,9 @@ def e2e_measure(muir, x, W, C, dev, ws_f, ws_b, steps, world):
         for k, v in host.items():
             dev_in[k].copy_(v, non_blocking=True)
         a = [dev_in[n] for n in NAMES]
-        o, S, Sc = muir.chunk_fwd(*a, dev_in.get("S0"), chunk=C, return_chunk_states=True, ws=ws_f)
-        gr = muir.chunk_bwd(*a, dev_in.get("S0"), dev_in["dO"], chunk=C, S_chunks=Sc, ws=ws_b)
+        o, S, Sc, Mc = muir.chunk_fwd(*a, dev_in.get("S0"), chunk=C, return_saved=True, ws=ws_f)
+        gr = muir.chunk_bwd(*a, dev_in.get("S0"), dev_in["dO"], chunk=C, S_chunks=Sc, M_chunks=Mc,
+                            ws=ws_b)
         res = [o, S] + [gr[k] for k in sorted(gr)]
         if outs_host is None:
             outs_host = [torch.empty_like(r, device="cpu").pin_memory() for r in res]

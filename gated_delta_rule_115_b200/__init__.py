@@ -64,9 +64,9 @@ def lib():
         L.muir_chunk_fwd_workspace.restype = S
         L.muir_chunk_bwd_workspace.argtypes = [SP]
         L.muir_chunk_bwd_workspace.restype = S
-        L.muir_chunk_fwd.argtypes = [SP] + [P] * 12 + [S, P]
+        L.muir_chunk_fwd.argtypes = [SP] + [P] * 13 + [S, P]
         L.muir_chunk_fwd.restype = I
-        L.muir_chunk_bwd.argtypes = [SP] + [P] * 20 + [S, P]
+        L.muir_chunk_bwd.argtypes = [SP] + [P] * 21 + [S, P]
         L.muir_chunk_bwd.restype = I
         L.muir_recurrent_step.argtypes = [I, I, I, I, I, I] + [P] * 7 + [I, P, P, P]
         L.muir_recurrent_step.restype = I
@@ -143,10 +143,12 @@ def _workspace(nbytes, dev, ws):
 
 
 def chunk_fwd(q, k, v, g, e, w, gamma, S0=None, chunk=64, out_dtype=None,
-              return_chunk_states=False, ws=None):
-    """Chunkwise forward.  Returns ``(o, S_final)`` or, with
-    ``return_chunk_states``, ``(o, S_final, S_chunks)`` where ``S_chunks[b,h,n]``
-    is the state at the start of chunk ``n`` (reusable by :func:`chunk_bwd`)."""
+              return_chunk_states=False, return_saved=False, ws=None):
+    """Chunkwise forward.  Returns ``(o, S_final)``; with ``return_chunk_states``
+    ``(o, S_final, S_chunks)`` where ``S_chunks[b,h,n]`` is the state at the start
+    of chunk ``n``; with ``return_saved`` ``(o, S_final, S_chunks, M_chunks)``
+    where ``M_chunks[b,h,n]`` is chunk n's transition.  Both are reusable by
+    :func:`chunk_bwd`."""
     L = lib()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -155,21 +157,26 @@ def chunk_fwd(q, k, v, g, e, w, gamma, S0=None, chunk=64, out_dtype=None,
     o = torch.empty(B, T, H, dv, dtype=od, device=q.device)
     S_final = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
     Sc = (torch.empty(B, H, T // chunk, dk, dv, dtype=torch.float32, device=q.device)
-          if return_chunk_states else None)
+          if (return_chunk_states or return_saved) else None)
+    Mc = (torch.empty(B, H, T // chunk, dk, dk, dtype=torch.float32, device=q.device)
+          if return_saved else None)
     need = int(L.muir_chunk_fwd_workspace(ctypes.byref(shp)))
     wsb = _workspace(need, q.device, ws)
     rc = L.muir_chunk_fwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(e),
                           _ptr(w), _ptr(gamma), _ptr(S0), _ptr(o), _ptr(S_final), _ptr(Sc),
-                          _ptr(wsb), ctypes.c_size_t(0 if wsb is None else wsb.numel()),
+                          _ptr(Mc), _ptr(wsb), ctypes.c_size_t(0 if wsb is None else wsb.numel()),
                           _stream(q.device))
     _check("muir_chunk_fwd", rc)
+    if return_saved:
+        return o, S_final, Sc, Mc
     return (o, S_final, Sc) if return_chunk_states else (o, S_final)
 
 
 def chunk_bwd(q, k, v, g, e, w, gamma, S0, dO, dS_final=None, chunk=64, S_chunks=None,
-              ws=None):
+              M_chunks=None, ws=None):
     """Gradients of ``sum(o*dO) + sum(S_final*dS_final)``.  Returns a dict with
-    ``dq, dk, dv, dg, de, dw, dgamma`` (input dtype) and ``dS0`` (float32)."""
+    ``dq, dk, dv, dg, de, dw, dgamma`` (input dtype) and ``dS0`` (float32).
+    ``S_chunks`` / ``M_chunks`` from :func:`chunk_fwd` skip recomputation."""
     L = lib()
     shp = _shape(q, v, chunk, None)
     grads = {n: torch.empty_like(x) for n, x in
@@ -179,7 +186,7 @@ def chunk_bwd(q, k, v, g, e, w, gamma, S0, dO, dS_final=None, chunk=64, S_chunks
     need = int(L.muir_chunk_bwd_workspace(ctypes.byref(shp)))
     wsb = _workspace(need, q.device, ws)
     rc = L.muir_chunk_bwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(e),
-                          _ptr(w), _ptr(gamma), _ptr(S0), _ptr(S_chunks), _ptr(dO),
+                          _ptr(w), _ptr(gamma), _ptr(S0), _ptr(S_chunks), _ptr(M_chunks), _ptr(dO),
                           _ptr(dS_final), _ptr(grads["dq"]), _ptr(grads["dk"]),
                           _ptr(grads["dv"]), _ptr(grads["dg"]), _ptr(grads["de"]),
                           _ptr(grads["dw"]), _ptr(grads["dgamma"]), _ptr(grads["dS0"]),
@@ -211,17 +218,17 @@ class MuirChunkFunction(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, g, e, w, gamma, S0, chunk):
-        o, S_final, Sc = chunk_fwd(q, k, v, g, e, w, gamma, S0, chunk=chunk,
-                                   return_chunk_states=True)
-        ctx.save_for_backward(q, k, v, g, e, w, gamma, S0, Sc)
+        o, S_final, Sc, Mc = chunk_fwd(q, k, v, g, e, w, gamma, S0, chunk=chunk,
+                                       return_saved=True)
+        ctx.save_for_backward(q, k, v, g, e, w, gamma, S0, Sc, Mc)
         ctx.chunk = chunk
         return o, S_final
 
     @staticmethod
     def backward(ctx, dO, dS_final):
-        q, k, v, g, e, w, gamma, S0, Sc = ctx.saved_tensors
+        q, k, v, g, e, w, gamma, S0, Sc, Mc = ctx.saved_tensors
         gr = chunk_bwd(q, k, v, g, e, w, gamma, S0, dO.contiguous().to(q.dtype),
                        None if dS_final is None else dS_final.contiguous().float(),
-                       chunk=ctx.chunk, S_chunks=Sc)
+                       chunk=ctx.chunk, S_chunks=Sc, M_chunks=Mc)
         return (gr["dq"], gr["dk"], gr["dv"], gr["dg"], gr["de"], gr["dw"], gr["dgamma"],
                 gr["dS0"] if S0 is not None else None, None)

@@ -83,42 +83,43 @@ size_t muir_chunk_bwd_workspace(const muir_shape* s) {
 
 muir_status muir_chunk_fwd(const muir_shape* s, const void* q, const void* k, const void* v,
                            const void* g, const void* e, const void* w, const void* gamma,
-                           const float* S0, void* o, float* S_final, float* S_chunks, void* ws,
-                           size_t ws_bytes, void* stream) {
+                           const float* S0, void* o, float* S_final, float* S_chunks,
+                           float* M_chunks, void* ws, size_t ws_bytes, void* stream) {
     muir_status st = check_shape(s);
     if (st != MUIR_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
-        !ok_ptr(gamma) || !ok_ptr(o) || !ok_opt(S0) || !ok_opt(S_final) || !ok_opt(S_chunks))
+        !ok_ptr(gamma) || !ok_ptr(o) || !ok_opt(S0) || !ok_opt(S_final) || !ok_opt(S_chunks) ||
+        !ok_opt(M_chunks))
         return MUIR_ERR_INVALID_ARG;
     const size_t need = muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk,
                                                  S_chunks != nullptr);
     if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
     if ((st = check_device()) != MUIR_OK) return st;
     muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);
-    return from_cuda(muir::run_chunk_fwd(P, S0, o, S_final, S_chunks, ws, ws_bytes,
+    return from_cuda(muir::run_chunk_fwd(P, S0, o, S_final, S_chunks, M_chunks, ws, ws_bytes,
                                          static_cast<cudaStream_t>(stream)));
 }
 
 muir_status muir_chunk_bwd(const muir_shape* s, const void* q, const void* k, const void* v,
                            const void* g, const void* e, const void* w, const void* gamma,
-                           const float* S0, const float* S_chunks, const void* dO,
-                           const float* dS_final, void* dq, void* dk, void* dv, void* dg,
-                           void* de, void* dw, void* dgamma, float* dS0, void* ws,
+                           const float* S0, const float* S_chunks, const float* M_chunks,
+                           const void* dO, const float* dS_final, void* dq, void* dk, void* dv,
+                           void* dg, void* de, void* dw, void* dgamma, float* dS0, void* ws,
                            size_t ws_bytes, void* stream) {
     muir_status st = check_shape(s);
     if (st != MUIR_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
         !ok_ptr(gamma) || !ok_ptr(dO) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) ||
         !ok_ptr(dg) || !ok_ptr(de) || !ok_ptr(dw) || !ok_ptr(dgamma) || !ok_opt(S0) ||
-        !ok_opt(S_chunks) || !ok_opt(dS_final) || !ok_opt(dS0))
+        !ok_opt(S_chunks) || !ok_opt(M_chunks) || !ok_opt(dS_final) || !ok_opt(dS0))
         return MUIR_ERR_INVALID_ARG;
     const size_t need = muir::chunk_bwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk,
                                                  S_chunks != nullptr);
     if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
     if ((st = check_device()) != MUIR_OK) return st;
     muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);
-    return from_cuda(muir::run_chunk_bwd(P, S0, S_chunks, dO, dS_final, dq, dk, dv, dg, de, dw,
-                                         dgamma, dS0, ws, ws_bytes,
+    return from_cuda(muir::run_chunk_bwd(P, S0, S_chunks, M_chunks, dO, dS_final, dq, dk, dv, dg,
+                                         de, dw, dgamma, dS0, ws, ws_bytes,
                                          static_cast<cudaStream_t>(stream)));
 }
 

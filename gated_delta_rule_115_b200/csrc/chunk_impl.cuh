@@ -1,0 +1,845 @@
+// chunk.cu -- chunkwise-parallel forward and backward of the Muir gated delta
+// rule ("Muir: Linear Attention with Sensitivity-Allocated Gating and
+// Matched-Filter Readout", arXiv 2611.08376; wolonglab.org page, section
+// "Methodology" and fig:kernel).
+//
+// Per chunk of C tokens with chunk-start state S (d = dk = dv, rows of S are
+// key channels), with Gam_t = sum_{i<=t} g_i inside the chunk, gbar = Gam_{C-1}:
+//
+//   [X (*) Z]_{ts} = sum_j X_tj Z_sj exp(Gam_tj - Gam_sj)          (s <= t)
+//   L_A = strict(K (*) A), L_K = strict(K (*) K),  A = e*K, U = w*V, Qh = gamma*Q
+//   M_QK = incl(Qh (*) K), M_QA = incl(Qh (*) A),  T = (I + L_A)^{-1}
+//   Y  = T (Kt S + L_K U),            Kt = K e^Gam      (y_t = k_t^T D_t S_{t-1})
+//   O  = Qt S + M_QK U - M_QA Y,      Qt = Qh e^Gam
+//   S' = diag(e^gbar) S + Kb^T U - Ab^T Y,   Kb = K e^{gbar-Gam}, Ab = A e^{gbar-Gam}
+//
+// Eliminating Y gives the chunk transition S' = M S + Bn with
+//   Psi = T^T Ab,  M = diag(e^gbar) - Psi^T Kt,  Bn = (Kb - L_K^T Psi)^T U,
+// so the sequential pass over chunks is one d x d x d product per chunk.
+//
+// Boundary pivots (fig:kernel "boundary-pivoted"): every exponential applied to
+// an operand is <= 1, except inside a diagonal 8-token block, where the pivot is
+// the block's 4th token and factors stay below exp(4 * 20) thanks to the clamp
+// g >= -20.  With 8-token blocks rb and J (rb > J), e(J) = last token of J and
+// b(rb) = token before rb:
+//   exp(Gam_t - Gam_s) = [exp(Gam_t - Gam_b(rb))] [exp(Gam_b(rb) - Gam_e(J))] [exp(Gam_e(J) - Gam_s)]
+//                      =        x8f_t          *        F[rb][J]            *      z8f_s
+// and inside one block with mid pivot m: exp(Gam_t - Gam_m) * exp(Gam_m - Gam_s) = xof_t * zof_s.
+//
+// Kernels (one CTA of 256 threads per chunk, persistent over chunks, with a
+// private float32 scratch slot in the workspace that stays resident in L2):
+//   k_intra : M, Bn per chunk                         (parallel over chunks)
+//   k_chain : S_{n+1} = M_n S_n + Bn_n, or its transpose for the gradient
+//             (sequential over chunks, parallel over (b, h, column slabs))
+//   k_out   : O per chunk from the chunk-start state  (parallel)
+//   k_bprep : B'_n = Qt^T dO - Kt^T T^T M_QA^T dO      (parallel)
+//   k_bwd   : all input gradients per chunk            (parallel)
+// Products run on tensor cores (TF32 mma.sync, float32 accumulate; three
+// split-TF32 passes for float32 inputs).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "mma.cuh"
+#include "tc.cuh"
+#include "profile.h"
+
+namespace muir {
+
+constexpr int kThreads = 256;
+constexpr int kMaxSlots = 296;  // 2 CTAs per SM on a 148-SM B200
+
+// ------------------------------------------------------------------ scratch
+
+struct Lay {
+    int C, D, nb8, nb16;
+    size_t LC, RC, BT, PRE, SUF, GBAR, LA, LK, MQK, MQA, TII, W[8], total;
+};
+
+__host__ __device__ inline Lay make_lay(int C, int D) {
+    Lay L;
+    L.C = C; L.D = D; L.nb8 = C / 8; L.nb16 = C / 16;
+    const size_t cd = (size_t)C * D, cc = (size_t)C * C, bd = (size_t)(C / 8) * D;
+    size_t o = 0;
+#define MUIR_TAKE(field, n) L.field = o; o += ((size_t)(n) + 63) & ~(size_t)63;
+    MUIR_TAKE(LC, cd) MUIR_TAKE(RC, cd) MUIR_TAKE(BT, bd) MUIR_TAKE(PRE, bd) MUIR_TAKE(SUF, bd)
+    MUIR_TAKE(GBAR, D)
+    MUIR_TAKE(LA, cc) MUIR_TAKE(LK, cc) MUIR_TAKE(MQK, cc) MUIR_TAKE(MQA, cc)
+    MUIR_TAKE(TII, (size_t)C * 16)
+    for (int i = 0; i < 8; ++i) { MUIR_TAKE(W[i], cd) }
+#undef MUIR_TAKE
+    L.total = o;
+    return L;
+}
+
+// ------------------------------------------------------------------ params
+
+struct KParams {
+    int B, T, H, C, N;
+    const void *q, *k, *v, *g, *e, *w, *gamma, *dO;
+    const float* S_chunks;   // chunk-start states   [B,H,N,D,D]
+    const float* dS_chunks;  // gradient at chunk end [B,H,N,D,D]
+    float* M;                // transition           [B,H,N,D,D]
+    float* Bn;               // affine term          [B,H,N,D,D]
+    void* o;
+    void *dq, *dk, *dv, *dg, *de, *dw, *dgamma;
+    float* scratch;
+    size_t slot;             // floats per scratch slot
+};
+
+// Accessors of one chunk's inputs; row t of a [B,T,H,D] tensor.
+template <typename Tin, int D>
+struct Chunk {
+    const Tin *q, *k, *v, *g, *e, *w, *gm, *dO;
+    size_t rs, base, sbase;  // row stride (H*D), element offset of row 0, state offset
+    float* s;                // scratch slot
+    Lay L;
+    __device__ float K(int t, int j) const { return ldf(k + base + t * rs + j); }
+    __device__ float Qh(int t, int j) const {
+        return ldf(gm + base + t * rs + j) * ldf(q + base + t * rs + j);
+    }
+    __device__ float A(int t, int j) const {
+        return ldf(e + base + t * rs + j) * ldf(k + base + t * rs + j);
+    }
+    __device__ float U(int t, int c) const {
+        return ldf(w + base + t * rs + c) * ldf(v + base + t * rs + c);
+    }
+    __device__ float dOv(int t, int c) const { return ldf(dO + base + t * rs + c); }
+    __device__ float& at(size_t off, int r, int c) const { return s[off + (size_t)r * D + c]; }
+};
+
+template <typename Tin, int D>
+__device__ Chunk<Tin, D> make_chunk(const KParams& p, int chunk, float* slot) {
+    Chunk<Tin, D> c;
+    const int n = chunk % p.N, bh = chunk / p.N, h = bh % p.H, b = bh / p.H;
+    c.q = (const Tin*)p.q; c.k = (const Tin*)p.k; c.v = (const Tin*)p.v; c.g = (const Tin*)p.g;
+    c.e = (const Tin*)p.e; c.w = (const Tin*)p.w; c.gm = (const Tin*)p.gamma;
+    c.dO = (const Tin*)p.dO;
+    c.rs = (size_t)p.H * D;
+    c.base = (((size_t)b * p.T + (size_t)n * p.C) * p.H + h) * D;
+    c.sbase = ((size_t)bh * p.N + n) * D * D;
+    c.s = slot;
+    c.L = make_lay(p.C, D);
+    return c;
+}
+
+// ------------------------------------------------------------------ masked products
+
+// Operand kinds for the masked products.
+enum Opnd { OP_K = 0, OP_Q = 1, OP_A = 2 };
+
+template <typename Tin, int D>
+__device__ __forceinline__ float opval(const Chunk<Tin, D>& c, int kind, int t, int j) {
+    return kind == OP_K ? c.K(t, j) : (kind == OP_Q ? c.Qh(t, j) : c.A(t, j));
+}
+
+#include "staged.cuh"
+
+// ------------------------------------------------------------------ triangular solves
+
+// T_II = (I + L_II)^{-1} for every 16 x 16 diagonal block of the unit lower
+// triangular I + L (forward substitution, float32).
+__device__ inline void compute_tii(float* s, const Lay& L, size_t Loff) {
+    const int C = L.C, warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    for (int blk = warp; blk < L.nb16; blk += kThreads / 32) {
+        const int b0 = 16 * blk;
+        if (lane < 16) {
+            const int col = lane;
+            float x[16];
+#pragma unroll
+            for (int r = 0; r < 16; ++r) {
+                float acc = (r == col) ? 1.f : 0.f;
+#pragma unroll
+                for (int q = 0; q < r; ++q) acc -= s[Loff + (size_t)(b0 + r) * C + b0 + q] * x[q];
+                x[r] = (r < col) ? 0.f : acc;
+            }
+#pragma unroll
+            for (int r = 0; r < 16; ++r) s[L.TII + ((size_t)blk * 16 + r) * 16 + col] = x[r];
+        }
+    }
+}
+
+// ------------------------------------------------------------------ tensor-core helpers
+
+// Four consecutive float32 scratch elements (16-byte aligned).
+__device__ __forceinline__ void ld4(const float* p, float* v) {
+    const float4 x = *reinterpret_cast<const float4*>(p);
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+// Four consecutive input elements (8- or 16-byte aligned).
+__device__ __forceinline__ void ld4in(const float* p, float* v) {
+    const float4 x = __ldg(reinterpret_cast<const float4*>(p));
+    v[0] = x.x; v[1] = x.y; v[2] = x.z; v[3] = x.w;
+}
+__device__ __forceinline__ void ld4in(const __nv_bfloat16* p, float* v) {
+    const uint2 x = __ldg(reinterpret_cast<const uint2*>(p));
+    const __nv_bfloat162 a = *reinterpret_cast<const __nv_bfloat162*>(&x.x);
+    const __nv_bfloat162 b = *reinterpret_cast<const __nv_bfloat162*>(&x.y);
+    const float2 fa = __bfloat1622float2(a), fb = __bfloat1622float2(b);
+    v[0] = fa.x; v[1] = fa.y; v[2] = fb.x; v[3] = fb.y;
+}
+
+// Tensor-core state shared by one CTA's products (TMEM columns, mbarrier).
+struct TcCta {
+    tc::State st;
+    unsigned char* sbuf;
+};
+
+constexpr int kTmemCols = 128;
+
+// Product over M rows (looped in 128-row tiles) and N = NT columns.
+template <int PASSES, int N, bool AR, bool BR, class FA4, class FB4, class EPI>
+__device__ __forceinline__ void tc_rows(TcCta& t, int M, int K, const FA4& fa4, const FB4& fb4,
+                                        const EPI& epi) {
+    for (int m0 = 0; m0 < M; m0 += 128) {
+        const int Mt = M - m0 < 128 ? M - m0 : 128;
+        tc::gemm<PASSES, N, AR, BR>(
+            t.st, t.sbuf, Mt, K, [&](int m, int k, float* v) { fa4(m0 + m, k, v); }, fb4,
+            [&](int m, int n, float x) { epi(m0 + m, n, x); });
+    }
+}
+
+// Same, storing raw rows (vectorised) into a row-major destination.
+template <int PASSES, int N, bool AR, bool BR, class FA4, class FB4>
+__device__ __forceinline__ void tc_rows(TcCta& t, int M, int K, const FA4& fa4, const FB4& fb4,
+                                        tc::RowStore dst) {
+    for (int m0 = 0; m0 < M; m0 += 128) {
+        const int Mt = M - m0 < 128 ? M - m0 : 128;
+        tc::RowStore d = {dst.dst + (size_t)m0 * dst.ld, dst.ld};
+        tc::gemm<PASSES, N, AR, BR>(
+            t.st, t.sbuf, Mt, K, [&](int m, int k, float* v) { fa4(m0 + m, k, v); }, fb4, d);
+    }
+}
+
+// ------------------------------------------------------------------ k_intra
+
+template <typename Tin, int D, int PASSES>
+__global__ void __launch_bounds__(kThreads) k_intra(KParams p) {
+    __shared__ uint32_t tmem_slot;
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ int tc_status;
+    extern __shared__ __align__(128) unsigned char dsm[];
+    TcCta tcx;
+    tcx.sbuf = dsm;
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    float* sm = reinterpret_cast<float*>(dsm);
+    float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
+    const int nch = p.B * p.H * p.N;
+    for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
+        const Chunk<Tin, D> c = make_chunk<Tin, D>(p, chunk, slot);
+        const Lay& L = c.L;
+        const int C = L.C;
+        float* s = c.s;
+        prologue2(c);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
+        __syncthreads();
+        compute_tii(s, L, L.LA);
+        for (int idx = threadIdx.x; idx < C * D; idx += kThreads)
+            s[L.W[0] + idx] = c.A(idx / D, idx % D) * facs(c).egb(idx / D, idx % D);  // Ab
+        __syncthreads();
+        solve_s<D, PASSES, true>(s, sm, L, L.LA, L.W[0]);  // Psi = T^T Ab
+        __syncthreads();
+        float* M = p.M + c.sbase;
+        const float* Psi = s + L.W[0];
+        const Fac<Tin, D> f = facs(c);
+        // M = diag(e^gbar) - Psi^T Kt      (rows i, contraction over tokens)
+        tc_rows<PASSES, D, true, true>(tcx, D, C,
+            [&](int i, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = Psi[(size_t)(t + u) * D + i]; },
+            [&](int j, int t, float* v) {
+                for (int u = 0; u < 4; ++u) v[u] = c.K(t + u, j) * f.eg(t + u, j);
+            },
+            [&](int i, int j, float x) {
+                const float d = (i == j) ? expf(f.gbar(i)) : 0.f;
+                M[(size_t)i * D + j] = d - x;
+            });
+        // Phi = Kb - L_K^T Psi              (rows t, contraction over tokens s)
+        float* Phi = s + L.W[1];
+        tc_rows<PASSES, D, true, true>(tcx, C, C,
+            [&](int t, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = s[L.LK + (size_t)(k + u) * C + t]; },
+            [&](int j, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = Psi[(size_t)(k + u) * D + j]; },
+            [&](int t, int j, float x) { Phi[(size_t)t * D + j] = c.K(t, j) * f.egb(t, j) - x; });
+        // Bn = Phi^T U
+        float* Bn = p.Bn + c.sbase;
+        tc_rows<PASSES, D, true, true>(tcx, D, C,
+            [&](int i, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = Phi[(size_t)(t + u) * D + i]; },
+            [&](int cc, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = c.U(t + u, cc); },
+            tc::RowStore{Bn, D});
+    }
+    tc::release(tcx.st, kTmemCols);
+}
+
+// ------------------------------------------------------------------ k_chain
+
+// Sequential pass over chunks for one (b, h) and a slab of SLAB columns.
+// Forward (REV = false): S_{n+1} = M_n S_n + Bn_n, records S_n.
+// Reverse (REV = true):  G_n = M_n^T G_{n+1} + Bn_n, records G_{n+1}.
+template <int D, int SLAB, int PASSES, bool REV>
+__global__ void __launch_bounds__(kThreads) k_chain(const float* __restrict__ M,
+                                                    const float* __restrict__ Bn,
+                                                    const float* __restrict__ S_in,
+                                                    float* __restrict__ S_rec,
+                                                    float* __restrict__ S_out, int N) {
+    constexpr int NT = SLAB / 8 < 4 ? SLAB / 8 : 4;
+    __shared__ float buf[2][D * SLAB];
+    constexpr int NSLAB = D / SLAB;
+    const int bh = blockIdx.x / NSLAB, c0 = (blockIdx.x % NSLAB) * SLAB;
+    const size_t DD = (size_t)D * D;
+    for (int idx = threadIdx.x; idx < D * SLAB; idx += kThreads) {
+        const int i = idx / SLAB, cc = idx % SLAB;
+        buf[0][idx] = S_in ? S_in[bh * DD + (size_t)i * D + c0 + cc] : 0.f;
+    }
+    __syncthreads();
+    int cur = 0;
+    for (int step = 0; step < N; ++step) {
+        const int n = REV ? N - 1 - step : step;
+        const size_t off = ((size_t)bh * N + n) * DD;
+        if (S_rec)
+            for (int idx = threadIdx.x; idx < D * SLAB; idx += kThreads)
+                S_rec[off + (size_t)(idx / SLAB) * D + c0 + idx % SLAB] = buf[cur][idx];
+        const float* Mn = M + off;
+        const float* Bb = Bn + off;
+        const float* Sc = buf[cur];
+        float* Sn = buf[cur ^ 1];
+        cta_tiles<NT>(D, SLAB,
+            [&](float (&acc)[1][NT][4], int m0, int n0) {
+                warp_gemm<PASSES, 1, NT>(acc, D,
+                    [&](int r, int k) {
+                        return REV ? __ldg(Mn + (size_t)k * D + m0 + r)
+                                   : __ldg(Mn + (size_t)(m0 + r) * D + k);
+                    },
+                    [&](int k, int n) { return Sc[k * SLAB + n0 + n]; });
+            },
+            [&](int i, int cc, float v) { Sn[i * SLAB + cc] = v + __ldg(Bb + (size_t)i * D + c0 + cc); });
+        __syncthreads();
+        cur ^= 1;
+    }
+    if (S_out)
+        for (int idx = threadIdx.x; idx < D * SLAB; idx += kThreads)
+            S_out[bh * DD + (size_t)(idx / SLAB) * D + c0 + idx % SLAB] = buf[cur][idx];
+}
+
+// ------------------------------------------------------------------ k_out
+
+// Y = T (Kt S + L_K U) into scratch at Yoff (needs LA, LK, TII).
+template <typename Tin, int D, int PASSES>
+__device__ void compute_Y(TcCta& tcx, const Chunk<Tin, D>& c, const float* S, size_t Yoff) {
+    const Lay& L = c.L;
+    const int C = L.C;
+    float* s = c.s;
+    const Fac<Tin, D> f = facs(c);
+    tc_rows<PASSES, D, false, true>(tcx, C, D + C,
+        [&](int t, int k, float* v) {
+            if (k < D) {
+                ld4in(c.k + c.base + t * c.rs + k, v);
+                for (int u = 0; u < 4; ++u) v[u] *= f.eg(t, k + u);
+            } else {
+                ld4(s + L.LK + (size_t)t * C + (k - D), v);
+            }
+        },
+        [&](int cc, int k, float* v) {
+            if (k < D) for (int u = 0; u < 4; ++u) v[u] = __ldg(S + (size_t)(k + u) * D + cc);
+            else for (int u = 0; u < 4; ++u) v[u] = c.U(k - D + u, cc);
+        },
+        tc::RowStore{s + Yoff, D});
+    solve_s<D, PASSES, false>(s, reinterpret_cast<float*>(tcx.sbuf), L, L.LA, Yoff);
+    __syncthreads();
+}
+
+template <typename Tin, typename Tout, int D, int PASSES>
+__global__ void __launch_bounds__(kThreads) k_out(KParams p) {
+    __shared__ uint32_t tmem_slot;
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ int tc_status;
+    extern __shared__ __align__(128) unsigned char dsm[];
+    TcCta tcx;
+    tcx.sbuf = dsm;
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    float* sm = reinterpret_cast<float*>(dsm);
+    float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
+    const int nch = p.B * p.H * p.N;
+    for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
+        const Chunk<Tin, D> c = make_chunk<Tin, D>(p, chunk, slot);
+        const Lay& L = c.L;
+        const int C = L.C;
+        float* s = c.s;
+        prologue2(c);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
+        __syncthreads();
+        compute_tii(s, L, L.LA);
+        __syncthreads();
+        const float* S = p.S_chunks + c.sbase;
+        compute_Y<Tin, D, PASSES>(tcx, c, S, L.W[0]);
+        Tout* o = (Tout*)p.o;
+        const Fac<Tin, D> f = facs(c);
+        const float* Y = s + L.W[0];
+        // O = Qt S + M_QK U - M_QA Y
+        tc_rows<PASSES, D, false, true>(tcx, C, D + 2 * C,
+            [&](int t, int k, float* v) {
+                if (k < D) {
+                    float g4[4];
+                    ld4in(c.q + c.base + t * c.rs + k, v);
+                    ld4in(c.gm + c.base + t * c.rs + k, g4);
+                    for (int u = 0; u < 4; ++u) v[u] *= g4[u] * f.eg(t, k + u);
+                } else if (k < D + C) {
+                    ld4(s + L.MQK + (size_t)t * C + (k - D), v);
+                } else {
+                    ld4(s + L.MQA + (size_t)t * C + (k - D - C), v);
+                    for (int u = 0; u < 4; ++u) v[u] = -v[u];
+                }
+            },
+            [&](int cc, int k, float* v) {
+                if (k < D) for (int u = 0; u < 4; ++u) v[u] = __ldg(S + (size_t)(k + u) * D + cc);
+                else if (k < D + C) for (int u = 0; u < 4; ++u) v[u] = c.U(k - D + u, cc);
+                else for (int u = 0; u < 4; ++u) v[u] = Y[(size_t)(k - D - C + u) * D + cc];
+            },
+            [&](int t, int j, float x) { stf(o + c.base + t * c.rs + j, x); });
+    }
+    tc::release(tcx.st, kTmemCols);
+}
+
+// ------------------------------------------------------------------ k_bprep
+
+template <typename Tin, int D, int PASSES>
+__global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
+    __shared__ uint32_t tmem_slot;
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ int tc_status;
+    extern __shared__ __align__(128) unsigned char dsm[];
+    TcCta tcx;
+    tcx.sbuf = dsm;
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    float* sm = reinterpret_cast<float*>(dsm);
+    float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
+    const int nch = p.B * p.H * p.N;
+    for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
+        const Chunk<Tin, D> c = make_chunk<Tin, D>(p, chunk, slot);
+        const Lay& L = c.L;
+        const int C = L.C;
+        float* s = c.s;
+        prologue2(c);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
+        __syncthreads();
+        compute_tii(s, L, L.LA);
+        __syncthreads();
+        float* Xi = s + L.W[0];
+        // Z0 = M_QA^T dO
+        tc_rows<PASSES, D, true, true>(tcx, C, C,
+            [&](int t, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = s[L.MQA + (size_t)(k + u) * C + t]; },
+            [&](int cc, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc); },
+            tc::RowStore{Xi, D});
+        solve_s<D, PASSES, true>(s, sm, L, L.LA, L.W[0]);  // Xi = T^T Z0
+        __syncthreads();
+        float* Bp = p.Bn + c.sbase;
+        const Fac<Tin, D> f = facs(c);
+        // B' = Qt^T dO - Kt^T Xi
+        tc_rows<PASSES, D, true, true>(tcx, D, 2 * C,
+            [&](int i, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.Qh(k + u, i) * f.eg(k + u, i);
+                else for (int u = 0; u < 4; ++u) v[u] = -c.K(k - C + u, i) * f.eg(k - C + u, i);
+            },
+            [&](int cc, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc);
+                else for (int u = 0; u < 4; ++u) v[u] = Xi[(size_t)(k - C + u) * D + cc];
+            },
+            tc::RowStore{Bp, D});
+    }
+    tc::release(tcx.st, kTmemCols);
+}
+
+// ------------------------------------------------------------------ k_bwd
+
+template <typename Tin, int D, int PASSES>
+__global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
+    __shared__ float s_colsum[D];
+    __shared__ float s_segtot[kThreads];
+    __shared__ float s_red[kThreads * 4];
+    __shared__ uint32_t tmem_slot;
+    __shared__ __align__(8) uint64_t mbar;
+    __shared__ int tc_status;
+    extern __shared__ __align__(128) unsigned char dsm[];
+    TcCta tcx;
+    tcx.sbuf = dsm;
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    float* sm = reinterpret_cast<float*>(dsm);
+    float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
+    const int nch = p.B * p.H * p.N;
+    for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
+        const Chunk<Tin, D> c = make_chunk<Tin, D>(p, chunk, slot);
+        const Lay& L = c.L;
+        const int C = L.C;
+        float* s = c.s;
+        const float* S = p.S_chunks + c.sbase;
+        const float* dS = p.dS_chunks + c.sbase;
+        const size_t Y = L.W[0], dR = L.W[1], dK = L.W[2], dQh = L.W[3], dA = L.W[4],
+                     dU = L.W[5], dGam = L.W[6];
+        prologue2(c);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
+        masked_pair_s<Tin, D, PASSES>(c, sm, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
+        __syncthreads();
+        compute_tii(s, L, L.LA);
+        __syncthreads();
+        compute_Y<Tin, D, PASSES>(tcx, c, S, Y);
+        const Fac<Tin, D> f = facs(c);
+        // dY = -M_QA^T dO - Ab dS'   (stored in dR, then dR = T^T dY)
+        tc_rows<PASSES, D, true, true>(tcx, C, C + D,
+            [&](int t, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = s[L.MQA + (size_t)(k + u) * C + t];
+                else {
+                    float k4[4];
+                    ld4in(c.e + c.base + t * c.rs + (k - C), v);
+                    ld4in(c.k + c.base + t * c.rs + (k - C), k4);
+                    for (int u = 0; u < 4; ++u) v[u] *= k4[u] * f.egb(t, k - C + u);
+                }
+            },
+            [&](int cc, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc);
+                else for (int u = 0; u < 4; ++u) v[u] = __ldg(dS + (size_t)(k - C + u) * D + cc);
+            },
+            [&](int t, int j, float x) { s[dR + (size_t)t * D + j] = -x; });
+        solve_s<D, PASSES, true>(s, sm, L, L.LA, dR);  // dR = T^T dY
+        __syncthreads();
+        // B(k = c, n = j) = S[j][c] or dS'[j][c]: rows of the staged B are rows of S
+        auto rowsS = [&](int j, int k, float* v) { ld4in(S + (size_t)j * D + k, v); };
+        auto rowsdS = [&](int j, int k, float* v) { ld4in(dS + (size_t)j * D + k, v); };
+        // raw products, then one elementwise pass applies the decay factors:
+        //   dQt = dO S^T, dKt = dR S^T, dKb = U dS'^T, dAb = -Y dS'^T
+        tc_rows<PASSES, D, false, false>(tcx, C, D,
+            [&](int t, int k, float* v) { ld4in(c.dO + c.base + t * c.rs + k, v); }, rowsS,
+            tc::RowStore{s + dQh, D});
+        tc_rows<PASSES, D, false, false>(tcx, C, D,
+            [&](int t, int k, float* v) { ld4(s + dR + (size_t)t * D + k, v); }, rowsS,
+            tc::RowStore{s + dK, D});
+        tc_rows<PASSES, D, false, false>(tcx, C, D,
+            [&](int t, int k, float* v) {
+                float w4[4];
+                ld4in(c.v + c.base + t * c.rs + k, v);
+                ld4in(c.w + c.base + t * c.rs + k, w4);
+                for (int u = 0; u < 4; ++u) v[u] *= w4[u];
+            },
+            rowsdS, tc::RowStore{s + dGam, D});
+        tc_rows<PASSES, D, false, false>(tcx, C, D,
+            [&](int t, int k, float* v) {
+                ld4(s + Y + (size_t)t * D + k, v);
+                for (int u = 0; u < 4; ++u) v[u] = -v[u];
+            },
+            rowsdS, tc::RowStore{s + dA, D});
+        float cpart[4] = {0.f, 0.f, 0.f, 0.f};  // this thread's share of the column sums
+        // dQh = dQt e^Gam;  dK = dKt e^Gam + dKb e^{gbar-Gam};  dA = dAb e^{gbar-Gam};
+        // dGam = dQt Qt + dKt Kt - dKb Kb - dAb Ab;  dgbar += sum_t (dKb Kb + dAb Ab)
+        for (int idx = threadIdx.x; idx < C * D / 4; idx += kThreads) {
+            const int t = idx / (D / 4), j = 4 * (idx % (D / 4));
+            const size_t i = (size_t)t * D + j;
+            float r1[4], r2[4], r3[4], r4[4], lc[4], rc[4], pre[4], suf[4], q4[4], gm4[4], k4[4], e4[4];
+            ld4(s + dQh + i, r1); ld4(s + dK + i, r2); ld4(s + dGam + i, r3); ld4(s + dA + i, r4);
+            ld4(s + L.LC + i, lc); ld4(s + L.RC + i, rc);
+            ld4(s + L.PRE + (size_t)(t >> 3) * D + j, pre); ld4(s + L.SUF + (size_t)(t >> 3) * D + j, suf);
+            const size_t gi = c.base + t * c.rs + j;
+            ld4in(c.q + gi, q4); ld4in(c.gm + gi, gm4); ld4in(c.k + gi, k4); ld4in(c.e + gi, e4);
+            float o1[4], o2[4], o3[4], o4[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float eg = fexp<Tin>(pre[u] + lc[u]), egb = fexp<Tin>(rc[u] + suf[u]);
+                const float kt = k4[u] * eg, qt = q4[u] * gm4[u] * eg;
+                const float kb = k4[u] * egb, ab = e4[u] * k4[u] * egb;
+                o1[u] = r1[u] * eg;
+                o2[u] = r2[u] * eg + r3[u] * egb;
+                o4[u] = r4[u] * egb;
+                o3[u] = r1[u] * qt + r2[u] * kt - r3[u] * kb - r4[u] * ab;
+                cpart[u] += r3[u] * kb + r4[u] * ab;
+            }
+            *reinterpret_cast<float4*>(s + dQh + i) = make_float4(o1[0], o1[1], o1[2], o1[3]);
+            *reinterpret_cast<float4*>(s + dK + i) = make_float4(o2[0], o2[1], o2[2], o2[3]);
+            *reinterpret_cast<float4*>(s + dGam + i) = make_float4(o3[0], o3[1], o3[2], o3[3]);
+            *reinterpret_cast<float4*>(s + dA + i) = make_float4(o4[0], o4[1], o4[2], o4[3]);
+        }
+        // column sums in a fixed order (deterministic): every thread always saw the
+        // same 4 channels, 4 * (threadIdx % (D/4)) .. + 3
+#pragma unroll
+        for (int u = 0; u < 4; ++u) s_red[threadIdx.x * 4 + u] = cpart[u];
+        __syncthreads();
+        if (threadIdx.x < D) {
+            const int jg = threadIdx.x / 4, u = threadIdx.x % 4;
+            float acc = 0.f;
+            for (int th = jg; th < kThreads; th += D / 4) acc += s_red[th * 4 + u];
+            s_colsum[threadIdx.x] = acc;
+        }
+        __syncthreads();
+        // dU = M_QK^T dO + L_K^T dR + Kb dS'
+        tc_rows<PASSES, D, true, true>(tcx, C, 2 * C + D,
+            [&](int t, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = s[L.MQK + (size_t)(k + u) * C + t];
+                else if (k < 2 * C) for (int u = 0; u < 4; ++u) v[u] = s[L.LK + (size_t)(k - C + u) * C + t];
+                else {
+                    ld4in(c.k + c.base + t * c.rs + (k - 2 * C), v);
+                    for (int u = 0; u < 4; ++u) v[u] *= f.egb(t, k - 2 * C + u);
+                }
+            },
+            [&](int cc, int k, float* v) {
+                if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc);
+                else if (k < 2 * C) for (int u = 0; u < 4; ++u) v[u] = s[dR + (size_t)(k - C + u) * D + cc];
+                else for (int u = 0; u < 4; ++u) v[u] = __ldg(dS + (size_t)(k - 2 * C + u) * D + cc);
+            },
+            tc::RowStore{s + dU, D});
+        // gradients of the masked products (overwrite them): dL_A = -strict(dR Y^T),
+        // dL_K = strict(dR U^T), dM_QK = incl(dO U^T), dM_QA = -incl(dO Y^T)
+        for (int which = 0; which < 4; ++which) {
+            const size_t out = which == 0 ? L.LA : which == 1 ? L.LK : which == 2 ? L.MQK : L.MQA;
+            const bool incl = which >= 2;
+            const float sg = (which == 0 || which == 3) ? -1.f : 1.f;
+            for (int n0 = 0; n0 < C; n0 += 128) {
+                tc_rows<PASSES, 128, false, false>(tcx, C, D,
+                    [&](int t, int k, float* v) {
+                        if (which < 2) ld4(s + dR + (size_t)t * D + k, v);
+                        else ld4in(c.dO + c.base + t * c.rs + k, v);
+                    },
+                    [&](int n, int k, float* v) {
+                        const int ss = n0 + n;
+                        if (ss >= C) { v[0] = v[1] = v[2] = v[3] = 0.f; return; }
+                        if (which == 0 || which == 3) ld4(s + Y + (size_t)ss * D + k, v);
+                        else {
+                            float w4[4];
+                            ld4in(c.v + c.base + ss * c.rs + k, v);
+                            ld4in(c.w + c.base + ss * c.rs + k, w4);
+                            for (int u = 0; u < 4; ++u) v[u] *= w4[u];
+                        }
+                    },
+                    [&](int t, int n, float x) {
+                        const int ss = n0 + n;
+                        if (ss >= C) return;
+                        const bool keep = incl ? ss <= t : ss < t;
+                        s[out + (size_t)t * C + ss] = keep ? sg * x : 0.f;
+                    });
+            }
+        }
+        __syncthreads();
+        // X side: dK += dL_A (*) A + dL_K (*) K ; dQh += dM_QK (*) K + dM_QA (*) A ; dGam += X * dX
+        decayed_grad_any<Tin, D, PASSES, true>(c, sm, L.LA, OP_A, L.LK, OP_K, [&](int t, int j, float v) {
+            const size_t x = (size_t)t * D + j;
+            s[dK + x] += v;
+            s[dGam + x] += c.K(t, j) * v;
+        });
+        decayed_grad_any<Tin, D, PASSES, true>(c, sm, L.MQK, OP_K, L.MQA, OP_A, [&](int t, int j, float v) {
+            const size_t x = (size_t)t * D + j;
+            s[dQh + x] += v;
+            s[dGam + x] += c.Qh(t, j) * v;
+        });
+        __syncthreads();
+        // Z side: dA += dL_A^T (*) K + dM_QA^T (*) Qh ; dK += dL_K^T (*) K + dM_QK^T (*) Qh ; dGam -= Z * dZ
+        decayed_grad_any<Tin, D, PASSES, false>(c, sm, L.LA, OP_K, L.MQA, OP_Q, [&](int t, int j, float v) {
+            const size_t x = (size_t)t * D + j;
+            s[dA + x] += v;
+            s[dGam + x] -= c.A(t, j) * v;
+        });
+        __syncthreads();
+        decayed_grad_any<Tin, D, PASSES, false>(c, sm, L.LK, OP_K, L.MQK, OP_Q, [&](int t, int j, float v) {
+            const size_t x = (size_t)t * D + j;
+            s[dK + x] += v;
+            s[dGam + x] -= c.K(t, j) * v;
+        });
+        __syncthreads();
+        // dgbar_j = e^gbar_j sum_c S[j][c] dS'[j][c] + sum_t (dKb Kb + dAb Ab)[t][j]
+        Tin* gq = (Tin*)p.dq; Tin* gk = (Tin*)p.dk; Tin* gv = (Tin*)p.dv; Tin* gg = (Tin*)p.dg;
+        Tin* ge = (Tin*)p.de; Tin* gw = (Tin*)p.dw; Tin* ggm = (Tin*)p.dgamma;
+        {
+            const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+            for (int j = warp; j < D; j += kThreads / 32) {
+                float acc = 0.f;
+                for (int cc = lane; cc < D; cc += 32)
+                    acc += __ldg(S + (size_t)j * D + cc) * __ldg(dS + (size_t)j * D + cc);
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+                if (lane == 0) s_colsum[j] += acc * expf(facs(c).gbar(j));
+            }
+        }
+        __syncthreads();
+        // dg_t = dgbar + sum_{t' >= t} dGam[t'] : token segments per thread, segment
+        // totals combined through shared memory
+        {
+            constexpr int SEG = kThreads / D;
+            const int j = threadIdx.x % D, seg = threadIdx.x / D, len = C / SEG;
+            const int t0 = seg * len;
+            float tot = 0.f;
+            for (int t = t0; t < t0 + len; t += 8) {
+                float v8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v8[u] = s[dGam + (size_t)(t + u) * D + j];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) tot += v8[u];
+            }
+            s_segtot[seg * D + j] = tot;
+            __syncthreads();
+            float run = s_colsum[j];
+            for (int sg = seg + 1; sg < SEG; ++sg) run += s_segtot[sg * D + j];
+            for (int t1 = t0 + len - 8; t1 >= t0; t1 -= 8) {
+                float v8[8], g8[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    v8[u] = s[dGam + (size_t)(t1 + u) * D + j];
+                    g8[u] = ldf(c.g + c.base + (size_t)(t1 + u) * c.rs + j);
+                }
+#pragma unroll
+                for (int u = 7; u >= 0; --u) {
+                    run += v8[u];
+                    stf(gg + c.base + (size_t)(t1 + u) * c.rs + j, g8[u] >= kLogDecayMin ? run : 0.f);
+                }
+            }
+        }
+        for (int idx = threadIdx.x; idx < C * D / 4; idx += kThreads) {
+            const int t = idx / (D / 4), j = 4 * (idx % (D / 4));
+            const size_t gi = c.base + t * c.rs + j;
+            const size_t li = (size_t)t * D + j;
+            float qv[4], gmv[4], kv[4], ev[4], vv[4], wv[4], dqh[4], da[4], du[4], dk4[4];
+            ld4in(c.q + gi, qv); ld4in(c.gm + gi, gmv); ld4in(c.k + gi, kv);
+            ld4in(c.e + gi, ev); ld4in(c.v + gi, vv); ld4in(c.w + gi, wv);
+            ld4(s + dQh + li, dqh); ld4(s + dA + li, da); ld4(s + dU + li, du); ld4(s + dK + li, dk4);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                stf(gq + gi + u, dqh[u] * gmv[u]);
+                stf(ggm + gi + u, dqh[u] * qv[u]);
+                stf(ge + gi + u, da[u] * kv[u]);
+                stf(gk + gi + u, dk4[u] + da[u] * ev[u]);
+                stf(gw + gi + u, du[u] * vv[u]);
+                stf(gv + gi + u, du[u] * wv[u]);
+            }
+        }
+        __syncthreads();
+    }
+    tc::release(tcx.st, kTmemCols);
+}
+
+// ------------------------------------------------------------------ host side
+
+// Dynamic shared memory of the per-chunk kernels: the largest staging area of
+// their phases (tensor-core slabs, masked products, gradient products, solves).
+template <int D, int PASSES>
+int dyn_bytes(int C) {
+    int f = tc::stage_bytes<PASSES, 128>() / 4;
+    const int m = masked_smem_floats(C, D), g = decayed_smem_floats(C), s = solve_smem_floats(C, D);
+    f = f > m ? f : m;
+    f = f > g ? f : g;
+    f = f > s ? f : s;
+    return f * 4;
+}
+
+// CTAs that fit on one SM next to each other with this much shared memory.
+inline int ctas_per_sm(int dyn) { return dyn <= 100 * 1024 ? 2 : 1; }
+
+template <typename Tin, int D, int PASSES>
+cudaError_t set_smem_attrs(int bytes) {
+    cudaError_t e = cudaFuncSetAttribute(k_intra<Tin, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_out<Tin, float, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_out<Tin, __nv_bfloat16, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_bprep<Tin, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_bwd<Tin, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    return e;
+}
+
+inline int num_slots(int nch) { return nch < kMaxSlots ? nch : kMaxSlots; }
+
+inline size_t slot_floats(int C, int D) { return make_lay(C, D).total; }
+
+template <int D, int PASSES, bool REV>
+cudaError_t launch_chain(int BH, int N, const float* M, const float* Bn, const float* S_in,
+                                float* S_rec, float* S_out, cudaStream_t st) {
+    // column slabs: enough CTAs to cover the GPU when B*H is small
+    if (BH >= 64) {
+        constexpr int SL = 32;
+        MUIR_TIMED(REV ? "k_chain_rev" : "k_chain", st, k_chain<D, SL, PASSES, REV><<<BH * (D / SL), kThreads, 0, st>>>(M, Bn, S_in, S_rec, S_out, N));
+    } else {
+        constexpr int SL = 16;
+        MUIR_TIMED(REV ? "k_chain_rev" : "k_chain", st, k_chain<D, SL, PASSES, REV><<<BH * (D / SL), kThreads, 0, st>>>(M, Bn, S_in, S_rec, S_out, N));
+    }
+    return cudaGetLastError();
+}
+
+template <typename Tin, int D, int PASSES>
+cudaError_t fwd_impl(const ChunkProblem& P, const float* S0, void* o, float* S_final,
+                            float* S_chunks, float* M_chunks, void* ws, cudaStream_t st) {
+    const int nch = P.B * P.H * P.N, BH = P.B * P.H;
+    const size_t DD = (size_t)D * D;
+    float* f = static_cast<float*>(ws);
+    KParams kp = {};
+    kp.B = P.B; kp.T = P.T; kp.H = P.H; kp.C = P.C; kp.N = P.N;
+    kp.q = P.q; kp.k = P.k; kp.v = P.v; kp.g = P.g; kp.e = P.e; kp.w = P.w; kp.gamma = P.gamma;
+    kp.M = f; f += nch * DD;
+    if (M_chunks) kp.M = M_chunks;
+    kp.Bn = f; f += nch * DD;
+    float* Sc = S_chunks;
+    if (!Sc) { Sc = f; f += nch * DD; }
+    kp.scratch = f;
+    kp.slot = slot_floats(P.C, D);
+    kp.S_chunks = Sc;
+    kp.o = o;
+    const int dyn = dyn_bytes<D, PASSES>(P.C);
+    int grid = num_slots(nch);
+    const int resident = 148 * ctas_per_sm(dyn);
+    if (grid > resident) grid = resident;
+    cudaError_t err = set_smem_attrs<Tin, D, PASSES>(dyn);
+    if (err != cudaSuccess) return err;
+    MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+    err = cudaGetLastError();
+    if (err != cudaSuccess) return err;
+    err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, S_final, st);
+    if (err != cudaSuccess) return err;
+    if (P.out_bf16)
+        MUIR_TIMED("k_out", st, k_out<Tin, __nv_bfloat16, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+    else
+        MUIR_TIMED("k_out", st, k_out<Tin, float, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+    return cudaGetLastError();
+}
+
+template <typename Tin, int D, int PASSES>
+cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chunks,
+                            const float* M_chunks, const void* dO, const float* dS_final, void* dq, void* dk, void* dv,
+                            void* dg, void* de, void* dw, void* dgamma, float* dS0, void* ws,
+                            cudaStream_t st) {
+    const int nch = P.B * P.H * P.N, BH = P.B * P.H;
+    const size_t DD = (size_t)D * D;
+    float* f = static_cast<float*>(ws);
+    KParams kp = {};
+    kp.B = P.B; kp.T = P.T; kp.H = P.H; kp.C = P.C; kp.N = P.N;
+    kp.q = P.q; kp.k = P.k; kp.v = P.v; kp.g = P.g; kp.e = P.e; kp.w = P.w; kp.gamma = P.gamma;
+    kp.dO = dO;
+    kp.M = f; f += nch * DD;
+    kp.Bn = f; f += nch * DD;
+    float* dSc = f; f += nch * DD;
+    float* Sc = const_cast<float*>(S_chunks);
+    const bool recompute = S_chunks == nullptr;
+    if (recompute) { Sc = f; f += nch * DD; }
+    kp.scratch = f;
+    kp.slot = slot_floats(P.C, D);
+    kp.S_chunks = Sc;
+    kp.dS_chunks = dSc;
+    kp.dq = dq; kp.dk = dk; kp.dv = dv; kp.dg = dg; kp.de = de; kp.dw = dw; kp.dgamma = dgamma;
+    const int dyn = dyn_bytes<D, PASSES>(P.C);
+    int grid = num_slots(nch);
+    const int resident = 148 * ctas_per_sm(dyn);
+    if (grid > resident) grid = resident;
+    cudaError_t err = set_smem_attrs<Tin, D, PASSES>(dyn);
+    if (err != cudaSuccess) return err;
+    const bool have_M = M_chunks != nullptr && !recompute;
+    if (have_M) {
+        kp.M = const_cast<float*>(M_chunks);  // the forward's transitions: nothing to recompute
+    } else {
+        MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+        err = cudaGetLastError();
+        if (err != cudaSuccess) return err;
+    }
+    if (recompute) {
+        err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, nullptr, st);
+        if (err != cudaSuccess) return err;
+    }
+    MUIR_TIMED("k_bprep", st, k_bprep<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    err = launch_chain<D, PASSES, true>(BH, P.N, kp.M, kp.Bn, dS_final, dSc, dS0, st);
+    if (err != cudaSuccess) return err;
+    MUIR_TIMED("k_bwd", st, k_bwd<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+    return cudaGetLastError();
+}
+
+}  // namespace muir

@@ -24,9 +24,10 @@ size_t chunk_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states);
 size_t chunk_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states);
 
 cudaError_t run_chunk_fwd(const ChunkProblem& P, const float* S0, void* o, float* S_final,
-                          float* S_chunks, void* ws, size_t ws_bytes, cudaStream_t st);
+                          float* S_chunks, float* M_chunks, void* ws, size_t ws_bytes,
+                          cudaStream_t st);
 cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S_chunks,
-                          const void* dO, const float* dS_final, void* dq, void* dk, void* dv,
+                          const float* M_chunks, const void* dO, const float* dS_final, void* dq, void* dk, void* dv,
                           void* dg, void* de, void* dw, void* dgamma, float* dS0, void* ws,
                           size_t ws_bytes, cudaStream_t st);
 

@@ -73,6 +73,15 @@ __device__ void prologue2(const Chunk<Tin, D>& c) {
     __syncthreads();
 }
 
+// exp for the factors: the fast hardware exp2-based form for bf16 inputs (its
+// ~1e-6 relative error is far below the bf16 tolerance), the accurate one for
+// float32 inputs.
+template <typename Tin>
+__device__ __forceinline__ float fexp(float x) {
+    if constexpr (std::is_same<Tin, float>::value) return expf(x);
+    else return __expf(x);
+}
+
 // Log factors (see the header comment).
 template <typename Tin, int D>
 struct Fac {
@@ -87,10 +96,10 @@ struct Fac {
         return s[L.LC + (size_t)((t & ~7) + 3) * D + j] - s[L.LC + (size_t)t * D + j];
     }
     __device__ float eg(int t, int j) const {
-        return expf(s[L.PRE + (size_t)(t >> 3) * D + j] + s[L.LC + (size_t)t * D + j]);
+        return fexp<Tin>(s[L.PRE + (size_t)(t >> 3) * D + j] + s[L.LC + (size_t)t * D + j]);
     }
     __device__ float egb(int t, int j) const {
-        return expf(s[L.RC + (size_t)t * D + j] + s[L.SUF + (size_t)(t >> 3) * D + j]);
+        return fexp<Tin>(s[L.RC + (size_t)t * D + j] + s[L.SUF + (size_t)(t >> 3) * D + j]);
     }
     __device__ float gbar(int j) const { return s[L.GBAR + j]; }
 };
@@ -117,9 +126,10 @@ __device__ __forceinline__ void mma_f(float (&d)[4], const float (&a)[4], const 
     }
 }
 
-// Channels per slab so that one C x slab fp32 tile is 16 KB.
+// Channels per slab so that one C x slab fp32 tile is 8 KB (small staging
+// areas leave most of the SM's unified L1 / shared memory to the L1 cache).
 __host__ __device__ constexpr int slab_channels(int C, int D) {
-    return (4096 / C) < D ? (4096 / C) : D;
+    return (2048 / C) < D ? (2048 / C) : D;
 }
 
 // Shared-memory floats masked_pair_s needs.
@@ -128,15 +138,23 @@ __host__ __device__ constexpr int masked_smem_floats(int C, int D) {
 }
 
 // Stage F[I][J][jj] = exp(sum_{J<K<I} Bt[K][j0 + jj]) for J < I (1 for J = I - 1).
+template <typename Tin>
 __device__ __forceinline__ void stage_F(float* FS, const float* s, const Lay& L, int D, int j0,
                                         int SL) {
-    const int nb8 = L.nb8;
+    const int nb8 = L.nb8;  // <= 32
     for (int idx = threadIdx.x; idx < nb8 * SL; idx += kThreads) {
         const int I = idx / SL, jj = idx % SL;
+        float bt[32];
+#pragma unroll
+        for (int J = 0; J < 32; ++J)  // all block totals first (independent loads)
+            bt[J] = J < I ? s[L.BT + (size_t)J * D + j0 + jj] : 0.f;
         float acc = 0.f;
-        for (int J = I - 1; J >= 0; --J) {
-            FS[((size_t)I * nb8 + J) * SL + jj] = expf(acc);
-            acc += s[L.BT + (size_t)J * D + j0 + jj];
+#pragma unroll
+        for (int J = 31; J >= 0; --J) {
+            if (J < I) {
+                FS[((size_t)I * nb8 + J) * SL + jj] = fexp<Tin>(acc);
+                acc += bt[J];
+            }
         }
     }
 }
@@ -173,20 +191,37 @@ __device__ void masked_pair_s(const Chunk<Tin, D>& c, float* sm, int X, int Z0, 
             for (int u = 0; u < 4; ++u) acc0[i][u] = acc1[i][u] = 0.f;
         for (int j0 = 0; j0 < D; j0 += SL) {
             __syncthreads();
-            for (int idx = threadIdx.x; idx < C * SL; idx += kThreads) {
-                const int t = idx / SL, jj = idx % SL, j = j0 + jj;
-                const float x = opval(c, X, t, j), z0 = opval(c, Z0, t, j), z1 = opval(c, Z1, t, j);
-                const float ex8 = expf(f.lx8(t, j)), exo = expf(f.lxo(t, j));
-                const float ez8 = expf(f.lz8(t, j)), ezo = expf(f.lzo(t, j));
-                const int o = t * SP + jj;
-                XH[o] = x * ex8;
-                XO[o] = x * exo;
-                ZH0[o] = z0 * ez8;
-                ZH1[o] = z1 * ez8;
-                ZO0[o] = z0 * ezo;
-                ZO1[o] = z1 * ezo;
+            for (int base = 0; base < C * SL; base += 4 * kThreads) {
+                float x[4], z0[4], z1[4], l8[4], lm[4], r8[4];
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {  // loads first, so they overlap
+                    const int idx = base + threadIdx.x + it * kThreads;
+                    const int t = idx / SL, j = j0 + idx % SL;
+                    const bool in = idx < C * SL;
+                    x[it] = in ? opval(c, X, t, j) : 0.f;
+                    z0[it] = in ? opval(c, Z0, t, j) : 0.f;
+                    z1[it] = in ? opval(c, Z1, t, j) : 0.f;
+                    l8[it] = in ? f.lx8(t, j) : 0.f;
+                    lm[it] = in ? c.s[L.LC + (size_t)((t & ~7) + 3) * D + j] : 0.f;
+                    r8[it] = in ? f.lz8(t, j) : 0.f;
+                }
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int idx = base + threadIdx.x + it * kThreads;
+                    if (idx >= C * SL) break;
+                    const int t = idx / SL, jj = idx % SL;
+                    const float ex8 = fexp<Tin>(l8[it]), exo = fexp<Tin>(l8[it] - lm[it]);
+                    const float ez8 = fexp<Tin>(r8[it]), ezo = fexp<Tin>(lm[it] - l8[it]);
+                    const int o = t * SP + jj;
+                    XH[o] = x[it] * ex8;
+                    XO[o] = x[it] * exo;
+                    ZH0[o] = z0[it] * ez8;
+                    ZH1[o] = z1[it] * ez8;
+                    ZO0[o] = z0[it] * ezo;
+                    ZO1[o] = z1[it] * ezo;
+                }
             }
-            stage_F(FS, c.s, L, D, j0, SL);
+            stage_F<Tin>(FS, c.s, L, D, j0, SL);
             __syncthreads();
 #pragma unroll
             for (int i = 0; i < TPW; ++i) {
@@ -255,14 +290,18 @@ __device__ void masked_pair_s(const Chunk<Tin, D>& c, float* sm, int X, int Z0, 
 
 // ------------------------------------------------------------------ gradients through masked products
 
-// Channels per output slab of decayed_grad_s (the F table must fit).
-__host__ __device__ constexpr int decayed_channels(int C) { return C > 128 ? 16 : 32; }
+// Slab shape of decayed_grad_s: channels per output slab (CH), tokens per
+// contraction slab (TS), 16-row blocks per warp (RB); C = 256 takes narrower
+// channel slabs so the F table fits.
+__host__ __device__ constexpr int decayed_ch(int C) { return C > 128 ? 16 : 32; }
+__host__ __device__ constexpr int decayed_ts(int C) { return 32; }
 
-// Shared-memory floats decayed_grad_s needs: two gradient slabs (C x 32 tokens or
-// 32 tokens x C, padded), four operand slabs (32 tokens x CH), the F table.
+// Shared-memory floats decayed_grad_s needs: two gradient slabs (C x TS or
+// TS x C, padded), four operand slabs (TS tokens x CH), the F table.
 __host__ __device__ constexpr int decayed_smem_floats(int C) {
-    return 2 * ((C * 36) > (32 * (C + 8)) ? (C * 36) : (32 * (C + 8))) +
-           4 * 32 * (decayed_channels(C) + 8) + (C / 8) * (C / 8) * decayed_channels(C);
+    return 2 * ((C * (decayed_ts(C) + 4)) > (decayed_ts(C) * (C + 8)) ? (C * (decayed_ts(C) + 4))
+                                                                       : (decayed_ts(C) * (C + 8))) +
+           4 * decayed_ts(C) * (decayed_ch(C) + 8) + (C / 8) * (C / 8) * decayed_ch(C);
 }
 
 // X side (XSIDE):  out[t][j] = sum_s Gm[t][s] Z_sj exp(Gam_tj - Gam_sj)
@@ -271,13 +310,12 @@ __host__ __device__ constexpr int decayed_smem_floats(int C) {
 // Output tiles: 16 rows x 32 channels; contraction in slabs of 32 tokens, one
 // 8-token block per MMA step; off-diagonal block pairs scale the step's result
 // by F, diagonal blocks use the mid-block pivot; output-side factors at the end.
-template <typename Tin, int D, int PASSES, bool XSIDE, int CH, class EPI>
+template <typename Tin, int D, int PASSES, bool XSIDE, int CH, int TS, int RB, class EPI>
 __device__ void decayed_grad_s(const Chunk<Tin, D>& c, float* sm, size_t G0, int op0, size_t G1,
                                int op1, const EPI& epi) {
     const Lay& L = c.L;
     const Fac<Tin, D> f = facs(c);
     const int C = L.C, nb8 = L.nb8, nb16 = L.nb16;
-    constexpr int TS = 32;                 // tokens per K slab
     constexpr int OP = CH + 8;             // operand slab row pitch
     const int GP = XSIDE ? TS + 4 : C + 8; // gradient slab row pitch
     float* GS0 = sm;
@@ -290,12 +328,12 @@ __device__ void decayed_grad_s(const Chunk<Tin, D>& c, float* sm, size_t G0, int
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, cq = lane & 3;
     for (int j0 = 0; j0 < D; j0 += CH) {
         __syncthreads();
-        stage_F(FS, c.s, L, D, j0, CH);
+        stage_F<Tin>(FS, c.s, L, D, j0, CH);
         // each warp owns row blocks I16 = warp, warp + 8, ... (at most 2 for C <= 256)
         constexpr int NT = CH / 8;
-        float off[2][NT][4], dia[2][NT][4];
+        float off[RB][NT][4], dia[RB][NT][4];
 #pragma unroll
-        for (int a = 0; a < 2; ++a)
+        for (int a = 0; a < RB; ++a)
 #pragma unroll
             for (int n = 0; n < NT; ++n)
 #pragma unroll
@@ -304,34 +342,63 @@ __device__ void decayed_grad_s(const Chunk<Tin, D>& c, float* sm, size_t G0, int
         for (int k0 = 0; k0 < C; k0 += ts) {
             __syncthreads();
             // gradient slabs
-            if (XSIDE) {
-                for (int idx = threadIdx.x; idx < C * ts; idx += kThreads) {
-                    const int t = idx / ts, kk = idx % ts;
-                    GS0[t * GP + kk] = c.s[G0 + (size_t)t * C + k0 + kk];
-                    GS1[t * GP + kk] = c.s[G1 + (size_t)t * C + k0 + kk];
-                }
-            } else {
-                for (int idx = threadIdx.x; idx < ts * C; idx += kThreads) {
-                    const int tt = idx / C, ss = idx % C;
-                    GS0[tt * GP + ss] = c.s[G0 + (size_t)(k0 + tt) * C + ss];
-                    GS1[tt * GP + ss] = c.s[G1 + (size_t)(k0 + tt) * C + ss];
+            {
+                // rows x cols of the slab (X side: all C rows x ts tokens; Z side: ts rows x C)
+                const int rows = XSIDE ? C : ts, cols = XSIDE ? ts : C, q4 = cols / 4;
+                const int n4 = rows * q4;
+                for (int base = 0; base < n4; base += 4 * kThreads) {
+                    float4 a0[4], a1[4];
+#pragma unroll
+                    for (int it = 0; it < 4; ++it) {
+                        const int idx = base + threadIdx.x + it * kThreads;
+                        if (idx < n4) {
+                            const int r = idx / q4, cc = 4 * (idx % q4);
+                            const size_t go = XSIDE ? (size_t)r * C + k0 + cc : (size_t)(k0 + r) * C + cc;
+                            a0[it] = *reinterpret_cast<const float4*>(c.s + G0 + go);
+                            a1[it] = *reinterpret_cast<const float4*>(c.s + G1 + go);
+                        }
+                    }
+#pragma unroll
+                    for (int it = 0; it < 4; ++it) {
+                        const int idx = base + threadIdx.x + it * kThreads;
+                        if (idx >= n4) break;
+                        const int r = idx / q4, cc = 4 * (idx % q4);
+                        float* d0 = GS0 + r * GP + cc;
+                        float* d1 = GS1 + r * GP + cc;
+                        d0[0] = a0[it].x; d0[1] = a0[it].y; d0[2] = a0[it].z; d0[3] = a0[it].w;
+                        d1[0] = a1[it].x; d1[1] = a1[it].y; d1[2] = a1[it].z; d1[3] = a1[it].w;
+                    }
                 }
             }
             // operand slabs: tokens k0.. of op0/op1 over channels j0.., scaled by the
             // pivot factors of the contraction side
-            for (int idx = threadIdx.x; idx < ts * CH; idx += kThreads) {
-                const int tt = idx / CH, jj = idx % CH, t = k0 + tt, j = j0 + jj;
-                const float v0 = opval(c, op0, t, j), v1 = opval(c, op1, t, j);
-                const float eh = XSIDE ? expf(f.lz8(t, j)) : expf(f.lx8(t, j));
-                const float eo = XSIDE ? expf(f.lzo(t, j)) : expf(f.lxo(t, j));
-                ZH0[tt * OP + jj] = v0 * eh;
-                ZO0[tt * OP + jj] = v0 * eo;
-                ZH1[tt * OP + jj] = v1 * eh;
-                ZO1[tt * OP + jj] = v1 * eo;
+            for (int base = 0; base < ts * CH; base += 2 * kThreads) {
+                float v0[2], v1[2], lh[2], lo[2];
+#pragma unroll
+                for (int it = 0; it < 2; ++it) {
+                    const int idx = base + threadIdx.x + it * kThreads;
+                    const int t = k0 + idx / CH, j = j0 + idx % CH;
+                    const bool in = idx < ts * CH;
+                    v0[it] = in ? opval(c, op0, t, j) : 0.f;
+                    v1[it] = in ? opval(c, op1, t, j) : 0.f;
+                    lh[it] = in ? (XSIDE ? f.lz8(t, j) : f.lx8(t, j)) : 0.f;
+                    lo[it] = in ? (XSIDE ? f.lzo(t, j) : f.lxo(t, j)) : 0.f;
+                }
+#pragma unroll
+                for (int it = 0; it < 2; ++it) {
+                    const int idx = base + threadIdx.x + it * kThreads;
+                    if (idx >= ts * CH) break;
+                    const int tt = idx / CH, jj = idx % CH;
+                    const float eh = fexp<Tin>(lh[it]), eo = fexp<Tin>(lo[it]);
+                    ZH0[tt * OP + jj] = v0[it] * eh;
+                    ZO0[tt * OP + jj] = v0[it] * eo;
+                    ZH1[tt * OP + jj] = v1[it] * eh;
+                    ZO1[tt * OP + jj] = v1[it] * eo;
+                }
             }
             __syncthreads();
 #pragma unroll
-            for (int a = 0; a < 2; ++a) {
+            for (int a = 0; a < RB; ++a) {
                 const int I16 = warp + 8 * a;
                 if (I16 >= nb16) break;
                 const int m0 = 16 * I16, rb0 = 2 * I16, rb1 = rb0 + 1;
@@ -395,7 +462,7 @@ __device__ void decayed_grad_s(const Chunk<Tin, D>& c, float* sm, size_t G0, int
         }
         // output-side pivot factors and the epilogue
 #pragma unroll
-        for (int a = 0; a < 2; ++a) {
+        for (int a = 0; a < RB; ++a) {
             const int I16 = warp + 8 * a;
             if (I16 >= nb16) break;
 #pragma unroll
@@ -404,8 +471,8 @@ __device__ void decayed_grad_s(const Chunk<Tin, D>& c, float* sm, size_t G0, int
                 for (int u = 0; u < 4; ++u) {
                     const int row = 16 * I16 + g + (u < 2 ? 0 : 8);
                     const int col = j0 + 8 * n + 2 * cq + (u & 1);
-                    const float fo = XSIDE ? expf(f.lx8(row, col)) : expf(f.lz8(row, col));
-                    const float fd = XSIDE ? expf(f.lxo(row, col)) : expf(f.lzo(row, col));
+                    const float fo = fexp<Tin>(XSIDE ? f.lx8(row, col) : f.lz8(row, col));
+                    const float fd = fexp<Tin>(XSIDE ? f.lxo(row, col) : f.lzo(row, col));
                     epi(row, col, fo * off[a][n][u] + fd * dia[a][n][u]);
                 }
         }
@@ -417,9 +484,9 @@ template <typename Tin, int D, int PASSES, bool XSIDE, class EPI>
 __device__ __forceinline__ void decayed_grad_any(const Chunk<Tin, D>& c, float* sm, size_t G0,
                                                  int op0, size_t G1, int op1, const EPI& epi) {
     if (c.L.C > 128)
-        decayed_grad_s<Tin, D, PASSES, XSIDE, 16>(c, sm, G0, op0, G1, op1, epi);
+        decayed_grad_s<Tin, D, PASSES, XSIDE, 16, 32, 2>(c, sm, G0, op0, G1, op1, epi);
     else
-        decayed_grad_s<Tin, D, PASSES, XSIDE, 32>(c, sm, G0, op0, G1, op1, epi);
+        decayed_grad_s<Tin, D, PASSES, XSIDE, 32, 32, 1>(c, sm, G0, op0, G1, op1, epi);
 }
 
 // ------------------------------------------------------------------ triangular solves
@@ -443,26 +510,49 @@ __device__ void solve_s(float* s, float* sm, const Lay& L, size_t Loff, size_t X
     constexpr int NT = D / 64;  // n8 tiles per warp
     const int c0 = warp * (D / 8);
     __syncthreads();
-    for (int idx = threadIdx.x; idx < C * D / 4; idx += kThreads) {
-        const int t = idx / (D / 4), j = 4 * (idx % (D / 4));
-        const float4 v = *reinterpret_cast<const float4*>(s + Xoff + (size_t)t * D + j);
-        XS[t * XP + j] = v.x; XS[t * XP + j + 1] = v.y; XS[t * XP + j + 2] = v.z; XS[t * XP + j + 3] = v.w;
+    for (int base = 0; base < C * D / 4; base += 4 * kThreads) {
+        float4 v[4];
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int idx = base + threadIdx.x + it * kThreads;
+            if (idx < C * D / 4) v[it] = *reinterpret_cast<const float4*>(s + Xoff + (size_t)4 * idx);
+        }
+#pragma unroll
+        for (int it = 0; it < 4; ++it) {
+            const int idx = base + threadIdx.x + it * kThreads;
+            if (idx >= C * D / 4) break;
+            const int t = idx / (D / 4), j = 4 * (idx % (D / 4));
+            XS[t * XP + j] = v[it].x; XS[t * XP + j + 1] = v[it].y;
+            XS[t * XP + j + 2] = v[it].z; XS[t * XP + j + 3] = v[it].w;
+        }
     }
     for (int idx = threadIdx.x; idx < C * 16; idx += kThreads) TS[idx] = s[L.TII + idx];
     for (int step = 0; step < nb16; ++step) {
         const int I = REV ? nb16 - 1 - step : step;
         __syncthreads();
         // stage L block: forward -> rows 16I.. (cols [0,16I)); reverse -> cols 16I.. (rows (16I+16, C))
-        if (!REV) {
-            for (int idx = threadIdx.x; idx < 16 * 16 * I; idx += kThreads) {
-                const int r = idx / (16 * I), k = idx % (16 * I);
-                LS[r * LP + k] = s[Loff + (size_t)(16 * I + r) * C + k];
-            }
-        } else {
+        {
+            // forward: rows 16I.. and columns [0, 16I); reverse: LS[r][k] = L[r1 + k][16I + r]
             const int r1 = 16 * (I + 1);
-            for (int idx = threadIdx.x; idx < 16 * (C - r1); idx += kThreads) {
-                const int k = idx / 16, r = idx % 16;  // LS[r][k] = L[r1 + k][16I + r]
-                LS[r * LP + k] = s[Loff + (size_t)(r1 + k) * C + 16 * I + r];
+            const int n = REV ? 16 * (C - r1) : 16 * 16 * I;
+            for (int base = 0; base < n; base += 4 * kThreads) {
+                float v[4];
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int idx = base + threadIdx.x + it * kThreads;
+                    v[it] = 0.f;
+                    if (idx < n) {
+                        if (!REV) v[it] = s[Loff + (size_t)(16 * I + idx / (16 * I)) * C + idx % (16 * I)];
+                        else v[it] = s[Loff + (size_t)(r1 + idx / 16) * C + 16 * I + idx % 16];
+                    }
+                }
+#pragma unroll
+                for (int it = 0; it < 4; ++it) {
+                    const int idx = base + threadIdx.x + it * kThreads;
+                    if (idx >= n) break;
+                    if (!REV) LS[(idx / (16 * I)) * LP + idx % (16 * I)] = v[it];
+                    else LS[(idx % 16) * LP + idx / 16] = v[it];
+                }
             }
         }
         __syncthreads();

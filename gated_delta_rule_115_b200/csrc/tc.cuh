@@ -19,6 +19,8 @@
 
 #include <stdint.h>
 
+#include <type_traits>
+
 namespace muir {
 namespace tc {
 
@@ -127,30 +129,47 @@ __host__ __device__ constexpr int stage_bytes() {
 
 // Stage one operand slab: rows [0, R) x K columns [k0, k0 + KS) into `dst`
 // (and `dst_lo` for PASSES == 3).  f4(row, k, out[4]) produces elements
-// (row, k..k+3) with k a multiple of 4 (zeros past kmax).  ROWMAJ_LANES: lanes
-// walk rows (source contiguous along rows) instead of K groups.
-template <int PASSES, bool ROW_LANES, class F4>
-__device__ __forceinline__ void stage(unsigned char* dst, unsigned char* dst_lo, int R, int k0,
-                                      int kmax, const F4& f4) {
+// (row, k..k+3) with k a multiple of 4 (zeros past kmax).  ROW_LANES: lanes
+// walk rows (source contiguous along rows) instead of K groups.  All loads of a
+// thread are issued before its shared-memory stores so they overlap.
+template <int PASSES, bool ROW_LANES, int R, class F4>
+__device__ __forceinline__ void stage(unsigned char* dst, unsigned char* dst_lo, int k0, int kmax,
+                                      const F4& f4) {
     constexpr int KG = KS / 4;
-    const int total = R * KG;
-    for (int idx = threadIdx.x; idx < total; idx += blockDim.x) {
+    constexpr int ITEMS = (R * KG + 255) / 256;
+    float v[ITEMS][4];
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) {
+        const int idx = threadIdx.x + it * 256;
         int row, kg;
         if (ROW_LANES) { row = idx % R; kg = idx / R; }
         else { kg = idx % KG; row = idx / KG; }
         const int k = k0 + 4 * kg;
-        float v[4] = {0.f, 0.f, 0.f, 0.f};
-        if (k < kmax) f4(row, k, v);
+        v[it][0] = v[it][1] = v[it][2] = v[it][3] = 0.f;
+        if (idx < R * KG && k < kmax) f4(row, k, v[it]);
+    }
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) {
+        const int idx = threadIdx.x + it * 256;
+        if (idx >= R * KG) break;
+        int row, kg;
+        if (ROW_LANES) { row = idx % R; kg = idx / R; }
+        else { kg = idx % KG; row = idx / KG; }
         float4 hi, lo;
-        hi.x = tf32_rn(v[0]); hi.y = tf32_rn(v[1]); hi.z = tf32_rn(v[2]); hi.w = tf32_rn(v[3]);
+        hi.x = tf32_rn(v[it][0]); hi.y = tf32_rn(v[it][1]); hi.z = tf32_rn(v[it][2]); hi.w = tf32_rn(v[it][3]);
         *reinterpret_cast<float4*>(dst + kmaj_off(row, 4 * kg)) = hi;
         if (PASSES == 3) {
-            lo.x = tf32_rn(v[0] - hi.x); lo.y = tf32_rn(v[1] - hi.y);
-            lo.z = tf32_rn(v[2] - hi.z); lo.w = tf32_rn(v[3] - hi.w);
+            lo.x = tf32_rn(v[it][0] - hi.x); lo.y = tf32_rn(v[it][1] - hi.y);
+            lo.z = tf32_rn(v[it][2] - hi.z); lo.w = tf32_rn(v[it][3] - hi.w);
             *reinterpret_cast<float4*>(dst_lo + kmaj_off(row, 4 * kg)) = lo;
         }
     }
 }
+
+struct RowStore {
+    float* dst;  // row-major destination, 16-byte aligned rows
+    int ld;      // floats between rows (multiple of 4)
+};
 
 // D (128 x N, TMEM) = sum over K of A(m, k) B(k, n).  fa4(m, k, v[4]) gives
 // A(m, k..k+3); fb4(n, k, v[4]) gives B(k..k+3, n).  Rows m >= M are zero.
@@ -169,10 +188,10 @@ __device__ void gemm(State& s, unsigned char* sbuf, int M, int K, const FA4& fa4
     const int nslab = (K + KS - 1) / KS;
     for (int sl = 0; sl < nslab; ++sl) {
         const int k0 = sl * KS;
-        stage<PASSES, A_ROW_LANES>(sA, sAl, 128, k0, K, [&](int m, int k, float* v) {
+        stage<PASSES, A_ROW_LANES, 128>(sA, sAl, k0, K, [&](int m, int k, float* v) {
             if (m < M) fa4(m, k, v);
         });
-        stage<PASSES, B_ROW_LANES>(sB, sBl, N, k0, K, fb4);
+        stage<PASSES, B_ROW_LANES, N>(sB, sBl, k0, K, fb4);
         asm volatile("fence.proxy.async.shared::cta;");
         __syncthreads();
         if (threadIdx.x == 0) {
@@ -208,8 +227,16 @@ __device__ void gemm(State& s, unsigned char* sbuf, int M, int K, const FA4& fa4
                      : "r"(taddr));
         asm volatile("tcgen05.wait::ld.sync.aligned;");
         if (row < M) {
+            if constexpr (std::is_same<EPI, RowStore>::value) {
+                float* d = epi.dst + (size_t)row * epi.ld + c0;
+                *reinterpret_cast<float4*>(d) = make_float4(__uint_as_float(r[0]), __uint_as_float(r[1]),
+                                                            __uint_as_float(r[2]), __uint_as_float(r[3]));
+                *reinterpret_cast<float4*>(d + 4) = make_float4(__uint_as_float(r[4]), __uint_as_float(r[5]),
+                                                                __uint_as_float(r[6]), __uint_as_float(r[7]));
+            } else {
 #pragma unroll
-            for (int j = 0; j < 8; ++j) epi(row, c0 + j, __uint_as_float(r[j]));
+                for (int j = 0; j < 8; ++j) epi(row, c0 + j, __uint_as_float(r[j]));
+            }
         }
     }
     asm volatile("tcgen05.fence::before_thread_sync;");

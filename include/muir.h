@@ -87,11 +87,15 @@ size_t muir_chunk_bwd_workspace(const muir_shape* shape);
  *   S_chunks          : [B][H][T/C][dk][dv] float32, may be NULL; receives the
  *                       state at the start of every chunk, which
  *                       muir_chunk_bwd can reuse instead of recomputing it.
+ *   M_chunks          : [B][H][T/C][dk][dk] float32, may be NULL; receives the
+ *                       chunk transitions M_n (S_{n+1} = M_n S_n + B_n), which
+ *                       muir_chunk_bwd reuses together with S_chunks.
  */
 muir_status muir_chunk_fwd(const muir_shape* shape, const void* q, const void* k,
                            const void* v, const void* g, const void* e, const void* w,
                            const void* gamma, const float* S0, void* o, float* S_final,
-                           float* S_chunks, void* ws, size_t ws_bytes, void* stream);
+                           float* S_chunks, float* M_chunks, void* ws, size_t ws_bytes,
+                           void* stream);
 
 /*
  * Backward of muir_chunk_fwd ("custom backward pass", same page,
@@ -101,13 +105,15 @@ muir_status muir_chunk_fwd(const muir_shape* shape, const void* q, const void* k
  *   dS_final [B][H][dk][dv] float32 or NULL (= 0);
  *   S_chunks: NULL (recompute the chunk states) or the array a previous
  *             muir_chunk_fwd with the same inputs wrote;
+ *   M_chunks: NULL, or (with S_chunks) the transitions that forward wrote:
+ *             then the per-chunk transitions are not recomputed;
  *   dq, dk, dg, de, dgamma [B][T][H][dk] and dv, dw [B][T][H][dv] are written
  *   in in_dtype; dS0 [B][H][dk][dv] float32 may be NULL.
  */
 muir_status muir_chunk_bwd(const muir_shape* shape, const void* q, const void* k,
                            const void* v, const void* g, const void* e, const void* w,
                            const void* gamma, const float* S0, const float* S_chunks,
-                           const void* dO, const float* dS_final, void* dq, void* dk,
+                           const float* M_chunks, const void* dO, const float* dS_final, void* dq, void* dk,
                            void* dv, void* dg, void* de, void* dw, void* dgamma,
                            float* dS0, void* ws, size_t ws_bytes, void* stream);
 

@@ -65,11 +65,11 @@ FAKE = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced: checks f
 
 def _fwd(L, shp, **over):
     args = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, e=FAKE, w=FAKE, gamma=FAKE, S0=None, o=FAKE,
-                S_final=None, S_chunks=None, ws=None, ws_bytes=0)
+                S_final=None, S_chunks=None, M_chunks=None, ws=None, ws_bytes=0)
     args.update(over)
     return L.muir_chunk_fwd(ctypes.byref(shp), args["q"], args["k"], args["v"], args["g"],
                             args["e"], args["w"], args["gamma"], args["S0"], args["o"],
-                            args["S_final"], args["S_chunks"], args["ws"],
+                            args["S_final"], args["S_chunks"], args["M_chunks"], args["ws"],
                             ctypes.c_size_t(args["ws_bytes"]), None)
 
 
@@ -83,7 +83,8 @@ def test_chunk_fwd_rejects_bad_arguments(L):
     assert _fwd(L, _shape(m, in_dtype=7)) == 1
     assert _fwd(L, _shape(m), q=None) == 1                  # null input
     assert _fwd(L, _shape(m), o=ctypes.c_void_p(0x10004)) == 1  # misaligned output
-    assert L.muir_chunk_fwd(None, *([FAKE] * 12), ctypes.c_size_t(0), None) == 1
+    assert _fwd(L, _shape(m), M_chunks=ctypes.c_void_p(0x10002)) == 1  # misaligned saved array
+    assert L.muir_chunk_fwd(None, *([FAKE] * 13), ctypes.c_size_t(0), None) == 1
 
 
 def test_chunk_workspace_query(L):
@@ -99,11 +100,11 @@ def test_chunk_workspace_query(L):
 def test_chunk_bwd_rejects_bad_arguments(L):
     import gated_delta_rule_115_b200 as m
     shp = _shape(m, dk=32, dv=32)
-    args = [FAKE] * 7 + [None, None, FAKE, None] + [FAKE] * 7 + [None, None]
+    args = [FAKE] * 7 + [None, None, None, FAKE, None] + [FAKE] * 7 + [None, None]
     assert L.muir_chunk_bwd(ctypes.byref(shp), *args, ctypes.c_size_t(0), None) == 2
     shp = _shape(m)
     args2 = list(args)
-    args2[10] = ctypes.c_void_p(0x10008)  # misaligned dS_final
+    args2[11] = ctypes.c_void_p(0x10008)  # misaligned dS_final
     assert L.muir_chunk_bwd(ctypes.byref(shp), *args2, ctypes.c_size_t(0), None) == 1
 
 

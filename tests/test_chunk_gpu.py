@@ -148,6 +148,13 @@ def test_chunk_bwd_reuses_states(muir):
     b = muir.chunk_bwd(*[x[n] for n in NAMES], x["S0"], x["dO"], chunk=128, S_chunks=Sc)
     for k in a:
         assert torch.equal(a[k], b[k]), k
+    # with the transitions as well, the backward skips recomputing them
+    o2, S2, Sc2, Mc2 = muir.chunk_fwd(*[x[n] for n in NAMES], x["S0"], chunk=128, return_saved=True)
+    assert torch.equal(Sc2, Sc) and torch.equal(o2, o)
+    c = muir.chunk_bwd(*[x[n] for n in NAMES], x["S0"], x["dO"], chunk=128, S_chunks=Sc2,
+                       M_chunks=Mc2)
+    for k in a:
+        assert torch.equal(a[k], c[k]), k
 
 
 # ------------------------------------------------------------ full-size workloads
@@ -183,8 +190,9 @@ def test_full_size_fwd_bwd_long_context(muir, oracle_mod):
     from gated_delta_rule_115_b200 import inputs as I
     x = I.chunk_inputs(2)
     d = to_dev(x)
-    o, S, Sc = muir.chunk_fwd(*[d[n] for n in NAMES], d["S0"], chunk=128, return_chunk_states=True)
-    gr = muir.chunk_bwd(*[d[n] for n in NAMES], d["S0"], d["dO"], chunk=128, S_chunks=Sc)
+    o, S, Sc, Mc = muir.chunk_fwd(*[d[n] for n in NAMES], d["S0"], chunk=128, return_saved=True)
+    gr = muir.chunk_bwd(*[d[n] for n in NAMES], d["S0"], d["dO"], chunk=128, S_chunks=Sc,
+                        M_chunks=Mc)
     torch.cuda.synchronize()
     hs = [11]
     xs = sub(x, [0], hs)
