@@ -111,7 +111,8 @@ struct Chunk {
     __device__ float& at(size_t off, int r, int c) const { return s[off + (size_t)r * D + c]; }
 };
 
-template <typename Tin, int D>
+// CF: the chunk size when it is fixed at compile time (0 = take it from p.C).
+template <typename Tin, int D, int CF>
 __device__ Chunk<Tin, D> make_chunk(const KParams& p, int chunk, float* slot) {
     Chunk<Tin, D> c;
     const int n = chunk % p.N, bh = chunk / p.N, h = bh % p.H, b = bh / p.H;
@@ -122,7 +123,7 @@ __device__ Chunk<Tin, D> make_chunk(const KParams& p, int chunk, float* slot) {
     c.base = (((size_t)b * p.T + (size_t)n * p.C) * p.H + h) * D;
     c.sbase = ((size_t)bh * p.N + n) * D * D;
     c.s = slot;
-    c.L = make_lay(p.C, D);
+    c.L = make_lay(CF ? CF : p.C, D);
     return c;
 }
 
@@ -216,7 +217,7 @@ __device__ __forceinline__ void tc_rows(TcCta& t, int M, int K, const FA4& fa4, 
 
 // ------------------------------------------------------------------ k_intra
 
-template <typename Tin, int D, int PASSES>
+template <typename Tin, int D, int PASSES, int CF>
 __global__ void __launch_bounds__(kThreads) k_intra(KParams p) {
     __shared__ uint32_t tmem_slot;
     __shared__ __align__(8) uint64_t mbar;
@@ -229,12 +230,12 @@ __global__ void __launch_bounds__(kThreads) k_intra(KParams p) {
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
-        const Chunk<Tin, D> c = make_chunk<Tin, D>(p, chunk, slot);
+        const Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
         const Lay& L = c.L;
         const int C = L.C;
         float* s = c.s;
         prologue2(c);
-        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
+        masked_pair_s<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, sm, L.LA, L.LK, false, false);
         __syncthreads();
         compute_tii(s, L, L.LA);
         for (int idx = threadIdx.x; idx < C * D; idx += kThreads)
@@ -348,7 +349,7 @@ __device__ void compute_Y(TcCta& tcx, const Chunk<Tin, D>& c, const float* S, si
     __syncthreads();
 }
 
-template <typename Tin, typename Tout, int D, int PASSES>
+template <typename Tin, typename Tout, int D, int PASSES, int CF>
 __global__ void __launch_bounds__(kThreads) k_out(KParams p) {
     __shared__ uint32_t tmem_slot;
     __shared__ __align__(8) uint64_t mbar;
@@ -361,13 +362,13 @@ __global__ void __launch_bounds__(kThreads) k_out(KParams p) {
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
-        const Chunk<Tin, D> c = make_chunk<Tin, D>(p, chunk, slot);
+        const Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
         const Lay& L = c.L;
         const int C = L.C;
         float* s = c.s;
         prologue2(c);
-        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
-        masked_pair_s<Tin, D, PASSES>(c, sm, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
+        masked_pair_s<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, sm, L.LA, L.LK, false, false);
+        masked_pair_s<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, sm, L.MQK, L.MQA, true, true);
         __syncthreads();
         compute_tii(s, L, L.LA);
         __syncthreads();
@@ -403,7 +404,7 @@ __global__ void __launch_bounds__(kThreads) k_out(KParams p) {
 
 // ------------------------------------------------------------------ k_bprep
 
-template <typename Tin, int D, int PASSES>
+template <typename Tin, int D, int PASSES, int CF>
 __global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
     __shared__ uint32_t tmem_slot;
     __shared__ __align__(8) uint64_t mbar;
@@ -416,13 +417,13 @@ __global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
-        const Chunk<Tin, D> c = make_chunk<Tin, D>(p, chunk, slot);
+        const Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
         const Lay& L = c.L;
         const int C = L.C;
         float* s = c.s;
         prologue2(c);
-        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
-        masked_pair_s<Tin, D, PASSES>(c, sm, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
+        masked_pair_s<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, sm, L.LA, L.LK, false, false);
+        masked_pair_s<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, sm, L.MQK, L.MQA, true, true);
         __syncthreads();
         compute_tii(s, L, L.LA);
         __syncthreads();
@@ -453,7 +454,7 @@ __global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
 
 // ------------------------------------------------------------------ k_bwd
 
-template <typename Tin, int D, int PASSES>
+template <typename Tin, int D, int PASSES, int CF>
 __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
     __shared__ float s_colsum[D];
     __shared__ float s_segtot[kThreads];
@@ -469,7 +470,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
-        const Chunk<Tin, D> c = make_chunk<Tin, D>(p, chunk, slot);
+        const Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
         const Lay& L = c.L;
         const int C = L.C;
         float* s = c.s;
@@ -478,8 +479,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         const size_t Y = L.W[0], dR = L.W[1], dK = L.W[2], dQh = L.W[3], dA = L.W[4],
                      dU = L.W[5], dGam = L.W[6];
         prologue2(c);
-        masked_pair_s<Tin, D, PASSES>(c, sm, OP_K, OP_A, OP_K, L.LA, L.LK, false, false);
-        masked_pair_s<Tin, D, PASSES>(c, sm, OP_Q, OP_K, OP_A, L.MQK, L.MQA, true, true);
+        masked_pair_s<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, sm, L.LA, L.LK, false, false);
+        masked_pair_s<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, sm, L.MQK, L.MQA, true, true);
         __syncthreads();
         compute_tii(s, L, L.LA);
         __syncthreads();
@@ -618,25 +619,25 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         }
         __syncthreads();
         // X side: dK += dL_A (*) A + dL_K (*) K ; dQh += dM_QK (*) K + dM_QA (*) A ; dGam += X * dX
-        decayed_grad_any<Tin, D, PASSES, true>(c, sm, L.LA, OP_A, L.LK, OP_K, [&](int t, int j, float v) {
+        decayed_grad_any<Tin, D, PASSES, true, OP_A, OP_K>(c, sm, L.LA, L.LK, [&](int t, int j, float v) {
             const size_t x = (size_t)t * D + j;
             s[dK + x] += v;
             s[dGam + x] += c.K(t, j) * v;
         });
-        decayed_grad_any<Tin, D, PASSES, true>(c, sm, L.MQK, OP_K, L.MQA, OP_A, [&](int t, int j, float v) {
+        decayed_grad_any<Tin, D, PASSES, true, OP_K, OP_A>(c, sm, L.MQK, L.MQA, [&](int t, int j, float v) {
             const size_t x = (size_t)t * D + j;
             s[dQh + x] += v;
             s[dGam + x] += c.Qh(t, j) * v;
         });
         __syncthreads();
         // Z side: dA += dL_A^T (*) K + dM_QA^T (*) Qh ; dK += dL_K^T (*) K + dM_QK^T (*) Qh ; dGam -= Z * dZ
-        decayed_grad_any<Tin, D, PASSES, false>(c, sm, L.LA, OP_K, L.MQA, OP_Q, [&](int t, int j, float v) {
+        decayed_grad_any<Tin, D, PASSES, false, OP_K, OP_Q>(c, sm, L.LA, L.MQA, [&](int t, int j, float v) {
             const size_t x = (size_t)t * D + j;
             s[dA + x] += v;
             s[dGam + x] -= c.A(t, j) * v;
         });
         __syncthreads();
-        decayed_grad_any<Tin, D, PASSES, false>(c, sm, L.LK, OP_K, L.MQK, OP_Q, [&](int t, int j, float v) {
+        decayed_grad_any<Tin, D, PASSES, false, OP_K, OP_Q>(c, sm, L.LK, L.MQK, [&](int t, int j, float v) {
             const size_t x = (size_t)t * D + j;
             s[dK + x] += v;
             s[dGam + x] -= c.K(t, j) * v;
@@ -729,13 +730,13 @@ int dyn_bytes(int C) {
 // CTAs that fit on one SM next to each other with this much shared memory.
 inline int ctas_per_sm(int dyn) { return dyn <= 100 * 1024 ? 2 : 1; }
 
-template <typename Tin, int D, int PASSES>
+template <typename Tin, int D, int PASSES, int CF>
 cudaError_t set_smem_attrs(int bytes) {
-    cudaError_t e = cudaFuncSetAttribute(k_intra<Tin, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_out<Tin, float, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_out<Tin, __nv_bfloat16, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_bprep<Tin, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_bwd<Tin, D, PASSES>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    cudaError_t e = cudaFuncSetAttribute(k_intra<Tin, D, PASSES, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_out<Tin, float, D, PASSES, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_out<Tin, __nv_bfloat16, D, PASSES, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_bprep<Tin, D, PASSES, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_bwd<Tin, D, PASSES, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     return e;
 }
 
@@ -757,7 +758,7 @@ cudaError_t launch_chain(int BH, int N, const float* M, const float* Bn, const f
     return cudaGetLastError();
 }
 
-template <typename Tin, int D, int PASSES>
+template <typename Tin, int D, int PASSES, int CF>
 cudaError_t fwd_impl(const ChunkProblem& P, const float* S0, void* o, float* S_final,
                             float* S_chunks, float* M_chunks, void* ws, cudaStream_t st) {
     const int nch = P.B * P.H * P.N, BH = P.B * P.H;
@@ -779,21 +780,21 @@ cudaError_t fwd_impl(const ChunkProblem& P, const float* S0, void* o, float* S_f
     int grid = num_slots(nch);
     const int resident = 148 * ctas_per_sm(dyn);
     if (grid > resident) grid = resident;
-    cudaError_t err = set_smem_attrs<Tin, D, PASSES>(dyn);
+    cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn);
     if (err != cudaSuccess) return err;
-    MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+    MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, S_final, st);
     if (err != cudaSuccess) return err;
     if (P.out_bf16)
-        MUIR_TIMED("k_out", st, k_out<Tin, __nv_bfloat16, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+        MUIR_TIMED("k_out", st, k_out<Tin, __nv_bfloat16, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
     else
-        MUIR_TIMED("k_out", st, k_out<Tin, float, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+        MUIR_TIMED("k_out", st, k_out<Tin, float, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
     return cudaGetLastError();
 }
 
-template <typename Tin, int D, int PASSES>
+template <typename Tin, int D, int PASSES, int CF>
 cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chunks,
                             const float* M_chunks, const void* dO, const float* dS_final, void* dq, void* dk, void* dv,
                             void* dg, void* de, void* dw, void* dgamma, float* dS0, void* ws,
@@ -820,13 +821,13 @@ cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chun
     int grid = num_slots(nch);
     const int resident = 148 * ctas_per_sm(dyn);
     if (grid > resident) grid = resident;
-    cudaError_t err = set_smem_attrs<Tin, D, PASSES>(dyn);
+    cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn);
     if (err != cudaSuccess) return err;
     const bool have_M = M_chunks != nullptr && !recompute;
     if (have_M) {
         kp.M = const_cast<float*>(M_chunks);  // the forward's transitions: nothing to recompute
     } else {
-        MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+        MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
         err = cudaGetLastError();
         if (err != cudaSuccess) return err;
     }
@@ -834,11 +835,11 @@ cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chun
         err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, nullptr, st);
         if (err != cudaSuccess) return err;
     }
-    MUIR_TIMED("k_bprep", st, k_bprep<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+    MUIR_TIMED("k_bprep", st, k_bprep<Tin, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     err = launch_chain<D, PASSES, true>(BH, P.N, kp.M, kp.Bn, dS_final, dSc, dS0, st);
     if (err != cudaSuccess) return err;
-    MUIR_TIMED("k_bwd", st, k_bwd<Tin, D, PASSES><<<grid, kThreads, dyn, st>>>(kp));
+    MUIR_TIMED("k_bwd", st, k_bwd<Tin, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
     return cudaGetLastError();
 }
 

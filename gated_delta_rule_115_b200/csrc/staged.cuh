@@ -166,9 +166,9 @@ __device__ __forceinline__ void stage_F(float* FS, const float* s, const Lay& L,
 // 8-blocks rb0 = 2*I16 and rb1 = rb0 + 1, columns in 8-block J8.  Off-diagonal
 // rows (rb > J8): A = X x8f F[rb][J8], B = Z z8f.  Diagonal rows (rb == J8):
 // A = X xof, B = Z zof.  Channels are streamed through shared memory in slabs.
-template <typename Tin, int D, int PASSES>
-__device__ void masked_pair_s(const Chunk<Tin, D>& c, float* sm, int X, int Z0, int Z1,
-                              size_t out0, size_t out1, bool incl0, bool incl1) {
+template <typename Tin, int D, int PASSES, int X, int Z0, int Z1>
+__device__ void masked_pair_s(const Chunk<Tin, D>& c, float* sm, size_t out0, size_t out1,
+                              bool incl0, bool incl1) {
     const Lay& L = c.L;
     const Fac<Tin, D> f = facs(c);
     const int C = L.C, nb8 = L.nb8, nb16 = L.nb16;
@@ -310,9 +310,10 @@ __host__ __device__ constexpr int decayed_smem_floats(int C) {
 // Output tiles: 16 rows x 32 channels; contraction in slabs of 32 tokens, one
 // 8-token block per MMA step; off-diagonal block pairs scale the step's result
 // by F, diagonal blocks use the mid-block pivot; output-side factors at the end.
-template <typename Tin, int D, int PASSES, bool XSIDE, int CH, int TS, int RB, class EPI>
-__device__ void decayed_grad_s(const Chunk<Tin, D>& c, float* sm, size_t G0, int op0, size_t G1,
-                               int op1, const EPI& epi) {
+template <typename Tin, int D, int PASSES, bool XSIDE, int CH, int TS, int RB, int op0, int op1,
+          class EPI>
+__device__ void decayed_grad_s(const Chunk<Tin, D>& c, float* sm, size_t G0, size_t G1,
+                               const EPI& epi) {
     const Lay& L = c.L;
     const Fac<Tin, D> f = facs(c);
     const int C = L.C, nb8 = L.nb8, nb16 = L.nb16;
@@ -480,13 +481,13 @@ __device__ void decayed_grad_s(const Chunk<Tin, D>& c, float* sm, size_t G0, int
     __syncthreads();
 }
 
-template <typename Tin, int D, int PASSES, bool XSIDE, class EPI>
+template <typename Tin, int D, int PASSES, bool XSIDE, int op0, int op1, class EPI>
 __device__ __forceinline__ void decayed_grad_any(const Chunk<Tin, D>& c, float* sm, size_t G0,
-                                                 int op0, size_t G1, int op1, const EPI& epi) {
+                                                 size_t G1, const EPI& epi) {
     if (c.L.C > 128)
-        decayed_grad_s<Tin, D, PASSES, XSIDE, 16, 32, 2>(c, sm, G0, op0, G1, op1, epi);
+        decayed_grad_s<Tin, D, PASSES, XSIDE, 16, 32, 2, op0, op1>(c, sm, G0, G1, epi);
     else
-        decayed_grad_s<Tin, D, PASSES, XSIDE, 32, 32, 1>(c, sm, G0, op0, G1, op1, epi);
+        decayed_grad_s<Tin, D, PASSES, XSIDE, 32, 32, 1, op0, op1>(c, sm, G0, G1, epi);
 }
 
 // ------------------------------------------------------------------ triangular solves
