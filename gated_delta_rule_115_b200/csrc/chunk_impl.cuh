@@ -215,6 +215,35 @@ __device__ __forceinline__ void tc_rows(TcCta& t, int M, int K, const FA4& fa4, 
     }
 }
 
+// Product with asynchronous staging of the K segments asrc / bsrc describe
+// (single-pass TF32); three-pass inputs take the element-producer engine.
+template <int PASSES, int N, bool AR, bool BR, class ASRC, class FA4, class BSRC, class FB4,
+          class EPI>
+__device__ __forceinline__ void tc_rows2(TcCta& t, int M, int K, const ASRC& asrc, const FA4& fa4,
+                                         const BSRC& bsrc, const FB4& fb4, const EPI& epi,
+                                         int NB = N) {
+    if constexpr (PASSES != 1) {
+        tc_rows<PASSES, N, AR, BR>(t, M, K, fa4, fb4, epi);
+    } else {
+        for (int m0 = 0; m0 < M; m0 += 128) {
+            const int Mt = M - m0 < 128 ? M - m0 : 128;
+            auto fa = [&](int m, int k, float* v) { fa4(m0 + m, k, v); };
+            auto as = [&](int k) {
+                tc::Src a = asrc(k);
+                if (a.p) a.p += a.mn ? (size_t)m0 : (size_t)m0 * a.ld;
+                return a;
+            };
+            if constexpr (std::is_same<EPI, tc::RowStore>::value) {
+                tc::RowStore d = {epi.dst + (size_t)m0 * epi.ld, epi.ld};
+                tc::gemm_async<N>(t.st, t.sbuf, Mt, NB, K, as, fa, bsrc, fb4, d);
+            } else {
+                tc::gemm_async<N>(t.st, t.sbuf, Mt, NB, K, as, fa, bsrc, fb4,
+                                  [&](int m, int n, float x) { epi(m0 + m, n, x); });
+            }
+        }
+    }
+}
+
 // ------------------------------------------------------------------ k_intra
 
 template <typename Tin, int D, int PASSES, int CF>
@@ -224,7 +253,7 @@ __global__ void __launch_bounds__(kThreads) k_intra(KParams p) {
     __shared__ int tc_status;
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
-    tcx.sbuf = dsm;
+    tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
     tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
@@ -247,8 +276,10 @@ __global__ void __launch_bounds__(kThreads) k_intra(KParams p) {
         const float* Psi = s + L.W[0];
         const Fac<Tin, D> f = facs(c);
         // M = diag(e^gbar) - Psi^T Kt      (rows i, contraction over tokens)
-        tc_rows<PASSES, D, true, true>(tcx, D, C,
+        tc_rows2<PASSES, D, true, true>(tcx, D, C,
+            [&](int) { return tc::Src{Psi, D, 0, true, false}; },
             [&](int i, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = Psi[(size_t)(t + u) * D + i]; },
+            [&](int) { return tc::no_src(); },
             [&](int j, int t, float* v) {
                 for (int u = 0; u < 4; ++u) v[u] = c.K(t + u, j) * f.eg(t + u, j);
             },
@@ -258,14 +289,18 @@ __global__ void __launch_bounds__(kThreads) k_intra(KParams p) {
             });
         // Phi = Kb - L_K^T Psi              (rows t, contraction over tokens s)
         float* Phi = s + L.W[1];
-        tc_rows<PASSES, D, true, true>(tcx, C, C,
+        tc_rows2<PASSES, D, true, true>(tcx, C, C,
+            [&](int) { return tc::Src{s + L.LK, C, 0, true, false}; },
             [&](int t, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = s[L.LK + (size_t)(k + u) * C + t]; },
+            [&](int) { return tc::Src{Psi, D, 0, true, false}; },
             [&](int j, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = Psi[(size_t)(k + u) * D + j]; },
             [&](int t, int j, float x) { Phi[(size_t)t * D + j] = c.K(t, j) * f.egb(t, j) - x; });
         // Bn = Phi^T U
         float* Bn = p.Bn + c.sbase;
-        tc_rows<PASSES, D, true, true>(tcx, D, C,
+        tc_rows2<PASSES, D, true, true>(tcx, D, C,
+            [&](int) { return tc::Src{Phi, D, 0, true, false}; },
             [&](int i, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = Phi[(size_t)(t + u) * D + i]; },
+            [&](int) { return tc::no_src(); },
             [&](int cc, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = c.U(t + u, cc); },
             tc::RowStore{Bn, D});
     }
@@ -331,7 +366,8 @@ __device__ void compute_Y(TcCta& tcx, const Chunk<Tin, D>& c, const float* S, si
     const int C = L.C;
     float* s = c.s;
     const Fac<Tin, D> f = facs(c);
-    tc_rows<PASSES, D, false, true>(tcx, C, D + C,
+    tc_rows2<PASSES, D, false, true>(tcx, C, D + C,
+        [&](int k) { return k < D ? tc::no_src() : tc::Src{s + L.LK, C, D, false, false}; },
         [&](int t, int k, float* v) {
             if (k < D) {
                 ld4in(c.k + c.base + t * c.rs + k, v);
@@ -340,6 +376,7 @@ __device__ void compute_Y(TcCta& tcx, const Chunk<Tin, D>& c, const float* S, si
                 ld4(s + L.LK + (size_t)t * C + (k - D), v);
             }
         },
+        [&](int k) { return k < D ? tc::Src{S, D, 0, true, false} : tc::no_src(); },
         [&](int cc, int k, float* v) {
             if (k < D) for (int u = 0; u < 4; ++u) v[u] = __ldg(S + (size_t)(k + u) * D + cc);
             else for (int u = 0; u < 4; ++u) v[u] = c.U(k - D + u, cc);
@@ -356,7 +393,7 @@ __global__ void __launch_bounds__(kThreads) k_out(KParams p) {
     __shared__ int tc_status;
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
-    tcx.sbuf = dsm;
+    tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
     tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
@@ -378,7 +415,12 @@ __global__ void __launch_bounds__(kThreads) k_out(KParams p) {
         const Fac<Tin, D> f = facs(c);
         const float* Y = s + L.W[0];
         // O = Qt S + M_QK U - M_QA Y
-        tc_rows<PASSES, D, false, true>(tcx, C, D + 2 * C,
+        tc_rows2<PASSES, D, false, true>(tcx, C, D + 2 * C,
+            [&](int k) {
+                return k < D ? tc::no_src()
+                             : (k < D + C ? tc::Src{s + L.MQK, C, D, false, false}
+                                          : tc::Src{s + L.MQA, C, D + C, false, true});
+            },
             [&](int t, int k, float* v) {
                 if (k < D) {
                     float g4[4];
@@ -391,6 +433,10 @@ __global__ void __launch_bounds__(kThreads) k_out(KParams p) {
                     ld4(s + L.MQA + (size_t)t * C + (k - D - C), v);
                     for (int u = 0; u < 4; ++u) v[u] = -v[u];
                 }
+            },
+            [&](int k) {
+                return k < D ? tc::Src{S, D, 0, true, false}
+                             : (k < D + C ? tc::no_src() : tc::Src{Y, D, D + C, true, false});
             },
             [&](int cc, int k, float* v) {
                 if (k < D) for (int u = 0; u < 4; ++u) v[u] = __ldg(S + (size_t)(k + u) * D + cc);
@@ -411,7 +457,7 @@ __global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
     __shared__ int tc_status;
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
-    tcx.sbuf = dsm;
+    tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
     tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
@@ -429,8 +475,10 @@ __global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
         __syncthreads();
         float* Xi = s + L.W[0];
         // Z0 = M_QA^T dO
-        tc_rows<PASSES, D, true, true>(tcx, C, C,
+        tc_rows2<PASSES, D, true, true>(tcx, C, C,
+            [&](int) { return tc::Src{s + L.MQA, C, 0, true, false}; },
             [&](int t, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = s[L.MQA + (size_t)(k + u) * C + t]; },
+            [&](int) { return tc::no_src(); },
             [&](int cc, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc); },
             tc::RowStore{Xi, D});
         solve_s<D, PASSES, true>(s, sm, L, L.LA, L.W[0]);  // Xi = T^T Z0
@@ -438,11 +486,13 @@ __global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
         float* Bp = p.Bn + c.sbase;
         const Fac<Tin, D> f = facs(c);
         // B' = Qt^T dO - Kt^T Xi
-        tc_rows<PASSES, D, true, true>(tcx, D, 2 * C,
+        tc_rows2<PASSES, D, true, true>(tcx, D, 2 * C,
+            [&](int) { return tc::no_src(); },
             [&](int i, int k, float* v) {
                 if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.Qh(k + u, i) * f.eg(k + u, i);
                 else for (int u = 0; u < 4; ++u) v[u] = -c.K(k - C + u, i) * f.eg(k - C + u, i);
             },
+            [&](int k) { return k < C ? tc::no_src() : tc::Src{Xi, D, C, true, false}; },
             [&](int cc, int k, float* v) {
                 if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc);
                 else for (int u = 0; u < 4; ++u) v[u] = Xi[(size_t)(k - C + u) * D + cc];
@@ -464,7 +514,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
     __shared__ int tc_status;
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
-    tcx.sbuf = dsm;
+    tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
     tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
@@ -487,7 +537,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         compute_Y<Tin, D, PASSES>(tcx, c, S, Y);
         const Fac<Tin, D> f = facs(c);
         // dY = -M_QA^T dO - Ab dS'   (stored in dR, then dR = T^T dY)
-        tc_rows<PASSES, D, true, true>(tcx, C, C + D,
+        tc_rows2<PASSES, D, true, true>(tcx, C, C + D,
+            [&](int k) { return k < C ? tc::Src{s + L.MQA, C, 0, true, false} : tc::no_src(); },
             [&](int t, int k, float* v) {
                 if (k < C) for (int u = 0; u < 4; ++u) v[u] = s[L.MQA + (size_t)(k + u) * C + t];
                 else {
@@ -497,6 +548,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                     for (int u = 0; u < 4; ++u) v[u] *= k4[u] * f.egb(t, k - C + u);
                 }
             },
+            [&](int k) { return k < C ? tc::no_src() : tc::Src{dS, D, C, true, false}; },
             [&](int cc, int k, float* v) {
                 if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc);
                 else for (int u = 0; u < 4; ++u) v[u] = __ldg(dS + (size_t)(k - C + u) * D + cc);
@@ -509,26 +561,30 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         auto rowsdS = [&](int j, int k, float* v) { ld4in(dS + (size_t)j * D + k, v); };
         // raw products, then one elementwise pass applies the decay factors:
         //   dQt = dO S^T, dKt = dR S^T, dKb = U dS'^T, dAb = -Y dS'^T
-        tc_rows<PASSES, D, false, false>(tcx, C, D,
-            [&](int t, int k, float* v) { ld4in(c.dO + c.base + t * c.rs + k, v); }, rowsS,
+        auto srcS = [&](int) { return tc::Src{S, D, 0, false, false}; };
+        auto srcdS = [&](int) { return tc::Src{dS, D, 0, false, false}; };
+        tc_rows2<PASSES, D, false, false>(tcx, C, D, [&](int) { return tc::no_src(); },
+            [&](int t, int k, float* v) { ld4in(c.dO + c.base + t * c.rs + k, v); }, srcS, rowsS,
             tc::RowStore{s + dQh, D});
-        tc_rows<PASSES, D, false, false>(tcx, C, D,
-            [&](int t, int k, float* v) { ld4(s + dR + (size_t)t * D + k, v); }, rowsS,
+        tc_rows2<PASSES, D, false, false>(tcx, C, D,
+            [&](int) { return tc::Src{s + dR, D, 0, false, false}; },
+            [&](int t, int k, float* v) { ld4(s + dR + (size_t)t * D + k, v); }, srcS, rowsS,
             tc::RowStore{s + dK, D});
-        tc_rows<PASSES, D, false, false>(tcx, C, D,
+        tc_rows2<PASSES, D, false, false>(tcx, C, D, [&](int) { return tc::no_src(); },
             [&](int t, int k, float* v) {
                 float w4[4];
                 ld4in(c.v + c.base + t * c.rs + k, v);
                 ld4in(c.w + c.base + t * c.rs + k, w4);
                 for (int u = 0; u < 4; ++u) v[u] *= w4[u];
             },
-            rowsdS, tc::RowStore{s + dGam, D});
-        tc_rows<PASSES, D, false, false>(tcx, C, D,
+            srcdS, rowsdS, tc::RowStore{s + dGam, D});
+        tc_rows2<PASSES, D, false, false>(tcx, C, D,
+            [&](int) { return tc::Src{s + Y, D, 0, false, true}; },
             [&](int t, int k, float* v) {
                 ld4(s + Y + (size_t)t * D + k, v);
                 for (int u = 0; u < 4; ++u) v[u] = -v[u];
             },
-            rowsdS, tc::RowStore{s + dA, D});
+            srcdS, rowsdS, tc::RowStore{s + dA, D});
         float cpart[4] = {0.f, 0.f, 0.f, 0.f};  // this thread's share of the column sums
         // dQh = dQt e^Gam;  dK = dKt e^Gam + dKb e^{gbar-Gam};  dA = dAb e^{gbar-Gam};
         // dGam = dQt Qt + dKt Kt - dKb Kb - dAb Ab;  dgbar += sum_t (dKb Kb + dAb Ab)
@@ -571,7 +627,11 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         }
         __syncthreads();
         // dU = M_QK^T dO + L_K^T dR + Kb dS'
-        tc_rows<PASSES, D, true, true>(tcx, C, 2 * C + D,
+        tc_rows2<PASSES, D, true, true>(tcx, C, 2 * C + D,
+            [&](int k) {
+                return k < C ? tc::Src{s + L.MQK, C, 0, true, false}
+                             : (k < 2 * C ? tc::Src{s + L.LK, C, C, true, false} : tc::no_src());
+            },
             [&](int t, int k, float* v) {
                 if (k < C) for (int u = 0; u < 4; ++u) v[u] = s[L.MQK + (size_t)(k + u) * C + t];
                 else if (k < 2 * C) for (int u = 0; u < 4; ++u) v[u] = s[L.LK + (size_t)(k - C + u) * C + t];
@@ -579,6 +639,11 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                     ld4in(c.k + c.base + t * c.rs + (k - 2 * C), v);
                     for (int u = 0; u < 4; ++u) v[u] *= f.egb(t, k - 2 * C + u);
                 }
+            },
+            [&](int k) {
+                return k < C ? tc::no_src()
+                             : (k < 2 * C ? tc::Src{s + dR, D, C, true, false}
+                                          : tc::Src{dS, D, 2 * C, true, false});
             },
             [&](int cc, int k, float* v) {
                 if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc);
@@ -593,10 +658,18 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
             const bool incl = which >= 2;
             const float sg = (which == 0 || which == 3) ? -1.f : 1.f;
             for (int n0 = 0; n0 < C; n0 += 128) {
-                tc_rows<PASSES, 128, false, false>(tcx, C, D,
+                tc_rows2<PASSES, 128, false, false>(tcx, C, D,
+                    [&](int) {
+                        return which < 2 ? tc::Src{s + dR, D, 0, false, false} : tc::no_src();
+                    },
                     [&](int t, int k, float* v) {
                         if (which < 2) ld4(s + dR + (size_t)t * D + k, v);
                         else ld4in(c.dO + c.base + t * c.rs + k, v);
+                    },
+                    [&](int) {
+                        return (which == 0 || which == 3)
+                                   ? tc::Src{s + Y + (size_t)n0 * D, D, 0, false, false}
+                                   : tc::no_src();
                     },
                     [&](int n, int k, float* v) {
                         const int ss = n0 + n;
@@ -614,7 +687,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                         if (ss >= C) return;
                         const bool keep = incl ? ss <= t : ss < t;
                         s[out + (size_t)t * C + ss] = keep ? sg * x : 0.f;
-                    });
+                    },
+                    C - n0 < 128 ? C - n0 : 128);
             }
         }
         __syncthreads();
@@ -720,11 +794,12 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
 template <int D, int PASSES>
 int dyn_bytes(int C) {
     int f = tc::stage_bytes<PASSES, 128>() / 4;
+    if (PASSES == 1 && tc::async_stage_bytes<128>() / 4 > f) f = tc::async_stage_bytes<128>() / 4;
     const int m = masked_smem_floats(C, D), g = decayed_smem_floats(C), s = solve_smem_floats(C, D);
     f = f > m ? f : m;
     f = f > g ? f : g;
     f = f > s ? f : s;
-    return f * 4;
+    return f * 4 + 1024;  // + alignment of the staging buffers
 }
 
 // CTAs that fit on one SM next to each other with this much shared memory.

@@ -40,6 +40,12 @@ __device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint
     return d;                // base offset 0, legacy LBO mode, no swizzle
 }
 
+// Descriptor of an MN-major block in the 128-byte swizzle with 32-byte atoms
+// (layout type 1); the block starts on a 1024-byte boundary.
+__device__ __forceinline__ uint64_t make_desc_mn32(uint32_t saddr, uint32_t sbo) {
+    return make_desc(saddr, 512, sbo) | ((uint64_t)1 << 61);
+}
+
 // Instruction descriptor: kind::tf32, D = f32, A = B = tf32, both K-major.
 __host__ __device__ constexpr uint32_t idesc_tf32(int M, int N) {
     return (1u << 4) | (2u << 7) | (2u << 10) | ((uint32_t)(N >> 3) << 17) |
@@ -214,6 +220,186 @@ __device__ void gemm(State& s, unsigned char* sbuf, int M, int K, const FA4& fa4
         wait_mma(s);  // the slab buffers are free again and, after the last slab, D is final
     }
     // epilogue: warp w reads TMEM lanes [32 (w % 4), +32) and half of the columns
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int quarter = warp & 3, half = warp >> 2;
+    const int row = 32 * quarter + lane;
+    constexpr int NH = N / 2;
+    for (int c0 = half * NH; c0 < (half + 1) * NH; c0 += 8) {
+        uint32_t r[8];
+        const uint32_t taddr = s.tmem + ((uint32_t)(32 * quarter) << 16) + (uint32_t)c0;
+        asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];"
+                     : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]),
+                       "=r"(r[6]), "=r"(r[7])
+                     : "r"(taddr));
+        asm volatile("tcgen05.wait::ld.sync.aligned;");
+        if (row < M) {
+            if constexpr (std::is_same<EPI, RowStore>::value) {
+                float* d = epi.dst + (size_t)row * epi.ld + c0;
+                *reinterpret_cast<float4*>(d) = make_float4(__uint_as_float(r[0]), __uint_as_float(r[1]),
+                                                            __uint_as_float(r[2]), __uint_as_float(r[3]));
+                *reinterpret_cast<float4*>(d + 4) = make_float4(__uint_as_float(r[4]), __uint_as_float(r[5]),
+                                                                __uint_as_float(r[6]), __uint_as_float(r[7]));
+            } else {
+#pragma unroll
+                for (int j = 0; j < 8; ++j) epi(row, c0 + j, __uint_as_float(r[j]));
+            }
+        }
+    }
+    asm volatile("tcgen05.fence::before_thread_sync;");
+    __syncthreads();
+}
+
+
+// ------------------------------------------------------------------ asynchronous staging
+
+// One K segment of an operand that is copied verbatim from float32 memory by
+// cp.async (the tensor core reads it as TF32 by truncation; used for
+// intermediates only, input-derived operands keep round-to-nearest producers).
+struct Src {
+    const float* p;  // nullptr: this K range comes from the element producer
+    int ld;          // floats between consecutive source rows
+    int k0;          // first operand K index of the segment
+    bool mn;         // false: source rows are the operand's rows (K contiguous);
+                     // true:  source rows are K (the operand's rows contiguous)
+    bool neg;        // negate the segment's products (A operand only)
+};
+
+__device__ __forceinline__ Src no_src() { return Src{nullptr, 0, 0, false, false}; }
+
+__device__ __forceinline__ void cp_async16(uint32_t saddr, const void* g, bool valid) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(saddr), "l"(g),
+                 "r"(valid ? 16 : 0));
+}
+
+// One 8-deep K block of R rows.  K-major: core matrices 8 rows x 16 B,
+// LBO = 128 B (second 4-element K group), SBO = 256 B (next 8 rows).  MN-major
+// (32-bit operands accept only this form): 128-byte rows of 32 consecutive
+// M/N elements, one row per k, 4 rows per 512-byte atom, the 32-byte chunk
+// index of a row XORed with k % 4; LBO = 512 B (next 32 M/N elements), SBO =
+// R / 32 * 512 B (next 4 k).
+__device__ __forceinline__ uint32_t kblk_off(int r, int kk) {
+    return (uint32_t)((r >> 3) * 256 + (kk >> 2) * 128 + (r & 7) * 16 + (kk & 3) * 4);
+}
+
+template <int R>
+__device__ __forceinline__ void copy_block(unsigned char* blk, const Src& a, int k, int rvalid,
+                                           int kmax) {
+    const uint32_t base = smem_addr(blk);
+    if (!a.mn) {
+        for (int idx = threadIdx.x; idx < R * 2; idx += blockDim.x) {
+            const int r = idx >> 1, h = idx & 1;
+            const bool ok = r < rvalid && k + 4 * h < kmax;
+            const float* g = a.p + (size_t)(ok ? r : 0) * a.ld + (ok ? (k - a.k0 + 4 * h) : 0);
+            cp_async16(base + (uint32_t)((r >> 3) * 256 + h * 128 + (r & 7) * 16), g, ok);
+        }
+    } else {
+        static_assert(R % 32 == 0, "MN-major blocks hold whole 32-element rows");
+        constexpr uint32_t SBO = (R / 32) * 512;
+        for (int idx = threadIdx.x; idx < R * 2; idx += blockDim.x) {
+            const int m = 4 * (idx % (R / 4)), kk = idx / (R / 4);
+            const bool ok = m < rvalid && k + kk < kmax;
+            const float* g = a.p + (size_t)(ok ? (k - a.k0 + kk) : 0) * a.ld + (ok ? m : 0);
+            const uint32_t off = (uint32_t)((kk >> 2) * SBO + (m >> 5) * 512 + (kk & 3) * 128 +
+                                            ((((m & 31) >> 3) ^ (kk & 3)) << 5) + (m & 4) * 4);
+            cp_async16(base + off, g, ok);
+        }
+    }
+}
+
+template <int R, class F4>
+__device__ __forceinline__ void produce_block(unsigned char* blk, int k, int rvalid, int kmax,
+                                              const F4& f4) {
+    constexpr int ITEMS = (R * 2 + 255) / 256;
+    float v[ITEMS][4];
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) {
+        const int idx = threadIdx.x + it * 256;
+        const int r = idx >> 1, h = idx & 1;
+        v[it][0] = v[it][1] = v[it][2] = v[it][3] = 0.f;
+        if (idx < R * 2 && r < rvalid && k + 4 * h < kmax) f4(r, k + 4 * h, v[it]);
+    }
+#pragma unroll
+    for (int it = 0; it < ITEMS; ++it) {
+        const int idx = threadIdx.x + it * 256;
+        if (idx >= R * 2) break;
+        const int r = idx >> 1, h = idx & 1;
+        float4 x;
+        x.x = tf32_rn(v[it][0]); x.y = tf32_rn(v[it][1]); x.z = tf32_rn(v[it][2]); x.w = tf32_rn(v[it][3]);
+        *reinterpret_cast<float4*>(blk + kblk_off(r, 4 * h)) = x;
+    }
+}
+
+template <int N>
+__host__ __device__ constexpr int async_stage_bytes() {
+    return 2 * 4 * (128 + N) * 32;
+}
+
+// Same product as gemm<1, N, ...> (single TF32 pass) with the K segments that
+// asrc(k) / bsrc(k) describe copied asynchronously, two slabs in flight.
+// sbuf starts on a 1024-byte boundary; an MN-major B segment needs N % 32 == 0.
+template <int N, class ASRC, class FA4, class BSRC, class FB4, class EPI>
+__device__ void gemm_async(State& s, unsigned char* sbuf, int M, int NB, int K, const ASRC& asrc,
+                           const FA4& fa4, const BSRC& bsrc, const FB4& fb4, const EPI& epi) {
+    static_assert(N % 16 == 0 && N <= 256, "N");
+    constexpr int ABLK = 128 * 32, BBLK = N * 32;
+    constexpr int SLAB = 4 * (ABLK + BBLK);
+    const int nslab = (K + 31) / 32;
+    auto blkA = [&](int buf, int ks) { return sbuf + buf * SLAB + ks * ABLK; };
+    auto blkB = [&](int buf, int ks) { return sbuf + buf * SLAB + 4 * ABLK + ks * BBLK; };
+    auto issue_copies = [&](int sl, int buf) {
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const int k = sl * 32 + ks * 8;
+            if (k >= K) break;
+            const Src a = asrc(k), b = bsrc(k);
+            if (a.p) copy_block<128>(blkA(buf, ks), a, k, M, K);
+            if (b.p) copy_block<N>(blkB(buf, ks), b, k, NB, K);
+        }
+        asm volatile("cp.async.commit_group;");
+    };
+    auto run_producers = [&](int sl, int buf) {
+#pragma unroll
+        for (int ks = 0; ks < 4; ++ks) {
+            const int k = sl * 32 + ks * 8;
+            if (k >= K) break;
+            if (!asrc(k).p) produce_block<128>(blkA(buf, ks), k, M, K, fa4);
+            if (!bsrc(k).p) produce_block<N>(blkB(buf, ks), k, NB, K, fb4);
+        }
+    };
+    issue_copies(0, 0);
+    run_producers(0, 0);
+    for (int sl = 0; sl < nslab; ++sl) {
+        const int buf = sl & 1;
+        if (sl + 1 < nslab) {
+            issue_copies(sl + 1, buf ^ 1);
+            asm volatile("cp.async.wait_group 1;");
+        } else {
+            asm volatile("cp.async.wait_group 0;");
+        }
+        asm volatile("fence.proxy.async.shared::cta;");
+        __syncthreads();
+        if (threadIdx.x == 0) {
+            asm volatile("tcgen05.fence::after_thread_sync;");
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const int k = sl * 32 + ks * 8;
+                if (k >= K) break;
+                const Src a = asrc(k), b = bsrc(k);
+                const bool amn = a.p && a.mn, bmn = b.p && b.mn;
+                const uint64_t da = amn ? make_desc_mn32(smem_addr(blkA(buf, ks)), 128 / 32 * 512)
+                                        : make_desc(smem_addr(blkA(buf, ks)), 128, 256);
+                const uint64_t db = bmn ? make_desc_mn32(smem_addr(blkB(buf, ks)), N / 32 * 512)
+                                        : make_desc(smem_addr(blkB(buf, ks)), 128, 256);
+                const uint32_t idesc = idesc_tf32(128, N) | ((a.p && a.neg) ? (1u << 13) : 0u) |
+                                       (amn ? (1u << 15) : 0u) | (bmn ? (1u << 16) : 0u);
+                issue_mma(s.tmem, da, db, idesc, k > 0 ? 1u : 0u);
+            }
+            commit(s);
+        }
+        if (sl + 1 < nslab) run_producers(sl + 1, buf ^ 1);  // overlaps this slab's MMAs
+        wait_mma(s);
+    }
+    // epilogue (as in gemm)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int quarter = warp & 3, half = warp >> 2;
     const int row = 32 * quarter + lane;
