@@ -58,6 +58,8 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         SP = ctypes.POINTER(MuirShape)
+        L.muir_device_wait_status.argtypes = []
+        L.muir_device_wait_status.restype = I
         L.muir_status_string.argtypes = [I]
         L.muir_status_string.restype = ctypes.c_char_p
         L.muir_chunk_fwd_workspace.argtypes = [SP]
@@ -122,6 +124,12 @@ def _shape(q, v, chunk, out_dtype):
     dv = v.shape[-1]
     od = _dt(q) if out_dtype is None else (MUIR_BF16 if out_dtype == torch.bfloat16 else MUIR_FP32)
     return MuirShape(B, T, H, dk, dv, chunk, _dt(q), od)
+
+
+def device_wait_status() -> None:
+    """Synchronise the device and raise MuirError if a bounded wait inside a
+    chunk kernel expired since the previous check (muir_device_wait_status)."""
+    _check("muir_device_wait_status", lib().muir_device_wait_status())
 
 
 def fwd_workspace_bytes(B, T, H, d, chunk, dtype=torch.bfloat16) -> int:

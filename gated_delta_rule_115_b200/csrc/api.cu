@@ -4,6 +4,7 @@
 #include <stdint.h>
 
 #include "../../include/muir.h"
+#include "chunk_units.h"
 #include "kernels.h"
 
 namespace {
@@ -69,6 +70,13 @@ const char* muir_status_string(muir_status s) {
         case MUIR_ERR_DEVICE_TIMEOUT: return "MUIR_ERR_DEVICE_TIMEOUT: a bounded device wait expired";
     }
     return "MUIR_ERR_UNKNOWN";
+}
+
+muir_status muir_device_wait_status(void) {
+    if (cudaDeviceSynchronize() != cudaSuccess) return MUIR_ERR_CUDA;
+    const unsigned int n = muir::timeouts_bf16_d128() + muir::timeouts_bf16_d64() +
+                           muir::timeouts_f32_d128() + muir::timeouts_f32_d64();
+    return n ? MUIR_ERR_DEVICE_TIMEOUT : MUIR_OK;
 }
 
 size_t muir_chunk_fwd_workspace(const muir_shape* s) {

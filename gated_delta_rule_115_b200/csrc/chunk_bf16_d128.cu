@@ -21,4 +21,6 @@ cudaError_t bwd_bf16_d128(const ChunkProblem& P, const float* S0, const float* S
                                    dS0, ws, st);
 }
 
+unsigned int timeouts_bf16_d128() { return take_wait_timeouts(); }
+
 }  // namespace muir

@@ -17,4 +17,6 @@ cudaError_t bwd_f32_d64(const ChunkProblem& P, const float* S0, const float* S_c
                                    dS0, ws, st);
 }
 
+unsigned int timeouts_f32_d64() { return take_wait_timeouts(); }
+
 }  // namespace muir

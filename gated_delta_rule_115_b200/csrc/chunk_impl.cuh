@@ -50,13 +50,25 @@
 namespace muir {
 
 constexpr int kThreads = 256;
-constexpr int kMaxSlots = 296;  // 2 CTAs per SM on a 148-SM B200
+
+// Expired bounded waits (tc::wait_mma) of the chunk kernels in this
+// translation unit, read and cleared by take_wait_timeouts().
+static __device__ unsigned int g_wait_timeouts;
+
+inline unsigned int take_wait_timeouts() {
+    unsigned int n = 0, zero = 0;
+    if (cudaMemcpyFromSymbol(&n, g_wait_timeouts, sizeof(n)) != cudaSuccess) return 0;
+    cudaMemcpyToSymbol(g_wait_timeouts, &zero, sizeof(zero));
+    return n;
+}
+constexpr int kMaxSlots = 296;  // scratch slots: at most 2 resident CTAs per SM on a 148-SM B200
 
 // ------------------------------------------------------------------ scratch
 
 struct Lay {
     int C, D, nb8, nb16;
-    size_t LC, RC, BT, PRE, SUF, GBAR, LA, LK, MQK, MQA, TII, W[8], total;
+    size_t LC, RC, BT, PRE, SUF, GBAR, LA, LK, MQK, MQA, TII, W[8], PXK, PXQ, PZA, PZK;
+    size_t OXK, OXQ, OZA, OZK, MXK, MXQ, MZA, MZK, GK[4], GM[4], total;
 };
 
 __host__ __device__ inline Lay make_lay(int C, int D) {
@@ -70,6 +82,11 @@ __host__ __device__ inline Lay make_lay(int C, int D) {
     MUIR_TAKE(LA, cc) MUIR_TAKE(LK, cc) MUIR_TAKE(MQK, cc) MUIR_TAKE(MQA, cc)
     MUIR_TAKE(TII, (size_t)C * 16)
     for (int i = 0; i < 8; ++i) { MUIR_TAKE(W[i], cd) }
+    MUIR_TAKE(PXK, cd) MUIR_TAKE(PXQ, cd) MUIR_TAKE(PZA, cd) MUIR_TAKE(PZK, cd)
+    const size_t pd = (size_t)128 * D, pc = (size_t)C * 128;  // tiles padded to 128 rows
+    MUIR_TAKE(OXK, pd) MUIR_TAKE(OXQ, pd) MUIR_TAKE(OZA, cd) MUIR_TAKE(OZK, cd)
+    MUIR_TAKE(MXK, pc) MUIR_TAKE(MXQ, pc) MUIR_TAKE(MZA, pc) MUIR_TAKE(MZK, pc)
+    for (int i = 0; i < 4; ++i) { MUIR_TAKE(GK[i], cc) MUIR_TAKE(GM[i], cc) }
 #undef MUIR_TAKE
     L.total = o;
     return L;
@@ -97,6 +114,7 @@ struct Chunk {
     size_t rs, base, sbase;  // row stride (H*D), element offset of row 0, state offset
     float* s;                // scratch slot
     Lay L;
+    bool tame;               // decay span small enough for the single-pivot products
     __device__ float K(int t, int j) const { return ldf(k + base + t * rs + j); }
     __device__ float Qh(int t, int j) const {
         return ldf(gm + base + t * rs + j) * ldf(q + base + t * rs + j);
@@ -124,6 +142,7 @@ __device__ Chunk<Tin, D> make_chunk(const KParams& p, int chunk, float* slot) {
     c.sbase = ((size_t)bh * p.N + n) * D * D;
     c.s = slot;
     c.L = make_lay(CF ? CF : p.C, D);
+    c.tame = false;
     return c;
 }
 
@@ -189,7 +208,9 @@ struct TcCta {
     unsigned char* sbuf;
 };
 
-constexpr int kTmemCols = 128;
+// TMEM columns a chunk CTA allocates: 512 with the panel products (one CTA
+// per SM), 128 for the three-pass products.
+__host__ __device__ constexpr int tmem_cols(int passes) { return passes == 1 ? 512 : 128; }
 
 // Product over M rows (looped in 128-row tiles) and N = NT columns.
 template <int PASSES, int N, bool AR, bool BR, class FA4, class FB4, class EPI>
@@ -197,9 +218,14 @@ __device__ __forceinline__ void tc_rows(TcCta& t, int M, int K, const FA4& fa4, 
                                         const EPI& epi) {
     for (int m0 = 0; m0 < M; m0 += 128) {
         const int Mt = M - m0 < 128 ? M - m0 : 128;
-        tc::gemm<PASSES, N, AR, BR>(
-            t.st, t.sbuf, Mt, K, [&](int m, int k, float* v) { fa4(m0 + m, k, v); }, fb4,
-            [&](int m, int n, float x) { epi(m0 + m, n, x); });
+        auto fa = [&](int m, int k, float* v) { fa4(m0 + m, k, v); };
+        if constexpr (tc::is_row8<EPI>::value) {
+            auto e8 = [&](int m, int n0, const float* v) { epi.f(m0 + m, n0, v); };
+            tc::gemm<PASSES, N, AR, BR>(t.st, t.sbuf, Mt, K, fa, fb4, tc::Row8<decltype(e8)>{e8});
+        } else {
+            tc::gemm<PASSES, N, AR, BR>(t.st, t.sbuf, Mt, K, fa, fb4,
+                                        [&](int m, int n, float x) { epi(m0 + m, n, x); });
+        }
     }
 }
 
@@ -236,11 +262,63 @@ __device__ __forceinline__ void tc_rows2(TcCta& t, int M, int K, const ASRC& asr
             if constexpr (std::is_same<EPI, tc::RowStore>::value) {
                 tc::RowStore d = {epi.dst + (size_t)m0 * epi.ld, epi.ld};
                 tc::gemm_async<N>(t.st, t.sbuf, Mt, NB, K, as, fa, bsrc, fb4, d);
+            } else if constexpr (tc::is_row8<EPI>::value) {
+                auto e8 = [&](int m, int n0, const float* v) { epi.f(m0 + m, n0, v); };
+                tc::gemm_async<N>(t.st, t.sbuf, Mt, NB, K, as, fa, bsrc, fb4, tc::Row8<decltype(e8)>{e8});
             } else {
                 tc::gemm_async<N>(t.st, t.sbuf, Mt, NB, K, as, fa, bsrc, fb4,
                                   [&](int m, int n, float x) { epi(m0 + m, n, x); });
             }
         }
+    }
+}
+
+#include "panel.cuh"
+#include "fast.cuh"
+
+// Decay-masked pair: tensor-core panels for single-pass chunks of at most 128
+// tokens, 8-block mma.sync tiles otherwise.
+template <typename Tin, int D, int PASSES>
+__device__ __forceinline__ bool use_panels(const Chunk<Tin, D>& c) {
+    return PASSES == 1 && c.L.C <= 128;
+}
+
+// Per-chunk operands of the decay-masked products; decides between the
+// single-pivot products (small decay span) and the 8-token panels.
+template <typename Tin, int D, int PASSES>
+__device__ __forceinline__ void masked_prep(Chunk<Tin, D>& c, bool with_q, bool bwd) {
+    c.tame = false;
+    if (!use_panels<Tin, D, PASSES>(c)) return;
+    if (c.L.C >= 32) c.tame = chunk_tame(c);
+    if (c.tame) fast_prep<Tin, D>(c, with_q, bwd);
+    else panel_prep<Tin, D>(c, with_q);
+}
+
+template <typename Tin, int D, int PASSES, int X, int Z0, int Z1>
+__device__ __forceinline__ void masked_pair(const Chunk<Tin, D>& c, TcCta& tcx, float* sm,
+                                            size_t out0, size_t out1, bool incl0, bool incl1) {
+    if (c.tame)
+        fast_masked_pair<Tin, D, X, Z0, Z1>(c, tcx, out0, out1, incl0, incl1);
+    else if (use_panels<Tin, D, PASSES>(c))
+        panel_masked_pair<Tin, D, X, Z0, Z1>(c, tcx, out0, out1, incl0, incl1);
+    else
+        masked_pair_s<Tin, D, PASSES, X, Z0, Z1>(c, sm, out0, out1, incl0, incl1);
+}
+
+// epi(integral_constant<int, N>, t0, j, v) consumes the results of N
+// consecutive tokens t0.. at channel j.
+template <typename Tin, int D, int PASSES, bool XSIDE, int op0, int op1, class EPI>
+__device__ __forceinline__ void decayed_grad(const Chunk<Tin, D>& c, TcCta& tcx, float* sm,
+                                             size_t G0, size_t G1, const EPI& epi) {
+    if (c.tame) {
+        fast_grad<Tin, D, XSIDE, op0, op1>(c, tcx, G0, G1, epi);
+    } else if (use_panels<Tin, D, PASSES>(c)) {
+        if constexpr (XSIDE) panel_grad_x<Tin, D, op0, op1>(c, tcx, G0, G1, epi);
+        else panel_grad_z<Tin, D, op0, op1>(c, tcx, G0, G1, epi);
+    } else {
+        decayed_grad_any<Tin, D, PASSES, XSIDE, op0, op1>(c, sm, G0, G1, [&](int t, int j, float v) {
+            epi(std::integral_constant<int, 1>{}, t, j, &v);
+        });
     }
 }
 
@@ -254,17 +332,18 @@ __global__ void __launch_bounds__(kThreads) k_intra(KParams p) {
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
     tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
-    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, tmem_cols(PASSES));
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
-        const Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
+        Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
         const Lay& L = c.L;
         const int C = L.C;
         float* s = c.s;
         prologue2(c);
-        masked_pair_s<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, sm, L.LA, L.LK, false, false);
+        masked_prep<Tin, D, PASSES>(c, false, false);
+        masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
         __syncthreads();
         compute_tii(s, L, L.LA);
         for (int idx = threadIdx.x; idx < C * D; idx += kThreads)
@@ -304,7 +383,8 @@ __global__ void __launch_bounds__(kThreads) k_intra(KParams p) {
             [&](int cc, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = c.U(t + u, cc); },
             tc::RowStore{Bn, D});
     }
-    tc::release(tcx.st, kTmemCols);
+    if (threadIdx.x == 0 && tc_status != 0) atomicAdd(&g_wait_timeouts, 1u);
+    tc::release(tcx.st, tmem_cols(PASSES));
 }
 
 // ------------------------------------------------------------------ k_chain
@@ -394,18 +474,19 @@ __global__ void __launch_bounds__(kThreads) k_out(KParams p) {
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
     tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
-    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, tmem_cols(PASSES));
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
-        const Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
+        Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
         const Lay& L = c.L;
         const int C = L.C;
         float* s = c.s;
         prologue2(c);
-        masked_pair_s<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, sm, L.LA, L.LK, false, false);
-        masked_pair_s<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, sm, L.MQK, L.MQA, true, true);
+        masked_prep<Tin, D, PASSES>(c, true, false);
+        masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
+        masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
         __syncthreads();
         compute_tii(s, L, L.LA);
         __syncthreads();
@@ -445,7 +526,8 @@ __global__ void __launch_bounds__(kThreads) k_out(KParams p) {
             },
             [&](int t, int j, float x) { stf(o + c.base + t * c.rs + j, x); });
     }
-    tc::release(tcx.st, kTmemCols);
+    if (threadIdx.x == 0 && tc_status != 0) atomicAdd(&g_wait_timeouts, 1u);
+    tc::release(tcx.st, tmem_cols(PASSES));
 }
 
 // ------------------------------------------------------------------ k_bprep
@@ -458,18 +540,19 @@ __global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
     tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
-    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, tmem_cols(PASSES));
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
-        const Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
+        Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
         const Lay& L = c.L;
         const int C = L.C;
         float* s = c.s;
         prologue2(c);
-        masked_pair_s<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, sm, L.LA, L.LK, false, false);
-        masked_pair_s<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, sm, L.MQK, L.MQA, true, true);
+        masked_prep<Tin, D, PASSES>(c, true, false);
+        masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
+        masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
         __syncthreads();
         compute_tii(s, L, L.LA);
         __syncthreads();
@@ -499,7 +582,8 @@ __global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
             },
             tc::RowStore{Bp, D});
     }
-    tc::release(tcx.st, kTmemCols);
+    if (threadIdx.x == 0 && tc_status != 0) atomicAdd(&g_wait_timeouts, 1u);
+    tc::release(tcx.st, tmem_cols(PASSES));
 }
 
 // ------------------------------------------------------------------ k_bwd
@@ -515,12 +599,12 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
     tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
-    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, kTmemCols);
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, tmem_cols(PASSES));
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
     for (int chunk = blockIdx.x; chunk < nch; chunk += gridDim.x) {
-        const Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
+        Chunk<Tin, D> c = make_chunk<Tin, D, CF>(p, chunk, slot);
         const Lay& L = c.L;
         const int C = L.C;
         float* s = c.s;
@@ -529,8 +613,9 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         const size_t Y = L.W[0], dR = L.W[1], dK = L.W[2], dQh = L.W[3], dA = L.W[4],
                      dU = L.W[5], dGam = L.W[6];
         prologue2(c);
-        masked_pair_s<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, sm, L.LA, L.LK, false, false);
-        masked_pair_s<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, sm, L.MQK, L.MQA, true, true);
+        masked_prep<Tin, D, PASSES>(c, true, true);
+        masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
+        masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
         __syncthreads();
         compute_tii(s, L, L.LA);
         __syncthreads();
@@ -658,6 +743,22 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
             const bool incl = which >= 2;
             const float sg = (which == 0 || which == 3) ? -1.f : 1.f;
             for (int n0 = 0; n0 < C; n0 += 128) {
+                // masked, signed rows (and, for the single-pivot products, the
+                // tensor-core layouts of the same rows)
+                auto gepi = [&](int t, int n, const float* x) {
+                    const int s0 = n0 + n;
+                    if (s0 >= C) return;
+                    float w[8];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int ss = s0 + u;
+                        w[u] = (incl ? ss <= t : ss < t) ? sg * x[u] : 0.f;
+                    }
+                    float* d = s + out + (size_t)t * C + s0;
+                    *reinterpret_cast<float4*>(d) = make_float4(w[0], w[1], w[2], w[3]);
+                    *reinterpret_cast<float4*>(d + 4) = make_float4(w[4], w[5], w[6], w[7]);
+                    if (c.tame) store_g_layouts(s, L, which, t, s0, w);
+                };
                 tc_rows2<PASSES, 128, false, false>(tcx, C, D,
                     [&](int) {
                         return which < 2 ? tc::Src{s + dR, D, 0, false, false} : tc::no_src();
@@ -682,40 +783,43 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                             for (int u = 0; u < 4; ++u) v[u] *= w4[u];
                         }
                     },
-                    [&](int t, int n, float x) {
-                        const int ss = n0 + n;
-                        if (ss >= C) return;
-                        const bool keep = incl ? ss <= t : ss < t;
-                        s[out + (size_t)t * C + ss] = keep ? sg * x : 0.f;
-                    },
+                    tc::Row8<decltype(gepi)>{gepi},
                     C - n0 < 128 ? C - n0 : 128);
             }
         }
         __syncthreads();
         // X side: dK += dL_A (*) A + dL_K (*) K ; dQh += dM_QK (*) K + dM_QA (*) A ; dGam += X * dX
-        decayed_grad_any<Tin, D, PASSES, true, OP_A, OP_K>(c, sm, L.LA, L.LK, [&](int t, int j, float v) {
-            const size_t x = (size_t)t * D + j;
-            s[dK + x] += v;
-            s[dGam + x] += c.K(t, j) * v;
-        });
-        decayed_grad_any<Tin, D, PASSES, true, OP_K, OP_A>(c, sm, L.MQK, L.MQA, [&](int t, int j, float v) {
-            const size_t x = (size_t)t * D + j;
-            s[dQh + x] += v;
-            s[dGam + x] += c.Qh(t, j) * v;
-        });
+        // dst[t][j] += v and dGam[t][j] += sg * op_tj * v for N consecutive tokens
+        // (all loads first, then the stores)
+        auto accum = [&](size_t dst, auto opk, float sg) {
+            return [&, dst, sg](auto NN, int t0, int j, const float* v) {
+                constexpr int N = decltype(NN)::value;
+                float a[N], gm[N], o[N];
+#pragma unroll
+                for (int u = 0; u < N; ++u) {
+                    const size_t x = (size_t)(t0 + u) * D + j;
+                    a[u] = s[dst + x];
+                    gm[u] = s[dGam + x];
+                    o[u] = opval(c, decltype(opk)::value, t0 + u, j);
+                }
+#pragma unroll
+                for (int u = 0; u < N; ++u) {
+                    const size_t x = (size_t)(t0 + u) * D + j;
+                    s[dst + x] = a[u] + v[u];
+                    s[dGam + x] = gm[u] + sg * o[u] * v[u];
+                }
+            };
+        };
+        using OK_ = std::integral_constant<int, OP_K>;
+        using OQ_ = std::integral_constant<int, OP_Q>;
+        using OA_ = std::integral_constant<int, OP_A>;
+        decayed_grad<Tin, D, PASSES, true, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, accum(dK, OK_{}, 1.f));
+        decayed_grad<Tin, D, PASSES, true, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, accum(dQh, OQ_{}, 1.f));
         __syncthreads();
         // Z side: dA += dL_A^T (*) K + dM_QA^T (*) Qh ; dK += dL_K^T (*) K + dM_QK^T (*) Qh ; dGam -= Z * dZ
-        decayed_grad_any<Tin, D, PASSES, false, OP_K, OP_Q>(c, sm, L.LA, L.MQA, [&](int t, int j, float v) {
-            const size_t x = (size_t)t * D + j;
-            s[dA + x] += v;
-            s[dGam + x] -= c.A(t, j) * v;
-        });
+        decayed_grad<Tin, D, PASSES, false, OP_K, OP_Q>(c, tcx, sm, L.LA, L.MQA, accum(dA, OA_{}, -1.f));
         __syncthreads();
-        decayed_grad_any<Tin, D, PASSES, false, OP_K, OP_Q>(c, sm, L.LK, L.MQK, [&](int t, int j, float v) {
-            const size_t x = (size_t)t * D + j;
-            s[dK + x] += v;
-            s[dGam + x] -= c.K(t, j) * v;
-        });
+        decayed_grad<Tin, D, PASSES, false, OP_K, OP_Q>(c, tcx, sm, L.LK, L.MQK, accum(dK, OK_{}, -1.f));
         __syncthreads();
         // dgbar_j = e^gbar_j sum_c S[j][c] dS'[j][c] + sum_t (dKb Kb + dAb Ab)[t][j]
         Tin* gq = (Tin*)p.dq; Tin* gk = (Tin*)p.dk; Tin* gv = (Tin*)p.dv; Tin* gg = (Tin*)p.dg;
@@ -784,7 +888,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         }
         __syncthreads();
     }
-    tc::release(tcx.st, kTmemCols);
+    if (threadIdx.x == 0 && tc_status != 0) atomicAdd(&g_wait_timeouts, 1u);
+    tc::release(tcx.st, tmem_cols(PASSES));
 }
 
 // ------------------------------------------------------------------ host side
@@ -799,11 +904,11 @@ int dyn_bytes(int C) {
     f = f > m ? f : m;
     f = f > g ? f : g;
     f = f > s ? f : s;
+    if (PASSES == 1 && panel_smem_bytes() / 4 > f) f = panel_smem_bytes() / 4;
+    if (PASSES == 1 && kFastSmem / 4 > f) f = kFastSmem / 4;
     return f * 4 + 1024;  // + alignment of the staging buffers
 }
 
-// CTAs that fit on one SM next to each other with this much shared memory.
-inline int ctas_per_sm(int dyn) { return dyn <= 100 * 1024 ? 2 : 1; }
 
 template <typename Tin, int D, int PASSES, int CF>
 cudaError_t set_smem_attrs(int bytes) {
@@ -818,6 +923,21 @@ cudaError_t set_smem_attrs(int bytes) {
 inline int num_slots(int nch) { return nch < kMaxSlots ? nch : kMaxSlots; }
 
 inline size_t slot_floats(int C, int D) { return make_lay(C, D).total; }
+
+// Persistent grid of a chunk kernel: one CTA per resident slot (SM count x
+// CTAs that fit per SM with this shared memory and register use), at most one
+// per scratch slot.  Call after the kernel's shared-memory attribute is set.
+template <class KERNEL>
+int persistent_grid(KERNEL kernel, int nch, int dyn) {
+    int dev = 0, nsm = 148, occ = 1;
+    if (cudaGetDevice(&dev) == cudaSuccess)
+        cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, dyn) != cudaSuccess ||
+        occ < 1)
+        occ = 1;
+    const int g = num_slots(nch);
+    return g < nsm * occ ? g : nsm * occ;
+}
 
 template <int D, int PASSES, bool REV>
 cudaError_t launch_chain(int BH, int N, const float* M, const float* Bn, const float* S_in,
@@ -852,20 +972,19 @@ cudaError_t fwd_impl(const ChunkProblem& P, const float* S0, void* o, float* S_f
     kp.S_chunks = Sc;
     kp.o = o;
     const int dyn = dyn_bytes<D, PASSES>(P.C);
-    int grid = num_slots(nch);
-    const int resident = 148 * ctas_per_sm(dyn);
-    if (grid > resident) grid = resident;
     cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn);
     if (err != cudaSuccess) return err;
+    const int grid = persistent_grid(k_intra<Tin, D, PASSES, CF>, nch, dyn);
+    const int grid_o = persistent_grid(k_out<Tin, float, D, PASSES, CF>, nch, dyn);
     MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
     err = cudaGetLastError();
     if (err != cudaSuccess) return err;
     err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, S_final, st);
     if (err != cudaSuccess) return err;
     if (P.out_bf16)
-        MUIR_TIMED("k_out", st, k_out<Tin, __nv_bfloat16, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
+        MUIR_TIMED("k_out", st, k_out<Tin, __nv_bfloat16, D, PASSES, CF><<<grid_o, kThreads, dyn, st>>>(kp));
     else
-        MUIR_TIMED("k_out", st, k_out<Tin, float, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
+        MUIR_TIMED("k_out", st, k_out<Tin, float, D, PASSES, CF><<<grid_o, kThreads, dyn, st>>>(kp));
     return cudaGetLastError();
 }
 
@@ -893,11 +1012,11 @@ cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chun
     kp.dS_chunks = dSc;
     kp.dq = dq; kp.dk = dk; kp.dv = dv; kp.dg = dg; kp.de = de; kp.dw = dw; kp.dgamma = dgamma;
     const int dyn = dyn_bytes<D, PASSES>(P.C);
-    int grid = num_slots(nch);
-    const int resident = 148 * ctas_per_sm(dyn);
-    if (grid > resident) grid = resident;
     cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn);
     if (err != cudaSuccess) return err;
+    const int grid = persistent_grid(k_intra<Tin, D, PASSES, CF>, nch, dyn);
+    const int grid_p = persistent_grid(k_bprep<Tin, D, PASSES, CF>, nch, dyn);
+    const int grid_b = persistent_grid(k_bwd<Tin, D, PASSES, CF>, nch, dyn);
     const bool have_M = M_chunks != nullptr && !recompute;
     if (have_M) {
         kp.M = const_cast<float*>(M_chunks);  // the forward's transitions: nothing to recompute
@@ -910,11 +1029,11 @@ cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chun
         err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, nullptr, st);
         if (err != cudaSuccess) return err;
     }
-    MUIR_TIMED("k_bprep", st, k_bprep<Tin, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
+    MUIR_TIMED("k_bprep", st, k_bprep<Tin, D, PASSES, CF><<<grid_p, kThreads, dyn, st>>>(kp));
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     err = launch_chain<D, PASSES, true>(BH, P.N, kp.M, kp.Bn, dS_final, dSc, dS0, st);
     if (err != cudaSuccess) return err;
-    MUIR_TIMED("k_bwd", st, k_bwd<Tin, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
+    MUIR_TIMED("k_bwd", st, k_bwd<Tin, D, PASSES, CF><<<grid_b, kThreads, dyn, st>>>(kp));
     return cudaGetLastError();
 }
 

@@ -30,4 +30,10 @@ cudaError_t bwd_f32_d64(const ChunkProblem& P, const float* S0, const float* S_c
                           void* dg, void* de, void* dw, void* dgamma, float* dS0, void* ws,
                           cudaStream_t st);
 
+// Expired bounded waits recorded by each unit's kernels since the last call.
+unsigned int timeouts_bf16_d128();
+unsigned int timeouts_bf16_d64();
+unsigned int timeouts_f32_d128();
+unsigned int timeouts_f32_d64();
+
 }  // namespace muir

@@ -177,6 +177,17 @@ struct RowStore {
     int ld;      // floats between rows (multiple of 4)
 };
 
+// Epilogue that takes eight consecutive columns of one row at once:
+// f(row, c0, v[8]) with v[j] = D[row][c0 + j].
+template <class F>
+struct Row8 {
+    F f;
+};
+template <class T>
+struct is_row8 : std::false_type {};
+template <class F>
+struct is_row8<Row8<F>> : std::true_type {};
+
 // D (128 x N, TMEM) = sum over K of A(m, k) B(k, n).  fa4(m, k, v[4]) gives
 // A(m, k..k+3); fb4(n, k, v[4]) gives B(k..k+3, n).  Rows m >= M are zero.
 // Then epi(m, n, value) for m < M, n < N.  All threads of the CTA call it.
@@ -239,6 +250,11 @@ __device__ void gemm(State& s, unsigned char* sbuf, int M, int K, const FA4& fa4
                                                             __uint_as_float(r[2]), __uint_as_float(r[3]));
                 *reinterpret_cast<float4*>(d + 4) = make_float4(__uint_as_float(r[4]), __uint_as_float(r[5]),
                                                                 __uint_as_float(r[6]), __uint_as_float(r[7]));
+            } else if constexpr (is_row8<EPI>::value) {
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r[j]);
+                epi.f(row, c0, v);
             } else {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) epi(row, c0 + j, __uint_as_float(r[j]));
@@ -281,6 +297,13 @@ __device__ __forceinline__ uint32_t kblk_off(int r, int kk) {
     return (uint32_t)((r >> 3) * 256 + (kk >> 2) * 128 + (r & 7) * 16 + (kk & 3) * 4);
 }
 
+// Byte offset of the four consecutive M/N elements starting at m (m % 4 == 0)
+// in row kk of an 8-deep MN-major K block whose 4-row groups lie sbo bytes apart.
+__device__ __forceinline__ uint32_t mn_off(int m, int kk, uint32_t sbo) {
+    return (uint32_t)((kk >> 2) * sbo + (m >> 5) * 512 + (kk & 3) * 128 +
+                      ((((m & 31) >> 3) ^ (kk & 3)) << 5) + (m & 4) * 4);
+}
+
 template <int R>
 __device__ __forceinline__ void copy_block(unsigned char* blk, const Src& a, int k, int rvalid,
                                            int kmax) {
@@ -299,9 +322,7 @@ __device__ __forceinline__ void copy_block(unsigned char* blk, const Src& a, int
             const int m = 4 * (idx % (R / 4)), kk = idx / (R / 4);
             const bool ok = m < rvalid && k + kk < kmax;
             const float* g = a.p + (size_t)(ok ? (k - a.k0 + kk) : 0) * a.ld + (ok ? m : 0);
-            const uint32_t off = (uint32_t)((kk >> 2) * SBO + (m >> 5) * 512 + (kk & 3) * 128 +
-                                            ((((m & 31) >> 3) ^ (kk & 3)) << 5) + (m & 4) * 4);
-            cp_async16(base + off, g, ok);
+            cp_async16(base + mn_off(m, kk, SBO), g, ok);
         }
     }
 }
@@ -419,6 +440,11 @@ __device__ void gemm_async(State& s, unsigned char* sbuf, int M, int NB, int K, 
                                                             __uint_as_float(r[2]), __uint_as_float(r[3]));
                 *reinterpret_cast<float4*>(d + 4) = make_float4(__uint_as_float(r[4]), __uint_as_float(r[5]),
                                                                 __uint_as_float(r[6]), __uint_as_float(r[7]));
+            } else if constexpr (is_row8<EPI>::value) {
+                float v[8];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) v[j] = __uint_as_float(r[j]);
+                epi.f(row, c0, v);
             } else {
 #pragma unroll
                 for (int j = 0; j < 8; ++j) epi(row, c0 + j, __uint_as_float(r[j]));

@@ -67,6 +67,15 @@ typedef struct {
 /* Human-readable name of a status code (static string, never NULL). */
 const char* muir_status_string(muir_status s);
 
+/* Bounded device waits.  The chunk kernels wait on tensor-core completion
+ * barriers with an iteration limit; a wait that runs out records the fact and
+ * lets the kernel finish (its results are then not to be trusted) instead of
+ * hanging the GPU.  This call synchronises the current device, returns
+ * MUIR_ERR_DEVICE_TIMEOUT if any such wait expired since the previous call
+ * (MUIR_ERR_CUDA if the synchronisation itself failed, else MUIR_OK) and
+ * clears the record. */
+muir_status muir_device_wait_status(void);
+
 /* Bytes of device workspace muir_chunk_fwd / muir_chunk_bwd need for this
  * shape (0 for an invalid shape).  Host-only; enqueues nothing. */
 size_t muir_chunk_fwd_workspace(const muir_shape* shape);

@@ -30,6 +30,14 @@ def muir():
     return m
 
 
+@pytest.fixture(autouse=True)
+def no_expired_waits(muir):
+    """Every test ends with no expired bounded wait in any chunk kernel."""
+    muir.device_wait_status()
+    yield
+    muir.device_wait_status()
+
+
 def to_dev(x):
     return {k: (v.cuda() if v is not None else None) for k, v in x.items()}
 
@@ -155,6 +163,61 @@ def test_chunk_bwd_reuses_states(muir):
                        M_chunks=Mc2)
     for k in a:
         assert torch.equal(a[k], c[k]), k
+
+
+# ------------------------------------------------- span-dependent product paths
+
+# Chunks whose per-channel log decay over the chunk stays within 140 take
+# single-pivot products; larger spans take the 8-token pivoted panels.  These
+# cases scale g so that every chunk, or every other chunk, needs the panels.
+SPAN_CASES = [
+    ("all-panels", 3.0, None),
+    ("mixed", 3.0, 2),
+]
+
+
+def _span_inputs(scale, every):
+    from gated_delta_rule_115_b200 import inputs as I
+    x = I.chunk_inputs(2, B=1, H=2, T=512, s0_std=1.0)
+    g = x["g"].float()
+    if every is None:
+        g = g * scale
+    else:  # scale the tokens of every other 128-token chunk
+        T = g.shape[1]
+        idx = torch.arange(T) // 128
+        sel = (idx % every == 0).view(1, T, 1, 1)
+        g = torch.where(sel, g * scale, g)
+    x["g"] = g.to(x["g"].dtype)
+    return x
+
+
+@pytest.mark.parametrize("name,scale,every", SPAN_CASES)
+def test_chunk_fwd_span_paths(muir, oracle_mod, name, scale, every):
+    x = _span_inputs(scale, every)
+    d = to_dev(x)
+    o, S, Sc = muir.chunk_fwd(*[d[n] for n in NAMES], d["S0"], chunk=128, out_dtype=torch.float32,
+                              return_chunk_states=True)
+    ro, rS, rSc = oracle_mod.chunk_fwd(*[x[n] for n in NAMES], S0=x["S0"], chunk=128)
+    torch.cuda.synchronize()
+    eo, eS, eC = nmax(o, ro), nmax(S, rS), nmax(Sc, rSc)
+    print(f"fwd span {name}: o {eo:.2e} S {eS:.2e} chunk states {eC:.2e}")
+    assert eo < TOL_FWD["bf16"] and eS < TOL_FWD["bf16"] and eC < TOL_FWD["bf16"]
+
+
+@pytest.mark.parametrize("name,scale,every", SPAN_CASES)
+def test_chunk_bwd_span_paths(muir, oracle_mod, name, scale, every):
+    x = _span_inputs(scale, every)
+    B, T, H, dk = x["q"].shape
+    dSf = torch.randn(B, H, dk, dk, generator=torch.Generator().manual_seed(7))
+    d = to_dev(x)
+    gr = muir.chunk_bwd(*[d[n] for n in NAMES], d["S0"], d["dO"], dSf.cuda(), chunk=128)
+    rg = oracle_mod.bwd(*[x[n] for n in NAMES], S0=x["S0"], dO=x["dO"], dS_final=dSf)
+    torch.cuda.synchronize()
+    errs = {n: nmax(gr["d" + n], rg["d" + n]) for n in NAMES}
+    errs["S0"] = nmax(gr["dS0"], rg["dS0"])
+    print(f"bwd span {name}: " + " ".join(f"d{k} {v:.2e}" for k, v in errs.items()))
+    for n, e in errs.items():
+        assert e < TOL_BWD["bf16"], (n, e)
 
 
 # ------------------------------------------------------------ full-size workloads
