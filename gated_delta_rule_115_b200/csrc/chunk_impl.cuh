@@ -208,9 +208,13 @@ struct TcCta {
     unsigned char* sbuf;
 };
 
-// TMEM columns a chunk CTA allocates: 512 with the panel products (one CTA
-// per SM), 128 for the three-pass products.
-__host__ __device__ constexpr int tmem_cols(int passes) { return passes == 1 ? 512 : 128; }
+// TMEM columns a chunk CTA allocates: single-pass k_bwd 512 (one CTA per SM);
+// the other single-pass kernels 256 (two CTAs per SM); three-pass 128.
+__host__ __device__ constexpr int tmem_cols(int passes, bool bwd = false) {
+    return passes == 1 ? (bwd ? 512 : 256) : 128;
+}
+// CTAs per SM the single-pass forward-side kernels are compiled for.
+__host__ __device__ constexpr int fwd_ctas(int passes) { return passes == 1 ? 2 : 1; }
 
 // Product over M rows (looped in 128-row tiles) and N = NT columns.
 template <int PASSES, int N, bool AR, bool BR, class FA4, class FB4, class EPI>
@@ -325,7 +329,7 @@ __device__ __forceinline__ void decayed_grad(const Chunk<Tin, D>& c, TcCta& tcx,
 // ------------------------------------------------------------------ k_intra
 
 template <typename Tin, int D, int PASSES, int CF>
-__global__ void __launch_bounds__(kThreads) k_intra(KParams p) {
+__global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_intra(KParams p) {
     __shared__ uint32_t tmem_slot;
     __shared__ __align__(8) uint64_t mbar;
     __shared__ int tc_status;
@@ -467,7 +471,7 @@ __device__ void compute_Y(TcCta& tcx, const Chunk<Tin, D>& c, const float* S, si
 }
 
 template <typename Tin, typename Tout, int D, int PASSES, int CF>
-__global__ void __launch_bounds__(kThreads) k_out(KParams p) {
+__global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_out(KParams p) {
     __shared__ uint32_t tmem_slot;
     __shared__ __align__(8) uint64_t mbar;
     __shared__ int tc_status;
@@ -533,7 +537,7 @@ __global__ void __launch_bounds__(kThreads) k_out(KParams p) {
 // ------------------------------------------------------------------ k_bprep
 
 template <typename Tin, int D, int PASSES, int CF>
-__global__ void __launch_bounds__(kThreads) k_bprep(KParams p) {
+__global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_bprep(KParams p) {
     __shared__ uint32_t tmem_slot;
     __shared__ __align__(8) uint64_t mbar;
     __shared__ int tc_status;
@@ -599,7 +603,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
     tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
-    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, tmem_cols(PASSES));
+    tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, tmem_cols(PASSES, true));
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
     const int nch = p.B * p.H * p.N;
@@ -889,7 +893,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         __syncthreads();
     }
     if (threadIdx.x == 0 && tc_status != 0) atomicAdd(&g_wait_timeouts, 1u);
-    tc::release(tcx.st, tmem_cols(PASSES));
+    tc::release(tcx.st, tmem_cols(PASSES, true));
 }
 
 // ------------------------------------------------------------------ host side
@@ -897,26 +901,46 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
 // Dynamic shared memory of the per-chunk kernels: the largest staging area of
 // their phases (tensor-core slabs, masked products, gradient products, solves).
 template <int D, int PASSES>
-int dyn_bytes(int C) {
+int dyn_bytes(int C, bool bwd) {
     int f = tc::stage_bytes<PASSES, 128>() / 4;
     if (PASSES == 1 && tc::async_stage_bytes<128>() / 4 > f) f = tc::async_stage_bytes<128>() / 4;
-    const int m = masked_smem_floats(C, D), g = decayed_smem_floats(C), s = solve_smem_floats(C, D);
+    const int m = masked_smem_floats(C, D), s = solve_smem_floats(C, D);
     f = f > m ? f : m;
-    f = f > g ? f : g;
     f = f > s ? f : s;
-    if (PASSES == 1 && panel_smem_bytes() / 4 > f) f = panel_smem_bytes() / 4;
-    if (PASSES == 1 && kFastSmem / 4 > f) f = kFastSmem / 4;
+    if (PASSES == 1 && C <= 128) {
+        const int pr = pair_smem_bytes() / 4, fp = kFastPairSmem / 4;
+        f = f > pr ? f : pr;
+        f = f > fp ? f : fp;
+    }
+    if (bwd) {
+        const int g = decayed_smem_floats(C);
+        f = f > g ? f : g;
+        if (PASSES == 1 && C <= 128) {
+            const int pg = panel_smem_bytes() / 4, fg = kFastGradSmem / 4;
+            f = f > pg ? f : pg;
+            f = f > fg ? f : fg;
+        }
+    }
     return f * 4 + 1024;  // + alignment of the staging buffers
 }
 
 
 template <typename Tin, int D, int PASSES, int CF>
-cudaError_t set_smem_attrs(int bytes) {
-    cudaError_t e = cudaFuncSetAttribute(k_intra<Tin, D, PASSES, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_out<Tin, float, D, PASSES, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_out<Tin, __nv_bfloat16, D, PASSES, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_bprep<Tin, D, PASSES, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
-    if (e == cudaSuccess) e = cudaFuncSetAttribute(k_bwd<Tin, D, PASSES, CF>, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+cudaError_t set_smem_attrs(int bytes, int bwd_bytes) {
+    // dynamic shared memory limit and the largest shared-memory carveout, so
+    // that as many CTAs as the budgets allow fit on one SM
+    auto set = [](const void* f, int n) {
+        cudaError_t e = cudaFuncSetAttribute(f, cudaFuncAttributeMaxDynamicSharedMemorySize, n);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(f, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                     (int)cudaSharedmemCarveoutMaxShared);
+        return e;
+    };
+    cudaError_t e = set((const void*)k_intra<Tin, D, PASSES, CF>, bytes);
+    if (e == cudaSuccess) e = set((const void*)k_out<Tin, float, D, PASSES, CF>, bytes);
+    if (e == cudaSuccess) e = set((const void*)k_out<Tin, __nv_bfloat16, D, PASSES, CF>, bytes);
+    if (e == cudaSuccess) e = set((const void*)k_bprep<Tin, D, PASSES, CF>, bytes);
+    if (e == cudaSuccess) e = set((const void*)k_bwd<Tin, D, PASSES, CF>, bwd_bytes);
     return e;
 }
 
@@ -925,16 +949,31 @@ inline int num_slots(int nch) { return nch < kMaxSlots ? nch : kMaxSlots; }
 inline size_t slot_floats(int C, int D) { return make_lay(C, D).total; }
 
 // Persistent grid of a chunk kernel: one CTA per resident slot (SM count x
-// CTAs that fit per SM with this shared memory and register use), at most one
-// per scratch slot.  Call after the kernel's shared-memory attribute is set.
+// CTAs that fit per SM by registers, shared memory and threads, from the
+// kernel's attributes), at most one per scratch slot.  Call after the
+// kernel's shared-memory attribute is set.  (The runtime occupancy query
+// reports one CTA per SM for these kernels where two fit.)  CTAs never wait
+// on one another, so an over-estimate only delays the surplus CTAs.
 template <class KERNEL>
 int persistent_grid(KERNEL kernel, int nch, int dyn) {
-    int dev = 0, nsm = 148, occ = 1;
-    if (cudaGetDevice(&dev) == cudaSuccess)
+    int dev = 0, nsm = 148, regs_sm = 65536, smem_sm = 233472, reserve = 1024;
+    if (cudaGetDevice(&dev) == cudaSuccess) {
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernel, kThreads, dyn) != cudaSuccess ||
-        occ < 1)
-        occ = 1;
+        cudaDeviceGetAttribute(&regs_sm, cudaDevAttrMaxRegistersPerMultiprocessor, dev);
+        cudaDeviceGetAttribute(&smem_sm, cudaDevAttrMaxSharedMemoryPerMultiprocessor, dev);
+        cudaDeviceGetAttribute(&reserve, cudaDevAttrReservedSharedMemoryPerBlock, dev);
+    }
+    int occ = 1;
+    cudaFuncAttributes fa;
+    if (cudaFuncGetAttributes(&fa, kernel) == cudaSuccess && fa.numRegs > 0) {
+        const int warp_regs = ((fa.numRegs * 32 + 255) / 256) * 256;  // per-warp allocation unit
+        const int by_regs = regs_sm / (warp_regs * (kThreads / 32));
+        const int by_smem = smem_sm / ((int)fa.sharedSizeBytes + dyn + reserve);
+        const int by_thr = 2048 / kThreads;
+        occ = by_regs < by_smem ? by_regs : by_smem;
+        occ = occ < by_thr ? occ : by_thr;
+        if (occ < 1) occ = 1;
+    }
     const int g = num_slots(nch);
     return g < nsm * occ ? g : nsm * occ;
 }
@@ -971,8 +1010,8 @@ cudaError_t fwd_impl(const ChunkProblem& P, const float* S0, void* o, float* S_f
     kp.slot = slot_floats(P.C, D);
     kp.S_chunks = Sc;
     kp.o = o;
-    const int dyn = dyn_bytes<D, PASSES>(P.C);
-    cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn);
+    const int dyn = dyn_bytes<D, PASSES>(P.C, false);
+    cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn, dyn_bytes<D, PASSES>(P.C, true));
     if (err != cudaSuccess) return err;
     const int grid = persistent_grid(k_intra<Tin, D, PASSES, CF>, nch, dyn);
     const int grid_o = persistent_grid(k_out<Tin, float, D, PASSES, CF>, nch, dyn);
@@ -1011,12 +1050,12 @@ cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chun
     kp.S_chunks = Sc;
     kp.dS_chunks = dSc;
     kp.dq = dq; kp.dk = dk; kp.dv = dv; kp.dg = dg; kp.de = de; kp.dw = dw; kp.dgamma = dgamma;
-    const int dyn = dyn_bytes<D, PASSES>(P.C);
-    cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn);
+    const int dyn = dyn_bytes<D, PASSES>(P.C, false), dyn_b = dyn_bytes<D, PASSES>(P.C, true);
+    cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn, dyn_b);
     if (err != cudaSuccess) return err;
     const int grid = persistent_grid(k_intra<Tin, D, PASSES, CF>, nch, dyn);
     const int grid_p = persistent_grid(k_bprep<Tin, D, PASSES, CF>, nch, dyn);
-    const int grid_b = persistent_grid(k_bwd<Tin, D, PASSES, CF>, nch, dyn);
+    const int grid_b = persistent_grid(k_bwd<Tin, D, PASSES, CF>, nch, dyn_b);
     const bool have_M = M_chunks != nullptr && !recompute;
     if (have_M) {
         kp.M = const_cast<float*>(M_chunks);  // the forward's transitions: nothing to recompute
@@ -1033,7 +1072,7 @@ cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chun
     if ((err = cudaGetLastError()) != cudaSuccess) return err;
     err = launch_chain<D, PASSES, true>(BH, P.N, kp.M, kp.Bn, dS_final, dSc, dS0, st);
     if (err != cudaSuccess) return err;
-    MUIR_TIMED("k_bwd", st, k_bwd<Tin, D, PASSES, CF><<<grid_b, kThreads, dyn, st>>>(kp));
+    MUIR_TIMED("k_bwd", st, k_bwd<Tin, D, PASSES, CF><<<grid_b, kThreads, dyn_b, st>>>(kp));
     return cudaGetLastError();
 }
 

@@ -27,7 +27,8 @@
 // (included inside namespace muir)
 
 constexpr float kTameSpan = 140.f;
-constexpr int kFastSmem = 3 * 65536;  // three 64 KB operand tiles
+constexpr int kFastPairSmem = 3 * 32768;  // masked pair: three 32 KB half tiles
+constexpr int kFastGradSmem = 2 * 65536;  // gradient products: two 64 KB tiles
 
 // True (for all threads) when every channel's chunk log decay |gbar| <= kTameSpan.
 template <typename Tin, int D>
@@ -134,35 +135,43 @@ __device__ __forceinline__ void fast_mma(tc::State& st, const ISSUE& issue) {
 // ------------------------------------------------------------------ masked products
 
 // out_p[t][s] = [X (*) Z_p]_{ts} masked to s < t (strict) or s <= t, p = 0, 1:
-// Xo Zo_p^T into TMEM columns 256 p + s (lane t).
+// Xo Zo_p^T into TMEM columns 128 p + s (lane t), the channels in two halves
+// (96 KB of shared memory, 256 TMEM columns).
 template <typename Tin, int D, int X, int Z0, int Z1>
 __device__ void fast_masked_pair(const Chunk<Tin, D>& c, TcCta& tcx, size_t out0, size_t out1,
                                  bool incl0, bool incl1) {
     const Lay& L = c.L;
     const int C = L.C, nb8 = L.nb8;
     const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    constexpr int KH = D / 16;                 // K blocks per channel half
+    const uint32_t ah = KH * 4096, bh = (uint32_t)KH * C * 32;
     unsigned char* A = tcx.sbuf;
-    unsigned char* B0 = A + 65536;
-    unsigned char* B1 = A + 131072;
-    const Bulk b[3] = {{A, c.s + (X == OP_Q ? L.OXQ : L.OXK), 128u * D * 4},
-                       {B0, c.s + (Z0 == OP_A ? L.OZA : L.OZK), (uint32_t)C * D * 4},
-                       {B1, c.s + (Z1 == OP_A ? L.OZA : L.OZK), (uint32_t)C * D * 4}};
-    bulk_load(tcx.st, b);
-    fast_mma(tcx.st, [&]() {
-        const uint32_t idesc = tc::idesc_tf32(128, C);
-        for (int kb = 0; kb < D / 8; ++kb) {
-            const uint64_t da = tc::make_desc(tc::smem_addr(A + kb * 4096), 128, 256);
-            const uint64_t d0 = tc::make_desc(tc::smem_addr(B0 + kb * C * 32), 128, 256);
-            const uint64_t d1 = tc::make_desc(tc::smem_addr(B1 + kb * C * 32), 128, 256);
-            tc::issue_mma(tcx.st.tmem, da, d0, idesc, kb > 0 ? 1u : 0u);
-            tc::issue_mma(tcx.st.tmem + 256, da, d1, idesc, kb > 0 ? 1u : 0u);
-        }
-    });
+    unsigned char* B0 = A + ah;
+    unsigned char* B1 = B0 + bh;
+    const unsigned char* gx = reinterpret_cast<const unsigned char*>(c.s + (X == OP_Q ? L.OXQ : L.OXK));
+    const unsigned char* g0 = reinterpret_cast<const unsigned char*>(c.s + (Z0 == OP_A ? L.OZA : L.OZK));
+    const unsigned char* g1 = reinterpret_cast<const unsigned char*>(c.s + (Z1 == OP_A ? L.OZA : L.OZK));
+#pragma unroll 1
+    for (int hf = 0; hf < 2; ++hf) {
+        const Bulk b[3] = {{A, gx + hf * ah, ah}, {B0, g0 + hf * bh, bh}, {B1, g1 + hf * bh, bh}};
+        bulk_load(tcx.st, b);
+        fast_mma(tcx.st, [&]() {
+            const uint32_t idesc = tc::idesc_tf32(128, C);
+            for (int kb = 0; kb < KH; ++kb) {
+                const uint64_t da = tc::make_desc(tc::smem_addr(A + kb * 4096), 128, 256);
+                const uint64_t d0 = tc::make_desc(tc::smem_addr(B0 + kb * C * 32), 128, 256);
+                const uint64_t d1 = tc::make_desc(tc::smem_addr(B1 + kb * C * 32), 128, 256);
+                const uint32_t acc = (hf > 0 || kb > 0) ? 1u : 0u;
+                tc::issue_mma(tcx.st.tmem, da, d0, idesc, acc);
+                tc::issue_mma(tcx.st.tmem + 128, da, d1, idesc, acc);
+            }
+        });
+    }
     const int q = warp & 3, pr = warp >> 2;
     const int t = 32 * q + lane;
     const size_t out = pr ? out1 : out0;
     const bool incl = pr ? incl1 : incl0;
-    const uint32_t lane_base = tcx.st.tmem + ((uint32_t)(32 * q) << 16) + 256 * pr;
+    const uint32_t lane_base = tcx.st.tmem + ((uint32_t)(32 * q) << 16) + 128 * pr;
     for (int J = 0; J < nb8; ++J) {
         float v[8];
         tmem_ld8(lane_base + 8 * J, v);

@@ -27,9 +27,12 @@ constexpr int kPanelA = 32 * 4096;      // A operand: up to 32 K blocks of 128 r
 constexpr int kPanelB = 30 * 1024;      // B operand
 constexpr int kPanelBt = 16 * 128 * 4;  // block totals Bt of the chunk
 constexpr int kPanelF = 16 * 128 * 4;   // F factors of one panel step
-constexpr uint32_t kDiagCol = 256;      // TMEM column of the in-block (diagonal) products
+constexpr uint32_t kDiagCol = 256;      // TMEM column of the in-block gradient products
+constexpr int kPairA = 16 * 4096;       // A region of the masked-pair panels (64 KB)
 
+// Shared memory of the gradient panels (k_bwd) and of the masked-pair panels.
 __host__ __device__ constexpr int panel_smem_bytes() { return kPanelA + kPanelB + kPanelBt + kPanelF; }
+__host__ __device__ constexpr int pair_smem_bytes() { return kPairA + 16 * 512 + kPanelBt + kPanelF; }
 
 // Shared-memory stores and loads by address; the stores carry no compiler
 // memory barrier, so global loads around them can be scheduled freely.
@@ -104,14 +107,16 @@ struct PanelSmem {
     float* f;   // [nb8][D]
 };
 
-// Carve the panel buffers and copy the chunk's block totals Bt (all threads).
+// Carve the panel buffers (A region of abytes, B region of bbytes) and copy
+// the chunk's block totals Bt (all threads).
 template <int D>
-__device__ __forceinline__ PanelSmem panel_smem(const float* s, const Lay& L, unsigned char* sbuf) {
+__device__ __forceinline__ PanelSmem panel_smem(const float* s, const Lay& L, unsigned char* sbuf,
+                                                int abytes = kPanelA, int bbytes = kPanelB) {
     PanelSmem m;
     m.A = sbuf;
-    m.B = sbuf + kPanelA;
-    m.bt = reinterpret_cast<float*>(sbuf + kPanelA + kPanelB);
-    m.f = reinterpret_cast<float*>(sbuf + kPanelA + kPanelB + kPanelBt);
+    m.B = sbuf + abytes;
+    m.bt = reinterpret_cast<float*>(sbuf + abytes + bbytes);
+    m.f = reinterpret_cast<float*>(sbuf + abytes + bbytes + kPanelBt);
     for (int i = threadIdx.x; i < L.nb8 * D / 4; i += kThreads)
         reinterpret_cast<float4*>(m.bt)[i] = *reinterpret_cast<const float4*>(s + L.BT + 4 * (size_t)i);
     __syncthreads();
@@ -259,94 +264,148 @@ __device__ void form_mid_mn(const Chunk<Tin, D>& c, unsigned char* dst, int kb0)
     }
 }
 
+// Channel half hf (K blocks [hf D/16, (hf+1) D/16)) of form_mid_k, stored from
+// K block 0 of dst.
+template <int OP, bool XSIDE, typename Tin, int D>
+__device__ void form_mid_k_half(const Chunk<Tin, D>& c, unsigned char* dst, int kstride, int hf) {
+    constexpr int QH = D / 8;   // channel quads per half
+    const Lay& L = c.L;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int r8 = lane & 7;
+    const int slot = warp * 4 + (lane >> 3);  // 0 .. 31
+    const int q4 = slot % QH, par = slot / QH, NPAR = 32 / QH;
+    const int j = 4 * (hf * QH + q4);
+    const uint32_t base = tc::smem_addr(dst) + (q4 >> 1) * kstride;
+#pragma unroll 4
+    for (int b = par; b < L.nb8; b += NPAR) {
+        const int t = 8 * b + r8;
+        float x[4], lc[4], lm[4];
+        opload4<OP>(c, t, j, x);
+        ld4(c.s + L.LC + (size_t)t * D + j, lc);
+        ld4(c.s + L.LC + (size_t)(8 * b + 3) * D + j, lm);
+        float4 o;
+        o.x = tc::tf32_rn(x[0] * fexp<Tin>(XSIDE ? lc[0] - lm[0] : lm[0] - lc[0]));
+        o.y = tc::tf32_rn(x[1] * fexp<Tin>(XSIDE ? lc[1] - lm[1] : lm[1] - lc[1]));
+        o.z = tc::tf32_rn(x[2] * fexp<Tin>(XSIDE ? lc[2] - lm[2] : lm[2] - lc[2]));
+        o.w = tc::tf32_rn(x[3] * fexp<Tin>(XSIDE ? lc[3] - lm[3] : lm[3] - lc[3]));
+        sts128(base + tc::kblk_off(t, 4 * (q4 & 1)), o);
+    }
+}
+
 // ------------------------------------------------------------------ masked products
 
 // out_p[t][s] = [X (*) Z_p]_{ts} masked to s < t (strict) or s <= t, p = 0, 1.
-//  - in-block pairs: Xo Zo_p^T with the mid-block pivots (full C x C product,
-//    only same-block entries are read), TMEM columns kDiagCol + 128 p + s;
 //  - earlier blocks: one chain per block J of s, B = [Zz_0 ; Zz_1] rows of J
 //    (N = 16), A = Xx F[.][J] over the later tokens (K-major, K = channels),
-//    TMEM column 16 J + 8 p + (s - 8 J); lane = t.
+//    TMEM column 16 J + 8 p + (s - 8 J); lane = t;
+//  - then the in-block pairs: Xo Zo_p^T with the mid-block pivots (full C x C
+//    product in two channel halves, only same-block entries are read), TMEM
+//    columns 128 p + s.  At most 256 TMEM columns and 96 KB of shared memory.
 template <typename Tin, int D, int X, int Z0, int Z1>
 __device__ void panel_masked_pair(const Chunk<Tin, D>& c, TcCta& tcx, size_t out0, size_t out1,
                                   bool incl0, bool incl1) {
     const Lay& L = c.L;
     const int C = L.C, nb8 = L.nb8;
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const PanelSmem m = panel_smem<D>(c.s, L, tcx.sbuf);
-    // in-block products
+    const PanelSmem m = panel_smem<D>(c.s, L, tcx.sbuf, kPairA, 16 * 512);
+    const int q = warp & 3, pr = warp >> 2;
+    const int t = 32 * q + lane;
+    const size_t out = pr ? out1 : out0;
+    const bool incl = pr ? incl1 : incl0;
+    const uint32_t lane_base = tcx.st.tmem + ((uint32_t)(32 * q) << 16);
+    // earlier blocks
     {
-        unsigned char* Bd = m.A + 64 * 1024;
-        form_mid_k<X, true>(c, m.A, 4096);
-#pragma unroll 1
-        for (int pr = 0; pr < 2; ++pr) {
-            if (pr == 0) form_mid_k<Z0, false>(c, Bd, C * 32);
-            else form_mid_k<Z1, false>(c, Bd, C * 32);
+        const size_t xx = panel_xx(L, X), zz0 = panel_zz(L, Z0), zz1 = panel_zz(L, Z1);
+        constexpr int NQ = D / 4, NPAR = kThreads / (8 * NQ);
+        const KRole<D> ro;
+        const uint32_t idesc = tc::idesc_tf32(128, 16);
+        const uint32_t aq = tc::smem_addr(m.A) + (ro.q4 >> 1) * 4096;
+        const uint32_t fq = tc::smem_addr(m.f) + 16 * ro.q4;
+        for (int J = 0; J + 1 < nb8; ++J) {
+            // B: rows n < 8 from Zz_0, n >= 8 from Zz_1 (tokens 8J + n % 8), already TF32
+            for (int idx = tid; idx < 16 * NQ; idx += kThreads) {
+                const int n = idx & 15, qq = idx >> 4;
+                const float* src = c.s + (n < 8 ? zz0 : zz1) + (size_t)(8 * J + (n & 7)) * D + 4 * qq;
+                tc::cp_async16(tc::smem_addr(m.B + (qq >> 1) * 512 + tc::kblk_off(n, 4 * (qq & 1))), src, true);
+            }
+            // A: raw Xx rows t >= 8(J + 1), each thread its own chunks
+            for (int I = J + 1 + ro.par; I < nb8; I += NPAR) {
+                const int tt = 8 * I + ro.r8;
+                tc::cp_async16(aq + tc::kblk_off(tt, 4 * (ro.q4 & 1)), c.s + xx + (size_t)tt * D + 4 * ro.q4, true);
+            }
+            panel_ftab<Tin, D, false>(m, nb8, J);
+            asm volatile("cp.async.wait_all;" ::: "memory");
+            __syncthreads();
+            for (int I = J + 1 + ro.par; I < nb8; I += NPAR)
+                scale_at(aq + tc::kblk_off(8 * I + ro.r8, 4 * (ro.q4 & 1)), fq + I * D * 4);
             panel_run(tcx.st, [&]() {
-                const uint32_t idesc = tc::idesc_tf32(128, C);
                 for (int kb = 0; kb < D / 8; ++kb) {
                     const uint64_t da = tc::make_desc(tc::smem_addr(m.A + kb * 4096), 128, 256);
-                    const uint64_t db = tc::make_desc(tc::smem_addr(Bd + kb * C * 32), 128, 256);
-                    tc::issue_mma(tcx.st.tmem + kDiagCol + 128 * pr, da, db, idesc, kb > 0 ? 1u : 0u);
+                    const uint64_t db = tc::make_desc(tc::smem_addr(m.B + kb * 512), 128, 256);
+                    tc::issue_mma(tcx.st.tmem + 16 * J, da, db, idesc, kb > 0 ? 1u : 0u);
                 }
             });
         }
-    }
-    // earlier blocks
-    const size_t xx = panel_xx(L, X), zz0 = panel_zz(L, Z0), zz1 = panel_zz(L, Z1);
-    constexpr int NQ = D / 4, NPAR = kThreads / (8 * NQ);
-    const KRole<D> ro;
-    const uint32_t idesc = tc::idesc_tf32(128, 16);
-    const uint32_t aq = tc::smem_addr(m.A) + (ro.q4 >> 1) * 4096;
-    const uint32_t fq = tc::smem_addr(m.f) + 16 * ro.q4;
-    for (int J = 0; J + 1 < nb8; ++J) {
-        // B: rows n < 8 from Zz_0, n >= 8 from Zz_1 (tokens 8J + n % 8), already TF32
-        for (int idx = tid; idx < 16 * NQ; idx += kThreads) {
-            const int n = idx & 15, qq = idx >> 4;
-            const float* src = c.s + (n < 8 ? zz0 : zz1) + (size_t)(8 * J + (n & 7)) * D + 4 * qq;
-            tc::cp_async16(tc::smem_addr(m.B + (qq >> 1) * 512 + tc::kblk_off(n, 4 * (qq & 1))), src, true);
-        }
-        // A: raw Xx rows t >= 8(J + 1), each thread its own chunks
-        for (int I = J + 1 + ro.par; I < nb8; I += NPAR) {
-            const int t = 8 * I + ro.r8;
-            tc::cp_async16(aq + tc::kblk_off(t, 4 * (ro.q4 & 1)), c.s + xx + (size_t)t * D + 4 * ro.q4, true);
-        }
-        panel_ftab<Tin, D, false>(m, nb8, J);
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        __syncthreads();
-        for (int I = J + 1 + ro.par; I < nb8; I += NPAR)
-            scale_at(aq + tc::kblk_off(8 * I + ro.r8, 4 * (ro.q4 & 1)), fq + I * D * 4);
-        panel_run(tcx.st, [&]() {
-            for (int kb = 0; kb < D / 8; ++kb) {
-                const uint64_t da = tc::make_desc(tc::smem_addr(m.A + kb * 4096), 128, 256);
-                const uint64_t db = tc::make_desc(tc::smem_addr(m.B + kb * 512), 128, 256);
-                tc::issue_mma(tcx.st.tmem + 16 * J, da, db, idesc, kb > 0 ? 1u : 0u);
-            }
-        });
-    }
-    // epilogue: lane t; earlier blocks, its own block (masked), zeros after it
-    {
-        const int q = warp & 3, pr = warp >> 2;
-        const int t = 32 * q + lane;
-        const size_t out = pr ? out1 : out0;
-        const bool incl = pr ? incl1 : incl0;
-        const uint32_t lane_base = tcx.st.tmem + ((uint32_t)(32 * q) << 16);
+        // blocks before t's block from TMEM, zeros after it (t's own block later)
         for (int J = 0; J < nb8; ++J) {
-            float v[8], dg[8];
+            float v[8];
             if (J + 1 < nb8) tmem_ld8(lane_base + (uint32_t)(16 * J + 8 * pr), v);
-            tmem_ld8(lane_base + kDiagCol + 128 * pr + 8 * J, dg);
             if (t < C) {
                 const int I = t >> 3;
                 float* d = c.s + out + (size_t)t * C + 8 * J;
-                float w[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int s = 8 * J + u;
-                    w[u] = J < I ? v[u] : (J == I && (incl ? s <= t : s < t) ? dg[u] : 0.f);
+                if (J < I) {
+                    *reinterpret_cast<float4*>(d) = make_float4(v[0], v[1], v[2], v[3]);
+                    *reinterpret_cast<float4*>(d + 4) = make_float4(v[4], v[5], v[6], v[7]);
+                } else if (J > I) {
+                    *reinterpret_cast<float4*>(d) = make_float4(0.f, 0.f, 0.f, 0.f);
+                    *reinterpret_cast<float4*>(d + 4) = make_float4(0.f, 0.f, 0.f, 0.f);
                 }
-                *reinterpret_cast<float4*>(d) = make_float4(w[0], w[1], w[2], w[3]);
-                *reinterpret_cast<float4*>(d + 4) = make_float4(w[4], w[5], w[6], w[7]);
             }
+        }
+        panel_end();
+    }
+    // in-block pairs, in two channel halves (A = Xo, B = Zo_p, 32 KB each)
+    {
+        unsigned char* Bd = m.A + 32 * 1024;
+        constexpr int KH = D / 16;  // K blocks per half
+#pragma unroll 1
+        for (int pr2 = 0; pr2 < 2; ++pr2) {
+#pragma unroll 1
+            for (int hf = 0; hf < 2; ++hf) {
+                form_mid_k_half<X, true>(c, m.A, 4096, hf);
+                if (pr2 == 0) form_mid_k_half<Z0, false>(c, Bd, C * 32, hf);
+                else form_mid_k_half<Z1, false>(c, Bd, C * 32, hf);
+                panel_run(tcx.st, [&]() {
+                    const uint32_t idesc = tc::idesc_tf32(128, C);
+                    for (int kb = 0; kb < KH; ++kb) {
+                        const uint64_t da = tc::make_desc(tc::smem_addr(m.A + kb * 4096), 128, 256);
+                        const uint64_t db = tc::make_desc(tc::smem_addr(Bd + kb * C * 32), 128, 256);
+                        tc::issue_mma(tcx.st.tmem + 128 * pr2, da, db, idesc, (hf > 0 || kb > 0) ? 1u : 0u);
+                    }
+                });
+            }
+        }
+        // t's own block (masked); the warp's 32 lanes span blocks 4q .. 4q + 3
+        float v[8];
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            float x[8];
+            tmem_ld8(lane_base + (uint32_t)(128 * pr + 8 * (4 * q + i)), x);
+            if ((lane >> 3) == i)
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = x[u];
+        }
+        if (t < C) {
+            const int I = t >> 3;
+            float w[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int s = 8 * I + u;
+                w[u] = (incl ? s <= t : s < t) ? v[u] : 0.f;
+            }
+            float* d = c.s + out + (size_t)t * C + 8 * I;
+            *reinterpret_cast<float4*>(d) = make_float4(w[0], w[1], w[2], w[3]);
+            *reinterpret_cast<float4*>(d + 4) = make_float4(w[4], w[5], w[6], w[7]);
         }
     }
     panel_end();
