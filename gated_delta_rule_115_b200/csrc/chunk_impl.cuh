@@ -314,9 +314,7 @@ __device__ __forceinline__ void masked_pair(const Chunk<Tin, D>& c, TcCta& tcx, 
 template <typename Tin, int D, int PASSES, bool XSIDE, int op0, int op1, class EPI>
 __device__ __forceinline__ void decayed_grad(const Chunk<Tin, D>& c, TcCta& tcx, float* sm,
                                              size_t G0, size_t G1, const EPI& epi) {
-    if (c.tame) {
-        fast_grad<Tin, D, XSIDE, op0, op1>(c, tcx, G0, G1, epi);
-    } else if (use_panels<Tin, D, PASSES>(c)) {
+    if (use_panels<Tin, D, PASSES>(c)) {
         if constexpr (XSIDE) panel_grad_x<Tin, D, op0, op1>(c, tcx, G0, G1, epi);
         else panel_grad_z<Tin, D, op0, op1>(c, tcx, G0, G1, epi);
     } else {
@@ -758,10 +756,13 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                         const int ss = s0 + u;
                         w[u] = (incl ? ss <= t : ss < t) ? sg * x[u] : 0.f;
                     }
-                    float* d = s + out + (size_t)t * C + s0;
-                    *reinterpret_cast<float4*>(d) = make_float4(w[0], w[1], w[2], w[3]);
-                    *reinterpret_cast<float4*>(d + 4) = make_float4(w[4], w[5], w[6], w[7]);
-                    if (c.tame) store_g_layouts(s, L, which, t, s0, w);
+                    if (c.tame) {
+                        store_g_layouts(s, L, which, t, s0, w);
+                    } else {
+                        float* d = s + out + (size_t)t * C + s0;
+                        *reinterpret_cast<float4*>(d) = make_float4(w[0], w[1], w[2], w[3]);
+                        *reinterpret_cast<float4*>(d + 4) = make_float4(w[4], w[5], w[6], w[7]);
+                    }
                 };
                 tc_rows2<PASSES, 128, false, false>(tcx, C, D,
                     [&](int) {
@@ -817,17 +818,64 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         using OK_ = std::integral_constant<int, OP_K>;
         using OQ_ = std::integral_constant<int, OP_Q>;
         using OA_ = std::integral_constant<int, OP_A>;
-        decayed_grad<Tin, D, PASSES, true, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, accum(dK, OK_{}, 1.f));
-        decayed_grad<Tin, D, PASSES, true, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, accum(dQh, OQ_{}, 1.f));
-        __syncthreads();
-        // Z side: dA += dL_A^T (*) K + dM_QA^T (*) Qh ; dK += dL_K^T (*) K + dM_QK^T (*) Qh ; dGam -= Z * dZ
-        decayed_grad<Tin, D, PASSES, false, OP_K, OP_Q>(c, tcx, sm, L.LA, L.MQA, accum(dA, OA_{}, -1.f));
-        __syncthreads();
-        decayed_grad<Tin, D, PASSES, false, OP_K, OP_Q>(c, tcx, sm, L.LK, L.MQK, accum(dK, OK_{}, -1.f));
-        __syncthreads();
-        // dgbar_j = e^gbar_j sum_c S[j][c] dS'[j][c] + sum_t (dKb Kb + dAb Ab)[t][j]
         Tin* gq = (Tin*)p.dq; Tin* gk = (Tin*)p.dk; Tin* gv = (Tin*)p.dv; Tin* gg = (Tin*)p.dg;
         Tin* ge = (Tin*)p.de; Tin* gw = (Tin*)p.dw; Tin* ggm = (Tin*)p.dgamma;
+        if (c.tame) {
+            // single-pivot products: the four gradient pairs accumulate in TMEM
+            // (X side: dK, dQh; Z side: dA, dK), then one pass finishes every
+            // token's gradients: dK, dQh, dA, dGam and the input gradients but dg
+            fast_grad_mma<Tin, D, true, OP_A, OP_K>(c, tcx, L.LA, L.LK, 0);
+            fast_grad_mma<Tin, D, true, OP_K, OP_A>(c, tcx, L.MQK, L.MQA, 128);
+            fast_grad_mma<Tin, D, false, OP_K, OP_Q>(c, tcx, L.LA, L.MQA, 256);
+            fast_grad_mma<Tin, D, false, OP_K, OP_Q>(c, tcx, L.LK, L.MQK, 384);
+            const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+            const int q = warp & 3, half = warp >> 2, cc = 32 * q + lane;
+            const uint32_t lane_base = tcx.st.tmem + ((uint32_t)(32 * q) << 16);
+            if (32 * q < D) {
+                const float hp = 0.5f * s[L.GBAR + cc];
+                for (int I = half; I < L.nb8; I += 2) {
+                    const int t0 = 8 * I;
+                    float x1[8], x2[8], z1[8], z2[8];
+                    tmem_ld8(lane_base + 8 * I, x1);
+                    tmem_ld8(lane_base + 128 + 8 * I, x2);
+                    tmem_ld8(lane_base + 256 + 8 * I, z1);
+                    tmem_ld8(lane_base + 384 + 8 * I, z2);
+                    const float pre = s[L.PRE + (size_t)I * D + cc];
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int t = t0 + u;
+                        const size_t x = (size_t)t * D + cc, gi = c.base + (size_t)t * c.rs + cc;
+                        const float lc = s[L.LC + x];
+                        const float kv = ldf(c.k + gi), qv = ldf(c.q + gi), gmv = ldf(c.gm + gi);
+                        const float ev = ldf(c.e + gi), vv = ldf(c.v + gi), wv = ldf(c.w + gi);
+                        const float dk0 = s[dK + x], dq0 = s[dQh + x], da0 = s[dA + x];
+                        const float dg0 = s[dGam + x], du0 = s[dU + x];
+                        const float d = pre + lc - hp;
+                        const float fx = fexp<Tin>(d), fz = fexp<Tin>(-d);
+                        const float vx1 = fx * x1[u], vx2 = fx * x2[u], vz1 = fz * z1[u], vz2 = fz * z2[u];
+                        const float DK = dk0 + vx1 + vz2, DQ = dq0 + vx2, DA = da0 + vz1;
+                        s[dGam + x] = dg0 + kv * (vx1 - vz2) + qv * gmv * vx2 - ev * kv * vz1;
+                        stf(gq + gi, DQ * gmv);
+                        stf(ggm + gi, DQ * qv);
+                        stf(ge + gi, DA * kv);
+                        stf(gk + gi, DK + DA * ev);
+                        stf(gw + gi, du0 * vv);
+                        stf(gv + gi, du0 * wv);
+                    }
+                }
+            }
+            panel_end();
+        } else {
+            decayed_grad<Tin, D, PASSES, true, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, accum(dK, OK_{}, 1.f));
+            decayed_grad<Tin, D, PASSES, true, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, accum(dQh, OQ_{}, 1.f));
+            __syncthreads();
+            // Z side: dA += dL_A^T (*) K + dM_QA^T (*) Qh ; dK += dL_K^T (*) K + dM_QK^T (*) Qh ; dGam -= Z * dZ
+            decayed_grad<Tin, D, PASSES, false, OP_K, OP_Q>(c, tcx, sm, L.LA, L.MQA, accum(dA, OA_{}, -1.f));
+            __syncthreads();
+            decayed_grad<Tin, D, PASSES, false, OP_K, OP_Q>(c, tcx, sm, L.LK, L.MQK, accum(dK, OK_{}, -1.f));
+            __syncthreads();
+        }
+        // dgbar_j = e^gbar_j sum_c S[j][c] dS'[j][c] + sum_t (dKb Kb + dAb Ab)[t][j]
         {
             const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
             for (int j = warp; j < D; j += kThreads / 32) {
@@ -872,7 +920,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                 }
             }
         }
-        for (int idx = threadIdx.x; idx < C * D / 4; idx += kThreads) {
+        for (int idx = threadIdx.x; !c.tame && idx < C * D / 4; idx += kThreads) {
             const int t = idx / (D / 4), j = 4 * (idx % (D / 4));
             const size_t gi = c.base + t * c.rs + j;
             const size_t li = (size_t)t * D + j;

@@ -196,17 +196,18 @@ __device__ __forceinline__ int gidx(const Lay& L, size_t G) {
     return G == L.LA ? 0 : G == L.LK ? 1 : G == L.MQK ? 2 : 3;
 }
 
-// X side:  out[t][c] = sum_s (G0[t][s] Z0_sc + G1[t][s] Z1_sc) exp(Gam_tc - Gam_sc)
-//   = exp(Gam_tc - P_c) sum_s (G0[t][s] Zo0[s][c] + G1[t][s] Zo1[s][c]):
-// A = Zo_p (MN-major), B = G_p (K-major rows t), TMEM lane c, column t.
-// Z side:  out[s][c] = exp(P_c - Gam_sc) sum_t (G0[t][s] Xo0[t][c] + G1[t][s] Xo1[t][c]):
-// A = Xo_p (MN-major), B[s][t] = G_p[t][s] (MN-major), TMEM lane c, column s.
-// Then epi(8, t0, c, v[8]) for 8 consecutive tokens.
-template <typename Tin, int D, bool XSIDE, int O0, int O1, class EPI>
-__device__ void fast_grad(const Chunk<Tin, D>& c, TcCta& tcx, size_t G0, size_t G1, const EPI& epi) {
+// Raw accumulators of the gradients through the masked products, into TMEM
+// columns col .. col + C (lane = channel):
+// X side:  acc[c][t] = sum_s (G0[t][s] Zo0[s][c] + G1[t][s] Zo1[s][c]), so that
+//   sum_s (G0[t][s] Z0_sc + G1[t][s] Z1_sc) exp(Gam_tc - Gam_sc) = exp(Gam_tc - P_c) acc[c][t];
+//   A = Zo_p (MN-major), B = G_p (K-major rows t);
+// Z side:  acc[c][s] = sum_t (G0[t][s] Xo0[t][c] + G1[t][s] Xo1[t][c]), so that
+//   sum_t (G0[t][s] X0_tc + G1[t][s] X1_tc) exp(Gam_tc - Gam_sc) = exp(P_c - Gam_sc) acc[c][s];
+//   A = Xo_p (MN-major), B[s][t] = G_p[t][s] (MN-major).
+template <typename Tin, int D, bool XSIDE, int O0, int O1>
+__device__ void fast_grad_mma(const Chunk<Tin, D>& c, TcCta& tcx, size_t G0, size_t G1, uint32_t col) {
     const Lay& L = c.L;
-    const int C = L.C, nb8 = L.nb8;
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int C = L.C;
     unsigned char* A = tcx.sbuf;
     unsigned char* B = A + 65536;
     const uint32_t idesc = tc::idesc_tf32(128, C) | (1u << 15) | (XSIDE ? 0u : (1u << 16));
@@ -223,31 +224,10 @@ __device__ void fast_grad(const Chunk<Tin, D>& c, TcCta& tcx, size_t G0, size_t 
                 const uint64_t da = tc::make_desc_mn32(tc::smem_addr(A + kb * 4096), 2048);
                 const uint64_t db = XSIDE ? tc::make_desc(tc::smem_addr(B + kb * C * 32), 128, 256)
                                           : tc::make_desc_mn32(tc::smem_addr(B + kb * C * 32), C / 32 * 512);
-                tc::issue_mma(tcx.st.tmem, da, db, idesc, (p > 0 || kb > 0) ? 1u : 0u);
+                tc::issue_mma(tcx.st.tmem + col, da, db, idesc, (p > 0 || kb > 0) ? 1u : 0u);
             }
         });
     }
-    const int q = warp & 3, half = warp >> 2;
-    const int cc = 32 * q + lane;
-    const uint32_t lane_base = tcx.st.tmem + ((uint32_t)(32 * q) << 16);
-    if (32 * q < D) {
-        const float hp = 0.5f * c.s[L.GBAR + cc];
-        for (int I = half; I < nb8; I += 2) {
-            const int t0 = 8 * I;
-            float lc[8], v[8];
-            const float pre = c.s[L.PRE + (size_t)I * D + cc];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) lc[u] = c.s[L.LC + (size_t)(t0 + u) * D + cc];
-            tmem_ld8(lane_base + 8 * I, v);
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const float d = pre + lc[u] - hp;
-                v[u] *= fexp<Tin>(XSIDE ? d : -d);
-            }
-            epi(std::integral_constant<int, 8>{}, t0, cc, v);
-        }
-    }
-    panel_end();
 }
 
 // Rows t of the masked-product gradient G_i in the two tensor-core layouts the
