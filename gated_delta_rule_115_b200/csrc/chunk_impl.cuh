@@ -394,6 +394,13 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_intra(KParams p)
 // Sequential pass over chunks for one (b, h) and a slab of SLAB columns.
 // Forward (REV = false): S_{n+1} = M_n S_n + Bn_n, records S_n.
 // Reverse (REV = true):  G_n = M_n^T G_{n+1} + Bn_n, records G_{n+1}.
+// M_{n+1} and the slab of Bn_{n+1} are copied into shared memory (cp.async,
+// rows padded to D + 4 floats) while step n computes from M_n.
+template <int D, int SLAB>
+__host__ __device__ constexpr int chain_smem_bytes() {
+    return (2 * D * (D + 4) + 2 * D * SLAB) * 4;
+}
+
 template <int D, int SLAB, int PASSES, bool REV>
 __global__ void __launch_bounds__(kThreads) k_chain(const float* __restrict__ M,
                                                     const float* __restrict__ Bn,
@@ -401,36 +408,59 @@ __global__ void __launch_bounds__(kThreads) k_chain(const float* __restrict__ M,
                                                     float* __restrict__ S_rec,
                                                     float* __restrict__ S_out, int N) {
     constexpr int NT = SLAB / 8 < 4 ? SLAB / 8 : 4;
+    constexpr int MP = D + 4;  // padded row of M in shared memory
     __shared__ float buf[2][D * SLAB];
+    extern __shared__ __align__(16) float csm[];
+    float* mbuf = csm;                    // [2][D][MP]
+    float* bbuf = csm + 2 * D * MP;       // [2][D][SLAB]
     constexpr int NSLAB = D / SLAB;
     const int bh = blockIdx.x / NSLAB, c0 = (blockIdx.x % NSLAB) * SLAB;
     const size_t DD = (size_t)D * D;
+    auto prefetch = [&](int step, int slot) {
+        const int n = REV ? N - 1 - step : step;
+        const size_t off = ((size_t)bh * N + n) * DD;
+        float* md = mbuf + slot * D * MP;
+        for (int idx = threadIdx.x; idx < D * D / 4; idx += kThreads) {
+            const int r = idx / (D / 4), j = 4 * (idx % (D / 4));
+            tc::cp_async16(tc::smem_addr(md + r * MP + j), M + off + (size_t)r * D + j, true);
+        }
+        float* bd = bbuf + slot * D * SLAB;
+        for (int idx = threadIdx.x; idx < D * SLAB / 4; idx += kThreads) {
+            const int r = idx / (SLAB / 4), j = 4 * (idx % (SLAB / 4));
+            tc::cp_async16(tc::smem_addr(bd + r * SLAB + j), Bn + off + (size_t)r * D + c0 + j, true);
+        }
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+    prefetch(0, 0);
     for (int idx = threadIdx.x; idx < D * SLAB; idx += kThreads) {
         const int i = idx / SLAB, cc = idx % SLAB;
         buf[0][idx] = S_in ? S_in[bh * DD + (size_t)i * D + c0 + cc] : 0.f;
     }
-    __syncthreads();
     int cur = 0;
     for (int step = 0; step < N; ++step) {
         const int n = REV ? N - 1 - step : step;
         const size_t off = ((size_t)bh * N + n) * DD;
+        if (step + 1 < N) {
+            prefetch(step + 1, (step + 1) & 1);
+            asm volatile("cp.async.wait_group 1;" ::: "memory");
+        } else {
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+        }
+        __syncthreads();
         if (S_rec)
             for (int idx = threadIdx.x; idx < D * SLAB; idx += kThreads)
                 S_rec[off + (size_t)(idx / SLAB) * D + c0 + idx % SLAB] = buf[cur][idx];
-        const float* Mn = M + off;
-        const float* Bb = Bn + off;
+        const float* Mn = mbuf + (step & 1) * D * MP;
+        const float* Bb = bbuf + (step & 1) * D * SLAB;
         const float* Sc = buf[cur];
         float* Sn = buf[cur ^ 1];
         cta_tiles<NT>(D, SLAB,
             [&](float (&acc)[1][NT][4], int m0, int n0) {
                 warp_gemm<PASSES, 1, NT>(acc, D,
-                    [&](int r, int k) {
-                        return REV ? __ldg(Mn + (size_t)k * D + m0 + r)
-                                   : __ldg(Mn + (size_t)(m0 + r) * D + k);
-                    },
-                    [&](int k, int n) { return Sc[k * SLAB + n0 + n]; });
+                    [&](int r, int k) { return REV ? Mn[k * MP + m0 + r] : Mn[(m0 + r) * MP + k]; },
+                    [&](int k, int nn) { return Sc[k * SLAB + n0 + nn]; });
             },
-            [&](int i, int cc, float v) { Sn[i * SLAB + cc] = v + __ldg(Bb + (size_t)i * D + c0 + cc); });
+            [&](int i, int cc, float v) { Sn[i * SLAB + cc] = v + Bb[i * SLAB + cc]; });
         __syncthreads();
         cur ^= 1;
     }
@@ -1026,18 +1056,24 @@ int persistent_grid(KERNEL kernel, int nch, int dyn) {
     return g < nsm * occ ? g : nsm * occ;
 }
 
+template <int D, int SL, int PASSES, bool REV>
+cudaError_t launch_chain_slab(int BH, int N, const float* M, const float* Bn, const float* S_in,
+                              float* S_rec, float* S_out, cudaStream_t st) {
+    constexpr int bytes = chain_smem_bytes<D, SL>();
+    cudaError_t e = cudaFuncSetAttribute(k_chain<D, SL, PASSES, REV>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+    if (e != cudaSuccess) return e;
+    MUIR_TIMED(REV ? "k_chain_rev" : "k_chain", st,
+               k_chain<D, SL, PASSES, REV><<<BH * (D / SL), kThreads, bytes, st>>>(M, Bn, S_in, S_rec, S_out, N));
+    return cudaGetLastError();
+}
+
 template <int D, int PASSES, bool REV>
 cudaError_t launch_chain(int BH, int N, const float* M, const float* Bn, const float* S_in,
                                 float* S_rec, float* S_out, cudaStream_t st) {
     // column slabs: enough CTAs to cover the GPU when B*H is small
-    if (BH >= 64) {
-        constexpr int SL = 32;
-        MUIR_TIMED(REV ? "k_chain_rev" : "k_chain", st, k_chain<D, SL, PASSES, REV><<<BH * (D / SL), kThreads, 0, st>>>(M, Bn, S_in, S_rec, S_out, N));
-    } else {
-        constexpr int SL = 16;
-        MUIR_TIMED(REV ? "k_chain_rev" : "k_chain", st, k_chain<D, SL, PASSES, REV><<<BH * (D / SL), kThreads, 0, st>>>(M, Bn, S_in, S_rec, S_out, N));
-    }
-    return cudaGetLastError();
+    if (BH >= 64) return launch_chain_slab<D, 32, PASSES, REV>(BH, N, M, Bn, S_in, S_rec, S_out, st);
+    return launch_chain_slab<D, 16, PASSES, REV>(BH, N, M, Bn, S_in, S_rec, S_out, st);
 }
 
 template <typename Tin, int D, int PASSES, int CF>
