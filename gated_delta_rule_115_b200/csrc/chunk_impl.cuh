@@ -68,7 +68,8 @@ constexpr int kMaxSlots = 296;  // scratch slots: at most 2 resident CTAs per SM
 struct Lay {
     int C, D, nb8, nb16;
     size_t LC, RC, BT, PRE, SUF, GBAR, LA, LK, MQK, MQA, TII, W[8], PXK, PXQ, PZA, PZK;
-    size_t OXK, OXQ, OZA, OZK, MXK, MXQ, MZA, MZK, GK[4], GM[4], total;
+    size_t OXK, OXQ, OZA, OZK, MXK, MXQ, MZA, MZK, GK[4], GM[4];
+    size_t RKT, RQT, RUU, RDO, RAB, RKB, total;  // input-derived operand rows (TF32)
 };
 
 __host__ __device__ inline Lay make_lay(int C, int D) {
@@ -87,6 +88,8 @@ __host__ __device__ inline Lay make_lay(int C, int D) {
     MUIR_TAKE(OXK, pd) MUIR_TAKE(OXQ, pd) MUIR_TAKE(OZA, cd) MUIR_TAKE(OZK, cd)
     MUIR_TAKE(MXK, pc) MUIR_TAKE(MXQ, pc) MUIR_TAKE(MZA, pc) MUIR_TAKE(MZK, pc)
     for (int i = 0; i < 4; ++i) { MUIR_TAKE(GK[i], cc) MUIR_TAKE(GM[i], cc) }
+    MUIR_TAKE(RKT, cd) MUIR_TAKE(RQT, cd) MUIR_TAKE(RUU, cd) MUIR_TAKE(RDO, cd) MUIR_TAKE(RAB, cd)
+    MUIR_TAKE(RKB, cd)
 #undef MUIR_TAKE
     L.total = o;
     return L;
@@ -298,6 +301,55 @@ __device__ __forceinline__ void masked_prep(Chunk<Tin, D>& c, bool with_q, bool 
     else panel_prep<Tin, D>(c, with_q);
 }
 
+// Input-derived operands of the dense products, once per chunk, as TF32-rounded
+// float32 rows [C][d] in scratch, so that the products copy them (cp.async)
+// instead of producing them element by element inside their K loops:
+//   R_KT  Kt = K e^Gam        R_QT  Qt = gamma q e^Gam     R_UU  U = w v
+//   R_DO  dO                  R_AB  Ab = e k e^{gbar-Gam}  R_KB  Kb = K e^{gbar-Gam}
+enum RowOps { R_KT = 1, R_QT = 2, R_UU = 4, R_DO = 8, R_AB = 16, R_KB = 32 };
+
+template <typename Tin, int D, int PASSES>
+__device__ void rows_prep(const Chunk<Tin, D>& c, int ops) {
+    if constexpr (PASSES != 1) return;
+    const Lay& L = c.L;
+    const int n4 = L.C * D / 4;
+    for (int idx = threadIdx.x; idx < n4; idx += kThreads) {
+        const int t = idx / (D / 4), j = 4 * (idx % (D / 4));
+        const size_t g = c.base + (size_t)t * c.rs + j, x = (size_t)t * D + j;
+        const size_t b = (size_t)(t >> 3) * D + j;
+        float k4[4] = {0.f, 0.f, 0.f, 0.f}, e4[4], q4[4], m4[4], v4[4], w4[4], o4[4];
+        float lc[4], pre[4], rc[4], suf[4];
+        if (ops & (R_KT | R_KB | R_AB)) ld4in(c.k + g, k4);
+        if (ops & R_AB) ld4in(c.e + g, e4);
+        if (ops & R_QT) { ld4in(c.q + g, q4); ld4in(c.gm + g, m4); }
+        if (ops & R_UU) { ld4in(c.v + g, v4); ld4in(c.w + g, w4); }
+        if (ops & R_DO) ld4in(c.dO + g, o4);
+        if (ops & (R_KT | R_QT)) { ld4(c.s + L.LC + x, lc); ld4(c.s + L.PRE + b, pre); }
+        if (ops & (R_KB | R_AB)) { ld4(c.s + L.RC + x, rc); ld4(c.s + L.SUF + b, suf); }
+        float4 kt, qt, uu, dd, ab, kb;
+        float* pkt = &kt.x; float* pqt = &qt.x; float* puu = &uu.x; float* pdd = &dd.x;
+        float* pab = &ab.x; float* pkb = &kb.x;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const float eg = (ops & (R_KT | R_QT)) ? fexp<Tin>(pre[u] + lc[u]) : 0.f;
+            const float egb = (ops & (R_KB | R_AB)) ? fexp<Tin>(rc[u] + suf[u]) : 0.f;
+            pkt[u] = tc::tf32_rn(k4[u] * eg);
+            pqt[u] = (ops & R_QT) ? tc::tf32_rn(q4[u] * m4[u] * eg) : 0.f;
+            puu[u] = (ops & R_UU) ? tc::tf32_rn(v4[u] * w4[u]) : 0.f;
+            pdd[u] = (ops & R_DO) ? tc::tf32_rn(o4[u]) : 0.f;
+            pab[u] = (ops & R_AB) ? tc::tf32_rn(e4[u] * k4[u] * egb) : 0.f;
+            pkb[u] = tc::tf32_rn(k4[u] * egb);
+        }
+        if (ops & R_KT) *reinterpret_cast<float4*>(c.s + L.RKT + x) = kt;
+        if (ops & R_QT) *reinterpret_cast<float4*>(c.s + L.RQT + x) = qt;
+        if (ops & R_UU) *reinterpret_cast<float4*>(c.s + L.RUU + x) = uu;
+        if (ops & R_DO) *reinterpret_cast<float4*>(c.s + L.RDO + x) = dd;
+        if (ops & R_AB) *reinterpret_cast<float4*>(c.s + L.RAB + x) = ab;
+        if (ops & R_KB) *reinterpret_cast<float4*>(c.s + L.RKB + x) = kb;
+    }
+    __syncthreads();
+}
+
 template <typename Tin, int D, int PASSES, int X, int Z0, int Z1>
 __device__ __forceinline__ void masked_pair(const Chunk<Tin, D>& c, TcCta& tcx, float* sm,
                                             size_t out0, size_t out1, bool incl0, bool incl1) {
@@ -345,6 +397,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_intra(KParams p)
         float* s = c.s;
         prologue2(c);
         masked_prep<Tin, D, PASSES>(c, false, false);
+        rows_prep<Tin, D, PASSES>(c, R_KT | R_UU);
         masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
         __syncthreads();
         compute_tii(s, L, L.LA);
@@ -360,7 +413,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_intra(KParams p)
         tc_rows2<PASSES, D, true, true>(tcx, D, C,
             [&](int) { return tc::Src{Psi, D, 0, true, false}; },
             [&](int i, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = Psi[(size_t)(t + u) * D + i]; },
-            [&](int) { return tc::no_src(); },
+            [&](int) { return tc::Src{s + L.RKT, D, 0, true, false}; },
             [&](int j, int t, float* v) {
                 for (int u = 0; u < 4; ++u) v[u] = c.K(t + u, j) * f.eg(t + u, j);
             },
@@ -381,7 +434,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_intra(KParams p)
         tc_rows2<PASSES, D, true, true>(tcx, D, C,
             [&](int) { return tc::Src{Phi, D, 0, true, false}; },
             [&](int i, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = Phi[(size_t)(t + u) * D + i]; },
-            [&](int) { return tc::no_src(); },
+            [&](int) { return tc::Src{s + L.RUU, D, 0, true, false}; },
             [&](int cc, int t, float* v) { for (int u = 0; u < 4; ++u) v[u] = c.U(t + u, cc); },
             tc::RowStore{Bn, D});
     }
@@ -479,7 +532,9 @@ __device__ void compute_Y(TcCta& tcx, const Chunk<Tin, D>& c, const float* S, si
     float* s = c.s;
     const Fac<Tin, D> f = facs(c);
     tc_rows2<PASSES, D, false, true>(tcx, C, D + C,
-        [&](int k) { return k < D ? tc::no_src() : tc::Src{s + L.LK, C, D, false, false}; },
+        [&](int k) {
+            return k < D ? tc::Src{s + L.RKT, D, 0, false, false} : tc::Src{s + L.LK, C, D, false, false};
+        },
         [&](int t, int k, float* v) {
             if (k < D) {
                 ld4in(c.k + c.base + t * c.rs + k, v);
@@ -488,7 +543,7 @@ __device__ void compute_Y(TcCta& tcx, const Chunk<Tin, D>& c, const float* S, si
                 ld4(s + L.LK + (size_t)t * C + (k - D), v);
             }
         },
-        [&](int k) { return k < D ? tc::Src{S, D, 0, true, false} : tc::no_src(); },
+        [&](int k) { return k < D ? tc::Src{S, D, 0, true, false} : tc::Src{s + L.RUU, D, D, true, false}; },
         [&](int cc, int k, float* v) {
             if (k < D) for (int u = 0; u < 4; ++u) v[u] = __ldg(S + (size_t)(k + u) * D + cc);
             else for (int u = 0; u < 4; ++u) v[u] = c.U(k - D + u, cc);
@@ -517,6 +572,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_out(KParams p) {
         float* s = c.s;
         prologue2(c);
         masked_prep<Tin, D, PASSES>(c, true, false);
+        rows_prep<Tin, D, PASSES>(c, R_KT | R_QT | R_UU);
         masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
         masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
         __syncthreads();
@@ -530,7 +586,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_out(KParams p) {
         // O = Qt S + M_QK U - M_QA Y
         tc_rows2<PASSES, D, false, true>(tcx, C, D + 2 * C,
             [&](int k) {
-                return k < D ? tc::no_src()
+                return k < D ? tc::Src{s + L.RQT, D, 0, false, false}
                              : (k < D + C ? tc::Src{s + L.MQK, C, D, false, false}
                                           : tc::Src{s + L.MQA, C, D + C, false, true});
             },
@@ -549,7 +605,8 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_out(KParams p) {
             },
             [&](int k) {
                 return k < D ? tc::Src{S, D, 0, true, false}
-                             : (k < D + C ? tc::no_src() : tc::Src{Y, D, D + C, true, false});
+                             : (k < D + C ? tc::Src{s + L.RUU, D, D, true, false}
+                                          : tc::Src{Y, D, D + C, true, false});
             },
             [&](int cc, int k, float* v) {
                 if (k < D) for (int u = 0; u < 4; ++u) v[u] = __ldg(S + (size_t)(k + u) * D + cc);
@@ -583,6 +640,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_bprep(KParams p)
         float* s = c.s;
         prologue2(c);
         masked_prep<Tin, D, PASSES>(c, true, false);
+        rows_prep<Tin, D, PASSES>(c, R_KT | R_QT | R_DO);
         masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
         masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
         __syncthreads();
@@ -593,7 +651,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_bprep(KParams p)
         tc_rows2<PASSES, D, true, true>(tcx, C, C,
             [&](int) { return tc::Src{s + L.MQA, C, 0, true, false}; },
             [&](int t, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = s[L.MQA + (size_t)(k + u) * C + t]; },
-            [&](int) { return tc::no_src(); },
+            [&](int) { return tc::Src{s + L.RDO, D, 0, true, false}; },
             [&](int cc, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc); },
             tc::RowStore{Xi, D});
         solve_s<D, PASSES, true>(s, sm, L, L.LA, L.W[0]);  // Xi = T^T Z0
@@ -602,12 +660,14 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_bprep(KParams p)
         const Fac<Tin, D> f = facs(c);
         // B' = Qt^T dO - Kt^T Xi
         tc_rows2<PASSES, D, true, true>(tcx, D, 2 * C,
-            [&](int) { return tc::no_src(); },
+            [&](int k) {
+                return k < C ? tc::Src{s + L.RQT, D, 0, true, false} : tc::Src{s + L.RKT, D, C, true, true};
+            },
             [&](int i, int k, float* v) {
                 if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.Qh(k + u, i) * f.eg(k + u, i);
                 else for (int u = 0; u < 4; ++u) v[u] = -c.K(k - C + u, i) * f.eg(k - C + u, i);
             },
-            [&](int k) { return k < C ? tc::no_src() : tc::Src{Xi, D, C, true, false}; },
+            [&](int k) { return k < C ? tc::Src{s + L.RDO, D, 0, true, false} : tc::Src{Xi, D, C, true, false}; },
             [&](int cc, int k, float* v) {
                 if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc);
                 else for (int u = 0; u < 4; ++u) v[u] = Xi[(size_t)(k - C + u) * D + cc];
@@ -646,6 +706,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                      dU = L.W[5], dGam = L.W[6];
         prologue2(c);
         masked_prep<Tin, D, PASSES>(c, true, true);
+        rows_prep<Tin, D, PASSES>(c, R_KT | R_UU | R_DO | R_AB | R_KB);
         masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
         masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
         __syncthreads();
@@ -655,7 +716,9 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         const Fac<Tin, D> f = facs(c);
         // dY = -M_QA^T dO - Ab dS'   (stored in dR, then dR = T^T dY)
         tc_rows2<PASSES, D, true, true>(tcx, C, C + D,
-            [&](int k) { return k < C ? tc::Src{s + L.MQA, C, 0, true, false} : tc::no_src(); },
+            [&](int k) {
+                return k < C ? tc::Src{s + L.MQA, C, 0, true, false} : tc::Src{s + L.RAB, D, C, false, false};
+            },
             [&](int t, int k, float* v) {
                 if (k < C) for (int u = 0; u < 4; ++u) v[u] = s[L.MQA + (size_t)(k + u) * C + t];
                 else {
@@ -665,7 +728,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                     for (int u = 0; u < 4; ++u) v[u] *= k4[u] * f.egb(t, k - C + u);
                 }
             },
-            [&](int k) { return k < C ? tc::no_src() : tc::Src{dS, D, C, true, false}; },
+            [&](int k) { return k < C ? tc::Src{s + L.RDO, D, 0, true, false} : tc::Src{dS, D, C, true, false}; },
             [&](int cc, int k, float* v) {
                 if (k < C) for (int u = 0; u < 4; ++u) v[u] = c.dOv(k + u, cc);
                 else for (int u = 0; u < 4; ++u) v[u] = __ldg(dS + (size_t)(k - C + u) * D + cc);
@@ -680,14 +743,14 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         //   dQt = dO S^T, dKt = dR S^T, dKb = U dS'^T, dAb = -Y dS'^T
         auto srcS = [&](int) { return tc::Src{S, D, 0, false, false}; };
         auto srcdS = [&](int) { return tc::Src{dS, D, 0, false, false}; };
-        tc_rows2<PASSES, D, false, false>(tcx, C, D, [&](int) { return tc::no_src(); },
+        tc_rows2<PASSES, D, false, false>(tcx, C, D, [&](int) { return tc::Src{s + L.RDO, D, 0, false, false}; },
             [&](int t, int k, float* v) { ld4in(c.dO + c.base + t * c.rs + k, v); }, srcS, rowsS,
             tc::RowStore{s + dQh, D});
         tc_rows2<PASSES, D, false, false>(tcx, C, D,
             [&](int) { return tc::Src{s + dR, D, 0, false, false}; },
             [&](int t, int k, float* v) { ld4(s + dR + (size_t)t * D + k, v); }, srcS, rowsS,
             tc::RowStore{s + dK, D});
-        tc_rows2<PASSES, D, false, false>(tcx, C, D, [&](int) { return tc::no_src(); },
+        tc_rows2<PASSES, D, false, false>(tcx, C, D, [&](int) { return tc::Src{s + L.RUU, D, 0, false, false}; },
             [&](int t, int k, float* v) {
                 float w4[4];
                 ld4in(c.v + c.base + t * c.rs + k, v);
@@ -747,7 +810,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         tc_rows2<PASSES, D, true, true>(tcx, C, 2 * C + D,
             [&](int k) {
                 return k < C ? tc::Src{s + L.MQK, C, 0, true, false}
-                             : (k < 2 * C ? tc::Src{s + L.LK, C, C, true, false} : tc::no_src());
+                             : (k < 2 * C ? tc::Src{s + L.LK, C, C, true, false}
+                                          : tc::Src{s + L.RKB, D, 2 * C, false, false});
             },
             [&](int t, int k, float* v) {
                 if (k < C) for (int u = 0; u < 4; ++u) v[u] = s[L.MQK + (size_t)(k + u) * C + t];
@@ -758,7 +822,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                 }
             },
             [&](int k) {
-                return k < C ? tc::no_src()
+                return k < C ? tc::Src{s + L.RDO, D, 0, true, false}
                              : (k < 2 * C ? tc::Src{s + dR, D, C, true, false}
                                           : tc::Src{dS, D, 2 * C, true, false});
             },
@@ -796,7 +860,8 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                 };
                 tc_rows2<PASSES, 128, false, false>(tcx, C, D,
                     [&](int) {
-                        return which < 2 ? tc::Src{s + dR, D, 0, false, false} : tc::no_src();
+                        return which < 2 ? tc::Src{s + dR, D, 0, false, false}
+                                         : tc::Src{s + L.RDO, D, 0, false, false};
                     },
                     [&](int t, int k, float* v) {
                         if (which < 2) ld4(s + dR + (size_t)t * D + k, v);
@@ -805,7 +870,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                     [&](int) {
                         return (which == 0 || which == 3)
                                    ? tc::Src{s + Y + (size_t)n0 * D, D, 0, false, false}
-                                   : tc::no_src();
+                                   : tc::Src{s + L.RUU + (size_t)n0 * D, D, 0, false, false};
                     },
                     [&](int n, int k, float* v) {
                         const int ss = n0 + n;
