@@ -208,7 +208,8 @@ __device__ __forceinline__ void ld4in(const __nv_bfloat16* p, float* v) {
 // Tensor-core state shared by one CTA's products (TMEM columns, mbarrier).
 struct TcCta {
     tc::State st;
-    unsigned char* sbuf;
+    unsigned char* sbuf;  // 1 KB aligned start of the dynamic shared memory
+    int sbytes;           // bytes from sbuf to the end of the dynamic shared memory
 };
 
 // TMEM columns a chunk CTA allocates: single-pass k_bwd 512 (one CTA per SM);
@@ -268,12 +269,12 @@ __device__ __forceinline__ void tc_rows2(TcCta& t, int M, int K, const ASRC& asr
             };
             if constexpr (std::is_same<EPI, tc::RowStore>::value) {
                 tc::RowStore d = {epi.dst + (size_t)m0 * epi.ld, epi.ld};
-                tc::gemm_async<N>(t.st, t.sbuf, Mt, NB, K, as, fa, bsrc, fb4, d);
+                tc::gemm_async<N>(t.st, t.sbuf, t.sbytes, Mt, NB, K, as, fa, bsrc, fb4, d);
             } else if constexpr (tc::is_row8<EPI>::value) {
                 auto e8 = [&](int m, int n0, const float* v) { epi.f(m0 + m, n0, v); };
-                tc::gemm_async<N>(t.st, t.sbuf, Mt, NB, K, as, fa, bsrc, fb4, tc::Row8<decltype(e8)>{e8});
+                tc::gemm_async<N>(t.st, t.sbuf, t.sbytes, Mt, NB, K, as, fa, bsrc, fb4, tc::Row8<decltype(e8)>{e8});
             } else {
-                tc::gemm_async<N>(t.st, t.sbuf, Mt, NB, K, as, fa, bsrc, fb4,
+                tc::gemm_async<N>(t.st, t.sbuf, t.sbytes, Mt, NB, K, as, fa, bsrc, fb4,
                                   [&](int m, int n, float x) { epi(m0 + m, n, x); });
             }
         }
@@ -386,6 +387,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_intra(KParams p)
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
     tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
+    tcx.sbytes = (int)tc::dynamic_smem_bytes() - (int)(tcx.sbuf - dsm);
     tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, tmem_cols(PASSES));
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
@@ -561,6 +563,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_out(KParams p) {
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
     tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
+    tcx.sbytes = (int)tc::dynamic_smem_bytes() - (int)(tcx.sbuf - dsm);
     tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, tmem_cols(PASSES));
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
@@ -629,6 +632,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_bprep(KParams p)
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
     tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
+    tcx.sbytes = (int)tc::dynamic_smem_bytes() - (int)(tcx.sbuf - dsm);
     tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, tmem_cols(PASSES));
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;
@@ -691,6 +695,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
     extern __shared__ __align__(128) unsigned char dsm[];
     TcCta tcx;
     tcx.sbuf = dsm + ((1024u - (tc::smem_addr(dsm) & 1023u)) & 1023u);  // 1 KB aligned
+    tcx.sbytes = (int)tc::dynamic_smem_bytes() - (int)(tcx.sbuf - dsm);
     tc::init(tcx.st, &tmem_slot, &mbar, &tc_status, tmem_cols(PASSES, true));
     float* sm = reinterpret_cast<float*>(dsm);
     float* slot = p.scratch + (size_t)blockIdx.x * p.slot;

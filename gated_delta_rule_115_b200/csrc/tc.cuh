@@ -358,67 +358,92 @@ __host__ __device__ constexpr int async_stage_bytes() {
 // Same product as gemm<1, N, ...> (single TF32 pass) with the K segments that
 // asrc(k) / bsrc(k) describe copied asynchronously, two slabs in flight.
 // sbuf starts on a 1024-byte boundary; an MN-major B segment needs N % 32 == 0.
+// cp.async.wait_group with a run-time count (the instruction takes an immediate).
+__device__ __forceinline__ void cp_async_wait_upto(int n) {
+    switch (n) {
+        case 0: asm volatile("cp.async.wait_group 0;" ::: "memory"); break;
+        case 1: asm volatile("cp.async.wait_group 1;" ::: "memory"); break;
+        case 2: asm volatile("cp.async.wait_group 2;" ::: "memory"); break;
+        case 3: asm volatile("cp.async.wait_group 3;" ::: "memory"); break;
+        case 4: asm volatile("cp.async.wait_group 4;" ::: "memory"); break;
+        case 5: asm volatile("cp.async.wait_group 5;" ::: "memory"); break;
+        case 6: asm volatile("cp.async.wait_group 6;" ::: "memory"); break;
+        default: asm volatile("cp.async.wait_group 7;" ::: "memory"); break;
+    }
+}
+
+// Bytes of dynamic shared memory of this launch.
+__device__ __forceinline__ uint32_t dynamic_smem_bytes() {
+    uint32_t n;
+    asm("mov.u32 %0, %%dynamic_smem_size;" : "=r"(n));
+    return n;
+}
+
+// Same product as gemm<1, N, ...> (single TF32 pass).  K is processed in
+// rounds of as many 32-deep slabs as the sbytes of staging memory hold (at
+// most 8): every slab's segments that asrc(k) / bsrc(k) describe are copied
+// with cp.async at the start of the round (one group per slab), the others
+// produced from their element functors; the MMAs of a slab are issued as soon
+// as its group has landed, and the round ends with one completion wait.
+// sbuf starts on a 1024-byte boundary; an MN-major B segment needs N % 32 == 0.
 template <int N, class ASRC, class FA4, class BSRC, class FB4, class EPI>
-__device__ void gemm_async(State& s, unsigned char* sbuf, int M, int NB, int K, const ASRC& asrc,
-                           const FA4& fa4, const BSRC& bsrc, const FB4& fb4, const EPI& epi) {
+__device__ void gemm_async(State& s, unsigned char* sbuf, int sbytes, int M, int NB, int K,
+                           const ASRC& asrc, const FA4& fa4, const BSRC& bsrc, const FB4& fb4,
+                           const EPI& epi) {
     static_assert(N % 16 == 0 && N <= 256, "N");
     constexpr int ABLK = 128 * 32, BBLK = N * 32;
     constexpr int SLAB = 4 * (ABLK + BBLK);
     const int nslab = (K + 31) / 32;
+    int nbuf = sbytes / SLAB;
+    nbuf = nbuf < 1 ? 1 : (nbuf > 8 ? 8 : nbuf);
     auto blkA = [&](int buf, int ks) { return sbuf + buf * SLAB + ks * ABLK; };
     auto blkB = [&](int buf, int ks) { return sbuf + buf * SLAB + 4 * ABLK + ks * BBLK; };
-    auto issue_copies = [&](int sl, int buf) {
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const int k = sl * 32 + ks * 8;
-            if (k >= K) break;
-            const Src a = asrc(k), b = bsrc(k);
-            if (a.p) copy_block<128>(blkA(buf, ks), a, k, M, K);
-            if (b.p) copy_block<N>(blkB(buf, ks), b, k, NB, K);
-        }
-        asm volatile("cp.async.commit_group;");
-    };
-    auto run_producers = [&](int sl, int buf) {
-#pragma unroll
-        for (int ks = 0; ks < 4; ++ks) {
-            const int k = sl * 32 + ks * 8;
-            if (k >= K) break;
-            if (!asrc(k).p) produce_block<128>(blkA(buf, ks), k, M, K, fa4);
-            if (!bsrc(k).p) produce_block<N>(blkB(buf, ks), k, NB, K, fb4);
-        }
-    };
-    issue_copies(0, 0);
-    run_producers(0, 0);
-    for (int sl = 0; sl < nslab; ++sl) {
-        const int buf = sl & 1;
-        if (sl + 1 < nslab) {
-            issue_copies(sl + 1, buf ^ 1);
-            asm volatile("cp.async.wait_group 1;");
-        } else {
-            asm volatile("cp.async.wait_group 0;");
-        }
-        asm volatile("fence.proxy.async.shared::cta;");
-        __syncthreads();
-        if (threadIdx.x == 0) {
-            asm volatile("tcgen05.fence::after_thread_sync;");
+    for (int r0 = 0; r0 < nslab; r0 += nbuf) {
+        const int nr = nslab - r0 < nbuf ? nslab - r0 : nbuf;
+        for (int i = 0; i < nr; ++i) {
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
-                const int k = sl * 32 + ks * 8;
+                const int k = (r0 + i) * 32 + ks * 8;
                 if (k >= K) break;
                 const Src a = asrc(k), b = bsrc(k);
-                const bool amn = a.p && a.mn, bmn = b.p && b.mn;
-                const uint64_t da = amn ? make_desc_mn32(smem_addr(blkA(buf, ks)), 128 / 32 * 512)
-                                        : make_desc(smem_addr(blkA(buf, ks)), 128, 256);
-                const uint64_t db = bmn ? make_desc_mn32(smem_addr(blkB(buf, ks)), N / 32 * 512)
-                                        : make_desc(smem_addr(blkB(buf, ks)), 128, 256);
-                const uint32_t idesc = idesc_tf32(128, N) | ((a.p && a.neg) ? (1u << 13) : 0u) |
-                                       (amn ? (1u << 15) : 0u) | (bmn ? (1u << 16) : 0u);
-                issue_mma(s.tmem, da, db, idesc, k > 0 ? 1u : 0u);
+                if (a.p) copy_block<128>(blkA(i, ks), a, k, M, K);
+                if (b.p) copy_block<N>(blkB(i, ks), b, k, NB, K);
             }
-            commit(s);
+            asm volatile("cp.async.commit_group;" ::: "memory");
         }
-        if (sl + 1 < nslab) run_producers(sl + 1, buf ^ 1);  // overlaps this slab's MMAs
-        wait_mma(s);
+        for (int i = 0; i < nr; ++i) {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+                const int k = (r0 + i) * 32 + ks * 8;
+                if (k >= K) break;
+                if (!asrc(k).p) produce_block<128>(blkA(i, ks), k, M, K, fa4);
+                if (!bsrc(k).p) produce_block<N>(blkB(i, ks), k, NB, K, fb4);
+            }
+        }
+        for (int i = 0; i < nr; ++i) {
+            cp_async_wait_upto(nr - 1 - i);
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            __syncthreads();
+            if (threadIdx.x == 0) {
+                asm volatile("tcgen05.fence::after_thread_sync;");
+#pragma unroll
+                for (int ks = 0; ks < 4; ++ks) {
+                    const int k = (r0 + i) * 32 + ks * 8;
+                    if (k >= K) break;
+                    const Src a = asrc(k), b = bsrc(k);
+                    const bool amn = a.p && a.mn, bmn = b.p && b.mn;
+                    const uint64_t da = amn ? make_desc_mn32(smem_addr(blkA(i, ks)), 128 / 32 * 512)
+                                            : make_desc(smem_addr(blkA(i, ks)), 128, 256);
+                    const uint64_t db = bmn ? make_desc_mn32(smem_addr(blkB(i, ks)), N / 32 * 512)
+                                            : make_desc(smem_addr(blkB(i, ks)), 128, 256);
+                    const uint32_t idesc = idesc_tf32(128, N) | ((a.p && a.neg) ? (1u << 13) : 0u) |
+                                           (amn ? (1u << 15) : 0u) | (bmn ? (1u << 16) : 0u);
+                    issue_mma(s.tmem, da, db, idesc, k > 0 ? 1u : 0u);
+                }
+                if (i == nr - 1) commit(s);
+            }
+        }
+        wait_mma(s);  // the round's buffers are free again; after the last round D is final
     }
     // epilogue (as in gemm)
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
