@@ -205,6 +205,21 @@ __device__ __forceinline__ void ld4in(const __nv_bfloat16* p, float* v) {
     v[0] = fa.x; v[1] = fa.y; v[2] = fb.x; v[3] = fb.y;
 }
 
+// Eight consecutive outputs (16-byte aligned for bf16, 32-byte for float32).
+__device__ __forceinline__ void st8(float* p, const float* x) {
+    *reinterpret_cast<float4*>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    *reinterpret_cast<float4*>(p + 4) = make_float4(x[4], x[5], x[6], x[7]);
+}
+__device__ __forceinline__ void st8(__nv_bfloat16* p, const float* x) {
+    uint4 u;
+    __nv_bfloat162 h[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) h[i] = __floats2bfloat162_rn(x[2 * i], x[2 * i + 1]);
+    u.x = *reinterpret_cast<uint32_t*>(&h[0]); u.y = *reinterpret_cast<uint32_t*>(&h[1]);
+    u.z = *reinterpret_cast<uint32_t*>(&h[2]); u.w = *reinterpret_cast<uint32_t*>(&h[3]);
+    *reinterpret_cast<uint4*>(p) = u;
+}
+
 // Tensor-core state shared by one CTA's products (TMEM columns, mbarrier).
 struct TcCta {
     tc::State st;
@@ -399,17 +414,20 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_intra(KParams p)
         float* s = c.s;
         prologue2(c);
         masked_prep<Tin, D, PASSES>(c, false, false);
-        rows_prep<Tin, D, PASSES>(c, R_KT | R_UU);
+        rows_prep<Tin, D, PASSES>(c, R_KT | R_UU | R_AB | R_KB);
         masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
         __syncthreads();
         compute_tii(s, L, L.LA);
-        for (int idx = threadIdx.x; idx < C * D; idx += kThreads)
-            s[L.W[0] + idx] = c.A(idx / D, idx % D) * facs(c).egb(idx / D, idx % D);  // Ab
+        // Ab (single-pass: the prepared rows; three-pass: formed here in full float32)
+        const size_t ab = PASSES == 1 ? L.RAB : L.W[0];
+        if (PASSES != 1)
+            for (int idx = threadIdx.x; idx < C * D; idx += kThreads)
+                s[ab + idx] = c.A(idx / D, idx % D) * facs(c).egb(idx / D, idx % D);
         __syncthreads();
-        solve_s<D, PASSES, true>(s, sm, L, L.LA, L.W[0]);  // Psi = T^T Ab
+        solve_s<D, PASSES, true>(s, sm, L, L.LA, ab);  // Psi = T^T Ab (in place)
         __syncthreads();
         float* M = p.M + c.sbase;
-        const float* Psi = s + L.W[0];
+        const float* Psi = s + ab;
         const Fac<Tin, D> f = facs(c);
         // M = diag(e^gbar) - Psi^T Kt      (rows i, contraction over tokens)
         tc_rows2<PASSES, D, true, true>(tcx, D, C,
@@ -430,7 +448,10 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_intra(KParams p)
             [&](int t, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = s[L.LK + (size_t)(k + u) * C + t]; },
             [&](int) { return tc::Src{Psi, D, 0, true, false}; },
             [&](int j, int k, float* v) { for (int u = 0; u < 4; ++u) v[u] = Psi[(size_t)(k + u) * D + j]; },
-            [&](int t, int j, float x) { Phi[(size_t)t * D + j] = c.K(t, j) * f.egb(t, j) - x; });
+            [&](int t, int j, float x) {
+                const float kb = PASSES == 1 ? s[L.RKB + (size_t)t * D + j] : c.K(t, j) * f.egb(t, j);
+                Phi[(size_t)t * D + j] = kb - x;
+            });
         // Bn = Phi^T U
         float* Bn = p.Bn + c.sbase;
         tc_rows2<PASSES, D, true, true>(tcx, D, C,
@@ -586,6 +607,8 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_out(KParams p) {
         Tout* o = (Tout*)p.o;
         const Fac<Tin, D> f = facs(c);
         const float* Y = s + L.W[0];
+        // eight consecutive outputs of one row per store (16 or 32 bytes)
+        auto ostore = [&](int t, int j, const float* x) { st8(o + c.base + (size_t)t * c.rs + j, x); };
         // O = Qt S + M_QK U - M_QA Y
         tc_rows2<PASSES, D, false, true>(tcx, C, D + 2 * C,
             [&](int k) {
@@ -616,7 +639,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_out(KParams p) {
                 else if (k < D + C) for (int u = 0; u < 4; ++u) v[u] = c.U(k - D + u, cc);
                 else for (int u = 0; u < 4; ++u) v[u] = Y[(size_t)(k - D - C + u) * D + cc];
             },
-            [&](int t, int j, float x) { stf(o + c.base + t * c.rs + j, x); });
+            tc::Row8<decltype(ostore)>{ostore});
     }
     if (threadIdx.x == 0 && tc_status != 0) atomicAdd(&g_wait_timeouts, 1u);
     tc::release(tcx.st, tmem_cols(PASSES));
