@@ -324,44 +324,58 @@ __device__ __forceinline__ void masked_prep(Chunk<Tin, D>& c, bool with_q, bool 
 //   R_DO  dO                  R_AB  Ab = e k e^{gbar-Gam}  R_KB  Kb = K e^{gbar-Gam}
 enum RowOps { R_KT = 1, R_QT = 2, R_UU = 4, R_DO = 8, R_AB = 16, R_KB = 32 };
 
-template <typename Tin, int D, int PASSES>
+// U2: items per thread whose loads are issued together (2 where registers allow).
+template <typename Tin, int D, int PASSES, int U2 = 1>
 __device__ void rows_prep(const Chunk<Tin, D>& c, int ops) {
     if constexpr (PASSES != 1) return;
     const Lay& L = c.L;
     const int n4 = L.C * D / 4;
-    for (int idx = threadIdx.x; idx < n4; idx += kThreads) {
-        const int t = idx / (D / 4), j = 4 * (idx % (D / 4));
-        const size_t g = c.base + (size_t)t * c.rs + j, x = (size_t)t * D + j;
-        const size_t b = (size_t)(t >> 3) * D + j;
-        float k4[4] = {0.f, 0.f, 0.f, 0.f}, e4[4], q4[4], m4[4], v4[4], w4[4], o4[4];
-        float lc[4], pre[4], rc[4], suf[4];
-        if (ops & (R_KT | R_KB | R_AB)) ld4in(c.k + g, k4);
-        if (ops & R_AB) ld4in(c.e + g, e4);
-        if (ops & R_QT) { ld4in(c.q + g, q4); ld4in(c.gm + g, m4); }
-        if (ops & R_UU) { ld4in(c.v + g, v4); ld4in(c.w + g, w4); }
-        if (ops & R_DO) ld4in(c.dO + g, o4);
-        if (ops & (R_KT | R_QT)) { ld4(c.s + L.LC + x, lc); ld4(c.s + L.PRE + b, pre); }
-        if (ops & (R_KB | R_AB)) { ld4(c.s + L.RC + x, rc); ld4(c.s + L.SUF + b, suf); }
-        float4 kt, qt, uu, dd, ab, kb;
-        float* pkt = &kt.x; float* pqt = &qt.x; float* puu = &uu.x; float* pdd = &dd.x;
-        float* pab = &ab.x; float* pkb = &kb.x;
+    for (int base = threadIdx.x; base < n4; base += U2 * kThreads) {
+        float k4[U2][4], e4[U2][4], q4[U2][4], m4[U2][4], v4[U2][4], w4[U2][4], o4[U2][4];
+        float lc[U2][4], pre[U2][4], rc[U2][4], suf[U2][4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const float eg = (ops & (R_KT | R_QT)) ? fexp<Tin>(pre[u] + lc[u]) : 0.f;
-            const float egb = (ops & (R_KB | R_AB)) ? fexp<Tin>(rc[u] + suf[u]) : 0.f;
-            pkt[u] = tc::tf32_rn(k4[u] * eg);
-            pqt[u] = (ops & R_QT) ? tc::tf32_rn(q4[u] * m4[u] * eg) : 0.f;
-            puu[u] = (ops & R_UU) ? tc::tf32_rn(v4[u] * w4[u]) : 0.f;
-            pdd[u] = (ops & R_DO) ? tc::tf32_rn(o4[u]) : 0.f;
-            pab[u] = (ops & R_AB) ? tc::tf32_rn(e4[u] * k4[u] * egb) : 0.f;
-            pkb[u] = tc::tf32_rn(k4[u] * egb);
+        for (int i = 0; i < U2; ++i) {
+            const int idx = base + i * kThreads;
+            if (idx >= n4) break;
+            const int t = idx / (D / 4), j = 4 * (idx % (D / 4));
+            const size_t g = c.base + (size_t)t * c.rs + j, x = (size_t)t * D + j;
+            const size_t b = (size_t)(t >> 3) * D + j;
+            if (ops & (R_KT | R_KB | R_AB)) ld4in(c.k + g, k4[i]);
+            if (ops & R_AB) ld4in(c.e + g, e4[i]);
+            if (ops & R_QT) { ld4in(c.q + g, q4[i]); ld4in(c.gm + g, m4[i]); }
+            if (ops & R_UU) { ld4in(c.v + g, v4[i]); ld4in(c.w + g, w4[i]); }
+            if (ops & R_DO) ld4in(c.dO + g, o4[i]);
+            if (ops & (R_KT | R_QT)) { ld4(c.s + L.LC + x, lc[i]); ld4(c.s + L.PRE + b, pre[i]); }
+            if (ops & (R_KB | R_AB)) { ld4(c.s + L.RC + x, rc[i]); ld4(c.s + L.SUF + b, suf[i]); }
         }
-        if (ops & R_KT) *reinterpret_cast<float4*>(c.s + L.RKT + x) = kt;
-        if (ops & R_QT) *reinterpret_cast<float4*>(c.s + L.RQT + x) = qt;
-        if (ops & R_UU) *reinterpret_cast<float4*>(c.s + L.RUU + x) = uu;
-        if (ops & R_DO) *reinterpret_cast<float4*>(c.s + L.RDO + x) = dd;
-        if (ops & R_AB) *reinterpret_cast<float4*>(c.s + L.RAB + x) = ab;
-        if (ops & R_KB) *reinterpret_cast<float4*>(c.s + L.RKB + x) = kb;
+#pragma unroll
+        for (int i = 0; i < U2; ++i) {
+            const int idx = base + i * kThreads;
+            if (idx >= n4) break;
+            const int t = idx / (D / 4), j = 4 * (idx % (D / 4));
+            const size_t x = (size_t)t * D + j;
+            float4 kt, qt, uu, dd, ab, kb;
+            float* pkt = &kt.x; float* pqt = &qt.x; float* puu = &uu.x; float* pdd = &dd.x;
+            float* pab = &ab.x; float* pkb = &kb.x;
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const float eg = (ops & (R_KT | R_QT)) ? fexp<Tin>(pre[i][u] + lc[i][u]) : 0.f;
+                const float egb = (ops & (R_KB | R_AB)) ? fexp<Tin>(rc[i][u] + suf[i][u]) : 0.f;
+                const float kk = (ops & (R_KT | R_KB | R_AB)) ? k4[i][u] : 0.f;
+                pkt[u] = tc::tf32_rn(kk * eg);
+                pqt[u] = (ops & R_QT) ? tc::tf32_rn(q4[i][u] * m4[i][u] * eg) : 0.f;
+                puu[u] = (ops & R_UU) ? tc::tf32_rn(v4[i][u] * w4[i][u]) : 0.f;
+                pdd[u] = (ops & R_DO) ? tc::tf32_rn(o4[i][u]) : 0.f;
+                pab[u] = (ops & R_AB) ? tc::tf32_rn(e4[i][u] * kk * egb) : 0.f;
+                pkb[u] = tc::tf32_rn(kk * egb);
+            }
+            if (ops & R_KT) *reinterpret_cast<float4*>(c.s + L.RKT + x) = kt;
+            if (ops & R_QT) *reinterpret_cast<float4*>(c.s + L.RQT + x) = qt;
+            if (ops & R_UU) *reinterpret_cast<float4*>(c.s + L.RUU + x) = uu;
+            if (ops & R_DO) *reinterpret_cast<float4*>(c.s + L.RDO + x) = dd;
+            if (ops & R_AB) *reinterpret_cast<float4*>(c.s + L.RAB + x) = ab;
+            if (ops & R_KB) *reinterpret_cast<float4*>(c.s + L.RKB + x) = kb;
+        }
     }
     __syncthreads();
 }
@@ -734,7 +748,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                      dU = L.W[5], dGam = L.W[6];
         prologue2(c);
         masked_prep<Tin, D, PASSES>(c, true, true);
-        rows_prep<Tin, D, PASSES>(c, R_KT | R_UU | R_DO | R_AB | R_KB);
+        rows_prep<Tin, D, PASSES, 2>(c, R_KT | R_UU | R_DO | R_AB | R_KB);
         masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
         masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
         __syncthreads();
@@ -964,26 +978,32 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                     tmem_ld8(lane_base + 256 + 8 * I, z1);
                     tmem_ld8(lane_base + 384 + 8 * I, z2);
                     const float pre = s[L.PRE + (size_t)I * D + cc];
+                    // all loads of the block first, then the arithmetic and the stores
+                    float lc[8], kv[8], qv[8], gmv[8], ev[8], vv[8], wv[8];
+                    float dk0[8], dq0[8], da0[8], dg0[8], du0[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        const int t = t0 + u;
-                        const size_t x = (size_t)t * D + cc, gi = c.base + (size_t)t * c.rs + cc;
-                        const float lc = s[L.LC + x];
-                        const float kv = ldf(c.k + gi), qv = ldf(c.q + gi), gmv = ldf(c.gm + gi);
-                        const float ev = ldf(c.e + gi), vv = ldf(c.v + gi), wv = ldf(c.w + gi);
-                        const float dk0 = s[dK + x], dq0 = s[dQh + x], da0 = s[dA + x];
-                        const float dg0 = s[dGam + x], du0 = s[dU + x];
-                        const float d = pre + lc - hp;
+                        const size_t x = (size_t)(t0 + u) * D + cc, gi = c.base + (size_t)(t0 + u) * c.rs + cc;
+                        lc[u] = s[L.LC + x];
+                        kv[u] = ldf(c.k + gi); qv[u] = ldf(c.q + gi); gmv[u] = ldf(c.gm + gi);
+                        ev[u] = ldf(c.e + gi); vv[u] = ldf(c.v + gi); wv[u] = ldf(c.w + gi);
+                        dk0[u] = s[dK + x]; dq0[u] = s[dQh + x]; da0[u] = s[dA + x];
+                        dg0[u] = s[dGam + x]; du0[u] = s[dU + x];
+                    }
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const size_t x = (size_t)(t0 + u) * D + cc, gi = c.base + (size_t)(t0 + u) * c.rs + cc;
+                        const float d = pre + lc[u] - hp;
                         const float fx = fexp<Tin>(d), fz = fexp<Tin>(-d);
                         const float vx1 = fx * x1[u], vx2 = fx * x2[u], vz1 = fz * z1[u], vz2 = fz * z2[u];
-                        const float DK = dk0 + vx1 + vz2, DQ = dq0 + vx2, DA = da0 + vz1;
-                        s[dGam + x] = dg0 + kv * (vx1 - vz2) + qv * gmv * vx2 - ev * kv * vz1;
-                        stf(gq + gi, DQ * gmv);
-                        stf(ggm + gi, DQ * qv);
-                        stf(ge + gi, DA * kv);
-                        stf(gk + gi, DK + DA * ev);
-                        stf(gw + gi, du0 * vv);
-                        stf(gv + gi, du0 * wv);
+                        const float DK = dk0[u] + vx1 + vz2, DQ = dq0[u] + vx2, DA = da0[u] + vz1;
+                        s[dGam + x] = dg0[u] + kv[u] * (vx1 - vz2) + qv[u] * gmv[u] * vx2 - ev[u] * kv[u] * vz1;
+                        stf(gq + gi, DQ * gmv[u]);
+                        stf(ggm + gi, DQ * qv[u]);
+                        stf(ge + gi, DA * kv[u]);
+                        stf(gk + gi, DK + DA * ev[u]);
+                        stf(gw + gi, du0[u] * vv[u]);
+                        stf(gv + gi, du0[u] * wv[u]);
                     }
                 }
             }
