@@ -254,8 +254,10 @@ def gpu_arm(args, rank, world, local):
     args_in = [d[n] for n in NAMES]
 
     def step():
-        o, S, Sc, Mc = muir.chunk_fwd(*args_in, d["S0"], chunk=C, return_saved=True, ws=ws_f)
-        gr = muir.chunk_bwd(*args_in, d["S0"], d["dO"], chunk=C, S_chunks=Sc, M_chunks=Mc, ws=ws_b)
+        o, S, Sc, Mc, aux = muir.chunk_fwd(*args_in, d["S0"], chunk=C, return_saved=True,
+                                           save_aux=True, ws=ws_f)
+        gr = muir.chunk_bwd(*args_in, d["S0"], d["dO"], chunk=C, S_chunks=Sc, M_chunks=Mc,
+                            aux=aux, ws=ws_b)
         return o, gr
 
     ws_f = torch.empty(muir.fwd_workspace_bytes(W.B, W.T, W.H, W.dk, C), dtype=torch.uint8, device=dev)
@@ -392,9 +394,10 @@ def e2e_measure(muir, x, W, C, dev, ws_f, ws_b, steps, world):
         for k, v in host.items():
             dev_in[k].copy_(v, non_blocking=True)
         a = [dev_in[n] for n in NAMES]
-        o, S, Sc, Mc = muir.chunk_fwd(*a, dev_in.get("S0"), chunk=C, return_saved=True, ws=ws_f)
+        o, S, Sc, Mc, aux = muir.chunk_fwd(*a, dev_in.get("S0"), chunk=C, return_saved=True,
+                                           save_aux=True, ws=ws_f)
         gr = muir.chunk_bwd(*a, dev_in.get("S0"), dev_in["dO"], chunk=C, S_chunks=Sc, M_chunks=Mc,
-                            ws=ws_b)
+                            aux=aux, ws=ws_b)
         res = [o, S] + [gr[k] for k in sorted(gr)]
         if outs_host is None:
             outs_host = [torch.empty_like(r, device="cpu").pin_memory() for r in res]

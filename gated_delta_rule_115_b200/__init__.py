@@ -62,13 +62,15 @@ def lib():
         L.muir_device_wait_status.restype = I
         L.muir_status_string.argtypes = [I]
         L.muir_status_string.restype = ctypes.c_char_p
+        L.muir_chunk_aux_floats.argtypes = [SP]
+        L.muir_chunk_aux_floats.restype = ctypes.c_size_t
         L.muir_chunk_fwd_workspace.argtypes = [SP]
         L.muir_chunk_fwd_workspace.restype = S
         L.muir_chunk_bwd_workspace.argtypes = [SP]
         L.muir_chunk_bwd_workspace.restype = S
-        L.muir_chunk_fwd.argtypes = [SP] + [P] * 13 + [S, P]
+        L.muir_chunk_fwd.argtypes = [SP] + [P] * 14 + [S, P]
         L.muir_chunk_fwd.restype = I
-        L.muir_chunk_bwd.argtypes = [SP] + [P] * 21 + [S, P]
+        L.muir_chunk_bwd.argtypes = [SP] + [P] * 22 + [S, P]
         L.muir_chunk_bwd.restype = I
         L.muir_recurrent_step.argtypes = [I, I, I, I, I, I] + [P] * 7 + [I, P, P, P]
         L.muir_recurrent_step.restype = I
@@ -151,12 +153,13 @@ def _workspace(nbytes, dev, ws):
 
 
 def chunk_fwd(q, k, v, g, e, w, gamma, S0=None, chunk=64, out_dtype=None,
-              return_chunk_states=False, return_saved=False, ws=None):
+              return_chunk_states=False, return_saved=False, save_aux=False, ws=None):
     """Chunkwise forward.  Returns ``(o, S_final)``; with ``return_chunk_states``
     ``(o, S_final, S_chunks)`` where ``S_chunks[b,h,n]`` is the state at the start
     of chunk ``n``; with ``return_saved`` ``(o, S_final, S_chunks, M_chunks)``
-    where ``M_chunks[b,h,n]`` is chunk n's transition.  Both are reusable by
-    :func:`chunk_bwd`."""
+    where ``M_chunks[b,h,n]`` is chunk n's transition, and with ``save_aux`` as
+    well a fifth element ``aux``, the per-chunk intermediates
+    (``muir_chunk_aux_floats``).  All are reusable by :func:`chunk_bwd`."""
     L = lib()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
@@ -168,23 +171,28 @@ def chunk_fwd(q, k, v, g, e, w, gamma, S0=None, chunk=64, out_dtype=None,
           if (return_chunk_states or return_saved) else None)
     Mc = (torch.empty(B, H, T // chunk, dk, dk, dtype=torch.float32, device=q.device)
           if return_saved else None)
+    aux = None
+    if return_saved and save_aux:
+        aux = torch.empty(int(L.muir_chunk_aux_floats(ctypes.byref(shp))), dtype=torch.float32,
+                          device=q.device)
     need = int(L.muir_chunk_fwd_workspace(ctypes.byref(shp)))
     wsb = _workspace(need, q.device, ws)
     rc = L.muir_chunk_fwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(e),
                           _ptr(w), _ptr(gamma), _ptr(S0), _ptr(o), _ptr(S_final), _ptr(Sc),
-                          _ptr(Mc), _ptr(wsb), ctypes.c_size_t(0 if wsb is None else wsb.numel()),
-                          _stream(q.device))
+                          _ptr(Mc), _ptr(aux), _ptr(wsb),
+                          ctypes.c_size_t(0 if wsb is None else wsb.numel()), _stream(q.device))
     _check("muir_chunk_fwd", rc)
     if return_saved:
-        return o, S_final, Sc, Mc
+        return (o, S_final, Sc, Mc, aux) if save_aux else (o, S_final, Sc, Mc)
     return (o, S_final, Sc) if return_chunk_states else (o, S_final)
 
 
 def chunk_bwd(q, k, v, g, e, w, gamma, S0, dO, dS_final=None, chunk=64, S_chunks=None,
-              M_chunks=None, ws=None):
+              M_chunks=None, aux=None, ws=None):
     """Gradients of ``sum(o*dO) + sum(S_final*dS_final)``.  Returns a dict with
     ``dq, dk, dv, dg, de, dw, dgamma`` (input dtype) and ``dS0`` (float32).
-    ``S_chunks`` / ``M_chunks`` from :func:`chunk_fwd` skip recomputation."""
+    ``S_chunks`` / ``M_chunks`` / ``aux`` from :func:`chunk_fwd` skip
+    recomputation (``aux`` only together with ``S_chunks``)."""
     L = lib()
     shp = _shape(q, v, chunk, None)
     grads = {n: torch.empty_like(x) for n, x in
@@ -194,7 +202,8 @@ def chunk_bwd(q, k, v, g, e, w, gamma, S0, dO, dS_final=None, chunk=64, S_chunks
     need = int(L.muir_chunk_bwd_workspace(ctypes.byref(shp)))
     wsb = _workspace(need, q.device, ws)
     rc = L.muir_chunk_bwd(ctypes.byref(shp), _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(e),
-                          _ptr(w), _ptr(gamma), _ptr(S0), _ptr(S_chunks), _ptr(M_chunks), _ptr(dO),
+                          _ptr(w), _ptr(gamma), _ptr(S0), _ptr(S_chunks), _ptr(M_chunks), _ptr(aux),
+                          _ptr(dO),
                           _ptr(dS_final), _ptr(grads["dq"]), _ptr(grads["dk"]),
                           _ptr(grads["dv"]), _ptr(grads["dg"]), _ptr(grads["de"]),
                           _ptr(grads["dw"]), _ptr(grads["dgamma"]), _ptr(grads["dS0"]),
@@ -226,17 +235,17 @@ class MuirChunkFunction(torch.autograd.Function):
 
     @staticmethod
     def forward(ctx, q, k, v, g, e, w, gamma, S0, chunk):
-        o, S_final, Sc, Mc = chunk_fwd(q, k, v, g, e, w, gamma, S0, chunk=chunk,
-                                       return_saved=True)
-        ctx.save_for_backward(q, k, v, g, e, w, gamma, S0, Sc, Mc)
+        o, S_final, Sc, Mc, aux = chunk_fwd(q, k, v, g, e, w, gamma, S0, chunk=chunk,
+                                            return_saved=True, save_aux=True)
+        ctx.save_for_backward(q, k, v, g, e, w, gamma, S0, Sc, Mc, aux)
         ctx.chunk = chunk
         return o, S_final
 
     @staticmethod
     def backward(ctx, dO, dS_final):
-        q, k, v, g, e, w, gamma, S0, Sc, Mc = ctx.saved_tensors
+        q, k, v, g, e, w, gamma, S0, Sc, Mc, aux = ctx.saved_tensors
         gr = chunk_bwd(q, k, v, g, e, w, gamma, S0, dO.contiguous().to(q.dtype),
                        None if dS_final is None else dS_final.contiguous().float(),
-                       chunk=ctx.chunk, S_chunks=Sc, M_chunks=Mc)
+                       chunk=ctx.chunk, S_chunks=Sc, M_chunks=Mc, aux=aux)
         return (gr["dq"], gr["dk"], gr["dv"], gr["dg"], gr["de"], gr["dw"], gr["dgamma"],
                 gr["dS0"] if S0 is not None else None, None)

@@ -47,6 +47,7 @@ muir::ChunkProblem make_problem(const muir_shape* s, const void* q, const void* 
     P.in_bf16 = s->in_dtype == MUIR_BF16;
     P.out_bf16 = s->out_dtype == MUIR_BF16;
     P.q = q; P.k = k; P.v = v; P.g = g; P.e = e; P.w = w; P.gamma = gamma;
+    P.aux = nullptr;
     return P;
 }
 
@@ -79,6 +80,11 @@ muir_status muir_device_wait_status(void) {
     return n ? MUIR_ERR_DEVICE_TIMEOUT : MUIR_OK;
 }
 
+size_t muir_chunk_aux_floats(const muir_shape* s) {
+    if (check_shape(s) != MUIR_OK) return 0;
+    return (size_t)s->B * s->H * (s->T / s->chunk) * muir::chunk_aux_floats(s->chunk, s->dk);
+}
+
 size_t muir_chunk_fwd_workspace(const muir_shape* s) {
     if (check_shape(s) != MUIR_OK) return 0;
     return muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false);
@@ -92,18 +98,19 @@ size_t muir_chunk_bwd_workspace(const muir_shape* s) {
 muir_status muir_chunk_fwd(const muir_shape* s, const void* q, const void* k, const void* v,
                            const void* g, const void* e, const void* w, const void* gamma,
                            const float* S0, void* o, float* S_final, float* S_chunks,
-                           float* M_chunks, void* ws, size_t ws_bytes, void* stream) {
+                           float* M_chunks, float* aux, void* ws, size_t ws_bytes, void* stream) {
     muir_status st = check_shape(s);
     if (st != MUIR_OK) return st;
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
         !ok_ptr(gamma) || !ok_ptr(o) || !ok_opt(S0) || !ok_opt(S_final) || !ok_opt(S_chunks) ||
-        !ok_opt(M_chunks))
+        !ok_opt(M_chunks) || !ok_opt(aux))
         return MUIR_ERR_INVALID_ARG;
     const size_t need = muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk,
                                                  S_chunks != nullptr);
     if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
     if ((st = check_device()) != MUIR_OK) return st;
     muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);
+    P.aux = aux;
     return from_cuda(muir::run_chunk_fwd(P, S0, o, S_final, S_chunks, M_chunks, ws, ws_bytes,
                                          static_cast<cudaStream_t>(stream)));
 }
@@ -111,7 +118,8 @@ muir_status muir_chunk_fwd(const muir_shape* s, const void* q, const void* k, co
 muir_status muir_chunk_bwd(const muir_shape* s, const void* q, const void* k, const void* v,
                            const void* g, const void* e, const void* w, const void* gamma,
                            const float* S0, const float* S_chunks, const float* M_chunks,
-                           const void* dO, const float* dS_final, void* dq, void* dk, void* dv,
+                           const float* aux, const void* dO, const float* dS_final, void* dq,
+                           void* dk, void* dv,
                            void* dg, void* de, void* dw, void* dgamma, float* dS0, void* ws,
                            size_t ws_bytes, void* stream) {
     muir_status st = check_shape(s);
@@ -119,13 +127,15 @@ muir_status muir_chunk_bwd(const muir_shape* s, const void* q, const void* k, co
     if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
         !ok_ptr(gamma) || !ok_ptr(dO) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) ||
         !ok_ptr(dg) || !ok_ptr(de) || !ok_ptr(dw) || !ok_ptr(dgamma) || !ok_opt(S0) ||
-        !ok_opt(S_chunks) || !ok_opt(M_chunks) || !ok_opt(dS_final) || !ok_opt(dS0))
+        !ok_opt(S_chunks) || !ok_opt(M_chunks) || !ok_opt(dS_final) || !ok_opt(dS0) ||
+        !ok_opt(aux) || (aux && !S_chunks))
         return MUIR_ERR_INVALID_ARG;
     const size_t need = muir::chunk_bwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk,
                                                  S_chunks != nullptr);
     if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
     if ((st = check_device()) != MUIR_OK) return st;
     muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);
+    P.aux = const_cast<float*>(aux);
     return from_cuda(muir::run_chunk_bwd(P, S0, S_chunks, M_chunks, dO, dS_final, dq, dk, dv, dg,
                                          de, dw, dgamma, dS0, ws, ws_bytes,
                                          static_cast<cudaStream_t>(stream)));

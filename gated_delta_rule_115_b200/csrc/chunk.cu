@@ -6,6 +6,8 @@
 
 namespace muir {
 
+size_t chunk_aux_floats(int C, int D) { return make_aux_lay(C, D).total; }
+
 size_t chunk_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states) {
     const size_t nch = (size_t)B * H * (T / C), DD = (size_t)D * D;
     size_t f = 2 * nch * DD;               // M, Bn

@@ -108,6 +108,7 @@ struct KParams {
     void *dq, *dk, *dv, *dg, *de, *dw, *dgamma;
     float* scratch;
     size_t slot;             // floats per scratch slot
+    float* aux;              // per-chunk saved intermediates or null
 };
 
 // Accessors of one chunk's inputs; row t of a [B,T,H,D] tensor.
@@ -147,6 +148,64 @@ __device__ Chunk<Tin, D> make_chunk(const KParams& p, int chunk, float* slot) {
     c.L = make_lay(CF ? CF : p.C, D);
     c.tame = false;
     return c;
+}
+
+// ------------------------------------------------------------------ saved intermediates
+
+// Per-chunk layout of the intermediates the forward saves for the backward:
+// L_A, L_K, M_QK, M_QA (C x C), the inverted 16 x 16 diagonal blocks (C x 16), Y (C x D).
+struct AuxLay {
+    size_t LA, LK, MQK, MQA, TII, Y, total;
+};
+
+__host__ __device__ inline AuxLay make_aux_lay(int C, int D) {
+    AuxLay A;
+    size_t o = 0;
+    auto take = [&](size_t n) { const size_t r = o; o += (n + 63) & ~(size_t)63; return r; };
+    const size_t cc = (size_t)C * C;
+    A.LA = take(cc); A.LK = take(cc); A.MQK = take(cc); A.MQA = take(cc);
+    A.TII = take((size_t)C * 16); A.Y = take((size_t)C * D);
+    A.total = o;
+    return A;
+}
+
+// Copy n floats (multiple of 4, 16-byte aligned) between global arrays, every
+// thread's loads of a batch issued before its stores.
+__device__ __forceinline__ void copy_floats(float* dst, const float* src, size_t n) {
+    constexpr int BATCH = 8;
+    const size_t n4 = n / 4;
+    for (size_t base = threadIdx.x; base < n4; base += (size_t)BATCH * kThreads) {
+        float4 v[BATCH];
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+            const size_t idx = base + (size_t)i * kThreads;
+            if (idx < n4) v[i] = reinterpret_cast<const float4*>(src)[idx];
+        }
+#pragma unroll
+        for (int i = 0; i < BATCH; ++i) {
+            const size_t idx = base + (size_t)i * kThreads;
+            if (idx < n4) reinterpret_cast<float4*>(dst)[idx] = v[i];
+        }
+    }
+}
+
+// Save (to_aux) or restore this chunk's intermediates between the scratch slot
+// and the chunk's aux record; y_off is Y's place in the scratch slot; mask
+// selects parts: 1 L_A, 2 L_K, 4 M_QK, 8 M_QA, 16 block inverses, 32 Y.
+template <typename Tin, int D>
+__device__ void aux_copy(const Chunk<Tin, D>& c, float* rec, bool to_aux, int mask, size_t y_off) {
+    const Lay& L = c.L;
+    const AuxLay A = make_aux_lay(L.C, D);
+    const size_t cc = (size_t)L.C * L.C;
+    const size_t so[6] = {L.LA, L.LK, L.MQK, L.MQA, L.TII, y_off};
+    const size_t ao[6] = {A.LA, A.LK, A.MQK, A.MQA, A.TII, A.Y};
+    const size_t n[6] = {cc, cc, cc, cc, (size_t)L.C * 16, (size_t)L.C * D};
+    for (int i = 0; i < 6; ++i) {
+        if (!(mask & (1 << i))) continue;
+        if (to_aux) copy_floats(rec + ao[i], c.s + so[i], n[i]);
+        else copy_floats(c.s + so[i], rec + ao[i], n[i]);
+    }
+    __syncthreads();
 }
 
 // ------------------------------------------------------------------ masked products
@@ -618,6 +677,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_out(KParams p) {
         __syncthreads();
         const float* S = p.S_chunks + c.sbase;
         compute_Y<Tin, D, PASSES>(tcx, c, S, L.W[0]);
+        if (p.aux) aux_copy(c, p.aux + (size_t)chunk * make_aux_lay(C, D).total, true, 63, L.W[0]);
         Tout* o = (Tout*)p.o;
         const Fac<Tin, D> f = facs(c);
         const float* Y = s + L.W[0];
@@ -680,13 +740,17 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_bprep(KParams p)
         const int C = L.C;
         float* s = c.s;
         prologue2(c);
-        masked_prep<Tin, D, PASSES>(c, true, false);
         rows_prep<Tin, D, PASSES>(c, R_KT | R_QT | R_DO);
-        masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
-        masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
-        __syncthreads();
-        compute_tii(s, L, L.LA);
-        __syncthreads();
+        if (p.aux) {  // L_A, M_QA and the block inverses the forward saved
+            aux_copy(c, p.aux + (size_t)chunk * make_aux_lay(C, D).total, false, 1 | 8 | 16, 0);
+        } else {
+            masked_prep<Tin, D, PASSES>(c, true, false);
+            masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
+            masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
+            __syncthreads();
+            compute_tii(s, L, L.LA);
+            __syncthreads();
+        }
         float* Xi = s + L.W[0];
         // Z0 = M_QA^T dO
         tc_rows2<PASSES, D, true, true>(tcx, C, C,
@@ -747,14 +811,18 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         const size_t Y = L.W[0], dR = L.W[1], dK = L.W[2], dQh = L.W[3], dA = L.W[4],
                      dU = L.W[5], dGam = L.W[6];
         prologue2(c);
-        masked_prep<Tin, D, PASSES>(c, true, true);
+        masked_prep<Tin, D, PASSES>(c, true, true);  // path choice and gradient operands
         rows_prep<Tin, D, PASSES, 2>(c, R_KT | R_UU | R_DO | R_AB | R_KB);
-        masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
-        masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
-        __syncthreads();
-        compute_tii(s, L, L.LA);
-        __syncthreads();
-        compute_Y<Tin, D, PASSES>(tcx, c, S, Y);
+        if (p.aux) {  // masked matrices, block inverses and Y the forward saved
+            aux_copy(c, p.aux + (size_t)chunk * make_aux_lay(C, D).total, false, 63, Y);
+        } else {
+            masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
+            masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
+            __syncthreads();
+            compute_tii(s, L, L.LA);
+            __syncthreads();
+            compute_Y<Tin, D, PASSES>(tcx, c, S, Y);
+        }
         const Fac<Tin, D> f = facs(c);
         // dY = -M_QA^T dO - Ab dS'   (stored in dR, then dR = T^T dY)
         tc_rows2<PASSES, D, true, true>(tcx, C, C + D,
@@ -1207,6 +1275,7 @@ cudaError_t fwd_impl(const ChunkProblem& P, const float* S0, void* o, float* S_f
     kp.slot = slot_floats(P.C, D);
     kp.S_chunks = Sc;
     kp.o = o;
+    kp.aux = P.aux;
     const int dyn = dyn_bytes<D, PASSES>(P.C, false);
     cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn, dyn_bytes<D, PASSES>(P.C, true));
     if (err != cudaSuccess) return err;
@@ -1247,6 +1316,7 @@ cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chun
     kp.S_chunks = Sc;
     kp.dS_chunks = dSc;
     kp.dq = dq; kp.dk = dk; kp.dv = dv; kp.dg = dg; kp.de = de; kp.dw = dw; kp.dgamma = dgamma;
+    kp.aux = recompute ? nullptr : P.aux;  // the saved Y belongs to the saved chunk states
     const int dyn = dyn_bytes<D, PASSES>(P.C, false), dyn_b = dyn_bytes<D, PASSES>(P.C, true);
     cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn, dyn_b);
     if (err != cudaSuccess) return err;

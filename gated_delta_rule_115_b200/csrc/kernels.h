@@ -17,7 +17,11 @@ struct ChunkProblem {
     int N;                 // chunks per sequence, T / C
     bool in_bf16, out_bf16;
     const void *q, *k, *v, *g, *e, *w, *gamma;
+    float* aux;            // per-chunk saved intermediates (forward: written; backward: read) or null
 };
+
+// Floats per chunk of the saved intermediates (muir_chunk_aux_floats).
+size_t chunk_aux_floats(int C, int D);
 
 // Workspace carving (bytes) for the chunk forward / backward.
 size_t chunk_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states);

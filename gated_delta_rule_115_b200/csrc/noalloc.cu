@@ -67,10 +67,10 @@ extern "C" muir_status muir_chunk_fwd_noalloc(const muir_shape* shape, const voi
     const size_t need = muir_chunk_fwd_workspace(shape);
     if (need == 0)  // invalid shape: let the regular entry point report which check failed
         return muir_chunk_fwd(shape, q, k, v, g, e, w, gamma, S0, o, S_final, nullptr, nullptr,
-                              nullptr, 0, stream);
+                              nullptr, nullptr, 0, stream);
     if (need > kStaticScratchBytes) return MUIR_ERR_WORKSPACE;
     void* ws = nullptr;
     if (scratch_address(&ws) != cudaSuccess) return MUIR_ERR_CUDA;
-    return muir_chunk_fwd(shape, q, k, v, g, e, w, gamma, S0, o, S_final, nullptr, nullptr, ws,
-                          kStaticScratchBytes, stream);
+    return muir_chunk_fwd(shape, q, k, v, g, e, w, gamma, S0, o, S_final, nullptr, nullptr, nullptr,
+                          ws, kStaticScratchBytes, stream);
 }

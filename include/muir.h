@@ -81,6 +81,13 @@ muir_status muir_device_wait_status(void);
 size_t muir_chunk_fwd_workspace(const muir_shape* shape);
 size_t muir_chunk_bwd_workspace(const muir_shape* shape);
 
+/* Floats of the optional per-chunk intermediates muir_chunk_fwd can save for
+ * muir_chunk_bwd (`aux`; 0 for an invalid shape).  Per chunk, in the order of
+ * S_chunks ([B][H][T/C]): the four decay-masked C x C matrices L_A, L_K, M_QK,
+ * M_QA, the C/16 inverted 16 x 16 diagonal blocks of I + L_A, and Y (C x dv),
+ * each padded to a multiple of 64 floats.  Host-only. */
+size_t muir_chunk_aux_floats(const muir_shape* shape);
+
 /*
  * Chunkwise-parallel forward.  Same page, "Methodology": each chunk of C
  * tokens is written as a unit-lower-triangular system (WY/UT form); the
@@ -99,12 +106,16 @@ size_t muir_chunk_bwd_workspace(const muir_shape* shape);
  *   M_chunks          : [B][H][T/C][dk][dk] float32, may be NULL; receives the
  *                       chunk transitions M_n (S_{n+1} = M_n S_n + B_n), which
  *                       muir_chunk_bwd reuses together with S_chunks.
+ *   aux               : muir_chunk_aux_floats(shape) float32, may be NULL;
+ *                       receives the per-chunk intermediates muir_chunk_bwd
+ *                       reuses together with S_chunks (masked matrices, block
+ *                       inverses, Y) instead of recomputing them.
  */
 muir_status muir_chunk_fwd(const muir_shape* shape, const void* q, const void* k,
                            const void* v, const void* g, const void* e, const void* w,
                            const void* gamma, const float* S0, void* o, float* S_final,
-                           float* S_chunks, float* M_chunks, void* ws, size_t ws_bytes,
-                           void* stream);
+                           float* S_chunks, float* M_chunks, float* aux, void* ws,
+                           size_t ws_bytes, void* stream);
 
 /*
  * Backward of muir_chunk_fwd ("custom backward pass", same page,
@@ -116,13 +127,16 @@ muir_status muir_chunk_fwd(const muir_shape* shape, const void* q, const void* k
  *             muir_chunk_fwd with the same inputs wrote;
  *   M_chunks: NULL, or (with S_chunks) the transitions that forward wrote:
  *             then the per-chunk transitions are not recomputed;
+ *   aux:      NULL, or (with S_chunks) the intermediates that forward wrote;
+ *             aux without S_chunks is MUIR_ERR_INVALID_ARG;
  *   dq, dk, dg, de, dgamma [B][T][H][dk] and dv, dw [B][T][H][dv] are written
  *   in in_dtype; dS0 [B][H][dk][dv] float32 may be NULL.
  */
 muir_status muir_chunk_bwd(const muir_shape* shape, const void* q, const void* k,
                            const void* v, const void* g, const void* e, const void* w,
                            const void* gamma, const float* S0, const float* S_chunks,
-                           const float* M_chunks, const void* dO, const float* dS_final, void* dq, void* dk,
+                           const float* M_chunks, const float* aux, const void* dO,
+                           const float* dS_final, void* dq, void* dk,
                            void* dv, void* dg, void* de, void* dw, void* dgamma,
                            float* dS0, void* ws, size_t ws_bytes, void* stream);
 

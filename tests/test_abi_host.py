@@ -65,12 +65,12 @@ FAKE = ctypes.c_void_p(0x10000)  # 16-byte aligned, never dereferenced: checks f
 
 def _fwd(L, shp, **over):
     args = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, e=FAKE, w=FAKE, gamma=FAKE, S0=None, o=FAKE,
-                S_final=None, S_chunks=None, M_chunks=None, ws=None, ws_bytes=0)
+                S_final=None, S_chunks=None, M_chunks=None, aux=None, ws=None, ws_bytes=0)
     args.update(over)
     return L.muir_chunk_fwd(ctypes.byref(shp), args["q"], args["k"], args["v"], args["g"],
                             args["e"], args["w"], args["gamma"], args["S0"], args["o"],
-                            args["S_final"], args["S_chunks"], args["M_chunks"], args["ws"],
-                            ctypes.c_size_t(args["ws_bytes"]), None)
+                            args["S_final"], args["S_chunks"], args["M_chunks"], args["aux"],
+                            args["ws"], ctypes.c_size_t(args["ws_bytes"]), None)
 
 
 def test_chunk_fwd_rejects_bad_arguments(L):
@@ -84,7 +84,15 @@ def test_chunk_fwd_rejects_bad_arguments(L):
     assert _fwd(L, _shape(m), q=None) == 1                  # null input
     assert _fwd(L, _shape(m), o=ctypes.c_void_p(0x10004)) == 1  # misaligned output
     assert _fwd(L, _shape(m), M_chunks=ctypes.c_void_p(0x10002)) == 1  # misaligned saved array
-    assert L.muir_chunk_fwd(None, *([FAKE] * 13), ctypes.c_size_t(0), None) == 1
+    assert _fwd(L, _shape(m), aux=ctypes.c_void_p(0x10004)) == 1       # misaligned intermediates
+    assert L.muir_chunk_fwd(None, *([FAKE] * 14), ctypes.c_size_t(0), None) == 1
+
+
+def test_chunk_aux_size(L):
+    import gated_delta_rule_115_b200 as m
+    # per chunk: 4 C x C masked matrices, C x 16 block inverses, C x d for Y
+    assert L.muir_chunk_aux_floats(ctypes.byref(_shape(m))) == 1 * 2 * 4 * (4 * 64 * 64 + 64 * 16 + 64 * 64)
+    assert L.muir_chunk_aux_floats(ctypes.byref(_shape(m, chunk=48))) == 0
 
 
 def test_chunk_workspace_query(L):
@@ -100,12 +108,16 @@ def test_chunk_workspace_query(L):
 def test_chunk_bwd_rejects_bad_arguments(L):
     import gated_delta_rule_115_b200 as m
     shp = _shape(m, dk=32, dv=32)
-    args = [FAKE] * 7 + [None, None, None, FAKE, None] + [FAKE] * 7 + [None, None]
+    # q k v g e w gamma | S0 S_chunks M_chunks aux | dO dS_final | dq .. dgamma | dS0 ws
+    args = [FAKE] * 7 + [None, None, None, None, FAKE, None] + [FAKE] * 7 + [None, None]
     assert L.muir_chunk_bwd(ctypes.byref(shp), *args, ctypes.c_size_t(0), None) == 2
     shp = _shape(m)
     args2 = list(args)
-    args2[11] = ctypes.c_void_p(0x10008)  # misaligned dS_final
+    args2[12] = ctypes.c_void_p(0x10008)  # misaligned dS_final
     assert L.muir_chunk_bwd(ctypes.byref(shp), *args2, ctypes.c_size_t(0), None) == 1
+    args3 = list(args)
+    args3[10] = FAKE  # saved intermediates without the saved chunk states
+    assert L.muir_chunk_bwd(ctypes.byref(shp), *args3, ctypes.c_size_t(0), None) == 1
 
 
 def test_recurrent_step_rejects_bad_arguments(L):

@@ -163,6 +163,15 @@ def test_chunk_bwd_reuses_states(muir):
                        M_chunks=Mc2)
     for k in a:
         assert torch.equal(a[k], c[k]), k
+    # with the saved intermediates too, the backward skips the masked products,
+    # the block inverses and Y, and the result does not change
+    o3, S3, Sc3, Mc3, aux = muir.chunk_fwd(*[x[n] for n in NAMES], x["S0"], chunk=128,
+                                           return_saved=True, save_aux=True)
+    assert torch.equal(o3, o) and torch.equal(Sc3, Sc)
+    e = muir.chunk_bwd(*[x[n] for n in NAMES], x["S0"], x["dO"], chunk=128, S_chunks=Sc3,
+                       M_chunks=Mc3, aux=aux)
+    for k in a:
+        assert torch.equal(a[k], e[k]), k
 
 
 # ------------------------------------------------- span-dependent product paths
@@ -218,6 +227,13 @@ def test_chunk_bwd_span_paths(muir, oracle_mod, name, scale, every):
     print(f"bwd span {name}: " + " ".join(f"d{k} {v:.2e}" for k, v in errs.items()))
     for n, e in errs.items():
         assert e < TOL_BWD["bf16"], (n, e)
+    # the saved-intermediates path gives the same gradients on both product paths
+    o, S, Sc, Mc, aux = muir.chunk_fwd(*[d[n] for n in NAMES], d["S0"], chunk=128,
+                                       return_saved=True, save_aux=True)
+    gs = muir.chunk_bwd(*[d[n] for n in NAMES], d["S0"], d["dO"], dSf.cuda(), chunk=128,
+                        S_chunks=Sc, M_chunks=Mc, aux=aux)
+    for k in gr:
+        assert torch.equal(gr[k], gs[k]), k
 
 
 # ------------------------------------------------------------ full-size workloads
@@ -253,9 +269,10 @@ def test_full_size_fwd_bwd_long_context(muir, oracle_mod):
     from gated_delta_rule_115_b200 import inputs as I
     x = I.chunk_inputs(2)
     d = to_dev(x)
-    o, S, Sc, Mc = muir.chunk_fwd(*[d[n] for n in NAMES], d["S0"], chunk=128, return_saved=True)
+    o, S, Sc, Mc, aux = muir.chunk_fwd(*[d[n] for n in NAMES], d["S0"], chunk=128,
+                                       return_saved=True, save_aux=True)
     gr = muir.chunk_bwd(*[d[n] for n in NAMES], d["S0"], d["dO"], chunk=128, S_chunks=Sc,
-                        M_chunks=Mc)
+                        M_chunks=Mc, aux=aux)
     torch.cuda.synchronize()
     hs = [11]
     xs = sub(x, [0], hs)
