@@ -368,11 +368,12 @@ __device__ __forceinline__ bool use_panels(const Chunk<Tin, D>& c) {
 // Per-chunk operands of the decay-masked products; decides between the
 // single-pivot products (small decay span) and the 8-token panels.
 template <typename Tin, int D, int PASSES>
-__device__ __forceinline__ void masked_prep(Chunk<Tin, D>& c, bool with_q, bool bwd) {
+__device__ __forceinline__ void masked_prep(Chunk<Tin, D>& c, bool with_q, bool bwd,
+                                            bool pairs = true) {
     c.tame = false;
     if (!use_panels<Tin, D, PASSES>(c)) return;
     if (c.L.C >= 32) c.tame = chunk_tame(c);
-    if (c.tame) fast_prep<Tin, D>(c, with_q, bwd);
+    if (c.tame) fast_prep<Tin, D>(c, with_q, bwd, pairs);
     else panel_prep<Tin, D>(c, with_q);
 }
 
@@ -811,7 +812,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         const size_t Y = L.W[0], dR = L.W[1], dK = L.W[2], dQh = L.W[3], dA = L.W[4],
                      dU = L.W[5], dGam = L.W[6];
         prologue2(c);
-        masked_prep<Tin, D, PASSES>(c, true, true);  // path choice and gradient operands
+        masked_prep<Tin, D, PASSES>(c, true, true, !p.aux);  // path choice and gradient operands
         rows_prep<Tin, D, PASSES, 2>(c, R_KT | R_UU | R_DO | R_AB | R_KB);
         if (p.aux) {  // masked matrices, block inverses and Y the forward saved
             aux_copy(c, p.aux + (size_t)chunk * make_aux_lay(C, D).total, false, 63, Y);

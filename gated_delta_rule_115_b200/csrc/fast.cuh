@@ -39,9 +39,10 @@ __device__ __forceinline__ bool chunk_tame(const Chunk<Tin, D>& c) {
 }
 
 // Xo (K-major, 128-row tiles) for X in {K, Qh}, Zo (K-major, C rows) for Z in
-// {A, K}; with_mn also the MN-major copies (rows = channels) for the gradients.
+// {A, K} (with_k: the masked products run); with_mn the MN-major copies
+// (rows = channels) the gradients read.
 template <typename Tin, int D>
-__device__ void fast_prep(const Chunk<Tin, D>& c, bool with_q, bool with_mn) {
+__device__ void fast_prep(const Chunk<Tin, D>& c, bool with_q, bool with_mn, bool with_k = true) {
     const Lay& L = c.L;
     const int C = L.C;
     unsigned char* base = reinterpret_cast<unsigned char*>(c.s);
@@ -71,10 +72,12 @@ __device__ void fast_prep(const Chunk<Tin, D>& c, bool with_q, bool with_mn) {
         }
         const size_t ox = (size_t)(j >> 3) * 4096 + tc::kblk_off(t, j & 7);
         const size_t oz = (size_t)(j >> 3) * C * 32 + tc::kblk_off(t, j & 7);
-        *reinterpret_cast<float4*>(base + 4 * L.OXK + ox) = xk;
-        if (with_q) *reinterpret_cast<float4*>(base + 4 * L.OXQ + ox) = xq;
-        *reinterpret_cast<float4*>(base + 4 * L.OZA + oz) = za;
-        *reinterpret_cast<float4*>(base + 4 * L.OZK + oz) = zk;
+        if (with_k) {
+            *reinterpret_cast<float4*>(base + 4 * L.OXK + ox) = xk;
+            if (with_q) *reinterpret_cast<float4*>(base + 4 * L.OXQ + ox) = xq;
+            *reinterpret_cast<float4*>(base + 4 * L.OZA + oz) = za;
+            *reinterpret_cast<float4*>(base + 4 * L.OZK + oz) = zk;
+        }
         if (with_mn) {
             const size_t om = (size_t)(t >> 3) * 4096 + tc::mn_off(j, t & 7, 2048);
             *reinterpret_cast<float4*>(base + 4 * L.MXK + om) = xk;
