@@ -813,7 +813,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
                      dU = L.W[5], dGam = L.W[6];
         prologue2(c);
         masked_prep<Tin, D, PASSES>(c, true, true, !p.aux);  // path choice and gradient operands
-        rows_prep<Tin, D, PASSES, 2>(c, R_KT | R_UU | R_DO | R_AB | R_KB);
+        rows_prep<Tin, D, PASSES, 2>(c, (p.aux ? 0 : R_KT) | R_UU | R_DO | R_AB | R_KB);  // Kt: for Y
         if (p.aux) {  // masked matrices, block inverses and Y the forward saved
             aux_copy(c, p.aux + (size_t)chunk * make_aux_lay(C, D).total, false, 63, Y);
         } else {
