@@ -327,6 +327,30 @@ __device__ __forceinline__ void copy_block(unsigned char* blk, const Src& a, int
     }
 }
 
+// K-major segments of a whole 32-deep slab (four 8-deep K blocks, block kb of
+// the slab at blk + kb * R * 32) in one pass: a warp copies 64 contiguous bytes
+// of each of 8 rows (sixteen 16-byte pieces of a row cover the slab), the 8
+// lanes of a store phase take 8 different rows (distinct bank groups).
+// MN-major segments are left to copy_block.
+template <int R, class SRC>
+__device__ __forceinline__ void copy_slab_k(unsigned char* blk, const SRC& src, int k0, int rvalid,
+                                            int kmax) {
+    constexpr int PIECES = R * 8;  // 8 pieces of 16 bytes per row per slab
+    for (int idx = threadIdx.x; idx < PIECES; idx += blockDim.x) {
+        const int lane = idx & 31, w = idx >> 5;
+        const int r = (lane & 7) + 8 * (w % (R / 8));
+        const int pc = (lane >> 3) + 4 * (w / (R / 8));  // piece of the row: 0 .. 7
+        const int kb = pc >> 1, h = pc & 1;
+        const int k = k0 + 8 * kb;
+        if (k >= kmax) continue;
+        const Src a = src(k);
+        if (!a.p || a.mn) continue;
+        const bool ok = r < rvalid && k + 4 * h < kmax;
+        const float* g = a.p + (size_t)(ok ? r : 0) * a.ld + (ok ? (k - a.k0 + 4 * h) : 0);
+        cp_async16(smem_addr(blk + kb * R * 32 + (r >> 3) * 256 + h * 128 + (r & 7) * 16), g, ok);
+    }
+}
+
 template <int R, class F4>
 __device__ __forceinline__ void produce_block(unsigned char* blk, int k, int rvalid, int kmax,
                                               const F4& f4) {
@@ -401,13 +425,15 @@ __device__ void gemm_async(State& s, unsigned char* sbuf, int sbytes, int M, int
     for (int r0 = 0; r0 < nslab; r0 += nbuf) {
         const int nr = nslab - r0 < nbuf ? nslab - r0 : nbuf;
         for (int i = 0; i < nr; ++i) {
+            copy_slab_k<128>(blkA(i, 0), asrc, (r0 + i) * 32, M, K);
+            copy_slab_k<N>(blkB(i, 0), bsrc, (r0 + i) * 32, NB, K);
 #pragma unroll
             for (int ks = 0; ks < 4; ++ks) {
                 const int k = (r0 + i) * 32 + ks * 8;
                 if (k >= K) break;
                 const Src a = asrc(k), b = bsrc(k);
-                if (a.p) copy_block<128>(blkA(i, ks), a, k, M, K);
-                if (b.p) copy_block<N>(blkB(i, ks), b, k, NB, K);
+                if (a.p && a.mn) copy_block<128>(blkA(i, ks), a, k, M, K);
+                if (b.p && b.mn) copy_block<N>(blkB(i, ks), b, k, NB, K);
             }
             asm volatile("cp.async.commit_group;" ::: "memory");
         }
