@@ -55,8 +55,8 @@ DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 6 * 128 * 2 + 128 * 2  # S read+writ
 # DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel; valid only while the kernel source hash matches.
 NCU_TRAFFIC = {
-    # profiles/k_bwd_k_out_B1_H16_T8192_d128_C128.md: 7.315 GB for 131,072 token-heads
-    "k_bwd": {"bytes_per_token_head": 7.315279e9 / 131072, "source": "8cd42fba42fd8606"},
+    # profiles/k_bwd_k_out_B1_H16_T8192_d128_C128.md: 6.406 GB for 131,072 token-heads
+    "k_bwd": {"bytes_per_token_head": 6.4061e9 / 131072, "source": "ef4679f7a70d3c06"},
 }
 
 
