@@ -167,9 +167,9 @@ def chunk_fwd(q, k, v, g, e, w, gamma, S0=None, chunk=64, out_dtype=None,
     od = torch.bfloat16 if shp.out_dtype == MUIR_BF16 else torch.float32
     o = torch.empty(B, T, H, dv, dtype=od, device=q.device)
     S_final = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
-    Sc = (torch.empty(B, H, T // chunk, dk, dv, dtype=torch.float32, device=q.device)
+    Sc = (torch.empty(B, H, -(-T // chunk), dk, dv, dtype=torch.float32, device=q.device)
           if (return_chunk_states or return_saved) else None)
-    Mc = (torch.empty(B, H, T // chunk, dk, dk, dtype=torch.float32, device=q.device)
+    Mc = (torch.empty(B, H, -(-T // chunk), dk, dk, dtype=torch.float32, device=q.device)
           if return_saved else None)
     aux = None
     if return_saved and save_aux:

@@ -33,9 +33,8 @@ muir_status check_shape(const muir_shape* s) {
     if (s->dk != s->dv || (s->dk != 64 && s->dk != 128)) return MUIR_ERR_UNSUPPORTED;
     const int C = s->chunk;
     if (C != 16 && C != 32 && C != 64 && C != 128 && C != 256) return MUIR_ERR_UNSUPPORTED;
-    if (s->T % C != 0) return MUIR_ERR_UNSUPPORTED;
     // index arithmetic inside the kernels is 64-bit for tensors; keep counts in int range
-    if ((long long)s->B * s->H * (s->T / C) > (1LL << 30)) return MUIR_ERR_UNSUPPORTED;
+    if ((long long)s->B * s->H * ((s->T + C - 1) / C) > (1LL << 30)) return MUIR_ERR_UNSUPPORTED;
     return MUIR_OK;
 }
 
@@ -43,7 +42,7 @@ muir::ChunkProblem make_problem(const muir_shape* s, const void* q, const void* 
                                 const void* v, const void* g, const void* e, const void* w,
                                 const void* gamma) {
     muir::ChunkProblem P;
-    P.B = s->B; P.T = s->T; P.H = s->H; P.D = s->dk; P.C = s->chunk; P.N = s->T / s->chunk;
+    P.B = s->B; P.T = s->T; P.H = s->H; P.D = s->dk; P.C = s->chunk; P.N = (s->T + s->chunk - 1) / s->chunk;
     P.in_bf16 = s->in_dtype == MUIR_BF16;
     P.out_bf16 = s->out_dtype == MUIR_BF16;
     P.q = q; P.k = k; P.v = v; P.g = g; P.e = e; P.w = w; P.gamma = gamma;
@@ -82,7 +81,7 @@ muir_status muir_device_wait_status(void) {
 
 size_t muir_chunk_aux_floats(const muir_shape* s) {
     if (check_shape(s) != MUIR_OK) return 0;
-    return (size_t)s->B * s->H * (s->T / s->chunk) * muir::chunk_aux_floats(s->chunk, s->dk);
+    return (size_t)s->B * s->H * ((s->T + s->chunk - 1) / s->chunk) * muir::chunk_aux_floats(s->chunk, s->dk);
 }
 
 size_t muir_chunk_fwd_workspace(const muir_shape* s) {

@@ -9,18 +9,20 @@ namespace muir {
 size_t chunk_aux_floats(int C, int D) { return make_aux_lay(C, D).total; }
 
 size_t chunk_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states) {
-    const size_t nch = (size_t)B * H * (T / C), DD = (size_t)D * D;
+    const size_t nch = (size_t)B * H * ((T + C - 1) / C), DD = (size_t)D * D;
     size_t f = 2 * nch * DD;               // M, Bn
     if (!have_states) f += nch * DD;       // chunk-start states
     f += (size_t)num_slots((int)nch) * slot_floats(C, D);
+    f += tail_side_floats(B, T, H, D, C);
     return f * sizeof(float);
 }
 
 size_t chunk_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states) {
-    const size_t nch = (size_t)B * H * (T / C), DD = (size_t)D * D;
+    const size_t nch = (size_t)B * H * ((T + C - 1) / C), DD = (size_t)D * D;
     size_t f = 3 * nch * DD;               // M, Bn / B', dS at chunk ends
     if (!have_states) f += nch * DD;
     f += (size_t)num_slots((int)nch) * slot_floats(C, D);
+    f += tail_side_floats(B, T, H, D, C);
     return f * sizeof(float);
 }
 

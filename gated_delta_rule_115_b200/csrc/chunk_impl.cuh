@@ -109,6 +109,11 @@ struct KParams {
     float* scratch;
     size_t slot;             // floats per scratch slot
     float* aux;              // per-chunk saved intermediates or null
+    // chunk n of sequence bh sits at index bh * nstride + noff + n of the
+    // per-chunk arrays (S_chunks, dS_chunks, M, Bn, aux); a launch may cover
+    // only some chunks of each sequence (the padded last chunk of a ragged
+    // sequence runs as its own launch over side buffers)
+    int nstride, noff;
 };
 
 // Accessors of one chunk's inputs; row t of a [B,T,H,D] tensor.
@@ -119,6 +124,7 @@ struct Chunk {
     float* s;                // scratch slot
     Lay L;
     bool tame;               // decay span small enough for the single-pivot products
+    size_t sidx;             // index of the chunk in the per-chunk arrays
     __device__ float K(int t, int j) const { return ldf(k + base + t * rs + j); }
     __device__ float Qh(int t, int j) const {
         return ldf(gm + base + t * rs + j) * ldf(q + base + t * rs + j);
@@ -143,7 +149,8 @@ __device__ Chunk<Tin, D> make_chunk(const KParams& p, int chunk, float* slot) {
     c.dO = (const Tin*)p.dO;
     c.rs = (size_t)p.H * D;
     c.base = (((size_t)b * p.T + (size_t)n * p.C) * p.H + h) * D;
-    c.sbase = ((size_t)bh * p.N + n) * D * D;
+    c.sidx = (size_t)bh * p.nstride + p.noff + n;
+    c.sbase = c.sidx * D * D;
     c.s = slot;
     c.L = make_lay(CF ? CF : p.C, D);
     c.tame = false;
@@ -678,7 +685,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_out(KParams p) {
         __syncthreads();
         const float* S = p.S_chunks + c.sbase;
         compute_Y<Tin, D, PASSES>(tcx, c, S, L.W[0]);
-        if (p.aux) aux_copy(c, p.aux + (size_t)chunk * make_aux_lay(C, D).total, true, 63, L.W[0]);
+        if (p.aux) aux_copy(c, p.aux + c.sidx * make_aux_lay(C, D).total, true, 63, L.W[0]);
         Tout* o = (Tout*)p.o;
         const Fac<Tin, D> f = facs(c);
         const float* Y = s + L.W[0];
@@ -743,7 +750,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_bprep(KParams p)
         prologue2(c);
         rows_prep<Tin, D, PASSES>(c, R_KT | R_QT | R_DO);
         if (p.aux) {  // L_A, M_QA and the block inverses the forward saved
-            aux_copy(c, p.aux + (size_t)chunk * make_aux_lay(C, D).total, false, 1 | 8 | 16, 0);
+            aux_copy(c, p.aux + c.sidx * make_aux_lay(C, D).total, false, 1 | 8 | 16, 0);
         } else {
             masked_prep<Tin, D, PASSES>(c, true, false);
             masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
@@ -815,7 +822,7 @@ __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
         masked_prep<Tin, D, PASSES>(c, true, true, !p.aux);  // path choice and gradient operands
         rows_prep<Tin, D, PASSES, 2>(c, (p.aux ? 0 : R_KT) | R_UU | R_DO | R_AB | R_KB);  // Kt: for Y
         if (p.aux) {  // masked matrices, block inverses and Y the forward saved
-            aux_copy(c, p.aux + (size_t)chunk * make_aux_lay(C, D).total, false, 63, Y);
+            aux_copy(c, p.aux + c.sidx * make_aux_lay(C, D).total, false, 63, Y);
         } else {
             masked_pair<Tin, D, PASSES, OP_K, OP_A, OP_K>(c, tcx, sm, L.LA, L.LK, false, false);
             masked_pair<Tin, D, PASSES, OP_Q, OP_K, OP_A>(c, tcx, sm, L.MQK, L.MQA, true, true);
@@ -1208,6 +1215,66 @@ inline int num_slots(int nch) { return nch < kMaxSlots ? nch : kMaxSlots; }
 
 inline size_t slot_floats(int C, int D) { return make_lay(C, D).total; }
 
+// Side buffers of a ragged last chunk, counted in floats (4-byte elements
+// bound both dtypes): 8 input tensors and 7 output tensors of [B*H][C][D].
+inline size_t tail_side_floats(int B, int T, int H, int D, int C) {
+    return T % C ? (size_t)15 * B * H * C * D : 0;
+}
+
+// A ragged problem (T % C != 0) runs its per-chunk kernels as two launches:
+// `main` over the N - 1 whole chunks of every sequence, and `tail` over the
+// last chunk of every sequence, read from a zero-padded side copy laid out
+// as a problem of B*H sequences, one head, C tokens (row stride D).  Both
+// address the same per-chunk arrays (nstride = N).  Staging copies the k
+// input tensors (dO included in the backward) into the side buffer and points
+// `tail` at it; `tail.o` / the gradient pointers go to the output side buffer.
+struct Launches {
+    KParams main, tail;
+    bool ragged;
+    size_t E;         // elements per side tensor, B*H*C*D
+    char* side_out;   // output side buffer (7 tensors of E elements)
+};
+
+template <typename Tin, int D>
+cudaError_t stage_tail(Launches& L, const KParams& kp, const void* const* in, int k, float* side,
+                       cudaStream_t st) {
+    L.main = kp;
+    L.main.nstride = kp.N;
+    L.main.noff = 0;
+    L.ragged = kp.T % kp.C != 0;
+    if (!L.ragged) return cudaSuccess;
+    L.main.N = kp.N - 1;
+    L.E = (size_t)kp.B * kp.H * kp.C * D;
+    Tin* tin = reinterpret_cast<Tin*>(side);
+    L.side_out = reinterpret_cast<char*>(side + 8 * L.E);
+    KParams& t = L.tail;
+    t = L.main;
+    t.B = kp.B * kp.H; t.H = 1; t.T = kp.C; t.N = 1; t.noff = kp.N - 1;
+    const void** dst[8] = {&t.q, &t.k, &t.v, &t.g, &t.e, &t.w, &t.gamma, &t.dO};
+    TailCopy io = {};
+    io.n = k;
+    for (int i = 0; i < k; ++i) {
+        io.src[i] = in[i];
+        io.dst[i] = tin + i * L.E;
+        *dst[i] = tin + i * L.E;
+    }
+    return tail_gather(io, kp.B, kp.H, kp.T, kp.C, D, (int)sizeof(Tin), st);
+}
+
+// Copy the tail rows of k output tensors (esize bytes per element) from the
+// output side buffer to their token-major destinations.
+inline cudaError_t unstage_tail(const Launches& L, const KParams& kp, void* const* out, int k,
+                                int D, int esize, cudaStream_t st) {
+    if (!L.ragged) return cudaSuccess;
+    TailCopy io = {};
+    io.n = k;
+    for (int i = 0; i < k; ++i) {
+        io.src[i] = L.side_out + i * L.E * esize;
+        io.dst[i] = out[i];
+    }
+    return tail_scatter(io, kp.B, kp.H, kp.T, kp.C, D, esize, st);
+}
+
 // Persistent grid of a chunk kernel: one CTA per resident slot (SM count x
 // CTAs that fit per SM by registers, shared memory and threads, from the
 // kernel's attributes), at most one per scratch slot.  Call after the
@@ -1280,18 +1347,31 @@ cudaError_t fwd_impl(const ChunkProblem& P, const float* S0, void* o, float* S_f
     const int dyn = dyn_bytes<D, PASSES>(P.C, false);
     cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn, dyn_bytes<D, PASSES>(P.C, true));
     if (err != cudaSuccess) return err;
-    const int grid = persistent_grid(k_intra<Tin, D, PASSES, CF>, nch, dyn);
-    const int grid_o = persistent_grid(k_out<Tin, float, D, PASSES, CF>, nch, dyn);
-    MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
-    err = cudaGetLastError();
+    const void* in[7] = {P.q, P.k, P.v, P.g, P.e, P.w, P.gamma};
+    Launches Ls;
+    err = stage_tail<Tin, D>(Ls, kp, in, 7, f + (size_t)num_slots(nch) * kp.slot, st);
     if (err != cudaSuccess) return err;
+    if (Ls.ragged) Ls.tail.o = Ls.side_out;
+    // per-chunk kernel over the whole chunks, then over the padded last chunks
+    auto each = [&](auto kernel, const char* name) -> cudaError_t {
+        for (int part = 0; part < 2; ++part) {
+            const KParams& q = part ? Ls.tail : Ls.main;
+            if ((part && !Ls.ragged) || q.N == 0) continue;
+            const int grid = persistent_grid(kernel, q.B * q.H * q.N, dyn);
+            MUIR_TIMED(name, st, kernel<<<grid, kThreads, dyn, st>>>(q));
+            const cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    };
+    if ((err = each(k_intra<Tin, D, PASSES, CF>, "k_intra")) != cudaSuccess) return err;
     err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, S_final, st);
     if (err != cudaSuccess) return err;
-    if (P.out_bf16)
-        MUIR_TIMED("k_out", st, k_out<Tin, __nv_bfloat16, D, PASSES, CF><<<grid_o, kThreads, dyn, st>>>(kp));
-    else
-        MUIR_TIMED("k_out", st, k_out<Tin, float, D, PASSES, CF><<<grid_o, kThreads, dyn, st>>>(kp));
-    return cudaGetLastError();
+    if (P.out_bf16) err = each(k_out<Tin, __nv_bfloat16, D, PASSES, CF>, "k_out");
+    else err = each(k_out<Tin, float, D, PASSES, CF>, "k_out");
+    if (err != cudaSuccess) return err;
+    void* out[1] = {o};
+    return unstage_tail(Ls, kp, out, 1, D, P.out_bf16 ? 2 : 4, st);
 }
 
 template <typename Tin, int D, int PASSES, int CF>
@@ -1321,27 +1401,41 @@ cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chun
     const int dyn = dyn_bytes<D, PASSES>(P.C, false), dyn_b = dyn_bytes<D, PASSES>(P.C, true);
     cudaError_t err = set_smem_attrs<Tin, D, PASSES, CF>(dyn, dyn_b);
     if (err != cudaSuccess) return err;
-    const int grid = persistent_grid(k_intra<Tin, D, PASSES, CF>, nch, dyn);
-    const int grid_p = persistent_grid(k_bprep<Tin, D, PASSES, CF>, nch, dyn);
-    const int grid_b = persistent_grid(k_bwd<Tin, D, PASSES, CF>, nch, dyn_b);
     const bool have_M = M_chunks != nullptr && !recompute;
-    if (have_M) {
-        kp.M = const_cast<float*>(M_chunks);  // the forward's transitions: nothing to recompute
-    } else {
-        MUIR_TIMED("k_intra", st, k_intra<Tin, D, PASSES, CF><<<grid, kThreads, dyn, st>>>(kp));
-        err = cudaGetLastError();
-        if (err != cudaSuccess) return err;
+    if (have_M) kp.M = const_cast<float*>(M_chunks);  // the forward's transitions: nothing to recompute
+    const void* in[8] = {P.q, P.k, P.v, P.g, P.e, P.w, P.gamma, dO};
+    Launches Ls;
+    err = stage_tail<Tin, D>(Ls, kp, in, 8, f + (size_t)num_slots(nch) * kp.slot, st);
+    if (err != cudaSuccess) return err;
+    if (Ls.ragged) {
+        void** g[7] = {&Ls.tail.dq, &Ls.tail.dk, &Ls.tail.dv, &Ls.tail.dg, &Ls.tail.de,
+                       &Ls.tail.dw, &Ls.tail.dgamma};
+        for (int i = 0; i < 7; ++i) *g[i] = Ls.side_out + i * Ls.E * sizeof(Tin);
     }
+    // per-chunk kernel over the whole chunks, then over the padded last chunks
+    auto each = [&](auto kernel, const char* name, int smem) -> cudaError_t {
+        for (int part = 0; part < 2; ++part) {
+            const KParams& q = part ? Ls.tail : Ls.main;
+            if ((part && !Ls.ragged) || q.N == 0) continue;
+            const int grid = persistent_grid(kernel, q.B * q.H * q.N, smem);
+            MUIR_TIMED(name, st, kernel<<<grid, kThreads, smem, st>>>(q));
+            const cudaError_t e = cudaGetLastError();
+            if (e != cudaSuccess) return e;
+        }
+        return cudaSuccess;
+    };
+    if (!have_M && (err = each(k_intra<Tin, D, PASSES, CF>, "k_intra", dyn)) != cudaSuccess)
+        return err;
     if (recompute) {
         err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, nullptr, st);
         if (err != cudaSuccess) return err;
     }
-    MUIR_TIMED("k_bprep", st, k_bprep<Tin, D, PASSES, CF><<<grid_p, kThreads, dyn, st>>>(kp));
-    if ((err = cudaGetLastError()) != cudaSuccess) return err;
+    if ((err = each(k_bprep<Tin, D, PASSES, CF>, "k_bprep", dyn)) != cudaSuccess) return err;
     err = launch_chain<D, PASSES, true>(BH, P.N, kp.M, kp.Bn, dS_final, dSc, dS0, st);
     if (err != cudaSuccess) return err;
-    MUIR_TIMED("k_bwd", st, k_bwd<Tin, D, PASSES, CF><<<grid_b, kThreads, dyn_b, st>>>(kp));
-    return cudaGetLastError();
+    if ((err = each(k_bwd<Tin, D, PASSES, CF>, "k_bwd", dyn_b)) != cudaSuccess) return err;
+    void* out[7] = {dq, dk, dv, dg, de, dw, dgamma};
+    return unstage_tail(Ls, kp, out, 7, D, (int)sizeof(Tin), st);
 }
 
 }  // namespace muir

@@ -14,11 +14,25 @@ cudaError_t launch_decode(int B, int H, int D, bool in_bf16, bool out_bf16, cons
 // Problem description shared by the chunk kernels.
 struct ChunkProblem {
     int B, T, H, D, C;     // D = dk = dv
-    int N;                 // chunks per sequence, T / C
+    int N;                 // chunks per sequence, ceil(T / C); the last one may be ragged
     bool in_bf16, out_bf16;
     const void *q, *k, *v, *g, *e, *w, *gamma;
     float* aux;            // per-chunk saved intermediates (forward: written; backward: read) or null
 };
+
+// Up to eight tensors moved between token-major [B][T][H][D] rows of the
+// ragged last chunk and a side buffer [B*H][C][D] (tail.cu).
+struct TailCopy {
+    const void* src[8];
+    void* dst[8];
+    int n;
+};
+// token-major -> side buffer (rows past the tail zeroed) / side -> token-major
+// (tail rows only); esize = bytes per element.
+cudaError_t tail_gather(const TailCopy& io, int B, int H, int T, int C, int D, int esize,
+                        cudaStream_t st);
+cudaError_t tail_scatter(const TailCopy& io, int B, int H, int T, int C, int D, int esize,
+                         cudaStream_t st);
 
 // Floats per chunk of the saved intermediates (muir_chunk_aux_floats).
 size_t chunk_aux_floats(int C, int D);

@@ -28,10 +28,15 @@
  * - Argument checks run on the host before anything is enqueued; a failed
  *   check returns MUIR_ERR_INVALID_ARG or MUIR_ERR_UNSUPPORTED and enqueues
  *   nothing.  A launch failure returns MUIR_ERR_CUDA.
- * - Supported: dk == dv in {64, 128}; chunk in {16, 32, 64, 128, 256};
- *   T % chunk == 0 (a ragged tail returns MUIR_ERR_UNSUPPORTED); a device of
- *   compute capability 10.x.  Inside the kernels g is clamped at -20 per
- *   token (exp(-20) ~ 2e-9; a row decayed that hard is already erased).
+ * - Supported: dk == dv in {64, 128}; chunk in {16, 32, 64, 128, 256}; any
+ *   T >= 1; a device of compute capability 10.x.  Inside the kernels g is
+ *   clamped at -20 per token (exp(-20) ~ 2e-9; a row decayed that hard is
+ *   already erased).
+ * - Ragged tails: N = ceil(T / chunk) chunks per sequence.  When T % chunk
+ *   != 0 the last chunk's rows are staged in the workspace, padded with zero
+ *   tokens (q = k = v = e = w = gamma = 0, g = 0: the state passes through
+ *   unchanged and o = 0), processed as a full chunk, and copied back; the
+ *   workspace queries include those side buffers.
  * - dtype MUIR_BF16 means bfloat16 inputs; MUIR_FP32 means float32 inputs.
  *   Internal arithmetic is float32 with tensor-core TF32 products (three TF32
  *   passes for float32 inputs).  out_dtype selects o's storage.
@@ -48,7 +53,7 @@ extern "C" {
 typedef enum {
     MUIR_OK = 0,
     MUIR_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, bad size */
-    MUIR_ERR_UNSUPPORTED = 2,   /* valid but not implemented (head dim, chunk, tail, device) */
+    MUIR_ERR_UNSUPPORTED = 2,   /* valid but not implemented (head dim, chunk, device) */
     MUIR_ERR_WORKSPACE = 3,     /* ws too small or NULL with ws_bytes > 0 */
     MUIR_ERR_CUDA = 4,          /* a CUDA runtime call or launch failed */
     MUIR_ERR_DEVICE_TIMEOUT = 5 /* a bounded device-side wait expired */
@@ -83,7 +88,7 @@ size_t muir_chunk_bwd_workspace(const muir_shape* shape);
 
 /* Floats of the optional per-chunk intermediates muir_chunk_fwd can save for
  * muir_chunk_bwd (`aux`; 0 for an invalid shape).  Per chunk, in the order of
- * S_chunks ([B][H][T/C]): the four decay-masked C x C matrices L_A, L_K, M_QK,
+ * S_chunks ([B][H][N], N = ceil(T/C)): the four decay-masked C x C matrices L_A, L_K, M_QK,
  * M_QA, the C/16 inverted 16 x 16 diagonal blocks of I + L_A, and Y (C x dv),
  * each padded to a multiple of 64 floats.  Host-only. */
 size_t muir_chunk_aux_floats(const muir_shape* shape);
@@ -100,10 +105,10 @@ size_t muir_chunk_aux_floats(const muir_shape* shape);
  *   S0                : [B][H][dk][dv]  float32, NULL = zero initial state
  *   o                 : [B][T][H][dv]   out_dtype (written)
  *   S_final           : [B][H][dk][dv]  float32, may be NULL (written)
- *   S_chunks          : [B][H][T/C][dk][dv] float32, may be NULL; receives the
+ *   S_chunks          : [B][H][N][dk][dv] float32 (N = ceil(T/C)), may be NULL; receives the
  *                       state at the start of every chunk, which
  *                       muir_chunk_bwd can reuse instead of recomputing it.
- *   M_chunks          : [B][H][T/C][dk][dk] float32, may be NULL; receives the
+ *   M_chunks          : [B][H][N][dk][dk] float32, may be NULL; receives the
  *                       chunk transitions M_n (S_{n+1} = M_n S_n + B_n), which
  *                       muir_chunk_bwd reuses together with S_chunks.
  *   aux               : muir_chunk_aux_floats(shape) float32, may be NULL;

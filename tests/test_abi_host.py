@@ -78,7 +78,8 @@ def test_chunk_fwd_rejects_bad_arguments(L):
     assert _fwd(L, _shape(m, dk=96, dv=96)) == 2            # head dim
     assert _fwd(L, _shape(m, dk=64, dv=128)) == 2           # dk != dv
     assert _fwd(L, _shape(m, chunk=48)) == 2                # chunk size
-    assert _fwd(L, _shape(m, T=250)) == 2                   # ragged tail
+    assert _fwd(L, _shape(m, T=0)) == 1                     # empty sequence
+    assert _fwd(L, _shape(m, T=250)) == 3                   # ragged tail: valid, needs workspace
     assert _fwd(L, _shape(m, B=0)) == 1
     assert _fwd(L, _shape(m, in_dtype=7)) == 1
     assert _fwd(L, _shape(m), q=None) == 1                  # null input
@@ -93,12 +94,19 @@ def test_chunk_aux_size(L):
     # per chunk: 4 C x C masked matrices, C x 16 block inverses, C x d for Y
     assert L.muir_chunk_aux_floats(ctypes.byref(_shape(m))) == 1 * 2 * 4 * (4 * 64 * 64 + 64 * 16 + 64 * 64)
     assert L.muir_chunk_aux_floats(ctypes.byref(_shape(m, chunk=48))) == 0
+    # ceil(T / C) chunks with a ragged tail
+    assert L.muir_chunk_aux_floats(ctypes.byref(_shape(m, T=250))) == \
+        L.muir_chunk_aux_floats(ctypes.byref(_shape(m)))
 
 
 def test_chunk_workspace_query(L):
     import gated_delta_rule_115_b200 as m
     assert L.muir_chunk_fwd_workspace(ctypes.byref(_shape(m, chunk=48))) == 0
-    assert L.muir_chunk_bwd_workspace(ctypes.byref(_shape(m, T=100))) == 0
+    assert L.muir_chunk_bwd_workspace(ctypes.byref(_shape(m, T=0))) == 0
+    # a ragged tail adds the side buffers of the padded last chunk
+    # (8 inputs + 7 outputs of B*H*C*d elements, 4 bytes each)
+    for q in (L.muir_chunk_fwd_workspace, L.muir_chunk_bwd_workspace):
+        assert q(ctypes.byref(_shape(m, T=250))) == q(ctypes.byref(_shape(m))) + 15 * 2 * 64 * 64 * 4
     need = L.muir_chunk_fwd_workspace(ctypes.byref(_shape(m)))
     if need > 0:
         assert _fwd(L, _shape(m), ws=FAKE, ws_bytes=need - 1) == 3

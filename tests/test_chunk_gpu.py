@@ -236,6 +236,88 @@ def test_chunk_bwd_span_paths(muir, oracle_mod, name, scale, every):
         assert torch.equal(gr[k], gs[k]), k
 
 
+# ------------------------------------------------------------ ragged tails
+
+# T not a multiple of C: the last chunk holds the remaining tokens (down to a
+# single one, and T < C where the whole sequence is one partial chunk).
+RAGGED_FWD = [
+    # (wid, overrides, chunk)
+    (0, dict(T=250), 64),                                         # fp32 d=64, tail 58
+    (0, dict(dtype="bf16", T=200, dk=128, dv=128, s0_std=1.0), 128),
+    (2, dict(B=2, H=2, T=300), 128),                              # batch stride, tail 44
+    (0, dict(dtype="fp32", T=37, dk=128, dv=128, s0_std=1.0), 64),  # T < C
+    (0, dict(dtype="bf16", T=1, s0_std=1.0), 16),                 # one token
+    (3, dict(B=1, H=2, T=700), 256),                              # tail 188
+    (0, dict(dtype="fp32", T=130, dk=128, dv=128, s0_std=2.0), 32),  # tail 2
+]
+
+
+@pytest.mark.parametrize("wid,over,C", RAGGED_FWD)
+def test_chunk_fwd_ragged_tail(muir, oracle_mod, wid, over, C):
+    from gated_delta_rule_115_b200 import inputs as I
+    x = I.chunk_inputs(wid, **over)
+    dt = over.get("dtype", I.WORKLOADS[wid].dtype)
+    d = to_dev(x)
+    o, S, Sc = muir.chunk_fwd(*[d[n] for n in NAMES], d["S0"], chunk=C, out_dtype=torch.float32,
+                              return_chunk_states=True)
+    ro, rS, rSc = oracle_mod.chunk_fwd(*[x[n] for n in NAMES], S0=x["S0"], chunk=C)
+    torch.cuda.synchronize()
+    assert Sc.shape[2] == -(-x["q"].shape[1] // C)
+    eo, eS, eC = nmax(o, ro), nmax(S, rS), nmax(Sc, rSc)
+    print(f"ragged fwd wid={wid} C={C} {dt}: o {eo:.2e} S {eS:.2e} chunk states {eC:.2e}")
+    assert eo < TOL_FWD[dt] and eS < TOL_FWD[dt] and eC < TOL_FWD[dt]
+
+
+RAGGED_BWD = [
+    (0, dict(T=250, s0_std=1.0), 64),
+    (2, dict(B=2, H=2, T=300), 128),
+    (0, dict(dtype="bf16", T=37, dk=128, dv=128, s0_std=1.0), 64),
+    (3, dict(B=1, H=1, T=600, with_dO=True), 256),
+    (0, dict(dtype="fp32", T=130, dk=128, dv=128, s0_std=1.0), 32),
+]
+
+
+@pytest.mark.parametrize("wid,over,C", RAGGED_BWD)
+def test_chunk_bwd_ragged_tail(muir, oracle_mod, wid, over, C):
+    from gated_delta_rule_115_b200 import inputs as I
+    x = I.chunk_inputs(wid, **over)
+    dt = over.get("dtype", I.WORKLOADS[wid].dtype)
+    B, T, H, dk = x["q"].shape
+    dSf = torch.randn(B, H, dk, dk, generator=torch.Generator().manual_seed(98))
+    d = to_dev(x)
+    gr = muir.chunk_bwd(*[d[n] for n in NAMES], d["S0"], d["dO"], dSf.cuda(), chunk=C)
+    rg = oracle_mod.bwd(*[x[n] for n in NAMES], S0=x["S0"], dO=x["dO"], dS_final=dSf)
+    torch.cuda.synchronize()
+    errs = {n: nmax(gr["d" + n], rg["d" + n]) for n in NAMES}
+    errs["S0"] = nmax(gr["dS0"], rg["dS0"])
+    print(f"ragged bwd wid={wid} C={C} {dt}: " + " ".join(f"d{k} {v:.2e}" for k, v in errs.items()))
+    for n, e in errs.items():
+        assert e < TOL_BWD[dt], (n, e)
+
+
+def test_ragged_tail_reuses_saved(muir):
+    """With a ragged tail, the backward from the forward's saved states,
+    transitions and intermediates equals the recomputing backward bit for bit,
+    and the forward equals the one over the sequences zero-padded by hand."""
+    from gated_delta_rule_115_b200 import inputs as I
+    x = to_dev(I.chunk_inputs(2, B=2, H=2, T=333, s0_std=1.0))
+    a = muir.chunk_bwd(*[x[n] for n in NAMES], x["S0"], x["dO"], chunk=128)
+    o, S, Sc, Mc, aux = muir.chunk_fwd(*[x[n] for n in NAMES], x["S0"], chunk=128,
+                                       return_saved=True, save_aux=True)
+    b = muir.chunk_bwd(*[x[n] for n in NAMES], x["S0"], x["dO"], chunk=128, S_chunks=Sc,
+                       M_chunks=Mc, aux=aux)
+    for k in a:
+        assert torch.equal(a[k], b[k]), k
+    # the same sequences padded by hand to 384 tokens with zero tokens give the
+    # same o on the real rows and the same final state
+    pad = {n: (torch.cat([x[n], torch.zeros_like(x[n][:, :51])], 1) if x[n].dim() == 4 and n != "S0"
+               else x[n]) for n in NAMES + ["S0"]}
+    op, Sp = muir.chunk_fwd(*[pad[n] for n in NAMES], pad["S0"], chunk=128)
+    torch.cuda.synchronize()
+    assert torch.equal(op[:, :333], o)
+    assert torch.equal(Sp, S)
+
+
 # ------------------------------------------------------------ full-size workloads
 
 FULL = [(1, 64), (2, 128), (3, 256)]
