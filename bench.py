@@ -5,7 +5,8 @@ One step = the whole hot path over one batch of the long-context workload
 (B=1, H=16, T=32768, dk=dv=128, chunk 128, bf16 inputs): ``muir_chunk_fwd``
 (saving chunk states) followed by ``muir_chunk_bwd`` with a random upstream
 gradient.  The streaming-decode step (B=64, H=16, d=128, float32 state) is
-measured in the same run and reported under ``"decode"``.
+measured in the same run and reported under ``"decode"``, the q/k feature
+prologue (forward and backward) under ``"qk_prologue"``.
 
 Usage::
 
@@ -325,6 +326,7 @@ def gpu_arm(args, rank, world, local):
         out["e2e"] = e2e_measure(muir, x, W, C, dev, ws_f, ws_b, max(1, min(args.steps, 3)), world)
     if not args.no_decode:
         out["decode"] = decode_measure(muir, I, dev, peaks)
+        out["qk_prologue"] = qk_measure(muir, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = len(os.sched_getaffinity(0))
         v, desc, dt = oracle_sample(args.cpu_seconds, threads)
@@ -478,6 +480,46 @@ def decode_measure(muir, I, dev, peaks, steps=50):
         "bytes_per_step": byts,
         "graph_replay_ms_per_step": ms_g, "graph_replay_gbs_l2_resident": byts / (ms_g / 1e3) / 1e9,
         "note": "graph replay keeps the 64 MiB state in L2; the flushed number is the HBM one",
+    }
+
+
+def qk_measure(muir, dev, peaks, steps=20):
+    """q/k prologue (SiLU + unit L2 norm per row, forward and backward) over
+    the long-context workload's q and k: 2 x 524,288 rows of 128 bf16.  Each
+    timed call moves 268 MB (forward: read + write) or 403 MB (backward: x and
+    dy read, dx written), beyond the 126 MB L2, with a 256 MB flush between
+    calls.  GB/s from those algorithmic bytes."""
+    import torch
+    g = torch.Generator(device=dev).manual_seed(11)
+    x = torch.randn(2, 32768, 16, 128, generator=g, device=dev).to(torch.bfloat16)
+    dy = torch.randn(2, 32768, 16, 128, generator=g, device=dev).to(torch.bfloat16)
+    y, dx = torch.empty_like(x), torch.empty_like(x)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    st = torch.cuda.current_stream(dev)
+    nbytes = x.numel() * 2
+
+    def timed(fn):
+        for _ in range(3):
+            fn()
+        ts = []
+        for _ in range(steps):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(st)
+            fn()
+            b.record(st)
+            b.synchronize()
+            ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    ms_f = timed(lambda: muir.qk_prologue(x, out=y))
+    ms_b = timed(lambda: muir.qk_prologue_bwd(x, dy, out=dx))
+    gf = 2 * nbytes / (ms_f / 1e3) / 1e9
+    gb = 3 * nbytes / (ms_b / 1e3) / 1e9
+    return {
+        "workload": "q and k of B=1 H=16 T=32768 d=128, bf16 (1,048,576 rows)",
+        "fwd_ms": ms_f, "fwd_gbs": gf, "fwd_hbm_frac": gf / peaks["hbm_gbs"],
+        "bwd_ms": ms_b, "bwd_gbs": gb, "bwd_hbm_frac": gb / peaks["hbm_gbs"],
     }
 
 

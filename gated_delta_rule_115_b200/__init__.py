@@ -22,8 +22,9 @@ import os
 import torch
 
 __all__ = [
-    "MuirError", "lib", "chunk_fwd", "chunk_bwd", "recurrent_step", "fwd_workspace_bytes",
-    "bwd_workspace_bytes", "MuirChunkFunction", "LIB_PATH",
+    "MuirError", "lib", "chunk_fwd", "chunk_bwd", "recurrent_step", "qk_prologue",
+    "qk_prologue_bwd", "fwd_workspace_bytes", "bwd_workspace_bytes", "MuirChunkFunction",
+    "LIB_PATH",
 ]
 
 LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libmuir.so")
@@ -74,6 +75,10 @@ def lib():
         L.muir_chunk_bwd.restype = I
         L.muir_recurrent_step.argtypes = [I, I, I, I, I, I] + [P] * 7 + [I, P, P, P]
         L.muir_recurrent_step.restype = I
+        L.muir_qk_prologue.argtypes = [ctypes.c_longlong, I, I, P, P, P]
+        L.muir_qk_prologue.restype = I
+        L.muir_qk_prologue_bwd.argtypes = [ctypes.c_longlong, I, I, P, P, P, P]
+        L.muir_qk_prologue_bwd.restype = I
         L.muir_chunk_fwd_noalloc.argtypes = [SP] + [P] * 10 + [P]
         L.muir_chunk_fwd_noalloc.restype = I
         L.muir_profile_enable.argtypes = [I]
@@ -228,6 +233,30 @@ def recurrent_step(q, k, v, g, e, w, gamma, S, gamma_static=False, out_dtype=Non
                                _ptr(S), _ptr(o), _stream(q.device))
     _check("muir_recurrent_step", rc)
     return o
+
+
+def qk_prologue(x, out=None):
+    """``SiLU(x) / max(||SiLU(x)||, 1e-12)`` over the last dim (64 or 128) of a
+    contiguous bf16/float32 tensor; ``out`` may be ``x`` (in place)."""
+    L = lib()
+    if out is None:
+        out = torch.empty_like(x)
+    d = x.shape[-1]
+    rc = L.muir_qk_prologue(x.numel() // d, d, _dt(x), _ptr(x), _ptr(out), _stream(x.device))
+    _check("muir_qk_prologue", rc)
+    return out
+
+
+def qk_prologue_bwd(x, dy, out=None):
+    """Gradient of :func:`qk_prologue` with respect to ``x`` for upstream ``dy``."""
+    L = lib()
+    if out is None:
+        out = torch.empty_like(x)
+    d = x.shape[-1]
+    rc = L.muir_qk_prologue_bwd(x.numel() // d, d, _dt(x), _ptr(x), _ptr(dy), _ptr(out),
+                                _stream(x.device))
+    _check("muir_qk_prologue_bwd", rc)
+    return out
 
 
 class MuirChunkFunction(torch.autograd.Function):

@@ -160,4 +160,28 @@ muir_status muir_recurrent_step(int B, int H, int dk, int dv, muir_dtype dtype,
                                          static_cast<cudaStream_t>(stream)));
 }
 
+muir_status muir_qk_prologue(long long rows, int d, muir_dtype dtype, const void* x, void* y,
+                             void* stream) {
+    if (rows < 0 || !ok_dtype(dtype)) return MUIR_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return MUIR_ERR_UNSUPPORTED;
+    if (rows == 0) return MUIR_OK;
+    if (!ok_ptr(x) || !ok_ptr(y)) return MUIR_ERR_INVALID_ARG;
+    muir_status st = check_device();
+    if (st != MUIR_OK) return st;
+    return from_cuda(muir::launch_qk_prologue(rows, d, dtype == MUIR_BF16, x, nullptr, y, false,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
+muir_status muir_qk_prologue_bwd(long long rows, int d, muir_dtype dtype, const void* x,
+                                 const void* dy, void* dx, void* stream) {
+    if (rows < 0 || !ok_dtype(dtype)) return MUIR_ERR_INVALID_ARG;
+    if (d != 64 && d != 128) return MUIR_ERR_UNSUPPORTED;
+    if (rows == 0) return MUIR_OK;
+    if (!ok_ptr(x) || !ok_ptr(dy) || !ok_ptr(dx)) return MUIR_ERR_INVALID_ARG;
+    muir_status st = check_device();
+    if (st != MUIR_OK) return st;
+    return from_cuda(muir::launch_qk_prologue(rows, d, dtype == MUIR_BF16, x, dy, dx, true,
+                                              static_cast<cudaStream_t>(stream)));
+}
+
 }  // extern "C"

@@ -11,6 +11,10 @@ cudaError_t launch_decode(int B, int H, int D, bool in_bf16, bool out_bf16, cons
                           const void* w, const void* gamma, int gamma_static, float* S,
                           void* o, cudaStream_t st);
 
+// q/k feature prologue y = SiLU(x) / ||SiLU(x)|| per row of d (bwd: dx from x, dy).
+cudaError_t launch_qk_prologue(long long rows, int d, bool bf16, const void* x, const void* dy,
+                               void* out, bool bwd, cudaStream_t st);
+
 // Problem description shared by the chunk kernels.
 struct ChunkProblem {
     int B, T, H, D, C;     // D = dk = dv

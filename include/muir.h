@@ -185,6 +185,36 @@ muir_status muir_recurrent_step(int B, int H, int dk, int dv, muir_dtype dtype,
                                 const void* gamma, int gamma_static, float* S, void* o,
                                 void* stream);
 
+/*
+ * q/k feature prologue (same page, "Methodology" and fig. 3(b): the query and
+ * key pathways end in SiLU, and q and k are unit-normalised per head before
+ * the recurrence).  Per row of d channels (one token of one head):
+ *
+ *     y = SiLU(x) / max(||SiLU(x)||_2, 1e-12),   SiLU(x) = x * sigmoid(x)
+ *
+ * so an all-zero row maps to zero.  The output is what muir_chunk_fwd and
+ * muir_recurrent_step expect as q and k.
+ *
+ *   rows : number of rows (B*T*H for token-major [B][T][H][d]); 0 enqueues
+ *          nothing and returns MUIR_OK
+ *   d    : 64 or 128 (else MUIR_ERR_UNSUPPORTED)
+ *   x, y : device [rows][d] in dtype; y may equal x (in place)
+ * Float32 arithmetic, y stored in dtype (round to nearest even).  Bound by
+ * HBM: each row is read once and written once.
+ */
+muir_status muir_qk_prologue(long long rows, int d, muir_dtype dtype, const void* x, void* y,
+                             void* stream);
+
+/*
+ * Backward of muir_qk_prologue: with s = SiLU(x), n = max(||s||, 1e-12),
+ *     ds = dy / n - s (s . dy) / n^3   (ds = dy / 1e-12 when ||s|| < 1e-12)
+ *     dx = ds * sigmoid(x) * (1 + x * (1 - sigmoid(x)))
+ *   x, dy, dx : device [rows][d] in dtype; dx may equal dy or x.
+ * Arguments and errors as muir_qk_prologue.
+ */
+muir_status muir_qk_prologue_bwd(long long rows, int d, muir_dtype dtype, const void* x,
+                                 const void* dy, void* dx, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -14,12 +14,16 @@ Two independent C sources are wrapped:
   derived by unrolling it over a chunk (same page, "Methodology": each chunk is
   a triangular system), with exact exponent differences.
 
+and, in numpy below, the q/k feature prologue (SiLU, then unit L2 norm per
+token-head row; same page, "Methodology" and fig. 3(b)) with its gradient.
+
 Every function takes numpy-convertible arrays, computes in float64 and returns
 float64 numpy arrays.  Per-token tensors are ``[B, T, H, d]``; states are
 ``[B, H, dk, dv]``.
 
 Pins (what fixes these functions other than themselves) live in
-``tests/test_oracle_pins.py``: linear-attention and gated-linear-attention
+``tests/test_oracle_pins.py`` and ``tests/test_qk_oracle.py`` (the prologue):
+linear-attention and gated-linear-attention
 closed forms, the delta rule (Widrow-Hoff), an exact-retrieval invariant,
 pure decay, chunk-size invariance, linearity, column equivariance, state
 passing, decode/recurrence equivalence, a hand-computed example in
@@ -168,3 +172,34 @@ def step(q, k, v, g, e, w, gamma, S, gamma_static=False):
     if rc:
         raise ValueError("muir_ref_step: bad shape")
     return o, S
+
+
+# ------------------------------------------------------------ q/k prologue
+
+QK_NORM_EPS = 1e-12  # guard of the norm: an all-zero row maps to zero
+
+
+def qk_prologue(x):
+    """``y = s / max(||s||, eps)`` with ``s = SiLU(x) = x * sigmoid(x)`` over the
+    last axis (one token-head row of d channels), in float64.  The pages end
+    the query and key pathways in SiLU and keep the key unit-normalised
+    ("Methodology", fig. 3(b)); eps only guards the zero row."""
+    x = _f64(x)
+    s = x / (1.0 + np.exp(-x))
+    n = np.maximum(np.sqrt((s * s).sum(axis=-1, keepdims=True)), QK_NORM_EPS)
+    return s / n
+
+
+def qk_prologue_bwd(x, dy):
+    """Gradient of ``sum(dy * qk_prologue(x))`` with respect to x, in float64:
+    the Jacobian of s -> s / ||s|| is (I - y y^T) / ||s|| (1 / eps times the
+    identity below the guard), and SiLU'(x) = sig(x) (1 + x (1 - sig(x)))."""
+    x, dy = _f64(x), _f64(dy)
+    sig = 1.0 / (1.0 + np.exp(-x))
+    s = x * sig
+    nrm = np.sqrt((s * s).sum(axis=-1, keepdims=True))
+    tiny = nrm < QK_NORM_EPS
+    n = np.maximum(nrm, QK_NORM_EPS)
+    y = s / n
+    ds = (dy - np.where(tiny, 0.0, y * (y * dy).sum(axis=-1, keepdims=True))) / n
+    return ds * sig * (1.0 + x * (1.0 - sig))

@@ -137,6 +137,20 @@ def test_recurrent_step_rejects_bad_arguments(L):
     assert L.muir_recurrent_step(2, 16, 128, 128, 3, 1, *P, None, 0, FAKE, FAKE, None) == 1
 
 
+def test_qk_prologue_rejects_bad_arguments(L):
+    # every case is rejected on the host before anything is enqueued
+    assert L.muir_qk_prologue(0, 128, 0, None, None, None) == 0          # empty: no-op
+    assert L.muir_qk_prologue(-1, 128, 0, FAKE, FAKE, None) == 1
+    assert L.muir_qk_prologue(16, 96, 0, FAKE, FAKE, None) == 2          # head dim
+    assert L.muir_qk_prologue(16, 128, 5, FAKE, FAKE, None) == 1         # dtype
+    assert L.muir_qk_prologue(16, 128, 0, None, FAKE, None) == 1
+    assert L.muir_qk_prologue(16, 128, 0, FAKE, ctypes.c_void_p(0x10008), None) == 1
+    assert L.muir_qk_prologue_bwd(0, 64, 1, None, None, None, None) == 0
+    assert L.muir_qk_prologue_bwd(16, 32, 1, FAKE, FAKE, FAKE, None) == 2
+    assert L.muir_qk_prologue_bwd(16, 64, 1, FAKE, None, FAKE, None) == 1
+    assert L.muir_qk_prologue_bwd(16, 64, 1, FAKE, FAKE, ctypes.c_void_p(0x10004), None) == 1
+
+
 def test_binding_refuses_cpu_tensors(L):
     import torch
     import gated_delta_rule_115_b200 as m
