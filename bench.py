@@ -56,15 +56,22 @@ DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 6 * 128 * 2 + 128 * 2  # S read+writ
 # DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel; valid only while the kernel source hash matches.
 NCU_TRAFFIC = {
-    # profiles/k_bwd_k_out_B1_H16_T8192_d128_C128.md: 6.406 GB for 131,072 token-heads
-    "k_bwd": {"bytes_per_token_head": 6.4061e9 / 131072, "source": "ef4679f7a70d3c06"},
+    # profiles/k_bwd_k_out_B1_H16_T8192_d128_C128.md: 6.410 GB for 131,072 token-heads;
+    # source = source_hash(chunk_kernels_only=True) of the captured build
+    "k_bwd": {"bytes_per_token_head": 6.4104e9 / 131072, "source": "0b6a614d9c25e16a"},
 }
 
 
-def source_hash() -> str:
+def source_hash(chunk_kernels_only: bool = False) -> str:
+    """Hash of the library sources; with ``chunk_kernels_only`` of the files the
+    chunk kernels are compiled from (``chunk*.cu`` and every header), so that
+    counters taken on those kernels stay valid across changes elsewhere."""
     h = hashlib.sha256()
-    for f in sorted(os.listdir(os.path.join(ROOT, "gated_delta_rule_115_b200", "csrc"))):
-        with open(os.path.join(ROOT, "gated_delta_rule_115_b200", "csrc", f), "rb") as fh:
+    csrc = os.path.join(ROOT, "gated_delta_rule_115_b200", "csrc")
+    for f in sorted(os.listdir(csrc)):
+        if chunk_kernels_only and not (f.startswith("chunk") or f.endswith((".cuh", ".h"))):
+            continue
+        with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
 
@@ -321,6 +328,7 @@ def gpu_arm(args, rank, world, local):
         "gpu_launches": launches,
         "clocks": clocks,
         "source": source_hash(),
+        "chunk_kernel_source": source_hash(chunk_kernels_only=True),
     }
     if not args.no_e2e:
         out["e2e"] = e2e_measure(muir, x, W, C, dev, ws_f, ws_b, max(1, min(args.steps, 3)), world)
@@ -367,7 +375,7 @@ def kernel_roofline(name, avg_ms, token_heads, C, d, peaks):
     f_hbm, f_tc = gbs / peaks["hbm_gbs"], tfl / tf32_peak
     traffic = None
     t = NCU_TRAFFIC.get(name)
-    if t and t.get("source") == source_hash():
+    if t and t.get("source") == source_hash(chunk_kernels_only=True):
         traffic = t["bytes_per_token_head"] * token_heads
     if f_hbm >= f_tc:
         r = {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s", "frac": f_hbm}

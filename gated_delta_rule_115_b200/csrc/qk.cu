@@ -19,7 +19,8 @@
 // (8 to 32), the row's sums reduce with butterfly shuffles inside that lane
 // group, and every lane keeps kRowsInFlight rows' loads in flight so enough
 // bytes are outstanding per SM to cover the HBM latency.  Arithmetic is
-// float32; the output is stored in the input dtype (round to nearest even).
+// float32 (the sigmoid from the fast exponential and division); the output is
+// stored in the input dtype (round to nearest even).
 #include "common.cuh"
 #include "kernels.h"
 #include "profile.h"
@@ -57,7 +58,10 @@ __device__ __forceinline__ void st16(__nv_bfloat16* p, const float* v) {
     *reinterpret_cast<uint4*>(p) = make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__device__ __forceinline__ float sigm(float x) { return 1.0f / (1.0f + expf(-x)); }
+// sigmoid from the fast exponential (2 + 1.173|x| ulp) and division (2 ulp): two
+// special-function ops per element, so the kernels stay bound by HBM rather than
+// by the longer exact expf / division sequences.  x < -88 gives exp = inf and 0.
+__device__ __forceinline__ float sigm(float x) { return __fdividef(1.0f, 1.0f + __expf(-x)); }
 
 // Sum over the G lanes of one row (groups of G consecutive lanes).
 template <int G>
@@ -130,10 +134,17 @@ template <typename T, int D, bool BWD>
 cudaError_t launch_qk(const void* x, const void* dy, void* out, long long rows, cudaStream_t st) {
     constexpr int RPB = (kQkThreads / 32) * (32 / (D * (int)sizeof(T) / 16)) * kRowsInFlight;
     long long blocks = (rows + RPB - 1) / RPB;
-    int dev = 0, nsm = 148;
+    int dev = 0, nsm = 148, occ = 1;
     if (cudaGetDevice(&dev) == cudaSuccess)
         cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-    const long long cap = (long long)nsm * (2048 / kQkThreads);
+    // one wave of resident CTAs: a grid-stride CTA beyond it would only start
+    // after a resident one has finished its whole share
+    if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_qk<T, D, BWD>, kQkThreads, 0) !=
+            cudaSuccess || occ < 1) {
+        (void)cudaGetLastError();  // a failed query is not a launch error
+        occ = 1;
+    }
+    const long long cap = (long long)nsm * occ;
     if (blocks > cap) blocks = cap;
     MUIR_TIMED(BWD ? "k_qk_bwd" : "k_qk", st,
                (k_qk<T, D, BWD><<<(unsigned)blocks, kQkThreads, 0, st>>>(

@@ -199,8 +199,9 @@ muir_status muir_recurrent_step(int B, int H, int dk, int dv, muir_dtype dtype,
  *          nothing and returns MUIR_OK
  *   d    : 64 or 128 (else MUIR_ERR_UNSUPPORTED)
  *   x, y : device [rows][d] in dtype; y may equal x (in place)
- * Float32 arithmetic, y stored in dtype (round to nearest even).  Bound by
- * HBM: each row is read once and written once.
+ * Float32 arithmetic (sigmoid from the fast exponential and division: within
+ * about 1e-6 relative for |x| <= 10), y stored in dtype (round to nearest
+ * even).  Bound by HBM: each row is read once and written once.
  */
 muir_status muir_qk_prologue(long long rows, int d, muir_dtype dtype, const void* x, void* y,
                              void* stream);

@@ -2,10 +2,14 @@
 against the fp64 oracle on seeded inputs.
 
 Error metric: max |gpu - oracle| / max |oracle| per tensor.  Both sides read
-the same stored inputs.  Tolerances from the arithmetic: float32 outputs
-1e-6 (forward) and 1e-5 (backward, one cancellation dy - y (y . dy));
-bfloat16 outputs are rounded once to nearest even, a relative error of at
-most 2^-8 per element, so 4e-3 (forward) and 5e-3 (backward).
+the same stored inputs.  Tolerances from the arithmetic: the kernel's sigmoid
+uses the fast exponential (at most 2 + 1.173|x| ulp) and division (2 ulp), so
+for the |x| <= 10 that carry a row's weight sigmoid is within 15 ulp (~9e-7
+relative), SiLU and the normalised row within about 2e-6: float32 outputs 5e-6
+(forward) and 1e-5 (backward, one more sigmoid and the cancellation
+dy - y (y . dy)); bfloat16 outputs are rounded once to nearest even, a
+relative error of at most 2^-8 per element, so 4e-3 (forward) and 5e-3
+(backward).
 """
 import numpy as np
 import pytest
@@ -13,7 +17,7 @@ import torch
 
 pytestmark = pytest.mark.gpu
 
-TOL_FWD = {torch.float32: 1e-6, torch.bfloat16: 4e-3}
+TOL_FWD = {torch.float32: 5e-6, torch.bfloat16: 4e-3}
 TOL_BWD = {torch.float32: 1e-5, torch.bfloat16: 5e-3}
 
 
