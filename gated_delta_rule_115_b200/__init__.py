@@ -22,7 +22,8 @@ import os
 import torch
 
 __all__ = [
-    "MuirError", "lib", "chunk_fwd", "chunk_bwd", "recurrent_step", "qk_prologue",
+    "MuirError", "lib", "chunk_fwd", "chunk_bwd", "chunk_fwd_varlen", "chunk_bwd_varlen",
+    "recurrent_step", "qk_prologue",
     "qk_prologue_bwd", "fwd_workspace_bytes", "bwd_workspace_bytes", "MuirChunkFunction",
     "LIB_PATH",
 ]
@@ -75,6 +76,13 @@ def lib():
         L.muir_chunk_bwd.restype = I
         L.muir_recurrent_step.argtypes = [I, I, I, I, I, I] + [P] * 7 + [I, P, P, P]
         L.muir_recurrent_step.restype = I
+        LLP = ctypes.POINTER(ctypes.c_longlong)
+        L.muir_chunk_varlen_workspace.argtypes = [SP, I, LLP, I]
+        L.muir_chunk_varlen_workspace.restype = S
+        L.muir_chunk_fwd_varlen.argtypes = [SP, I, LLP] + [P] * 11 + [S, P]
+        L.muir_chunk_fwd_varlen.restype = I
+        L.muir_chunk_bwd_varlen.argtypes = [SP, I, LLP] + [P] * 19 + [S, P]
+        L.muir_chunk_bwd_varlen.restype = I
         L.muir_qk_prologue.argtypes = [ctypes.c_longlong, I, I, P, P, P]
         L.muir_qk_prologue.restype = I
         L.muir_qk_prologue_bwd.argtypes = [ctypes.c_longlong, I, I, P, P, P, P]
@@ -233,6 +241,60 @@ def recurrent_step(q, k, v, g, e, w, gamma, S, gamma_static=False, out_dtype=Non
                                _ptr(S), _ptr(o), _stream(q.device))
     _check("muir_recurrent_step", rc)
     return o
+
+
+def _cu(cu_seqlens):
+    vals = [int(c) for c in (cu_seqlens.tolist() if hasattr(cu_seqlens, "tolist") else cu_seqlens)]
+    return len(vals) - 1, (ctypes.c_longlong * len(vals))(*vals)
+
+
+def chunk_fwd_varlen(q, k, v, g, e, w, gamma, cu_seqlens, S0=None, chunk=64, out_dtype=None,
+                     ws=None):
+    """Forward over packed sequences: per-token tensors ``[1, T, H, d]`` with
+    sequence i at rows ``cu_seqlens[i]:cu_seqlens[i+1]`` (a host list or CPU
+    tensor).  ``S0`` is ``[num_seqs, H, dk, dv]`` or None.  Returns
+    ``(o, S_final)`` with ``S_final`` of shape ``[num_seqs, H, dk, dv]``."""
+    L = lib()
+    n, cu = _cu(cu_seqlens)
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    shp = _shape(q, v, chunk, out_dtype)
+    od = torch.bfloat16 if shp.out_dtype == MUIR_BF16 else torch.float32
+    o = torch.empty(B, T, H, dv, dtype=od, device=q.device)
+    S_final = torch.empty(n, H, dk, dv, dtype=torch.float32, device=q.device)
+    need = int(L.muir_chunk_varlen_workspace(ctypes.byref(shp), n, cu, 0))
+    wsb = _workspace(need, q.device, ws)
+    rc = L.muir_chunk_fwd_varlen(ctypes.byref(shp), n, cu, _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                 _ptr(e), _ptr(w), _ptr(gamma), _ptr(S0), _ptr(o), _ptr(S_final),
+                                 _ptr(wsb), ctypes.c_size_t(0 if wsb is None else wsb.numel()),
+                                 _stream(q.device))
+    _check("muir_chunk_fwd_varlen", rc)
+    return o, S_final
+
+
+def chunk_bwd_varlen(q, k, v, g, e, w, gamma, cu_seqlens, S0, dO, dS_final=None, chunk=64,
+                     ws=None):
+    """Gradients of ``sum(o*dO) + sum(S_final*dS_final)`` over packed sequences
+    (see :func:`chunk_fwd_varlen`); returns the dict of :func:`chunk_bwd` with
+    ``dS0`` of shape ``[num_seqs, H, dk, dv]``."""
+    L = lib()
+    n, cu = _cu(cu_seqlens)
+    shp = _shape(q, v, chunk, None)
+    grads = {nm: torch.empty_like(x) for nm, x in
+             dict(dq=q, dk=k, dv=v, dg=g, de=e, dw=w, dgamma=gamma).items()}
+    _, _, H, dk = q.shape
+    grads["dS0"] = torch.empty(n, H, dk, v.shape[-1], dtype=torch.float32, device=q.device)
+    need = int(L.muir_chunk_varlen_workspace(ctypes.byref(shp), n, cu, 1))
+    wsb = _workspace(need, q.device, ws)
+    rc = L.muir_chunk_bwd_varlen(ctypes.byref(shp), n, cu, _ptr(q), _ptr(k), _ptr(v), _ptr(g),
+                                 _ptr(e), _ptr(w), _ptr(gamma), _ptr(S0), _ptr(dO),
+                                 _ptr(dS_final), *[_ptr(grads[nm]) for nm in
+                                                   ("dq", "dk", "dv", "dg", "de", "dw", "dgamma")],
+                                 _ptr(grads["dS0"]), _ptr(wsb),
+                                 ctypes.c_size_t(0 if wsb is None else wsb.numel()),
+                                 _stream(q.device))
+    _check("muir_chunk_bwd_varlen", rc)
+    return grads
 
 
 def qk_prologue(x, out=None):

@@ -50,6 +50,35 @@ muir::ChunkProblem make_problem(const muir_shape* s, const void* q, const void* 
     return P;
 }
 
+// Packed variable-length batch: B == 1, T = total tokens, cu_seqlens (host)
+// holds num_seqs + 1 non-decreasing offsets from 0 to T.  A batch whose
+// sequences are all empty (T == 0) is valid.
+muir_status check_varlen(const muir_shape* s, int num_seqs, const long long* cu) {
+    if (!s || num_seqs <= 0 || !cu || s->B != 1 || s->T < 0) return MUIR_ERR_INVALID_ARG;
+    if (cu[0] != 0 || cu[num_seqs] != s->T) return MUIR_ERR_INVALID_ARG;
+    for (int i = 0; i < num_seqs; ++i)
+        if (cu[i + 1] < cu[i]) return MUIR_ERR_INVALID_ARG;
+    muir_shape t = *s;
+    if (t.T == 0) t.T = t.chunk > 0 ? t.chunk : 1;  // the remaining checks only
+    return check_shape(&t);
+}
+
+size_t varlen_ws_bytes(const muir_shape* s, int num_seqs, const long long* cu, bool bwd) {
+    size_t need = 0;
+    for (int i = 0; i < num_seqs; ++i) {
+        const int L = (int)(cu[i + 1] - cu[i]);
+        if (L == 0) continue;
+        const size_t b = bwd ? muir::chunk_bwd_ws_bytes(1, L, s->H, s->dk, s->chunk, false)
+                             : muir::chunk_fwd_ws_bytes(1, L, s->H, s->dk, s->chunk, false);
+        if (b > need) need = b;
+    }
+    return need;
+}
+
+const void* at_row(const void* p, long long row, size_t row_bytes) {
+    return static_cast<const char*>(p) + (size_t)row * row_bytes;
+}
+
 muir_status from_cuda(cudaError_t err) {
     if (err == cudaSuccess) return MUIR_OK;
     if (err == cudaErrorNotSupported) return MUIR_ERR_UNSUPPORTED;
@@ -64,7 +93,7 @@ const char* muir_status_string(muir_status s) {
     switch (s) {
         case MUIR_OK: return "MUIR_OK";
         case MUIR_ERR_INVALID_ARG: return "MUIR_ERR_INVALID_ARG: null, misaligned or out-of-range argument";
-        case MUIR_ERR_UNSUPPORTED: return "MUIR_ERR_UNSUPPORTED: shape, chunk, tail or device not supported";
+        case MUIR_ERR_UNSUPPORTED: return "MUIR_ERR_UNSUPPORTED: shape, chunk or device not supported";
         case MUIR_ERR_WORKSPACE: return "MUIR_ERR_WORKSPACE: workspace missing or too small";
         case MUIR_ERR_CUDA: return "MUIR_ERR_CUDA: a CUDA runtime call or kernel launch failed";
         case MUIR_ERR_DEVICE_TIMEOUT: return "MUIR_ERR_DEVICE_TIMEOUT: a bounded device wait expired";
@@ -158,6 +187,102 @@ muir_status muir_recurrent_step(int B, int H, int dk, int dv, muir_dtype dtype,
     return from_cuda(muir::launch_decode(B, H, dk, dtype == MUIR_BF16, out_dtype == MUIR_BF16,
                                          q, k, v, g, e, w, gamma, gamma_static, S, o,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+size_t muir_chunk_varlen_workspace(const muir_shape* s, int num_seqs, const long long* cu_seqlens,
+                                   int backward) {
+    if (check_varlen(s, num_seqs, cu_seqlens) != MUIR_OK) return 0;
+    return varlen_ws_bytes(s, num_seqs, cu_seqlens, backward != 0);
+}
+
+muir_status muir_chunk_fwd_varlen(const muir_shape* s, int num_seqs, const long long* cu_seqlens,
+                                  const void* q, const void* k, const void* v, const void* g,
+                                  const void* e, const void* w, const void* gamma,
+                                  const float* S0, void* o, float* S_final, void* ws,
+                                  size_t ws_bytes, void* stream) {
+    muir_status st = check_varlen(s, num_seqs, cu_seqlens);
+    if (st != MUIR_OK) return st;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
+        !ok_ptr(gamma) || !ok_ptr(o) || !ok_opt(S0) || !ok_opt(S_final))
+        return MUIR_ERR_INVALID_ARG;
+    const size_t need = varlen_ws_bytes(s, num_seqs, cu_seqlens, false);
+    if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
+    if ((st = check_device()) != MUIR_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const size_t DD = (size_t)s->dk * s->dv, row = (size_t)s->H * s->dk;
+    const size_t ein = s->in_dtype == MUIR_BF16 ? 2 : 4, eout = s->out_dtype == MUIR_BF16 ? 2 : 4;
+    for (int i = 0; i < num_seqs; ++i) {
+        const long long r0 = cu_seqlens[i];
+        const int L = (int)(cu_seqlens[i + 1] - r0);
+        const float* s0 = S0 ? S0 + (size_t)i * s->H * DD : nullptr;
+        float* sf = S_final ? S_final + (size_t)i * s->H * DD : nullptr;
+        cudaError_t err = cudaSuccess;
+        if (L == 0) {  // empty sequence: the final state is the initial one
+            if (sf && s0) err = cudaMemcpyAsync(sf, s0, s->H * DD * 4, cudaMemcpyDeviceToDevice, cs);
+            else if (sf) err = cudaMemsetAsync(sf, 0, s->H * DD * 4, cs);
+            if (err != cudaSuccess) return from_cuda(err);
+            continue;
+        }
+        muir_shape si = *s;
+        si.T = L;
+        const size_t rb = row * ein;
+        muir::ChunkProblem P = make_problem(&si, at_row(q, r0, rb), at_row(k, r0, rb),
+                                            at_row(v, r0, rb), at_row(g, r0, rb),
+                                            at_row(e, r0, rb), at_row(w, r0, rb),
+                                            at_row(gamma, r0, rb));
+        err = muir::run_chunk_fwd(P, s0, const_cast<void*>(at_row(o, r0, row * eout)), sf,
+                                  nullptr, nullptr, ws, ws_bytes, cs);
+        if (err != cudaSuccess) return from_cuda(err);
+    }
+    return MUIR_OK;
+}
+
+muir_status muir_chunk_bwd_varlen(const muir_shape* s, int num_seqs, const long long* cu_seqlens,
+                                  const void* q, const void* k, const void* v, const void* g,
+                                  const void* e, const void* w, const void* gamma,
+                                  const float* S0, const void* dO, const float* dS_final,
+                                  void* dq, void* dk, void* dv, void* dg, void* de, void* dw,
+                                  void* dgamma, float* dS0, void* ws, size_t ws_bytes,
+                                  void* stream) {
+    muir_status st = check_varlen(s, num_seqs, cu_seqlens);
+    if (st != MUIR_OK) return st;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
+        !ok_ptr(gamma) || !ok_ptr(dO) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) ||
+        !ok_ptr(dg) || !ok_ptr(de) || !ok_ptr(dw) || !ok_ptr(dgamma) || !ok_opt(S0) ||
+        !ok_opt(dS_final) || !ok_opt(dS0))
+        return MUIR_ERR_INVALID_ARG;
+    const size_t need = varlen_ws_bytes(s, num_seqs, cu_seqlens, true);
+    if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
+    if ((st = check_device()) != MUIR_OK) return st;
+    cudaStream_t cs = static_cast<cudaStream_t>(stream);
+    const size_t DD = (size_t)s->dk * s->dv, row = (size_t)s->H * s->dk;
+    const size_t rb = row * (s->in_dtype == MUIR_BF16 ? 2 : 4);
+    for (int i = 0; i < num_seqs; ++i) {
+        const long long r0 = cu_seqlens[i];
+        const int L = (int)(cu_seqlens[i + 1] - r0);
+        const float* s0 = S0 ? S0 + (size_t)i * s->H * DD : nullptr;
+        const float* dsf = dS_final ? dS_final + (size_t)i * s->H * DD : nullptr;
+        float* ds0 = dS0 ? dS0 + (size_t)i * s->H * DD : nullptr;
+        cudaError_t err = cudaSuccess;
+        if (L == 0) {  // empty sequence: the state passes through unchanged
+            if (ds0 && dsf) err = cudaMemcpyAsync(ds0, dsf, s->H * DD * 4, cudaMemcpyDeviceToDevice, cs);
+            else if (ds0) err = cudaMemsetAsync(ds0, 0, s->H * DD * 4, cs);
+            if (err != cudaSuccess) return from_cuda(err);
+            continue;
+        }
+        muir_shape si = *s;
+        si.T = L;
+        auto out = [&](void* p) { return const_cast<void*>(at_row(p, r0, rb)); };
+        muir::ChunkProblem P = make_problem(&si, at_row(q, r0, rb), at_row(k, r0, rb),
+                                            at_row(v, r0, rb), at_row(g, r0, rb),
+                                            at_row(e, r0, rb), at_row(w, r0, rb),
+                                            at_row(gamma, r0, rb));
+        err = muir::run_chunk_bwd(P, s0, nullptr, nullptr, at_row(dO, r0, rb), dsf, out(dq),
+                                  out(dk), out(dv), out(dg), out(de), out(dw), out(dgamma), ds0,
+                                  ws, ws_bytes, cs);
+        if (err != cudaSuccess) return from_cuda(err);
+    }
+    return MUIR_OK;
 }
 
 muir_status muir_qk_prologue(long long rows, int d, muir_dtype dtype, const void* x, void* y,

@@ -146,6 +146,41 @@ muir_status muir_chunk_bwd(const muir_shape* shape, const void* q, const void* k
                            float* dS0, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * Packed variable-length sequences (streaming prefill of documents of mixed
+ * length; same page, "Experiments": long streams): num_seqs independent
+ * sequences stored back to back in one token-major buffer.
+ *
+ *   shape      : B must be 1; T = total tokens (0 allowed); other fields as above
+ *   cu_seqlens : HOST array of num_seqs + 1 offsets, cu_seqlens[0] = 0,
+ *                non-decreasing, cu_seqlens[num_seqs] = T; sequence i is
+ *                rows [cu_seqlens[i], cu_seqlens[i+1]) of every per-token tensor
+ *   S0, S_final, dS_final, dS0 : [num_seqs][H][dk][dv] float32, each may be NULL
+ *   other tensors as muir_chunk_fwd / muir_chunk_bwd with B = 1
+ * Each sequence runs the chunkwise path on its own rows (its own chunk grid and
+ * ragged tail), one after another on `stream`, sharing the workspace; an empty
+ * sequence copies S0 to S_final (dS_final to dS0), or writes zeros.  No chunk
+ * states are saved: the backward recomputes them.  Bad offsets return
+ * MUIR_ERR_INVALID_ARG before anything is enqueued.
+ *
+ * muir_chunk_varlen_workspace: bytes of workspace for the forward (backward != 0:
+ * the backward); 0 for invalid arguments.  Host-only.
+ */
+size_t muir_chunk_varlen_workspace(const muir_shape* shape, int num_seqs,
+                                   const long long* cu_seqlens, int backward);
+muir_status muir_chunk_fwd_varlen(const muir_shape* shape, int num_seqs,
+                                  const long long* cu_seqlens, const void* q, const void* k,
+                                  const void* v, const void* g, const void* e, const void* w,
+                                  const void* gamma, const float* S0, void* o, float* S_final,
+                                  void* ws, size_t ws_bytes, void* stream);
+muir_status muir_chunk_bwd_varlen(const muir_shape* shape, int num_seqs,
+                                  const long long* cu_seqlens, const void* q, const void* k,
+                                  const void* v, const void* g, const void* e, const void* w,
+                                  const void* gamma, const float* S0, const void* dO,
+                                  const float* dS_final, void* dq, void* dk, void* dv, void* dg,
+                                  void* de, void* dw, void* dgamma, float* dS0, void* ws,
+                                  size_t ws_bytes, void* stream);
+
+/*
  * muir_chunk_fwd for callers that cannot allocate device memory.  The paper
  * has no counterpart; this is a deployment convenience.  Some hosts hand a
  * library only input and output pointers (plugin interfaces of runtimes that

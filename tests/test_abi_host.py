@@ -137,6 +137,36 @@ def test_recurrent_step_rejects_bad_arguments(L):
     assert L.muir_recurrent_step(2, 16, 128, 128, 3, 1, *P, None, 0, FAKE, FAKE, None) == 1
 
 
+def _cu(vals):
+    return (ctypes.c_longlong * len(vals))(*vals)
+
+
+def test_varlen_rejects_bad_offsets(L):
+    import gated_delta_rule_115_b200 as m
+    shp = _shape(m, T=100)
+    fwd = lambda s, n, cu, **kw: L.muir_chunk_fwd_varlen(  # noqa: E731
+        ctypes.byref(s), n, cu, *([FAKE] * 7), None, FAKE, None, kw.get("ws"),
+        ctypes.c_size_t(kw.get("ws_bytes", 0)), None)
+    # every case is rejected on the host before anything is enqueued
+    assert fwd(_shape(m, B=2, T=100), 2, _cu([0, 40, 100])) == 1   # B must be 1
+    assert fwd(shp, 2, _cu([1, 40, 100])) == 1                     # cu[0] != 0
+    assert fwd(shp, 2, _cu([0, 60, 40])) == 1                      # decreasing
+    assert fwd(shp, 2, _cu([0, 40, 99])) == 1                      # last != T
+    assert fwd(shp, 0, _cu([0])) == 1                              # no sequence
+    assert fwd(shp, 2, None) == 1
+    assert fwd(_shape(m, T=100, dk=96, dv=96), 2, _cu([0, 40, 100])) == 2
+    assert fwd(shp, 2, _cu([0, 40, 100])) == 3                     # valid, needs workspace
+    assert L.muir_chunk_varlen_workspace(ctypes.byref(shp), 2, _cu([0, 60, 40]), 0) == 0
+    # the workspace is the largest single sequence's
+    one = L.muir_chunk_fwd_workspace(ctypes.byref(_shape(m, T=60)))
+    assert L.muir_chunk_varlen_workspace(ctypes.byref(shp), 2, _cu([0, 40, 100]), 0) == one
+    oneb = L.muir_chunk_bwd_workspace(ctypes.byref(_shape(m, T=60)))
+    assert L.muir_chunk_varlen_workspace(ctypes.byref(shp), 2, _cu([0, 40, 100]), 1) == oneb
+    args = [FAKE] * 7 + [None, FAKE, None] + [FAKE] * 7 + [None, None]
+    assert L.muir_chunk_bwd_varlen(ctypes.byref(shp), 2, _cu([0, 50, 49]), *args,
+                                   ctypes.c_size_t(0), None) == 1
+
+
 def test_qk_prologue_rejects_bad_arguments(L):
     # every case is rejected on the host before anything is enqueued
     assert L.muir_qk_prologue(0, 128, 0, None, None, None) == 0          # empty: no-op
