@@ -73,7 +73,7 @@ __device__ __forceinline__ float group_sum(float a) {
 
 // BWD = false: y = SiLU(x) / max(||SiLU(x)||, eps).  BWD = true: dx from (x, dy).
 template <typename T, int D, bool BWD>
-__global__ void __launch_bounds__(kQkThreads)
+__global__ void __launch_bounds__(kQkThreads, BWD ? 4 : 8)
 k_qk(const T* x, const T* dy, T* out, long long rows) {
     constexpr int V = 16 / (int)sizeof(T);  // elements per lane
     constexpr int G = D / V;                // lanes per row
