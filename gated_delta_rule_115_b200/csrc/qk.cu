@@ -32,12 +32,13 @@ constexpr int kQkThreads = 256;
 constexpr int kRowsInFlight = 2;
 constexpr float kNormEps = 1e-12f;
 
-__device__ __forceinline__ void ld16(const float* p, float* v) {
-    const float4 a = *reinterpret_cast<const float4*>(p);
-    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+// 16 bytes of a row as raw bits (kept packed while in flight), unpacked to float32.
+__device__ __forceinline__ uint4 ld16raw(const void* p) { return *reinterpret_cast<const uint4*>(p); }
+__device__ __forceinline__ void unpack16(const uint4& a, float* v, float) {
+    v[0] = __uint_as_float(a.x); v[1] = __uint_as_float(a.y);
+    v[2] = __uint_as_float(a.z); v[3] = __uint_as_float(a.w);
 }
-__device__ __forceinline__ void ld16(const __nv_bfloat16* p, float* v) {
-    const uint4 a = *reinterpret_cast<const uint4*>(p);
+__device__ __forceinline__ void unpack16(const uint4& a, float* v, __nv_bfloat16) {
     const uint32_t w[4] = {a.x, a.y, a.z, a.w};
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
@@ -72,8 +73,10 @@ __device__ __forceinline__ float group_sum(float a) {
 }
 
 // BWD = false: y = SiLU(x) / max(||SiLU(x)||, eps).  BWD = true: dx from (x, dy).
+// The next pass's rows are loaded (packed) before this pass's are computed, so
+// every lane keeps loads in flight while it does arithmetic.
 template <typename T, int D, bool BWD>
-__global__ void __launch_bounds__(kQkThreads, BWD ? 4 : 8)
+__global__ void __launch_bounds__(kQkThreads, BWD ? 3 : 6)
 k_qk(const T* x, const T* dy, T* out, long long rows) {
     constexpr int V = 16 / (int)sizeof(T);  // elements per lane
     constexpr int G = D / V;                // lanes per row
@@ -81,30 +84,36 @@ k_qk(const T* x, const T* dy, T* out, long long rows) {
     constexpr int U = kRowsInFlight;
     const int lane = threadIdx.x & 31, sub = lane / G, col = (lane % G) * V;
     const long long warp = ((long long)blockIdx.x * kQkThreads + threadIdx.x) >> 5;
-    const long long nwarp = (long long)gridDim.x * (kQkThreads / 32);
-    for (long long r0 = warp * RPW * U; r0 < rows; r0 += nwarp * RPW * U) {
-        float xv[U][V], dv[U][V];
-        bool ok[U];
+    const long long step = (long long)gridDim.x * (kQkThreads / 32) * RPW * U;
+    auto fetch = [&](long long base, uint4* bx, uint4* bd) {
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            const long long r = r0 + (long long)u * RPW + sub;
-            ok[u] = r < rows;
-#pragma unroll
-            for (int i = 0; i < V; ++i) { xv[u][i] = 0.f; dv[u][i] = 0.f; }
-            if (ok[u]) {
-                ld16(x + r * D + col, xv[u]);
-                if (BWD) ld16(dy + r * D + col, dv[u]);
+            const long long r = base + (long long)u * RPW + sub;
+            bx[u] = make_uint4(0u, 0u, 0u, 0u);
+            bd[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (r < rows) {
+                bx[u] = ld16raw(x + r * D + col);
+                if (BWD) bd[u] = ld16raw(dy + r * D + col);
             }
         }
+    };
+    long long r0 = warp * RPW * U;
+    uint4 cx[U], cd[U];
+    fetch(r0, cx, cd);
+    for (; r0 < rows; r0 += step) {
+        uint4 nx[U], nd[U];
+        fetch(r0 + step, nx, nd);
 #pragma unroll
         for (int u = 0; u < U; ++u) {
-            float sv[V], sg[V], ss = 0.f, sd = 0.f;
+            float xv[V], dv[V], sv[V], sg[V], ss = 0.f, sd = 0.f;
+            unpack16(cx[u], xv, T());
+            if (BWD) unpack16(cd[u], dv, T());
 #pragma unroll
             for (int i = 0; i < V; ++i) {
-                sg[i] = sigm(xv[u][i]);
-                sv[i] = xv[u][i] * sg[i];
+                sg[i] = sigm(xv[i]);
+                sv[i] = xv[i] * sg[i];
                 ss += sv[i] * sv[i];
-                if (BWD) sd += sv[i] * dv[u][i];
+                if (BWD) sd += sv[i] * dv[i];
             }
             // every lane takes part in the shuffles, rows past the end with zeros
             ss = group_sum<G>(ss);
@@ -120,13 +129,15 @@ k_qk(const T* x, const T* dy, T* out, long long rows) {
                 const float c = tiny ? 0.f : sd * inv * inv * inv;
 #pragma unroll
                 for (int i = 0; i < V; ++i) {
-                    const float ds = dv[u][i] * inv - sv[i] * c;
-                    r[i] = ds * sg[i] * (1.0f + xv[u][i] * (1.0f - sg[i]));
+                    const float ds = dv[i] * inv - sv[i] * c;
+                    r[i] = ds * sg[i] * (1.0f + xv[i] * (1.0f - sg[i]));
                 }
             }
             const long long row = r0 + (long long)u * RPW + sub;
-            if (ok[u]) st16(out + row * D + col, r);
+            if (row < rows) st16(out + row * D + col, r);
         }
+#pragma unroll
+        for (int u = 0; u < U; ++u) { cx[u] = nx[u]; cd[u] = nd[u]; }
     }
 }
 
