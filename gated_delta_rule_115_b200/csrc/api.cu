@@ -5,6 +5,7 @@
 
 #include "../../include/muir.h"
 #include "chunk_units.h"
+#include "fwd2.h"
 #include "kernels.h"
 
 namespace {
@@ -47,6 +48,7 @@ muir::ChunkProblem make_problem(const muir_shape* s, const void* q, const void* 
     P.out_bf16 = s->out_dtype == MUIR_BF16;
     P.q = q; P.k = k; P.v = v; P.g = g; P.e = e; P.w = w; P.gamma = gamma;
     P.aux = nullptr;
+    P.gate = nullptr;
     return P;
 }
 
@@ -69,7 +71,7 @@ size_t varlen_ws_bytes(const muir_shape* s, int num_seqs, const long long* cu, b
         const int L = (int)(cu[i + 1] - cu[i]);
         if (L == 0) continue;
         const size_t b = bwd ? muir::chunk_bwd_ws_bytes(1, L, s->H, s->dk, s->chunk, false)
-                             : muir::chunk_fwd_ws_bytes(1, L, s->H, s->dk, s->chunk, false);
+                             : muir::chunk_fwd_ws_bytes(1, L, s->H, s->dk, s->chunk, false, s->in_dtype == MUIR_BF16);
         if (b > need) need = b;
     }
     return need;
@@ -104,7 +106,8 @@ const char* muir_status_string(muir_status s) {
 muir_status muir_device_wait_status(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MUIR_ERR_CUDA;
     const unsigned int n = muir::timeouts_bf16_d128() + muir::timeouts_bf16_d64() +
-                           muir::timeouts_f32_d128() + muir::timeouts_f32_d64();
+                           muir::timeouts_f32_d128() + muir::timeouts_f32_d64() +
+                           muir::v2::timeouts_v2();
     return n ? MUIR_ERR_DEVICE_TIMEOUT : MUIR_OK;
 }
 
@@ -115,7 +118,8 @@ size_t muir_chunk_aux_floats(const muir_shape* s) {
 
 size_t muir_chunk_fwd_workspace(const muir_shape* s) {
     if (check_shape(s) != MUIR_OK) return 0;
-    return muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false);
+    return muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false,
+                                    s->in_dtype == MUIR_BF16);
 }
 
 size_t muir_chunk_bwd_workspace(const muir_shape* s) {
@@ -134,7 +138,7 @@ muir_status muir_chunk_fwd(const muir_shape* s, const void* q, const void* k, co
         !ok_opt(M_chunks) || !ok_opt(aux))
         return MUIR_ERR_INVALID_ARG;
     const size_t need = muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk,
-                                                 S_chunks != nullptr);
+                                                 S_chunks != nullptr, s->in_dtype == MUIR_BF16);
     if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
     if ((st = check_device()) != MUIR_OK) return st;
     muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);

@@ -3,18 +3,34 @@
 // instantiated in chunk_{bf16,f32}_d{64,128}.cu.
 #include "chunk_impl.cuh"
 #include "chunk_units.h"
+#include "fwd2.h"
 
 namespace muir {
 
 size_t chunk_aux_floats(int C, int D) { return make_aux_lay(C, D).total; }
 
-size_t chunk_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states) {
+static size_t old_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states) {
     const size_t nch = (size_t)B * H * ((T + C - 1) / C), DD = (size_t)D * D;
     size_t f = 2 * nch * DD;               // M, Bn
     if (!have_states) f += nch * DD;       // chunk-start states
     f += (size_t)num_slots((int)nch) * slot_floats(C, D);
     f += tail_side_floats(B, T, H, D, C);
     return f * sizeof(float);
+}
+
+// The on-chip tensor-core forward (fwd2.cu) runs when the shape allows it;
+// its first 256 bytes of workspace hold the device flags (span flag first),
+// the rest is shared with the boundary-pivot path, which runs after it and
+// only when the span flag is set.
+static bool use_v2_fwd(const ChunkProblem& P) {
+    return P.aux == nullptr && v2::fwd2_supported(P.B, P.T, P.H, P.D, P.C, P.in_bf16);
+}
+
+size_t chunk_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states, bool in_bf16) {
+    const size_t old = old_fwd_ws_bytes(B, T, H, D, C, have_states);
+    if (!v2::fwd2_supported(B, T, H, D, C, in_bf16)) return old;
+    const size_t nv2 = v2::fwd2_ws_bytes(B, T, H);
+    return 256 + (old > nv2 ? old : nv2);
 }
 
 size_t chunk_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states) {
@@ -28,6 +44,31 @@ size_t chunk_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states) {
 
 cudaError_t run_chunk_fwd(const ChunkProblem& P, const float* S0, void* o, float* S_final,
                           float* S_chunks, float* M_chunks, void* ws, size_t, cudaStream_t st) {
+    if (use_v2_fwd(P)) {
+        int* flags = static_cast<int*>(ws);
+        char* shared = static_cast<char*>(ws) + 256;
+        const size_t blk = (size_t)128 * 128;
+        const size_t nch = (size_t)P.B * P.H * P.N;
+        float* f = reinterpret_cast<float*>(shared);
+        v2::Fwd2Args a = {};
+        a.B = P.B; a.T = P.T; a.H = P.H; a.out_bf16 = P.out_bf16;
+        a.q = P.q; a.k = P.k; a.v = P.v; a.g = P.g; a.e = P.e; a.w = P.w; a.gamma = P.gamma;
+        a.S0 = S0; a.o = o; a.S_final = S_final;
+        a.M = M_chunks ? M_chunks : f; if (!M_chunks) f += nch * blk;
+        a.Mt = nullptr;
+        a.Bn = f; f += nch * blk;
+        a.Qp = f; f += nch * blk;
+        a.Oi = f; f += nch * blk;
+        a.S_chunks = S_chunks ? S_chunks : f;
+        a.flags = flags;
+        cudaError_t e = cudaMemsetAsync(flags, 0, 16, st);
+        if (e == cudaSuccess) e = v2::span_check(P.g, P.B, P.T, P.H, flags, st);
+        if (e == cudaSuccess) e = v2::run_fwd2(a, st);
+        if (e != cudaSuccess) return e;
+        ChunkProblem G = P;
+        G.gate = flags;  // boundary-pivot path only when a chunk's span exceeds the single pivot
+        return fwd_bf16_d128(G, S0, o, S_final, S_chunks, M_chunks, shared, st);
+    }
     if (P.in_bf16) {
         if (P.D == 128) return fwd_bf16_d128(P, S0, o, S_final, S_chunks, M_chunks, ws, st);
         return fwd_bf16_d64(P, S0, o, S_final, S_chunks, M_chunks, ws, st);

@@ -114,6 +114,9 @@ struct KParams {
     // only some chunks of each sequence (the padded last chunk of a ragged
     // sequence runs as its own launch over side buffers)
     int nstride, noff;
+    // device word that must be non-zero for the launch to do any work (the
+    // single-pivot span flag when the on-chip path ran first), or null
+    const int* gate;
 };
 
 // Accessors of one chunk's inputs; row t of a [B,T,H,D] tensor.
@@ -477,6 +480,7 @@ __device__ __forceinline__ void decayed_grad(const Chunk<Tin, D>& c, TcCta& tcx,
 
 template <typename Tin, int D, int PASSES, int CF>
 __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_intra(KParams p) {
+    if (p.gate && *p.gate == 0) return;
     __shared__ uint32_t tmem_slot;
     __shared__ __align__(8) uint64_t mbar;
     __shared__ int tc_status;
@@ -563,7 +567,9 @@ __global__ void __launch_bounds__(kThreads) k_chain(const float* __restrict__ M,
                                                     const float* __restrict__ Bn,
                                                     const float* __restrict__ S_in,
                                                     float* __restrict__ S_rec,
-                                                    float* __restrict__ S_out, int N) {
+                                                    float* __restrict__ S_out, int N,
+                                                    const int* __restrict__ gate) {
+    if (gate && *gate == 0) return;
     constexpr int NT = SLAB / 8 < 4 ? SLAB / 8 : 4;
     constexpr int MP = D + 4;  // padded row of M in shared memory
     __shared__ float buf[2][D * SLAB];
@@ -659,6 +665,7 @@ __device__ void compute_Y(TcCta& tcx, const Chunk<Tin, D>& c, const float* S, si
 
 template <typename Tin, typename Tout, int D, int PASSES, int CF>
 __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_out(KParams p) {
+    if (p.gate && *p.gate == 0) return;
     __shared__ uint32_t tmem_slot;
     __shared__ __align__(8) uint64_t mbar;
     __shared__ int tc_status;
@@ -731,6 +738,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_out(KParams p) {
 
 template <typename Tin, int D, int PASSES, int CF>
 __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_bprep(KParams p) {
+    if (p.gate && *p.gate == 0) return;
     __shared__ uint32_t tmem_slot;
     __shared__ __align__(8) uint64_t mbar;
     __shared__ int tc_status;
@@ -795,6 +803,7 @@ __global__ void __launch_bounds__(kThreads, fwd_ctas(PASSES)) k_bprep(KParams p)
 
 template <typename Tin, int D, int PASSES, int CF>
 __global__ void __launch_bounds__(kThreads) k_bwd(KParams p) {
+    if (p.gate && *p.gate == 0) return;
     __shared__ float s_colsum[D];
     __shared__ float s_segtot[kThreads];
     __shared__ float s_red[kThreads * 4];
@@ -1307,22 +1316,22 @@ int persistent_grid(KERNEL kernel, int nch, int dyn) {
 
 template <int D, int SL, int PASSES, bool REV>
 cudaError_t launch_chain_slab(int BH, int N, const float* M, const float* Bn, const float* S_in,
-                              float* S_rec, float* S_out, cudaStream_t st) {
+                              float* S_rec, float* S_out, const int* gate, cudaStream_t st) {
     constexpr int bytes = chain_smem_bytes<D, SL>();
     cudaError_t e = cudaFuncSetAttribute(k_chain<D, SL, PASSES, REV>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
     if (e != cudaSuccess) return e;
     MUIR_TIMED(REV ? "k_chain_rev" : "k_chain", st,
-               k_chain<D, SL, PASSES, REV><<<BH * (D / SL), kThreads, bytes, st>>>(M, Bn, S_in, S_rec, S_out, N));
+               k_chain<D, SL, PASSES, REV><<<BH * (D / SL), kThreads, bytes, st>>>(M, Bn, S_in, S_rec, S_out, N, gate));
     return cudaGetLastError();
 }
 
 template <int D, int PASSES, bool REV>
 cudaError_t launch_chain(int BH, int N, const float* M, const float* Bn, const float* S_in,
-                                float* S_rec, float* S_out, cudaStream_t st) {
+                                float* S_rec, float* S_out, const int* gate, cudaStream_t st) {
     // column slabs: enough CTAs to cover the GPU when B*H is small
-    if (BH >= 64) return launch_chain_slab<D, 32, PASSES, REV>(BH, N, M, Bn, S_in, S_rec, S_out, st);
-    return launch_chain_slab<D, 16, PASSES, REV>(BH, N, M, Bn, S_in, S_rec, S_out, st);
+    if (BH >= 64) return launch_chain_slab<D, 32, PASSES, REV>(BH, N, M, Bn, S_in, S_rec, S_out, gate, st);
+    return launch_chain_slab<D, 16, PASSES, REV>(BH, N, M, Bn, S_in, S_rec, S_out, gate, st);
 }
 
 template <typename Tin, int D, int PASSES, int CF>
@@ -1334,6 +1343,7 @@ cudaError_t fwd_impl(const ChunkProblem& P, const float* S0, void* o, float* S_f
     KParams kp = {};
     kp.B = P.B; kp.T = P.T; kp.H = P.H; kp.C = P.C; kp.N = P.N;
     kp.q = P.q; kp.k = P.k; kp.v = P.v; kp.g = P.g; kp.e = P.e; kp.w = P.w; kp.gamma = P.gamma;
+    kp.gate = P.gate;
     kp.M = f; f += nch * DD;
     if (M_chunks) kp.M = M_chunks;
     kp.Bn = f; f += nch * DD;
@@ -1365,7 +1375,7 @@ cudaError_t fwd_impl(const ChunkProblem& P, const float* S0, void* o, float* S_f
         return cudaSuccess;
     };
     if ((err = each(k_intra<Tin, D, PASSES, CF>, "k_intra")) != cudaSuccess) return err;
-    err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, S_final, st);
+    err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, S_final, P.gate, st);
     if (err != cudaSuccess) return err;
     if (P.out_bf16) err = each(k_out<Tin, __nv_bfloat16, D, PASSES, CF>, "k_out");
     else err = each(k_out<Tin, float, D, PASSES, CF>, "k_out");
@@ -1385,6 +1395,7 @@ cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chun
     KParams kp = {};
     kp.B = P.B; kp.T = P.T; kp.H = P.H; kp.C = P.C; kp.N = P.N;
     kp.q = P.q; kp.k = P.k; kp.v = P.v; kp.g = P.g; kp.e = P.e; kp.w = P.w; kp.gamma = P.gamma;
+    kp.gate = P.gate;
     kp.dO = dO;
     kp.M = f; f += nch * DD;
     kp.Bn = f; f += nch * DD;
@@ -1427,11 +1438,11 @@ cudaError_t bwd_impl(const ChunkProblem& P, const float* S0, const float* S_chun
     if (!have_M && (err = each(k_intra<Tin, D, PASSES, CF>, "k_intra", dyn)) != cudaSuccess)
         return err;
     if (recompute) {
-        err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, nullptr, st);
+        err = launch_chain<D, PASSES, false>(BH, P.N, kp.M, kp.Bn, S0, Sc, nullptr, P.gate, st);
         if (err != cudaSuccess) return err;
     }
     if ((err = each(k_bprep<Tin, D, PASSES, CF>, "k_bprep", dyn)) != cudaSuccess) return err;
-    err = launch_chain<D, PASSES, true>(BH, P.N, kp.M, kp.Bn, dS_final, dSc, dS0, st);
+    err = launch_chain<D, PASSES, true>(BH, P.N, kp.M, kp.Bn, dS_final, dSc, dS0, P.gate, st);
     if (err != cudaSuccess) return err;
     if ((err = each(k_bwd<Tin, D, PASSES, CF>, "k_bwd", dyn_b)) != cudaSuccess) return err;
     void* out[7] = {dq, dk, dv, dg, de, dw, dgamma};

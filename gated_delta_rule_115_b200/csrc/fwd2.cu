@@ -1,0 +1,885 @@
+// fwd2.cu -- chunkwise forward on the 5th-generation tensor cores with every
+// per-chunk intermediate held in shared memory and tensor memory.
+//
+// Scope: bf16 inputs, dk = dv = 128, chunk C = 128, T a multiple of 128, and
+// chunks whose per-channel log decay over the chunk stays within the
+// single-pivot range (|sum g| <= 140, checked on the device by k2_span; larger
+// spans take the 8-token boundary-pivot path in chunk_impl.cuh).
+//
+// Per chunk (wolonglab.org page, "Methodology": each chunk is a unit-lower-
+// triangular system; fig:kernel: fused right-hand side, block inversion on the
+// matrix unit), with L = chunk-local cumulative log decay (log2 units inside),
+// P = L_C / 2 the per-channel pivot, q^ = gamma*q, a = e*k, u = w*v:
+//
+//   Kp = k 2^(L-P), Km = k 2^(P-L), Am = a 2^(P-L), Qp = q^ 2^(L-P)
+//   L_A = strict(Kp Am^T), L_K = strict(Kp Km^T)           (bf16 operands)
+//   M_QK = incl(Qp Km^T)  (bf16 hi/lo split: hi hi + hi lo + lo hi)
+//   M_QA = incl(Qp Am^T)                                     (bf16 operands)
+//   T = (I + L_A)^-1: 32x32 diagonal blocks by forward substitution (fp32),
+//       then block merges T21 = -T22 (L21 T11) for 32 -> 64 -> 128 on tcgen05
+//   X = [W | U'] = T [K~ | L_K U]   (K~ = k 2^L; one N = 256 MMA chain)
+//   Z = [Q' | O_intra] = [Q~ | M_QK U] - M_QA X              (Q~ = q^ 2^L)
+//   [M_n | B_n] = [diag(2^Lbar) | Kbar^T U] - Abar^T X       (Kbar = k 2^(Lbar-L), Abar = a 2^(Lbar-L))
+//
+// so that the chunk's output is O_n = Q'_n S_n + O_intra_n and the state
+// passes as S_{n+1} = M_n S_n + B_n (k2_chain, then k2_out).  Bounded-range
+// operands (T, U, L_K, L_K U, K~, X, M_QK, M_QA, Kbar, Abar) are fp16; the
+// pivoted ones span up to 2^+-101 and are bf16.  Accumulation is fp32 in TMEM.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "fwd2.h"
+#include "profile.h"
+#include "tc2.cuh"
+
+namespace muir {
+namespace v2 {
+
+using namespace t2;
+
+constexpr int kC = 128, kD = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLogDecayMin = -20.f;      // per-token clamp of g (natural log units)
+constexpr float kSpanMax = 140.f;          // single-pivot limit of |sum g| over a chunk
+
+__device__ unsigned int g_v2_timeouts;
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void bf16_split(float x, float& hi, float& lo) {
+    hi = __bfloat162float(__float2bfloat16_rn(x));
+    lo = x - hi;
+}
+
+// ------------------------------------------------------------------ span pre-pass
+
+// flags[0] = 1 if any chunk has a channel whose clamped log decay summed over
+// the chunk is below -kSpanMax.  One warp per (chunk, 32-channel quarter).
+__global__ void k2_span(const __nv_bfloat16* __restrict__ g, int B, int T, int H, int* flags) {
+    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
+    const int N = T / kC;
+    const long long nwork = (long long)B * H * N * 4;
+    if (warp >= nwork) return;
+    const int quarter = warp & 3;
+    const long long c = warp >> 2;
+    const int n = (int)(c % N);
+    const long long bh = c / N;
+    const int h = (int)(bh % H), b = (int)(bh / H);
+    const int j = 32 * quarter + lane;
+    const __nv_bfloat16* p = g + (((size_t)b * T + (size_t)n * kC) * H + h) * kD + j;
+    float s = 0.f;
+    for (int t = 0; t < kC; ++t) s += fmaxf(__bfloat162float(p[(size_t)t * H * kD]), kLogDecayMin);
+    if (__any_sync(0xffffffffu, s < -kSpanMax) && lane == 0) atomicOr(flags, 1);
+}
+
+// ------------------------------------------------------------------ k2_intra
+
+struct IntraSmem {
+    float tot[4][kC];   // per-quarter totals of the log-decay scan
+    float P2[kD];       // pivot (log2 units)
+    float eP2[kD];      // 2^P2
+    float Lb[kD];       // chunk total (log2 units)
+    uint64_t bar[16];
+    uint32_t tslot;
+    int bad;
+};
+
+enum { BA = 0, BB, BC, BD, BE, BF, BM1, BM2, BM3, BM4, BM5, BM6, BG };
+
+__device__ __forceinline__ bool waitb(IntraSmem& s, int i, uint32_t parity) {
+    const bool ok = mbar_wait(&s.bar[i], parity);
+    if (!ok) s.bad = 1;
+    return ok;
+}
+
+__device__ __forceinline__ void sync_all() {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+}
+
+// Load 64 values (this thread's row t, columns 64h..64h+63) of a bf16 T16 tile.
+__device__ __forceinline__ void row_ld64(const unsigned char* tile, int t, int h, float* v) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) ld_chunk16<true>(tile, t, 8 * h + i, v + 8 * i);
+}
+
+template <bool BF16>
+__device__ __forceinline__ void row_st64(unsigned char* tile, int t, int h, const float* v) {
+#pragma unroll
+    for (int i = 0; i < 8; ++i) st_chunk16<BF16>(tile, t, 8 * h + i, v + 8 * i);
+}
+
+// Read 64 TMEM columns [col, col + 64) of this thread's lane.
+__device__ __forceinline__ void tm_ld64(uint32_t tm, int q, int col, float* v) {
+    float a[32], b[32];
+    tmem_ld32(taddr(tm, 32 * q, col), a);
+    tmem_ld32(taddr(tm, 32 * q, col + 32), b);
+    tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) { v[i] = a[i]; v[32 + i] = b[i]; }
+}
+
+__global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ IntraParams p) {
+    extern __shared__ __align__(1024) unsigned char smraw[];
+    unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    unsigned char* S[6];
+#pragma unroll
+    for (int i = 0; i < 6; ++i) S[i] = sm + i * kT16Bytes;
+    IntraSmem& s = *reinterpret_cast<IntraSmem*>(sm + 6 * kT16Bytes);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, h = warp >> 2;
+    const int t = 32 * q + lane;  // row owned by this thread
+    const int N = p.T / kC;
+    const int nch = p.B * p.H * N;
+
+    if (tid == 0) {
+        for (int i = 0; i < 16; ++i) mbar_init(&s.bar[i], 1);
+        s.bad = 0;
+        fence_barrier_init();
+        prefetch_tmap(&p.tq); prefetch_tmap(&p.tk); prefetch_tmap(&p.tv); prefetch_tmap(&p.tg);
+        prefetch_tmap(&p.te); prefetch_tmap(&p.tw); prefetch_tmap(&p.tgam);
+    }
+    if (warp == 0) tmem_alloc(&s.tslot, 512);
+    sync_all();
+    const uint32_t tm = s.tslot;
+    const uint32_t a0 = saddr(S[0]), a1 = saddr(S[1]), a2 = saddr(S[2]), a3 = saddr(S[3]),
+                   a4 = saddr(S[4]), a5 = saddr(S[5]);
+
+    auto coords = [&](int c, int& y, int& z) {
+        const int n = c % N, bh = c / N;
+        y = bh % p.H;
+        z = (bh / p.H) * p.T + n * kC;
+    };
+    auto load_tile = [&](unsigned char* dst, const CUtensorMap* map, int y, int z, int bar) {
+        tma_load_3d(dst, map, 0, y, z, &s.bar[bar]);
+        tma_load_3d(dst + kT16Block, map, 64, y, z, &s.bar[bar]);
+    };
+    auto issue_first = [&](int c) {  // g, k, e on BA; q, gamma on BB
+        int y, z;
+        coords(c, y, z);
+        mbar_arrive_expect_tx(&s.bar[BA], 3 * kT16Bytes);
+        load_tile(S[0], &p.tg, y, z, BA);
+        load_tile(S[1], &p.tk, y, z, BA);
+        load_tile(S[2], &p.te, y, z, BA);
+        mbar_arrive_expect_tx(&s.bar[BB], 2 * kT16Bytes);
+        load_tile(S[3], &p.tq, y, z, BB);
+        load_tile(S[4], &p.tgam, y, z, BB);
+    };
+    if (tid == 0 && (int)blockIdx.x < nch) issue_first(blockIdx.x);
+
+    int it = 0;
+    for (int c = blockIdx.x; c < nch; c += gridDim.x, ++it) {
+        const uint32_t ph = (uint32_t)(it & 1);
+        uint32_t pg = 0;  // parity of the merge barrier within this chunk
+        int y, z;
+        coords(c, y, z);
+        const size_t cbase = (size_t)c * kC * kD;  // chunk offset in the per-chunk fp32 arrays
+
+        // ---- 1. log-decay prefix (warp scan over tokens), pivots, span
+        waitb(s, BA, ph);
+        float L[64];
+        row_ld64(S[0], t, h, L);
+#pragma unroll
+        for (int j = 0; j < 64; ++j) L[j] = fmaxf(L[j], kLogDecayMin) * kLog2e;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) {
+                const float o = __shfl_up_sync(0xffffffffu, L[j], off);
+                if (lane >= off) L[j] += o;
+            }
+        }
+        if (lane == 31) {
+#pragma unroll
+            for (int j = 0; j < 64; ++j) s.tot[q][64 * h + j] = L[j];
+        }
+        __syncthreads();
+#pragma unroll
+        for (int j = 0; j < 64; ++j) {
+            const int col = 64 * h + j;
+            float pre = 0.f;
+            for (int qq = 0; qq < q; ++qq) pre += s.tot[qq][col];
+            L[j] += pre;
+        }
+        if (q == 0) {
+            for (int jj = lane; jj < 64; jj += 32) {
+                const int col = 64 * h + jj;
+                const float lb = s.tot[0][col] + s.tot[1][col] + s.tot[2][col] + s.tot[3][col];
+                s.Lb[col] = lb;
+                s.P2[col] = 0.5f * lb;
+                s.eP2[col] = ex2(0.5f * lb);
+            }
+        }
+        __syncthreads();
+
+        // ---- 2. pivoted key operands: Kp -> S0, Km (hi) -> S1, Km (lo) -> S2, Am -> S5
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {
+            float kv[8], ev[8], kp[8], kmh[8], kml[8], am[8];
+            ld_chunk16<true>(S[1], t, 8 * h + i, kv);
+            ld_chunk16<true>(S[2], t, 8 * h + i, ev);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = 8 * i + u;
+                const float pv = s.P2[64 * h + j];
+                const float ep = ex2(L[j] - pv), em = ex2(pv - L[j]);
+                kp[u] = kv[u] * ep;
+                bf16_split(kv[u] * em, kmh[u], kml[u]);
+                am[u] = ev[u] * kv[u] * em;
+            }
+            st_chunk16<true>(S[0], t, 8 * h + i, kp);
+            st_chunk16<true>(S[1], t, 8 * h + i, kmh);
+            st_chunk16<true>(S[2], t, 8 * h + i, kml);
+            st_chunk16<true>(S[5], t, 8 * h + i, am);
+        }
+        fence_async_smem();
+        sync_all();
+        if (tid == 0) {
+            gemm_kk16(tm + 0, a0, 0, a5, 0, 0, 128, 128, kBF16, false);    // L_A
+            gemm_kk16(tm + 128, a0, 0, a1, 0, 0, 128, 128, kBF16, false);  // L_K
+            mma_commit(&s.bar[BM1]);
+        }
+
+        // ---- 3. query operands: Qp hi -> S3, Qp lo -> S4; Q~ -> Qp_out (fp32, completed in step 8)
+        waitb(s, BB, ph);
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {
+            float qv[8], gv[8], qh[8], ql[8];
+            ld_chunk16<true>(S[3], t, 8 * h + i, qv);
+            ld_chunk16<true>(S[4], t, 8 * h + i, gv);
+            float qt[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = 8 * i + u;
+                const float pv = s.P2[64 * h + j];
+                const float qhat = qv[u] * gv[u];
+                const float qp = qhat * ex2(L[j] - pv);
+                bf16_split(qp, qh[u], ql[u]);
+                qt[u] = qhat * ex2(L[j]);
+            }
+            st_chunk16<true>(S[3], t, 8 * h + i, qh);
+            st_chunk16<true>(S[4], t, 8 * h + i, ql);
+            float* dst = p.Qp + cbase + (size_t)t * kD + 64 * h + 8 * i;
+            *reinterpret_cast<float4*>(dst) = make_float4(qt[0], qt[1], qt[2], qt[3]);
+            *reinterpret_cast<float4*>(dst + 4) = make_float4(qt[4], qt[5], qt[6], qt[7]);
+        }
+        fence_async_smem();
+        sync_all();
+        if (tid == 0) {
+            gemm_kk16(tm + 256, a3, 0, a1, 0, 0, 128, 128, kBF16, false);  // M_QK: hi hi
+            gemm_kk16(tm + 256, a3, 0, a2, 0, 0, 128, 128, kBF16, true);   //       hi lo
+            gemm_kk16(tm + 256, a4, 0, a1, 0, 0, 128, 128, kBF16, true);   //       lo hi
+            gemm_kk16(tm + 384, a3, 0, a5, 0, 0, 128, 128, kBF16, false);  // M_QA
+            mma_commit(&s.bar[BM2]);
+        }
+
+        // ---- 4. L_A -> LA16 (S0), leaves of T, L_K -> LK16 (S1)
+        waitb(s, BM1, ph);
+        tc_fence_after();
+        float la[64];
+        tm_ld64(tm + 64 * h, q, 0, la);  // L_A row t, columns 64h..
+        {
+            float v[64];
+#pragma unroll
+            for (int j = 0; j < 64; ++j) v[j] = (64 * h + j < t) ? la[j] : 0.f;
+            row_st64<false>(S[0], t, h, v);
+        }
+        // diagonal 32x32 block q of T: warp (q, q >> 1) holds L_A[32q + lane][32q .. 32q + 31]
+        float tcol[32];
+        const bool leaf = (h == (q >> 1));
+        if (leaf) {
+            const int off = 32 * (q & 1);  // block columns inside this thread's 64
+            float lrow[32];
+#pragma unroll
+            for (int k = 0; k < 32; ++k) lrow[k] = (k < lane) ? la[off + k] : 0.f;
+            // lane = column c of the block; tcol[r] = T[r][c]
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                float acc = (r == lane) ? 1.f : 0.f;
+#pragma unroll
+                for (int k = 0; k < r; ++k) acc -= __shfl_sync(0xffffffffu, lrow[k], r) * tcol[k];
+                tcol[r] = acc;
+            }
+        }
+        waitb(s, BM2, ph);  // S1..S5 free
+        tc_fence_after();
+        {
+            float lk[64];
+            tm_ld64(tm + 128 + 64 * h, q, 0, lk);
+#pragma unroll
+            for (int j = 0; j < 64; ++j) lk[j] = (64 * h + j < t) ? lk[j] : 0.f;
+            row_st64<false>(S[1], t, h, lk);
+        }
+        // T (S2): zeros outside the diagonal blocks, leaves written column-wise
+        {
+            float z8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const int c0 = 64 * h + 8 * i;
+                if (c0 >= 32 * q && c0 < 32 * q + 32) continue;  // diagonal block
+                st_chunk16<false>(S[2], t, 8 * h + i, z8);
+            }
+        }
+        if (leaf) {
+            const int col = 32 * q + lane;
+#pragma unroll
+            for (int r = 0; r < 32; ++r) {
+                const int row = 32 * q + r;
+                __half hv = __float2half_rn(tcol[r]);
+                *reinterpret_cast<__half*>(S[2] + t16_off(row, col >> 3) + (col & 7) * 2) = hv;
+            }
+        }
+        if (tid == 0) {  // v -> S4, w -> S5
+            mbar_arrive_expect_tx(&s.bar[BC], 2 * kT16Bytes);
+            load_tile(S[4], &p.tv, y, z, BC);
+            load_tile(S[5], &p.tw, y, z, BC);
+        }
+        fence_async_smem();
+        sync_all();
+
+        // ---- 5. block merges of T on tcgen05: P = L21 T11 (into B0), T21 = -T22 P (into B1)
+        for (int lvl = 0; lvl < 2; ++lvl) {
+            const int b = lvl == 0 ? 32 : 64;
+            if (tid == 0) {
+                for (int pr = 0; pr < 128 / (2 * b); ++pr) {
+                    const int F = 2 * b * pr;
+                    gemm_km16(tm + F, a0, F, a2, F, F, b, b, kF16, false);
+                }
+                mma_commit(&s.bar[BG]);
+            }
+            waitb(s, BG, pg); pg ^= 1;
+            tc_fence_after();
+            // rows of the second halves: level 32 -> quarters 1, 3 (pair q >> 1, columns 64 (q>>1) .. +32)
+            //                            level 64 -> quarters 2, 3 (columns 0 .. 63)
+            const bool mine = (lvl == 0) ? ((q & 1) && h == (q >> 1)) : (q >= 2 && h == 0);
+            const int F = (lvl == 0) ? 64 * (q >> 1) : 0;
+            if (mine) {
+                float v[64];
+                if (b == 32) {
+                    float a[32];
+                    tmem_ld32(taddr(tm, 32 * q, F), a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) st_chunk16<false>(S[3], t, F / 8 + i, a + 8 * i);
+                } else {
+                    tm_ld64(tm, q, 0, v);
+                    row_st64<false>(S[3], t, 0, v);
+                }
+            } else if (b == 32) {
+                tmem_wait_ld();  // keep the warp's tcgen05.ld bookkeeping uniform
+            }
+            fence_async_smem();
+            sync_all();
+            if (tid == 0) {
+                for (int pr = 0; pr < 128 / (2 * b); ++pr) {
+                    const int F2 = 2 * b * pr;
+                    gemm_km16(tm + 128 + F2, a2, F2 + b, a3, F2 + b, F2, b, b, kF16, false, true);
+                }
+                mma_commit(&s.bar[BG]);
+            }
+            waitb(s, BG, pg); pg ^= 1;
+            tc_fence_after();
+            if (mine) {
+                if (b == 32) {
+                    float a[32];
+                    tmem_ld32(taddr(tm + 128, 32 * q, F), a);
+                    tmem_wait_ld();
+#pragma unroll
+                    for (int i = 0; i < 4; ++i) st_chunk16<false>(S[2], t, F / 8 + i, a + 8 * i);
+                } else {
+                    float v[64];
+                    tm_ld64(tm + 128, q, 0, v);
+                    row_st64<false>(S[2], t, 0, v);
+                }
+            }
+            fence_async_smem();
+            sync_all();
+        }
+
+        // ---- 6. U = w v (S4, in place); L_K U (B0); K~ (S0); X = T [K~ | L_K U] (B0..B1)
+        waitb(s, BC, ph);
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {
+            float vv[8], wv[8];
+            ld_chunk16<true>(S[4], t, 8 * h + i, vv);
+            ld_chunk16<true>(S[5], t, 8 * h + i, wv);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) vv[u] *= wv[u];
+            st_chunk16<false>(S[4], t, 8 * h + i, vv);
+        }
+        fence_async_smem();
+        sync_all();
+        if (tid == 0) {
+            gemm_km16(tm + 0, a1, 0, a4, 0, 0, 128, 128, kF16, false);  // L_K U
+            mma_commit(&s.bar[BM3]);
+            mbar_arrive_expect_tx(&s.bar[BD], kT16Bytes);                // k -> S0
+            load_tile(S[0], &p.tk, y, z, BD);
+        }
+        waitb(s, BD, ph);
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {
+            float kv[8];
+            ld_chunk16<true>(S[0], t, 8 * h + i, kv);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) kv[u] *= ex2(L[8 * i + u]);
+            st_chunk16<false>(S[0], t, 8 * h + i, kv);
+        }
+        waitb(s, BM3, ph);
+        tc_fence_after();
+        {
+            float v[64];
+            tm_ld64(tm + 64 * h, q, 0, v);
+            row_st64<false>(S[1], t, h, v);
+        }
+        fence_async_smem();
+        sync_all();
+        if (tid == 0) {
+            gemm_km16(tm + 0, a2, 0, a0, 0, 0, 256, 128, kF16, false);  // X = T [K~ | L_K U]
+            mma_commit(&s.bar[BM4]);
+        }
+        // M_QK (B2) -> S3, M_QA (B3) -> S5 (inclusive masks)
+        {
+            float v[64];
+            tm_ld64(tm + 256 + 64 * h, q, 0, v);
+#pragma unroll
+            for (int j = 0; j < 64; ++j) v[j] = (64 * h + j <= t) ? v[j] : 0.f;
+            row_st64<false>(S[3], t, h, v);
+            tm_ld64(tm + 384 + 64 * h, q, 0, v);
+#pragma unroll
+            for (int j = 0; j < 64; ++j) v[j] = (64 * h + j <= t) ? v[j] : 0.f;
+            row_st64<false>(S[5], t, h, v);
+        }
+        waitb(s, BM4, ph);
+        tc_fence_after();
+        {
+            float v[64];
+            tm_ld64(tm + 64 * h, q, 0, v);        // W
+            row_st64<false>(S[0], t, h, v);
+            tm_ld64(tm + 128 + 64 * h, q, 0, v);  // U'
+            row_st64<false>(S[1], t, h, v);
+        }
+        fence_async_smem();
+        sync_all();
+
+        // ---- 7. Z = [Q~ | M_QK U] - M_QA [W | U'] (B2..B3)
+        if (tid == 0) {
+            gemm_km16(tm + 256, a5, 0, a0, 0, 0, 256, 128, kF16, false, true);
+            gemm_km16(tm + 384, a3, 0, a4, 0, 0, 128, 128, kF16, true);
+            mma_commit(&s.bar[BM5]);
+            mbar_arrive_expect_tx(&s.bar[BE], kT16Bytes);  // k -> S2
+            load_tile(S[2], &p.tk, y, z, BE);
+        }
+        waitb(s, BM5, ph);
+        tc_fence_after();
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&s.bar[BF], kT16Bytes);  // e -> S3
+            load_tile(S[3], &p.te, y, z, BF);
+        }
+        {
+            float v[64];
+            tm_ld64(tm + 256 + 64 * h, q, 0, v);
+            float* qd = p.Qp + cbase + (size_t)t * kD + 64 * h;
+#pragma unroll
+            for (int j = 0; j < 64; j += 4) {
+                float4 a = *reinterpret_cast<const float4*>(qd + j);
+                a.x += v[j]; a.y += v[j + 1]; a.z += v[j + 2]; a.w += v[j + 3];
+                *reinterpret_cast<float4*>(qd + j) = a;
+            }
+            tm_ld64(tm + 384 + 64 * h, q, 0, v);
+            float* od = p.Oi + cbase + (size_t)t * kD + 64 * h;
+#pragma unroll
+            for (int j = 0; j < 64; j += 4)
+                *reinterpret_cast<float4*>(od + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        }
+        waitb(s, BE, ph);
+        waitb(s, BF, ph);
+#pragma unroll 1
+        for (int i = 0; i < 8; ++i) {
+            float kv[8], ev[8];
+            ld_chunk16<true>(S[2], t, 8 * h + i, kv);
+            ld_chunk16<true>(S[3], t, 8 * h + i, ev);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const int j = 8 * i + u;
+                const float pv = s.P2[64 * h + j];
+                const float f = ex2(pv - L[j]) * s.eP2[64 * h + j];  // 2^(Lbar - L)
+                kv[u] *= f;
+                ev[u] *= kv[u];
+            }
+            st_chunk16<false>(S[2], t, 8 * h + i, kv);
+            st_chunk16<false>(S[3], t, 8 * h + i, ev);
+        }
+        fence_async_smem();
+        sync_all();
+
+        // ---- 8. [M_n | B_n] = [diag 2^Lbar | Kbar^T U] - Abar^T [W | U'] (B0..B1)
+        if (tid == 0) {
+            gemm_mm16(tm + 0, a3, 0, 0, a0, 0, 0, 256, 128, kF16, false, true);
+            gemm_mm16(tm + 128, a2, 0, 0, a4, 0, 0, 128, 128, kF16, true);
+            mma_commit(&s.bar[BM6]);
+        }
+        waitb(s, BM6, ph);
+        tc_fence_after();
+        const int cn = c + gridDim.x;
+        if (tid == 0 && cn < nch) issue_first(cn);
+        {
+            float v[64];
+            tm_ld64(tm + 64 * h, q, 0, v);
+            float* md = p.M + cbase + (size_t)t * kD + 64 * h;
+            const float dg = ex2(s.Lb[t]);
+#pragma unroll
+            for (int j = 0; j < 64; ++j)
+                if (64 * h + j == t) v[j] += dg;
+#pragma unroll
+            for (int j = 0; j < 64; j += 4)
+                *reinterpret_cast<float4*>(md + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            if (p.Mt) {
+                float* mt = p.Mt + cbase + t;
+#pragma unroll 8
+                for (int j = 0; j < 64; ++j) mt[(size_t)(64 * h + j) * kD] = v[j];
+            }
+            tm_ld64(tm + 128 + 64 * h, q, 0, v);
+            float* bd = p.Bn + cbase + (size_t)t * kD + 64 * h;
+#pragma unroll
+            for (int j = 0; j < 64; j += 4)
+                *reinterpret_cast<float4*>(bd + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        }
+        sync_all();  // TMEM read out before the next chunk's products
+    }
+    if (tid == 0 && s.bad) atomicAdd(&g_v2_timeouts, 1u);
+    sync_all();
+    if (warp == 0) tmem_dealloc(tm, 512);
+}
+
+// ------------------------------------------------------------------ k2_chain
+
+// S_{n+1} = M_n S_n + B_n for one head and SLAB value columns; 128 threads,
+// thread j owns row j.  M_n streams through a 3-stage TMA ring (K-major TF32
+// tiles); S_n^T sits in a K-major TF32 tile of SLAB rows (the B operand).
+// Records S_n (chunk-start states) and writes S_N to S_final.
+template <int SLAB>
+__global__ void __launch_bounds__(128, 1) k2_chain(const __grid_constant__ ChainParams p) {
+    constexpr int STAGES = 3;
+    constexpr uint32_t MT = 128 * 128 * 4;  // one transition tile
+    extern __shared__ __align__(1024) unsigned char smraw[];
+    unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    unsigned char* Mst = sm;                       // STAGES x 64 KB
+    unsigned char* St = sm + STAGES * MT;          // SLAB x 128 fp32, K-major
+    __shared__ uint64_t bar[STAGES + 1];
+    __shared__ uint32_t tslot;
+    __shared__ int bad;
+
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int nslab = kD / SLAB;
+    const int bh = blockIdx.x / nslab, c0 = (blockIdx.x % nslab) * SLAB;
+    const int N = p.N;
+    const int j = tid;
+    if (tid == 0) {
+        for (int i = 0; i <= STAGES; ++i) mbar_init(&bar[i], 1);
+        bad = 0;
+        fence_barrier_init();
+        prefetch_tmap(&p.tM);
+    }
+    if (warp == 0) tmem_alloc(&tslot, 32 < SLAB ? SLAB : 32);
+    sync_all();
+    const uint32_t tm = tslot;
+    const long long row0 = (long long)bh * N * kD;  // first row of this head's transitions
+    auto issue = [&](int n) {
+        const int st = n % STAGES;
+        mbar_arrive_expect_tx(&bar[st], MT);
+        for (int kb = 0; kb < 4; ++kb)
+            tma_load_3d(Mst + st * MT + kb * 128 * 128, &p.tM, 32 * kb, (int)(row0 + (long long)n * kD), 0,
+                        &bar[st]);
+    };
+    if (tid == 0)
+        for (int n = 0; n < STAGES && n < N; ++n) issue(n);
+
+    // initial state row j, columns c0 .. c0 + SLAB
+    float Sr[SLAB];
+    const size_t sbase = ((size_t)bh * kD + j) * kD + c0;
+#pragma unroll
+    for (int c = 0; c < SLAB; ++c) Sr[c] = p.S0 ? p.S0[sbase + c] : 0.f;
+    auto put_state = [&]() {
+#pragma unroll
+        for (int c = 0; c < SLAB; ++c)
+            *reinterpret_cast<float*>(St + t32_off<SLAB>(c, j >> 2) + (j & 3) * 4) = Sr[c];
+    };
+    put_state();
+    float Bnext[SLAB];
+    auto load_B = [&](int n, float* dst) {
+        const float* src = p.Bn + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
+#pragma unroll
+        for (int c = 0; c < SLAB; c += 4) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(src + c));
+            dst[c] = v.x; dst[c + 1] = v.y; dst[c + 2] = v.z; dst[c + 3] = v.w;
+        }
+    };
+    if (N > 0) load_B(0, Bnext);
+    fence_async_smem();
+    sync_all();
+    for (int n = 0; n < N; ++n) {
+        const int st = n % STAGES;
+        if (p.S_chunks) {
+            float* d = p.S_chunks + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
+#pragma unroll
+            for (int c = 0; c < SLAB; c += 4) *reinterpret_cast<float4*>(d + c) = make_float4(Sr[c], Sr[c + 1], Sr[c + 2], Sr[c + 3]);
+        }
+        if (!mbar_wait(&bar[st], (uint32_t)((n / STAGES) & 1))) bad = 1;
+        if (tid == 0) {
+            tc_fence_after();
+            gemm_kk32<128, SLAB>(tm, saddr(Mst + st * MT), saddr(St), 0, SLAB, 128, false);
+            mma_commit(&bar[STAGES]);
+        }
+        float Bc[SLAB];
+#pragma unroll
+        for (int c = 0; c < SLAB; ++c) Bc[c] = Bnext[c];
+        if (n + 1 < N) load_B(n + 1, Bnext);
+        if (!mbar_wait(&bar[STAGES], (uint32_t)(n & 1))) bad = 1;
+        tc_fence_after();
+        if (tid == 0 && n + STAGES < N) issue(n + STAGES);
+        float d[32];
+        tmem_ld32(taddr(tm, 32 * warp, 0), d);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < SLAB; ++c) Sr[c] = d[c] + Bc[c];
+        put_state();
+        fence_async_smem();
+        sync_all();
+    }
+    if (p.S_final) {
+        float* d = p.S_final + sbase;
+#pragma unroll
+        for (int c = 0; c < SLAB; c += 4) *reinterpret_cast<float4*>(d + c) = make_float4(Sr[c], Sr[c + 1], Sr[c + 2], Sr[c + 3]);
+    }
+    if (tid == 0 && bad) atomicAdd(&g_v2_timeouts, 1u);
+    sync_all();
+    if (warp == 0) tmem_dealloc(tm, 32 < SLAB ? SLAB : 32);
+}
+
+// ------------------------------------------------------------------ k2_out
+
+// O_n = Q'_n S_n + O_intra_n per chunk (TF32 products, fp32 accumulation).
+// Persistent, 256 threads; Q'_n by TMA (K-major TF32 tile), S_n^T written by
+// the threads into a K-major TF32 tile.
+template <typename Tout>
+__global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutParams p) {
+    constexpr uint32_t MT = 128 * 128 * 4;
+    extern __shared__ __align__(1024) unsigned char smraw[];
+    unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    unsigned char* Qt = sm;
+    unsigned char* St = sm + MT;
+    __shared__ uint64_t bar[2];
+    __shared__ uint32_t tslot;
+    __shared__ int bad;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, h = warp >> 2, t = 32 * q + lane;
+    const int N = p.T / kC, nch = p.B * p.H * N;
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        bad = 0;
+        fence_barrier_init();
+        prefetch_tmap(&p.tQ);
+    }
+    if (warp == 0) tmem_alloc(&tslot, 128);
+    sync_all();
+    const uint32_t tm = tslot;
+    auto issue = [&](int c) {
+        mbar_arrive_expect_tx(&bar[0], MT);
+        for (int kb = 0; kb < 4; ++kb)
+            tma_load_3d(Qt + kb * 128 * 128, &p.tQ, 32 * kb, c * kC, 0, &bar[0]);
+    };
+    if (tid == 0 && (int)blockIdx.x < nch) issue(blockIdx.x);
+    int it = 0;
+    for (int c = blockIdx.x; c < nch; c += gridDim.x, ++it) {
+        // S_n^T into St: thread (row r = tid / 2, half) reads 64 values of S_n row r
+        {
+            const int r = tid >> 1, hf = tid & 1;
+            const float* src = p.S_chunks + (size_t)c * kD * kD + (size_t)r * kD + 64 * hf;
+#pragma unroll 4
+            for (int cc = 0; cc < 64; cc += 4) {
+                const float4 v = __ldg(reinterpret_cast<const float4*>(src + cc));
+                const float vv[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const int col = 64 * hf + cc + u;  // B row (value column), K index r
+                    *reinterpret_cast<float*>(St + t32_off<128>(col, r >> 2) + (r & 3) * 4) = vv[u];
+                }
+            }
+        }
+        fence_async_smem();
+        sync_all();
+        if (!mbar_wait(&bar[0], (uint32_t)(it & 1))) bad = 1;
+        if (tid == 0) {
+            tc_fence_after();
+            gemm_kk32<128, 128>(tm, saddr(Qt), saddr(St), 0, 128, 128, false);
+            mma_commit(&bar[1]);
+        }
+        if (!mbar_wait(&bar[1], (uint32_t)(it & 1))) bad = 1;
+        tc_fence_after();
+        const int cn = c + gridDim.x;
+        if (tid == 0 && cn < nch) issue(cn);
+        // epilogue: o[b][n*C + t][h][64 hh ..] = D + O_intra
+        const int n = c % N, bh = c / N, hd = bh % p.H, b = bh / p.H;
+        float v[64];
+        tm_ld64(tm + 64 * h, q, 0, v);
+        const float* oi = p.Oi + (size_t)c * kC * kD + (size_t)t * kD + 64 * h;
+        Tout* od = reinterpret_cast<Tout*>(p.o) + (((size_t)b * p.T + (size_t)n * kC + t) * p.H + hd) * kD + 64 * h;
+#pragma unroll
+        for (int jj = 0; jj < 64; jj += 4) {
+            const float4 a = __ldg(reinterpret_cast<const float4*>(oi + jj));
+            const float r0 = v[jj] + a.x, r1 = v[jj + 1] + a.y, r2 = v[jj + 2] + a.z, r3 = v[jj + 3] + a.w;
+            if constexpr (sizeof(Tout) == 4) {
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(od) + jj) = make_float4(r0, r1, r2, r3);
+            } else {
+                uint2 u;
+                u.x = pack_bf16(r0, r1);
+                u.y = pack_bf16(r2, r3);
+                *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(od) + jj) = u;
+            }
+        }
+        sync_all();
+    }
+    if (tid == 0 && bad) atomicAdd(&g_v2_timeouts, 1u);
+    sync_all();
+    if (warp == 0) tmem_dealloc(tm, 128);
+}
+
+// ------------------------------------------------------------------ host side
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+static EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    if (!fn) {
+        void* f = nullptr;
+        cudaDriverEntryPointQueryResult qr;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &f, cudaEnableDefault, &qr) ==
+                cudaSuccess &&
+            qr == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(f);
+    }
+    return fn;
+}
+
+// Map over a token-major [B*T][H][128] bf16 tensor: box of 64 channels x 1 head x 128 tokens.
+static bool map_tokens(CUtensorMap* m, const void* base, int B, int T, int H) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)B * T};
+    cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
+    cuuint32_t box[3] = {64, 1, (cuuint32_t)kC};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Map over rows of 128 fp32 (a [rows][128] array): box of 32 columns x 128 rows.
+static bool map_rows32(CUtensorMap* m, const float* base, long long rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc) return false;
+    cuuint64_t dims[3] = {128, (cuuint64_t)rows, 1};
+    cuuint64_t strides[2] = {128 * 4, (cuuint64_t)rows * 128 * 4};
+    cuuint32_t box[3] = {32, 128, 1};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<float*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+static int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+constexpr int kIntraSmem = 6 * kT16Bytes + sizeof(IntraSmem) + 1024;
+constexpr int kOutSmem = 2 * 128 * 128 * 4 + 1024;
+template <int SLAB>
+constexpr int chain_smem() { return 3 * 128 * 128 * 4 + SLAB * 512 + 1024; }
+
+size_t fwd2_ws_bytes(int B, int T, int H) {
+    const size_t nch = (size_t)B * H * (T / kC), CD = (size_t)kC * kD;
+    // M, Bn, Q', O_intra, S_chunks, flags
+    return (5 * nch * CD) * sizeof(float) + 256;
+}
+
+bool fwd2_supported(int B, int T, int H, int D, int C, bool in_bf16) {
+    return in_bf16 && D == kD && C == kC && T > 0 && T % kC == 0 && B > 0 && H > 0;
+}
+
+cudaError_t span_check(const void* g, int B, int T, int H, int* flags, cudaStream_t st) {
+    const long long warps = (long long)B * H * (T / kC) * 4;
+    const int blocks = (int)((warps * 32 + 255) / 256);
+    MUIR_TIMED("k2_span", st, k2_span<<<blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(g), B, T, H, flags));
+    return cudaGetLastError();
+}
+
+cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st) {
+    if (!encode_fn()) return cudaErrorNotSupported;
+    const int N = a.T / kC, nch = a.B * a.H * N, BH = a.B * a.H;
+    IntraParams ip;
+    if (!map_tokens(&ip.tq, a.q, a.B, a.T, a.H) || !map_tokens(&ip.tk, a.k, a.B, a.T, a.H) ||
+        !map_tokens(&ip.tv, a.v, a.B, a.T, a.H) || !map_tokens(&ip.tg, a.g, a.B, a.T, a.H) ||
+        !map_tokens(&ip.te, a.e, a.B, a.T, a.H) || !map_tokens(&ip.tw, a.w, a.B, a.T, a.H) ||
+        !map_tokens(&ip.tgam, a.gamma, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    ip.B = a.B; ip.T = a.T; ip.H = a.H;
+    ip.M = a.M; ip.Mt = a.Mt; ip.Bn = a.Bn; ip.Qp = a.Qp; ip.Oi = a.Oi; ip.flags = a.flags;
+    cudaError_t e = cudaFuncSetAttribute(k2_intra, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);
+    if (e != cudaSuccess) return e;
+    const int nsm = sm_count();
+    const int grid = nch < nsm ? nch : nsm;
+    MUIR_TIMED("k2_intra", st, k2_intra<<<grid, 256, kIntraSmem, st>>>(ip));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    constexpr int SLAB = 32;
+    ChainParams cp;
+    if (!map_rows32(&cp.tM, a.M, (long long)nch * kD)) return cudaErrorInvalidValue;
+    cp.Bn = a.Bn; cp.S0 = a.S0; cp.S_chunks = a.S_chunks; cp.S_final = a.S_final; cp.N = N;
+    e = cudaFuncSetAttribute(k2_chain<SLAB>, cudaFuncAttributeMaxDynamicSharedMemorySize, chain_smem<SLAB>());
+    if (e != cudaSuccess) return e;
+    MUIR_TIMED("k2_chain", st, k2_chain<SLAB><<<BH * (kD / SLAB), 128, chain_smem<SLAB>(), st>>>(cp));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    if (a.o) {
+        OutParams op;
+        if (!map_rows32(&op.tQ, a.Qp, (long long)nch * kC)) return cudaErrorInvalidValue;
+        op.B = a.B; op.T = a.T; op.H = a.H;
+        op.S_chunks = a.S_chunks; op.Oi = a.Oi; op.o = a.o;
+        if (a.out_bf16) {
+            e = cudaFuncSetAttribute(k2_out<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
+            if (e != cudaSuccess) return e;
+            MUIR_TIMED("k2_out", st, k2_out<__nv_bfloat16><<<grid, 256, kOutSmem, st>>>(op));
+        } else {
+            e = cudaFuncSetAttribute(k2_out<float>, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
+            if (e != cudaSuccess) return e;
+            MUIR_TIMED("k2_out", st, k2_out<float><<<grid, 256, kOutSmem, st>>>(op));
+        }
+        if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+    return cudaSuccess;
+}
+
+unsigned int timeouts_v2() {
+    unsigned int n = 0;
+    cudaMemcpyFromSymbol(&n, g_v2_timeouts, sizeof(n));
+    const unsigned int z = 0;
+    cudaMemcpyToSymbol(g_v2_timeouts, &z, sizeof(z));
+    return n;
+}
+
+}  // namespace v2
+}  // namespace muir

@@ -22,6 +22,7 @@ struct ChunkProblem {
     bool in_bf16, out_bf16;
     const void *q, *k, *v, *g, *e, *w, *gamma;
     float* aux;            // per-chunk saved intermediates (forward: written; backward: read) or null
+    const int* gate;       // non-null: every kernel returns at once unless *gate != 0
 };
 
 // Up to eight tensors moved between token-major [B][T][H][D] rows of the
@@ -42,7 +43,7 @@ cudaError_t tail_scatter(const TailCopy& io, int B, int H, int T, int C, int D, 
 size_t chunk_aux_floats(int C, int D);
 
 // Workspace carving (bytes) for the chunk forward / backward.
-size_t chunk_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states);
+size_t chunk_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states, bool in_bf16);
 size_t chunk_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states);
 
 cudaError_t run_chunk_fwd(const ChunkProblem& P, const float* S0, void* o, float* S_final,
