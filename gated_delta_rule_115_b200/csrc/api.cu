@@ -5,6 +5,7 @@
 
 #include "../../include/muir.h"
 #include "chunk_units.h"
+#include "bwd2.h"
 #include "fwd2.h"
 #include "kernels.h"
 
@@ -70,7 +71,7 @@ size_t varlen_ws_bytes(const muir_shape* s, int num_seqs, const long long* cu, b
     for (int i = 0; i < num_seqs; ++i) {
         const int L = (int)(cu[i + 1] - cu[i]);
         if (L == 0) continue;
-        const size_t b = bwd ? muir::chunk_bwd_ws_bytes(1, L, s->H, s->dk, s->chunk, false)
+        const size_t b = bwd ? muir::chunk_bwd_ws_bytes(1, L, s->H, s->dk, s->chunk, false, s->in_dtype == MUIR_BF16)
                              : muir::chunk_fwd_ws_bytes(1, L, s->H, s->dk, s->chunk, false, s->in_dtype == MUIR_BF16);
         if (b > need) need = b;
     }
@@ -107,13 +108,13 @@ muir_status muir_device_wait_status(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MUIR_ERR_CUDA;
     const unsigned int n = muir::timeouts_bf16_d128() + muir::timeouts_bf16_d64() +
                            muir::timeouts_f32_d128() + muir::timeouts_f32_d64() +
-                           muir::v2::timeouts_v2();
+                           muir::v2::timeouts_v2() + muir::v2::timeouts_bwd2();
     return n ? MUIR_ERR_DEVICE_TIMEOUT : MUIR_OK;
 }
 
 size_t muir_chunk_aux_floats(const muir_shape* s) {
     if (check_shape(s) != MUIR_OK) return 0;
-    return (size_t)s->B * s->H * ((s->T + s->chunk - 1) / s->chunk) * muir::chunk_aux_floats(s->chunk, s->dk);
+    return muir::chunk_aux_total_floats(s->B, s->T, s->H, s->dk, s->chunk, s->in_dtype == MUIR_BF16);
 }
 
 size_t muir_chunk_fwd_workspace(const muir_shape* s) {
@@ -124,7 +125,8 @@ size_t muir_chunk_fwd_workspace(const muir_shape* s) {
 
 size_t muir_chunk_bwd_workspace(const muir_shape* s) {
     if (check_shape(s) != MUIR_OK) return 0;
-    return muir::chunk_bwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false);
+    return muir::chunk_bwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false,
+                                    s->in_dtype == MUIR_BF16);
 }
 
 muir_status muir_chunk_fwd(const muir_shape* s, const void* q, const void* k, const void* v,
@@ -163,7 +165,7 @@ muir_status muir_chunk_bwd(const muir_shape* s, const void* q, const void* k, co
         !ok_opt(aux) || (aux && !S_chunks))
         return MUIR_ERR_INVALID_ARG;
     const size_t need = muir::chunk_bwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk,
-                                                 S_chunks != nullptr);
+                                                 S_chunks != nullptr, s->in_dtype == MUIR_BF16);
     if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
     if ((st = check_device()) != MUIR_OK) return st;
     muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);

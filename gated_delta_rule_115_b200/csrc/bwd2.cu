@@ -1,0 +1,1079 @@
+// bwd2.cu -- chunkwise backward on the 5th-generation tensor cores, every
+// per-chunk intermediate on chip (companion of fwd2.cu: bf16 inputs,
+// dk = dv = 128, chunk 128).
+//
+// Gradients of L = sum(o * dO) + sum(S_N * dS_N) ("custom backward pass",
+// wolonglab.org page, "Methodology"), from the chunk form the forward uses,
+//   O_n = Q'_n S_n + O_intra_n,   S_{n+1} = M_n S_n + B_n,
+// with Y = W S + U' (Y_t = k_t^T D_t S_{t-1}):
+//
+//   reverse state pass  G_n = M_n^T G_{n+1} + Q'_n^T dO_n      (G_n = dL/dS_n)
+//   per chunk, with G = G_{n+1}:
+//     dY  = -M_QA^T dO - Abar G            dYR = T^T dY
+//     dU  = M_QK^T dO + Kbar G + L_K^T dYR          -> dv = dU w, dw = dU v
+//     dQ~ = dO S^T,  dK~ = dYR S^T,  dKbar = U G^T,  dAbar = -Y G^T
+//     dL_A = -strict(dYR Y^T), dL_K = strict(dYR U^T),
+//     dM_QA = -incl(dO Y^T),   dM_QK = incl(dO U^T)
+//     decay-masked gradients (pivoted operands as in the forward):
+//       dKp = dL_A Am + dL_K Km,      dQp = dM_QK Km + dM_QA Am,
+//       dAm = dL_A^T Kp + dM_QA^T Qp, dKm = dL_K^T Kp + dM_QK^T Qp
+//     dq^ = dQp 2^(L-P) + dQ~ 2^L,  da = dAm 2^(P-L) + dAbar 2^(Lbar-L)
+//     dk  = dKp 2^(L-P) + dKm 2^(P-L) + dK~ 2^L + dKbar 2^(Lbar-L) + e da
+//     dLog = dKp Kp + dQp Qp - dKm Km - dAm Am + dK~ K~ + dQ~ Q~ - dKbar Kbar - dAbar Abar
+//     dg_t = sum_{t' >= t} dLog_t' + dLbar,   dLbar_j = sum_c G[j][c] S_{n+1}[j][c]
+//
+// Kernels: k2_bprep (Q'^T dO), k2_chain_rev (reverse pass, dLbar), k2_bwd1
+// (dY, dYR, dU -> dv, dw; the state-side terms; Y and dYR for k2_bwd2),
+// k2_bwd2 (the decay-masked gradients in TF32 with the dL matrices as
+// tensor-memory operands, one 64-channel half at a time; final dq, dk, dg, de,
+// dgamma).  Precision: products with a state (S, G) use bf16 operands, the
+// bounded-range products fp16, the decay-masked gradients TF32; fp32
+// accumulation throughout.
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "bwd2.h"
+#include "fwd2.h"
+#include "profile.h"
+#include "tc2.cuh"
+
+namespace muir {
+namespace v2 {
+
+using namespace t2;
+
+// Expired bounded waits of this file's kernels (bit i: wait site i), read and
+// cleared by timeouts_bwd2().
+__device__ unsigned int g_bwd2_timeouts;
+
+namespace {
+
+constexpr int kC = 128, kD = 128;
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr float kLogDecayMin = -20.f;
+constexpr uint32_t kT32Half = 64 * 128 * 4;  // T32 tile of 64 rows
+
+__device__ __forceinline__ float ex2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+__device__ __forceinline__ void sync_all() {
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+}
+
+// 8 consecutive bf16 of a token-major row -> floats.
+__device__ __forceinline__ void ld8_bf16(const __nv_bfloat16* p, float* v) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    unpack16<true>(u.x, v[0], v[1]);
+    unpack16<true>(u.y, v[2], v[3]);
+    unpack16<true>(u.z, v[4], v[5]);
+    unpack16<true>(u.w, v[6], v[7]);
+}
+
+__device__ __forceinline__ void st8_bf16(__nv_bfloat16* p, const float* v) {
+    uint4 u;
+    u.x = pack_bf16(v[0], v[1]);
+    u.y = pack_bf16(v[2], v[3]);
+    u.z = pack_bf16(v[4], v[5]);
+    u.w = pack_bf16(v[6], v[7]);
+    *reinterpret_cast<uint4*>(p) = u;
+}
+
+// Store 32 values at columns 32 * c32 .. +32 of row t of a T16 tile.
+template <bool BF16>
+__device__ __forceinline__ void row_st32(unsigned char* tile, int t, int c32, const float* v) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) st_chunk16<BF16>(tile, t, 4 * c32 + i, v + 8 * i);
+}
+
+template <bool BF16>
+__device__ __forceinline__ void row_ld32(const unsigned char* tile, int t, int c32, float* v) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ld_chunk16<BF16>(tile, t, 4 * c32 + i, v + 8 * i);
+}
+
+__device__ __forceinline__ void tm_ld32w(uint32_t tm, int q, int col, float (&v)[32]) {
+    tmem_ld32(taddr(tm, 32 * q, col), v);
+    tmem_wait_ld();
+}
+
+// Chunk-local cumulative log decay (log2 units) of this thread's row t and 32
+// channels j0..j0+31, by a warp scan over tokens plus the totals of the
+// earlier 32-token quarters (tot: [4][128] floats in shared memory, written
+// here).  Ends with a block barrier; tot then holds the quarter totals.
+__device__ __forceinline__ void log_decay(const __nv_bfloat16* g, int lane, int q, int j0,
+                                          float (*tot)[kD], float (&L)[32]) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) ld8_bf16(g + j0 + 8 * i, L + 8 * i);
+#pragma unroll
+    for (int j = 0; j < 32; ++j) L[j] = fmaxf(L[j], kLogDecayMin) * kLog2e;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {
+            const float o = __shfl_up_sync(0xffffffffu, L[j], off);
+            if (lane >= off) L[j] += o;
+        }
+    }
+    if (lane == 31) {
+#pragma unroll
+        for (int j = 0; j < 32; ++j) tot[q][j0 + j] = L[j];
+    }
+    __syncthreads();
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        float pre = 0.f;
+        for (int qq = 0; qq < q; ++qq) pre += tot[qq][j0 + j];
+        L[j] += pre;
+    }
+}
+
+__device__ __forceinline__ float chunk_total(float (*tot)[kD], int j) {
+    return tot[0][j] + tot[1][j] + tot[2][j] + tot[3][j];
+}
+
+}  // namespace
+
+// ------------------------------------------------------------------ k2_bprep
+
+// B'_n = Q'_n^T dO_n (fp16 operands, fp32 accumulation); one chunk per CTA.
+__global__ void __launch_bounds__(256) k2_bprep(const __grid_constant__ BprepParams p) {
+    extern __shared__ __align__(1024) unsigned char smraw[];
+    unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    unsigned char* Qt = sm;
+    unsigned char* Dt = sm + kT16Bytes;
+    __shared__ uint64_t bar[2];
+    __shared__ uint32_t tslot;
+    __shared__ int bad;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, h = warp >> 2, t = 32 * q + lane;
+    const int c = blockIdx.x, N = p.T / kC;
+    const int n = c % N, bh = c / N;
+    if (tid == 0) {
+        mbar_init(&bar[0], 1);
+        mbar_init(&bar[1], 1);
+        bad = 0;
+        fence_barrier_init();
+    }
+    if (warp == 0) tmem_alloc(&tslot, 128);
+    sync_all();
+    const uint32_t tm = tslot;
+    if (tid == 0) {
+        mbar_arrive_expect_tx(&bar[0], kT16Bytes);
+        const int z = (bh / p.H) * p.T + n * kC, y = bh % p.H;
+        tma_load_3d(Dt, &p.tdO, 0, y, z, &bar[0]);
+        tma_load_3d(Dt + kT16Block, &p.tdO, 64, y, z, &bar[0]);
+    }
+    {  // Q' row t, columns 64h .. +64 -> fp16
+        const float* src = p.Qp + (size_t)c * kC * kD + (size_t)t * kD + 64 * h;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            float v[8];
+            const float4 a = __ldg(reinterpret_cast<const float4*>(src + 8 * i));
+            const float4 b = __ldg(reinterpret_cast<const float4*>(src + 8 * i + 4));
+            v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+            st_chunk16<false>(Qt, t, 8 * h + i, v);
+        }
+    }
+    if (!mbar_wait(&bar[0], 0)) atomicOr(&bad, 1);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {  // dO bf16 -> fp16 in place (own chunks)
+        float v[8];
+        ld_chunk16<true>(Dt, t, 8 * h + i, v);
+        st_chunk16<false>(Dt, t, 8 * h + i, v);
+    }
+    fence_async_smem();
+    sync_all();
+    if (tid == 0) {
+        gemm_mm16(tm, saddr(Qt), 0, 0, saddr(Dt), 0, 0, 128, 128, kF16, false);
+        mma_commit(&bar[1]);
+    }
+    if (!mbar_wait(&bar[1], 0)) atomicOr(&bad, 2);
+    tc_fence_after();
+    {
+        float* dst = p.Bp + (size_t)c * kD * kD + (size_t)t * kD + 64 * h;
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh) {
+            float v[32];
+            tm_ld32w(tm, q, 64 * h + 32 * hh, v);
+#pragma unroll
+            for (int j = 0; j < 32; j += 4)
+                *reinterpret_cast<float4*>(dst + 32 * hh + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+        }
+    }
+    if (tid == 0 && bad) atomicOr(&g_bwd2_timeouts, (unsigned)bad);
+    sync_all();
+    if (warp == 0) tmem_dealloc(tm, 128);
+}
+
+// ------------------------------------------------------------------ k2_chain_rev
+
+// G_n = M_n^T G_{n+1} + B'_n for one head and SLAB value columns, n = N-1 .. 0;
+// records G_{n+1} in dSc[n], adds this slab's share of
+// dLbar[n][j] = sum_c G_{n+1}[j][c] S_{n+1}[j][c] (dLbar zeroed beforehand) and
+// writes G_0 to dS0.  M_n^T streams through a 3-stage TMA ring (K-major TF32).
+template <int SLAB>
+__global__ void __launch_bounds__(128, 1) k2_chain_rev(const __grid_constant__ RevParams p) {
+    constexpr int STAGES = 3;
+    constexpr uint32_t MT = 128 * 128 * 4;
+    extern __shared__ __align__(1024) unsigned char smraw[];
+    unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    unsigned char* Mst = sm;
+    unsigned char* Gt = sm + STAGES * MT;
+    __shared__ uint64_t bar[STAGES + 1];
+    __shared__ uint32_t tslot;
+    __shared__ int bad;
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const int nslab = kD / SLAB;
+    const int bh = blockIdx.x / nslab, c0 = (blockIdx.x % nslab) * SLAB;
+    const int N = p.N, j = tid;
+    if (tid == 0) {
+        for (int i = 0; i <= STAGES; ++i) mbar_init(&bar[i], 1);
+        bad = 0;
+        fence_barrier_init();
+        prefetch_tmap(&p.tMt);
+    }
+    if (warp == 0) tmem_alloc(&tslot, 32 < SLAB ? SLAB : 32);
+    sync_all();
+    const uint32_t tm = tslot;
+    const long long row0 = (long long)bh * N * kD;
+    // step s handles chunk n = N - 1 - s
+    auto issue = [&](int s) {
+        const int st = s % STAGES, n = N - 1 - s;
+        mbar_arrive_expect_tx(&bar[st], MT);
+        for (int kb = 0; kb < 4; ++kb)
+            tma_load_3d(Mst + st * MT + kb * 128 * 128, &p.tMt, 32 * kb, (int)(row0 + (long long)n * kD), 0,
+                        &bar[st]);
+    };
+    if (tid == 0)
+        for (int s = 0; s < STAGES && s < N; ++s) issue(s);
+    float Gr[SLAB];
+    const size_t gbase = ((size_t)bh * kD + j) * kD + c0;
+#pragma unroll
+    for (int c = 0; c < SLAB; ++c) Gr[c] = p.dS_final ? p.dS_final[gbase + c] : 0.f;
+    auto put = [&]() {
+#pragma unroll
+        for (int c = 0; c < SLAB; ++c)
+            *reinterpret_cast<float*>(Gt + t32_off<SLAB>(c, j >> 2) + (j & 3) * 4) = Gr[c];
+    };
+    put();
+    fence_async_smem();
+    sync_all();
+    for (int s = 0; s < N; ++s) {
+        const int st = s % STAGES, n = N - 1 - s;
+        // record G_{n+1} and this slab's share of dLbar_n
+        {
+            float* d = p.dSc + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
+            const float* sn1 = (n + 1 < N) ? p.S_chunks + ((size_t)bh * N + n + 1) * kD * kD + (size_t)j * kD + c0
+                                           : p.S_last + gbase;
+            float acc = 0.f;
+#pragma unroll
+            for (int c = 0; c < SLAB; c += 4) {
+                *reinterpret_cast<float4*>(d + c) = make_float4(Gr[c], Gr[c + 1], Gr[c + 2], Gr[c + 3]);
+                const float4 sv = __ldg(reinterpret_cast<const float4*>(sn1 + c));
+                acc += Gr[c] * sv.x + Gr[c + 1] * sv.y + Gr[c + 2] * sv.z + Gr[c + 3] * sv.w;
+            }
+            atomicAdd(p.dgb + ((size_t)bh * N + n) * kD + j, acc);
+        }
+        // only the issuing thread waits for M_n^T (see k2_chain)
+        if (tid == 0) {
+            if (!mbar_wait(&bar[st], (uint32_t)((s / STAGES) & 1))) atomicOr(&bad, 4);
+            tc_fence_after();
+            gemm_kk32<128, SLAB>(tm, saddr(Mst + st * MT), saddr(Gt), 0, SLAB, 128, false);
+            mma_commit(&bar[STAGES]);
+        }
+        float Bc[SLAB];
+        {
+            const float* src = p.Bp + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
+#pragma unroll
+            for (int c = 0; c < SLAB; c += 4) {
+                const float4 v = __ldg(reinterpret_cast<const float4*>(src + c));
+                Bc[c] = v.x; Bc[c + 1] = v.y; Bc[c + 2] = v.z; Bc[c + 3] = v.w;
+            }
+        }
+        if (!mbar_wait(&bar[STAGES], (uint32_t)(s & 1))) atomicOr(&bad, 8);
+        tc_fence_after();
+        if (tid == 0 && s + STAGES < N) issue(s + STAGES);
+        float d[32];
+        tmem_ld32(taddr(tm, 32 * warp, 0), d);
+        tmem_wait_ld();
+#pragma unroll
+        for (int c = 0; c < SLAB; ++c) Gr[c] = d[c] + Bc[c];
+        put();
+        fence_async_smem();
+        sync_all();
+    }
+    if (p.dS0) {
+        float* d = p.dS0 + gbase;
+#pragma unroll
+        for (int c = 0; c < SLAB; c += 4) *reinterpret_cast<float4*>(d + c) = make_float4(Gr[c], Gr[c + 1], Gr[c + 2], Gr[c + 3]);
+    }
+    if (tid == 0 && bad) atomicOr(&g_bwd2_timeouts, (unsigned)bad);
+    sync_all();
+    if (warp == 0) tmem_dealloc(tm, 32 < SLAB ? SLAB : 32);
+}
+
+// ------------------------------------------------------------------ k2_bwd1
+
+namespace {
+struct Bwd1Smem {
+    float tot[4][kD];
+    float Lb[kD];
+    float red[16];
+    uint64_t bar[16];
+    uint32_t tslot;
+    int bad;
+};
+enum { B1D = 0, B1W, B1U, B1Q, B1A, B1T, B1K, B1L, B1KB, B1M1, B1M2, B1M3, B1M4, B1M5, B1M6 };
+
+// Largest |x| over the block (512 threads, 32 values each); ends with a barrier.
+__device__ __forceinline__ float block_absmax(const float (&v)[32], float* red, int warp, int lane) {
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+    if (lane == 0) red[warp] = m;
+    __syncthreads();
+    float r = 0.f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) r = fmaxf(r, red[i]);
+    __syncthreads();
+    return r;
+}
+
+// Power of two s with max|x| / s below 2^14 (fp16 operands keep their range); 1 for zero.
+__device__ __forceinline__ float pow2_scale(float amax) {
+    if (!(amax > 0.f)) return 1.f;
+    return exp2f((float)(ilogbf(amax) - 13));
+}
+}  // namespace
+
+// 512 threads; thread t = 32 (warp % 4) + lane owns row t, columns 32 (warp / 4) .. +32.
+// Products with a state use fp16 operands with S / sS and G / sG (sS, sG per-chunk
+// powers of two), every other product fp16; accumulation fp32 in tensor memory.
+__global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Params p) {
+    extern __shared__ __align__(1024) unsigned char smraw[];
+    unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    unsigned char* S[6];
+#pragma unroll
+    for (int i = 0; i < 6; ++i) S[i] = sm + i * kT16Bytes;
+    Bwd1Smem& s = *reinterpret_cast<Bwd1Smem*>(sm + 6 * kT16Bytes);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, h = warp >> 2, t = 32 * q + lane, c0 = 32 * h;
+    const int N = p.T / kC, nch = p.B * p.H * N;
+    if (tid == 0) {
+        for (int i = 0; i < 16; ++i) mbar_init(&s.bar[i], 1);
+        s.bad = 0;
+        fence_barrier_init();
+        prefetch_tmap(&p.tdO);
+    }
+    if (warp == 0) tmem_alloc(&s.tslot, 512);
+    sync_all();
+    const uint32_t tm = s.tslot;
+    uint32_t a[6];
+#pragma unroll
+    for (int i = 0; i < 6; ++i) a[i] = saddr(S[i]);
+    auto waitb = [&](int i, uint32_t ph) {
+        if (!mbar_wait(&s.bar[i], ph)) atomicOr(&s.bad, 1 << (8 + i));
+    };
+    auto bulk = [&](unsigned char* dst, const unsigned char* src, int bar) {
+        mbar_arrive_expect_tx(&s.bar[bar], kT16Bytes);
+        bulk_load(dst, src, kT16Bytes, &s.bar[bar]);
+    };
+    int it = 0;
+    for (int c = blockIdx.x; c < nch; c += gridDim.x, ++it) {
+        const uint32_t ph = (uint32_t)(it & 1);
+        const int n = c % N, bh = c / N, hd = bh % p.H, b = bh / p.H;
+        const size_t tok = ((size_t)b * p.T + (size_t)n * kC + t) * p.H + hd;  // token-major row
+        const size_t ro = tok * kD + c0;                                      // this thread's 32 elements
+        const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + c0;          // per-chunk fp32 arrays
+        const unsigned char* ax = p.aux + (size_t)c * AuxLayout::kBytes;
+        unsigned char* y16 = p.Y16 + (size_t)c * kT16Bytes;
+        unsigned char* r16 = p.dYR16 + (size_t)c * kT16Bytes;
+
+        if (tid == 0) {  // dO -> S1; W -> S2, U -> S4, M_QA -> S5
+            bulk_wait_read();  // the previous chunk's tile stores have left S2 and S5
+            mbar_arrive_expect_tx(&s.bar[B1D], kT16Bytes);
+            const int z = b * p.T + n * kC;
+            tma_load_3d(S[1], &p.tdO, 0, hd, z, &s.bar[B1D]);
+            tma_load_3d(S[1] + kT16Block, &p.tdO, 64, hd, z, &s.bar[B1D]);
+            bulk(S[2], ax + AuxLayout::kW16, B1W);
+            bulk(S[4], ax + AuxLayout::kU16, B1U);
+            bulk(S[5], ax + AuxLayout::kMQA16, B1Q);
+        }
+        // log decay of row t, columns c0..; E = 2^L, Eb = 2^(Lbar - L)
+        float L[32];
+        log_decay(reinterpret_cast<const __nv_bfloat16*>(p.g) + tok * kD, lane, q, c0, s.tot, L);
+        if (q == 0) s.Lb[c0 + lane] = chunk_total(s.tot, c0 + lane);
+        // S_n / sS -> fp16 tile S0, G / sG -> fp16 tile S3 (row j = t)
+        float sS, sG;
+        {
+            float v[32];
+            const float* src = p.S_chunks + cb;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 x = __ldg(reinterpret_cast<const float4*>(src + j));
+                v[j] = x.x; v[j + 1] = x.y; v[j + 2] = x.z; v[j + 3] = x.w;
+            }
+            sS = pow2_scale(block_absmax(v, s.red, warp, lane));
+            const float is = 1.f / sS;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= is;
+            row_st32<false>(S[0], t, h, v);
+            src = p.dSc + cb;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 x = __ldg(reinterpret_cast<const float4*>(src + j));
+                v[j] = x.x; v[j + 1] = x.y; v[j + 2] = x.z; v[j + 3] = x.w;
+            }
+            sG = pow2_scale(block_absmax(v, s.red, warp, lane));
+            const float ig = 1.f / sG;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) v[j] *= ig;
+            row_st32<false>(S[3], t, h, v);
+        }
+        waitb(B1D, ph);
+        {  // dO bf16 -> fp16 in place (own chunks)
+            float v[32];
+            row_ld32<true>(S[1], t, h, v);
+            row_st32<false>(S[1], t, h, v);
+        }
+        fence_async_smem();
+        __syncthreads();
+        waitb(B1W, ph);
+        tc_fence_after();
+        // ---- phase 1: dQ~ / sS = dO S^T (B0), W S / sS (B1)
+        if (tid == 0) {
+            gemm_kk16(tm + 0, a[1], 0, a[0], 0, 0, 128, 128, kF16, false);
+            gemm_km16(tm + 128, a[2], 0, a[0], 0, 0, 128, 128, kF16, false);
+            mma_commit(&s.bar[B1M1]);
+        }
+        float kv[32], ev[32];
+        {
+            const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(p.k) + ro;
+            const __nv_bfloat16* ep = reinterpret_cast<const __nv_bfloat16*>(p.e) + ro;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) { ld8_bf16(kp + 8 * i, kv + 8 * i); ld8_bf16(ep + 8 * i, ev + 8 * i); }
+        }
+        waitb(B1M1, ph);
+        tc_fence_after();
+        // ---- phase 2: Pq, PL (dQ~ part); Y = W S + U' -> fp16 tile S2 (also saved for k2_bwd2)
+        float PL[32];
+        {
+            float d[32], qv[8], gv[8];
+            tm_ld32w(tm, q, c0, d);
+            const __nv_bfloat16* qp = reinterpret_cast<const __nv_bfloat16*>(p.q) + ro;
+            const __nv_bfloat16* gp = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + ro;
+            float* pq = p.Pq + cb;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                ld8_bf16(qp + 8 * i, qv);
+                ld8_bf16(gp + 8 * i, gv);
+                float o[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const int j = 8 * i + u;
+                    o[u] = d[j] * sS * ex2(L[j]);
+                    PL[j] = o[u] * qv[u] * gv[u];  // dQ~ . Q~
+                }
+                *reinterpret_cast<float4*>(pq + 8 * i) = make_float4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<float4*>(pq + 8 * i + 4) = make_float4(o[4], o[5], o[6], o[7]);
+            }
+            tm_ld32w(tm, q, 128 + c0, d);
+            const float* up = reinterpret_cast<const float*>(ax + AuxLayout::kUp) + (size_t)t * kD + c0;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                const float4 x = __ldg(reinterpret_cast<const float4*>(up + j));
+                d[j] = d[j] * sS + x.x; d[j + 1] = d[j + 1] * sS + x.y;
+                d[j + 2] = d[j + 2] * sS + x.z; d[j + 3] = d[j + 3] * sS + x.w;
+            }
+            row_st32<false>(S[2], t, h, d);  // Y over W
+        }
+        fence_async_smem();
+        sync_all();
+        waitb(B1U, ph);
+        waitb(B1Q, ph);
+        tc_fence_after();
+        if (tid == 0) {
+            bulk_store(y16, S[2], kT16Bytes);
+            bulk_commit();
+            gemm_kk16(tm + 0, a[4], 0, a[3], 0, 0, 128, 128, kF16, false);         // dKbar / sG = U G^T
+            gemm_kk16(tm + 128, a[2], 0, a[3], 0, 0, 128, 128, kF16, false, true);  // dAbar / sG = -Y G^T
+            gemm_mm16(tm + 256, a[5], 0, 0, a[1], 0, 0, 128, 128, kF16, false, true); // -M_QA^T dO
+            mma_commit(&s.bar[B1M2]);
+        }
+        waitb(B1M2, ph);
+        tc_fence_after();
+        if (tid == 0) {  // Abar -> S4, T -> S5 (U, M_QA consumed)
+            bulk(S[4], ax + AuxLayout::kAbar16, B1A);
+            bulk(S[5], ax + AuxLayout::kT16, B1T);
+        }
+        // ---- phase 3: Pk (dKbar part), Pa, PL
+        {
+            float d[32];
+            tm_ld32w(tm, q, c0, d);  // dKbar / sG
+            float* pk = p.Pk + cb;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                float o[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float Eb = ex2(s.Lb[c0 + j + u] - L[j + u]);
+                    o[u] = d[j + u] * sG * Eb;
+                    PL[j + u] -= o[u] * kv[j + u];  // dKbar . Kbar
+                }
+                *reinterpret_cast<float4*>(pk + j) = make_float4(o[0], o[1], o[2], o[3]);
+            }
+            tm_ld32w(tm, q, 128 + c0, d);  // dAbar / sG
+            float* pa = p.Pa + cb;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                float o[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    const float Eb = ex2(s.Lb[c0 + j + u] - L[j + u]);
+                    o[u] = d[j + u] * sG * Eb;
+                    PL[j + u] -= o[u] * ev[j + u] * kv[j + u];  // dAbar . Abar
+                }
+                *reinterpret_cast<float4*>(pa + j) = make_float4(o[0], o[1], o[2], o[3]);
+            }
+        }
+        waitb(B1A, ph);
+        sync_all();  // every warp has read B0 before it is overwritten
+        // ---- phase 4: Abar G / sG (B0); dY = -M_QA^T dO - Abar G
+        if (tid == 0) {
+            gemm_km16(tm + 0, a[4], 0, a[3], 0, 0, 128, 128, kF16, false);
+            mma_commit(&s.bar[B1M3]);
+        }
+        waitb(B1M3, ph);
+        tc_fence_after();
+        if (tid == 0) {
+            bulk_wait_read();  // Y left S2
+            bulk(S[4], ax + AuxLayout::kMQK16, B1K);  // Abar consumed
+        }
+        {
+            float d[32], e2[32];
+            tm_ld32w(tm, q, 256 + c0, d);
+            tm_ld32w(tm, q, c0, e2);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) d[j] -= sG * e2[j];
+            __syncthreads();                 // Y (S2) no longer read by the bulk store
+            row_st32<false>(S[2], t, h, d);  // dY over Y
+        }
+        fence_async_smem();
+        sync_all();
+        waitb(B1T, ph);
+        tc_fence_after();
+        // ---- phase 5: dYR = T^T dY (B3)
+        if (tid == 0) {
+            gemm_mm16(tm + 384, a[5], 0, 0, a[2], 0, 0, 128, 128, kF16, false);
+            mma_commit(&s.bar[B1M4]);
+        }
+        waitb(B1M4, ph);
+        tc_fence_after();
+        if (tid == 0) bulk(S[2], ax + AuxLayout::kLK16, B1L);  // dY consumed
+        {
+            float d[32];
+            tm_ld32w(tm, q, 384 + c0, d);
+            row_st32<false>(S[5], t, h, d);  // dYR over T
+        }
+        fence_async_smem();
+        sync_all();
+        waitb(B1K, ph);
+        tc_fence_after();
+        // ---- phase 6: dK~ / sS = dYR S^T (B0); M_QK^T dO (B1)
+        if (tid == 0) {
+            bulk_store(r16, S[5], kT16Bytes);
+            bulk_commit();
+            gemm_kk16(tm + 0, a[5], 0, a[0], 0, 0, 128, 128, kF16, false);
+            gemm_mm16(tm + 128, a[4], 0, 0, a[1], 0, 0, 128, 128, kF16, false);
+            mma_commit(&s.bar[B1M5]);
+        }
+        waitb(B1M5, ph);
+        tc_fence_after();
+        if (tid == 0) bulk(S[0], ax + AuxLayout::kKbar16, B1KB);  // S consumed
+        {
+            float d[32];
+            tm_ld32w(tm, q, c0, d);  // dK~ / sS
+            float* pk = p.Pk + cb;
+            float* pl = p.PL + cb;
+#pragma unroll
+            for (int j = 0; j < 32; j += 4) {
+                float4 x = *reinterpret_cast<float4*>(pk + j);
+                float o[4];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    o[u] = d[j + u] * sS * ex2(L[j + u]);
+                    PL[j + u] += o[u] * kv[j + u];  // dK~ . K~
+                }
+                x.x += o[0]; x.y += o[1]; x.z += o[2]; x.w += o[3];
+                *reinterpret_cast<float4*>(pk + j) = x;
+                *reinterpret_cast<float4*>(pl + j) = make_float4(PL[j], PL[j + 1], PL[j + 2], PL[j + 3]);
+            }
+        }
+        waitb(B1L, ph);
+        waitb(B1KB, ph);
+        tc_fence_after();
+        // ---- phase 7: dU = M_QK^T dO + L_K^T dYR (B1) + Kbar G (B2, times sG)
+        if (tid == 0) {
+            gemm_mm16(tm + 128, a[2], 0, 0, a[5], 0, 0, 128, 128, kF16, true);
+            gemm_km16(tm + 256, a[0], 0, a[3], 0, 0, 128, 128, kF16, false);
+            mma_commit(&s.bar[B1M6]);
+        }
+        waitb(B1M6, ph);
+        tc_fence_after();
+        {
+            float d[32], e2[32], vv[8], wv[8];
+            tm_ld32w(tm, q, 128 + c0, d);
+            tm_ld32w(tm, q, 256 + c0, e2);
+            const __nv_bfloat16* vp = reinterpret_cast<const __nv_bfloat16*>(p.v) + ro;
+            const __nv_bfloat16* wp = reinterpret_cast<const __nv_bfloat16*>(p.w) + ro;
+            __nv_bfloat16* dvp = reinterpret_cast<__nv_bfloat16*>(p.dv) + ro;
+            __nv_bfloat16* dwp = reinterpret_cast<__nv_bfloat16*>(p.dw) + ro;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                ld8_bf16(vp + 8 * i, vv);
+                ld8_bf16(wp + 8 * i, wv);
+                float o1[8], o2[8];
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    const float du = d[8 * i + u] + sG * e2[8 * i + u];
+                    o1[u] = du * wv[u];
+                    o2[u] = du * vv[u];
+                }
+                st8_bf16(dvp + 8 * i, o1);
+                st8_bf16(dwp + 8 * i, o2);
+            }
+        }
+        sync_all();
+    }
+    if (tid == 0) bulk_wait_all();
+    if (tid == 0 && s.bad) atomicOr(&g_bwd2_timeouts, (unsigned)s.bad);
+    sync_all();
+    if (warp == 0) tmem_dealloc(tm, 512);
+}
+
+// ------------------------------------------------------------------ k2_bwd2
+
+namespace {
+struct Bwd2Smem {
+    float tot[4][kD];
+    float P2[kD];
+    float sfx[4][kD];  // per-quarter totals of the reverse scan
+    uint64_t bar[8];
+    uint32_t tslot;
+    int bad;
+};
+enum { B2IN = 0, B2M };
+}  // namespace
+
+// 256 threads; thread t = 32 (warp % 4) + lane owns row t; for channel half hj
+// it handles channels 64 hj + 32 (warp / 4) .. +32.
+__global__ void __launch_bounds__(256, 1) k2_bwd2(const __grid_constant__ Bwd2Params p) {
+    extern __shared__ __align__(1024) unsigned char smraw[];
+    unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
+    unsigned char* tdO = sm;
+    unsigned char* tU = sm + 1 * kT16Bytes;
+    unsigned char* tY = sm + 2 * kT16Bytes;
+    unsigned char* tR = sm + 3 * kT16Bytes;
+    unsigned char* Bt0 = sm + 4 * kT16Bytes;
+    unsigned char* Bt1 = Bt0 + kT32Half;
+    Bwd2Smem& s = *reinterpret_cast<Bwd2Smem*>(Bt1 + kT32Half);
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int q = warp & 3, h = warp >> 2, t = 32 * q + lane;
+    const int N = p.T / kC, nch = p.B * p.H * N;
+    if (tid == 0) {
+        for (int i = 0; i < 8; ++i) mbar_init(&s.bar[i], 1);
+        s.bad = 0;
+        fence_barrier_init();
+        prefetch_tmap(&p.tdO);
+    }
+    if (warp == 0) tmem_alloc(&s.tslot, 512);
+    sync_all();
+    const uint32_t tm = s.tslot;
+    const uint32_t aO = saddr(tdO), aU = saddr(tU), aY = saddr(tY), aR = saddr(tR);
+    const uint32_t aB0 = saddr(Bt0), aB1 = saddr(Bt1);
+    uint32_t pm = 0;  // parity of the MMA barrier
+    // Every thread waits; the barrier that follows keeps the next commit on
+    // B2M from completing before the slowest thread has seen this phase.
+    auto mma_wait = [&]() {
+        if (!mbar_wait(&s.bar[B2M], pm)) atomicOr(&s.bad, 1 << 24);
+        pm ^= 1u;
+        sync_all();
+    };
+    // dL products into TMEM columns 0..127 (x) and 128..255 (y), then masked in
+    // place: keep(col) for this lane's row; values rounded to TF32.
+    auto mask_rows = [&](auto keep0, auto keep1) {
+#pragma unroll 1
+        for (int part = 0; part < 4; ++part) {
+            const int bank = part >> 1, col0 = 64 * h + 32 * (part & 1);
+            float v[32];
+            tm_ld32w(tm, q, 128 * bank + col0, v);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                const bool k = bank == 0 ? keep0(col0 + j) : keep1(col0 + j);
+                v[j] = k ? tf32_round(v[j]) : 0.f;
+            }
+#pragma unroll
+            for (int hh = 0; hh < 2; ++hh) {
+                float w[16];
+#pragma unroll
+                for (int j = 0; j < 16; ++j) w[j] = v[16 * hh + j];
+                tmem_st16(taddr(tm, 32 * q, 128 * bank + col0 + 16 * hh), w);
+            }
+        }
+        tmem_wait_st();
+    };
+    // ACC[128 x 64] (+)= A0 (TMEM cols 0..127) Bt0 + A1 (TMEM cols 128..255) Bt1, TF32
+    auto acc_pair = [&](int acc_col) {
+        const uint32_t id = idesc(kTF32, 128, 64, false, false);
+        for (int k = 0; k < 128; k += 8)
+            mma_tf32_ta(tm + acc_col, tm + k, kdesc32<64>(aB0, 0, k), id, k ? 1u : 0u);
+        for (int k = 0; k < 128; k += 8)
+            mma_tf32_ta(tm + acc_col, tm + 128 + k, kdesc32<64>(aB1, 0, k), id, 1u);
+    };
+    // pivoted operand (row t, this thread's 32 channels) -> column t of a
+    // transposed K-major TF32 tile (row = channel inside the half)
+    auto put_t = [&](unsigned char* tile, int r0, const float* v) {
+#pragma unroll
+        for (int u = 0; u < 32; ++u)
+            *reinterpret_cast<float*>(tile + t32_off<64>(r0 + u, t >> 2) + (t & 3) * 4) = tf32_round(v[u]);
+    };
+
+    int it = 0;
+    for (int c = blockIdx.x; c < nch; c += gridDim.x, ++it) {
+        const uint32_t ph = (uint32_t)(it & 1);
+        const int n = c % N, bh = c / N, hd = bh % p.H, b = bh / p.H;
+        const size_t tok = ((size_t)b * p.T + (size_t)n * kC + t) * p.H + hd;
+        if (tid == 0) {
+            mbar_arrive_expect_tx(&s.bar[B2IN], 4 * kT16Bytes);
+            const int z = b * p.T + n * kC;
+            tma_load_3d(tdO, &p.tdO, 0, hd, z, &s.bar[B2IN]);
+            tma_load_3d(tdO + kT16Block, &p.tdO, 64, hd, z, &s.bar[B2IN]);
+            bulk_load(tU, p.aux + (size_t)c * AuxLayout::kBytes + AuxLayout::kU16, kT16Bytes, &s.bar[B2IN]);
+            bulk_load(tY, p.Y16 + (size_t)c * kT16Bytes, kT16Bytes, &s.bar[B2IN]);
+            bulk_load(tR, p.dYR16 + (size_t)c * kT16Bytes, kT16Bytes, &s.bar[B2IN]);
+        }
+        if (!mbar_wait(&s.bar[B2IN], ph)) atomicOr(&s.bad, 1 << 25);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {  // dO bf16 -> fp16 in place (row t, columns 64h ..)
+            float v[8];
+            ld_chunk16<true>(tdO, t, 8 * h + i, v);
+            st_chunk16<false>(tdO, t, 8 * h + i, v);
+        }
+        fence_async_smem();
+        sync_all();
+
+#pragma unroll 1
+        for (int hj = 0; hj < 2; ++hj) {
+            const int j0 = 64 * hj + 32 * h;  // this thread's channels
+            const int r0 = 32 * h;            // their rows in the half tiles
+            float L[32];
+            log_decay(reinterpret_cast<const __nv_bfloat16*>(p.g) + tok * kD, lane, q, j0, s.tot, L);
+            if (q == 0) s.P2[j0 + lane] = 0.5f * chunk_total(s.tot, j0 + lane);
+            __syncthreads();
+            float kv[32], ev[32];
+            {
+                const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(p.k) + tok * kD + j0;
+                const __nv_bfloat16* ep = reinterpret_cast<const __nv_bfloat16*>(p.e) + tok * kD + j0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) { ld8_bf16(kp + 8 * i, kv + 8 * i); ld8_bf16(ep + 8 * i, ev + 8 * i); }
+            }
+            // Am -> Bt0, Km -> Bt1
+            {
+                float am[32], km[32];
+#pragma unroll
+                for (int u = 0; u < 32; ++u) {
+                    const float em = ex2(s.P2[j0 + u] - L[u]);
+                    km[u] = kv[u] * em;
+                    am[u] = ev[u] * km[u];
+                }
+                put_t(Bt0, r0, am);
+                put_t(Bt1, r0, km);
+            }
+            fence_async_smem();
+            sync_all();
+            // R1: dL_A = -dYR Y^T, dL_K = dYR U^T (strict) -> dKp
+            if (tid == 0) {
+                gemm_kk16(tm + 0, aR, 0, aY, 0, 0, 128, 128, kF16, false, true);
+                gemm_kk16(tm + 128, aR, 0, aU, 0, 0, 128, 128, kF16, false);
+                mma_commit(&s.bar[B2M]);
+            }
+            mma_wait();
+            mask_rows([&](int col) { return col < t; }, [&](int col) { return col < t; });
+            sync_all();
+            if (tid == 0) {
+                acc_pair(256);
+                mma_commit(&s.bar[B2M]);
+            }
+            mma_wait();
+            // R2: dM_QA = -dO Y^T (x), dM_QK = dO U^T (y) (inclusive) -> dQp = x Am + y Km
+            if (tid == 0) {
+                gemm_kk16(tm + 0, aO, 0, aY, 0, 0, 128, 128, kF16, false, true);
+                gemm_kk16(tm + 128, aO, 0, aU, 0, 0, 128, 128, kF16, false);
+                mma_commit(&s.bar[B2M]);
+            }
+            mma_wait();
+            mask_rows([&](int col) { return col <= t; }, [&](int col) { return col <= t; });
+            sync_all();
+            if (tid == 0) {
+                acc_pair(320);
+                mma_commit(&s.bar[B2M]);
+            }
+            mma_wait();
+            // Kp -> Bt0, Qp -> Bt1
+            {
+                float kp[32], qp[32], qv[8], gv[8];
+                const __nv_bfloat16* qsrc = reinterpret_cast<const __nv_bfloat16*>(p.q) + tok * kD + j0;
+                const __nv_bfloat16* gsrc = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + tok * kD + j0;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    ld8_bf16(qsrc + 8 * i, qv);
+                    ld8_bf16(gsrc + 8 * i, gv);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = 8 * i + u;
+                        const float ep = ex2(L[j] - s.P2[j0 + j]);
+                        kp[j] = kv[j] * ep;
+                        qp[j] = qv[u] * gv[u] * ep;
+                    }
+                }
+                put_t(Bt0, r0, kp);
+                put_t(Bt1, r0, qp);
+            }
+            fence_async_smem();
+            sync_all();
+            // R3: dL_A^T = -Y dYR^T (x, strict upper), dM_QA^T = -Y dO^T (y, inclusive upper) -> dAm
+            if (tid == 0) {
+                gemm_kk16(tm + 0, aY, 0, aR, 0, 0, 128, 128, kF16, false, true);
+                gemm_kk16(tm + 128, aY, 0, aO, 0, 0, 128, 128, kF16, false, true);
+                mma_commit(&s.bar[B2M]);
+            }
+            mma_wait();
+            mask_rows([&](int col) { return col > t; }, [&](int col) { return col >= t; });
+            sync_all();
+            if (tid == 0) {
+                acc_pair(384);
+                mma_commit(&s.bar[B2M]);
+            }
+            mma_wait();
+            // R4: dL_K^T = U dYR^T (x, strict upper), dM_QK^T = U dO^T (y, inclusive upper) -> dKm
+            if (tid == 0) {
+                gemm_kk16(tm + 0, aU, 0, aR, 0, 0, 128, 128, kF16, false);
+                gemm_kk16(tm + 128, aU, 0, aO, 0, 0, 128, 128, kF16, false);
+                mma_commit(&s.bar[B2M]);
+            }
+            mma_wait();
+            mask_rows([&](int col) { return col > t; }, [&](int col) { return col >= t; });
+            sync_all();
+            if (tid == 0) {
+                acc_pair(448);
+                mma_commit(&s.bar[B2M]);
+            }
+            mma_wait();
+            // ---- readout: final gradients of channels j0 .. j0 + 31 of row t
+            {
+                const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + j0;
+                const size_t ro = tok * kD + j0;
+                float dL[32];
+                float akp[32], aq[32];
+                tm_ld32w(tm, q, 256 + 32 * h, akp);
+                tm_ld32w(tm, q, 320 + 32 * h, aq);
+                const __nv_bfloat16* qsrc = reinterpret_cast<const __nv_bfloat16*>(p.q) + ro;
+                const __nv_bfloat16* gsrc = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + ro;
+                __nv_bfloat16* dq = reinterpret_cast<__nv_bfloat16*>(p.dq) + ro;
+                __nv_bfloat16* dgm = reinterpret_cast<__nv_bfloat16*>(p.dgamma) + ro;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float qv[8], gv[8], o1[8], o2[8];
+                    ld8_bf16(qsrc + 8 * i, qv);
+                    ld8_bf16(gsrc + 8 * i, gv);
+                    const float4 pq0 = __ldg(reinterpret_cast<const float4*>(p.Pq + cb + 8 * i));
+                    const float4 pq1 = __ldg(reinterpret_cast<const float4*>(p.Pq + cb + 8 * i + 4));
+                    const float pq[8] = {pq0.x, pq0.y, pq0.z, pq0.w, pq1.x, pq1.y, pq1.z, pq1.w};
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = 8 * i + u;
+                        const float ep = ex2(L[j] - s.P2[j0 + j]);
+                        const float dqh = aq[j] * ep + pq[u];
+                        o1[u] = dqh * gv[u];
+                        o2[u] = dqh * qv[u];
+                        // dKp Kp + dQp Qp
+                        dL[j] = akp[j] * kv[j] * ep + aq[j] * qv[u] * gv[u] * ep;
+                        akp[j] *= ep;  // dKp 2^(L-P)
+                    }
+                    st8_bf16(dq + 8 * i, o1);
+                    st8_bf16(dgm + 8 * i, o2);
+                }
+                float aa[32], akm[32];
+                tm_ld32w(tm, q, 384 + 32 * h, aa);
+                tm_ld32w(tm, q, 448 + 32 * h, akm);
+                __nv_bfloat16* dk = reinterpret_cast<__nv_bfloat16*>(p.dk) + ro;
+                __nv_bfloat16* de = reinterpret_cast<__nv_bfloat16*>(p.de) + ro;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float o1[8], o2[8];
+                    const float4 pa0 = __ldg(reinterpret_cast<const float4*>(p.Pa + cb + 8 * i));
+                    const float4 pa1 = __ldg(reinterpret_cast<const float4*>(p.Pa + cb + 8 * i + 4));
+                    const float4 pk0 = __ldg(reinterpret_cast<const float4*>(p.Pk + cb + 8 * i));
+                    const float4 pk1 = __ldg(reinterpret_cast<const float4*>(p.Pk + cb + 8 * i + 4));
+                    const float4 pl0 = __ldg(reinterpret_cast<const float4*>(p.PL + cb + 8 * i));
+                    const float4 pl1 = __ldg(reinterpret_cast<const float4*>(p.PL + cb + 8 * i + 4));
+                    const float pa[8] = {pa0.x, pa0.y, pa0.z, pa0.w, pa1.x, pa1.y, pa1.z, pa1.w};
+                    const float pk[8] = {pk0.x, pk0.y, pk0.z, pk0.w, pk1.x, pk1.y, pk1.z, pk1.w};
+                    const float pl[8] = {pl0.x, pl0.y, pl0.z, pl0.w, pl1.x, pl1.y, pl1.z, pl1.w};
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = 8 * i + u;
+                        const float em = ex2(s.P2[j0 + j] - L[j]);
+                        const float da = aa[j] * em + pa[u];
+                        o2[u] = da * kv[j];
+                        o1[u] = akp[j] + akm[j] * em + pk[u] + ev[j] * da;
+                        // - dKm Km - dAm Am + state-side part
+                        dL[j] += -akm[j] * kv[j] * em - aa[j] * ev[j] * kv[j] * em + pl[u];
+                    }
+                    st8_bf16(dk + 8 * i, o1);
+                    st8_bf16(de + 8 * i, o2);
+                }
+                // dg_t = sum_{t' >= t} dL_t' + dLbar: warp suffix scan, then later quarters
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) {
+                        const float o = __shfl_down_sync(0xffffffffu, dL[j], off);
+                        if (lane + off < 32) dL[j] += o;
+                    }
+                }
+                if (lane == 0) {
+#pragma unroll
+                    for (int j = 0; j < 32; ++j) s.sfx[q][j0 + j] = dL[j];
+                }
+                __syncthreads();
+                const float* gin = reinterpret_cast<const float*>(p.dgb) + (size_t)c * kD + j0;
+                __nv_bfloat16* dg = reinterpret_cast<__nv_bfloat16*>(p.dg) + ro;
+                const __nv_bfloat16* graw = reinterpret_cast<const __nv_bfloat16*>(p.g) + ro;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float o[8], gv[8];
+                    ld8_bf16(graw + 8 * i, gv);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const int j = 8 * i + u;
+                        float post = gin[j];
+                        for (int qq = q + 1; qq < 4; ++qq) post += s.sfx[qq][j0 + j];
+                        // the clamp g >= -20 passes no gradient below it
+                        o[u] = gv[u] >= kLogDecayMin ? dL[j] + post : 0.f;
+                    }
+                    st8_bf16(dg + 8 * i, o);
+                }
+            }
+            sync_all();
+        }
+    }
+    if (tid == 0 && s.bad) atomicOr(&g_bwd2_timeouts, (unsigned)s.bad);
+    sync_all();
+    if (warp == 0) tmem_dealloc(tm, 512);
+}
+
+// ------------------------------------------------------------------ host side
+
+namespace {
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                  const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                  const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+int sm_count() {
+    int dev = 0, n = 148;
+    if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    return n;
+}
+
+constexpr int kBprepSmem = 2 * kT16Bytes + 1024;
+constexpr int kBwd1Smem = 6 * kT16Bytes + sizeof(Bwd1Smem) + 1024;
+constexpr int kBwd2Smem = 4 * kT16Bytes + 2 * kT32Half + sizeof(Bwd2Smem) + 1024;
+template <int SLAB>
+constexpr int rev_smem() { return 3 * 128 * 128 * 4 + SLAB * 512 + 1024; }
+
+}  // namespace
+
+size_t bwd2_ws_bytes(int B, int T, int H) {
+    const size_t nch = (size_t)B * H * (T / kC), blk = (size_t)kC * kD * 4;
+    // Bp, dSc, Pq, Pk, Pa, PL (fp32 blocks), Y16, dYR16 (fp16 tiles), dLbar
+    return nch * (6 * blk + 2 * (size_t)kT16Bytes + kD * 4) + 256;
+}
+
+cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
+    const int N = a.T / kC, nch = a.B * a.H * N, BH = a.B * a.H;
+    const size_t blk = (size_t)kC * kD;
+    float* f = reinterpret_cast<float*>(a.ws);
+    float* Bp = f; f += nch * blk;
+    float* dSc = f; f += nch * blk;
+    float* Pq = f; f += nch * blk;
+    float* Pk = f; f += nch * blk;
+    float* Pa = f; f += nch * blk;
+    float* PL = f; f += nch * blk;
+    float* dgb = f; f += (size_t)nch * kD;
+    unsigned char* Y16 = reinterpret_cast<unsigned char*>(f);
+    unsigned char* dYR16 = Y16 + (size_t)nch * kT16Bytes;
+    const int nsm = sm_count();
+    cudaError_t e;
+
+    CUtensorMap tdO;
+    if (!map_tokens16(&tdO, a.dO, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+
+    BprepParams bp;
+    bp.tdO = tdO; bp.T = a.T; bp.H = a.H; bp.Qp = a.Qp; bp.Bp = Bp;
+    if ((e = cudaFuncSetAttribute(k2_bprep, cudaFuncAttributeMaxDynamicSharedMemorySize, kBprepSmem)) != cudaSuccess) return e;
+    MUIR_TIMED("k2_bprep", st, k2_bprep<<<nch, 256, kBprepSmem, st>>>(bp));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    constexpr int SLAB = 32;
+    RevParams rp;
+    if (!map_rows32f(&rp.tMt, a.Mt, (long long)nch * kD)) return cudaErrorInvalidValue;
+    rp.Bp = Bp; rp.S_chunks = a.S_chunks; rp.S_last = a.S_last; rp.dS_final = a.dS_final;
+    rp.dSc = dSc; rp.dS0 = a.dS0; rp.dgb = dgb; rp.N = N;
+    if ((e = cudaMemsetAsync(dgb, 0, (size_t)nch * kD * sizeof(float), st)) != cudaSuccess) return e;
+    if ((e = cudaFuncSetAttribute(k2_chain_rev<SLAB>, cudaFuncAttributeMaxDynamicSharedMemorySize, rev_smem<SLAB>())) != cudaSuccess) return e;
+    MUIR_TIMED("k2_chain_rev", st, k2_chain_rev<SLAB><<<BH * (kD / SLAB), 128, rev_smem<SLAB>(), st>>>(rp));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    const int grid = nch < nsm ? nch : nsm;
+    Bwd1Params p1;
+    p1.tdO = tdO; p1.B = a.B; p1.T = a.T; p1.H = a.H;
+    p1.q = a.q; p1.k = a.k; p1.v = a.v; p1.g = a.g; p1.e = a.e; p1.w = a.w; p1.gamma = a.gamma;
+    p1.aux = a.aux; p1.S_chunks = a.S_chunks; p1.dSc = dSc;
+    p1.Pq = Pq; p1.Pk = Pk; p1.Pa = Pa; p1.PL = PL; p1.Y16 = Y16; p1.dYR16 = dYR16;
+    p1.dv = a.dv; p1.dw = a.dw;
+    if ((e = cudaFuncSetAttribute(k2_bwd1, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwd1Smem)) != cudaSuccess) return e;
+    MUIR_TIMED("k2_bwd1", st, k2_bwd1<<<grid, 512, kBwd1Smem, st>>>(p1));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+    Bwd2Params p2;
+    p2.tdO = tdO; p2.B = a.B; p2.T = a.T; p2.H = a.H;
+    p2.q = a.q; p2.k = a.k; p2.g = a.g; p2.e = a.e; p2.gamma = a.gamma;
+    p2.aux = a.aux; p2.Y16 = Y16; p2.dYR16 = dYR16; p2.Pq = Pq; p2.Pk = Pk; p2.Pa = Pa; p2.PL = PL;
+    p2.dgb = dgb;
+    p2.dq = a.dq; p2.dk = a.dk; p2.dg = a.dg; p2.de = a.de; p2.dgamma = a.dgamma;
+    if ((e = cudaFuncSetAttribute(k2_bwd2, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwd2Smem)) != cudaSuccess) return e;
+    MUIR_TIMED("k2_bwd2", st, k2_bwd2<<<grid, 256, kBwd2Smem, st>>>(p2));
+    return cudaGetLastError();
+}
+
+unsigned int timeouts_bwd2() {
+    unsigned int n = 0;
+    cudaMemcpyFromSymbol(&n, g_bwd2_timeouts, sizeof(n));
+    const unsigned int z = 0;
+    cudaMemcpyToSymbol(g_bwd2_timeouts, &z, sizeof(z));
+    return n;
+}
+
+}  // namespace v2
+}  // namespace muir

@@ -1,0 +1,74 @@
+// bwd2.h -- internal interface of the tensor-core chunk backward with on-chip
+// intermediates (companion of fwd2.h); not part of the C ABI.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stddef.h>
+
+namespace muir {
+namespace v2 {
+
+struct BprepParams {
+    CUtensorMap tdO;
+    int T, H;
+    const float* Qp;  // [nch][128][128]
+    float* Bp;        // Q'^T dO per chunk
+};
+
+struct RevParams {
+    CUtensorMap tMt;        // M_n^T rows of 128 fp32
+    const float* Bp;
+    const float* S_chunks;  // chunk-start states
+    const float* S_last;    // [B*H][128][128] final states (S_N)
+    const float* dS_final;  // or null
+    float* dSc;             // G_{n+1} per chunk
+    float* dS0;             // or null
+    float* dgb;             // dLbar per chunk and channel (zeroed by the host)
+    int N;
+};
+
+struct Bwd1Params {
+    CUtensorMap tdO;
+    int B, T, H;
+    const void *q, *k, *v, *g, *e, *w, *gamma;
+    const unsigned char* aux;
+    const float* S_chunks;
+    const float* dSc;
+    float *Pq, *Pk, *Pa, *PL;
+    unsigned char *Y16, *dYR16;
+    void *dv, *dw;
+};
+
+struct Bwd2Params {
+    CUtensorMap tdO;
+    int B, T, H;
+    const void *q, *k, *g, *e, *gamma;
+    const unsigned char* aux;
+    const unsigned char *Y16, *dYR16;
+    const float *Pq, *Pk, *Pa, *PL, *dgb;
+    void *dq, *dk, *dg, *de, *dgamma;
+};
+
+struct Bwd2Args {
+    int B, T, H;
+    const void *q, *k, *v, *g, *e, *w, *gamma, *dO;
+    const float* dS_final;                  // or null
+    const unsigned char* aux;               // forward's saved records
+    const float *Qp, *Mt, *S_chunks, *S_last;
+    void *dq, *dk, *dv, *dg, *de, *dw, *dgamma;
+    float* dS0;                             // or null
+    void* ws;                               // bwd2_ws_bytes
+};
+
+size_t bwd2_ws_bytes(int B, int T, int H);
+cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st);
+// Bitmask of the wait sites whose bounded wait expired since the last call (then cleared).
+unsigned int timeouts_bwd2();
+
+// Tensor maps shared with fwd2.cu.
+bool map_tokens16(CUtensorMap* m, const void* base, int B, int T, int H);
+bool map_rows32f(CUtensorMap* m, const float* base, long long rows);
+
+}  // namespace v2
+}  // namespace muir

@@ -3,6 +3,7 @@
 // instantiated in chunk_{bf16,f32}_d{64,128}.cu.
 #include "chunk_impl.cuh"
 #include "chunk_units.h"
+#include "bwd2.h"
 #include "fwd2.h"
 
 namespace muir {
@@ -22,18 +23,46 @@ static size_t old_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_stat
 // its first 256 bytes of workspace hold the device flags (span flag first),
 // the rest is shared with the boundary-pivot path, which runs after it and
 // only when the span flag is set.
-static bool use_v2_fwd(const ChunkProblem& P) {
-    return P.aux == nullptr && v2::fwd2_supported(P.B, P.T, P.H, P.D, P.C, P.in_bf16);
+static bool use_v2(const ChunkProblem& P) {
+    return v2::fwd2_supported(P.B, P.T, P.H, P.D, P.C, P.in_bf16);
 }
+
+// Floats of the saved per-chunk intermediates (muir_chunk_aux_floats): the
+// larger of the two paths' formats (the boundary-pivot path writes its own
+// when a chunk's span exceeds the single pivot).
+size_t chunk_aux_total_floats(int B, int T, int H, int D, int C, bool in_bf16) {
+    const size_t nch = (size_t)B * H * ((T + C - 1) / C);
+    const size_t old = nch * chunk_aux_floats(C, D);
+    if (!v2::fwd2_supported(B, T, H, D, C, in_bf16)) return old;
+    const size_t nv2 = v2::aux_bytes(nch, (size_t)B * H) / sizeof(float);
+    return old > nv2 ? old : nv2;
+}
+
+// Workspace of the on-chip forward: flags, then M (unless given), Bn, Q'
+// (unless saved), O_intra, chunk states (unless given).
+static size_t v2_fwd_arrays(size_t nch) { return 5 * nch * 128 * 128 * sizeof(float); }
 
 size_t chunk_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states, bool in_bf16) {
     const size_t old = old_fwd_ws_bytes(B, T, H, D, C, have_states);
     if (!v2::fwd2_supported(B, T, H, D, C, in_bf16)) return old;
-    const size_t nv2 = v2::fwd2_ws_bytes(B, T, H);
+    const size_t nv2 = v2_fwd_arrays((size_t)B * H * (T / C));
     return 256 + (old > nv2 ? old : nv2);
 }
 
-size_t chunk_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states) {
+static size_t old_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states);
+
+// Backward workspace: flags; then (shared with the boundary-pivot path) the
+// on-chip backward's arrays and, when the forward's intermediates are not
+// passed in, a recomputed forward (its arrays and saved records).
+size_t chunk_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states, bool in_bf16) {
+    const size_t old = old_bwd_ws_bytes(B, T, H, D, C, have_states);
+    if (!v2::fwd2_supported(B, T, H, D, C, in_bf16)) return old;
+    const size_t nch = (size_t)B * H * (T / C);
+    const size_t nv2 = v2::bwd2_ws_bytes(B, T, H) + v2_fwd_arrays(nch) + v2::aux_bytes(nch, (size_t)B * H);
+    return 256 + (old > nv2 ? old : nv2);
+}
+
+static size_t old_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states) {
     const size_t nch = (size_t)B * H * ((T + C - 1) / C), DD = (size_t)D * D;
     size_t f = 3 * nch * DD;               // M, Bn / B', dS at chunk ends
     if (!have_states) f += nch * DD;
@@ -44,7 +73,7 @@ size_t chunk_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states) {
 
 cudaError_t run_chunk_fwd(const ChunkProblem& P, const float* S0, void* o, float* S_final,
                           float* S_chunks, float* M_chunks, void* ws, size_t, cudaStream_t st) {
-    if (use_v2_fwd(P)) {
+    if (use_v2(P)) {
         int* flags = static_cast<int*>(ws);
         char* shared = static_cast<char*>(ws) + 256;
         const size_t blk = (size_t)128 * 128;
@@ -55,11 +84,18 @@ cudaError_t run_chunk_fwd(const ChunkProblem& P, const float* S0, void* o, float
         a.q = P.q; a.k = P.k; a.v = P.v; a.g = P.g; a.e = P.e; a.w = P.w; a.gamma = P.gamma;
         a.S0 = S0; a.o = o; a.S_final = S_final;
         a.M = M_chunks ? M_chunks : f; if (!M_chunks) f += nch * blk;
-        a.Mt = nullptr;
         a.Bn = f; f += nch * blk;
-        a.Qp = f; f += nch * blk;
         a.Oi = f; f += nch * blk;
-        a.S_chunks = S_chunks ? S_chunks : f;
+        a.S_chunks = S_chunks ? S_chunks : f; f += nch * blk;
+        if (P.aux) {  // save the intermediates the backward reuses
+            unsigned char* ax = reinterpret_cast<unsigned char*>(P.aux);
+            a.aux = ax;
+            a.Qp = v2::aux_Qp(ax, nch);
+            a.Mt = v2::aux_Mt(ax, nch);
+            a.S_last = v2::aux_SN(ax, nch);
+        } else {
+            a.Qp = f; f += nch * blk;
+        }
         a.flags = flags;
         cudaError_t e = cudaMemsetAsync(flags, 0, 16, st);
         if (e == cudaSuccess) e = v2::span_check(P.g, P.B, P.T, P.H, flags, st);
@@ -81,6 +117,52 @@ cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S
                           const float* M_chunks, const void* dO, const float* dS_final, void* dq, void* dk, void* dv,
                           void* dg, void* de, void* dw, void* dgamma, float* dS0, void* ws,
                           size_t, cudaStream_t st) {
+    if (use_v2(P)) {
+        int* flags = static_cast<int*>(ws);
+        char* shared = static_cast<char*>(ws) + 256;
+        const size_t blk = (size_t)128 * 128;
+        const size_t nch = (size_t)P.B * P.H * P.N;
+        cudaError_t e = cudaMemsetAsync(flags, 0, 16, st);
+        if (e == cudaSuccess) e = v2::span_check(P.g, P.B, P.T, P.H, flags, st);
+        if (e != cudaSuccess) return e;
+        v2::Bwd2Args b = {};
+        b.B = P.B; b.T = P.T; b.H = P.H;
+        b.q = P.q; b.k = P.k; b.v = P.v; b.g = P.g; b.e = P.e; b.w = P.w; b.gamma = P.gamma;
+        b.dO = dO; b.dS_final = dS_final;
+        b.dq = dq; b.dk = dk; b.dv = dv; b.dg = dg; b.de = de; b.dw = dw; b.dgamma = dgamma;
+        b.dS0 = dS0;
+        char* rest = shared;
+        if (P.aux && S_chunks) {  // intermediates saved by the forward
+            unsigned char* ax = reinterpret_cast<unsigned char*>(P.aux);
+            b.aux = ax;
+            b.Qp = v2::aux_Qp(ax, nch);
+            b.Mt = v2::aux_Mt(ax, nch);
+            b.S_last = v2::aux_SN(ax, nch);
+            b.S_chunks = S_chunks;
+        } else {  // recompute the forward's state pass and intermediates
+            float* f = reinterpret_cast<float*>(shared);
+            unsigned char* ax = reinterpret_cast<unsigned char*>(f + 4 * nch * blk);
+            v2::Fwd2Args a = {};
+            a.B = P.B; a.T = P.T; a.H = P.H; a.out_bf16 = false;
+            a.q = P.q; a.k = P.k; a.v = P.v; a.g = P.g; a.e = P.e; a.w = P.w; a.gamma = P.gamma;
+            a.S0 = S0; a.o = nullptr; a.S_final = nullptr;
+            a.M = f; a.Bn = f + nch * blk; a.Oi = f + 2 * nch * blk; a.S_chunks = f + 3 * nch * blk;
+            a.aux = ax;
+            a.Qp = v2::aux_Qp(ax, nch);
+            a.Mt = v2::aux_Mt(ax, nch);
+            a.S_last = v2::aux_SN(ax, nch);
+            a.flags = flags;
+            if ((e = v2::run_fwd2(a, st)) != cudaSuccess) return e;
+            b.aux = ax; b.Qp = a.Qp; b.Mt = a.Mt; b.S_last = a.S_last; b.S_chunks = a.S_chunks;
+            rest = reinterpret_cast<char*>(ax) + v2::aux_bytes(nch, (size_t)P.B * P.H);
+        }
+        b.ws = rest;
+        if ((e = v2::run_bwd2(b, st)) != cudaSuccess) return e;
+        ChunkProblem G = P;
+        G.gate = flags;
+        return bwd_bf16_d128(G, S0, S_chunks, M_chunks, dO, dS_final, dq, dk, dv, dg, de, dw,
+                             dgamma, dS0, shared, st);
+    }
 #define MUIR_BWD_ARGS P, S0, S_chunks, M_chunks, dO, dS_final, dq, dk, dv, dg, de, dw, dgamma, dS0, ws, st
     if (P.in_bf16) {
         if (P.D == 128) return bwd_bf16_d128(MUIR_BWD_ARGS);

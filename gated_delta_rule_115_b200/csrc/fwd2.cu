@@ -29,6 +29,7 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include "bwd2.h"
 #include "fwd2.h"
 #include "profile.h"
 #include "tc2.cuh"
@@ -49,6 +50,19 @@ __device__ __forceinline__ float ex2(float x) {
     float y;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
     return y;
+}
+
+// Rotate a 32-entry register array left by 8: after four calls it is back in
+// order.  Lets a rolled loop over four 8-column chunks use L[0..7] with
+// compile-time indices (the array stays in registers).
+__device__ __forceinline__ void rot8(float (&L)[32]) {
+    float t[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) t[u] = L[u];
+#pragma unroll
+    for (int j = 0; j < 24; ++j) L[j] = L[j + 8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) L[24 + u] = t[u];
 }
 
 __device__ __forceinline__ void bf16_split(float x, float& hi, float& lo) {
@@ -84,6 +98,7 @@ struct IntraSmem {
     float P2[kD];       // pivot (log2 units)
     float eP2[kD];      // 2^P2
     float Lb[kD];       // chunk total (log2 units)
+    float lblk[4][32][33];  // strictly lower 32x32 diagonal blocks of L_A (leaf inverses)
     uint64_t bar[16];
     uint32_t tslot;
     int bad;
@@ -115,6 +130,35 @@ __device__ __forceinline__ void row_st64(unsigned char* tile, int t, int h, cons
     for (int i = 0; i < 8; ++i) st_chunk16<BF16>(tile, t, 8 * h + i, v + 8 * i);
 }
 
+// Store 32 values at columns 32 * c32 .. +32 of row t.
+template <bool BF16>
+__device__ __forceinline__ void row_st32(unsigned char* tile, int t, int c32, const float* v) {
+#pragma unroll
+    for (int i = 0; i < 4; ++i) st_chunk16<BF16>(tile, t, 4 * c32 + i, v + 8 * i);
+}
+
+// TMEM columns [col, col + 32) of this thread's lane, waited.
+__device__ __forceinline__ void tm_ld32w(uint32_t tm, int q, int col, float (&v)[32]) {
+    tmem_ld32(taddr(tm, 32 * q, col), v);
+    tmem_wait_ld();
+}
+
+// Copy 64 TMEM columns (this thread's half h of the 128 columns at tm + base)
+// into row t of a fp16 tile, 32 at a time; mask(col) decides which survive.
+template <class MASK>
+__device__ __forceinline__ void tm_to_tile(uint32_t tm, int base, int q, int h, int t,
+                                           unsigned char* tile, const MASK& mask) {
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+        float v[32];
+        tm_ld32w(tm, q, base + 64 * h + 32 * hh, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (!mask(64 * h + 32 * hh + j)) v[j] = 0.f;
+        row_st32<false>(tile, t, 2 * h + hh, v);
+    }
+}
+
 // Read 64 TMEM columns [col, col + 64) of this thread's lane.
 __device__ __forceinline__ void tm_ld64(uint32_t tm, int q, int col, float* v) {
     float a[32], b[32];
@@ -125,7 +169,10 @@ __device__ __forceinline__ void tm_ld64(uint32_t tm, int q, int col, float* v) {
     for (int i = 0; i < 32; ++i) { v[i] = a[i]; v[32 + i] = b[i]; }
 }
 
-__global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ IntraParams p) {
+// 512 threads: warp w owns rows 32 (w % 4) .. +32 (its TMEM lane quarter q) and
+// columns 32 (w / 4) .. +32 (h); thread t = 32 q + lane owns row t of every
+// per-chunk tile in those columns.  Thread 0 issues the TMA loads and the MMAs.
+__global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ IntraParams p) {
     extern __shared__ __align__(1024) unsigned char smraw[];
     unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
     unsigned char* S[6];
@@ -136,6 +183,7 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = warp & 3, h = warp >> 2;
     const int t = 32 * q + lane;  // row owned by this thread
+    const int c0 = 32 * h;        // first of its 32 columns
     const int N = p.T / kC;
     const int nch = p.B * p.H * N;
 
@@ -172,6 +220,20 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
         load_tile(S[3], &p.tq, y, z, BB);
         load_tile(S[4], &p.tgam, y, z, BB);
     };
+    // this thread's 4 chunks of 8 columns: chunk index 4h + i
+    auto ld32 = [&](const unsigned char* tile, float* v) {
+#pragma unroll
+        for (int i = 0; i < 4; ++i) ld_chunk16<true>(tile, t, 4 * h + i, v + 8 * i);
+    };
+    // TMEM columns base + c0 .. +32 of row t -> fp16 tile, masked by keep(col)
+    auto tm_to_row = [&](int base, unsigned char* tile, auto keep) {
+        float v[32];
+        tm_ld32w(tm, q, base + c0, v);
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+            if (!keep(c0 + j)) v[j] = 0.f;
+        row_st32<false>(tile, t, h, v);
+    };
     if (tid == 0 && (int)blockIdx.x < nch) issue_first(blockIdx.x);
 
     int it = 0;
@@ -180,64 +242,60 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
         uint32_t pg = 0;  // parity of the merge barrier within this chunk
         int y, z;
         coords(c, y, z);
-        const size_t cbase = (size_t)c * kC * kD;  // chunk offset in the per-chunk fp32 arrays
+        const size_t rbase = (size_t)c * kC * kD + (size_t)t * kD + c0;  // row t, column c0
 
-        // ---- 1. log-decay prefix (warp scan over tokens), pivots, span
+        // ---- 1. log-decay prefix (warp scan over tokens), pivots
         waitb(s, BA, ph);
-        float L[64];
-        row_ld64(S[0], t, h, L);
+        float L[32];
+        ld32(S[0], L);
 #pragma unroll
-        for (int j = 0; j < 64; ++j) L[j] = fmaxf(L[j], kLogDecayMin) * kLog2e;
+        for (int j = 0; j < 32; ++j) L[j] = fmaxf(L[j], kLogDecayMin) * kLog2e;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) {
+            for (int j = 0; j < 32; ++j) {
                 const float o = __shfl_up_sync(0xffffffffu, L[j], off);
                 if (lane >= off) L[j] += o;
             }
         }
         if (lane == 31) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) s.tot[q][64 * h + j] = L[j];
+            for (int j = 0; j < 32; ++j) s.tot[q][c0 + j] = L[j];
         }
         __syncthreads();
 #pragma unroll
-        for (int j = 0; j < 64; ++j) {
-            const int col = 64 * h + j;
+        for (int j = 0; j < 32; ++j) {
             float pre = 0.f;
-            for (int qq = 0; qq < q; ++qq) pre += s.tot[qq][col];
+            for (int qq = 0; qq < q; ++qq) pre += s.tot[qq][c0 + j];
             L[j] += pre;
         }
         if (q == 0) {
-            for (int jj = lane; jj < 64; jj += 32) {
-                const int col = 64 * h + jj;
-                const float lb = s.tot[0][col] + s.tot[1][col] + s.tot[2][col] + s.tot[3][col];
-                s.Lb[col] = lb;
-                s.P2[col] = 0.5f * lb;
-                s.eP2[col] = ex2(0.5f * lb);
-            }
+            const int col = c0 + lane;
+            const float lb = s.tot[0][col] + s.tot[1][col] + s.tot[2][col] + s.tot[3][col];
+            s.Lb[col] = lb;
+            s.P2[col] = 0.5f * lb;
+            s.eP2[col] = ex2(0.5f * lb);
         }
         __syncthreads();
 
         // ---- 2. pivoted key operands: Kp -> S0, Km (hi) -> S1, Km (lo) -> S2, Am -> S5
 #pragma unroll 1
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i, rot8(L)) {
             float kv[8], ev[8], kp[8], kmh[8], kml[8], am[8];
-            ld_chunk16<true>(S[1], t, 8 * h + i, kv);
-            ld_chunk16<true>(S[2], t, 8 * h + i, ev);
+            ld_chunk16<true>(S[1], t, 4 * h + i, kv);
+            ld_chunk16<true>(S[2], t, 4 * h + i, ev);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int j = 8 * i + u;
-                const float pv = s.P2[64 * h + j];
-                const float ep = ex2(L[j] - pv), em = ex2(pv - L[j]);
+                const float pv = s.P2[c0 + 8 * i + u];
+                const float ep = ex2(L[u] - pv), em = ex2(pv - L[u]);
                 kp[u] = kv[u] * ep;
                 bf16_split(kv[u] * em, kmh[u], kml[u]);
                 am[u] = ev[u] * kv[u] * em;
             }
-            st_chunk16<true>(S[0], t, 8 * h + i, kp);
-            st_chunk16<true>(S[1], t, 8 * h + i, kmh);
-            st_chunk16<true>(S[2], t, 8 * h + i, kml);
-            st_chunk16<true>(S[5], t, 8 * h + i, am);
+            st_chunk16<true>(S[0], t, 4 * h + i, kp);
+            st_chunk16<true>(S[1], t, 4 * h + i, kmh);
+            st_chunk16<true>(S[2], t, 4 * h + i, kml);
+            st_chunk16<true>(S[5], t, 4 * h + i, am);
         }
         fence_async_smem();
         sync_all();
@@ -247,26 +305,23 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
             mma_commit(&s.bar[BM1]);
         }
 
-        // ---- 3. query operands: Qp hi -> S3, Qp lo -> S4; Q~ -> Qp_out (fp32, completed in step 8)
+        // ---- 3. query operands: Qp hi -> S3, Qp lo -> S4; Q~ -> Qp_out (completed in step 7)
         waitb(s, BB, ph);
 #pragma unroll 1
-        for (int i = 0; i < 8; ++i) {
-            float qv[8], gv[8], qh[8], ql[8];
-            ld_chunk16<true>(S[3], t, 8 * h + i, qv);
-            ld_chunk16<true>(S[4], t, 8 * h + i, gv);
-            float qt[8];
+        for (int i = 0; i < 4; ++i, rot8(L)) {
+            float qv[8], gv[8], qh[8], ql[8], qt[8];
+            ld_chunk16<true>(S[3], t, 4 * h + i, qv);
+            ld_chunk16<true>(S[4], t, 4 * h + i, gv);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int j = 8 * i + u;
-                const float pv = s.P2[64 * h + j];
+                const float pv = s.P2[c0 + 8 * i + u];
                 const float qhat = qv[u] * gv[u];
-                const float qp = qhat * ex2(L[j] - pv);
-                bf16_split(qp, qh[u], ql[u]);
-                qt[u] = qhat * ex2(L[j]);
+                bf16_split(qhat * ex2(L[u] - pv), qh[u], ql[u]);
+                qt[u] = qhat * ex2(L[u]);
             }
-            st_chunk16<true>(S[3], t, 8 * h + i, qh);
-            st_chunk16<true>(S[4], t, 8 * h + i, ql);
-            float* dst = p.Qp + cbase + (size_t)t * kD + 64 * h + 8 * i;
+            st_chunk16<true>(S[3], t, 4 * h + i, qh);
+            st_chunk16<true>(S[4], t, 4 * h + i, ql);
+            float* dst = p.Qp + rbase + 8 * i;
             *reinterpret_cast<float4*>(dst) = make_float4(qt[0], qt[1], qt[2], qt[3]);
             *reinterpret_cast<float4*>(dst + 4) = make_float4(qt[4], qt[5], qt[6], qt[7]);
         }
@@ -280,61 +335,45 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
             mma_commit(&s.bar[BM2]);
         }
 
-        // ---- 4. L_A -> LA16 (S0), leaves of T, L_K -> LK16 (S1)
+        // ---- 4. L_A -> LA16 (S0), leaves of T (32 x 32 diagonal blocks), L_K -> LK16 (S1)
         waitb(s, BM1, ph);
         tc_fence_after();
-        float la[64];
-        tm_ld64(tm + 64 * h, q, 0, la);  // L_A row t, columns 64h..
+        const bool leaf = (h == q);  // warp (q, q) holds L_A[32q + lane][32q .. 32q + 31]
         {
-            float v[64];
+            float la[32];
+            tm_ld32w(tm, q, c0, la);
+            if (leaf) {
 #pragma unroll
-            for (int j = 0; j < 64; ++j) v[j] = (64 * h + j < t) ? la[j] : 0.f;
-            row_st64<false>(S[0], t, h, v);
+                for (int k = 0; k < 32; ++k) s.lblk[q][lane][k] = (k < lane) ? la[k] : 0.f;
+            }
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (c0 + j >= t) la[j] = 0.f;
+            row_st32<false>(S[0], t, h, la);
         }
-        // diagonal 32x32 block q of T: warp (q, q >> 1) holds L_A[32q + lane][32q .. 32q + 31]
-        float tcol[32];
-        const bool leaf = (h == (q >> 1));
-        if (leaf) {
-            const int off = 32 * (q & 1);  // block columns inside this thread's 64
-            float lrow[32];
+        waitb(s, BM2, ph);  // S1..S5 free
+        tc_fence_after();
+        tm_to_row(128, S[1], [&](int col) { return col < t; });
+        // T (S2): zeros outside the diagonal blocks, leaves written column-wise
+        if (!leaf) {
+            float z8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-            for (int k = 0; k < 32; ++k) lrow[k] = (k < lane) ? la[off + k] : 0.f;
-            // lane = column c of the block; tcol[r] = T[r][c]
+            for (int i = 0; i < 4; ++i) st_chunk16<false>(S[2], t, 4 * h + i, z8);
+        } else {
+            // lane = column c of the block; tcol[r] = T[r][c] by forward substitution
+            float tcol[32];
 #pragma unroll
             for (int r = 0; r < 32; ++r) {
                 float acc = (r == lane) ? 1.f : 0.f;
 #pragma unroll
-                for (int k = 0; k < r; ++k) acc -= __shfl_sync(0xffffffffu, lrow[k], r) * tcol[k];
+                for (int k = 0; k < r; ++k) acc -= s.lblk[q][r][k] * tcol[k];
                 tcol[r] = acc;
             }
-        }
-        waitb(s, BM2, ph);  // S1..S5 free
-        tc_fence_after();
-        {
-            float lk[64];
-            tm_ld64(tm + 128 + 64 * h, q, 0, lk);
+            const int col = c0 + lane;
 #pragma unroll
-            for (int j = 0; j < 64; ++j) lk[j] = (64 * h + j < t) ? lk[j] : 0.f;
-            row_st64<false>(S[1], t, h, lk);
-        }
-        // T (S2): zeros outside the diagonal blocks, leaves written column-wise
-        {
-            float z8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-                const int c0 = 64 * h + 8 * i;
-                if (c0 >= 32 * q && c0 < 32 * q + 32) continue;  // diagonal block
-                st_chunk16<false>(S[2], t, 8 * h + i, z8);
-            }
-        }
-        if (leaf) {
-            const int col = 32 * q + lane;
-#pragma unroll
-            for (int r = 0; r < 32; ++r) {
-                const int row = 32 * q + r;
-                __half hv = __float2half_rn(tcol[r]);
-                *reinterpret_cast<__half*>(S[2] + t16_off(row, col >> 3) + (col & 7) * 2) = hv;
-            }
+            for (int r = 0; r < 32; ++r)
+                *reinterpret_cast<__half*>(S[2] + t16_off(32 * q + r, col >> 3) + (col & 7) * 2) =
+                    __float2half_rn(tcol[r]);
         }
         if (tid == 0) {  // v -> S4, w -> S5
             mbar_arrive_expect_tx(&s.bar[BC], 2 * kT16Bytes);
@@ -345,6 +384,12 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
         sync_all();
 
         // ---- 5. block merges of T on tcgen05: P = L21 T11 (into B0), T21 = -T22 P (into B1)
+        unsigned char* ax = p.aux ? p.aux + (size_t)c * AuxLayout::kBytes : nullptr;
+        if (ax && tid == 0) {  // L_K (S1) is final
+            bulk_store(ax + AuxLayout::kLK16, S[1], kT16Bytes);
+            bulk_commit();
+        }
+#pragma unroll 1
         for (int lvl = 0; lvl < 2; ++lvl) {
             const int b = lvl == 0 ? 32 : 64;
             if (tid == 0) {
@@ -356,24 +401,13 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
             }
             waitb(s, BG, pg); pg ^= 1;
             tc_fence_after();
-            // rows of the second halves: level 32 -> quarters 1, 3 (pair q >> 1, columns 64 (q>>1) .. +32)
-            //                            level 64 -> quarters 2, 3 (columns 0 .. 63)
-            const bool mine = (lvl == 0) ? ((q & 1) && h == (q >> 1)) : (q >= 2 && h == 0);
-            const int F = (lvl == 0) ? 64 * (q >> 1) : 0;
+            // second-half rows of each pair and the pair's first-half columns:
+            // level 32: quarters 1 and 3, columns 0..31 / 64..95; level 64: quarters 2, 3, columns 0..63
+            const bool mine = (lvl == 0) ? ((q & 1) && h == 2 * (q >> 1)) : (q >= 2 && h < 2);
             if (mine) {
-                float v[64];
-                if (b == 32) {
-                    float a[32];
-                    tmem_ld32(taddr(tm, 32 * q, F), a);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) st_chunk16<false>(S[3], t, F / 8 + i, a + 8 * i);
-                } else {
-                    tm_ld64(tm, q, 0, v);
-                    row_st64<false>(S[3], t, 0, v);
-                }
-            } else if (b == 32) {
-                tmem_wait_ld();  // keep the warp's tcgen05.ld bookkeeping uniform
+                float a[32];
+                tm_ld32w(tm, q, c0, a);
+                row_st32<false>(S[3], t, h, a);
             }
             fence_async_smem();
             sync_all();
@@ -387,35 +421,36 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
             waitb(s, BG, pg); pg ^= 1;
             tc_fence_after();
             if (mine) {
-                if (b == 32) {
-                    float a[32];
-                    tmem_ld32(taddr(tm + 128, 32 * q, F), a);
-                    tmem_wait_ld();
-#pragma unroll
-                    for (int i = 0; i < 4; ++i) st_chunk16<false>(S[2], t, F / 8 + i, a + 8 * i);
-                } else {
-                    float v[64];
-                    tm_ld64(tm + 128, q, 0, v);
-                    row_st64<false>(S[2], t, 0, v);
-                }
+                float a[32];
+                tm_ld32w(tm + 128, q, c0, a);
+                row_st32<false>(S[2], t, h, a);
             }
             fence_async_smem();
             sync_all();
         }
 
+        if (ax && tid == 0) {  // T (S2) is final
+            bulk_store(ax + AuxLayout::kT16, S[2], kT16Bytes);
+            bulk_commit();
+        }
         // ---- 6. U = w v (S4, in place); L_K U (B0); K~ (S0); X = T [K~ | L_K U] (B0..B1)
         waitb(s, BC, ph);
 #pragma unroll 1
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i) {
             float vv[8], wv[8];
-            ld_chunk16<true>(S[4], t, 8 * h + i, vv);
-            ld_chunk16<true>(S[5], t, 8 * h + i, wv);
+            ld_chunk16<true>(S[4], t, 4 * h + i, vv);
+            ld_chunk16<true>(S[5], t, 4 * h + i, wv);
 #pragma unroll
             for (int u = 0; u < 8; ++u) vv[u] *= wv[u];
-            st_chunk16<false>(S[4], t, 8 * h + i, vv);
+            st_chunk16<false>(S[4], t, 4 * h + i, vv);
         }
         fence_async_smem();
         sync_all();
+        if (ax && tid == 0) {  // U (S4) is final; L_K (S1) is overwritten below
+            bulk_store(ax + AuxLayout::kU16, S[4], kT16Bytes);
+            bulk_commit();
+            bulk_wait_read();
+        }
         if (tid == 0) {
             gemm_km16(tm + 0, a1, 0, a4, 0, 0, 128, 128, kF16, false);  // L_K U
             mma_commit(&s.bar[BM3]);
@@ -424,20 +459,16 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
         }
         waitb(s, BD, ph);
 #pragma unroll 1
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i, rot8(L)) {
             float kv[8];
-            ld_chunk16<true>(S[0], t, 8 * h + i, kv);
+            ld_chunk16<true>(S[0], t, 4 * h + i, kv);
 #pragma unroll
-            for (int u = 0; u < 8; ++u) kv[u] *= ex2(L[8 * i + u]);
-            st_chunk16<false>(S[0], t, 8 * h + i, kv);
+            for (int u = 0; u < 8; ++u) kv[u] *= ex2(L[u]);
+            st_chunk16<false>(S[0], t, 4 * h + i, kv);
         }
         waitb(s, BM3, ph);
         tc_fence_after();
-        {
-            float v[64];
-            tm_ld64(tm + 64 * h, q, 0, v);
-            row_st64<false>(S[1], t, h, v);
-        }
+        tm_to_row(0, S[1], [](int) { return true; });
         fence_async_smem();
         sync_all();
         if (tid == 0) {
@@ -445,34 +476,38 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
             mma_commit(&s.bar[BM4]);
         }
         // M_QK (B2) -> S3, M_QA (B3) -> S5 (inclusive masks)
-        {
-            float v[64];
-            tm_ld64(tm + 256 + 64 * h, q, 0, v);
-#pragma unroll
-            for (int j = 0; j < 64; ++j) v[j] = (64 * h + j <= t) ? v[j] : 0.f;
-            row_st64<false>(S[3], t, h, v);
-            tm_ld64(tm + 384 + 64 * h, q, 0, v);
-#pragma unroll
-            for (int j = 0; j < 64; ++j) v[j] = (64 * h + j <= t) ? v[j] : 0.f;
-            row_st64<false>(S[5], t, h, v);
-        }
+        tm_to_row(256, S[3], [&](int col) { return col <= t; });
+        tm_to_row(384, S[5], [&](int col) { return col <= t; });
         waitb(s, BM4, ph);
         tc_fence_after();
         {
-            float v[64];
-            tm_ld64(tm + 64 * h, q, 0, v);        // W
-            row_st64<false>(S[0], t, h, v);
-            tm_ld64(tm + 128 + 64 * h, q, 0, v);  // U'
-            row_st64<false>(S[1], t, h, v);
+            float v[32];
+            tm_ld32w(tm, q, c0, v);  // W
+            row_st32<false>(S[0], t, h, v);
+            tm_ld32w(tm, q, 128 + c0, v);  // U'
+            row_st32<false>(S[1], t, h, v);
+            if (ax) {
+                float* up = reinterpret_cast<float*>(ax + AuxLayout::kUp) + (size_t)t * kD + c0;
+#pragma unroll
+                for (int j = 0; j < 32; j += 4)
+                    *reinterpret_cast<float4*>(up + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            }
         }
         fence_async_smem();
         sync_all();
+        if (ax && tid == 0) {  // M_QK (S3), M_QA (S5), W (S0) are final
+            bulk_store(ax + AuxLayout::kMQK16, S[3], kT16Bytes);
+            bulk_store(ax + AuxLayout::kMQA16, S[5], kT16Bytes);
+            bulk_store(ax + AuxLayout::kW16, S[0], kT16Bytes);
+            bulk_commit();
+        }
 
         // ---- 7. Z = [Q~ | M_QK U] - M_QA [W | U'] (B2..B3)
         if (tid == 0) {
             gemm_km16(tm + 256, a5, 0, a0, 0, 0, 256, 128, kF16, false, true);
             gemm_km16(tm + 384, a3, 0, a4, 0, 0, 128, 128, kF16, true);
             mma_commit(&s.bar[BM5]);
+            if (ax) bulk_wait_read();                       // T (S2), M_QK (S3) stored
             mbar_arrive_expect_tx(&s.bar[BE], kT16Bytes);  // k -> S2
             load_tile(S[2], &p.tk, y, z, BE);
         }
@@ -483,43 +518,48 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
             load_tile(S[3], &p.te, y, z, BF);
         }
         {
-            float v[64];
-            tm_ld64(tm + 256 + 64 * h, q, 0, v);
-            float* qd = p.Qp + cbase + (size_t)t * kD + 64 * h;
+            float v[32];
+            tm_ld32w(tm + 256, q, c0, v);
+            float* qd = p.Qp + rbase;
 #pragma unroll
-            for (int j = 0; j < 64; j += 4) {
+            for (int j = 0; j < 32; j += 4) {
                 float4 a = *reinterpret_cast<const float4*>(qd + j);
                 a.x += v[j]; a.y += v[j + 1]; a.z += v[j + 2]; a.w += v[j + 3];
                 *reinterpret_cast<float4*>(qd + j) = a;
             }
-            tm_ld64(tm + 384 + 64 * h, q, 0, v);
-            float* od = p.Oi + cbase + (size_t)t * kD + 64 * h;
+            tm_ld32w(tm + 384, q, c0, v);
+            float* od = p.Oi + rbase;
 #pragma unroll
-            for (int j = 0; j < 64; j += 4)
+            for (int j = 0; j < 32; j += 4)
                 *reinterpret_cast<float4*>(od + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         }
         waitb(s, BE, ph);
         waitb(s, BF, ph);
 #pragma unroll 1
-        for (int i = 0; i < 8; ++i) {
+        for (int i = 0; i < 4; ++i, rot8(L)) {
             float kv[8], ev[8];
-            ld_chunk16<true>(S[2], t, 8 * h + i, kv);
-            ld_chunk16<true>(S[3], t, 8 * h + i, ev);
+            ld_chunk16<true>(S[2], t, 4 * h + i, kv);
+            ld_chunk16<true>(S[3], t, 4 * h + i, ev);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const int j = 8 * i + u;
-                const float pv = s.P2[64 * h + j];
-                const float f = ex2(pv - L[j]) * s.eP2[64 * h + j];  // 2^(Lbar - L)
+                const float f = ex2(s.P2[c0 + j] - L[u]) * s.eP2[c0 + j];  // 2^(Lbar - L)
                 kv[u] *= f;
                 ev[u] *= kv[u];
             }
-            st_chunk16<false>(S[2], t, 8 * h + i, kv);
-            st_chunk16<false>(S[3], t, 8 * h + i, ev);
+            st_chunk16<false>(S[2], t, 4 * h + i, kv);
+            st_chunk16<false>(S[3], t, 4 * h + i, ev);
+
         }
         fence_async_smem();
         sync_all();
 
         // ---- 8. [M_n | B_n] = [diag 2^Lbar | Kbar^T U] - Abar^T [W | U'] (B0..B1)
+        if (ax && tid == 0) {  // Kbar (S2), Abar (S3) are final
+            bulk_store(ax + AuxLayout::kKbar16, S[2], kT16Bytes);
+            bulk_store(ax + AuxLayout::kAbar16, S[3], kT16Bytes);
+            bulk_commit();
+        }
         if (tid == 0) {
             gemm_mm16(tm + 0, a3, 0, 0, a0, 0, 0, 256, 128, kF16, false, true);
             gemm_mm16(tm + 128, a2, 0, 0, a4, 0, 0, 128, 128, kF16, true);
@@ -528,31 +568,35 @@ __global__ void __launch_bounds__(256, 1) k2_intra(const __grid_constant__ Intra
         waitb(s, BM6, ph);
         tc_fence_after();
         const int cn = c + gridDim.x;
+        if (tid == 0 && ax) bulk_wait_read();  // M_QA (S5) stored before S5 is reused
         if (tid == 0 && cn < nch) issue_first(cn);
         {
-            float v[64];
-            tm_ld64(tm + 64 * h, q, 0, v);
-            float* md = p.M + cbase + (size_t)t * kD + 64 * h;
-            const float dg = ex2(s.Lb[t]);
+            float v[32];
+            tm_ld32w(tm, q, c0, v);
+            if (t >= c0 && t < c0 + 32) {
+                const float dg = ex2(s.Lb[t]);
 #pragma unroll
-            for (int j = 0; j < 64; ++j)
-                if (64 * h + j == t) v[j] += dg;
+                for (int j = 0; j < 32; ++j)
+                    if (c0 + j == t) v[j] += dg;
+            }
+            float* md = p.M + rbase;
 #pragma unroll
-            for (int j = 0; j < 64; j += 4)
+            for (int j = 0; j < 32; j += 4)
                 *reinterpret_cast<float4*>(md + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
             if (p.Mt) {
-                float* mt = p.Mt + cbase + t;
+                float* mt = p.Mt + (size_t)c * kC * kD + t;
 #pragma unroll 8
-                for (int j = 0; j < 64; ++j) mt[(size_t)(64 * h + j) * kD] = v[j];
+                for (int j = 0; j < 32; ++j) mt[(size_t)(c0 + j) * kD] = v[j];
             }
-            tm_ld64(tm + 128 + 64 * h, q, 0, v);
-            float* bd = p.Bn + cbase + (size_t)t * kD + 64 * h;
+            tm_ld32w(tm + 128, q, c0, v);
+            float* bd = p.Bn + rbase;
 #pragma unroll
-            for (int j = 0; j < 64; j += 4)
+            for (int j = 0; j < 32; j += 4)
                 *reinterpret_cast<float4*>(bd + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         }
         sync_all();  // TMEM read out before the next chunk's products
     }
+    if (tid == 0) bulk_wait_all();
     if (tid == 0 && s.bad) atomicAdd(&g_v2_timeouts, 1u);
     sync_all();
     if (warp == 0) tmem_dealloc(tm, 512);
@@ -631,8 +675,11 @@ __global__ void __launch_bounds__(128, 1) k2_chain(const __grid_constant__ Chain
 #pragma unroll
             for (int c = 0; c < SLAB; c += 4) *reinterpret_cast<float4*>(d + c) = make_float4(Sr[c], Sr[c + 1], Sr[c + 2], Sr[c + 3]);
         }
-        if (!mbar_wait(&bar[st], (uint32_t)((n / STAGES) & 1))) bad = 1;
+        // only the issuing thread waits for the transition tile: it alone reads it
+        // (through the MMA), and it reloads the stage later in this step, so a
+        // second waiter could see the barrier two phases on and miss its phase
         if (tid == 0) {
+            if (!mbar_wait(&bar[st], (uint32_t)((n / STAGES) & 1))) bad = 1;
             tc_fence_after();
             gemm_kk32<128, SLAB>(tm, saddr(Mst + st * MT), saddr(St), 0, SLAB, 128, false);
             mma_commit(&bar[STAGES]);
@@ -653,8 +700,10 @@ __global__ void __launch_bounds__(128, 1) k2_chain(const __grid_constant__ Chain
         fence_async_smem();
         sync_all();
     }
-    if (p.S_final) {
-        float* d = p.S_final + sbase;
+    float* fin[2] = {p.S_final, p.S_last};
+    for (int i = 0; i < 2; ++i) {
+        if (!fin[i]) continue;
+        float* d = fin[i] + sbase;
 #pragma unroll
         for (int c = 0; c < SLAB; c += 4) *reinterpret_cast<float4*>(d + c) = make_float4(Sr[c], Sr[c + 1], Sr[c + 2], Sr[c + 3]);
     }
@@ -716,8 +765,8 @@ __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutPara
         }
         fence_async_smem();
         sync_all();
-        if (!mbar_wait(&bar[0], (uint32_t)(it & 1))) bad = 1;
-        if (tid == 0) {
+        if (tid == 0) {  // Q' is read by the MMA only; its issuer alone waits for it
+            if (!mbar_wait(&bar[0], (uint32_t)(it & 1))) bad = 1;
             tc_fence_after();
             gemm_kk32<128, 128>(tm, saddr(Qt), saddr(St), 0, 128, 128, false);
             mma_commit(&bar[1]);
@@ -773,7 +822,7 @@ static EncodeTiledFn encode_fn() {
 }
 
 // Map over a token-major [B*T][H][128] bf16 tensor: box of 64 channels x 1 head x 128 tokens.
-static bool map_tokens(CUtensorMap* m, const void* base, int B, int T, int H) {
+bool map_tokens16(CUtensorMap* m, const void* base, int B, int T, int H) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)B * T};
@@ -786,7 +835,7 @@ static bool map_tokens(CUtensorMap* m, const void* base, int B, int T, int H) {
 }
 
 // Map over rows of 128 fp32 (a [rows][128] array): box of 32 columns x 128 rows.
-static bool map_rows32(CUtensorMap* m, const float* base, long long rows) {
+bool map_rows32f(CUtensorMap* m, const float* base, long long rows) {
     EncodeTiledFn enc = encode_fn();
     if (!enc) return false;
     cuuint64_t dims[3] = {128, (cuuint64_t)rows, 1};
@@ -831,24 +880,26 @@ cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st) {
     if (!encode_fn()) return cudaErrorNotSupported;
     const int N = a.T / kC, nch = a.B * a.H * N, BH = a.B * a.H;
     IntraParams ip;
-    if (!map_tokens(&ip.tq, a.q, a.B, a.T, a.H) || !map_tokens(&ip.tk, a.k, a.B, a.T, a.H) ||
-        !map_tokens(&ip.tv, a.v, a.B, a.T, a.H) || !map_tokens(&ip.tg, a.g, a.B, a.T, a.H) ||
-        !map_tokens(&ip.te, a.e, a.B, a.T, a.H) || !map_tokens(&ip.tw, a.w, a.B, a.T, a.H) ||
-        !map_tokens(&ip.tgam, a.gamma, a.B, a.T, a.H))
+    if (!map_tokens16(&ip.tq, a.q, a.B, a.T, a.H) || !map_tokens16(&ip.tk, a.k, a.B, a.T, a.H) ||
+        !map_tokens16(&ip.tv, a.v, a.B, a.T, a.H) || !map_tokens16(&ip.tg, a.g, a.B, a.T, a.H) ||
+        !map_tokens16(&ip.te, a.e, a.B, a.T, a.H) || !map_tokens16(&ip.tw, a.w, a.B, a.T, a.H) ||
+        !map_tokens16(&ip.tgam, a.gamma, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
     ip.B = a.B; ip.T = a.T; ip.H = a.H;
     ip.M = a.M; ip.Mt = a.Mt; ip.Bn = a.Bn; ip.Qp = a.Qp; ip.Oi = a.Oi; ip.flags = a.flags;
+    ip.aux = a.aux;
     cudaError_t e = cudaFuncSetAttribute(k2_intra, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);
     if (e != cudaSuccess) return e;
     const int nsm = sm_count();
     const int grid = nch < nsm ? nch : nsm;
-    MUIR_TIMED("k2_intra", st, k2_intra<<<grid, 256, kIntraSmem, st>>>(ip));
+    MUIR_TIMED("k2_intra", st, k2_intra<<<grid, 512, kIntraSmem, st>>>(ip));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     constexpr int SLAB = 32;
     ChainParams cp;
-    if (!map_rows32(&cp.tM, a.M, (long long)nch * kD)) return cudaErrorInvalidValue;
+    if (!map_rows32f(&cp.tM, a.M, (long long)nch * kD)) return cudaErrorInvalidValue;
     cp.Bn = a.Bn; cp.S0 = a.S0; cp.S_chunks = a.S_chunks; cp.S_final = a.S_final; cp.N = N;
+    cp.S_last = a.S_last;
     e = cudaFuncSetAttribute(k2_chain<SLAB>, cudaFuncAttributeMaxDynamicSharedMemorySize, chain_smem<SLAB>());
     if (e != cudaSuccess) return e;
     MUIR_TIMED("k2_chain", st, k2_chain<SLAB><<<BH * (kD / SLAB), 128, chain_smem<SLAB>(), st>>>(cp));
@@ -856,7 +907,7 @@ cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st) {
 
     if (a.o) {
         OutParams op;
-        if (!map_rows32(&op.tQ, a.Qp, (long long)nch * kC)) return cudaErrorInvalidValue;
+        if (!map_rows32f(&op.tQ, a.Qp, (long long)nch * kC)) return cudaErrorInvalidValue;
         op.B = a.B; op.T = a.T; op.H = a.H;
         op.S_chunks = a.S_chunks; op.Oi = a.Oi; op.o = a.o;
         if (a.out_bf16) {

@@ -11,6 +11,39 @@ namespace v2 {
 
 // Per-chunk fp32 arrays are indexed by chunk c = (b * H + h) * N + n, each
 // chunk a row-major 128 x 128 block.
+
+// Per-chunk intermediates the forward saves for the backward ("aux"), byte
+// offsets inside one chunk's record.  16-bit tiles are stored byte for byte in
+// the 128B-swizzled shared-memory tile layout (tc2.cuh, T16) so the backward
+// reloads them with plain bulk copies; fp32 blocks are row-major 128 x 128.
+struct AuxLayout {
+    static constexpr size_t kT16 = 0;                 // T = (I + L_A)^-1, fp16 tile
+    static constexpr size_t kLK16 = 1 * 32768;        // strict(L_K), fp16 tile
+    static constexpr size_t kMQK16 = 2 * 32768;       // incl(M_QK), fp16 tile
+    static constexpr size_t kMQA16 = 3 * 32768;       // incl(M_QA), fp16 tile
+    static constexpr size_t kU16 = 4 * 32768;         // U = w * v, fp16 tile
+    static constexpr size_t kW16 = 5 * 32768;         // W = T K~, fp16 tile
+    static constexpr size_t kAbar16 = 6 * 32768;      // Abar, fp16 tile
+    static constexpr size_t kKbar16 = 7 * 32768;      // Kbar, fp16 tile
+    static constexpr size_t kUp = 8 * 32768;          // U' = T L_K U, fp32 [t][c]
+    static constexpr size_t kBytes = 8 * 32768 + 65536;
+};
+// The aux buffer: nch records, then Q' [nch][128][128] fp32, then M^T
+// [nch][128][128] fp32 (the reverse state pass reads M_n^T), then the final
+// states S_N [B*H][128][128] fp32.
+inline size_t aux_bytes(size_t nch, size_t bh) {
+    return nch * (AuxLayout::kBytes + 2 * 65536) + bh * 65536;
+}
+inline float* aux_SN(unsigned char* aux, size_t nch) {
+    return reinterpret_cast<float*>(aux + nch * (AuxLayout::kBytes + 2 * 65536));
+}
+inline float* aux_Qp(unsigned char* aux, size_t nch) {
+    return reinterpret_cast<float*>(aux + nch * AuxLayout::kBytes);
+}
+inline float* aux_Mt(unsigned char* aux, size_t nch) {
+    return reinterpret_cast<float*>(aux + nch * (AuxLayout::kBytes + 65536));
+}
+
 struct IntraParams {
     CUtensorMap tq, tk, tv, tg, te, tw, tgam;  // token-major [B*T][H][128] bf16
     int B, T, H;
@@ -19,6 +52,7 @@ struct IntraParams {
     float* Bn;     // B_n [j][c]
     float* Qp;     // Q'_n [t][i]: O_n = Q'_n S_n + O_intra_n
     float* Oi;     // O_intra_n [t][c]
+    unsigned char* aux;  // per-chunk AuxLayout records, or null (nothing saved)
     int* flags;
 };
 
@@ -28,6 +62,7 @@ struct ChainParams {
     const float* S0;     // [B*H][128][128] or null
     float* S_chunks;     // [B*H][N][128][128] or null
     float* S_final;      // [B*H][128][128] or null
+    float* S_last;       // second copy of S_N (saved for the backward) or null
     int N;
 };
 
@@ -48,6 +83,8 @@ struct Fwd2Args {
     float* S_final;      // may be null
     float* S_chunks;     // required
     float *M, *Mt, *Bn, *Qp, *Oi;
+    float* S_last;       // copy of S_N for the backward, or null
+    unsigned char* aux;  // null, or nch AuxLayout records
     int* flags;
 };
 

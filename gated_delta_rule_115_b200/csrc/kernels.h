@@ -44,7 +44,8 @@ size_t chunk_aux_floats(int C, int D);
 
 // Workspace carving (bytes) for the chunk forward / backward.
 size_t chunk_fwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states, bool in_bf16);
-size_t chunk_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states);
+size_t chunk_bwd_ws_bytes(int B, int T, int H, int D, int C, bool have_states, bool in_bf16);
+size_t chunk_aux_total_floats(int B, int T, int H, int D, int C, bool in_bf16);
 
 cudaError_t run_chunk_fwd(const ChunkProblem& P, const float* S0, void* o, float* S_final,
                           float* S_chunks, float* M_chunks, void* ws, size_t ws_bytes,

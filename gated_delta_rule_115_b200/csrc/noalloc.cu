@@ -20,8 +20,11 @@
 //   every scratch element before reading it, so nothing has to be cleared
 //   between calls.
 // - The first call on each device looks up the array's device address
-//   (cudaGetSymbolAddress) with that device current; make that first call
-//   before any stream capture.
+//   (cudaGetSymbolAddress) with that device current and keeps it for later
+//   calls; make that first call before any stream capture.  The address
+//   belongs to the device's primary context: after cudaDeviceReset (or any
+//   other teardown of that context) the kept address is stale, so a process
+//   that resets a device must not call this entry point on it again.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -69,6 +72,13 @@ extern "C" muir_status muir_chunk_fwd_noalloc(const muir_shape* shape, const voi
         return muir_chunk_fwd(shape, q, k, v, g, e, w, gamma, S0, o, S_final, nullptr, nullptr,
                               nullptr, nullptr, 0, stream);
     if (need > kStaticScratchBytes) return MUIR_ERR_WORKSPACE;
+    // The library holds sm_100a code only: on another device the symbol lookup
+    // would fail; report that as every other entry point does.
+    int dev = 0, major = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess)
+        return MUIR_ERR_CUDA;
+    if (major != 10) return MUIR_ERR_UNSUPPORTED;
     void* ws = nullptr;
     if (scratch_address(&ws) != cudaSuccess) return MUIR_ERR_CUDA;
     return muir_chunk_fwd(shape, q, k, v, g, e, w, gamma, S0, o, S_final, nullptr, nullptr, nullptr,

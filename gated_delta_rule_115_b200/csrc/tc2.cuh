@@ -94,6 +94,36 @@ __device__ __forceinline__ void tma_load_3d(void* dst, const CUtensorMap* map, i
         : "memory");
 }
 
+// Untiled bulk copy global -> shared (bytes % 16 == 0, both 16-byte aligned),
+// completion counted on `bar`.  No multicast.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            saddr(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(saddr(bar))
+        : "memory");
+}
+
+// Untiled bulk copy shared -> global in this thread's bulk group; call
+// bulk_commit() after a batch and bulk_wait_read() before the shared source
+// is overwritten (fence_async_smem() + barrier before issuing, so generic
+// writes to the source are visible).
+__device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(
+                     reinterpret_cast<uint64_t>(dst)),
+                 "r"(saddr(src)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() {
+    asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+
 __device__ __forceinline__ void prefetch_tmap(const CUtensorMap* map) {
     asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(map)) : "memory");
 }
@@ -242,6 +272,22 @@ __device__ __forceinline__ void mma_tf32(uint32_t d, uint64_t a, uint64_t b, uin
         "l"(a), "l"(b), "r"(id), "r"(acc));
 }
 
+// kind::tf32 with A read from tensor memory (lane m = row m, one fp32 per
+// column along K) and B from a shared-memory descriptor.
+__device__ __forceinline__ void mma_tf32_ta(uint32_t d, uint32_t a_tmem, uint64_t b, uint32_t id,
+                                            uint32_t acc) {
+    asm volatile(
+        "{\n.reg .pred p;\nsetp.ne.b32 p, %4, 0;\n"
+        "tcgen05.mma.cta_group::1.kind::tf32 [%0], [%1], %2, %3, p;\n}" ::"r"(d),
+        "r"(a_tmem), "l"(b), "r"(id), "r"(acc));
+}
+
+__device__ __forceinline__ float tf32_round(float x) {
+    uint32_t r;
+    asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+    return __uint_as_float(r);
+}
+
 // Arrive on `bar` once every MMA this thread issued so far has completed.
 __device__ __forceinline__ void mma_commit(uint64_t* bar) {
     asm volatile(
@@ -306,12 +352,12 @@ __device__ __forceinline__ uint32_t t32_off(int r, int c) {
 }
 
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
-    __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
+    return (uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(a)) |
+           ((uint32_t)__bfloat16_as_ushort(__float2bfloat16_rn(b)) << 16);
 }
 __device__ __forceinline__ uint32_t pack_f16(float a, float b) {
-    __half2 h = __floats2half2_rn(a, b);
-    return *reinterpret_cast<uint32_t*>(&h);
+    return (uint32_t)__half_as_ushort(__float2half_rn(a)) |
+           ((uint32_t)__half_as_ushort(__float2half_rn(b)) << 16);
 }
 
 template <bool BF16>
@@ -330,23 +376,26 @@ __device__ __forceinline__ void st_chunk16(unsigned char* tile, int r, int c, co
     *reinterpret_cast<uint4*>(tile + t16_off(r, c)) = u;
 }
 
+// Two 16-bit values packed in a word -> floats.
+template <bool BF16>
+__device__ __forceinline__ void unpack16(uint32_t w, float& lo, float& hi) {
+    if (BF16) {
+        lo = __uint_as_float(w << 16);
+        hi = __uint_as_float(w & 0xFFFF0000u);
+    } else {
+        lo = __half2float(__ushort_as_half((unsigned short)(w & 0xFFFFu)));
+        hi = __half2float(__ushort_as_half((unsigned short)(w >> 16)));
+    }
+}
+
 // Load 8 values of chunk c of row r of a T16 tile.
 template <bool BF16>
 __device__ __forceinline__ void ld_chunk16(const unsigned char* tile, int r, int c, float* v) {
     const uint4 u = *reinterpret_cast<const uint4*>(tile + t16_off(r, c));
-    const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-        if (BF16) {
-            const __nv_bfloat162 h = *reinterpret_cast<const __nv_bfloat162*>(&w[i]);
-            const float2 f = __bfloat1622float2(h);
-            v[2 * i] = f.x; v[2 * i + 1] = f.y;
-        } else {
-            const __half2 h = *reinterpret_cast<const __half2*>(&w[i]);
-            const float2 f = __half22float2(h);
-            v[2 * i] = f.x; v[2 * i + 1] = f.y;
-        }
-    }
+    unpack16<BF16>(u.x, v[0], v[1]);
+    unpack16<BF16>(u.y, v[2], v[3]);
+    unpack16<BF16>(u.z, v[4], v[5]);
+    unpack16<BF16>(u.w, v[6], v[7]);
 }
 
 }  // namespace t2

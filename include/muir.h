@@ -195,7 +195,10 @@ muir_status muir_chunk_bwd_varlen(const muir_shape* shape, int num_seqs,
  *   - All calls share the array: calls that overlap on the GPU race; order
  *     them (one stream).  No state carries over between calls.
  *   - The first call on each device looks up the array's device address with
- *     that device current; make it before any stream capture.
+ *     that device current and keeps it; make it before any stream capture.
+ *     A device reset (cudaDeviceReset) after that first call is not
+ *     supported: the kept address would be stale.
+ *   - MUIR_ERR_UNSUPPORTED on a device that is not compute capability 10.x.
  */
 muir_status muir_chunk_fwd_noalloc(const muir_shape* shape, const void* q, const void* k,
                                    const void* v, const void* g, const void* e, const void* w,
