@@ -54,12 +54,8 @@ BYTES_BWD = 8 * 256 + 7 * 256        # 7 inputs + dO read, 7 gradients written
 DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 6 * 128 * 2 + 128 * 2  # S read+write, tokens, o
 
 # DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
-# keyed by kernel; valid only while the kernel source hash matches.
-NCU_TRAFFIC = {
-    # profiles/k_bwd_k_out_B1_H16_T8192_d128_C128.md: 6.410 GB for 131,072 token-heads;
-    # source = source_hash(chunk_kernels_only=True) of the captured build
-    "k_bwd": {"bytes_per_token_head": 6.4104e9 / 131072, "source": "0b6a614d9c25e16a"},
-}
+# keyed by kernel; valid only while the chunk-kernel source hash matches.
+NCU_TRAFFIC = {}
 
 
 def source_hash(chunk_kernels_only: bool = False) -> str:
@@ -319,7 +315,7 @@ def gpu_arm(args, rank, world, local):
     out = {
         "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms,
-        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "tf32",
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16+fp16+tf32",
         "data": "synthetic", "config": workload_config(W.T),
         "tflops": tflops, "tc_peak_frac": tflops / peaks["bf16_tflops"],
         "hbm_gbs_algorithmic": (BYTES_FWD + BYTES_BWD) * token_heads * world / (ms / 1e3) / 1e9,
@@ -356,17 +352,30 @@ def load_peaks():
                 "source": "fallback"}
 
 
-def kernel_roofline(name, avg_ms, token_heads, C, d, peaks):
-    """Roofline of one launch of the dominant kernel from its algorithmic work."""
+def kernel_work(name, C, d):
+    """Algorithmic (bytes, flops) per token-head credited to one launch of a
+    chunk kernel: each product counted once at 2 flops per multiply-add, the
+    decay-masked and triangular ones at half size; bytes = the bf16 inputs the
+    kernel reads and the outputs it writes (saved intermediates excluded)."""
     F = flops_fwd_per_token_head(C, d)
-    work = {  # (algorithmic bytes, algorithmic flops) per token-head
-        "k_bwd": (BYTES_BWD, 2 * F),
-        "k_out": (BYTES_FWD, F),
-        "k_intra": (5 * 256, F),
-        "k_bprep": (6 * 256, F),
-        "k_chain": (2 * d * d * 4 / C, 2 * d * d * d / C),
-        "k_chain_rev": (2 * d * d * 4 / C, 2 * d * d * d / C),
+    return {
+        # 8 decay-masked gradient products and the 4 dL matrices they use
+        "k2_bwd2": (11 * 256, 12 * C * d),
+        # Y, dY, dYR, dU and the four state-side products
+        "k2_bwd1": (10 * 256, 4 * C * d + 14 * d * d),
+        # masked products, inverse, solve, Z and the chunk transition
+        "k2_intra": (7 * 256, 10 * C * d + C * C / 3 + 6 * d * d),
+        "k2_chain": (2 * d * d * 4 / C, 2 * d * d * d / C),
+        "k2_chain_rev": (2 * d * d * 4 / C, 2 * d * d * d / C),
+        "k2_out": (256, 2 * d * d),
     }.get(name, (BYTES_FWD, F))
+
+
+def kernel_roofline(name, avg_ms, token_heads, C, d, peaks):
+    """Roofline of one launch of the dominant kernel from its algorithmic work.
+    The tensor peak is TF32 (sustained bf16 x 1.1/2.25): the kernels mix TF32
+    products with 16-bit ones, so TF32 is the lower of the two ceilings."""
+    work = kernel_work(name, C, d)
     byts = work[0] * token_heads
     fl = work[1] * token_heads
     gbs = byts / (avg_ms / 1e3) / 1e9

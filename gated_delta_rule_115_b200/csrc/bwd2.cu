@@ -102,31 +102,32 @@ __device__ __forceinline__ void tm_ld32w(uint32_t tm, int q, int col, float (&v)
     tmem_wait_ld();
 }
 
-// Chunk-local cumulative log decay (log2 units) of this thread's row t and 32
-// channels j0..j0+31, by a warp scan over tokens plus the totals of the
+// Chunk-local cumulative log decay (log2 units) of this thread's row t and W
+// channels j0..j0+W-1, by a warp scan over tokens plus the totals of the
 // earlier 32-token quarters (tot: [4][128] floats in shared memory, written
-// here).  Ends with a block barrier; tot then holds the quarter totals.
+// here).  Ends after a block barrier; tot then holds the quarter totals.
+template <int W>
 __device__ __forceinline__ void log_decay(const __nv_bfloat16* g, int lane, int q, int j0,
-                                          float (*tot)[kD], float (&L)[32]) {
+                                          float (*tot)[kD], float (&L)[W]) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) ld8_bf16(g + j0 + 8 * i, L + 8 * i);
+    for (int i = 0; i < W / 8; ++i) ld8_bf16(g + j0 + 8 * i, L + 8 * i);
 #pragma unroll
-    for (int j = 0; j < 32; ++j) L[j] = fmaxf(L[j], kLogDecayMin) * kLog2e;
+    for (int j = 0; j < W; ++j) L[j] = fmaxf(L[j], kLogDecayMin) * kLog2e;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
+        for (int j = 0; j < W; ++j) {
             const float o = __shfl_up_sync(0xffffffffu, L[j], off);
             if (lane >= off) L[j] += o;
         }
     }
     if (lane == 31) {
 #pragma unroll
-        for (int j = 0; j < 32; ++j) tot[q][j0 + j] = L[j];
+        for (int j = 0; j < W; ++j) tot[q][j0 + j] = L[j];
     }
     __syncthreads();
 #pragma unroll
-    for (int j = 0; j < 32; ++j) {
+    for (int j = 0; j < W; ++j) {
         float pre = 0.f;
         for (int qq = 0; qq < q; ++qq) pre += tot[qq][j0 + j];
         L[j] += pre;
@@ -214,9 +215,9 @@ __global__ void __launch_bounds__(256) k2_bprep(const __grid_constant__ BprepPar
 // ------------------------------------------------------------------ k2_chain_rev
 
 // G_n = M_n^T G_{n+1} + B'_n for one head and SLAB value columns, n = N-1 .. 0;
-// records G_{n+1} in dSc[n], adds this slab's share of
-// dLbar[n][j] = sum_c G_{n+1}[j][c] S_{n+1}[j][c] (dLbar zeroed beforehand) and
-// writes G_0 to dS0.  M_n^T streams through a 3-stage TMA ring (K-major TF32).
+// records G_{n+1} in dSc[n], writes this slab's share of
+// dLbar[n][j] = sum_c G_{n+1}[j][c] S_{n+1}[j][c] to its own slot (dgb[slab][n][j])
+// and writes G_0 to dS0.  M_n^T streams through a 3-stage TMA ring (K-major TF32).
 template <int SLAB>
 __global__ void __launch_bounds__(128, 1) k2_chain_rev(const __grid_constant__ RevParams p) {
     constexpr int STAGES = 3;
@@ -278,7 +279,8 @@ __global__ void __launch_bounds__(128, 1) k2_chain_rev(const __grid_constant__ R
                 const float4 sv = __ldg(reinterpret_cast<const float4*>(sn1 + c));
                 acc += Gr[c] * sv.x + Gr[c + 1] * sv.y + Gr[c + 2] * sv.z + Gr[c + 3] * sv.w;
             }
-            atomicAdd(p.dgb + ((size_t)bh * N + n) * kD + j, acc);
+            // one partial per value slab, summed in a fixed order by k2_bwd2
+            p.dgb[((size_t)(c0 / SLAB) * p.nch + (size_t)bh * N + n) * kD + j] = acc;
         }
         // only the issuing thread waits for M_n^T (see k2_chain)
         if (tid == 0) {
@@ -409,7 +411,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
         }
         // log decay of row t, columns c0..; E = 2^L, Eb = 2^(Lbar - L)
         float L[32];
-        log_decay(reinterpret_cast<const __nv_bfloat16*>(p.g) + tok * kD, lane, q, c0, s.tot, L);
+        log_decay<32>(reinterpret_cast<const __nv_bfloat16*>(p.g) + tok * kD, lane, q, c0, s.tot, L);
         if (q == 0) s.Lb[c0 + lane] = chunk_total(s.tot, c0 + lane);
         // S_n / sS -> fp16 tile S0, G / sG -> fp16 tile S3 (row j = t)
         float sS, sG;
@@ -454,17 +456,12 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             gemm_km16(tm + 128, a[2], 0, a[0], 0, 0, 128, 128, kF16, false);
             mma_commit(&s.bar[B1M1]);
         }
-        float kv[32], ev[32];
-        {
-            const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(p.k) + ro;
-            const __nv_bfloat16* ep = reinterpret_cast<const __nv_bfloat16*>(p.e) + ro;
-#pragma unroll
-            for (int i = 0; i < 4; ++i) { ld8_bf16(kp + 8 * i, kv + 8 * i); ld8_bf16(ep + 8 * i, ev + 8 * i); }
-        }
+        const __nv_bfloat16* kin = reinterpret_cast<const __nv_bfloat16*>(p.k) + ro;
+        const __nv_bfloat16* ein = reinterpret_cast<const __nv_bfloat16*>(p.e) + ro;
         waitb(B1M1, ph);
         tc_fence_after();
         // ---- phase 2: Pq, PL (dQ~ part); Y = W S + U' -> fp16 tile S2 (also saved for k2_bwd2)
-        float PL[32];
+        float* pl = p.PL + cb;  // the state-side part of dLog, accumulated over phases 2, 3, 6
         {
             float d[32], qv[8], gv[8];
             tm_ld32w(tm, q, c0, d);
@@ -475,15 +472,17 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             for (int i = 0; i < 4; ++i) {
                 ld8_bf16(qp + 8 * i, qv);
                 ld8_bf16(gp + 8 * i, gv);
-                float o[8];
+                float o[8], r[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int j = 8 * i + u;
                     o[u] = d[j] * sS * ex2(L[j]);
-                    PL[j] = o[u] * qv[u] * gv[u];  // dQ~ . Q~
+                    r[u] = o[u] * qv[u] * gv[u];  // dQ~ . Q~
                 }
                 *reinterpret_cast<float4*>(pq + 8 * i) = make_float4(o[0], o[1], o[2], o[3]);
                 *reinterpret_cast<float4*>(pq + 8 * i + 4) = make_float4(o[4], o[5], o[6], o[7]);
+                *reinterpret_cast<float4*>(pl + 8 * i) = make_float4(r[0], r[1], r[2], r[3]);
+                *reinterpret_cast<float4*>(pl + 8 * i + 4) = make_float4(r[4], r[5], r[6], r[7]);
             }
             tm_ld32w(tm, q, 128 + c0, d);
             const float* up = reinterpret_cast<const float*>(ax + AuxLayout::kUp) + (size_t)t * kD + c0;
@@ -516,32 +515,33 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
         }
         // ---- phase 3: Pk (dKbar part), Pa, PL
         {
-            float d[32];
-            tm_ld32w(tm, q, c0, d);  // dKbar / sG
+            float d[32], e2[32];
+            tm_ld32w(tm, q, c0, d);         // dKbar / sG
+            tm_ld32w(tm, q, 128 + c0, e2);  // dAbar / sG
             float* pk = p.Pk + cb;
-#pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                float o[4];
-#pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float Eb = ex2(s.Lb[c0 + j + u] - L[j + u]);
-                    o[u] = d[j + u] * sG * Eb;
-                    PL[j + u] -= o[u] * kv[j + u];  // dKbar . Kbar
-                }
-                *reinterpret_cast<float4*>(pk + j) = make_float4(o[0], o[1], o[2], o[3]);
-            }
-            tm_ld32w(tm, q, 128 + c0, d);  // dAbar / sG
             float* pa = p.Pa + cb;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                float o[4];
+            for (int i = 0; i < 4; ++i) {
+                float kv[8], ev[8], o1[8], o2[8], r[8];
+                ld8_bf16(kin + 8 * i, kv);
+                ld8_bf16(ein + 8 * i, ev);
+                const float4 r0 = *reinterpret_cast<const float4*>(pl + 8 * i);
+                const float4 r1 = *reinterpret_cast<const float4*>(pl + 8 * i + 4);
+                r[0] = r0.x; r[1] = r0.y; r[2] = r0.z; r[3] = r0.w; r[4] = r1.x; r[5] = r1.y; r[6] = r1.z; r[7] = r1.w;
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    const float Eb = ex2(s.Lb[c0 + j + u] - L[j + u]);
-                    o[u] = d[j + u] * sG * Eb;
-                    PL[j + u] -= o[u] * ev[j + u] * kv[j + u];  // dAbar . Abar
+                for (int u = 0; u < 8; ++u) {
+                    const int j = 8 * i + u;
+                    const float Eb = ex2(s.Lb[c0 + j] - L[j]) * sG;
+                    o1[u] = d[j] * Eb;
+                    o2[u] = e2[j] * Eb;
+                    r[u] -= (o1[u] + o2[u] * ev[u]) * kv[u];  // dKbar . Kbar + dAbar . Abar
                 }
-                *reinterpret_cast<float4*>(pa + j) = make_float4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<float4*>(pl + 8 * i) = make_float4(r[0], r[1], r[2], r[3]);
+                *reinterpret_cast<float4*>(pl + 8 * i + 4) = make_float4(r[4], r[5], r[6], r[7]);
+                *reinterpret_cast<float4*>(pk + 8 * i) = make_float4(o1[0], o1[1], o1[2], o1[3]);
+                *reinterpret_cast<float4*>(pk + 8 * i + 4) = make_float4(o1[4], o1[5], o1[6], o1[7]);
+                *reinterpret_cast<float4*>(pa + 8 * i) = make_float4(o2[0], o2[1], o2[2], o2[3]);
+                *reinterpret_cast<float4*>(pa + 8 * i + 4) = make_float4(o2[4], o2[5], o2[6], o2[7]);
             }
         }
         waitb(B1A, ph);
@@ -602,19 +602,21 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             float d[32];
             tm_ld32w(tm, q, c0, d);  // dK~ / sS
             float* pk = p.Pk + cb;
-            float* pl = p.PL + cb;
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
                 float4 x = *reinterpret_cast<float4*>(pk + j);
+                float4 y = *reinterpret_cast<float4*>(pl + j);
+                const uint2 kw = __ldg(reinterpret_cast<const uint2*>(kin + j));
+                float kv[4];
+                unpack16<true>(kw.x, kv[0], kv[1]);
+                unpack16<true>(kw.y, kv[2], kv[3]);
                 float o[4];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) {
-                    o[u] = d[j + u] * sS * ex2(L[j + u]);
-                    PL[j + u] += o[u] * kv[j + u];  // dK~ . K~
-                }
+                for (int u = 0; u < 4; ++u) o[u] = d[j + u] * sS * ex2(L[j + u]);
                 x.x += o[0]; x.y += o[1]; x.z += o[2]; x.w += o[3];
+                y.x += o[0] * kv[0]; y.y += o[1] * kv[1]; y.z += o[2] * kv[2]; y.w += o[3] * kv[3];  // dK~ . K~
                 *reinterpret_cast<float4*>(pk + j) = x;
-                *reinterpret_cast<float4*>(pl + j) = make_float4(PL[j], PL[j + 1], PL[j + 2], PL[j + 3]);
+                *reinterpret_cast<float4*>(pl + j) = y;
             }
         }
         waitb(B1L, ph);
@@ -671,11 +673,21 @@ struct Bwd2Smem {
     int bad;
 };
 enum { B2IN = 0, B2M };
+// which part of a dL product survives, in row/column terms of the lane's row r:
+// strictly / inclusively below the diagonal (col < r / col <= r) or above it
+enum { kStrictLow = 0, kInclLow, kStrictUp, kInclUp };
+__device__ __forceinline__ bool keep_col(int mode, int col, int r) {
+    return mode == kStrictLow ? col < r : mode == kInclLow ? col <= r : mode == kStrictUp ? col > r : col >= r;
+}
 }  // namespace
 
-// 256 threads; thread t = 32 (warp % 4) + lane owns row t; for channel half hj
-// it handles channels 64 hj + 32 (warp / 4) .. +32.
-__global__ void __launch_bounds__(256, 1) k2_bwd2(const __grid_constant__ Bwd2Params p) {
+// 512 threads; thread t = 32 (warp % 4) + lane owns row t; for channel half hj
+// it handles the 16 channels 64 hj + 16 (warp / 4) .. +16.  Per half, four
+// rounds each form two dL matrices (fp16 products into TMEM columns 0..255),
+// mask them in place (rounded to TF32) and use them as the A operands of TF32
+// products with a pivoted operand (K-major TF32 tile, 64 rows = the half's
+// channels) into one of four 64-column accumulators (TMEM 256..511).
+__global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Params p) {
     extern __shared__ __align__(1024) unsigned char smraw[];
     unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
     unsigned char* tdO = sm;
@@ -686,7 +698,7 @@ __global__ void __launch_bounds__(256, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
     unsigned char* Bt1 = Bt0 + kT32Half;
     Bwd2Smem& s = *reinterpret_cast<Bwd2Smem*>(Bt1 + kT32Half);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int q = warp & 3, h = warp >> 2, t = 32 * q + lane;
+    const int q = warp & 3, g4 = warp >> 2, t = 32 * q + lane;
     const int N = p.T / kC, nch = p.B * p.H * N;
     if (tid == 0) {
         for (int i = 0; i < 8; ++i) mbar_init(&s.bar[i], 1);
@@ -707,19 +719,16 @@ __global__ void __launch_bounds__(256, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
         pm ^= 1u;
         sync_all();
     };
-    // dL products into TMEM columns 0..127 (x) and 128..255 (y), then masked in
-    // place: keep(col) for this lane's row; values rounded to TF32.
-    auto mask_rows = [&](auto keep0, auto keep1) {
-#pragma unroll 1
-        for (int part = 0; part < 4; ++part) {
-            const int bank = part >> 1, col0 = 64 * h + 32 * (part & 1);
+    // mask the two dL products in place: this thread's 64 columns of bank g4 >> 1
+    auto mask_rows = [&](int mode0, int mode1) {
+        const int bank = g4 >> 1, mode = bank ? mode1 : mode0;
+#pragma unroll
+        for (int part = 0; part < 2; ++part) {
+            const int col0 = 64 * (g4 & 1) + 32 * part;
             float v[32];
             tm_ld32w(tm, q, 128 * bank + col0, v);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const bool k = bank == 0 ? keep0(col0 + j) : keep1(col0 + j);
-                v[j] = k ? tf32_round(v[j]) : 0.f;
-            }
+            for (int j = 0; j < 32; ++j) v[j] = keep_col(mode, col0 + j, t) ? tf32_round(v[j]) : 0.f;
 #pragma unroll
             for (int hh = 0; hh < 2; ++hh) {
                 float w[16];
@@ -730,7 +739,7 @@ __global__ void __launch_bounds__(256, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
         }
         tmem_wait_st();
     };
-    // ACC[128 x 64] (+)= A0 (TMEM cols 0..127) Bt0 + A1 (TMEM cols 128..255) Bt1, TF32
+    // ACC[128 x 64] = A0 (TMEM cols 0..127) Bt0 + A1 (TMEM cols 128..255) Bt1, TF32
     auto acc_pair = [&](int acc_col) {
         const uint32_t id = idesc(kTF32, 128, 64, false, false);
         for (int k = 0; k < 128; k += 8)
@@ -738,12 +747,27 @@ __global__ void __launch_bounds__(256, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
         for (int k = 0; k < 128; k += 8)
             mma_tf32_ta(tm + acc_col, tm + 128 + k, kdesc32<64>(aB1, 0, k), id, 1u);
     };
-    // pivoted operand (row t, this thread's 32 channels) -> column t of a
-    // transposed K-major TF32 tile (row = channel inside the half)
+    // 16 values of row t -> column t of a transposed K-major TF32 tile, rows r0 ..
     auto put_t = [&](unsigned char* tile, int r0, const float* v) {
 #pragma unroll
-        for (int u = 0; u < 32; ++u)
+        for (int u = 0; u < 16; ++u)
             *reinterpret_cast<float*>(tile + t32_off<64>(r0 + u, t >> 2) + (t & 3) * 4) = tf32_round(v[u]);
+    };
+    auto round_ = [&](uint32_t ax0, uint32_t bx0, bool negx, uint32_t ax1, uint32_t bx1, bool negy,
+                      int mode0, int mode1, int acc_col) {
+        if (tid == 0) {
+            gemm_kk16(tm + 0, ax0, 0, bx0, 0, 0, 128, 128, kF16, false, negx);
+            gemm_kk16(tm + 128, ax1, 0, bx1, 0, 0, 128, 128, kF16, false, negy);
+            mma_commit(&s.bar[B2M]);
+        }
+        mma_wait();
+        mask_rows(mode0, mode1);
+        sync_all();
+        if (tid == 0) {
+            acc_pair(acc_col);
+            mma_commit(&s.bar[B2M]);
+        }
+        mma_wait();
     };
 
     int it = 0;
@@ -762,36 +786,33 @@ __global__ void __launch_bounds__(256, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
         }
         if (!mbar_wait(&s.bar[B2IN], ph)) atomicOr(&s.bad, 1 << 25);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) {  // dO bf16 -> fp16 in place (row t, columns 64h ..)
+        for (int i = 0; i < 4; ++i) {  // dO bf16 -> fp16 in place (row t, columns 32 g4 ..)
             float v[8];
-            ld_chunk16<true>(tdO, t, 8 * h + i, v);
-            st_chunk16<false>(tdO, t, 8 * h + i, v);
+            ld_chunk16<true>(tdO, t, 4 * g4 + i, v);
+            st_chunk16<false>(tdO, t, 4 * g4 + i, v);
         }
         fence_async_smem();
         sync_all();
 
 #pragma unroll 1
         for (int hj = 0; hj < 2; ++hj) {
-            const int j0 = 64 * hj + 32 * h;  // this thread's channels
-            const int r0 = 32 * h;            // their rows in the half tiles
-            float L[32];
-            log_decay(reinterpret_cast<const __nv_bfloat16*>(p.g) + tok * kD, lane, q, j0, s.tot, L);
-            if (q == 0) s.P2[j0 + lane] = 0.5f * chunk_total(s.tot, j0 + lane);
+            const int j0 = 64 * hj + 16 * g4;  // this thread's channels
+            const int r0 = 16 * g4;            // their rows in the half tiles
+            float L[16];
+            log_decay<16>(reinterpret_cast<const __nv_bfloat16*>(p.g) + tok * kD, lane, q, j0, s.tot, L);
+            if (q == 0 && lane < 16) s.P2[j0 + lane] = 0.5f * chunk_total(s.tot, j0 + lane);
             __syncthreads();
-            float kv[32], ev[32];
-            {
-                const __nv_bfloat16* kp = reinterpret_cast<const __nv_bfloat16*>(p.k) + tok * kD + j0;
-                const __nv_bfloat16* ep = reinterpret_cast<const __nv_bfloat16*>(p.e) + tok * kD + j0;
+            const __nv_bfloat16* kin = reinterpret_cast<const __nv_bfloat16*>(p.k) + tok * kD + j0;
+            const __nv_bfloat16* ein = reinterpret_cast<const __nv_bfloat16*>(p.e) + tok * kD + j0;
+            const __nv_bfloat16* qin = reinterpret_cast<const __nv_bfloat16*>(p.q) + tok * kD + j0;
+            const __nv_bfloat16* gin_ = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + tok * kD + j0;
+            {  // Am -> Bt0, Km -> Bt1
+                float kv[16], ev[16], am[16], km[16];
+                ld8_bf16(kin, kv); ld8_bf16(kin + 8, kv + 8);
+                ld8_bf16(ein, ev); ld8_bf16(ein + 8, ev + 8);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) { ld8_bf16(kp + 8 * i, kv + 8 * i); ld8_bf16(ep + 8 * i, ev + 8 * i); }
-            }
-            // Am -> Bt0, Km -> Bt1
-            {
-                float am[32], km[32];
-#pragma unroll
-                for (int u = 0; u < 32; ++u) {
-                    const float em = ex2(s.P2[j0 + u] - L[u]);
-                    km[u] = kv[u] * em;
+                for (int u = 0; u < 16; ++u) {
+                    km[u] = kv[u] * ex2(s.P2[j0 + u] - L[u]);
                     am[u] = ev[u] * km[u];
                 }
                 put_t(Bt0, r0, am);
@@ -799,178 +820,115 @@ __global__ void __launch_bounds__(256, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             }
             fence_async_smem();
             sync_all();
-            // R1: dL_A = -dYR Y^T, dL_K = dYR U^T (strict) -> dKp
-            if (tid == 0) {
-                gemm_kk16(tm + 0, aR, 0, aY, 0, 0, 128, 128, kF16, false, true);
-                gemm_kk16(tm + 128, aR, 0, aU, 0, 0, 128, 128, kF16, false);
-                mma_commit(&s.bar[B2M]);
-            }
-            mma_wait();
-            mask_rows([&](int col) { return col < t; }, [&](int col) { return col < t; });
-            sync_all();
-            if (tid == 0) {
-                acc_pair(256);
-                mma_commit(&s.bar[B2M]);
-            }
-            mma_wait();
-            // R2: dM_QA = -dO Y^T (x), dM_QK = dO U^T (y) (inclusive) -> dQp = x Am + y Km
-            if (tid == 0) {
-                gemm_kk16(tm + 0, aO, 0, aY, 0, 0, 128, 128, kF16, false, true);
-                gemm_kk16(tm + 128, aO, 0, aU, 0, 0, 128, 128, kF16, false);
-                mma_commit(&s.bar[B2M]);
-            }
-            mma_wait();
-            mask_rows([&](int col) { return col <= t; }, [&](int col) { return col <= t; });
-            sync_all();
-            if (tid == 0) {
-                acc_pair(320);
-                mma_commit(&s.bar[B2M]);
-            }
-            mma_wait();
-            // Kp -> Bt0, Qp -> Bt1
-            {
-                float kp[32], qp[32], qv[8], gv[8];
-                const __nv_bfloat16* qsrc = reinterpret_cast<const __nv_bfloat16*>(p.q) + tok * kD + j0;
-                const __nv_bfloat16* gsrc = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + tok * kD + j0;
+            // R1: dL_A = -dYR Y^T, dL_K = dYR U^T (strict) -> dKp = dL_A Am + dL_K Km
+            round_(aR, aY, true, aR, aU, false, kStrictLow, kStrictLow, 256);
+            // R2: dM_QA = -dO Y^T, dM_QK = dO U^T (inclusive) -> dQp = dM_QA Am + dM_QK Km
+            round_(aO, aY, true, aO, aU, false, kInclLow, kInclLow, 320);
+            {  // Kp -> Bt0, Qp -> Bt1
+                float kv[16], qv[16], gv[16], kp[16], qp[16];
+                ld8_bf16(kin, kv); ld8_bf16(kin + 8, kv + 8);
+                ld8_bf16(qin, qv); ld8_bf16(qin + 8, qv + 8);
+                ld8_bf16(gin_, gv); ld8_bf16(gin_ + 8, gv + 8);
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    ld8_bf16(qsrc + 8 * i, qv);
-                    ld8_bf16(gsrc + 8 * i, gv);
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int j = 8 * i + u;
-                        const float ep = ex2(L[j] - s.P2[j0 + j]);
-                        kp[j] = kv[j] * ep;
-                        qp[j] = qv[u] * gv[u] * ep;
-                    }
+                for (int u = 0; u < 16; ++u) {
+                    const float ep = ex2(L[u] - s.P2[j0 + u]);
+                    kp[u] = kv[u] * ep;
+                    qp[u] = qv[u] * gv[u] * ep;
                 }
                 put_t(Bt0, r0, kp);
                 put_t(Bt1, r0, qp);
             }
             fence_async_smem();
             sync_all();
-            // R3: dL_A^T = -Y dYR^T (x, strict upper), dM_QA^T = -Y dO^T (y, inclusive upper) -> dAm
-            if (tid == 0) {
-                gemm_kk16(tm + 0, aY, 0, aR, 0, 0, 128, 128, kF16, false, true);
-                gemm_kk16(tm + 128, aY, 0, aO, 0, 0, 128, 128, kF16, false, true);
-                mma_commit(&s.bar[B2M]);
-            }
-            mma_wait();
-            mask_rows([&](int col) { return col > t; }, [&](int col) { return col >= t; });
-            sync_all();
-            if (tid == 0) {
-                acc_pair(384);
-                mma_commit(&s.bar[B2M]);
-            }
-            mma_wait();
-            // R4: dL_K^T = U dYR^T (x, strict upper), dM_QK^T = U dO^T (y, inclusive upper) -> dKm
-            if (tid == 0) {
-                gemm_kk16(tm + 0, aU, 0, aR, 0, 0, 128, 128, kF16, false);
-                gemm_kk16(tm + 128, aU, 0, aO, 0, 0, 128, 128, kF16, false);
-                mma_commit(&s.bar[B2M]);
-            }
-            mma_wait();
-            mask_rows([&](int col) { return col > t; }, [&](int col) { return col >= t; });
-            sync_all();
-            if (tid == 0) {
-                acc_pair(448);
-                mma_commit(&s.bar[B2M]);
-            }
-            mma_wait();
-            // ---- readout: final gradients of channels j0 .. j0 + 31 of row t
+            // R3: dL_A^T = -Y dYR^T (strict upper), dM_QA^T = -Y dO^T (inclusive upper) -> dAm
+            round_(aY, aR, true, aY, aO, true, kStrictUp, kInclUp, 384);
+            // R4: dL_K^T = U dYR^T (strict upper), dM_QK^T = U dO^T (inclusive upper) -> dKm
+            round_(aU, aR, false, aU, aO, false, kStrictUp, kInclUp, 448);
+            // ---- readout: final gradients of channels j0 .. j0 + 15 of row t
             {
                 const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + j0;
                 const size_t ro = tok * kD + j0;
-                float dL[32];
-                float akp[32], aq[32];
-                tm_ld32w(tm, q, 256 + 32 * h, akp);
-                tm_ld32w(tm, q, 320 + 32 * h, aq);
-                const __nv_bfloat16* qsrc = reinterpret_cast<const __nv_bfloat16*>(p.q) + ro;
-                const __nv_bfloat16* gsrc = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + ro;
-                __nv_bfloat16* dq = reinterpret_cast<__nv_bfloat16*>(p.dq) + ro;
-                __nv_bfloat16* dgm = reinterpret_cast<__nv_bfloat16*>(p.dgamma) + ro;
+                float dL[16];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float qv[8], gv[8], o1[8], o2[8];
-                    ld8_bf16(qsrc + 8 * i, qv);
-                    ld8_bf16(gsrc + 8 * i, gv);
-                    const float4 pq0 = __ldg(reinterpret_cast<const float4*>(p.Pq + cb + 8 * i));
-                    const float4 pq1 = __ldg(reinterpret_cast<const float4*>(p.Pq + cb + 8 * i + 4));
-                    const float pq[8] = {pq0.x, pq0.y, pq0.z, pq0.w, pq1.x, pq1.y, pq1.z, pq1.w};
+                for (int hh = 0; hh < 2; ++hh) {  // 8 channels at a time
+                    const int u0 = 8 * hh;
+                    float a_kp[8], a_q[8], a_a[8], a_km[8];
+                    tmem_ld8(taddr(tm, 32 * q, 256 + 16 * g4 + u0), a_kp);
+                    tmem_ld8(taddr(tm, 32 * q, 320 + 16 * g4 + u0), a_q);
+                    tmem_ld8(taddr(tm, 32 * q, 384 + 16 * g4 + u0), a_a);
+                    tmem_ld8(taddr(tm, 32 * q, 448 + 16 * g4 + u0), a_km);
+                    tmem_wait_ld();
+                    float kv[8], ev[8], qv[8], gv[8];
+                    ld8_bf16(kin + u0, kv);
+                    ld8_bf16(ein + u0, ev);
+                    ld8_bf16(qin + u0, qv);
+                    ld8_bf16(gin_ + u0, gv);
+                    float pq[8], pk[8], pa[8], pl[8];
+#pragma unroll
+                    for (int u = 0; u < 8; u += 4) {
+                        const float4 x0 = __ldg(reinterpret_cast<const float4*>(p.Pq + cb + u0 + u));
+                        const float4 x1 = __ldg(reinterpret_cast<const float4*>(p.Pk + cb + u0 + u));
+                        const float4 x2 = __ldg(reinterpret_cast<const float4*>(p.Pa + cb + u0 + u));
+                        const float4 x3 = __ldg(reinterpret_cast<const float4*>(p.PL + cb + u0 + u));
+                        pq[u] = x0.x; pq[u + 1] = x0.y; pq[u + 2] = x0.z; pq[u + 3] = x0.w;
+                        pk[u] = x1.x; pk[u + 1] = x1.y; pk[u + 2] = x1.z; pk[u + 3] = x1.w;
+                        pa[u] = x2.x; pa[u + 1] = x2.y; pa[u + 2] = x2.z; pa[u + 3] = x2.w;
+                        pl[u] = x3.x; pl[u + 1] = x3.y; pl[u + 2] = x3.z; pl[u + 3] = x3.w;
+                    }
+                    float oq[8], og[8], ok[8], oe[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        const int j = 8 * i + u;
+                        const int j = u0 + u;
                         const float ep = ex2(L[j] - s.P2[j0 + j]);
-                        const float dqh = aq[j] * ep + pq[u];
-                        o1[u] = dqh * gv[u];
-                        o2[u] = dqh * qv[u];
-                        // dKp Kp + dQp Qp
-                        dL[j] = akp[j] * kv[j] * ep + aq[j] * qv[u] * gv[u] * ep;
-                        akp[j] *= ep;  // dKp 2^(L-P)
-                    }
-                    st8_bf16(dq + 8 * i, o1);
-                    st8_bf16(dgm + 8 * i, o2);
-                }
-                float aa[32], akm[32];
-                tm_ld32w(tm, q, 384 + 32 * h, aa);
-                tm_ld32w(tm, q, 448 + 32 * h, akm);
-                __nv_bfloat16* dk = reinterpret_cast<__nv_bfloat16*>(p.dk) + ro;
-                __nv_bfloat16* de = reinterpret_cast<__nv_bfloat16*>(p.de) + ro;
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    float o1[8], o2[8];
-                    const float4 pa0 = __ldg(reinterpret_cast<const float4*>(p.Pa + cb + 8 * i));
-                    const float4 pa1 = __ldg(reinterpret_cast<const float4*>(p.Pa + cb + 8 * i + 4));
-                    const float4 pk0 = __ldg(reinterpret_cast<const float4*>(p.Pk + cb + 8 * i));
-                    const float4 pk1 = __ldg(reinterpret_cast<const float4*>(p.Pk + cb + 8 * i + 4));
-                    const float4 pl0 = __ldg(reinterpret_cast<const float4*>(p.PL + cb + 8 * i));
-                    const float4 pl1 = __ldg(reinterpret_cast<const float4*>(p.PL + cb + 8 * i + 4));
-                    const float pa[8] = {pa0.x, pa0.y, pa0.z, pa0.w, pa1.x, pa1.y, pa1.z, pa1.w};
-                    const float pk[8] = {pk0.x, pk0.y, pk0.z, pk0.w, pk1.x, pk1.y, pk1.z, pk1.w};
-                    const float pl[8] = {pl0.x, pl0.y, pl0.z, pl0.w, pl1.x, pl1.y, pl1.z, pl1.w};
-#pragma unroll
-                    for (int u = 0; u < 8; ++u) {
-                        const int j = 8 * i + u;
                         const float em = ex2(s.P2[j0 + j] - L[j]);
-                        const float da = aa[j] * em + pa[u];
-                        o2[u] = da * kv[j];
-                        o1[u] = akp[j] + akm[j] * em + pk[u] + ev[j] * da;
-                        // - dKm Km - dAm Am + state-side part
-                        dL[j] += -akm[j] * kv[j] * em - aa[j] * ev[j] * kv[j] * em + pl[u];
+                        const float qh = qv[u] * gv[u];
+                        const float dqh = a_q[u] * ep + pq[u];
+                        oq[u] = dqh * gv[u];
+                        og[u] = dqh * qv[u];
+                        const float da = a_a[u] * em + pa[u];
+                        oe[u] = da * kv[u];
+                        ok[u] = a_kp[u] * ep + a_km[u] * em + pk[u] + ev[u] * da;
+                        // dKp Kp + dQp Qp - dKm Km - dAm Am + state-side part
+                        dL[j] = (a_kp[u] * kv[u] + a_q[u] * qh) * ep -
+                                (a_km[u] * kv[u] + a_a[u] * ev[u] * kv[u]) * em + pl[u];
                     }
-                    st8_bf16(dk + 8 * i, o1);
-                    st8_bf16(de + 8 * i, o2);
+                    st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dq) + ro + u0, oq);
+                    st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dgamma) + ro + u0, og);
+                    st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dk) + ro + u0, ok);
+                    st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.de) + ro + u0, oe);
                 }
                 // dg_t = sum_{t' >= t} dL_t' + dLbar: warp suffix scan, then later quarters
 #pragma unroll
                 for (int off = 1; off < 32; off <<= 1) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
+                    for (int j = 0; j < 16; ++j) {
                         const float o = __shfl_down_sync(0xffffffffu, dL[j], off);
                         if (lane + off < 32) dL[j] += o;
                     }
                 }
                 if (lane == 0) {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) s.sfx[q][j0 + j] = dL[j];
+                    for (int j = 0; j < 16; ++j) s.sfx[q][j0 + j] = dL[j];
                 }
                 __syncthreads();
-                const float* gin = reinterpret_cast<const float*>(p.dgb) + (size_t)c * kD + j0;
-                __nv_bfloat16* dg = reinterpret_cast<__nv_bfloat16*>(p.dg) + ro;
+                // dLbar of this chunk: the value slabs' partial sums in a fixed order
+                const float* gbar = p.dgb + (size_t)c * kD + j0;
+                const size_t gstride = (size_t)nch * kD;
                 const __nv_bfloat16* graw = reinterpret_cast<const __nv_bfloat16*>(p.g) + ro;
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
+                for (int hh = 0; hh < 2; ++hh) {
                     float o[8], gv[8];
-                    ld8_bf16(graw + 8 * i, gv);
+                    ld8_bf16(graw + 8 * hh, gv);
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        const int j = 8 * i + u;
-                        float post = gin[j];
+                        const int j = 8 * hh + u;
+                        float post = 0.f;
+                        for (int sl = 0; sl < p.nslab; ++sl) post += gbar[sl * gstride + j];
                         for (int qq = q + 1; qq < 4; ++qq) post += s.sfx[qq][j0 + j];
                         // the clamp g >= -20 passes no gradient below it
                         o[u] = gv[u] >= kLogDecayMin ? dL[j] + post : 0.f;
                     }
-                    st8_bf16(dg + 8 * i, o);
+                    st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dg) + ro + 8 * hh, o);
                 }
             }
             sync_all();
@@ -1006,8 +964,8 @@ constexpr int rev_smem() { return 3 * 128 * 128 * 4 + SLAB * 512 + 1024; }
 
 size_t bwd2_ws_bytes(int B, int T, int H) {
     const size_t nch = (size_t)B * H * (T / kC), blk = (size_t)kC * kD * 4;
-    // Bp, dSc, Pq, Pk, Pa, PL (fp32 blocks), Y16, dYR16 (fp16 tiles), dLbar
-    return nch * (6 * blk + 2 * (size_t)kT16Bytes + kD * 4) + 256;
+    // Bp, dSc, Pq, Pk, Pa, PL (fp32 blocks), Y16, dYR16 (fp16 tiles), dLbar per value slab
+    return nch * (6 * blk + 2 * (size_t)kT16Bytes + 4 * kD * 4) + 256;
 }
 
 cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
@@ -1020,7 +978,8 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     float* Pk = f; f += nch * blk;
     float* Pa = f; f += nch * blk;
     float* PL = f; f += nch * blk;
-    float* dgb = f; f += (size_t)nch * kD;
+    constexpr int SLAB = 32;
+    float* dgb = f; f += (size_t)(kD / SLAB) * nch * kD;
     unsigned char* Y16 = reinterpret_cast<unsigned char*>(f);
     unsigned char* dYR16 = Y16 + (size_t)nch * kT16Bytes;
     const int nsm = sm_count();
@@ -1035,12 +994,10 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     MUIR_TIMED("k2_bprep", st, k2_bprep<<<nch, 256, kBprepSmem, st>>>(bp));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    constexpr int SLAB = 32;
     RevParams rp;
     if (!map_rows32f(&rp.tMt, a.Mt, (long long)nch * kD)) return cudaErrorInvalidValue;
     rp.Bp = Bp; rp.S_chunks = a.S_chunks; rp.S_last = a.S_last; rp.dS_final = a.dS_final;
-    rp.dSc = dSc; rp.dS0 = a.dS0; rp.dgb = dgb; rp.N = N;
-    if ((e = cudaMemsetAsync(dgb, 0, (size_t)nch * kD * sizeof(float), st)) != cudaSuccess) return e;
+    rp.dSc = dSc; rp.dS0 = a.dS0; rp.dgb = dgb; rp.N = N; rp.nch = nch;
     if ((e = cudaFuncSetAttribute(k2_chain_rev<SLAB>, cudaFuncAttributeMaxDynamicSharedMemorySize, rev_smem<SLAB>())) != cudaSuccess) return e;
     MUIR_TIMED("k2_chain_rev", st, k2_chain_rev<SLAB><<<BH * (kD / SLAB), 128, rev_smem<SLAB>(), st>>>(rp));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1060,10 +1017,10 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     p2.tdO = tdO; p2.B = a.B; p2.T = a.T; p2.H = a.H;
     p2.q = a.q; p2.k = a.k; p2.g = a.g; p2.e = a.e; p2.gamma = a.gamma;
     p2.aux = a.aux; p2.Y16 = Y16; p2.dYR16 = dYR16; p2.Pq = Pq; p2.Pk = Pk; p2.Pa = Pa; p2.PL = PL;
-    p2.dgb = dgb;
+    p2.dgb = dgb; p2.nslab = kD / SLAB;
     p2.dq = a.dq; p2.dk = a.dk; p2.dg = a.dg; p2.de = a.de; p2.dgamma = a.dgamma;
     if ((e = cudaFuncSetAttribute(k2_bwd2, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwd2Smem)) != cudaSuccess) return e;
-    MUIR_TIMED("k2_bwd2", st, k2_bwd2<<<grid, 256, kBwd2Smem, st>>>(p2));
+    MUIR_TIMED("k2_bwd2", st, k2_bwd2<<<grid, 512, kBwd2Smem, st>>>(p2));
     return cudaGetLastError();
 }
 

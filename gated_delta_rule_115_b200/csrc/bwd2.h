@@ -24,8 +24,8 @@ struct RevParams {
     const float* dS_final;  // or null
     float* dSc;             // G_{n+1} per chunk
     float* dS0;             // or null
-    float* dgb;             // dLbar per chunk and channel (zeroed by the host)
-    int N;
+    float* dgb;             // dLbar partials [128 / SLAB][nch][128]
+    int N, nch;
 };
 
 struct Bwd1Params {
@@ -46,7 +46,8 @@ struct Bwd2Params {
     const void *q, *k, *g, *e, *gamma;
     const unsigned char* aux;
     const unsigned char *Y16, *dYR16;
-    const float *Pq, *Pk, *Pa, *PL, *dgb;
+    const float *Pq, *Pk, *Pa, *PL, *dgb;  // dgb: [nslab][nch][128] partials of dLbar
+    int nslab;
     void *dq, *dk, *dg, *de, *dgamma;
 };
 

@@ -305,25 +305,20 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             mma_commit(&s.bar[BM1]);
         }
 
-        // ---- 3. query operands: Qp hi -> S3, Qp lo -> S4; Q~ -> Qp_out (completed in step 7)
+        // ---- 3. query operands: Qp hi -> S3, Qp lo -> S4
         waitb(s, BB, ph);
 #pragma unroll 1
         for (int i = 0; i < 4; ++i, rot8(L)) {
-            float qv[8], gv[8], qh[8], ql[8], qt[8];
+            float qv[8], gv[8], qh[8], ql[8];
             ld_chunk16<true>(S[3], t, 4 * h + i, qv);
             ld_chunk16<true>(S[4], t, 4 * h + i, gv);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const float pv = s.P2[c0 + 8 * i + u];
-                const float qhat = qv[u] * gv[u];
-                bf16_split(qhat * ex2(L[u] - pv), qh[u], ql[u]);
-                qt[u] = qhat * ex2(L[u]);
+                bf16_split(qv[u] * gv[u] * ex2(L[u] - pv), qh[u], ql[u]);
             }
             st_chunk16<true>(S[3], t, 4 * h + i, qh);
             st_chunk16<true>(S[4], t, 4 * h + i, ql);
-            float* dst = p.Qp + rbase + 8 * i;
-            *reinterpret_cast<float4*>(dst) = make_float4(qt[0], qt[1], qt[2], qt[3]);
-            *reinterpret_cast<float4*>(dst + 4) = make_float4(qt[4], qt[5], qt[6], qt[7]);
         }
         fence_async_smem();
         sync_all();
@@ -518,14 +513,29 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             load_tile(S[3], &p.te, y, z, BF);
         }
         {
+            // Q' = Q~ - M_QA W with Q~ = gamma q 2^L from the bf16 inputs
             float v[32];
             tm_ld32w(tm + 256, q, c0, v);
             float* qd = p.Qp + rbase;
+            const size_t ri = (((size_t)(c / N / p.H) * p.T + (size_t)(c % N) * kC + t) * p.H + y) * kD + c0;
+            const __nv_bfloat16* qsrc = reinterpret_cast<const __nv_bfloat16*>(p.q) + ri;
+            const __nv_bfloat16* gsrc = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + ri;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                float4 a = *reinterpret_cast<const float4*>(qd + j);
-                a.x += v[j]; a.y += v[j + 1]; a.z += v[j + 2]; a.w += v[j + 3];
-                *reinterpret_cast<float4*>(qd + j) = a;
+            for (int j = 0; j < 32; j += 8) {
+                const uint4 qw = __ldg(reinterpret_cast<const uint4*>(qsrc + j));
+                const uint4 gw = __ldg(reinterpret_cast<const uint4*>(gsrc + j));
+                const uint32_t qa[4] = {qw.x, qw.y, qw.z, qw.w}, ga[4] = {gw.x, gw.y, gw.z, gw.w};
+                float r[8];
+#pragma unroll
+                for (int u = 0; u < 4; ++u) {
+                    float q0, q1, g0, g1;
+                    unpack16<true>(qa[u], q0, q1);
+                    unpack16<true>(ga[u], g0, g1);
+                    r[2 * u] = v[j + 2 * u] + q0 * g0 * ex2(L[j + 2 * u]);
+                    r[2 * u + 1] = v[j + 2 * u + 1] + q1 * g1 * ex2(L[j + 2 * u + 1]);
+                }
+                *reinterpret_cast<float4*>(qd + j) = make_float4(r[0], r[1], r[2], r[3]);
+                *reinterpret_cast<float4*>(qd + j + 4) = make_float4(r[4], r[5], r[6], r[7]);
             }
             tm_ld32w(tm + 384, q, c0, v);
             float* od = p.Oi + rbase;
@@ -886,6 +896,7 @@ cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st) {
         !map_tokens16(&ip.tgam, a.gamma, a.B, a.T, a.H))
         return cudaErrorInvalidValue;
     ip.B = a.B; ip.T = a.T; ip.H = a.H;
+    ip.q = a.q; ip.gamma = a.gamma;
     ip.M = a.M; ip.Mt = a.Mt; ip.Bn = a.Bn; ip.Qp = a.Qp; ip.Oi = a.Oi; ip.flags = a.flags;
     ip.aux = a.aux;
     cudaError_t e = cudaFuncSetAttribute(k2_intra, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);

@@ -309,13 +309,19 @@ def test_ragged_tail_reuses_saved(muir):
     for k in a:
         assert torch.equal(a[k], b[k]), k
     # the same sequences padded by hand to 384 tokens with zero tokens give the
-    # same o on the real rows and the same final state
+    # same o on the real rows and the same final state.  The padded call
+    # (T a multiple of 128) runs the on-chip tensor-core path, the ragged one
+    # the boundary-pivot path, so they agree within the forward tolerance
+    # rather than bit for bit (o is bf16: one rounding step on each side).
     pad = {n: (torch.cat([x[n], torch.zeros_like(x[n][:, :51])], 1) if x[n].dim() == 4 and n != "S0"
                else x[n]) for n in NAMES + ["S0"]}
-    op, Sp = muir.chunk_fwd(*[pad[n] for n in NAMES], pad["S0"], chunk=128)
+    op, Sp = muir.chunk_fwd(*[pad[n] for n in NAMES], pad["S0"], chunk=128, out_dtype=torch.float32)
+    o32, S32 = muir.chunk_fwd(*[x[n] for n in NAMES], x["S0"], chunk=128, out_dtype=torch.float32)
     torch.cuda.synchronize()
-    assert torch.equal(op[:, :333], o)
-    assert torch.equal(Sp, S)
+    ref_o = o32.double().cpu().numpy()
+    assert nmax(op[:, :333], ref_o) < 2 * TOL_FWD["bf16"]
+    assert nmax(Sp, S32.double().cpu().numpy()) < 2 * TOL_FWD["bf16"]
+    assert torch.equal(S32, S)
 
 
 # ------------------------------------------------------------ full-size workloads
