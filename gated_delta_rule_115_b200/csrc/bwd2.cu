@@ -20,6 +20,8 @@
 //     dq^ = dQp 2^(L-P) + dQ~ 2^L,  da = dAm 2^(P-L) + dAbar 2^(Lbar-L)
 //     dk  = dKp 2^(L-P) + dKm 2^(P-L) + dK~ 2^L + dKbar 2^(Lbar-L) + e da
 //     dLog = dKp Kp + dQp Qp - dKm Km - dAm Am + dK~ K~ + dQ~ Q~ - dKbar Kbar - dAbar Abar
+//          (the last four = Pd k + Pq q^ - Pa a with Pq = dQ~ 2^L, Pa = dAbar 2^(Lbar-L),
+//           Pd = dK~ 2^L - dKbar 2^(Lbar-L))
 //     dg_t = sum_{t' >= t} dLog_t' + dLbar,   dLbar_j = sum_c G[j][c] S_{n+1}[j][c]
 //
 // Kernels: k2_bprep (Q'^T dO), k2_chain_rev (reverse pass, dLbar), k2_bwd1
@@ -181,7 +183,7 @@ __global__ void __launch_bounds__(256) k2_bprep(const __grid_constant__ BprepPar
             st_chunk16<false>(Qt, t, 8 * h + i, v);
         }
     }
-    if (!mbar_wait(&bar[0], 0)) atomicOr(&bad, 1);
+    if (!cta_wait(&bar[0], 0) && tid == 0) atomicOr(&bad, 1);
 #pragma unroll
     for (int i = 0; i < 8; ++i) {  // dO bf16 -> fp16 in place (own chunks)
         float v[8];
@@ -194,8 +196,7 @@ __global__ void __launch_bounds__(256) k2_bprep(const __grid_constant__ BprepPar
         gemm_mm16(tm, saddr(Qt), 0, 0, saddr(Dt), 0, 0, 128, 128, kF16, false);
         mma_commit(&bar[1]);
     }
-    if (!mbar_wait(&bar[1], 0)) atomicOr(&bad, 2);
-    tc_fence_after();
+    if (!cta_wait(&bar[1], 0) && tid == 0) atomicOr(&bad, 2);
     {
         float* dst = p.Bp + (size_t)c * kD * kD + (size_t)t * kD + 64 * h;
 #pragma unroll
@@ -298,8 +299,7 @@ __global__ void __launch_bounds__(128, 1) k2_chain_rev(const __grid_constant__ R
                 Bc[c] = v.x; Bc[c + 1] = v.y; Bc[c + 2] = v.z; Bc[c + 3] = v.w;
             }
         }
-        if (!mbar_wait(&bar[STAGES], (uint32_t)(s & 1))) atomicOr(&bad, 8);
-        tc_fence_after();
+        if (!cta_wait(&bar[STAGES], (uint32_t)(s & 1)) && tid == 0) atomicOr(&bad, 8);
         if (tid == 0 && s + STAGES < N) issue(s + STAGES);
         float d[32];
         tmem_ld32(taddr(tm, 32 * warp, 0), d);
@@ -381,8 +381,8 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
     uint32_t a[6];
 #pragma unroll
     for (int i = 0; i < 6; ++i) a[i] = saddr(S[i]);
-    auto waitb = [&](int i, uint32_t ph) {
-        if (!mbar_wait(&s.bar[i], ph)) atomicOr(&s.bad, 1 << (8 + i));
+    auto waitb = [&](int i, uint32_t ph) {  // all threads: warp 0 polls, the rest sleep
+        if (!cta_wait(&s.bar[i], ph) && tid == 0) atomicOr(&s.bad, 1 << (8 + i));
     };
     auto bulk = [&](unsigned char* dst, const unsigned char* src, int bar) {
         mbar_arrive_expect_tx(&s.bar[bar], kT16Bytes);
@@ -456,33 +456,20 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             gemm_km16(tm + 128, a[2], 0, a[0], 0, 0, 128, 128, kF16, false);
             mma_commit(&s.bar[B1M1]);
         }
-        const __nv_bfloat16* kin = reinterpret_cast<const __nv_bfloat16*>(p.k) + ro;
-        const __nv_bfloat16* ein = reinterpret_cast<const __nv_bfloat16*>(p.e) + ro;
         waitb(B1M1, ph);
         tc_fence_after();
-        // ---- phase 2: Pq, PL (dQ~ part); Y = W S + U' -> fp16 tile S2 (also saved for k2_bwd2)
-        float* pl = p.PL + cb;  // the state-side part of dLog, accumulated over phases 2, 3, 6
+        // ---- phase 2: Pq; Y = W S + U' -> fp16 tile S2 (also saved for k2_bwd2)
         {
-            float d[32], qv[8], gv[8];
+            float d[32];
             tm_ld32w(tm, q, c0, d);
-            const __nv_bfloat16* qp = reinterpret_cast<const __nv_bfloat16*>(p.q) + ro;
-            const __nv_bfloat16* gp = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + ro;
             float* pq = p.Pq + cb;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                ld8_bf16(qp + 8 * i, qv);
-                ld8_bf16(gp + 8 * i, gv);
-                float o[8], r[8];
+                float o[8];
 #pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int j = 8 * i + u;
-                    o[u] = d[j] * sS * ex2(L[j]);
-                    r[u] = o[u] * qv[u] * gv[u];  // dQ~ . Q~
-                }
+                for (int u = 0; u < 8; ++u) o[u] = d[8 * i + u] * sS * ex2(L[8 * i + u]);
                 *reinterpret_cast<float4*>(pq + 8 * i) = make_float4(o[0], o[1], o[2], o[3]);
                 *reinterpret_cast<float4*>(pq + 8 * i + 4) = make_float4(o[4], o[5], o[6], o[7]);
-                *reinterpret_cast<float4*>(pl + 8 * i) = make_float4(r[0], r[1], r[2], r[3]);
-                *reinterpret_cast<float4*>(pl + 8 * i + 4) = make_float4(r[4], r[5], r[6], r[7]);
             }
             tm_ld32w(tm, q, 128 + c0, d);
             const float* up = reinterpret_cast<const float*>(ax + AuxLayout::kUp) + (size_t)t * kD + c0;
@@ -498,61 +485,43 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
         sync_all();
         waitb(B1U, ph);
         waitb(B1Q, ph);
-        tc_fence_after();
         if (tid == 0) {
             bulk_store(y16, S[2], kT16Bytes);
             bulk_commit();
-            gemm_kk16(tm + 0, a[4], 0, a[3], 0, 0, 128, 128, kF16, false);         // dKbar / sG = U G^T
+            gemm_kk16(tm + 384, a[4], 0, a[3], 0, 0, 128, 128, kF16, false);         // dKbar / sG = U G^T (kept)
             gemm_kk16(tm + 128, a[2], 0, a[3], 0, 0, 128, 128, kF16, false, true);  // dAbar / sG = -Y G^T
             gemm_mm16(tm + 256, a[5], 0, 0, a[1], 0, 0, 128, 128, kF16, false, true); // -M_QA^T dO
             mma_commit(&s.bar[B1M2]);
         }
         waitb(B1M2, ph);
-        tc_fence_after();
         if (tid == 0) {  // Abar -> S4, T -> S5 (U, M_QA consumed)
             bulk(S[4], ax + AuxLayout::kAbar16, B1A);
             bulk(S[5], ax + AuxLayout::kT16, B1T);
         }
-        // ---- phase 3: Pk (dKbar part), Pa, PL
+        // ---- phase 3: Pa = dAbar 2^(Lbar - L)
         {
-            float d[32], e2[32];
-            tm_ld32w(tm, q, c0, d);         // dKbar / sG
-            tm_ld32w(tm, q, 128 + c0, e2);  // dAbar / sG
-            float* pk = p.Pk + cb;
+            float d[32];
+            tm_ld32w(tm, q, 128 + c0, d);  // dAbar / sG
             float* pa = p.Pa + cb;
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-                float kv[8], ev[8], o1[8], o2[8], r[8];
-                ld8_bf16(kin + 8 * i, kv);
-                ld8_bf16(ein + 8 * i, ev);
-                const float4 r0 = *reinterpret_cast<const float4*>(pl + 8 * i);
-                const float4 r1 = *reinterpret_cast<const float4*>(pl + 8 * i + 4);
-                r[0] = r0.x; r[1] = r0.y; r[2] = r0.z; r[3] = r0.w; r[4] = r1.x; r[5] = r1.y; r[6] = r1.z; r[7] = r1.w;
+                float o[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
                     const int j = 8 * i + u;
-                    const float Eb = ex2(s.Lb[c0 + j] - L[j]) * sG;
-                    o1[u] = d[j] * Eb;
-                    o2[u] = e2[j] * Eb;
-                    r[u] -= (o1[u] + o2[u] * ev[u]) * kv[u];  // dKbar . Kbar + dAbar . Abar
+                    o[u] = d[j] * sG * ex2(s.Lb[c0 + j] - L[j]);
                 }
-                *reinterpret_cast<float4*>(pl + 8 * i) = make_float4(r[0], r[1], r[2], r[3]);
-                *reinterpret_cast<float4*>(pl + 8 * i + 4) = make_float4(r[4], r[5], r[6], r[7]);
-                *reinterpret_cast<float4*>(pk + 8 * i) = make_float4(o1[0], o1[1], o1[2], o1[3]);
-                *reinterpret_cast<float4*>(pk + 8 * i + 4) = make_float4(o1[4], o1[5], o1[6], o1[7]);
-                *reinterpret_cast<float4*>(pa + 8 * i) = make_float4(o2[0], o2[1], o2[2], o2[3]);
-                *reinterpret_cast<float4*>(pa + 8 * i + 4) = make_float4(o2[4], o2[5], o2[6], o2[7]);
+                *reinterpret_cast<float4*>(pa + 8 * i) = make_float4(o[0], o[1], o[2], o[3]);
+                *reinterpret_cast<float4*>(pa + 8 * i + 4) = make_float4(o[4], o[5], o[6], o[7]);
             }
         }
-        waitb(B1A, ph);
-        sync_all();  // every warp has read B0 before it is overwritten
+        waitb(B1A, ph);  // (its block barrier also orders the reads of B1 above)
         // ---- phase 4: Abar G / sG (B0); dY = -M_QA^T dO - Abar G
         if (tid == 0) {
             gemm_km16(tm + 0, a[4], 0, a[3], 0, 0, 128, 128, kF16, false);
             mma_commit(&s.bar[B1M3]);
         }
         waitb(B1M3, ph);
-        tc_fence_after();
         if (tid == 0) {
             bulk_wait_read();  // Y left S2
             bulk(S[4], ax + AuxLayout::kMQK16, B1K);  // Abar consumed
@@ -569,71 +538,67 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
         fence_async_smem();
         sync_all();
         waitb(B1T, ph);
-        tc_fence_after();
-        // ---- phase 5: dYR = T^T dY (B3)
+        // ---- phase 5: dYR = T^T dY (B1)
         if (tid == 0) {
-            gemm_mm16(tm + 384, a[5], 0, 0, a[2], 0, 0, 128, 128, kF16, false);
+            gemm_mm16(tm + 128, a[5], 0, 0, a[2], 0, 0, 128, 128, kF16, false);
             mma_commit(&s.bar[B1M4]);
         }
         waitb(B1M4, ph);
-        tc_fence_after();
         if (tid == 0) bulk(S[2], ax + AuxLayout::kLK16, B1L);  // dY consumed
         {
             float d[32];
-            tm_ld32w(tm, q, 384 + c0, d);
+            tm_ld32w(tm, q, 128 + c0, d);
             row_st32<false>(S[5], t, h, d);  // dYR over T
         }
         fence_async_smem();
         sync_all();
         waitb(B1K, ph);
-        tc_fence_after();
-        // ---- phase 6: dK~ / sS = dYR S^T (B0); M_QK^T dO (B1)
+        // ---- phase 6: dK~ / sS = dYR S^T (B0); M_QK^T dO (B2); Pk, Pd from dK~ and dKbar (B3)
         if (tid == 0) {
             bulk_store(r16, S[5], kT16Bytes);
             bulk_commit();
             gemm_kk16(tm + 0, a[5], 0, a[0], 0, 0, 128, 128, kF16, false);
-            gemm_mm16(tm + 128, a[4], 0, 0, a[1], 0, 0, 128, 128, kF16, false);
+            gemm_mm16(tm + 256, a[4], 0, 0, a[1], 0, 0, 128, 128, kF16, false);
             mma_commit(&s.bar[B1M5]);
         }
         waitb(B1M5, ph);
-        tc_fence_after();
         if (tid == 0) bulk(S[0], ax + AuxLayout::kKbar16, B1KB);  // S consumed
         {
-            float d[32];
-            tm_ld32w(tm, q, c0, d);  // dK~ / sS
+            float d[32], e2[32];
+            tm_ld32w(tm, q, c0, d);         // dK~ / sS
+            tm_ld32w(tm, q, 384 + c0, e2);  // dKbar / sG
             float* pk = p.Pk + cb;
+            float* pd = p.Pd + cb;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4) {
-                float4 x = *reinterpret_cast<float4*>(pk + j);
-                float4 y = *reinterpret_cast<float4*>(pl + j);
-                const uint2 kw = __ldg(reinterpret_cast<const uint2*>(kin + j));
-                float kv[4];
-                unpack16<true>(kw.x, kv[0], kv[1]);
-                unpack16<true>(kw.y, kv[2], kv[3]);
-                float o[4];
+            for (int i = 0; i < 4; ++i) {
+                float o1[8], o2[8];
 #pragma unroll
-                for (int u = 0; u < 4; ++u) o[u] = d[j + u] * sS * ex2(L[j + u]);
-                x.x += o[0]; x.y += o[1]; x.z += o[2]; x.w += o[3];
-                y.x += o[0] * kv[0]; y.y += o[1] * kv[1]; y.z += o[2] * kv[2]; y.w += o[3] * kv[3];  // dK~ . K~
-                *reinterpret_cast<float4*>(pk + j) = x;
-                *reinterpret_cast<float4*>(pl + j) = y;
+                for (int u = 0; u < 8; ++u) {
+                    const int j = 8 * i + u;
+                    const float x1 = d[j] * sS * ex2(L[j]);                          // dK~ 2^L
+                    const float x2 = e2[j] * sG * ex2(s.Lb[c0 + j] - L[j]);         // dKbar 2^(Lbar-L)
+                    o1[u] = x1 + x2;
+                    o2[u] = x1 - x2;
+                }
+                *reinterpret_cast<float4*>(pk + 8 * i) = make_float4(o1[0], o1[1], o1[2], o1[3]);
+                *reinterpret_cast<float4*>(pk + 8 * i + 4) = make_float4(o1[4], o1[5], o1[6], o1[7]);
+                *reinterpret_cast<float4*>(pd + 8 * i) = make_float4(o2[0], o2[1], o2[2], o2[3]);
+                *reinterpret_cast<float4*>(pd + 8 * i + 4) = make_float4(o2[4], o2[5], o2[6], o2[7]);
             }
         }
         waitb(B1L, ph);
         waitb(B1KB, ph);
-        tc_fence_after();
-        // ---- phase 7: dU = M_QK^T dO + L_K^T dYR (B1) + Kbar G (B2, times sG)
+        // ---- phase 7: dU = M_QK^T dO + L_K^T dYR (B2) + Kbar G (B1, times sG)
         if (tid == 0) {
-            gemm_mm16(tm + 128, a[2], 0, 0, a[5], 0, 0, 128, 128, kF16, true);
-            gemm_km16(tm + 256, a[0], 0, a[3], 0, 0, 128, 128, kF16, false);
+            gemm_mm16(tm + 256, a[2], 0, 0, a[5], 0, 0, 128, 128, kF16, true);
+            gemm_km16(tm + 128, a[0], 0, a[3], 0, 0, 128, 128, kF16, false);
             mma_commit(&s.bar[B1M6]);
         }
         waitb(B1M6, ph);
-        tc_fence_after();
         {
             float d[32], e2[32], vv[8], wv[8];
-            tm_ld32w(tm, q, 128 + c0, d);
-            tm_ld32w(tm, q, 256 + c0, e2);
+            tm_ld32w(tm, q, 256 + c0, d);
+            tm_ld32w(tm, q, 128 + c0, e2);
             const __nv_bfloat16* vp = reinterpret_cast<const __nv_bfloat16*>(p.v) + ro;
             const __nv_bfloat16* wp = reinterpret_cast<const __nv_bfloat16*>(p.w) + ro;
             __nv_bfloat16* dvp = reinterpret_cast<__nv_bfloat16*>(p.dv) + ro;
@@ -715,9 +680,8 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
     // Every thread waits; the barrier that follows keeps the next commit on
     // B2M from completing before the slowest thread has seen this phase.
     auto mma_wait = [&]() {
-        if (!mbar_wait(&s.bar[B2M], pm)) atomicOr(&s.bad, 1 << 24);
+        if (!cta_wait(&s.bar[B2M], pm) && tid == 0) atomicOr(&s.bad, 1 << 24);
         pm ^= 1u;
-        sync_all();
     };
     // mask the two dL products in place: this thread's 64 columns of bank g4 >> 1
     auto mask_rows = [&](int mode0, int mode1) {
@@ -784,7 +748,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             bulk_load(tY, p.Y16 + (size_t)c * kT16Bytes, kT16Bytes, &s.bar[B2IN]);
             bulk_load(tR, p.dYR16 + (size_t)c * kT16Bytes, kT16Bytes, &s.bar[B2IN]);
         }
-        if (!mbar_wait(&s.bar[B2IN], ph)) atomicOr(&s.bad, 1 << 25);
+        if (!cta_wait(&s.bar[B2IN], ph) && tid == 0) atomicOr(&s.bad, 1 << 25);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {  // dO bf16 -> fp16 in place (row t, columns 32 g4 ..)
             float v[8];
@@ -869,7 +833,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                         const float4 x0 = __ldg(reinterpret_cast<const float4*>(p.Pq + cb + u0 + u));
                         const float4 x1 = __ldg(reinterpret_cast<const float4*>(p.Pk + cb + u0 + u));
                         const float4 x2 = __ldg(reinterpret_cast<const float4*>(p.Pa + cb + u0 + u));
-                        const float4 x3 = __ldg(reinterpret_cast<const float4*>(p.PL + cb + u0 + u));
+                        const float4 x3 = __ldg(reinterpret_cast<const float4*>(p.Pd + cb + u0 + u));
                         pq[u] = x0.x; pq[u + 1] = x0.y; pq[u + 2] = x0.z; pq[u + 3] = x0.w;
                         pk[u] = x1.x; pk[u + 1] = x1.y; pk[u + 2] = x1.z; pk[u + 3] = x1.w;
                         pa[u] = x2.x; pa[u + 1] = x2.y; pa[u + 2] = x2.z; pa[u + 3] = x2.w;
@@ -888,9 +852,11 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                         const float da = a_a[u] * em + pa[u];
                         oe[u] = da * kv[u];
                         ok[u] = a_kp[u] * ep + a_km[u] * em + pk[u] + ev[u] * da;
-                        // dKp Kp + dQp Qp - dKm Km - dAm Am + state-side part
+                        // dKp Kp + dQp Qp - dKm Km - dAm Am, plus the state-side part
+                        // dK~ K~ + dQ~ Q~ - dKbar Kbar - dAbar Abar = Pd k + Pq q^ - Pa a
                         dL[j] = (a_kp[u] * kv[u] + a_q[u] * qh) * ep -
-                                (a_km[u] * kv[u] + a_a[u] * ev[u] * kv[u]) * em + pl[u];
+                                (a_km[u] * kv[u] + a_a[u] * ev[u] * kv[u]) * em +
+                                pl[u] * kv[u] + pq[u] * qh - pa[u] * ev[u] * kv[u];
                     }
                     st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dq) + ro + u0, oq);
                     st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dgamma) + ro + u0, og);
@@ -977,7 +943,7 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     float* Pq = f; f += nch * blk;
     float* Pk = f; f += nch * blk;
     float* Pa = f; f += nch * blk;
-    float* PL = f; f += nch * blk;
+    float* Pd = f; f += nch * blk;
     constexpr int SLAB = 32;
     float* dgb = f; f += (size_t)(kD / SLAB) * nch * kD;
     unsigned char* Y16 = reinterpret_cast<unsigned char*>(f);
@@ -1007,7 +973,7 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     p1.tdO = tdO; p1.B = a.B; p1.T = a.T; p1.H = a.H;
     p1.q = a.q; p1.k = a.k; p1.v = a.v; p1.g = a.g; p1.e = a.e; p1.w = a.w; p1.gamma = a.gamma;
     p1.aux = a.aux; p1.S_chunks = a.S_chunks; p1.dSc = dSc;
-    p1.Pq = Pq; p1.Pk = Pk; p1.Pa = Pa; p1.PL = PL; p1.Y16 = Y16; p1.dYR16 = dYR16;
+    p1.Pq = Pq; p1.Pk = Pk; p1.Pa = Pa; p1.Pd = Pd; p1.Y16 = Y16; p1.dYR16 = dYR16;
     p1.dv = a.dv; p1.dw = a.dw;
     if ((e = cudaFuncSetAttribute(k2_bwd1, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwd1Smem)) != cudaSuccess) return e;
     MUIR_TIMED("k2_bwd1", st, k2_bwd1<<<grid, 512, kBwd1Smem, st>>>(p1));
@@ -1016,7 +982,7 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     Bwd2Params p2;
     p2.tdO = tdO; p2.B = a.B; p2.T = a.T; p2.H = a.H;
     p2.q = a.q; p2.k = a.k; p2.g = a.g; p2.e = a.e; p2.gamma = a.gamma;
-    p2.aux = a.aux; p2.Y16 = Y16; p2.dYR16 = dYR16; p2.Pq = Pq; p2.Pk = Pk; p2.Pa = Pa; p2.PL = PL;
+    p2.aux = a.aux; p2.Y16 = Y16; p2.dYR16 = dYR16; p2.Pq = Pq; p2.Pk = Pk; p2.Pa = Pa; p2.Pd = Pd;
     p2.dgb = dgb; p2.nslab = kD / SLAB;
     p2.dq = a.dq; p2.dk = a.dk; p2.dg = a.dg; p2.de = a.de; p2.dgamma = a.dgamma;
     if ((e = cudaFuncSetAttribute(k2_bwd2, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwd2Smem)) != cudaSuccess) return e;

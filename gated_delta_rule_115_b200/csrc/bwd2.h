@@ -35,7 +35,7 @@ struct Bwd1Params {
     const unsigned char* aux;
     const float* S_chunks;
     const float* dSc;
-    float *Pq, *Pk, *Pa, *PL;
+    float *Pq, *Pk, *Pa, *Pd;
     unsigned char *Y16, *dYR16;
     void *dv, *dw;
 };
@@ -46,7 +46,7 @@ struct Bwd2Params {
     const void *q, *k, *g, *e, *gamma;
     const unsigned char* aux;
     const unsigned char *Y16, *dYR16;
-    const float *Pq, *Pk, *Pa, *PL, *dgb;  // dgb: [nslab][nch][128] partials of dLbar
+    const float *Pq, *Pk, *Pa, *Pd, *dgb;  // dgb: [nslab][nch][128] partials of dLbar
     int nslab;
     void *dq, *dk, *dg, *de, *dgamma;
 };

@@ -106,9 +106,10 @@ struct IntraSmem {
 
 enum { BA = 0, BB, BC, BD, BE, BF, BM1, BM2, BM3, BM4, BM5, BM6, BG };
 
+// All threads call: warp 0 polls, the block barrier releases the rest.
 __device__ __forceinline__ bool waitb(IntraSmem& s, int i, uint32_t parity) {
-    const bool ok = mbar_wait(&s.bar[i], parity);
-    if (!ok) s.bad = 1;
+    const bool ok = cta_wait(&s.bar[i], parity);
+    if (!ok && threadIdx.x == 0) s.bad = 1;
     return ok;
 }
 
@@ -698,8 +699,7 @@ __global__ void __launch_bounds__(128, 1) k2_chain(const __grid_constant__ Chain
 #pragma unroll
         for (int c = 0; c < SLAB; ++c) Bc[c] = Bnext[c];
         if (n + 1 < N) load_B(n + 1, Bnext);
-        if (!mbar_wait(&bar[STAGES], (uint32_t)(n & 1))) bad = 1;
-        tc_fence_after();
+        if (!cta_wait(&bar[STAGES], (uint32_t)(n & 1)) && tid == 0) bad = 1;
         if (tid == 0 && n + STAGES < N) issue(n + STAGES);
         float d[32];
         tmem_ld32(taddr(tm, 32 * warp, 0), d);
@@ -781,8 +781,7 @@ __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutPara
             gemm_kk32<128, 128>(tm, saddr(Qt), saddr(St), 0, 128, 128, false);
             mma_commit(&bar[1]);
         }
-        if (!mbar_wait(&bar[1], (uint32_t)(it & 1))) bad = 1;
-        tc_fence_after();
+        if (!cta_wait(&bar[1], (uint32_t)(it & 1)) && tid == 0) bad = 1;
         const int cn = c + gridDim.x;
         if (tid == 0 && cn < nch) issue(cn);
         // epilogue: o[b][n*C + t][h][64 hh ..] = D + O_intra

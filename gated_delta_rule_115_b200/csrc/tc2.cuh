@@ -81,6 +81,17 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
     }
 }
 
+// Block-wide wait for a phase: warp 0 polls the barrier, every other warp
+// sleeps at the block barrier instead of spending issue slots on polling.
+// Returns false if the bounded wait expired.  All threads of the block call it.
+__device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity) {
+    int ok = 1;
+    if (threadIdx.x < 32) ok = mbar_wait(bar, parity) ? 1 : 0;
+    ok = __syncthreads_and(ok);
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    return ok != 0;
+}
+
 // ------------------------------------------------------------------ TMA
 
 // 3-D tiled load of one box into shared memory, completion counted in bytes
