@@ -633,23 +633,21 @@ struct Bwd2Smem {
     float tot[4][kD];
     float P2[kD];
     float sfx[4][kD];  // per-quarter totals of the reverse scan
+    float dgb[kD];     // dLbar of the chunk (value slabs summed in a fixed order)
     uint64_t bar[8];
     uint32_t tslot;
     int bad;
 };
 enum { B2IN = 0, B2M };
-// which part of a dL product survives, in row/column terms of the lane's row r:
-// strictly / inclusively below the diagonal (col < r / col <= r) or above it
+// which part of a dL product survives, for row r and column col:
+// col < r, col <= r, col > r, col >= r
 enum { kStrictLow = 0, kInclLow, kStrictUp, kInclUp };
-__device__ __forceinline__ bool keep_col(int mode, int col, int r) {
-    return mode == kStrictLow ? col < r : mode == kInclLow ? col <= r : mode == kStrictUp ? col > r : col >= r;
-}
 }  // namespace
 
 // 512 threads; thread t = 32 (warp % 4) + lane owns row t; for channel half hj
 // it handles the 16 channels 64 hj + 16 (warp / 4) .. +16.  Per half, four
 // rounds each form two dL matrices (fp16 products into TMEM columns 0..255),
-// mask them in place (rounded to TF32) and use them as the A operands of TF32
+// mask them in place and use them as the A operands of TF32
 // products with a pivoted operand (K-major TF32 tile, 64 rows = the half's
 // channels) into one of four 64-column accumulators (TMEM 256..511).
 __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Params p) {
@@ -683,22 +681,35 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
         if (!cta_wait(&s.bar[B2M], pm) && tid == 0) atomicOr(&s.bad, 1 << 24);
         pm ^= 1u;
     };
-    // mask the two dL products in place: this thread's 64 columns of bank g4 >> 1
+    // Mask the two dL products in place: this warp's two 32-column blocks of bank
+    // g4 >> 1.  A block wholly on the kept side of the diagonal is left as it is
+    // (the TF32 product truncates it), a block wholly on the other side is
+    // zeroed, and only the diagonal block (block index q) is read and masked.
     auto mask_rows = [&](int mode0, int mode1) {
-        const int bank = g4 >> 1, mode = bank ? mode1 : mode0;
+        const int mode = (g4 >> 1) ? mode1 : mode0;
+        const bool low = mode == kStrictLow || mode == kInclLow;
+        const bool incl = mode == kInclLow || mode == kInclUp;
 #pragma unroll
         for (int part = 0; part < 2; ++part) {
-            const int col0 = 64 * (g4 & 1) + 32 * part;
-            float v[32];
-            tm_ld32w(tm, q, 128 * bank + col0, v);
+            const int col0 = 64 * (g4 & 1) + 32 * part, cb = col0 >> 5;
+            const uint32_t at = taddr(tm, 32 * q, 128 * (g4 >> 1) + col0);
+            if (cb == q) {
+                float v[32];
+                tmem_ld32(at, v);
+                tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 32; ++j) v[j] = keep_col(mode, col0 + j, t) ? tf32_round(v[j]) : 0.f;
+                for (int j = 0; j < 32; ++j) {
+                    const bool keep = low ? (j < lane || (incl && j == lane)) : (j > lane || (incl && j == lane));
+                    if (!keep) v[j] = 0.f;
+                }
+                tmem_st16(at, *reinterpret_cast<const float(*)[16]>(v));
+                tmem_st16(at + 16, *reinterpret_cast<const float(*)[16]>(v + 16));
+            } else if (low ? cb > q : cb < q) {
+                float z[16];
 #pragma unroll
-            for (int hh = 0; hh < 2; ++hh) {
-                float w[16];
-#pragma unroll
-                for (int j = 0; j < 16; ++j) w[j] = v[16 * hh + j];
-                tmem_st16(taddr(tm, 32 * q, 128 * bank + col0 + 16 * hh), w);
+                for (int j = 0; j < 16; ++j) z[j] = 0.f;
+                tmem_st16(at, z);
+                tmem_st16(at + 16, z);
             }
         }
         tmem_wait_st();
@@ -747,6 +758,29 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             bulk_load(tU, p.aux + (size_t)c * AuxLayout::kBytes + AuxLayout::kU16, kT16Bytes, &s.bar[B2IN]);
             bulk_load(tY, p.Y16 + (size_t)c * kT16Bytes, kT16Bytes, &s.bar[B2IN]);
             bulk_load(tR, p.dYR16 + (size_t)c * kT16Bytes, kT16Bytes, &s.bar[B2IN]);
+        }
+        {  // this chunk's rows of the inputs the readout reads late -> L2
+            const char* rows[5] = {static_cast<const char*>(p.k), static_cast<const char*>(p.e),
+                                   static_cast<const char*>(p.q), static_cast<const char*>(p.gamma),
+                                   static_cast<const char*>(p.g)};
+            const size_t off = tok * kD * 2;
+#pragma unroll
+            for (int i = 0; i < 5; ++i) {
+                if (((i * 2) & 3) == g4) prefetch_l2(rows[i] + off);
+                if (((i * 2 + 1) & 3) == g4) prefetch_l2(rows[i] + off + 128);
+            }
+            if (tid == 32) {
+                const size_t cb = (size_t)c * kC * kD * sizeof(float);
+                bulk_prefetch_l2(reinterpret_cast<const char*>(p.Pq) + cb, kC * kD * 4);
+                bulk_prefetch_l2(reinterpret_cast<const char*>(p.Pk) + cb, kC * kD * 4);
+                bulk_prefetch_l2(reinterpret_cast<const char*>(p.Pa) + cb, kC * kD * 4);
+                bulk_prefetch_l2(reinterpret_cast<const char*>(p.Pd) + cb, kC * kD * 4);
+            }
+        }
+        if (tid < kD) {  // dLbar: the value slabs' partial sums in a fixed order
+            float acc = 0.f;
+            for (int sl = 0; sl < p.nslab; ++sl) acc += p.dgb[((size_t)sl * nch + c) * kD + tid];
+            s.dgb[tid] = acc;
         }
         if (!cta_wait(&s.bar[B2IN], ph) && tid == 0) atomicOr(&s.bad, 1 << 25);
 #pragma unroll
@@ -877,9 +911,6 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                     for (int j = 0; j < 16; ++j) s.sfx[q][j0 + j] = dL[j];
                 }
                 __syncthreads();
-                // dLbar of this chunk: the value slabs' partial sums in a fixed order
-                const float* gbar = p.dgb + (size_t)c * kD + j0;
-                const size_t gstride = (size_t)nch * kD;
                 const __nv_bfloat16* graw = reinterpret_cast<const __nv_bfloat16*>(p.g) + ro;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -888,8 +919,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const int j = 8 * hh + u;
-                        float post = 0.f;
-                        for (int sl = 0; sl < p.nslab; ++sl) post += gbar[sl * gstride + j];
+                        float post = s.dgb[j0 + j];
                         for (int qq = q + 1; qq < 4; ++qq) post += s.sfx[qq][j0 + j];
                         // the clamp g >= -20 passes no gradient below it
                         o[u] = gv[u] >= kLogDecayMin ? dL[j] + post : 0.f;
