@@ -15,14 +15,17 @@ Two independent C sources are wrapped:
   a triangular system), with exact exponent differences.
 
 and, in numpy below, the q/k feature prologue (SiLU, then unit L2 norm per
-token-head row; same page, "Methodology" and fig. 3(b)) with its gradient.
+token-head row; same page, "Methodology" and fig. 3(b)) with its gradient, the
+output gate o * sigmoid(z) with its gradient, and the fused layer composed of
+the three (``fwd_fused`` / ``bwd_fused``).
 
 Every function takes numpy-convertible arrays, computes in float64 and returns
 float64 numpy arrays.  Per-token tensors are ``[B, T, H, d]``; states are
 ``[B, H, dk, dv]``.
 
 Pins (what fixes these functions other than themselves) live in
-``tests/test_oracle_pins.py`` and ``tests/test_qk_oracle.py`` (the prologue):
+``tests/test_oracle_pins.py``, ``tests/test_qk_oracle.py`` (the prologue) and
+``tests/test_fused_oracle.py`` (output gate, fused composition):
 linear-attention and gated-linear-attention
 closed forms, the delta rule (Widrow-Hoff), an exact-retrieval invariant,
 pure decay, chunk-size invariance, linearity, column equivariance, state
@@ -203,3 +206,57 @@ def qk_prologue_bwd(x, dy):
     y = s / n
     ds = (dy - np.where(tiny, 0.0, y * (y * dy).sum(axis=-1, keepdims=True))) / n
     return ds * sig * (1.0 + x * (1.0 - sig))
+
+
+# ------------------------------------------------------------ output gate
+
+def out_gate(o, z):
+    """Output gate applied after the mixer: ``o * sigmoid(z)``, elementwise, in
+    float64.  The pages name a rank-128 gate g_t among the five gate families
+    ("Methodology", fig. 3(b)-(c): ranks (r_f, r_b, r_g, r_w, r_q)) and call it
+    the output gate (tab:abl caption, "wider output-gate"); z is its
+    pre-activation per token, head and value channel, produced upstream."""
+    o, z = _f64(o), _f64(z)
+    return o / (1.0 + np.exp(-z))
+
+
+def out_gate_bwd(o, z, dy):
+    """Gradients of ``sum(dy * out_gate(o, z))``: ``(do, dz)`` with
+    ``do = dy sig(z)`` and ``dz = dy o sig(z) (1 - sig(z))``."""
+    o, z, dy = _f64(o), _f64(z), _f64(dy)
+    sig = 1.0 / (1.0 + np.exp(-z))
+    return dy * sig, dy * o * sig * (1.0 - sig)
+
+
+# ------------------------------------------------------------ fused layer
+
+def fwd_fused(q, k, v, g, e, w, gamma=None, S0=None, z_out=None, qk_raw=False, threads=None):
+    """The mixer with its optional fused stages, composed from the functions
+    above in the order the pages' block applies them (fig. 3(b)): the q/k
+    prologue on raw q and k (``qk_raw``), the recurrence, then the output gate
+    on o (``z_out``).  Returns ``(o_gated, S_T, o)``: o is the pre-gate output
+    (equal to o_gated without a gate)."""
+    if qk_raw:
+        q, k = qk_prologue(q), qk_prologue(k)
+    o, S = fwd(q, k, v, g, e, w, gamma, S0, threads=threads)
+    og = out_gate(o, z_out) if z_out is not None else o
+    return og, S, o
+
+
+def bwd_fused(q, k, v, g, e, w, gamma=None, S0=None, dO=None, dS_final=None, z_out=None,
+              qk_raw=False, threads=None):
+    """Gradients of ``sum(o_gated * dO) + sum(S_T * dS_final)`` through
+    ``fwd_fused`` by the chain rule: the output gate's gradient, then the
+    recurrence's back-propagation through time, then the prologue's Jacobian
+    on dq and dk (gradients with respect to the raw q and k when ``qk_raw``).
+    Returns the dict of ``bwd`` plus ``dz_out`` when a gate is given."""
+    qh, kh = (qk_prologue(q), qk_prologue(k)) if qk_raw else (q, k)
+    out = {}
+    if z_out is not None:
+        o, _ = fwd(qh, kh, v, g, e, w, gamma, S0, threads=threads)
+        dO, out["dz_out"] = out_gate_bwd(o, z_out, dO)
+    out.update(bwd(qh, kh, v, g, e, w, gamma, S0, dO=dO, dS_final=dS_final, threads=threads))
+    if qk_raw:
+        out["dq"] = qk_prologue_bwd(q, out["dq"])
+        out["dk"] = qk_prologue_bwd(k, out["dk"])
+    return out
