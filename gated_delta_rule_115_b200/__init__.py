@@ -23,7 +23,7 @@ import torch
 
 __all__ = [
     "MuirError", "lib", "chunk_fwd", "chunk_bwd", "chunk_fwd_varlen", "chunk_bwd_varlen",
-    "recurrent_step", "qk_prologue",
+    "recurrent_step", "qk_prologue", "chunk_fwd_fused", "chunk_bwd_fused", "MuirFusion",
     "qk_prologue_bwd", "fwd_workspace_bytes", "bwd_workspace_bytes", "MuirChunkFunction",
     "LIB_PATH",
 ]
@@ -46,6 +46,10 @@ class MuirShape(ctypes.Structure):
     _fields_ = [("B", ctypes.c_int), ("T", ctypes.c_int), ("H", ctypes.c_int),
                 ("dk", ctypes.c_int), ("dv", ctypes.c_int), ("chunk", ctypes.c_int),
                 ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int)]
+
+
+class MuirFusion(ctypes.Structure):
+    _fields_ = [("z_out", ctypes.c_void_p), ("qk_raw", ctypes.c_int)]
 
 
 _lib = None
@@ -87,6 +91,13 @@ def lib():
         L.muir_qk_prologue.restype = I
         L.muir_qk_prologue_bwd.argtypes = [ctypes.c_longlong, I, I, P, P, P, P]
         L.muir_qk_prologue_bwd.restype = I
+        FP = ctypes.POINTER(MuirFusion)
+        L.muir_chunk_fused_workspace.argtypes = [SP, FP, I]
+        L.muir_chunk_fused_workspace.restype = S
+        L.muir_chunk_fwd_fused.argtypes = [SP, FP] + [P] * 15 + [S, P]
+        L.muir_chunk_fwd_fused.restype = I
+        L.muir_chunk_bwd_fused.argtypes = [SP, FP] + [P] * 24 + [S, P]
+        L.muir_chunk_bwd_fused.restype = I
         L.muir_chunk_fwd_noalloc.argtypes = [SP] + [P] * 10 + [P]
         L.muir_chunk_fwd_noalloc.restype = I
         L.muir_profile_enable.argtypes = [I]
@@ -223,6 +234,85 @@ def chunk_bwd(q, k, v, g, e, w, gamma, S0, dO, dS_final=None, chunk=64, S_chunks
                           _ptr(wsb), ctypes.c_size_t(0 if wsb is None else wsb.numel()),
                           _stream(q.device))
     _check("muir_chunk_bwd", rc)
+    return grads
+
+
+def _fusion(z_out, qk_raw):
+    return MuirFusion(None if z_out is None else _ptr(z_out).value, int(bool(qk_raw)))
+
+
+def chunk_fwd_fused(q, k, v, g, e, w, gamma, S0=None, z_out=None, qk_raw=False, chunk=128,
+                    out_dtype=None, save=True, ws=None):
+    """Forward with the fused stages (``muir_chunk_fwd_fused``): ``qk_raw``
+    means q and k are the raw pre-activations (SiLU and the unit L2 norm are
+    applied in the kernels); ``z_out`` is the output gate's pre-activation
+    (the output is ``o * sigmoid(z_out)``).  Returns ``(o, S_final, saved)``;
+    ``saved`` (None unless ``save``) holds what :func:`chunk_bwd_fused` reuses:
+    ``S_chunks``, ``M_chunks``, ``aux`` and, with a gate, ``o_pre``."""
+    L = lib()
+    B, T, H, dk = q.shape
+    dv = v.shape[-1]
+    shp = _shape(q, v, chunk, out_dtype)
+    fu = _fusion(z_out, qk_raw)
+    od = torch.bfloat16 if shp.out_dtype == MUIR_BF16 else torch.float32
+    o = torch.empty(B, T, H, dv, dtype=od, device=q.device)
+    o_pre = torch.empty_like(o) if z_out is not None else None
+    S_final = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
+    Sc = Mc = aux = None
+    if save:
+        n = -(-T // chunk)
+        Sc = torch.empty(B, H, n, dk, dv, dtype=torch.float32, device=q.device)
+        Mc = torch.empty(B, H, n, dk, dk, dtype=torch.float32, device=q.device)
+        aux = torch.empty(int(L.muir_chunk_aux_floats(ctypes.byref(shp))), dtype=torch.float32,
+                          device=q.device)
+    need = int(L.muir_chunk_fused_workspace(ctypes.byref(shp), ctypes.byref(fu), 0))
+    if need == 0:
+        raise MuirError("muir_chunk_fused_workspace", 2)
+    wsb = _workspace(need, q.device, ws)
+    rc = L.muir_chunk_fwd_fused(ctypes.byref(shp), ctypes.byref(fu), _ptr(q), _ptr(k), _ptr(v),
+                                _ptr(g), _ptr(e), _ptr(w), _ptr(gamma), _ptr(S0), _ptr(o),
+                                _ptr(o_pre), _ptr(S_final), _ptr(Sc), _ptr(Mc), _ptr(aux),
+                                _ptr(wsb), ctypes.c_size_t(wsb.numel()), _stream(q.device))
+    _check("muir_chunk_fwd_fused", rc)
+    saved = dict(S_chunks=Sc, M_chunks=Mc, aux=aux, o_pre=o_pre) if save else None
+    return o, S_final, saved
+
+
+def chunk_bwd_fused(q, k, v, g, e, w, gamma, S0, dO, dS_final=None, z_out=None, qk_raw=False,
+                    o_pre=None, saved=None, chunk=128, ws=None):
+    """Gradients through :func:`chunk_fwd_fused` (``muir_chunk_bwd_fused``):
+    ``dO`` is the gradient of the (gated) output.  Returns the dict of
+    :func:`chunk_bwd` plus ``dz_out`` with a gate; dq and dk are with respect
+    to the raw q and k when ``qk_raw``.  ``saved`` from the forward skips
+    recomputation; with a gate, ``o_pre`` (or ``saved["o_pre"]``) is required."""
+    L = lib()
+    shp = _shape(q, v, chunk, None)
+    if saved is not None and o_pre is None:
+        o_pre = saved.get("o_pre")
+    if o_pre is not None:
+        shp.out_dtype = MUIR_BF16 if o_pre.dtype == torch.bfloat16 else MUIR_FP32
+    fu = _fusion(z_out, qk_raw)
+    grads = {n: torch.empty_like(x) for n, x in
+             dict(dq=q, dk=k, dv=v, dg=g, de=e, dw=w, dgamma=gamma).items()}
+    B, T, H, dk = q.shape
+    grads["dS0"] = torch.empty(B, H, dk, v.shape[-1], dtype=torch.float32, device=q.device)
+    dz = torch.empty_like(z_out) if z_out is not None else None
+    Sc, Mc, aux = ((saved["S_chunks"], saved["M_chunks"], saved["aux"]) if saved is not None
+                   else (None, None, None))
+    need = int(L.muir_chunk_fused_workspace(ctypes.byref(shp), ctypes.byref(fu), 1))
+    if need == 0:
+        raise MuirError("muir_chunk_fused_workspace", 2)
+    wsb = _workspace(need, q.device, ws)
+    rc = L.muir_chunk_bwd_fused(ctypes.byref(shp), ctypes.byref(fu), _ptr(q), _ptr(k), _ptr(v),
+                                _ptr(g), _ptr(e), _ptr(w), _ptr(gamma), _ptr(S0), _ptr(Sc),
+                                _ptr(Mc), _ptr(aux), _ptr(o_pre), _ptr(dO), _ptr(dS_final),
+                                *[_ptr(grads[n]) for n in ("dq", "dk", "dv", "dg", "de", "dw",
+                                                           "dgamma")],
+                                _ptr(dz), _ptr(grads["dS0"]), _ptr(wsb),
+                                ctypes.c_size_t(wsb.numel()), _stream(q.device))
+    _check("muir_chunk_bwd_fused", rc)
+    if dz is not None:
+        grads["dz_out"] = dz
     return grads
 
 

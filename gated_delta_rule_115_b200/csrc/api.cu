@@ -316,3 +316,106 @@ muir_status muir_qk_prologue_bwd(long long rows, int d, muir_dtype dtype, const 
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------ fused stages
+
+namespace {
+
+bool fused_any(const muir_fusion* f) { return f && (f->z_out || f->qk_raw); }
+
+// The fused stages run inside the on-chip kernels: bf16 inputs, dk = dv = 128,
+// chunk 128, T a multiple of 128.
+muir_status check_fusion(const muir_shape* s, const muir_fusion* f) {
+    if (!f) return MUIR_ERR_INVALID_ARG;
+    if (f->qk_raw != 0 && f->qk_raw != 1) return MUIR_ERR_INVALID_ARG;
+    if (!ok_opt(f->z_out)) return MUIR_ERR_INVALID_ARG;
+    if (fused_any(f) && !muir::v2::fwd2_supported(s->B, s->T, s->H, s->dk, s->chunk,
+                                                  s->in_dtype == MUIR_BF16))
+        return MUIR_ERR_UNSUPPORTED;
+    return MUIR_OK;
+}
+
+size_t fused_ws(const muir_shape* s, const muir_fusion* f, bool backward) {
+    const size_t base = backward
+        ? muir::chunk_bwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false, s->in_dtype == MUIR_BF16)
+        : muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false, s->in_dtype == MUIR_BF16);
+    if (!fused_any(f)) return base;
+    return ((base + 255) & ~(size_t)255) + muir::fused_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk);
+}
+
+char* fused_region(const muir_shape* s, void* ws, bool backward) {
+    const size_t base = backward
+        ? muir::chunk_bwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false, s->in_dtype == MUIR_BF16)
+        : muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false, s->in_dtype == MUIR_BF16);
+    return static_cast<char*>(ws) + ((base + 255) & ~(size_t)255);
+}
+
+}  // namespace
+
+size_t muir_chunk_fused_workspace(const muir_shape* s, const muir_fusion* f, int backward) {
+    if (check_shape(s) != MUIR_OK || check_fusion(s, f) != MUIR_OK) return 0;
+    return fused_ws(s, f, backward != 0);
+}
+
+muir_status muir_chunk_fwd_fused(const muir_shape* s, const muir_fusion* f, const void* q,
+                                 const void* k, const void* v, const void* g, const void* e,
+                                 const void* w, const void* gamma, const float* S0, void* o,
+                                 void* o_pre, float* S_final, float* S_chunks, float* M_chunks,
+                                 float* aux, void* ws, size_t ws_bytes, void* stream) {
+    muir_status st = check_shape(s);
+    if (st != MUIR_OK) return st;
+    if ((st = check_fusion(s, f)) != MUIR_OK) return st;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
+        !ok_ptr(gamma) || !ok_ptr(o) || !ok_opt(o_pre) || !ok_opt(S0) || !ok_opt(S_final) ||
+        !ok_opt(S_chunks) || !ok_opt(M_chunks) || !ok_opt(aux) || (o_pre && !f->z_out))
+        return MUIR_ERR_INVALID_ARG;
+    const size_t need = fused_ws(s, f, false);
+    if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
+    if ((st = check_device()) != MUIR_OK) return st;
+    muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);
+    P.aux = aux;
+    if (fused_any(f)) {
+        P.zo = f->z_out;
+        P.o_pre = o_pre;
+        P.qk_raw = f->qk_raw;
+        P.fused_ws = fused_region(s, ws, false);
+    }
+    return from_cuda(muir::run_chunk_fwd(P, S0, o, S_final, S_chunks, M_chunks, ws, ws_bytes,
+                                         static_cast<cudaStream_t>(stream)));
+}
+
+muir_status muir_chunk_bwd_fused(const muir_shape* s, const muir_fusion* f, const void* q,
+                                 const void* k, const void* v, const void* g, const void* e,
+                                 const void* w, const void* gamma, const float* S0,
+                                 const float* S_chunks, const float* M_chunks, const float* aux,
+                                 const void* o_pre, const void* dO, const float* dS_final,
+                                 void* dq, void* dk, void* dv, void* dg, void* de, void* dw,
+                                 void* dgamma, void* dz_out, float* dS0, void* ws, size_t ws_bytes,
+                                 void* stream) {
+    muir_status st = check_shape(s);
+    if (st != MUIR_OK) return st;
+    if ((st = check_fusion(s, f)) != MUIR_OK) return st;
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
+        !ok_ptr(gamma) || !ok_ptr(dO) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) ||
+        !ok_ptr(dg) || !ok_ptr(de) || !ok_ptr(dw) || !ok_ptr(dgamma) || !ok_opt(S0) ||
+        !ok_opt(S_chunks) || !ok_opt(M_chunks) || !ok_opt(dS_final) || !ok_opt(dS0) ||
+        !ok_opt(aux) || (aux && !S_chunks) || !ok_opt(o_pre) || !ok_opt(dz_out))
+        return MUIR_ERR_INVALID_ARG;
+    if (f->z_out && (!o_pre || !dz_out)) return MUIR_ERR_INVALID_ARG;
+    const size_t need = fused_ws(s, f, true);
+    if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
+    if ((st = check_device()) != MUIR_OK) return st;
+    muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);
+    P.aux = const_cast<float*>(aux);
+    if (fused_any(f)) {
+        P.zo = f->z_out;
+        P.o_pre = const_cast<void*>(o_pre);
+        P.o_pre_f32 = s->out_dtype == MUIR_FP32;
+        P.dzo = dz_out;
+        P.qk_raw = f->qk_raw;
+        P.fused_ws = fused_region(s, ws, true);
+    }
+    return from_cuda(muir::run_chunk_bwd(P, S0, S_chunks, M_chunks, dO, dS_final, dq, dk, dv, dg,
+                                         de, dw, dgamma, dS0, ws, ws_bytes,
+                                         static_cast<cudaStream_t>(stream)));
+}

@@ -86,6 +86,13 @@ __device__ __forceinline__ void st8_bf16(__nv_bfloat16* p, const float* v) {
     *reinterpret_cast<uint4*>(p) = u;
 }
 
+// Fused q/k prologue: x -> SiLU(x) r with r the row's inverse norm (the
+// forward applies the same arithmetic).
+__device__ __forceinline__ void prologue8(float* v, float r) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = v[u] * sigmoid_f(v[u]) * r;
+}
+
 // Store 32 values at columns 32 * c32 .. +32 of row t of a T16 tile.
 template <bool BF16>
 __device__ __forceinline__ void row_st32(unsigned char* tile, int t, int c32, const float* v) {
@@ -184,11 +191,43 @@ __global__ void __launch_bounds__(256) k2_bprep(const __grid_constant__ BprepPar
         }
     }
     if (!cta_wait(&bar[0], 0) && tid == 0) atomicOr(&bad, 1);
+    if (p.zo) {  // fused output gate: dO = dO' sig(z) (bf16), dz = dO' o sig (1 - sig)
+        const size_t ro = (((size_t)(bh / p.H) * p.T + (size_t)n * kC + t) * p.H + bh % p.H) * kD + 64 * h;
+        const __nv_bfloat16* zr = reinterpret_cast<const __nv_bfloat16*>(p.zo) + ro;
+        __nv_bfloat16* er = reinterpret_cast<__nv_bfloat16*>(p.dO_eff) + ro;
+        __nv_bfloat16* dzr = reinterpret_cast<__nv_bfloat16*>(p.dzo) + ro;
+#pragma unroll 2
+        for (int i = 0; i < 8; ++i) {
+            float dy[8], zv[8], ov[8], dov[8], dzv[8];
+            ld_chunk16<true>(Dt, t, 8 * h + i, dy);
+            ld8_bf16(zr + 8 * i, zv);
+            if (p.o_pre_f32) {
+                const float* op = reinterpret_cast<const float*>(p.o_pre) + ro + 8 * i;
+                const float4 a = __ldg(reinterpret_cast<const float4*>(op));
+                const float4 b = __ldg(reinterpret_cast<const float4*>(op + 4));
+                ov[0] = a.x; ov[1] = a.y; ov[2] = a.z; ov[3] = a.w;
+                ov[4] = b.x; ov[5] = b.y; ov[6] = b.z; ov[7] = b.w;
+            } else {
+                ld8_bf16(reinterpret_cast<const __nv_bfloat16*>(p.o_pre) + ro + 8 * i, ov);
+            }
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {  // dO bf16 -> fp16 in place (own chunks)
-        float v[8];
-        ld_chunk16<true>(Dt, t, 8 * h + i, v);
-        st_chunk16<false>(Dt, t, 8 * h + i, v);
+            for (int u = 0; u < 8; ++u) {
+                const float sg = sigmoid_f(zv[u]);
+                // the bf16 value the later kernels read
+                dov[u] = __bfloat162float(__float2bfloat16_rn(dy[u] * sg));
+                dzv[u] = dy[u] * ov[u] * sg * (1.f - sg);
+            }
+            st8_bf16(er + 8 * i, dov);
+            st8_bf16(dzr + 8 * i, dzv);
+            st_chunk16<false>(Dt, t, 8 * h + i, dov);
+        }
+    } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {  // dO bf16 -> fp16 in place (own chunks)
+            float v[8];
+            ld_chunk16<true>(Dt, t, 8 * h + i, v);
+            st_chunk16<false>(Dt, t, 8 * h + i, v);
+        }
     }
     fence_async_smem();
     sync_all();
@@ -634,6 +673,7 @@ struct Bwd2Smem {
     float P2[kD];
     float sfx[4][kD];  // per-quarter totals of the reverse scan
     float dgb[kD];     // dLbar of the chunk (value slabs summed in a fixed order)
+    float dot[2][8][kC];  // fused prologue: row dots dq^.q^ and dk^.k^ per (half, warp group)
     uint64_t bar[8];
     uint32_t tslot;
     int bad;
@@ -650,6 +690,7 @@ enum { kStrictLow = 0, kInclLow, kStrictUp, kInclUp };
 // mask them in place and use them as the A operands of TF32
 // products with a pivoted operand (K-major TF32 tile, 64 rows = the half's
 // channels) into one of four 64-column accumulators (TMEM 256..511).
+template <bool QKRAW>
 __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Params p) {
     extern __shared__ __align__(1024) unsigned char smraw[];
     unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
@@ -750,6 +791,8 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
         const uint32_t ph = (uint32_t)(it & 1);
         const int n = c % N, bh = c / N, hd = bh % p.H, b = bh / p.H;
         const size_t tok = ((size_t)b * p.T + (size_t)n * kC + t) * p.H + hd;
+        const float rq = QKRAW ? __ldg(p.rnorm + (size_t)c * 2 * kC + t) : 1.f;
+        const float rk = QKRAW ? __ldg(p.rnorm + (size_t)c * 2 * kC + kC + t) : 1.f;
         if (tid == 0) {
             mbar_arrive_expect_tx(&s.bar[B2IN], 4 * kT16Bytes);
             const int z = b * p.T + n * kC;
@@ -807,6 +850,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             {  // Am -> Bt0, Km -> Bt1
                 float kv[16], ev[16], am[16], km[16];
                 ld8_bf16(kin, kv); ld8_bf16(kin + 8, kv + 8);
+                if (QKRAW) { prologue8(kv, rk); prologue8(kv + 8, rk); }
                 ld8_bf16(ein, ev); ld8_bf16(ein + 8, ev + 8);
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
@@ -826,6 +870,10 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 float kv[16], qv[16], gv[16], kp[16], qp[16];
                 ld8_bf16(kin, kv); ld8_bf16(kin + 8, kv + 8);
                 ld8_bf16(qin, qv); ld8_bf16(qin + 8, qv + 8);
+                if (QKRAW) {
+                    prologue8(kv, rk); prologue8(kv + 8, rk);
+                    prologue8(qv, rq); prologue8(qv + 8, rq);
+                }
                 ld8_bf16(gin_, gv); ld8_bf16(gin_ + 8, gv + 8);
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
@@ -847,6 +895,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + j0;
                 const size_t ro = tok * kD + j0;
                 float dL[16];
+                float dotq = 0.f, dotk = 0.f;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {  // 8 channels at a time
                     const int u0 = 8 * hh;
@@ -861,11 +910,15 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                     ld8_bf16(ein + u0, ev);
                     ld8_bf16(qin + u0, qv);
                     ld8_bf16(gin_ + u0, gv);
+                    if (QKRAW) { prologue8(kv, rk); prologue8(qv, rq); }
                     float pq[8], pk[8], pa[8], pl[8];
 #pragma unroll
                     for (int u = 0; u < 8; u += 4) {
-                        const float4 x0 = __ldg(reinterpret_cast<const float4*>(p.Pq + cb + u0 + u));
-                        const float4 x1 = __ldg(reinterpret_cast<const float4*>(p.Pk + cb + u0 + u));
+                        // (plain loads with the fused prologue: this kernel overwrites them)
+                        const float4 x0 = QKRAW ? *reinterpret_cast<const float4*>(p.Pq + cb + u0 + u)
+                                                : __ldg(reinterpret_cast<const float4*>(p.Pq + cb + u0 + u));
+                        const float4 x1 = QKRAW ? *reinterpret_cast<const float4*>(p.Pk + cb + u0 + u)
+                                                : __ldg(reinterpret_cast<const float4*>(p.Pk + cb + u0 + u));
                         const float4 x2 = __ldg(reinterpret_cast<const float4*>(p.Pa + cb + u0 + u));
                         const float4 x3 = __ldg(reinterpret_cast<const float4*>(p.Pd + cb + u0 + u));
                         pq[u] = x0.x; pq[u + 1] = x0.y; pq[u + 2] = x0.z; pq[u + 3] = x0.w;
@@ -892,10 +945,28 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                                 (a_km[u] * kv[u] + a_a[u] * ev[u] * kv[u]) * em +
                                 pl[u] * kv[u] + pq[u] * qh - pa[u] * ev[u] * kv[u];
                     }
-                    st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dq) + ro + u0, oq);
+                    if (QKRAW) {  // dq^, dk^ (fp32, over the P entries just read) and row dots
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) {
+                            dotq = fmaf(oq[u], qv[u], dotq);
+                            dotk = fmaf(ok[u], kv[u], dotk);
+                        }
+                        float* pq_ = p.Pq + cb + u0;
+                        float* pk_ = p.Pk + cb + u0;
+                        *reinterpret_cast<float4*>(pq_) = make_float4(oq[0], oq[1], oq[2], oq[3]);
+                        *reinterpret_cast<float4*>(pq_ + 4) = make_float4(oq[4], oq[5], oq[6], oq[7]);
+                        *reinterpret_cast<float4*>(pk_) = make_float4(ok[0], ok[1], ok[2], ok[3]);
+                        *reinterpret_cast<float4*>(pk_ + 4) = make_float4(ok[4], ok[5], ok[6], ok[7]);
+                    } else {
+                        st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dq) + ro + u0, oq);
+                        st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dk) + ro + u0, ok);
+                    }
                     st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dgamma) + ro + u0, og);
-                    st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dk) + ro + u0, ok);
                     st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.de) + ro + u0, oe);
+                }
+                if (QKRAW) {
+                    s.dot[0][4 * hj + g4][t] = dotq;
+                    s.dot[1][4 * hj + g4][t] = dotk;
                 }
                 // dg_t = sum_{t' >= t} dL_t' + dLbar: warp suffix scan, then later quarters
 #pragma unroll
@@ -925,6 +996,42 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                         o[u] = gv[u] >= kLogDecayMin ? dL[j] + post : 0.f;
                     }
                     st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dg) + ro + 8 * hh, o);
+                }
+            }
+            sync_all();
+        }
+        if (QKRAW) {
+            // the prologue's Jacobian: dx = SiLU'(x) r (dy^ - y^ (y^ . dy^)), row t,
+            // channels 32 g4 .. +32 (dy^ written above by this block; its barrier
+            // makes the writes visible)
+            float dq_dot = 0.f, dk_dot = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                dq_dot += s.dot[0][i][t];
+                dk_dot += s.dot[1][i][t];
+            }
+            const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + 32 * g4;
+            const size_t ro = tok * kD + 32 * g4;
+#pragma unroll 1
+            for (int which = 0; which < 2; ++which) {
+                const float* dy = (which ? p.Pk : p.Pq) + cb;
+                const __nv_bfloat16* xr = reinterpret_cast<const __nv_bfloat16*>(which ? p.k : p.q) + ro;
+                __nv_bfloat16* dx = reinterpret_cast<__nv_bfloat16*>(which ? p.dk : p.dq) + ro;
+                const float r = which ? rk : rq, dot = which ? dk_dot : dq_dot;
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    float xv[8], o[8];
+                    ld8_bf16(xr + 8 * i, xv);
+                    const float4 a0 = *reinterpret_cast<const float4*>(dy + 8 * i);
+                    const float4 a1 = *reinterpret_cast<const float4*>(dy + 8 * i + 4);
+                    const float dv8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) {
+                        const float sg = sigmoid_f(xv[u]);
+                        const float yh = xv[u] * sg * r;
+                        o[u] = (dv8[u] - yh * dot) * r * sg * (1.f + xv[u] * (1.f - sg));
+                    }
+                    st8_bf16(dx + 8 * i, o);
                 }
             }
             sync_all();
@@ -981,11 +1088,20 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     const int nsm = sm_count();
     cudaError_t e;
 
-    CUtensorMap tdO;
-    if (!map_tokens16(&tdO, a.dO, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+    // with a fused output gate, k2_bprep reads the gated output's gradient and
+    // writes the mixer's dO (dO_eff), which the later kernels read
+    CUtensorMap tdO, tdO_in;
+    if (!map_tokens16(&tdO_in, a.dO, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+    if (a.zo) {
+        if (!a.o_pre || !a.dO_eff || !a.dzo) return cudaErrorInvalidValue;
+        if (!map_tokens16(&tdO, a.dO_eff, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+    } else {
+        tdO = tdO_in;
+    }
 
     BprepParams bp;
-    bp.tdO = tdO; bp.T = a.T; bp.H = a.H; bp.Qp = a.Qp; bp.Bp = Bp;
+    bp.tdO = tdO_in; bp.T = a.T; bp.H = a.H; bp.Qp = a.Qp; bp.Bp = Bp;
+    bp.zo = a.zo; bp.o_pre = a.o_pre; bp.o_pre_f32 = a.o_pre_f32; bp.dO_eff = a.dO_eff; bp.dzo = a.dzo;
     if ((e = cudaFuncSetAttribute(k2_bprep, cudaFuncAttributeMaxDynamicSharedMemorySize, kBprepSmem)) != cudaSuccess) return e;
     MUIR_TIMED("k2_bprep", st, k2_bprep<<<nch, 256, kBprepSmem, st>>>(bp));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1015,8 +1131,10 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     p2.aux = a.aux; p2.Y16 = Y16; p2.dYR16 = dYR16; p2.Pq = Pq; p2.Pk = Pk; p2.Pa = Pa; p2.Pd = Pd;
     p2.dgb = dgb; p2.nslab = kD / SLAB;
     p2.dq = a.dq; p2.dk = a.dk; p2.dg = a.dg; p2.de = a.de; p2.dgamma = a.dgamma;
-    if ((e = cudaFuncSetAttribute(k2_bwd2, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwd2Smem)) != cudaSuccess) return e;
-    MUIR_TIMED("k2_bwd2", st, k2_bwd2<<<grid, 512, kBwd2Smem, st>>>(p2));
+    p2.rnorm = a.rnorm;
+    auto k2 = a.rnorm ? k2_bwd2<true> : k2_bwd2<false>;
+    if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwd2Smem)) != cudaSuccess) return e;
+    MUIR_TIMED("k2_bwd2", st, k2<<<grid, 512, kBwd2Smem, st>>>(p2));
     return cudaGetLastError();
 }
 

@@ -14,6 +14,14 @@ struct BprepParams {
     int T, H;
     const float* Qp;  // [nch][128][128]
     float* Bp;        // Q'^T dO per chunk
+    // fused output gate (zo non-null): tdO holds the gradient of the gated
+    // output; dO = dO' sigmoid(zo) is written to dO_eff (bf16, read by the
+    // later kernels) and dzo = dO' o_pre sigmoid'(zo) to dzo (bf16)
+    const void* zo;
+    const void* o_pre;
+    bool o_pre_f32;
+    void* dO_eff;
+    void* dzo;
 };
 
 struct RevParams {
@@ -46,14 +54,22 @@ struct Bwd2Params {
     const void *q, *k, *g, *e, *gamma;
     const unsigned char* aux;
     const unsigned char *Y16, *dYR16;
-    const float *Pq, *Pk, *Pa, *Pd, *dgb;  // dgb: [nslab][nch][128] partials of dLbar
+    float *Pq, *Pk;                       // with the fused prologue, reused for dq^, dk^
+    const float *Pa, *Pd, *dgb;           // dgb: [nslab][nch][128] partials of dLbar
     int nslab;
     void *dq, *dk, *dg, *de, *dgamma;
+    const float* rnorm;                   // fused prologue: [nch][2][128] inverse row norms
 };
 
 struct Bwd2Args {
     int B, T, H;
     const void *q, *k, *v, *g, *e, *w, *gamma, *dO;
+    const void* zo;                         // fused output gate: pre-activation, or null
+    const void* o_pre;                      // with zo: the forward's pre-gate output
+    bool o_pre_f32;                         // its dtype (fp32, else bf16)
+    void* dO_eff;                           // with zo: B*T*H*128 bf16 of workspace
+    void* dzo;                              // with zo: gradient of zo (bf16)
+    const float* rnorm;                     // fused q/k prologue: the forward's inverse row norms, or null
     const float* dS_final;                  // or null
     const unsigned char* aux;               // forward's saved records
     const float *Qp, *Mt, *S_chunks, *S_last;

@@ -97,13 +97,32 @@ cudaError_t run_chunk_fwd(const ChunkProblem& P, const float* S0, void* o, float
             a.Qp = f; f += nch * blk;
         }
         a.flags = flags;
+        // fused stages: output gate in k2_out, q/k prologue in k2_intra (its
+        // inverse row norms saved with the intermediates, else in fused_ws)
+        const long long rows = (long long)P.B * P.T * P.H;
+        char* fw = P.fused_ws;
+        if ((P.zo || P.qk_raw) && !fw) return cudaErrorInvalidValue;
+        a.zo = P.zo; a.o_pre = P.o_pre;
+        a.qk_raw = P.qk_raw;
+        if (P.qk_raw)
+            a.rnorm = P.aux ? v2::aux_rn(reinterpret_cast<unsigned char*>(P.aux), nch, (size_t)P.B * P.H)
+                            : reinterpret_cast<float*>(fw + 256);
         cudaError_t e = cudaMemsetAsync(flags, 0, 16, st);
         if (e == cudaSuccess) e = v2::span_check(P.g, P.B, P.T, P.H, flags, st);
         if (e == cudaSuccess) e = v2::run_fwd2(a, st);
         if (e != cudaSuccess) return e;
         ChunkProblem G = P;
         G.gate = flags;  // boundary-pivot path only when a chunk's span exceeds the single pivot
-        return fwd_bf16_d128(G, S0, o, S_final, S_chunks, M_chunks, shared, st);
+        if (P.qk_raw) {  // that path reads q^ and k^ as tensors
+            char* qh = fw + 256 + nch * 2 * 128 * 4;
+            char* kh = qh + rows * 128 * 2;
+            if ((e = qk_materialise_gated(flags, P.q, qh, rows, st)) != cudaSuccess) return e;
+            if ((e = qk_materialise_gated(flags, P.k, kh, rows, st)) != cudaSuccess) return e;
+            G.q = qh; G.k = kh;
+        }
+        if ((e = fwd_bf16_d128(G, S0, o, S_final, S_chunks, M_chunks, shared, st)) != cudaSuccess) return e;
+        if (P.zo && o) return out_gate_fix_gated(flags, o, P.o_pre, P.zo, rows * 128, P.out_bf16, st);
+        return cudaSuccess;
     }
     if (P.in_bf16) {
         if (P.D == 128) return fwd_bf16_d128(P, S0, o, S_final, S_chunks, M_chunks, ws, st);
@@ -131,6 +150,16 @@ cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S
         b.dO = dO; b.dS_final = dS_final;
         b.dq = dq; b.dk = dk; b.dv = dv; b.dg = dg; b.de = de; b.dw = dw; b.dgamma = dgamma;
         b.dS0 = dS0;
+        const long long rows = (long long)P.B * P.T * P.H;
+        char* fw = P.fused_ws;
+        if ((P.zo || P.qk_raw) && !fw) return cudaErrorInvalidValue;
+        char* qh = fw ? fw + 256 + nch * 2 * 128 * 4 : nullptr;
+        char* kh = qh ? qh + rows * 128 * 2 : nullptr;
+        if (P.zo) {  // fused output gate: k2_bprep forms the mixer's dO and dzo
+            if (!P.o_pre || !P.dzo) return cudaErrorInvalidValue;
+            b.zo = P.zo; b.o_pre = P.o_pre; b.o_pre_f32 = P.o_pre_f32; b.dzo = P.dzo;
+            b.dO_eff = kh + rows * 128 * 2;
+        }
         char* rest = shared;
         if (P.aux && S_chunks) {  // intermediates saved by the forward
             unsigned char* ax = reinterpret_cast<unsigned char*>(P.aux);
@@ -139,6 +168,7 @@ cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S
             b.Mt = v2::aux_Mt(ax, nch);
             b.S_last = v2::aux_SN(ax, nch);
             b.S_chunks = S_chunks;
+            if (P.qk_raw) b.rnorm = v2::aux_rn(ax, nch, (size_t)P.B * P.H);
         } else {  // recompute the forward's state pass and intermediates
             float* f = reinterpret_cast<float*>(shared);
             unsigned char* ax = reinterpret_cast<unsigned char*>(f + 4 * nch * blk);
@@ -152,16 +182,31 @@ cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S
             a.Mt = v2::aux_Mt(ax, nch);
             a.S_last = v2::aux_SN(ax, nch);
             a.flags = flags;
+            a.qk_raw = P.qk_raw;
+            if (P.qk_raw) a.rnorm = reinterpret_cast<float*>(fw + 256);
             if ((e = v2::run_fwd2(a, st)) != cudaSuccess) return e;
             b.aux = ax; b.Qp = a.Qp; b.Mt = a.Mt; b.S_last = a.S_last; b.S_chunks = a.S_chunks;
+            b.rnorm = a.rnorm;
             rest = reinterpret_cast<char*>(ax) + v2::aux_bytes(nch, (size_t)P.B * P.H);
         }
         b.ws = rest;
         if ((e = v2::run_bwd2(b, st)) != cudaSuccess) return e;
         ChunkProblem G = P;
         G.gate = flags;
-        return bwd_bf16_d128(G, S0, S_chunks, M_chunks, dO, dS_final, dq, dk, dv, dg, de, dw,
-                             dgamma, dS0, shared, st);
+        if (P.qk_raw) {  // the boundary-pivot path reads q^, k^ and returns dq^, dk^
+            if ((e = qk_materialise_gated(flags, P.q, qh, rows, st)) != cudaSuccess) return e;
+            if ((e = qk_materialise_gated(flags, P.k, kh, rows, st)) != cudaSuccess) return e;
+            G.q = qh; G.k = kh;
+        }
+        const void* dO_mix = P.zo ? static_cast<const void*>(b.dO_eff) : dO;
+        if ((e = bwd_bf16_d128(G, S0, S_chunks, M_chunks, dO_mix, dS_final, dq, dk, dv, dg, de, dw,
+                               dgamma, dS0, shared, st)) != cudaSuccess)
+            return e;
+        if (P.qk_raw) {
+            if ((e = qk_jacobian_gated(flags, P.q, dq, rows, st)) != cudaSuccess) return e;
+            if ((e = qk_jacobian_gated(flags, P.k, dk, rows, st)) != cudaSuccess) return e;
+        }
+        return cudaSuccess;
     }
 #define MUIR_BWD_ARGS P, S0, S_chunks, M_chunks, dO, dS_final, dq, dk, dv, dg, de, dw, dgamma, dS0, ws, st
     if (P.in_bf16) {

@@ -99,6 +99,7 @@ struct IntraSmem {
     float eP2[kD];      // 2^P2
     float Lb[kD];       // chunk total (log2 units)
     float lblk[4][32][33];  // strictly lower 32x32 diagonal blocks of L_A (leaf inverses)
+    float nrm[4][kC];   // fused prologue: per-quarter sums of SiLU(x)^2 of each row
     uint64_t bar[16];
     uint32_t tslot;
     int bad;
@@ -117,6 +118,33 @@ __device__ __forceinline__ void sync_all() {
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
+}
+
+// Fused q/k prologue: x -> SiLU(x) r with r the row's inverse norm.
+__device__ __forceinline__ void prologue8(float* v, float r) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) v[u] = v[u] * sigmoid_f(v[u]) * r;
+}
+
+// Sum of SiLU(x)^2 over this thread's 32 columns of row t of a raw tile.
+__device__ __forceinline__ float silu_sq32(const unsigned char* tile, int t, int h) {
+    float acc = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        float v[8];
+        ld_chunk16<true>(tile, t, 4 * h + i, v);
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+            const float sv = v[u] * sigmoid_f(v[u]);
+            acc = fmaf(sv, sv, acc);
+        }
+    }
+    return acc;
+}
+
+// Inverse row norm from the four quarter sums (the guard maps a zero row to zero).
+__device__ __forceinline__ float row_rnorm(const float (*nrm)[kC], int t) {
+    return rsqrtf(fmaxf(((nrm[0][t] + nrm[1][t]) + nrm[2][t]) + nrm[3][t], 1e-24f));
 }
 
 // Load 64 values (this thread's row t, columns 64h..64h+63) of a bf16 T16 tile.
@@ -173,6 +201,7 @@ __device__ __forceinline__ void tm_ld64(uint32_t tm, int q, int col, float* v) {
 // 512 threads: warp w owns rows 32 (w % 4) .. +32 (its TMEM lane quarter q) and
 // columns 32 (w / 4) .. +32 (h); thread t = 32 q + lane owns row t of every
 // per-chunk tile in those columns.  Thread 0 issues the TMA loads and the MMAs.
+template <bool QKRAW>
 __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ IntraParams p) {
     extern __shared__ __align__(1024) unsigned char smraw[];
     unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
@@ -263,7 +292,10 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
 #pragma unroll
             for (int j = 0; j < 32; ++j) s.tot[q][c0 + j] = L[j];
         }
+        if (QKRAW) s.nrm[h][t] = silu_sq32(S[1], t, h);
         __syncthreads();
+        const float rk = QKRAW ? row_rnorm(s.nrm, t) : 1.f;
+        if (QKRAW && h == 0) p.rnorm[(size_t)c * 2 * kC + kC + t] = rk;
 #pragma unroll
         for (int j = 0; j < 32; ++j) {
             float pre = 0.f;
@@ -284,6 +316,7 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         for (int i = 0; i < 4; ++i, rot8(L)) {
             float kv[8], ev[8], kp[8], kmh[8], kml[8], am[8];
             ld_chunk16<true>(S[1], t, 4 * h + i, kv);
+            if (QKRAW) prologue8(kv, rk);
             ld_chunk16<true>(S[2], t, 4 * h + i, ev);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -308,10 +341,18 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
 
         // ---- 3. query operands: Qp hi -> S3, Qp lo -> S4
         waitb(s, BB, ph);
+        float rq = 1.f;
+        if (QKRAW) {  // (the barrier of the wait above ordered the reads of nrm for k)
+            s.nrm[h][t] = silu_sq32(S[3], t, h);
+            __syncthreads();
+            rq = row_rnorm(s.nrm, t);
+            if (h == 0) p.rnorm[(size_t)c * 2 * kC + t] = rq;
+        }
 #pragma unroll 1
         for (int i = 0; i < 4; ++i, rot8(L)) {
             float qv[8], gv[8], qh[8], ql[8];
             ld_chunk16<true>(S[3], t, 4 * h + i, qv);
+            if (QKRAW) prologue8(qv, rq);
             ld_chunk16<true>(S[4], t, 4 * h + i, gv);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -458,6 +499,7 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         for (int i = 0; i < 4; ++i, rot8(L)) {
             float kv[8];
             ld_chunk16<true>(S[0], t, 4 * h + i, kv);
+            if (QKRAW) prologue8(kv, rk);
 #pragma unroll
             for (int u = 0; u < 8; ++u) kv[u] *= ex2(L[u]);
             st_chunk16<false>(S[0], t, 4 * h + i, kv);
@@ -532,6 +574,10 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
                     float q0, q1, g0, g1;
                     unpack16<true>(qa[u], q0, q1);
                     unpack16<true>(ga[u], g0, g1);
+                    if (QKRAW) {
+                        q0 = q0 * sigmoid_f(q0) * rq;
+                        q1 = q1 * sigmoid_f(q1) * rq;
+                    }
                     r[2 * u] = v[j + 2 * u] + q0 * g0 * ex2(L[j + 2 * u]);
                     r[2 * u + 1] = v[j + 2 * u + 1] + q1 * g1 * ex2(L[j + 2 * u + 1]);
                 }
@@ -550,6 +596,7 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         for (int i = 0; i < 4; ++i, rot8(L)) {
             float kv[8], ev[8];
             ld_chunk16<true>(S[2], t, 4 * h + i, kv);
+            if (QKRAW) prologue8(kv, rk);
             ld_chunk16<true>(S[3], t, 4 * h + i, ev);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
@@ -784,24 +831,39 @@ __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutPara
         if (!cta_wait(&bar[1], (uint32_t)(it & 1)) && tid == 0) bad = 1;
         const int cn = c + gridDim.x;
         if (tid == 0 && cn < nch) issue(cn);
-        // epilogue: o[b][n*C + t][h][64 hh ..] = D + O_intra
+        // epilogue: o[b][n*C + t][h][64 hh ..] = D + O_intra, times sigmoid(zo)
+        // when the output gate is fused (the pre-gate value then also to o_pre)
         const int n = c % N, bh = c / N, hd = bh % p.H, b = bh / p.H;
         float v[64];
         tm_ld64(tm + 64 * h, q, 0, v);
         const float* oi = p.Oi + (size_t)c * kC * kD + (size_t)t * kD + 64 * h;
-        Tout* od = reinterpret_cast<Tout*>(p.o) + (((size_t)b * p.T + (size_t)n * kC + t) * p.H + hd) * kD + 64 * h;
-#pragma unroll
-        for (int jj = 0; jj < 64; jj += 4) {
-            const float4 a = __ldg(reinterpret_cast<const float4*>(oi + jj));
-            const float r0 = v[jj] + a.x, r1 = v[jj + 1] + a.y, r2 = v[jj + 2] + a.z, r3 = v[jj + 3] + a.w;
+        const size_t ro = (((size_t)b * p.T + (size_t)n * kC + t) * p.H + hd) * kD + 64 * h;
+        Tout* od = reinterpret_cast<Tout*>(p.o) + ro;
+        Tout* pd = p.o_pre ? reinterpret_cast<Tout*>(p.o_pre) + ro : nullptr;
+        const __nv_bfloat16* zr = p.zo ? reinterpret_cast<const __nv_bfloat16*>(p.zo) + ro : nullptr;
+        auto put4 = [&](Tout* dst, int jj, float r0, float r1, float r2, float r3) {
             if constexpr (sizeof(Tout) == 4) {
-                *reinterpret_cast<float4*>(reinterpret_cast<float*>(od) + jj) = make_float4(r0, r1, r2, r3);
+                *reinterpret_cast<float4*>(reinterpret_cast<float*>(dst) + jj) = make_float4(r0, r1, r2, r3);
             } else {
                 uint2 u;
                 u.x = pack_bf16(r0, r1);
                 u.y = pack_bf16(r2, r3);
-                *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(od) + jj) = u;
+                *reinterpret_cast<uint2*>(reinterpret_cast<__nv_bfloat16*>(dst) + jj) = u;
             }
+        };
+#pragma unroll
+        for (int jj = 0; jj < 64; jj += 4) {
+            const float4 a = __ldg(reinterpret_cast<const float4*>(oi + jj));
+            float r0 = v[jj] + a.x, r1 = v[jj + 1] + a.y, r2 = v[jj + 2] + a.z, r3 = v[jj + 3] + a.w;
+            if (zr) {
+                if (pd) put4(pd, jj, r0, r1, r2, r3);
+                const uint2 zw = __ldg(reinterpret_cast<const uint2*>(zr + jj));
+                float z0, z1, z2, z3;
+                unpack16<true>(zw.x, z0, z1);
+                unpack16<true>(zw.y, z2, z3);
+                r0 *= sigmoid_f(z0); r1 *= sigmoid_f(z1); r2 *= sigmoid_f(z2); r3 *= sigmoid_f(z3);
+            }
+            put4(od, jj, r0, r1, r2, r3);
         }
         sync_all();
     }
@@ -898,11 +960,14 @@ cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st) {
     ip.q = a.q; ip.gamma = a.gamma;
     ip.M = a.M; ip.Mt = a.Mt; ip.Bn = a.Bn; ip.Qp = a.Qp; ip.Oi = a.Oi; ip.flags = a.flags;
     ip.aux = a.aux;
-    cudaError_t e = cudaFuncSetAttribute(k2_intra, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);
+    ip.qk_raw = a.qk_raw; ip.rnorm = a.rnorm;
+    if (a.qk_raw && !a.rnorm) return cudaErrorInvalidValue;
+    auto kern = a.qk_raw ? k2_intra<true> : k2_intra<false>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, kIntraSmem);
     if (e != cudaSuccess) return e;
     const int nsm = sm_count();
     const int grid = nch < nsm ? nch : nsm;
-    MUIR_TIMED("k2_intra", st, k2_intra<<<grid, 512, kIntraSmem, st>>>(ip));
+    MUIR_TIMED("k2_intra", st, kern<<<grid, 512, kIntraSmem, st>>>(ip));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     constexpr int SLAB = 32;
@@ -920,6 +985,7 @@ cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st) {
         if (!map_rows32f(&op.tQ, a.Qp, (long long)nch * kC)) return cudaErrorInvalidValue;
         op.B = a.B; op.T = a.T; op.H = a.H;
         op.S_chunks = a.S_chunks; op.Oi = a.Oi; op.o = a.o;
+        op.zo = a.zo; op.o_pre = a.zo ? a.o_pre : nullptr;
         if (a.out_bf16) {
             e = cudaFuncSetAttribute(k2_out<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
             if (e != cudaSuccess) return e;

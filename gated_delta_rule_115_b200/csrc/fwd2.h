@@ -32,7 +32,11 @@ struct AuxLayout {
 // [nch][128][128] fp32 (the reverse state pass reads M_n^T), then the final
 // states S_N [B*H][128][128] fp32.
 inline size_t aux_bytes(size_t nch, size_t bh) {
-    return nch * (AuxLayout::kBytes + 2 * 65536) + bh * 65536;
+    return nch * (AuxLayout::kBytes + 2 * 65536 + 1024) + bh * 65536;
+}
+// Inverse row norms of the fused q/k prologue: [nch][2][128] floats after S_N.
+inline float* aux_rn(unsigned char* aux, size_t nch, size_t bh) {
+    return reinterpret_cast<float*>(aux + nch * (AuxLayout::kBytes + 2 * 65536) + bh * 65536);
 }
 inline float* aux_SN(unsigned char* aux, size_t nch) {
     return reinterpret_cast<float*>(aux + nch * (AuxLayout::kBytes + 2 * 65536));
@@ -55,6 +59,11 @@ struct IntraParams {
     float* Oi;     // O_intra_n [t][c]
     unsigned char* aux;  // per-chunk AuxLayout records, or null (nothing saved)
     int* flags;
+    // fused q/k prologue: q and k hold raw x; every read applies
+    // SiLU(x) / ||SiLU(x)|| per token-head row, and the row's inverse norms
+    // go to rnorm[c][0][t] (q) and rnorm[c][1][t] (k) for the backward
+    int qk_raw;
+    float* rnorm;
 };
 
 struct ChainParams {
@@ -73,6 +82,8 @@ struct OutParams {
     const float* S_chunks;
     const float* Oi;
     void* o;             // token-major [B][T][H][128], fp32 or bf16
+    const void* zo;      // output-gate pre-activation [B][T][H][128] bf16, or null
+    void* o_pre;         // pre-gate output (as o), or null
 };
 
 struct Fwd2Args {
@@ -81,12 +92,16 @@ struct Fwd2Args {
     const void *q, *k, *v, *g, *e, *w, *gamma;
     const float* S0;
     void* o;             // may be null (state pass only)
+    const void* zo;      // output-gate pre-activation, or null (no gate)
+    void* o_pre;         // receives the pre-gate output when zo is set, or null
     float* S_final;      // may be null
     float* S_chunks;     // required
     float *M, *Mt, *Bn, *Qp, *Oi;
     float* S_last;       // copy of S_N for the backward, or null
     unsigned char* aux;  // null, or nch AuxLayout records
     int* flags;
+    int qk_raw;          // q and k are raw: the prologue is fused (needs rnorm)
+    float* rnorm;        // with qk_raw: [nch][2][128] inverse row norms (q, k)
 };
 
 bool fwd2_supported(int B, int T, int H, int D, int C, bool in_bf16);

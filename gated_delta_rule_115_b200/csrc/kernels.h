@@ -23,7 +23,31 @@ struct ChunkProblem {
     const void *q, *k, *v, *g, *e, *w, *gamma;
     float* aux;            // per-chunk saved intermediates (forward: written; backward: read) or null
     const int* gate;       // non-null: every kernel returns at once unless *gate != 0
+    // Stages fused around the recurrence (on-chip path only; all off by default):
+    const void* zo = nullptr;   // output gate pre-activation [B][T][H][D] bf16, or null
+    void* o_pre = nullptr;      // forward: pre-gate output (out dtype) or null; backward: read
+    bool o_pre_f32 = false;     // dtype of o_pre in the backward
+    void* dzo = nullptr;        // backward: gradient of zo (bf16)
+    int qk_raw = 0;             // q, k hold raw x; SiLU and the unit L2 norm are fused
+    char* fused_ws = nullptr;   // fused_ws_bytes() of workspace for the stages above
 };
+
+// Workspace the fused stages add (inverse row norms, materialised q^ / k^ and
+// the mixer's dO for the large-span fallback).
+inline size_t fused_ws_bytes(int B, int T, int H, int D, int C) {
+    const size_t nch = (size_t)B * H * ((T + C - 1) / C);
+    const size_t rows = (size_t)B * T * H;
+    return 256 + nch * 2 * C * 4 + 3 * rows * D * 2;
+}
+
+// Flag-gated helpers of the fused stages (fused.cu): each returns at once
+// unless *flag != 0 (the large-span fallback ran and needs them).
+cudaError_t qk_materialise_gated(const int* flag, const void* x, void* y, long long rows,
+                                 cudaStream_t st);
+cudaError_t qk_jacobian_gated(const int* flag, const void* x, void* dy, long long rows,
+                              cudaStream_t st);
+cudaError_t out_gate_fix_gated(const int* flag, void* o, void* o_pre, const void* z, long long n,
+                               bool out_bf16, cudaStream_t st);
 
 // Up to eight tensors moved between token-major [B][T][H][D] rows of the
 // ragged last chunk and a side buffer [B*H][C][D] (tail.cu).

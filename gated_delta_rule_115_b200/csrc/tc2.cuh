@@ -135,6 +135,14 @@ __device__ __forceinline__ void bulk_wait_all() {
     asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
 }
 
+// Logistic sigmoid 1 / (1 + e^-z) through the base-2 exponential
+// (e^-z = 2^(-z log2 e)); saturates to 0 and 1 without NaN.
+__device__ __forceinline__ float sigmoid_f(float z) {
+    float e;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-1.4426950408889634f * z));
+    return 1.f / (1.f + e);
+}
+
 // Fetch the 128-byte line holding `ptr` into L2 (no register result).
 __device__ __forceinline__ void prefetch_l2(const void* ptr) {
     asm volatile("prefetch.global.L2 [%0];" ::"l"(ptr) : "memory");

@@ -179,3 +179,19 @@ def decode_tokens(step: int, wid: int = 4, *, B=None, H=None, dk=None, dv=None, 
     td = TORCH_DTYPE[dtype]
     return {n: t.to(td).contiguous() for n, t in
             dict(q=q, k=k, v=v, g=g, e=e, w=w).items()}
+
+
+def fused_inputs(wid: int, *, seed=None, **over):
+    """Inputs of the fused layer: those of :func:`chunk_inputs` (same
+    overrides), plus raw q/k pre-activations ``xq``, ``xk`` ~ N(0,1) (the
+    prologue's inputs) and the output gate's pre-activation ``z_out`` ~ N(0,1),
+    all ``[B,T,H,d]`` in the workload dtype, drawn from their own seed."""
+    x = chunk_inputs(wid, **over)
+    B, T, H, dk = x["q"].shape
+    dv = x["v"].shape[-1]
+    gen = torch.Generator("cpu").manual_seed((5000 + wid) if seed is None else seed)
+    td = x["q"].dtype
+    x["xq"] = _randn(gen, B, T, H, dk).to(td).contiguous()
+    x["xk"] = _randn(gen, B, T, H, dk).to(td).contiguous()
+    x["z_out"] = _randn(gen, B, T, H, dv).to(td).contiguous()
+    return x

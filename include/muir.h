@@ -87,10 +87,11 @@ size_t muir_chunk_fwd_workspace(const muir_shape* shape);
 size_t muir_chunk_bwd_workspace(const muir_shape* shape);
 
 /* Floats of the optional per-chunk intermediates muir_chunk_fwd can save for
- * muir_chunk_bwd (`aux`; 0 for an invalid shape).  Per chunk, in the order of
- * S_chunks ([B][H][N], N = ceil(T/C)): the four decay-masked C x C matrices L_A, L_K, M_QK,
- * M_QA, the C/16 inverted 16 x 16 diagonal blocks of I + L_A, and Y (C x dv),
- * each padded to a multiple of 64 floats.  Host-only. */
+ * muir_chunk_bwd (`aux`; 0 for an invalid shape): the decay-masked C x C
+ * matrices, the inverse of the chunk's triangular system, the chunk's
+ * transformed keys and values and its chunk-end quantities, in a layout
+ * private to the library (it differs between the on-chip path and the
+ * boundary-pivot path, and the size covers both).  Host-only. */
 size_t muir_chunk_aux_floats(const muir_shape* shape);
 
 /*
@@ -204,6 +205,74 @@ muir_status muir_chunk_fwd_noalloc(const muir_shape* shape, const void* q, const
                                    const void* v, const void* g, const void* e, const void* w,
                                    const void* gamma, const float* S0, void* o, float* S_final,
                                    void* stream);
+
+/*
+ * Stages fused around the recurrence ("Muir", wolonglab.org page,
+ * "Methodology" and fig. 3(b)): the block's q/k pathways end in SiLU with a
+ * unit-normalised key, and a rank-128 gate g_t (the output gate, tab:abl
+ * caption "wider output-gate") multiplies the mixer's output.
+ *
+ *   z_out  : output-gate pre-activation [B][T][H][dv] in_dtype, or NULL (no
+ *            gate).  The forward writes o * sigmoid(z_out); the backward takes
+ *            the gradient of that gated output.
+ *   qk_raw : 0, or 1 = the q and k arguments hold the raw pre-activations
+ *            x_q, x_k: the kernels use SiLU(x) / ||SiLU(x)|| per token-head
+ *            row (the same prologue as muir_qk_prologue), and the backward
+ *            returns dq, dk with respect to x_q, x_k.
+ * Runs where the on-chip path runs (in_dtype MUIR_BF16, dk = dv = 128,
+ * chunk 128, T a multiple of 128); with any stage enabled, other shapes are
+ * MUIR_ERR_UNSUPPORTED.  With both stages off the calls equal muir_chunk_fwd /
+ * muir_chunk_bwd.
+ */
+typedef struct {
+    const void* z_out;
+    int qk_raw;
+} muir_fusion;
+
+/* Workspace bytes of muir_chunk_fwd_fused (backward == 0) or
+ * muir_chunk_bwd_fused (backward != 0); 0 for an invalid shape or fusion.
+ * Host-only. */
+size_t muir_chunk_fused_workspace(const muir_shape* shape, const muir_fusion* fusion,
+                                  int backward);
+
+/*
+ * muir_chunk_fwd with the fused stages.  Arguments as muir_chunk_fwd, plus:
+ *   o      : [B][T][H][dv] out_dtype, the gated output when z_out is set
+ *   o_pre  : [B][T][H][dv] out_dtype or NULL (NULL required without z_out):
+ *            receives the pre-gate output, which muir_chunk_bwd_fused needs
+ *   aux    : as muir_chunk_fwd; with qk_raw it also keeps the inverse row norms
+ *            of q^ and k^ for the backward
+ * A large decay span (a chunk whose channel log-decay total exceeds the single
+ * pivot) runs the boundary-pivot path on q^, k^ materialised in the workspace
+ * (bf16) and gates its output afterwards.
+ */
+muir_status muir_chunk_fwd_fused(const muir_shape* shape, const muir_fusion* fusion,
+                                 const void* q, const void* k, const void* v, const void* g,
+                                 const void* e, const void* w, const void* gamma,
+                                 const float* S0, void* o, void* o_pre, float* S_final,
+                                 float* S_chunks, float* M_chunks, float* aux, void* ws,
+                                 size_t ws_bytes, void* stream);
+
+/*
+ * muir_chunk_bwd with the fused stages.  Arguments as muir_chunk_bwd, plus:
+ *   o_pre  : the pre-gate output muir_chunk_fwd_fused wrote (required with
+ *            z_out, else ignored), out_dtype of the shape
+ *   dO     : gradient of the (gated) output, in_dtype
+ *   dz_out : [B][T][H][dv] in_dtype, receives the gradient of z_out (required
+ *            with z_out, else ignored)
+ *   aux    : as muir_chunk_bwd; with qk_raw it must come from a forward called
+ *            with qk_raw
+ * dq, dk are gradients with respect to the raw x_q, x_k when qk_raw is set.
+ * Missing o_pre / dz_out with z_out is MUIR_ERR_INVALID_ARG.
+ */
+muir_status muir_chunk_bwd_fused(const muir_shape* shape, const muir_fusion* fusion,
+                                 const void* q, const void* k, const void* v, const void* g,
+                                 const void* e, const void* w, const void* gamma,
+                                 const float* S0, const float* S_chunks, const float* M_chunks,
+                                 const float* aux, const void* o_pre, const void* dO,
+                                 const float* dS_final, void* dq, void* dk, void* dv, void* dg,
+                                 void* de, void* dw, void* dgamma, void* dz_out, float* dS0,
+                                 void* ws, size_t ws_bytes, void* stream);
 
 /*
  * One decode token for every (b, h) against a resident float32 state (same

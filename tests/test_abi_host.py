@@ -188,3 +188,25 @@ def test_binding_refuses_cpu_tensors(L):
     with pytest.raises(ValueError):
         m.recurrent_step(x, x, x, x, x, x, None, torch.zeros(1, 2, 64, 64), out_dtype=torch.float32,
                          o=torch.zeros(1, 2, 64))
+
+
+def test_fused_workspace_host_checks(L):
+    """muir_chunk_fused_workspace: 0 where a fused stage cannot run (ragged T,
+    fp32 inputs, head dim 64, chunk 64) or for a bad fusion; more than the
+    plain workspace where it can; equal to it with both stages off."""
+    import gated_delta_rule_115_b200 as m
+    on = m.MuirFusion(None, 1)
+    off = m.MuirFusion(None, 0)
+    good = _shape(m, T=512, dk=128, dv=128, chunk=128)
+    for backward in (0, 1):
+        plain = (L.muir_chunk_bwd_workspace if backward else L.muir_chunk_fwd_workspace)(
+            ctypes.byref(good))
+        assert L.muir_chunk_fused_workspace(ctypes.byref(good), ctypes.byref(on), backward) > plain
+        assert L.muir_chunk_fused_workspace(ctypes.byref(good), ctypes.byref(off), backward) == plain
+    for bad in (_shape(m, T=500, dk=128, dv=128, chunk=128),
+                _shape(m, T=512, dk=128, dv=128, chunk=128, in_dtype=1),
+                _shape(m, T=512, chunk=128),
+                _shape(m, T=512, dk=128, dv=128, chunk=64)):
+        assert L.muir_chunk_fused_workspace(ctypes.byref(bad), ctypes.byref(on), 0) == 0
+    assert L.muir_chunk_fused_workspace(ctypes.byref(good), ctypes.byref(m.MuirFusion(None, 2)), 0) == 0
+    assert L.muir_chunk_fused_workspace(ctypes.byref(good), None, 0) == 0
