@@ -12,7 +12,8 @@ Usage::
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl muir|reference]
 
-N > 1 runs one process per GPU (launched by torch.distributed.run); every rank
+N > 1 runs one process per GPU (launched by torch.distributed.run; started as
+a single process, the script relaunches itself that way); every rank
 processes its own batch (weak scaling, no data-path collective); the time is
 the max over ranks.  ``--impl reference`` times the fp64 CPU oracle on a
 bounded sample of the same workload (rank 0 only).  Prints ONE JSON line.
@@ -114,6 +115,47 @@ def max_over_ranks(value: float, world: int, device=None) -> float:
 def rank_seed(rank: int) -> int:
     """Seed of this rank's batch: rank 0 draws the canonical workload."""
     return 1000 + WID + 7919 * rank
+
+
+def rank_batch(rank: int, **over):
+    """This rank's batch of the workload (CPU tensors): every rank draws its
+    own inputs from its own seed (weak scaling: no data is exchanged)."""
+    from gated_delta_rule_115_b200 import inputs as I
+    return I.chunk_inputs(WID, seed=rank_seed(rank), **over)
+
+
+def timed_steps(step, steps: int, warmup: int, world: int, timer, barrier=None,
+                device=None) -> float:
+    """The timing protocol of every arm: ``warmup`` untimed steps, a barrier,
+    exactly ``steps`` timed steps, a barrier; returns ms per step, the max over
+    ranks.  ``timer()`` returns ``(start, stop)`` callables, stop() giving the
+    elapsed ms (CUDA events on the launching stream for the GPU arm)."""
+    for _ in range(warmup):
+        step()
+    if barrier is not None:
+        barrier()
+    start, stop = timer()
+    start()
+    for _ in range(steps):
+        step()
+    ms = stop()
+    if barrier is not None:
+        barrier()
+    return max_over_ranks(ms, world, device) / steps
+
+
+def job_tokens_per_s(ms_per_step: float, tokens_per_rank: int, world: int) -> float:
+    """Whole-job throughput: the tokens all ranks processed per step over the
+    slowest rank's step time."""
+    return tokens_per_rank * world / (ms_per_step / 1e3)
+
+
+def spawn_command(args_list, gpus: int, port: int):
+    """The command that runs this script once per GPU (one process per GPU,
+    rendezvous on 127.0.0.1), forwarding the script's own arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={gpus}", "--master-addr", "127.0.0.1", "--master-port", str(port),
+            os.path.abspath(__file__)] + list(args_list)
 
 
 # ------------------------------------------------------------------ clocks
@@ -252,7 +294,7 @@ def gpu_arm(args, rank, world, local):
     if args.T is not None:
         import dataclasses
         W = dataclasses.replace(W, T=args.T)
-    x = I.chunk_inputs(WID, seed=rank_seed(rank), T=W.T)
+    x = rank_batch(rank, T=W.T)
     d = {k: (v.to(dev) if v is not None else None) for k, v in x.items()}
     C = W.chunk
     args_in = [d[n] for n in NAMES]
@@ -266,41 +308,46 @@ def gpu_arm(args, rank, world, local):
 
     ws_f = torch.empty(muir.fwd_workspace_bytes(W.B, W.T, W.H, W.dk, C), dtype=torch.uint8, device=dev)
     ws_b = torch.empty(muir.bwd_workspace_bytes(W.B, W.T, W.H, W.dk, C), dtype=torch.uint8, device=dev)
-    for _ in range(args.warmup):
-        step()
-    torch.cuda.synchronize()
     gpu_id = ""
     try:
         gpu_id = "GPU-" + str(torch.cuda.get_device_properties(dev).uuid)
     except Exception:
         pass
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    torch.cuda.synchronize()
-    sampler = ClockSampler(gpu_id)
-    L.muir_profile_reset()
-    L.muir_profile_enable(1)
     st = torch.cuda.current_stream(dev)
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record(st)
-    for _ in range(args.steps):
-        step()
-    e1.record(st)
-    torch.cuda.synchronize()
-    L.muir_profile_enable(0)
+    sampler = None
+
+    def barrier():
+        torch.cuda.synchronize()
+        if world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def timer():
+        nonlocal sampler
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+        def start():
+            nonlocal sampler
+            sampler = ClockSampler(gpu_id)
+            L.muir_profile_reset()
+            L.muir_profile_enable(1)
+            e0.record(st)
+
+        def stop():
+            e1.record(st)
+            torch.cuda.synchronize()
+            L.muir_profile_enable(0)
+            return e0.elapsed_time(e1)
+        return start, stop
+
+    ms = timed_steps(step, args.steps, args.warmup, world, timer, barrier, dev)
     L.muir_profile_collect()
     clocks = sampler.stop()
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
-    ms_total = max_over_ranks(e0.elapsed_time(e1), world, dev)
-    ms = ms_total / args.steps
     prof = {L.muir_profile_name(i).decode(): (L.muir_profile_total_ms(i), L.muir_profile_launches(i))
             for i in range(L.muir_profile_count())}
     launches = sum(n for _, n in prof.values())
-    tokens = W.B * W.T * world
-    value = tokens / (ms / 1e3)
+    value = job_tokens_per_s(ms, W.B * W.T, world)
     token_heads = W.B * W.T * W.H
     fl = 3 * flops_fwd_per_token_head(C, W.dk) * token_heads * world
     tflops = fl / (ms / 1e3) / 1e12
@@ -331,6 +378,7 @@ def gpu_arm(args, rank, world, local):
     if not args.no_decode:
         out["decode"] = decode_measure(muir, I, dev, peaks)
         out["qk_prologue"] = qk_measure(muir, dev, peaks)
+        out["other_workloads"] = configs_measure(muir, I, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = len(os.sched_getaffinity(0))
         v, desc, dt = oracle_sample(args.cpu_seconds, threads)
@@ -512,14 +560,107 @@ def decode_measure(muir, I, dev, peaks, steps=50):
     b.record(st)
     torch.cuda.synchronize()
     ms_g = a.elapsed_time(b) / 1000
+    # a batch whose state (1 GiB) is far beyond the 126 MB L2: back-to-back
+    # steps read and write it from HBM without any flush
+    BL = 1024
+    S_l, g_l = I.decode_state(B=BL)
+    S_l = S_l.to(dev)
+    tok_l = {k: v.to(dev) for k, v in I.decode_tokens(0, B=BL).items()}
+    g_l = g_l.to(dev)
+    o_l = torch.empty(BL, W.H, W.dv, dtype=torch.bfloat16, device=dev)
+
+    def one_l():
+        muir.recurrent_step(tok_l["q"], tok_l["k"], tok_l["v"], tok_l["g"], tok_l["e"],
+                            tok_l["w"], g_l, S_l, gamma_static=True, o=o_l)
+
+    for _ in range(5):
+        one_l()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(steps):
+        one_l()
+    b.record(st)
+    torch.cuda.synchronize()
+    ms_l = a.elapsed_time(b) / steps
+    byts_l = DECODE_BYTES_PER_HEAD * BL * W.H
+    large = {"B": BL, "H": W.H, "state_bytes": BL * W.H * 128 * 128 * 4, "ms_per_step": ms_l,
+             "gbs": byts_l / (ms_l / 1e3) / 1e9,
+             "hbm_frac": byts_l / (ms_l / 1e3) / 1e9 / peaks["hbm_gbs"],
+             "tokens_per_s": BL / (ms_l / 1e3),
+             "note": "state 1 GiB >> L2: consecutive steps stream it from HBM, no flush"}
+    del S_l, tok_l, o_l
     return {
         "workload": "decode step B=64 H=16 d=128, fp32 state, bf16 tokens, static gamma",
+        "large_batch": large,
         "ms_per_step_l2_flushed": ms, "gbs_l2_flushed": gbs,
         "hbm_frac": gbs / peaks["hbm_gbs"], "tokens_per_s": W.B / (ms / 1e3),
         "bytes_per_step": byts,
         "graph_replay_ms_per_step": ms_g, "graph_replay_gbs_l2_resident": byts / (ms_g / 1e3) / 1e9,
         "note": "graph replay keeps the 64 MiB state in L2; the flushed number is the HBM one",
     }
+
+
+def configs_measure(muir, I, dev, peaks, steps=5, warmup=3):
+    """The other chunked workloads, each timed with CUDA events over ``steps``
+    back-to-back calls after ``warmup`` (inputs far beyond L2):
+    the layer-shaped forward (B=8, H=16, T=4096, d=128, its chunk 64, and
+    chunk 128, the on-chip path) and the large-chunk stress workload's
+    forward+backward (B=2, H=8, T=8192, chunk 256, the 8-token panel path for
+    its large decay spans, and chunk 128)."""
+    import torch
+    st = torch.cuda.current_stream(dev)
+
+    def timeit(fn):
+        for _ in range(warmup):
+            fn()
+        torch.cuda.synchronize()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(st)
+        for _ in range(steps):
+            fn()
+        b.record(st)
+        torch.cuda.synchronize()
+        return a.elapsed_time(b) / steps
+
+    out = {}
+    W1 = I.WORKLOADS[1]
+    x = I.chunk_inputs(1)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in x.items()}
+    del x
+    th = W1.B * W1.T * W1.H
+    for C in (W1.chunk, 128):
+        ws = torch.empty(muir.fwd_workspace_bytes(W1.B, W1.T, W1.H, W1.dk, C), dtype=torch.uint8,
+                         device=dev)
+        ms = timeit(lambda: muir.chunk_fwd(*[d[n] for n in NAMES], d["S0"], chunk=C, ws=ws))
+        out[f"layer_fwd_chunk{C}"] = {
+            "workload": f"layer-shaped forward B={W1.B} H={W1.H} T={W1.T} d={W1.dk} chunk {C}, bf16",
+            "ms": ms, "tokens_per_s": W1.B * W1.T / (ms / 1e3),
+            "gbs_algorithmic": BYTES_FWD * th / (ms / 1e3) / 1e9,
+            "hbm_frac": BYTES_FWD * th / (ms / 1e3) / 1e9 / peaks["hbm_gbs"]}
+        del ws
+    del d
+    W3 = I.WORKLOADS[3]
+    x = I.chunk_inputs(3, with_dO=True)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in x.items()}
+    del x
+    for C in (W3.chunk, 128):
+        wf = torch.empty(muir.fwd_workspace_bytes(W3.B, W3.T, W3.H, W3.dk, C), dtype=torch.uint8,
+                         device=dev)
+        wb = torch.empty(muir.bwd_workspace_bytes(W3.B, W3.T, W3.H, W3.dk, C), dtype=torch.uint8,
+                         device=dev)
+
+        def fb():
+            _, _, Sc, Mc, aux = muir.chunk_fwd(*[d[n] for n in NAMES], d["S0"], chunk=C,
+                                               return_saved=True, save_aux=True, ws=wf)
+            muir.chunk_bwd(*[d[n] for n in NAMES], d["S0"], d["dO"], chunk=C, S_chunks=Sc,
+                           M_chunks=Mc, aux=aux, ws=wb)
+        ms = timeit(fb)
+        out[f"stress_fwd_bwd_chunk{C}"] = {
+            "workload": f"large-chunk stress fwd+bwd B={W3.B} H={W3.H} T={W3.T} d={W3.dk} chunk {C}, bf16",
+            "ms": ms, "tokens_per_s": W3.B * W3.T / (ms / 1e3)}
+        del wf, wb
+    return out
 
 
 def qk_measure(muir, dev, peaks, steps=20):
@@ -565,6 +706,15 @@ def qk_measure(muir, dev, peaks, steps=20):
 def main(argv=None):
     args = parse_args(argv)
     rank, world, local = dist_env()
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # started as one process: run one rank per GPU under torch.distributed.run
+        import socket
+        sk = socket.socket()
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+        sk.close()
+        argv_list = sys.argv[1:] if argv is None else list(argv)
+        return subprocess.call(spawn_command(argv_list, args.gpus, port))
     if world != args.gpus:
         print(f"warning: --gpus {args.gpus} but WORLD_SIZE={world}", file=sys.stderr)
     if args.impl == "reference":

@@ -64,6 +64,8 @@ def lib():
         L = ctypes.CDLL(LIB_PATH)
         P, I, S = ctypes.c_void_p, ctypes.c_int, ctypes.c_size_t
         SP = ctypes.POINTER(MuirShape)
+        L.muir_selftest_expired_wait.argtypes = [I, P]
+        L.muir_selftest_expired_wait.restype = I
         L.muir_device_wait_status.argtypes = []
         L.muir_device_wait_status.restype = I
         L.muir_status_string.argtypes = [I]

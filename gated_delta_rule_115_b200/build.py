@@ -2,6 +2,9 @@
 
 Usage: ``python -m gated_delta_rule_115_b200.build [--force] [--debug]``.
 The shared library lands next to this file; object files go to ``_build/``.
+``--debug`` (with ``--force`` to rebuild every object) defines MUIR_DEBUG: the
+C-ABI entry points then also ask the CUDA runtime where every pointer lives and
+refuse, with MUIR_ERR_INVALID_ARG, memory the device cannot address.
 """
 from __future__ import annotations
 

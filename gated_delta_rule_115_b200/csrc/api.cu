@@ -12,8 +12,24 @@
 namespace {
 
 bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+#ifdef MUIR_DEBUG
+// Debug builds (build.py --debug) also ask the CUDA runtime where each
+// pointer lives and refuse host memory the device cannot address.
+bool device_addressable(const void* p) {
+    cudaPointerAttributes a;
+    if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+        cudaGetLastError();
+        return false;
+    }
+    return a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged ||
+           (a.type == cudaMemoryTypeHost && a.devicePointer != nullptr);
+}
+bool ok_ptr(const void* p) { return p != nullptr && aligned16(p) && device_addressable(p); }
+bool ok_opt(const void* p) { return p == nullptr || (aligned16(p) && device_addressable(p)); }
+#else
 bool ok_ptr(const void* p) { return p != nullptr && aligned16(p); }
 bool ok_opt(const void* p) { return p == nullptr || aligned16(p); }
+#endif
 bool ok_dtype(muir_dtype d) { return d == MUIR_BF16 || d == MUIR_FP32; }
 
 // The kernels use sm_100a instructions: require compute capability 10.x.
@@ -108,7 +124,8 @@ muir_status muir_device_wait_status(void) {
     if (cudaDeviceSynchronize() != cudaSuccess) return MUIR_ERR_CUDA;
     const unsigned int n = muir::timeouts_bf16_d128() + muir::timeouts_bf16_d64() +
                            muir::timeouts_f32_d128() + muir::timeouts_f32_d64() +
-                           muir::v2::timeouts_v2() + muir::v2::timeouts_bwd2();
+                           muir::v2::timeouts_v2() + muir::v2::timeouts_bwd2() +
+                           muir::timeouts_selftest();
     return n ? MUIR_ERR_DEVICE_TIMEOUT : MUIR_OK;
 }
 
@@ -418,4 +435,11 @@ muir_status muir_chunk_bwd_fused(const muir_shape* s, const muir_fusion* f, cons
     return from_cuda(muir::run_chunk_bwd(P, S0, S_chunks, M_chunks, dO, dS_final, dq, dk, dv, dg,
                                          de, dw, dgamma, dS0, ws, ws_bytes,
                                          static_cast<cudaStream_t>(stream)));
+}
+
+muir_status muir_selftest_expired_wait(int limit_us, void* stream) {
+    if (limit_us < 1 || limit_us > 1000000) return MUIR_ERR_INVALID_ARG;
+    muir_status st = check_device();
+    if (st != MUIR_OK) return st;
+    return from_cuda(muir::launch_expired_wait(limit_us, static_cast<cudaStream_t>(stream)));
 }

@@ -40,6 +40,11 @@ inline size_t fused_ws_bytes(int B, int T, int H, int D, int C) {
     return 256 + nch * 2 * C * 4 + 3 * rows * D * 2;
 }
 
+// Self-test of the bounded device waits (selftest.cu): one block waits
+// limit_us microseconds on a barrier nothing arrives on and records the expiry.
+cudaError_t launch_expired_wait(int limit_us, cudaStream_t st);
+unsigned int timeouts_selftest();
+
 // Flag-gated helpers of the fused stages (fused.cu): each returns at once
 // unless *flag != 0 (the large-span fallback ran and needs them).
 cudaError_t qk_materialise_gated(const int* flag, const void* x, void* y, long long rows,

@@ -71,13 +71,14 @@ __device__ __forceinline__ bool mbar_try(uint64_t* bar, uint32_t parity) {
     return done != 0;
 }
 
-// Wait for the phase of parity `parity` to complete; false after kWaitNs.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) {
+// Wait for the phase of parity `parity` to complete; false after limit_ns.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
+                                          uint64_t limit_ns = kWaitNs) {
     if (mbar_try(bar, parity)) return true;
     const uint64_t t0 = globaltimer();
     for (;;) {
         if (mbar_try(bar, parity)) return true;
-        if (globaltimer() - t0 > kWaitNs) return false;
+        if (globaltimer() - t0 > limit_ns) return false;
     }
 }
 

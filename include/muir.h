@@ -81,6 +81,14 @@ const char* muir_status_string(muir_status s);
  * clears the record. */
 muir_status muir_device_wait_status(void);
 
+/* Self-test of the bounded device waits: enqueues one block that waits
+ * limit_us microseconds (1 .. 1000000) on a shared-memory barrier that nothing
+ * ever arrives on, with no copy or tensor-core operation in flight.  The wait
+ * runs out, the expiry is recorded as for the chunk kernels' waits, and the
+ * block exits, so the next muir_device_wait_status returns
+ * MUIR_ERR_DEVICE_TIMEOUT.  Any other limit is MUIR_ERR_INVALID_ARG. */
+muir_status muir_selftest_expired_wait(int limit_us, void* stream);
+
 /* Bytes of device workspace muir_chunk_fwd / muir_chunk_bwd need for this
  * shape (0 for an invalid shape).  Host-only; enqueues nothing. */
 size_t muir_chunk_fwd_workspace(const muir_shape* shape);

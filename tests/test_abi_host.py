@@ -210,3 +210,19 @@ def test_fused_workspace_host_checks(L):
         assert L.muir_chunk_fused_workspace(ctypes.byref(bad), ctypes.byref(on), 0) == 0
     assert L.muir_chunk_fused_workspace(ctypes.byref(good), ctypes.byref(m.MuirFusion(None, 2)), 0) == 0
     assert L.muir_chunk_fused_workspace(ctypes.byref(good), None, 0) == 0
+
+
+def test_debug_build_compiles(tmp_path):
+    """The MUIR_DEBUG variant of the C-ABI layer (pointer residency checks)
+    compiles for sm_100a."""
+    import subprocess
+    src = os.path.join(ROOT, "gated_delta_rule_115_b200", "csrc", "api.cu")
+    r = subprocess.run(["/usr/local/cuda/bin/nvcc", "-gencode", "arch=compute_100a,code=sm_100a",
+                        "-std=c++17", "-Xcompiler", "-fPIC", "-DMUIR_DEBUG=1", "-c", src, "-o",
+                        str(tmp_path / "api_debug.o")], capture_output=True, text=True)
+    assert r.returncode == 0, r.stderr
+
+
+def test_selftest_rejects_bad_limits(L):
+    for bad in (0, -5, 1000001):
+        assert L.muir_selftest_expired_wait(bad, None) == 1  # MUIR_ERR_INVALID_ARG

@@ -89,3 +89,80 @@ def test_max_over_ranks_gloo_world2(tmp_path):
     assert all(x["world"] == 2 for x in res)
     assert all(x["worst"] == 15.0 for x in res)
     assert res[0]["seed"] != res[1]["seed"]
+
+
+def _rank_step_main(rank, world, port, out_dir):
+    """One rank of the bench's per-rank step logic on a CPU stand-in: its own
+    seeded batch, the oracle's chunked forward as the step, the bench's timing
+    protocol (warm-up, barrier, timed steps, barrier, max over ranks)."""
+    import time
+
+    import torch.distributed as dist
+    import oracle
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank),
+                      WORLD_SIZE=str(world), LOCAL_RANK=str(rank))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    r, w, _ = bench.dist_env()
+    T = 32
+    x = bench.rank_batch(r, B=1, H=1, T=T, dk=8, dv=8)
+    calls = []
+
+    def step():
+        calls.append(1)
+        oracle.chunk_fwd(*[x[n] for n in bench.NAMES], S0=x["S0"], chunk=8, threads=1)
+        if r == 1:
+            time.sleep(0.01)  # the slower rank sets the job time
+
+    own = {}
+
+    def timer():
+        t = {}
+
+        def start():
+            t["0"] = time.perf_counter()
+
+        def stop():
+            own["ms"] = (time.perf_counter() - t["0"]) * 1e3
+            return own["ms"]
+        return start, stop
+
+    ms = bench.timed_steps(step, 3, 2, w, timer, dist.barrier, device="cpu")
+    value = bench.job_tokens_per_s(ms, T, w)
+    with open(os.path.join(out_dir, f"step{rank}.json"), "w") as f:
+        json.dump({"ms": ms, "own_ms": own["ms"] / 3, "value": value, "calls": len(calls),
+                   "q0": float(x["q"].float().flatten()[0])}, f)
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_per_rank_step_gloo_world2(tmp_path):
+    port = _free_port()
+    mp.spawn(_rank_step_main, args=(2, port, str(tmp_path)), nprocs=2, join=True)
+    res = [json.load(open(tmp_path / f"step{r}.json")) for r in range(2)]
+    assert all(x["calls"] == 5 for x in res)          # 2 warm-up + 3 timed steps
+    assert res[0]["ms"] == res[1]["ms"]               # one job time: the max over ranks
+    assert res[0]["ms"] >= max(x["own_ms"] for x in res) - 1e-9
+    assert res[1]["own_ms"] >= 10.0                   # the slow rank's own time ...
+    assert res[0]["ms"] >= 10.0                       # ... is the job's
+    assert res[0]["value"] == pytest.approx(32 * 2 / (res[0]["ms"] / 1e3))
+    assert res[0]["q0"] != res[1]["q0"]               # each rank has its own batch
+
+
+def test_gpus_flag_spawns_one_rank_per_gpu(monkeypatch):
+    """bench.py --gpus N started as one process relaunches itself under
+    torch.distributed.run with N ranks on 127.0.0.1, forwarding its arguments."""
+    seen = {}
+
+    def fake_call(cmd):
+        seen["cmd"] = cmd
+        return 0
+
+    monkeypatch.delenv("WORLD_SIZE", raising=False)
+    monkeypatch.setattr(bench.subprocess, "call", fake_call)
+    assert bench.main(["--gpus", "4", "--steps", "3", "--warmup", "3"]) == 0
+    cmd = seen["cmd"]
+    assert cmd[1:3] == ["-m", "torch.distributed.run"]
+    assert "--nproc-per-node=4" in cmd and "--nnodes=1" in cmd
+    assert cmd[cmd.index("--master-addr") + 1] == "127.0.0.1"
+    assert cmd[-7].endswith("bench.py")
+    assert cmd[-6:] == ["--gpus", "4", "--steps", "3", "--warmup", "3"]
