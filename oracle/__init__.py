@@ -16,8 +16,10 @@ Two independent C sources are wrapped:
 
 and, in numpy below, the q/k feature prologue (SiLU, then unit L2 norm per
 token-head row; same page, "Methodology" and fig. 3(b)) with its gradient, the
-output gate o * sigmoid(z) with its gradient, and the fused layer composed of
-the three (``fwd_fused`` / ``bwd_fused``).
+output gate o * sigmoid(z) with its gradient, the fused layer composed of the
+three (``fwd_fused`` / ``bwd_fused``), and the fused low-rank gate projection
+(one latent per token, five up-projections with channel biases, eq:ours_proj)
+with its gradient.
 
 Every function takes numpy-convertible arrays, computes in float64 and returns
 float64 numpy arrays.  Per-token tensors are ``[B, T, H, d]``; states are
@@ -25,7 +27,8 @@ float64 numpy arrays.  Per-token tensors are ``[B, T, H, d]``; states are
 
 Pins (what fixes these functions other than themselves) live in
 ``tests/test_oracle_pins.py``, ``tests/test_qk_oracle.py`` (the prologue) and
-``tests/test_fused_oracle.py`` (output gate, fused composition):
+``tests/test_fused_oracle.py`` (output gate, fused composition),
+``tests/test_gate_oracle.py`` (gate projection):
 linear-attention and gated-linear-attention
 closed forms, the delta rule (Widrow-Hoff), an exact-retrieval invariant,
 pure decay, chunk-size invariance, linearity, column equivariance, state
@@ -260,3 +263,99 @@ def bwd_fused(q, k, v, g, e, w, gamma=None, S0=None, dO=None, dS_final=None, z_o
         out["dq"] = qk_prologue_bwd(q, out["dq"])
         out["dk"] = qk_prologue_bwd(k, out["dk"])
     return out
+
+
+# ------------------------------------------------------------ gate projection
+
+# The five gate families of the fused low-rank projection ("Methodology";
+# fig. 3(c): ranks (r_f, r_b, r_g, r_w, r_q) = (64, 64, 128, 128, 128), R_tot =
+# 512), in the order their latent columns are laid out, with what each yields:
+# f -> log decay g, b -> erase e, g -> the output gate's pre-activation z_out,
+# w -> write w, q -> readout gain gamma.
+GATE_FAMILIES = ("f", "b", "g", "w", "q")
+GATE_OUTPUT = {"f": "g", "b": "e", "g": "z_out", "w": "w", "q": "gamma"}
+
+
+def _sig(x):
+    return 1.0 / (1.0 + np.exp(-x))
+
+
+def _softplus(x):
+    return np.logaddexp(0.0, x)
+
+
+def _gate_act(fam, pre):
+    """g = -softplus(pre) (log decay, <= 0); e, w, gamma = sigmoid(pre); the
+    output gate's pre-activation passes through (its sigmoid is applied after
+    the mixer)."""
+    if fam == "f":
+        return -_softplus(pre)
+    if fam == "g":
+        return pre
+    return _sig(pre)
+
+
+def _gate_act_grad(fam, pre):
+    if fam == "f":
+        return -_sig(pre)
+    if fam == "g":
+        return np.ones_like(pre)
+    s = _sig(pre)
+    return s * (1.0 - s)
+
+
+def round_bf16(x):
+    """Round to bfloat16 the way the kernels store a float32 value: first to
+    float32 (the precision the kernels compute in), then to the nearest bf16,
+    ties to even.  Returns float64 holding the bf16 values."""
+    f = np.ascontiguousarray(np.asarray(x, dtype=np.float64).astype(np.float32))
+    u = f.view(np.uint32).astype(np.uint64)
+    r = (u + 0x7FFF + ((u >> 16) & 1)) & 0xFFFF0000
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def gate_pre(lat, ups, H):
+    """Pre-activations of the fused projection.  ``lat`` [B, T, R] is the
+    per-token latent (shared by all heads); ``ups`` maps a family to
+    ``(offset, U [r, H*d], bias [H*d])``: the family's latent columns are
+    ``offset .. offset + r``.  Returns ``{family: pre [B, T, H, d]}``."""
+    lat = _f64(lat)
+    B, T, _ = lat.shape
+    out = {}
+    for fam, (off, U, bias) in ups.items():
+        U, bias = _f64(U), _f64(bias)
+        r = U.shape[0]
+        pre = lat[:, :, off:off + r] @ U + bias
+        out[fam] = pre.reshape(B, T, H, -1)
+    return out
+
+
+def gate_projection(lat, ups, H, rounded=True):
+    """The gates the fused projection yields (``GATE_OUTPUT`` names), each
+    [B, T, H, d]: activation of ``gate_pre``, rounded to bf16 when
+    ``rounded`` (the gate dtype the kernels consume)."""
+    pre = gate_pre(lat, ups, H)
+    out = {}
+    for fam, p in pre.items():
+        a = _gate_act(fam, p)
+        out[GATE_OUTPUT[fam]] = round_bf16(a) if rounded else a
+    return out
+
+
+def gate_projection_bwd(lat, ups, H, dgates):
+    """Gradients of ``sum_X dgates[X] * gate_X`` through ``gate_projection``
+    (the bf16 rounding passes gradients unchanged): returns ``dlat`` [B, T, R]
+    and, per family, ``dU`` [r, H*d] and ``dbias`` [H*d]."""
+    lat = _f64(lat)
+    B, T, R = lat.shape
+    pre = gate_pre(lat, ups, H)
+    dlat = np.zeros_like(lat)
+    res = {"dlat": dlat}
+    for fam, (off, U, bias) in ups.items():
+        U = _f64(U)
+        r = U.shape[0]
+        dp = (_f64(dgates[GATE_OUTPUT[fam]]) * _gate_act_grad(fam, pre[fam])).reshape(B, T, -1)
+        dlat[:, :, off:off + r] += dp @ U.T
+        res["dU_" + fam] = np.einsum("bti,btn->in", lat[:, :, off:off + r], dp)
+        res["dbias_" + fam] = dp.sum(axis=(0, 1))
+    return res
