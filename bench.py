@@ -56,17 +56,26 @@ DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 6 * 128 * 2 + 128 * 2  # S read+writ
 
 # DRAM traffic per launch from ncu (dram__bytes_read.sum + dram__bytes_write.sum),
 # keyed by kernel; valid only while the chunk-kernel source hash matches.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    # ncu --set full of one k2_bwd2 launch at B=1 H=16 T=8192 (131,072 token-heads):
+    # 619.2 MB read + 168.4 MB written; traffic scales with the chunks processed
+    "k2_bwd2": {"bytes_per_token_head": (619.170304e6 + 168.362496e6) / 131072,
+                "source": "27ad89fbb9ea1c69"},
+}
+
+
+CHUNK_KERNEL_FILES = ("chunk", "fwd2.cu", "bwd2.cu")
 
 
 def source_hash(chunk_kernels_only: bool = False) -> str:
     """Hash of the library sources; with ``chunk_kernels_only`` of the files the
-    chunk kernels are compiled from (``chunk*.cu`` and every header), so that
-    counters taken on those kernels stay valid across changes elsewhere."""
+    chunk kernels are compiled from (``chunk*.cu``, ``fwd2.cu``, ``bwd2.cu`` and
+    every header), so that counters taken on those kernels stay valid across
+    changes elsewhere and are dropped when those kernels change."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "gated_delta_rule_115_b200", "csrc")
     for f in sorted(os.listdir(csrc)):
-        if chunk_kernels_only and not (f.startswith("chunk") or f.endswith((".cuh", ".h"))):
+        if chunk_kernels_only and not (f.startswith(CHUNK_KERNEL_FILES) or f.endswith((".cuh", ".h"))):
             continue
         with open(os.path.join(csrc, f), "rb") as fh:
             h.update(f.encode() + fh.read())

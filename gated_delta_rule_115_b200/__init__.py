@@ -48,8 +48,23 @@ class MuirShape(ctypes.Structure):
                 ("in_dtype", ctypes.c_int), ("out_dtype", ctypes.c_int)]
 
 
+class MuirGateFamily(ctypes.Structure):
+    _fields_ = [("off", ctypes.c_int), ("rank", ctypes.c_int), ("U", ctypes.c_void_p),
+                ("bias", ctypes.c_void_p)]
+
+
 class MuirFusion(ctypes.Structure):
-    _fields_ = [("z_out", ctypes.c_void_p), ("qk_raw", ctypes.c_int)]
+    _fields_ = [("z_out", ctypes.c_void_p), ("qk_raw", ctypes.c_int),
+                ("latent", ctypes.c_void_p), ("R", ctypes.c_int), ("fam", MuirGateFamily * 5)]
+
+
+class MuirFusionGrads(ctypes.Structure):
+    _fields_ = [("dlatent", ctypes.c_void_p), ("dU", ctypes.c_void_p * 5),
+                ("dbias", ctypes.c_void_p * 5)]
+
+
+# gate families of the fused projection, in the latent's column order
+GATE_FAMILIES = ("f", "b", "g", "w", "q")
 
 
 _lib = None
@@ -98,7 +113,7 @@ def lib():
         L.muir_chunk_fused_workspace.restype = S
         L.muir_chunk_fwd_fused.argtypes = [SP, FP] + [P] * 15 + [S, P]
         L.muir_chunk_fwd_fused.restype = I
-        L.muir_chunk_bwd_fused.argtypes = [SP, FP] + [P] * 24 + [S, P]
+        L.muir_chunk_bwd_fused.argtypes = [SP, FP] + [P] * 25 + [S, P]
         L.muir_chunk_bwd_fused.restype = I
         L.muir_chunk_fwd_noalloc.argtypes = [SP] + [P] * 10 + [P]
         L.muir_chunk_fwd_noalloc.restype = I
@@ -239,26 +254,41 @@ def chunk_bwd(q, k, v, g, e, w, gamma, S0, dO, dS_final=None, chunk=64, S_chunks
     return grads
 
 
-def _fusion(z_out, qk_raw):
-    return MuirFusion(None if z_out is None else _ptr(z_out).value, int(bool(qk_raw)))
+def _fusion(z_out, qk_raw, latent=None, proj=None):
+    """``proj`` maps a family name (``GATE_FAMILIES``) to ``(offset, U, bias)``:
+    U [rank, H*dk] bf16, bias [H*dk] float32."""
+    f = MuirFusion()
+    f.z_out = None if z_out is None else _ptr(z_out).value
+    f.qk_raw = int(bool(qk_raw))
+    if latent is not None:
+        f.latent = _ptr(latent).value
+        f.R = latent.shape[-1]
+        for name, (off, U, bias) in (proj or {}).items():
+            fam = f.fam[GATE_FAMILIES.index(name)]
+            fam.off, fam.rank = int(off), U.shape[0]
+            fam.U, fam.bias = _ptr(U).value, _ptr(bias).value
+    return f
 
 
 def chunk_fwd_fused(q, k, v, g, e, w, gamma, S0=None, z_out=None, qk_raw=False, chunk=128,
-                    out_dtype=None, save=True, ws=None):
+                    out_dtype=None, save=True, ws=None, latent=None, proj=None):
     """Forward with the fused stages (``muir_chunk_fwd_fused``): ``qk_raw``
     means q and k are the raw pre-activations (SiLU and the unit L2 norm are
     applied in the kernels); ``z_out`` is the output gate's pre-activation
-    (the output is ``o * sigmoid(z_out)``).  Returns ``(o, S_final, saved)``;
+    (the output is ``o * sigmoid(z_out)``); ``latent`` [B, T, R] with ``proj``
+    (family -> (offset, U, bias)) projects those families' gates from the
+    latent (their tensor arguments may be None).  Returns ``(o, S_final, saved)``;
     ``saved`` (None unless ``save``) holds what :func:`chunk_bwd_fused` reuses:
     ``S_chunks``, ``M_chunks``, ``aux`` and, with a gate, ``o_pre``."""
     L = lib()
     B, T, H, dk = q.shape
     dv = v.shape[-1]
     shp = _shape(q, v, chunk, out_dtype)
-    fu = _fusion(z_out, qk_raw)
+    fu = _fusion(z_out, qk_raw, latent, proj)
     od = torch.bfloat16 if shp.out_dtype == MUIR_BF16 else torch.float32
     o = torch.empty(B, T, H, dv, dtype=od, device=q.device)
-    o_pre = torch.empty_like(o) if z_out is not None else None
+    gated = z_out is not None or (proj is not None and "g" in proj)
+    o_pre = torch.empty_like(o) if gated else None
     S_final = torch.empty(B, H, dk, dv, dtype=torch.float32, device=q.device)
     Sc = Mc = aux = None
     if save:
@@ -281,7 +311,7 @@ def chunk_fwd_fused(q, k, v, g, e, w, gamma, S0=None, z_out=None, qk_raw=False, 
 
 
 def chunk_bwd_fused(q, k, v, g, e, w, gamma, S0, dO, dS_final=None, z_out=None, qk_raw=False,
-                    o_pre=None, saved=None, chunk=128, ws=None):
+                    o_pre=None, saved=None, chunk=128, ws=None, latent=None, proj=None):
     """Gradients through :func:`chunk_fwd_fused` (``muir_chunk_bwd_fused``):
     ``dO`` is the gradient of the (gated) output.  Returns the dict of
     :func:`chunk_bwd` plus ``dz_out`` with a gate; dq and dk are with respect
@@ -293,12 +323,23 @@ def chunk_bwd_fused(q, k, v, g, e, w, gamma, S0, dO, dS_final=None, z_out=None, 
         o_pre = saved.get("o_pre")
     if o_pre is not None:
         shp.out_dtype = MUIR_BF16 if o_pre.dtype == torch.bfloat16 else MUIR_FP32
-    fu = _fusion(z_out, qk_raw)
-    grads = {n: torch.empty_like(x) for n, x in
+    fu = _fusion(z_out, qk_raw, latent, proj)
+    grads = {n: (torch.empty_like(x) if x is not None else None) for n, x in
              dict(dq=q, dk=k, dv=v, dg=g, de=e, dw=w, dgamma=gamma).items()}
     B, T, H, dk = q.shape
     grads["dS0"] = torch.empty(B, H, dk, v.shape[-1], dtype=torch.float32, device=q.device)
     dz = torch.empty_like(z_out) if z_out is not None else None
+    fg = None
+    if latent is not None:
+        fg = MuirFusionGrads()
+        grads["dlatent"] = torch.empty_like(latent)
+        fg.dlatent = _ptr(grads["dlatent"]).value
+        for name, (off, U, bias) in proj.items():
+            i = GATE_FAMILIES.index(name)
+            grads["dU_" + name] = torch.empty(U.shape, dtype=torch.float32, device=q.device)
+            grads["dbias_" + name] = torch.empty(bias.shape, dtype=torch.float32, device=q.device)
+            fg.dU[i] = _ptr(grads["dU_" + name]).value
+            fg.dbias[i] = _ptr(grads["dbias_" + name]).value
     Sc, Mc, aux = ((saved["S_chunks"], saved["M_chunks"], saved["aux"]) if saved is not None
                    else (None, None, None))
     need = int(L.muir_chunk_fused_workspace(ctypes.byref(shp), ctypes.byref(fu), 1))
@@ -310,9 +351,13 @@ def chunk_bwd_fused(q, k, v, g, e, w, gamma, S0, dO, dS_final=None, z_out=None, 
                                 _ptr(Mc), _ptr(aux), _ptr(o_pre), _ptr(dO), _ptr(dS_final),
                                 *[_ptr(grads[n]) for n in ("dq", "dk", "dv", "dg", "de", "dw",
                                                            "dgamma")],
-                                _ptr(dz), _ptr(grads["dS0"]), _ptr(wsb),
+                                _ptr(dz), _ptr(grads["dS0"]),
+                                ctypes.byref(fg) if fg is not None else None, _ptr(wsb),
                                 ctypes.c_size_t(wsb.numel()), _stream(q.device))
     _check("muir_chunk_bwd_fused", rc)
+    for n in ("dg", "de", "dw", "dgamma"):
+        if grads[n] is None:
+            del grads[n]
     if dz is not None:
         grads["dz_out"] = dz
     return grads

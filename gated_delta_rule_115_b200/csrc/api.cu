@@ -7,6 +7,7 @@
 #include "chunk_units.h"
 #include "bwd2.h"
 #include "fwd2.h"
+#include "gates.h"
 #include "kernels.h"
 
 namespace {
@@ -125,7 +126,7 @@ muir_status muir_device_wait_status(void) {
     const unsigned int n = muir::timeouts_bf16_d128() + muir::timeouts_bf16_d64() +
                            muir::timeouts_f32_d128() + muir::timeouts_f32_d64() +
                            muir::v2::timeouts_v2() + muir::v2::timeouts_bwd2() +
-                           muir::timeouts_selftest();
+                           muir::timeouts_selftest() + muir::v2::timeouts_gates();
     return n ? MUIR_ERR_DEVICE_TIMEOUT : MUIR_OK;
 }
 
@@ -338,7 +339,9 @@ muir_status muir_qk_prologue_bwd(long long rows, int d, muir_dtype dtype, const 
 
 namespace {
 
-bool fused_any(const muir_fusion* f) { return f && (f->z_out || f->qk_raw); }
+bool fused_any(const muir_fusion* f) { return f && (f->z_out || f->qk_raw || f->latent); }
+
+int projected(const muir_fusion* f, int X) { return f && f->latent && f->fam[X].rank > 0; }
 
 // The fused stages run inside the on-chip kernels: bf16 inputs, dk = dv = 128,
 // chunk 128, T a multiple of 128.
@@ -346,25 +349,96 @@ muir_status check_fusion(const muir_shape* s, const muir_fusion* f) {
     if (!f) return MUIR_ERR_INVALID_ARG;
     if (f->qk_raw != 0 && f->qk_raw != 1) return MUIR_ERR_INVALID_ARG;
     if (!ok_opt(f->z_out)) return MUIR_ERR_INVALID_ARG;
+    if (f->latent) {
+        if (!ok_ptr(f->latent) || f->R <= 0 || f->R % 8) return MUIR_ERR_INVALID_ARG;
+        int n = 0;
+        for (int X = 0; X < 5; ++X) {
+            const muir_gate_family& a = f->fam[X];
+            if (a.rank == 0) continue;
+            if (a.rank != 64 && a.rank != 128) return MUIR_ERR_UNSUPPORTED;
+            if (a.off < 0 || a.off % 8 || a.off + a.rank > f->R) return MUIR_ERR_INVALID_ARG;
+            if (!ok_ptr(a.U) || !ok_ptr(a.bias)) return MUIR_ERR_INVALID_ARG;
+            for (int Y = 0; Y < X; ++Y) {  // latent columns of two families must not overlap
+                const muir_gate_family& b = f->fam[Y];
+                if (b.rank > 0 && a.off < b.off + b.rank && b.off < a.off + a.rank)
+                    return MUIR_ERR_INVALID_ARG;
+            }
+            ++n;
+        }
+        if (n == 0) return MUIR_ERR_INVALID_ARG;
+        if (projected(f, MUIR_FAM_OUTGATE) && f->z_out) return MUIR_ERR_INVALID_ARG;
+    }
     if (fused_any(f) && !muir::v2::fwd2_supported(s->B, s->T, s->H, s->dk, s->chunk,
                                                   s->in_dtype == MUIR_BF16))
         return MUIR_ERR_UNSUPPORTED;
     return MUIR_OK;
 }
 
-size_t fused_ws(const muir_shape* s, const muir_fusion* f, bool backward) {
-    const size_t base = backward
+size_t base_ws(const muir_shape* s, bool backward) {
+    return backward
         ? muir::chunk_bwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false, s->in_dtype == MUIR_BF16)
         : muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false, s->in_dtype == MUIR_BF16);
+}
+
+// Per projected family: its gate, and in the backward the gate's gradient and
+// dpre (a bf16 hi / lo pair).
+size_t gate_buf_bytes(const muir_shape* s) { return (size_t)s->B * s->T * s->H * s->dk * 2; }
+
+size_t fused_ws(const muir_shape* s, const muir_fusion* f, bool backward) {
+    const size_t base = base_ws(s, backward);
     if (!fused_any(f)) return base;
-    return ((base + 255) & ~(size_t)255) + muir::fused_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk);
+    size_t extra = muir::fused_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk);
+    if (f->latent) extra += 5 * (backward ? 4 : 1) * gate_buf_bytes(s);
+    return ((base + 255) & ~(size_t)255) + extra;
 }
 
 char* fused_region(const muir_shape* s, void* ws, bool backward) {
-    const size_t base = backward
-        ? muir::chunk_bwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false, s->in_dtype == MUIR_BF16)
-        : muir::chunk_fwd_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, false, s->in_dtype == MUIR_BF16);
-    return static_cast<char*>(ws) + ((base + 255) & ~(size_t)255);
+    return static_cast<char*>(ws) + ((base_ws(s, backward) + 255) & ~(size_t)255);
+}
+
+// The gate projection's launch description; the projected gates (and in the
+// backward their gradients and dpre) live in the workspace after the stages'
+// own region.  Replaces the tensor arguments of projected families in P.
+void setup_projection(const muir_shape* s, const muir_fusion* f, char* fw, bool backward,
+                      muir::v2::GatesArgs& ga, muir::ChunkProblem& P, void** dgate_ptrs,
+                      const muir_fusion_grads* fg) {
+    static const int act[5] = {muir::v2::kActNegSoftplus, muir::v2::kActSigmoid,
+                               muir::v2::kActIdentity, muir::v2::kActSigmoid,
+                               muir::v2::kActSigmoid};
+    const size_t gb = gate_buf_bytes(s);
+    char* buf = fw + muir::fused_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk);
+    ga = muir::v2::GatesArgs{};
+    ga.latent = f->latent;
+    ga.R = f->R;
+    ga.H = s->H;
+    ga.rows = (long long)s->B * s->T;
+    ga.dlatent = fg ? fg->dlatent : nullptr;
+    for (int X = 0; X < 5; ++X) {
+        if (!projected(f, X)) continue;
+        muir::v2::GateFamily& g = ga.fam[ga.nfam++];
+        g.off = f->fam[X].off;
+        g.r = f->fam[X].rank;
+        g.act = act[X];
+        g.U = f->fam[X].U;
+        g.bias = f->fam[X].bias;
+        g.out = buf + (size_t)X * gb;
+        if (backward) {
+            g.dout = buf + (size_t)(5 + X) * gb;
+            g.dpre = buf + (size_t)(10 + X) * gb;
+            g.dpre_lo = buf + (size_t)(15 + X) * gb;
+            g.dU = fg->dU[X];
+            g.dbias = fg->dbias[X];
+            dgate_ptrs[X] = const_cast<void*>(g.dout);
+        }
+        switch (X) {
+            case MUIR_FAM_DECAY: P.g = g.out; break;
+            case MUIR_FAM_ERASE: P.e = g.out; break;
+            case MUIR_FAM_OUTGATE: P.zo = g.out; break;
+            case MUIR_FAM_WRITE: P.w = g.out; break;
+            default: P.gamma = g.out; break;
+        }
+    }
+    P.gate_proj = &ga;
 }
 
 }  // namespace
@@ -382,20 +456,27 @@ muir_status muir_chunk_fwd_fused(const muir_shape* s, const muir_fusion* f, cons
     muir_status st = check_shape(s);
     if (st != MUIR_OK) return st;
     if ((st = check_fusion(s, f)) != MUIR_OK) return st;
-    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
-        !ok_ptr(gamma) || !ok_ptr(o) || !ok_opt(o_pre) || !ok_opt(S0) || !ok_opt(S_final) ||
-        !ok_opt(S_chunks) || !ok_opt(M_chunks) || !ok_opt(aux) || (o_pre && !f->z_out))
+    const bool gate = f->z_out || projected(f, MUIR_FAM_OUTGATE);
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(o) || !ok_opt(o_pre) || !ok_opt(S0) ||
+        !ok_opt(S_final) || !ok_opt(S_chunks) || !ok_opt(M_chunks) || !ok_opt(aux) ||
+        (o_pre && !gate))
+        return MUIR_ERR_INVALID_ARG;
+    if ((!projected(f, MUIR_FAM_DECAY) && !ok_ptr(g)) || (!projected(f, MUIR_FAM_ERASE) && !ok_ptr(e)) ||
+        (!projected(f, MUIR_FAM_WRITE) && !ok_ptr(w)) ||
+        (!projected(f, MUIR_FAM_READOUT) && !ok_ptr(gamma)))
         return MUIR_ERR_INVALID_ARG;
     const size_t need = fused_ws(s, f, false);
     if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
     if ((st = check_device()) != MUIR_OK) return st;
     muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);
     P.aux = aux;
+    muir::v2::GatesArgs ga;
     if (fused_any(f)) {
         P.zo = f->z_out;
         P.o_pre = o_pre;
         P.qk_raw = f->qk_raw;
         P.fused_ws = fused_region(s, ws, false);
+        if (f->latent) setup_projection(s, f, P.fused_ws, false, ga, P, nullptr, nullptr);
     }
     return from_cuda(muir::run_chunk_fwd(P, S0, o, S_final, S_chunks, M_chunks, ws, ws_bytes,
                                          static_cast<cudaStream_t>(stream)));
@@ -407,23 +488,38 @@ muir_status muir_chunk_bwd_fused(const muir_shape* s, const muir_fusion* f, cons
                                  const float* S_chunks, const float* M_chunks, const float* aux,
                                  const void* o_pre, const void* dO, const float* dS_final,
                                  void* dq, void* dk, void* dv, void* dg, void* de, void* dw,
-                                 void* dgamma, void* dz_out, float* dS0, void* ws, size_t ws_bytes,
+                                 void* dgamma, void* dz_out, float* dS0,
+                                 const muir_fusion_grads* fg, void* ws, size_t ws_bytes,
                                  void* stream) {
     muir_status st = check_shape(s);
     if (st != MUIR_OK) return st;
     if ((st = check_fusion(s, f)) != MUIR_OK) return st;
-    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(g) || !ok_ptr(e) || !ok_ptr(w) ||
-        !ok_ptr(gamma) || !ok_ptr(dO) || !ok_ptr(dq) || !ok_ptr(dk) || !ok_ptr(dv) ||
-        !ok_ptr(dg) || !ok_ptr(de) || !ok_ptr(dw) || !ok_ptr(dgamma) || !ok_opt(S0) ||
-        !ok_opt(S_chunks) || !ok_opt(M_chunks) || !ok_opt(dS_final) || !ok_opt(dS0) ||
-        !ok_opt(aux) || (aux && !S_chunks) || !ok_opt(o_pre) || !ok_opt(dz_out))
+    const bool gate = f->z_out || projected(f, MUIR_FAM_OUTGATE);
+    if (!ok_ptr(q) || !ok_ptr(k) || !ok_ptr(v) || !ok_ptr(dO) || !ok_ptr(dq) || !ok_ptr(dk) ||
+        !ok_ptr(dv) || !ok_opt(S0) || !ok_opt(S_chunks) || !ok_opt(M_chunks) ||
+        !ok_opt(dS_final) || !ok_opt(dS0) || !ok_opt(aux) || (aux && !S_chunks) ||
+        !ok_opt(o_pre) || !ok_opt(dz_out))
         return MUIR_ERR_INVALID_ARG;
-    if (f->z_out && (!o_pre || !dz_out)) return MUIR_ERR_INVALID_ARG;
+    const void* gin[5] = {g, e, nullptr, w, gamma};
+    void* gout[5] = {dg, de, dz_out, dw, dgamma};
+    for (int X = 0; X < 5; ++X) {
+        if (X == MUIR_FAM_OUTGATE || projected(f, X)) continue;
+        if (!ok_ptr(gin[X]) || !ok_ptr(gout[X])) return MUIR_ERR_INVALID_ARG;
+    }
+    if (gate && !o_pre) return MUIR_ERR_INVALID_ARG;
+    if (f->z_out && !dz_out) return MUIR_ERR_INVALID_ARG;
+    if (f->latent) {
+        if (!fg || !ok_ptr(fg->dlatent)) return MUIR_ERR_INVALID_ARG;
+        for (int X = 0; X < 5; ++X)
+            if (projected(f, X) && (!ok_ptr(fg->dU[X]) || !ok_ptr(fg->dbias[X])))
+                return MUIR_ERR_INVALID_ARG;
+    }
     const size_t need = fused_ws(s, f, true);
     if (ws_bytes < need || (need > 0 && !ok_ptr(ws))) return MUIR_ERR_WORKSPACE;
     if ((st = check_device()) != MUIR_OK) return st;
     muir::ChunkProblem P = make_problem(s, q, k, v, g, e, w, gamma);
     P.aux = const_cast<float*>(aux);
+    muir::v2::GatesArgs ga;
     if (fused_any(f)) {
         P.zo = f->z_out;
         P.o_pre = const_cast<void*>(o_pre);
@@ -431,10 +527,15 @@ muir_status muir_chunk_bwd_fused(const muir_shape* s, const muir_fusion* f, cons
         P.dzo = dz_out;
         P.qk_raw = f->qk_raw;
         P.fused_ws = fused_region(s, ws, true);
+        if (f->latent) {
+            setup_projection(s, f, P.fused_ws, true, ga, P, gout, fg);
+            P.dzo = gout[MUIR_FAM_OUTGATE];
+        }
     }
-    return from_cuda(muir::run_chunk_bwd(P, S0, S_chunks, M_chunks, dO, dS_final, dq, dk, dv, dg,
-                                         de, dw, dgamma, dS0, ws, ws_bytes,
-                                         static_cast<cudaStream_t>(stream)));
+    return from_cuda(muir::run_chunk_bwd(P, S0, S_chunks, M_chunks, dO, dS_final, dq, dk, dv,
+                                         gout[MUIR_FAM_DECAY], gout[MUIR_FAM_ERASE],
+                                         gout[MUIR_FAM_WRITE], gout[MUIR_FAM_READOUT], dS0, ws,
+                                         ws_bytes, static_cast<cudaStream_t>(stream)));
 }
 
 muir_status muir_selftest_expired_wait(int limit_us, void* stream) {

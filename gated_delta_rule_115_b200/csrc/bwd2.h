@@ -86,6 +86,7 @@ unsigned int timeouts_bwd2();
 // Tensor maps shared with fwd2.cu.
 bool map_tokens16(CUtensorMap* m, const void* base, int B, int T, int H);
 bool map_rows32f(CUtensorMap* m, const float* base, long long rows);
+bool map_2d16(CUtensorMap* m, const void* base, long long cols, long long rows, int box_rows);
 
 }  // namespace v2
 }  // namespace muir

@@ -5,6 +5,7 @@
 #include "chunk_units.h"
 #include "bwd2.h"
 #include "fwd2.h"
+#include "gates.h"
 
 namespace muir {
 
@@ -107,7 +108,10 @@ cudaError_t run_chunk_fwd(const ChunkProblem& P, const float* S0, void* o, float
         if (P.qk_raw)
             a.rnorm = P.aux ? v2::aux_rn(reinterpret_cast<unsigned char*>(P.aux), nch, (size_t)P.B * P.H)
                             : reinterpret_cast<float*>(fw + 256);
-        cudaError_t e = cudaMemsetAsync(flags, 0, 16, st);
+        cudaError_t e = cudaSuccess;
+        if (P.gate_proj)  // projected gates first: everything below reads them
+            e = v2::run_gates_fwd(*static_cast<const v2::GatesArgs*>(P.gate_proj), st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(flags, 0, 16, st);
         if (e == cudaSuccess) e = v2::span_check(P.g, P.B, P.T, P.H, flags, st);
         if (e == cudaSuccess) e = v2::run_fwd2(a, st);
         if (e != cudaSuccess) return e;
@@ -141,7 +145,10 @@ cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S
         char* shared = static_cast<char*>(ws) + 256;
         const size_t blk = (size_t)128 * 128;
         const size_t nch = (size_t)P.B * P.H * P.N;
-        cudaError_t e = cudaMemsetAsync(flags, 0, 16, st);
+        cudaError_t e = cudaSuccess;
+        if (P.gate_proj)  // the forward's projected gates, recomputed
+            e = v2::run_gates_fwd(*static_cast<const v2::GatesArgs*>(P.gate_proj), st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(flags, 0, 16, st);
         if (e == cudaSuccess) e = v2::span_check(P.g, P.B, P.T, P.H, flags, st);
         if (e != cudaSuccess) return e;
         v2::Bwd2Args b = {};
@@ -206,6 +213,8 @@ cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S
             if ((e = qk_jacobian_gated(flags, P.q, dq, rows, st)) != cudaSuccess) return e;
             if ((e = qk_jacobian_gated(flags, P.k, dk, rows, st)) != cudaSuccess) return e;
         }
+        if (P.gate_proj)  // the projected gates' gradients -> latent, U, bias
+            return v2::run_gates_bwd(*static_cast<const v2::GatesArgs*>(P.gate_proj), st);
         return cudaSuccess;
     }
 #define MUIR_BWD_ARGS P, S0, S_chunks, M_chunks, dO, dS_final, dq, dk, dv, dg, de, dw, dgamma, dS0, ws, st

@@ -14,7 +14,7 @@
 //   Kp = k 2^(L-P), Km = k 2^(P-L), Am = a 2^(P-L), Qp = q^ 2^(L-P)
 //   L_A = strict(Kp Am^T), L_K = strict(Kp Km^T)           (bf16 operands)
 //   M_QK = incl(Qp Km^T)  (bf16 hi/lo split: hi hi + hi lo + lo hi)
-//   M_QA = incl(Qp Am^T)                                     (bf16 operands)
+//   M_QA = incl(Qp Am^T)                      (Qp as bf16 hi + lo, Am bf16)
 //   T = (I + L_A)^-1: 32x32 diagonal blocks by forward substitution (fp32),
 //       then block merges T21 = -T22 (L21 T11) for 32 -> 64 -> 128 on tcgen05
 //   X = [W | U'] = T [K~ | L_K U]   (K~ = k 2^L; one N = 256 MMA chain)
@@ -368,7 +368,8 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             gemm_kk16(tm + 256, a3, 0, a1, 0, 0, 128, 128, kBF16, false);  // M_QK: hi hi
             gemm_kk16(tm + 256, a3, 0, a2, 0, 0, 128, 128, kBF16, true);   //       hi lo
             gemm_kk16(tm + 256, a4, 0, a1, 0, 0, 128, 128, kBF16, true);   //       lo hi
-            gemm_kk16(tm + 384, a3, 0, a5, 0, 0, 128, 128, kBF16, false);  // M_QA
+            gemm_kk16(tm + 384, a3, 0, a5, 0, 0, 128, 128, kBF16, false);  // M_QA: hi Am
+            gemm_kk16(tm + 384, a4, 0, a5, 0, 0, 128, 128, kBF16, true);   //       lo Am
             mma_commit(&s.bar[BM2]);
         }
 
@@ -899,6 +900,20 @@ bool map_tokens16(CUtensorMap* m, const void* base, int B, int T, int H) {
     cuuint64_t dims[3] = {(cuuint64_t)kD, (cuuint64_t)H, (cuuint64_t)B * T};
     cuuint64_t strides[2] = {(cuuint64_t)kD * 2, (cuuint64_t)H * kD * 2};
     cuuint32_t box[3] = {64, 1, (cuuint32_t)kC};
+    cuuint32_t es[3] = {1, 1, 1};
+    return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
+               CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+               CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Map over a row-major [rows][cols] bf16 matrix: box of 64 columns x box_rows rows
+// (cols a multiple of 8, so that every row starts 16-byte aligned).
+bool map_2d16(CUtensorMap* m, const void* base, long long cols, long long rows, int box_rows) {
+    EncodeTiledFn enc = encode_fn();
+    if (!enc || cols % 8 || box_rows < 1 || box_rows > 256) return false;
+    cuuint64_t dims[3] = {(cuuint64_t)cols, (cuuint64_t)rows, 1};
+    cuuint64_t strides[2] = {(cuuint64_t)cols * 2, (cuuint64_t)cols * rows * 2};
+    cuuint32_t box[3] = {64, (cuuint32_t)box_rows, 1};
     cuuint32_t es[3] = {1, 1, 1};
     return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, es,
                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,

@@ -30,6 +30,7 @@ struct ChunkProblem {
     void* dzo = nullptr;        // backward: gradient of zo (bf16)
     int qk_raw = 0;             // q, k hold raw x; SiLU and the unit L2 norm are fused
     char* fused_ws = nullptr;   // fused_ws_bytes() of workspace for the stages above
+    const void* gate_proj = nullptr;  // v2::GatesArgs: gates projected from a latent (gates.cu)
 };
 
 // Workspace the fused stages add (inverse row norms, materialised q^ / k^ and

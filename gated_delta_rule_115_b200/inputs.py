@@ -195,3 +195,30 @@ def fused_inputs(wid: int, *, seed=None, **over):
     x["xk"] = _randn(gen, B, T, H, dk).to(td).contiguous()
     x["z_out"] = _randn(gen, B, T, H, dv).to(td).contiguous()
     return x
+
+
+GATE_RANKS = {"f": 64, "b": 64, "g": 128, "w": 128, "q": 128}  # (r_f, r_b, r_g, r_w, r_q)
+
+
+def gate_latent_inputs(B: int, T: int, H: int, d: int = 128, *, seed=None, dtype="bf16",
+                       families=("f", "b", "g", "w", "q"), bias_f=-1.5):
+    """Parameters of the fused gate projection: a per-token latent
+    ``[B, T, R]`` ~ N(0,1) (R = 512, families laid out in the order f, b, g, w,
+    q with ranks 64, 64, 128, 128, 128), per family an up-projection
+    ``U [r, H*d]`` ~ N(0, 1/r) (so pre-activations are ~N(0,1)) and a channel
+    bias ~ N(0, 0.25) in float32 (the decay family's centred at ``bias_f``, so
+    the log decays stay moderate).  Returns ``(latent, {family: (offset, U,
+    bias)})`` as CPU tensors."""
+    gen = torch.Generator("cpu").manual_seed(7000 if seed is None else seed)
+    td = TORCH_DTYPE[dtype]
+    R = sum(GATE_RANKS.values())
+    lat = _randn(gen, B, T, R).to(td).contiguous()
+    proj, off = {}, 0
+    for fam in ("f", "b", "g", "w", "q"):
+        r = GATE_RANKS[fam]
+        U = (_randn(gen, r, H * d) / math.sqrt(r)).to(td).contiguous()
+        bias = _randn(gen, H * d) * 0.5 + (bias_f if fam == "f" else 0.0)
+        if fam in families:
+            proj[fam] = (off, U, bias.contiguous())
+        off += r
+    return lat, proj

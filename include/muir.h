@@ -233,9 +233,41 @@ muir_status muir_chunk_fwd_noalloc(const muir_shape* shape, const void* q, const
  * muir_chunk_bwd.
  */
 typedef struct {
+    int off;            /* first latent column of the family (multiple of 8) */
+    int rank;           /* 0 = the family is not projected; else 64 or 128 */
+    const void* U;      /* [rank][H*dk] in_dtype: the family's up-projection */
+    const float* bias;  /* [H*dk] float32: its channel biases */
+} muir_gate_family;
+
+/* Families of the fused gate projection, in the pages' order (fig. 3(c)). */
+enum { MUIR_FAM_DECAY = 0, MUIR_FAM_ERASE = 1, MUIR_FAM_OUTGATE = 2, MUIR_FAM_WRITE = 3,
+       MUIR_FAM_READOUT = 4 };
+
+typedef struct {
     const void* z_out;
     int qk_raw;
+    /* Fused low-rank gate projection (same page, "Methodology", eq:ours_proj):
+     * latent [B][T][R] in_dtype, one row per token shared by every head, or
+     * NULL.  A family with rank > 0 takes its gate from
+     *   pre[t][h][c] = sum_i latent[t][off + i] U[i][h*dk + c] + bias[h*dk + c]
+     * instead of the tensor argument (which may then be NULL): log decay
+     * g = -softplus(pre), erase e, write w and readout gain gamma = sigmoid(pre),
+     * and the output gate's pre-activation z_out = pre (then fusion.z_out must
+     * be NULL).  The gates are formed on the tensor cores in float32 and kept
+     * in bf16, like gate inputs.  Families' latent columns must not overlap;
+     * R is a multiple of 8. */
+    const void* latent;
+    int R;
+    muir_gate_family fam[5];
 } muir_fusion;
+
+/* Gradients of the projection's parameters, written by muir_chunk_bwd_fused
+ * when fusion.latent is set (NULL otherwise). */
+typedef struct {
+    void* dlatent;      /* [B][T][R] in_dtype (columns of no family: 0) */
+    float* dU[5];       /* per projected family: [rank][H*dk] float32 */
+    float* dbias[5];    /* per projected family: [H*dk] float32 */
+} muir_fusion_grads;
 
 /* Workspace bytes of muir_chunk_fwd_fused (backward == 0) or
  * muir_chunk_bwd_fused (backward != 0); 0 for an invalid shape or fusion.
@@ -252,7 +284,9 @@ size_t muir_chunk_fused_workspace(const muir_shape* shape, const muir_fusion* fu
  *            of q^ and k^ for the backward
  * A large decay span (a chunk whose channel log-decay total exceeds the single
  * pivot) runs the boundary-pivot path on q^, k^ materialised in the workspace
- * (bf16) and gates its output afterwards.
+ * (bf16) and gates its output afterwards.  With a latent, the projected gates
+ * are formed in the workspace by a tensor-core pre-pass before the chunk
+ * kernels read them.
  */
 muir_status muir_chunk_fwd_fused(const muir_shape* shape, const muir_fusion* fusion,
                                  const void* q, const void* k, const void* v, const void* g,
@@ -271,7 +305,10 @@ muir_status muir_chunk_fwd_fused(const muir_shape* shape, const muir_fusion* fus
  *   aux    : as muir_chunk_bwd; with qk_raw it must come from a forward called
  *            with qk_raw
  * dq, dk are gradients with respect to the raw x_q, x_k when qk_raw is set.
- * Missing o_pre / dz_out with z_out is MUIR_ERR_INVALID_ARG.
+ * Missing o_pre / dz_out with z_out is MUIR_ERR_INVALID_ARG.  With a latent,
+ * the gradients of projected families go to fgrads (required) and their
+ * dg / de / dw / dgamma / dz_out arguments may be NULL; the forward's gates
+ * are recomputed from the latent.
  */
 muir_status muir_chunk_bwd_fused(const muir_shape* shape, const muir_fusion* fusion,
                                  const void* q, const void* k, const void* v, const void* g,
@@ -280,7 +317,8 @@ muir_status muir_chunk_bwd_fused(const muir_shape* shape, const muir_fusion* fus
                                  const float* aux, const void* o_pre, const void* dO,
                                  const float* dS_final, void* dq, void* dk, void* dv, void* dg,
                                  void* de, void* dw, void* dgamma, void* dz_out, float* dS0,
-                                 void* ws, size_t ws_bytes, void* stream);
+                                 const muir_fusion_grads* fgrads, void* ws, size_t ws_bytes,
+                                 void* stream);
 
 /*
  * One decode token for every (b, h) against a resident float32 state (same
