@@ -217,8 +217,8 @@ muir_status muir_chunk_fwd_noalloc(const muir_shape* shape, const void* q, const
 /*
  * Stages fused around the recurrence ("Muir", wolonglab.org page,
  * "Methodology" and fig. 3(b)): the block's q/k pathways end in SiLU with a
- * unit-normalised key, and a rank-128 gate g_t (the output gate, tab:abl
- * caption "wider output-gate") multiplies the mixer's output.
+ * unit-normalised key, and a rank-128 gate g_t (the output gate; the tab:abl
+ * caption compares against a widened one) multiplies the mixer's output.
  *
  *   z_out  : output-gate pre-activation [B][T][H][dv] in_dtype, or NULL (no
  *            gate).  The forward writes o * sigmoid(z_out); the backward takes

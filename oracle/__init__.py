@@ -216,9 +216,9 @@ def qk_prologue_bwd(x, dy):
 def out_gate(o, z):
     """Output gate applied after the mixer: ``o * sigmoid(z)``, elementwise, in
     float64.  The pages name a rank-128 gate g_t among the five gate families
-    ("Methodology", fig. 3(b)-(c): ranks (r_f, r_b, r_g, r_w, r_q)) and call it
-    the output gate (tab:abl caption, "wider output-gate"); z is its
-    pre-activation per token, head and value channel, produced upstream."""
+    ("Methodology", fig. 3(b)-(c): ranks (r_f, r_b, r_g, r_w, r_q)); the tab:abl
+    caption compares against a widened output gate, which identifies g_t as the
+    output gate.  z is its pre-activation per token, head and value channel."""
     o, z = _f64(o), _f64(z)
     return o / (1.0 + np.exp(-z))
 
