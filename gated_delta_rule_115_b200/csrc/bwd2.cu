@@ -54,6 +54,7 @@ namespace {
 constexpr int kC = 128, kD = 128;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLogDecayMin = -20.f;
+constexpr float kSpanMax = 140.f;  // single-pivot limit of |sum g| over a chunk (natural log)
 constexpr uint32_t kT32Half = 64 * 128 * 4;  // T32 tile of 64 rows
 
 __device__ __forceinline__ float ex2(float x) {
@@ -841,7 +842,13 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             const int r0 = 16 * g4;            // their rows in the half tiles
             float L[16];
             log_decay<16>(reinterpret_cast<const __nv_bfloat16*>(p.g) + tok * kD, lane, q, j0, s.tot, L);
-            if (q == 0 && lane < 16) s.P2[j0 + lane] = 0.5f * chunk_total(s.tot, j0 + lane);
+            if (q == 0 && lane < 16) {
+                const float lb = chunk_total(s.tot, j0 + lane);
+                s.P2[j0 + lane] = 0.5f * lb;
+                // (the forward's test, on the same sums: the call then also runs the
+                // boundary-pivot path, which overwrites this kernel's results)
+                if (lb < -kSpanMax * kLog2e) atomicOr(p.flags, 1);
+            }
             __syncthreads();
             const __nv_bfloat16* kin = reinterpret_cast<const __nv_bfloat16*>(p.k) + tok * kD + j0;
             const __nv_bfloat16* ein = reinterpret_cast<const __nv_bfloat16*>(p.e) + tok * kD + j0;
@@ -862,34 +869,40 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             }
             fence_async_smem();
             sync_all();
-            // R1: dL_A = -dYR Y^T, dL_K = dYR U^T (strict) -> dKp = dL_A Am + dL_K Km
-            round_(aR, aY, true, aR, aU, false, kStrictLow, kStrictLow, 256);
-            // R2: dM_QA = -dO Y^T, dM_QK = dO U^T (inclusive) -> dQp = dM_QA Am + dM_QK Km
-            round_(aO, aY, true, aO, aU, false, kInclLow, kInclLow, 320);
-            {  // Kp -> Bt0, Qp -> Bt1
-                float kv[16], qv[16], gv[16], kp[16], qp[16];
-                ld8_bf16(kin, kv); ld8_bf16(kin + 8, kv + 8);
-                ld8_bf16(qin, qv); ld8_bf16(qin + 8, qv + 8);
-                if (QKRAW) {
-                    prologue8(kv, rk); prologue8(kv + 8, rk);
-                    prologue8(qv, rq); prologue8(qv + 8, rq);
-                }
-                ld8_bf16(gin_, gv); ld8_bf16(gin_ + 8, gv + 8);
+            // Four rounds (one loop, so that their code is issued once):
+            //  R1: dL_A = -dYR Y^T, dL_K = dYR U^T (strict) -> dKp = dL_A Am + dL_K Km
+            //  R2: dM_QA = -dO Y^T, dM_QK = dO U^T (inclusive) -> dQp = dM_QA Am + dM_QK Km
+            //  R3: dL_A^T = -Y dYR^T (strict upper), dM_QA^T = -Y dO^T (inclusive upper) -> dAm
+            //  R4: dL_K^T = U dYR^T (strict upper), dM_QK^T = U dO^T (inclusive upper) -> dKm
+            // with Am, Km in Bt0, Bt1 for R1, R2 and Kp, Qp for R3, R4.
+#pragma unroll 1
+            for (int r = 0; r < 4; ++r) {
+                if (r == 2) {  // Kp -> Bt0, Qp -> Bt1
+                    float kv[16], qv[16], gv[16], kp[16], qp[16];
+                    ld8_bf16(kin, kv); ld8_bf16(kin + 8, kv + 8);
+                    ld8_bf16(qin, qv); ld8_bf16(qin + 8, qv + 8);
+                    if (QKRAW) {
+                        prologue8(kv, rk); prologue8(kv + 8, rk);
+                        prologue8(qv, rq); prologue8(qv + 8, rq);
+                    }
+                    ld8_bf16(gin_, gv); ld8_bf16(gin_ + 8, gv + 8);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    const float ep = ex2(L[u] - s.P2[j0 + u]);
-                    kp[u] = kv[u] * ep;
-                    qp[u] = qv[u] * gv[u] * ep;
+                    for (int u = 0; u < 16; ++u) {
+                        const float ep = ex2(L[u] - s.P2[j0 + u]);
+                        kp[u] = kv[u] * ep;
+                        qp[u] = qv[u] * gv[u] * ep;
+                    }
+                    put_t(Bt0, r0, kp);
+                    put_t(Bt1, r0, qp);
+                    fence_async_smem();
+                    sync_all();
                 }
-                put_t(Bt0, r0, kp);
-                put_t(Bt1, r0, qp);
+                const uint32_t ax = r == 0 ? aR : r == 1 ? aO : r == 2 ? aY : aU;
+                const uint32_t bx0 = r < 2 ? aY : aR, bx1 = r < 2 ? aU : aO;
+                const int mode0 = r == 0 ? kStrictLow : r == 1 ? kInclLow : kStrictUp;
+                const int mode1 = r == 0 ? kStrictLow : r == 1 ? kInclLow : kInclUp;
+                round_(ax, bx0, r != 3, ax, bx1, r == 2, mode0, mode1, 256 + 64 * r);
             }
-            fence_async_smem();
-            sync_all();
-            // R3: dL_A^T = -Y dYR^T (strict upper), dM_QA^T = -Y dO^T (inclusive upper) -> dAm
-            round_(aY, aR, true, aY, aO, true, kStrictUp, kInclUp, 384);
-            // R4: dL_K^T = U dYR^T (strict upper), dM_QK^T = U dO^T (inclusive upper) -> dKm
-            round_(aU, aR, false, aU, aO, false, kStrictUp, kInclUp, 448);
             // ---- readout: final gradients of channels j0 .. j0 + 15 of row t
             {
                 const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + j0;
@@ -1068,7 +1081,7 @@ constexpr int rev_smem() { return 3 * 128 * 128 * 4 + SLAB * 512 + 1024; }
 size_t bwd2_ws_bytes(int B, int T, int H) {
     const size_t nch = (size_t)B * H * (T / kC), blk = (size_t)kC * kD * 4;
     // Bp, dSc, Pq, Pk, Pa, PL (fp32 blocks), Y16, dYR16 (fp16 tiles), dLbar per value slab
-    return nch * (6 * blk + 2 * (size_t)kT16Bytes + 4 * kD * 4) + 256;
+    return nch * (6 * blk + 2 * (size_t)kT16Bytes + 8 * kD * 4) + 256;  // dLbar: up to 8 slabs
 }
 
 cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
@@ -1081,7 +1094,7 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     float* Pk = f; f += nch * blk;
     float* Pa = f; f += nch * blk;
     float* Pd = f; f += nch * blk;
-    constexpr int SLAB = 32;
+    const int SLAB = chain_slab(BH);  // column slabs of the reverse state pass
     float* dgb = f; f += (size_t)(kD / SLAB) * nch * kD;
     unsigned char* Y16 = reinterpret_cast<unsigned char*>(f);
     unsigned char* dYR16 = Y16 + (size_t)nch * kT16Bytes;
@@ -1110,8 +1123,13 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     if (!map_rows32f(&rp.tMt, a.Mt, (long long)nch * kD)) return cudaErrorInvalidValue;
     rp.Bp = Bp; rp.S_chunks = a.S_chunks; rp.S_last = a.S_last; rp.dS_final = a.dS_final;
     rp.dSc = dSc; rp.dS0 = a.dS0; rp.dgb = dgb; rp.N = N; rp.nch = nch;
-    if ((e = cudaFuncSetAttribute(k2_chain_rev<SLAB>, cudaFuncAttributeMaxDynamicSharedMemorySize, rev_smem<SLAB>())) != cudaSuccess) return e;
-    MUIR_TIMED("k2_chain_rev", st, k2_chain_rev<SLAB><<<BH * (kD / SLAB), 128, rev_smem<SLAB>(), st>>>(rp));
+    if (SLAB == 16) {
+        if ((e = cudaFuncSetAttribute(k2_chain_rev<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, rev_smem<16>())) != cudaSuccess) return e;
+        MUIR_TIMED("k2_chain_rev", st, k2_chain_rev<16><<<BH * (kD / 16), 128, rev_smem<16>(), st>>>(rp));
+    } else {
+        if ((e = cudaFuncSetAttribute(k2_chain_rev<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, rev_smem<32>())) != cudaSuccess) return e;
+        MUIR_TIMED("k2_chain_rev", st, k2_chain_rev<32><<<BH * (kD / 32), 128, rev_smem<32>(), st>>>(rp));
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     const int grid = nch < nsm ? nch : nsm;
@@ -1132,6 +1150,8 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     p2.dgb = dgb; p2.nslab = kD / SLAB;
     p2.dq = a.dq; p2.dk = a.dk; p2.dg = a.dg; p2.de = a.de; p2.dgamma = a.dgamma;
     p2.rnorm = a.rnorm;
+    p2.flags = a.flags;
+    if (!a.flags) return cudaErrorInvalidValue;
     auto k2 = a.rnorm ? k2_bwd2<true> : k2_bwd2<false>;
     if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwd2Smem)) != cudaSuccess) return e;
     MUIR_TIMED("k2_bwd2", st, k2<<<grid, 512, kBwd2Smem, st>>>(p2));

@@ -59,6 +59,7 @@ struct Bwd2Params {
     int nslab;
     void *dq, *dk, *dg, *de, *dgamma;
     const float* rnorm;                   // fused prologue: [nch][2][128] inverse row norms
+    int* flags;                           // flags[0] |= 1 when a chunk's decay span exceeds the single pivot
 };
 
 struct Bwd2Args {
@@ -76,6 +77,7 @@ struct Bwd2Args {
     void *dq, *dk, *dv, *dg, *de, *dw, *dgamma;
     float* dS0;                             // or null
     void* ws;                               // bwd2_ws_bytes
+    int* flags;                             // raised when a chunk exceeds the single pivot
 };
 
 size_t bwd2_ws_bytes(int B, int T, int H);

@@ -111,8 +111,7 @@ cudaError_t run_chunk_fwd(const ChunkProblem& P, const float* S0, void* o, float
         cudaError_t e = cudaSuccess;
         if (P.gate_proj)  // projected gates first: everything below reads them
             e = v2::run_gates_fwd(*static_cast<const v2::GatesArgs*>(P.gate_proj), st);
-        if (e == cudaSuccess) e = cudaMemsetAsync(flags, 0, 16, st);
-        if (e == cudaSuccess) e = v2::span_check(P.g, P.B, P.T, P.H, flags, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(flags, 0, 16, st);  // k2_intra raises the span flag
         if (e == cudaSuccess) e = v2::run_fwd2(a, st);
         if (e != cudaSuccess) return e;
         ChunkProblem G = P;
@@ -148,8 +147,7 @@ cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S
         cudaError_t e = cudaSuccess;
         if (P.gate_proj)  // the forward's projected gates, recomputed
             e = v2::run_gates_fwd(*static_cast<const v2::GatesArgs*>(P.gate_proj), st);
-        if (e == cudaSuccess) e = cudaMemsetAsync(flags, 0, 16, st);
-        if (e == cudaSuccess) e = v2::span_check(P.g, P.B, P.T, P.H, flags, st);
+        if (e == cudaSuccess) e = cudaMemsetAsync(flags, 0, 16, st);  // k2_bwd2 (and a recomputed k2_intra) raise it
         if (e != cudaSuccess) return e;
         v2::Bwd2Args b = {};
         b.B = P.B; b.T = P.T; b.H = P.H;
@@ -197,6 +195,7 @@ cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S
             rest = reinterpret_cast<char*>(ax) + v2::aux_bytes(nch, (size_t)P.B * P.H);
         }
         b.ws = rest;
+        b.flags = flags;
         if ((e = v2::run_bwd2(b, st)) != cudaSuccess) return e;
         ChunkProblem G = P;
         G.gate = flags;

@@ -3,8 +3,9 @@
 //
 // Scope: bf16 inputs, dk = dv = 128, chunk C = 128, T a multiple of 128, and
 // chunks whose per-channel log decay over the chunk stays within the
-// single-pivot range (|sum g| <= 140, checked on the device by k2_span; larger
-// spans take the 8-token boundary-pivot path in chunk_impl.cuh).
+// single-pivot range (|sum g| <= 140; k2_intra raises a device flag for a
+// chunk beyond it, and the call then also runs the 8-token boundary-pivot path
+// of chunk_impl.cuh, whose results replace these).
 //
 // Per chunk (wolonglab.org page, "Methodology": each chunk is a unit-lower-
 // triangular system; fig:kernel: fused right-hand side, block inversion on the
@@ -68,27 +69,6 @@ __device__ __forceinline__ void rot8(float (&L)[32]) {
 __device__ __forceinline__ void bf16_split(float x, float& hi, float& lo) {
     hi = __bfloat162float(__float2bfloat16_rn(x));
     lo = x - hi;
-}
-
-// ------------------------------------------------------------------ span pre-pass
-
-// flags[0] = 1 if any chunk has a channel whose clamped log decay summed over
-// the chunk is below -kSpanMax.  One warp per (chunk, 32-channel quarter).
-__global__ void k2_span(const __nv_bfloat16* __restrict__ g, int B, int T, int H, int* flags) {
-    const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5, lane = threadIdx.x & 31;
-    const int N = T / kC;
-    const long long nwork = (long long)B * H * N * 4;
-    if (warp >= nwork) return;
-    const int quarter = warp & 3;
-    const long long c = warp >> 2;
-    const int n = (int)(c % N);
-    const long long bh = c / N;
-    const int h = (int)(bh % H), b = (int)(bh / H);
-    const int j = 32 * quarter + lane;
-    const __nv_bfloat16* p = g + (((size_t)b * T + (size_t)n * kC) * H + h) * kD + j;
-    float s = 0.f;
-    for (int t = 0; t < kC; ++t) s += fmaxf(__bfloat162float(p[(size_t)t * H * kD]), kLogDecayMin);
-    if (__any_sync(0xffffffffu, s < -kSpanMax) && lane == 0) atomicOr(flags, 1);
 }
 
 // ------------------------------------------------------------------ k2_intra
@@ -308,6 +288,8 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             s.Lb[col] = lb;
             s.P2[col] = 0.5f * lb;
             s.eP2[col] = ex2(0.5f * lb);
+            // a span beyond the single pivot sends the call to the boundary-pivot path
+            if (__any_sync(0xffffffffu, lb < -kSpanMax * kLog2e) && lane == 0) atomicOr(p.flags, 1);
         }
         __syncthreads();
 
@@ -944,6 +926,8 @@ constexpr int kOutSmem = 2 * 128 * 128 * 4 + 1024;
 template <int SLAB>
 constexpr int chain_smem() { return 3 * 128 * 128 * 4 + SLAB * 512 + 1024; }
 
+int chain_slab(int BH) { return BH * (kD / 32) < sm_count() ? 16 : 32; }
+
 size_t fwd2_ws_bytes(int B, int T, int H) {
     const size_t nch = (size_t)B * H * (T / kC), CD = (size_t)kC * kD;
     // M, Bn, Q', O_intra, S_chunks, flags
@@ -952,14 +936,6 @@ size_t fwd2_ws_bytes(int B, int T, int H) {
 
 bool fwd2_supported(int B, int T, int H, int D, int C, bool in_bf16) {
     return in_bf16 && D == kD && C == kC && T > 0 && T % kC == 0 && B > 0 && H > 0;
-}
-
-cudaError_t span_check(const void* g, int B, int T, int H, int* flags, cudaStream_t st) {
-    const long long warps = (long long)B * H * (T / kC) * 4;
-    const int blocks = (int)((warps * 32 + 255) / 256);
-    MUIR_TIMED("k2_span", st, k2_span<<<blocks, 256, 0, st>>>(
-        static_cast<const __nv_bfloat16*>(g), B, T, H, flags));
-    return cudaGetLastError();
 }
 
 cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st) {
@@ -985,14 +961,21 @@ cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st) {
     MUIR_TIMED("k2_intra", st, kern<<<grid, 512, kIntraSmem, st>>>(ip));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-    constexpr int SLAB = 32;
+    // one CTA per (head, column slab): 16-column slabs when 32-column ones
+    // would leave SMs idle (each CTA is a sequential pass over the chunks)
     ChainParams cp;
     if (!map_rows32f(&cp.tM, a.M, (long long)nch * kD)) return cudaErrorInvalidValue;
     cp.Bn = a.Bn; cp.S0 = a.S0; cp.S_chunks = a.S_chunks; cp.S_final = a.S_final; cp.N = N;
     cp.S_last = a.S_last;
-    e = cudaFuncSetAttribute(k2_chain<SLAB>, cudaFuncAttributeMaxDynamicSharedMemorySize, chain_smem<SLAB>());
-    if (e != cudaSuccess) return e;
-    MUIR_TIMED("k2_chain", st, k2_chain<SLAB><<<BH * (kD / SLAB), 128, chain_smem<SLAB>(), st>>>(cp));
+    if (chain_slab(BH) == 16) {
+        e = cudaFuncSetAttribute(k2_chain<16>, cudaFuncAttributeMaxDynamicSharedMemorySize, chain_smem<16>());
+        if (e != cudaSuccess) return e;
+        MUIR_TIMED("k2_chain", st, k2_chain<16><<<BH * (kD / 16), 128, chain_smem<16>(), st>>>(cp));
+    } else {
+        e = cudaFuncSetAttribute(k2_chain<32>, cudaFuncAttributeMaxDynamicSharedMemorySize, chain_smem<32>());
+        if (e != cudaSuccess) return e;
+        MUIR_TIMED("k2_chain", st, k2_chain<32><<<BH * (kD / 32), 128, chain_smem<32>(), st>>>(cp));
+    }
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
     if (a.o) {

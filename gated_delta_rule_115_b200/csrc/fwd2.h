@@ -58,7 +58,7 @@ struct IntraParams {
     float* Qp;     // Q'_n [t][i]: O_n = Q'_n S_n + O_intra_n
     float* Oi;     // O_intra_n [t][c]
     unsigned char* aux;  // per-chunk AuxLayout records, or null (nothing saved)
-    int* flags;
+    int* flags;          // flags[0] |= 1 when a chunk's decay span exceeds the single pivot
     // fused q/k prologue: q and k hold raw x; every read applies
     // SiLU(x) / ||SiLU(x)|| per token-head row, and the row's inverse norms
     // go to rnorm[c][0][t] (q) and rnorm[c][1][t] (k) for the backward
@@ -105,8 +105,9 @@ struct Fwd2Args {
 };
 
 bool fwd2_supported(int B, int T, int H, int D, int C, bool in_bf16);
+// Column-slab width of the two state passes for B*H heads (16 or 32).
+int chain_slab(int BH);
 size_t fwd2_ws_bytes(int B, int T, int H);
-cudaError_t span_check(const void* g, int B, int T, int H, int* flags, cudaStream_t st);
 cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st);
 unsigned int timeouts_v2();
 
