@@ -94,6 +94,76 @@ __device__ __forceinline__ void prologue8(float* v, float r) {
     for (int u = 0; u < 8; ++u) v[u] = v[u] * sigmoid_f(v[u]) * r;
 }
 
+// 32 values as fp16 times a power of two: the scale puts the largest
+// magnitude just below 2^15 (fp16 keeps 11 significant bits of every value
+// within 2^-14 of it; the sums these partials join are dominated by larger
+// terms).  dst: 32 halves (64 bytes, 16-byte aligned); *scale: the factor.
+__device__ __forceinline__ void st_scaled32(__half* dst, float* scale, const float* v) {
+    float m = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
+    int ex = 0;
+    frexpf(m, &ex);                       // m < 2^ex (m = 0: ex = 0)
+    const int e = max(ex - 15, -126);
+    const float inv = __int_as_float((127 - e) << 23), sc = __int_as_float((127 + e) << 23);
+    *scale = sc;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint4 u;
+        u.x = pack_f16(v[8 * i] * inv, v[8 * i + 1] * inv);
+        u.y = pack_f16(v[8 * i + 2] * inv, v[8 * i + 3] * inv);
+        u.z = pack_f16(v[8 * i + 4] * inv, v[8 * i + 5] * inv);
+        u.w = pack_f16(v[8 * i + 6] * inv, v[8 * i + 7] * inv);
+        reinterpret_cast<uint4*>(dst)[i] = u;
+    }
+}
+
+// The same for the two groups a + b and a - b (each with its own scale),
+// without forming them in registers first.
+__device__ __forceinline__ void st_scaled32_pm(__half* dp, float* sp, __half* dm, float* sm_,
+                                               const float* a, const float* b) {
+    float mp = 0.f, mm = 0.f;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        mp = fmaxf(mp, fabsf(a[j] + b[j]));
+        mm = fmaxf(mm, fabsf(a[j] - b[j]));
+    }
+    int ep = 0, em = 0;
+    frexpf(mp, &ep);
+    frexpf(mm, &em);
+    ep = max(ep - 15, -126);
+    em = max(em - 15, -126);
+    const float ip = __int_as_float((127 - ep) << 23), im = __int_as_float((127 - em) << 23);
+    *sp = __int_as_float((127 + ep) << 23);
+    *sm_ = __int_as_float((127 + em) << 23);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        uint4 u, w;
+        const int j = 8 * i;
+        u.x = pack_f16((a[j] + b[j]) * ip, (a[j + 1] + b[j + 1]) * ip);
+        u.y = pack_f16((a[j + 2] + b[j + 2]) * ip, (a[j + 3] + b[j + 3]) * ip);
+        u.z = pack_f16((a[j + 4] + b[j + 4]) * ip, (a[j + 5] + b[j + 5]) * ip);
+        u.w = pack_f16((a[j + 6] + b[j + 6]) * ip, (a[j + 7] + b[j + 7]) * ip);
+        w.x = pack_f16((a[j] - b[j]) * im, (a[j + 1] - b[j + 1]) * im);
+        w.y = pack_f16((a[j + 2] - b[j + 2]) * im, (a[j + 3] - b[j + 3]) * im);
+        w.z = pack_f16((a[j + 4] - b[j + 4]) * im, (a[j + 5] - b[j + 5]) * im);
+        w.w = pack_f16((a[j + 6] - b[j + 6]) * im, (a[j + 7] - b[j + 7]) * im);
+        reinterpret_cast<uint4*>(dp)[i] = u;
+        reinterpret_cast<uint4*>(dm)[i] = w;
+    }
+}
+
+// 8 scaled fp16 values -> floats.
+__device__ __forceinline__ void ld8_scaled(const __half* p, float sc, float* v) {
+    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+    unpack16<false>(u.x, v[0], v[1]);
+    unpack16<false>(u.y, v[2], v[3]);
+    unpack16<false>(u.z, v[4], v[5]);
+    unpack16<false>(u.w, v[6], v[7]);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v[i] *= sc;
+}
+
 // Store 32 values at columns 32 * c32 .. +32 of row t of a T16 tile.
 template <bool BF16>
 __device__ __forceinline__ void row_st32(unsigned char* tile, int t, int c32, const float* v) {
@@ -434,7 +504,8 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
         const int n = c % N, bh = c / N, hd = bh % p.H, b = bh / p.H;
         const size_t tok = ((size_t)b * p.T + (size_t)n * kC + t) * p.H + hd;  // token-major row
         const size_t ro = tok * kD + c0;                                      // this thread's 32 elements
-        const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + c0;          // per-chunk fp32 arrays
+        const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + c0;          // per-chunk arrays
+        const size_t scb = ((size_t)c * kC + t) * 4 + h;                      // their group scales
         const unsigned char* ax = p.aux + (size_t)c * AuxLayout::kBytes;
         unsigned char* y16 = p.Y16 + (size_t)c * kT16Bytes;
         unsigned char* r16 = p.dYR16 + (size_t)c * kT16Bytes;
@@ -502,15 +573,9 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
         {
             float d[32];
             tm_ld32w(tm, q, c0, d);
-            float* pq = p.Pq + cb;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float o[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) o[u] = d[8 * i + u] * sS * ex2(L[8 * i + u]);
-                *reinterpret_cast<float4*>(pq + 8 * i) = make_float4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<float4*>(pq + 8 * i + 4) = make_float4(o[4], o[5], o[6], o[7]);
-            }
+            for (int j = 0; j < 32; ++j) d[j] *= sS * ex2(L[j]);
+            st_scaled32(p.Pq + cb, p.sq + scb, d);
             tm_ld32w(tm, q, 128 + c0, d);
             const float* up = reinterpret_cast<const float*>(ax + AuxLayout::kUp) + (size_t)t * kD + c0;
 #pragma unroll
@@ -542,18 +607,9 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
         {
             float d[32];
             tm_ld32w(tm, q, 128 + c0, d);  // dAbar / sG
-            float* pa = p.Pa + cb;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float o[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int j = 8 * i + u;
-                    o[u] = d[j] * sG * ex2(s.Lb[c0 + j] - L[j]);
-                }
-                *reinterpret_cast<float4*>(pa + 8 * i) = make_float4(o[0], o[1], o[2], o[3]);
-                *reinterpret_cast<float4*>(pa + 8 * i + 4) = make_float4(o[4], o[5], o[6], o[7]);
-            }
+            for (int j = 0; j < 32; ++j) d[j] *= sG * ex2(s.Lb[c0 + j] - L[j]);
+            st_scaled32(p.Pa + cb, p.sa + scb, d);
         }
         waitb(B1A, ph);  // (its block barrier also orders the reads of B1 above)
         // ---- phase 4: Abar G / sG (B0); dY = -M_QA^T dO - Abar G
@@ -607,24 +663,12 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             float d[32], e2[32];
             tm_ld32w(tm, q, c0, d);         // dK~ / sS
             tm_ld32w(tm, q, 384 + c0, e2);  // dKbar / sG
-            float* pk = p.Pk + cb;
-            float* pd = p.Pd + cb;
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                float o1[8], o2[8];
-#pragma unroll
-                for (int u = 0; u < 8; ++u) {
-                    const int j = 8 * i + u;
-                    const float x1 = d[j] * sS * ex2(L[j]);                          // dK~ 2^L
-                    const float x2 = e2[j] * sG * ex2(s.Lb[c0 + j] - L[j]);         // dKbar 2^(Lbar-L)
-                    o1[u] = x1 + x2;
-                    o2[u] = x1 - x2;
-                }
-                *reinterpret_cast<float4*>(pk + 8 * i) = make_float4(o1[0], o1[1], o1[2], o1[3]);
-                *reinterpret_cast<float4*>(pk + 8 * i + 4) = make_float4(o1[4], o1[5], o1[6], o1[7]);
-                *reinterpret_cast<float4*>(pd + 8 * i) = make_float4(o2[0], o2[1], o2[2], o2[3]);
-                *reinterpret_cast<float4*>(pd + 8 * i + 4) = make_float4(o2[4], o2[5], o2[6], o2[7]);
+            for (int j = 0; j < 32; ++j) {
+                d[j] *= sS * ex2(L[j]);                    // dK~ 2^L
+                e2[j] *= sG * ex2(s.Lb[c0 + j] - L[j]);  // dKbar 2^(Lbar-L)
             }
+            st_scaled32_pm(p.Pk + cb, p.sk + scb, p.Pd + cb, p.sd + scb, d, e2);  // Pk, Pd
         }
         waitb(B1L, ph);
         waitb(B1KB, ph);
@@ -814,11 +858,14 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 if (((i * 2 + 1) & 3) == g4) prefetch_l2(rows[i] + off + 128);
             }
             if (tid == 32) {
-                const size_t cb = (size_t)c * kC * kD * sizeof(float);
-                bulk_prefetch_l2(reinterpret_cast<const char*>(p.Pq) + cb, kC * kD * 4);
-                bulk_prefetch_l2(reinterpret_cast<const char*>(p.Pk) + cb, kC * kD * 4);
-                bulk_prefetch_l2(reinterpret_cast<const char*>(p.Pa) + cb, kC * kD * 4);
-                bulk_prefetch_l2(reinterpret_cast<const char*>(p.Pd) + cb, kC * kD * 4);
+                const size_t cb = (size_t)c * kC * kD * 2, sb = (size_t)c * kC * 16;
+                const __half* P[4] = {p.Pq, p.Pk, p.Pa, p.Pd};
+                const float* S4[4] = {p.sq, p.sk, p.sa, p.sd};
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    bulk_prefetch_l2(reinterpret_cast<const char*>(P[i]) + cb, kC * kD * 2);
+                    bulk_prefetch_l2(reinterpret_cast<const char*>(S4[i]) + sb, kC * 16);
+                }
             }
         }
         if (tid < kD) {  // dLbar: the value slabs' partial sums in a fixed order
@@ -907,6 +954,9 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             {
                 const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + j0;
                 const size_t ro = tok * kD + j0;
+                const size_t scb = ((size_t)c * kC + t) * 4 + (j0 >> 5);  // channels j0 .. +16 share a group
+                const float s_q = __ldg(p.sq + scb), s_k = __ldg(p.sk + scb);
+                const float s_a = __ldg(p.sa + scb), s_d = __ldg(p.sd + scb);
                 float dL[16];
                 float dotq = 0.f, dotk = 0.f;
 #pragma unroll
@@ -925,20 +975,10 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                     ld8_bf16(gin_ + u0, gv);
                     if (QKRAW) { prologue8(kv, rk); prologue8(qv, rq); }
                     float pq[8], pk[8], pa[8], pl[8];
-#pragma unroll
-                    for (int u = 0; u < 8; u += 4) {
-                        // (plain loads with the fused prologue: this kernel overwrites them)
-                        const float4 x0 = QKRAW ? *reinterpret_cast<const float4*>(p.Pq + cb + u0 + u)
-                                                : __ldg(reinterpret_cast<const float4*>(p.Pq + cb + u0 + u));
-                        const float4 x1 = QKRAW ? *reinterpret_cast<const float4*>(p.Pk + cb + u0 + u)
-                                                : __ldg(reinterpret_cast<const float4*>(p.Pk + cb + u0 + u));
-                        const float4 x2 = __ldg(reinterpret_cast<const float4*>(p.Pa + cb + u0 + u));
-                        const float4 x3 = __ldg(reinterpret_cast<const float4*>(p.Pd + cb + u0 + u));
-                        pq[u] = x0.x; pq[u + 1] = x0.y; pq[u + 2] = x0.z; pq[u + 3] = x0.w;
-                        pk[u] = x1.x; pk[u + 1] = x1.y; pk[u + 2] = x1.z; pk[u + 3] = x1.w;
-                        pa[u] = x2.x; pa[u + 1] = x2.y; pa[u + 2] = x2.z; pa[u + 3] = x2.w;
-                        pl[u] = x3.x; pl[u + 1] = x3.y; pl[u + 2] = x3.z; pl[u + 3] = x3.w;
-                    }
+                    ld8_scaled(p.Pq + cb + u0, s_q, pq);
+                    ld8_scaled(p.Pk + cb + u0, s_k, pk);
+                    ld8_scaled(p.Pa + cb + u0, s_a, pa);
+                    ld8_scaled(p.Pd + cb + u0, s_d, pl);
                     float oq[8], og[8], ok[8], oe[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
@@ -958,14 +998,14 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                                 (a_km[u] * kv[u] + a_a[u] * ev[u] * kv[u]) * em +
                                 pl[u] * kv[u] + pq[u] * qh - pa[u] * ev[u] * kv[u];
                     }
-                    if (QKRAW) {  // dq^, dk^ (fp32, over the P entries just read) and row dots
+                    if (QKRAW) {  // dq^, dk^ (fp32, for the last pass) and row dots
 #pragma unroll
                         for (int u = 0; u < 8; ++u) {
                             dotq = fmaf(oq[u], qv[u], dotq);
                             dotk = fmaf(ok[u], kv[u], dotk);
                         }
-                        float* pq_ = p.Pq + cb + u0;
-                        float* pk_ = p.Pk + cb + u0;
+                        float* pq_ = p.dqh + cb + u0;
+                        float* pk_ = p.dkh + cb + u0;
                         *reinterpret_cast<float4*>(pq_) = make_float4(oq[0], oq[1], oq[2], oq[3]);
                         *reinterpret_cast<float4*>(pq_ + 4) = make_float4(oq[4], oq[5], oq[6], oq[7]);
                         *reinterpret_cast<float4*>(pk_) = make_float4(ok[0], ok[1], ok[2], ok[3]);
@@ -1027,7 +1067,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             const size_t ro = tok * kD + 32 * g4;
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
-                const float* dy = (which ? p.Pk : p.Pq) + cb;
+                const float* dy = (which ? p.dkh : p.dqh) + cb;
                 const __nv_bfloat16* xr = reinterpret_cast<const __nv_bfloat16*>(which ? p.k : p.q) + ro;
                 __nv_bfloat16* dx = reinterpret_cast<__nv_bfloat16*>(which ? p.dk : p.dq) + ro;
                 const float r = which ? rk : rq, dot = which ? dk_dot : dq_dot;
@@ -1080,8 +1120,9 @@ constexpr int rev_smem() { return 3 * 128 * 128 * 4 + SLAB * 512 + 1024; }
 
 size_t bwd2_ws_bytes(int B, int T, int H) {
     const size_t nch = (size_t)B * H * (T / kC), blk = (size_t)kC * kD * 4;
-    // Bp, dSc, Pq, Pk, Pa, PL (fp32 blocks), Y16, dYR16 (fp16 tiles), dLbar per value slab
-    return nch * (6 * blk + 2 * (size_t)kT16Bytes + 8 * kD * 4) + 256;  // dLbar: up to 8 slabs
+    // Bp, dSc, dq^, dk^ (fp32 blocks), Pq, Pk, Pa, Pd (fp16 blocks) and their
+    // group scales, Y16, dYR16 (fp16 tiles), dLbar per value slab (up to 8)
+    return nch * (4 * blk + 4 * blk / 2 + 4 * (size_t)kC * 16 + 2 * (size_t)kT16Bytes + 8 * kD * 4) + 256;
 }
 
 cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
@@ -1090,10 +1131,12 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     float* f = reinterpret_cast<float*>(a.ws);
     float* Bp = f; f += nch * blk;
     float* dSc = f; f += nch * blk;
-    float* Pq = f; f += nch * blk;
-    float* Pk = f; f += nch * blk;
-    float* Pa = f; f += nch * blk;
-    float* Pd = f; f += nch * blk;
+    float* dqh = f; f += nch * blk;
+    float* dkh = f; f += nch * blk;
+    __half* P16[4];
+    for (int i = 0; i < 4; ++i) { P16[i] = reinterpret_cast<__half*>(f); f += nch * blk / 2; }
+    float* Psc[4];
+    for (int i = 0; i < 4; ++i) { Psc[i] = f; f += (size_t)nch * kC * 4; }
     const int SLAB = chain_slab(BH);  // column slabs of the reverse state pass
     float* dgb = f; f += (size_t)(kD / SLAB) * nch * kD;
     unsigned char* Y16 = reinterpret_cast<unsigned char*>(f);
@@ -1137,7 +1180,9 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     p1.tdO = tdO; p1.B = a.B; p1.T = a.T; p1.H = a.H;
     p1.q = a.q; p1.k = a.k; p1.v = a.v; p1.g = a.g; p1.e = a.e; p1.w = a.w; p1.gamma = a.gamma;
     p1.aux = a.aux; p1.S_chunks = a.S_chunks; p1.dSc = dSc;
-    p1.Pq = Pq; p1.Pk = Pk; p1.Pa = Pa; p1.Pd = Pd; p1.Y16 = Y16; p1.dYR16 = dYR16;
+    p1.Pq = P16[0]; p1.Pk = P16[1]; p1.Pa = P16[2]; p1.Pd = P16[3];
+    p1.sq = Psc[0]; p1.sk = Psc[1]; p1.sa = Psc[2]; p1.sd = Psc[3];
+    p1.Y16 = Y16; p1.dYR16 = dYR16;
     p1.dv = a.dv; p1.dw = a.dw;
     if ((e = cudaFuncSetAttribute(k2_bwd1, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwd1Smem)) != cudaSuccess) return e;
     MUIR_TIMED("k2_bwd1", st, k2_bwd1<<<grid, 512, kBwd1Smem, st>>>(p1));
@@ -1146,7 +1191,10 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     Bwd2Params p2;
     p2.tdO = tdO; p2.B = a.B; p2.T = a.T; p2.H = a.H;
     p2.q = a.q; p2.k = a.k; p2.g = a.g; p2.e = a.e; p2.gamma = a.gamma;
-    p2.aux = a.aux; p2.Y16 = Y16; p2.dYR16 = dYR16; p2.Pq = Pq; p2.Pk = Pk; p2.Pa = Pa; p2.Pd = Pd;
+    p2.aux = a.aux; p2.Y16 = Y16; p2.dYR16 = dYR16;
+    p2.Pq = P16[0]; p2.Pk = P16[1]; p2.Pa = P16[2]; p2.Pd = P16[3];
+    p2.sq = Psc[0]; p2.sk = Psc[1]; p2.sa = Psc[2]; p2.sd = Psc[3];
+    p2.dqh = dqh; p2.dkh = dkh;
     p2.dgb = dgb; p2.nslab = kD / SLAB;
     p2.dq = a.dq; p2.dk = a.dk; p2.dg = a.dg; p2.de = a.de; p2.dgamma = a.dgamma;
     p2.rnorm = a.rnorm;

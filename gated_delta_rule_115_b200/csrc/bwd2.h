@@ -3,6 +3,7 @@
 #pragma once
 
 #include <cuda.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stddef.h>
 
@@ -43,7 +44,10 @@ struct Bwd1Params {
     const unsigned char* aux;
     const float* S_chunks;
     const float* dSc;
-    float *Pq, *Pk, *Pa, *Pd;
+    // state-side partials as fp16 [nch][128][128] with one power-of-two scale
+    // per row and 32-column group ([nch][128][4] fp32)
+    __half *Pq, *Pk, *Pa, *Pd;
+    float *sq, *sk, *sa, *sd;
     unsigned char *Y16, *dYR16;
     void *dv, *dw;
 };
@@ -54,8 +58,10 @@ struct Bwd2Params {
     const void *q, *k, *g, *e, *gamma;
     const unsigned char* aux;
     const unsigned char *Y16, *dYR16;
-    float *Pq, *Pk;                       // with the fused prologue, reused for dq^, dk^
-    const float *Pa, *Pd, *dgb;           // dgb: [nslab][nch][128] partials of dLbar
+    const __half *Pq, *Pk, *Pa, *Pd;      // k2_bwd1's partials (scaled fp16, see Bwd1Params)
+    const float *sq, *sk, *sa, *sd;
+    float *dqh, *dkh;                     // fused prologue: dq^, dk^ before its Jacobian (fp32)
+    const float* dgb;                     // [nslab][nch][128] partials of dLbar
     int nslab;
     void *dq, *dk, *dg, *de, *dgamma;
     const float* rnorm;                   // fused prologue: [nch][2][128] inverse row norms
