@@ -831,6 +831,20 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
         mma_wait();
     };
 
+    // dO, U, Y, dYR of chunk cc into the four tiles; a chunk's loads are issued
+    // as soon as the previous chunk's last products have read the tiles
+    auto load_tiles = [&](int cc) {
+        const int nn = cc % N, bb = cc / N;
+        mbar_arrive_expect_tx(&s.bar[B2IN], 4 * kT16Bytes);
+        const int z = (bb / p.H) * p.T + nn * kC;
+        tma_load_3d(tdO, &p.tdO, 0, bb % p.H, z, &s.bar[B2IN]);
+        tma_load_3d(tdO + kT16Block, &p.tdO, 64, bb % p.H, z, &s.bar[B2IN]);
+        bulk_load(tU, p.aux + (size_t)cc * AuxLayout::kBytes + AuxLayout::kU16, kT16Bytes, &s.bar[B2IN]);
+        bulk_load(tY, p.Y16 + (size_t)cc * kT16Bytes, kT16Bytes, &s.bar[B2IN]);
+        bulk_load(tR, p.dYR16 + (size_t)cc * kT16Bytes, kT16Bytes, &s.bar[B2IN]);
+    };
+    if (tid == 0 && (int)blockIdx.x < nch) load_tiles(blockIdx.x);
+
     int it = 0;
     for (int c = blockIdx.x; c < nch; c += gridDim.x, ++it) {
         const uint32_t ph = (uint32_t)(it & 1);
@@ -838,15 +852,6 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
         const size_t tok = ((size_t)b * p.T + (size_t)n * kC + t) * p.H + hd;
         const float rq = QKRAW ? __ldg(p.rnorm + (size_t)c * 2 * kC + t) : 1.f;
         const float rk = QKRAW ? __ldg(p.rnorm + (size_t)c * 2 * kC + kC + t) : 1.f;
-        if (tid == 0) {
-            mbar_arrive_expect_tx(&s.bar[B2IN], 4 * kT16Bytes);
-            const int z = b * p.T + n * kC;
-            tma_load_3d(tdO, &p.tdO, 0, hd, z, &s.bar[B2IN]);
-            tma_load_3d(tdO + kT16Block, &p.tdO, 64, hd, z, &s.bar[B2IN]);
-            bulk_load(tU, p.aux + (size_t)c * AuxLayout::kBytes + AuxLayout::kU16, kT16Bytes, &s.bar[B2IN]);
-            bulk_load(tY, p.Y16 + (size_t)c * kT16Bytes, kT16Bytes, &s.bar[B2IN]);
-            bulk_load(tR, p.dYR16 + (size_t)c * kT16Bytes, kT16Bytes, &s.bar[B2IN]);
-        }
         {  // this chunk's rows of the inputs the readout reads late -> L2
             const char* rows[5] = {static_cast<const char*>(p.k), static_cast<const char*>(p.e),
                                    static_cast<const char*>(p.q), static_cast<const char*>(p.gamma),
@@ -950,6 +955,8 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 const int mode1 = r == 0 ? kStrictLow : r == 1 ? kInclLow : kInclUp;
                 round_(ax, bx0, r != 3, ax, bx1, r == 2, mode0, mode1, 256 + 64 * r);
             }
+            // the second half's rounds were the tiles' last readers
+            if (hj == 1 && tid == 0 && c + (int)gridDim.x < nch) load_tiles(c + gridDim.x);
             // ---- readout: final gradients of channels j0 .. j0 + 15 of row t
             {
                 const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + j0;
