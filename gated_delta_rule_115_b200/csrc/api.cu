@@ -387,7 +387,7 @@ size_t gate_buf_bytes(const muir_shape* s) { return (size_t)s->B * s->T * s->H *
 size_t fused_ws(const muir_shape* s, const muir_fusion* f, bool backward) {
     const size_t base = base_ws(s, backward);
     if (!fused_any(f)) return base;
-    size_t extra = muir::fused_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk);
+    size_t extra = muir::fused_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, f->qk_raw != 0);
     if (f->latent) extra += 5 * (backward ? 4 : 1) * gate_buf_bytes(s);
     return ((base + 255) & ~(size_t)255) + extra;
 }
@@ -406,7 +406,7 @@ void setup_projection(const muir_shape* s, const muir_fusion* f, char* fw, bool 
                                muir::v2::kActIdentity, muir::v2::kActSigmoid,
                                muir::v2::kActSigmoid};
     const size_t gb = gate_buf_bytes(s);
-    char* buf = fw + muir::fused_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk);
+    char* buf = fw + muir::fused_ws_bytes(s->B, s->T, s->H, s->dk, s->chunk, f->qk_raw != 0);
     ga = muir::v2::GatesArgs{};
     ga.latent = f->latent;
     ga.R = f->R;

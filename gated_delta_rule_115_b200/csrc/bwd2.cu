@@ -262,10 +262,11 @@ __global__ void __launch_bounds__(256) k2_bprep(const __grid_constant__ BprepPar
         }
     }
     if (!cta_wait(&bar[0], 0) && tid == 0) atomicOr(&bad, 1);
-    if (p.zo) {  // fused output gate: dO = dO' sig(z) (bf16), dz = dO' o sig (1 - sig)
+    if (p.zo) {  // fused output gate: dO = dO' sig(z) (fp16, and bf16), dz = dO' o sig (1 - sig)
         const size_t ro = (((size_t)(bh / p.H) * p.T + (size_t)n * kC + t) * p.H + bh % p.H) * kD + 64 * h;
         const __nv_bfloat16* zr = reinterpret_cast<const __nv_bfloat16*>(p.zo) + ro;
-        __nv_bfloat16* er = reinterpret_cast<__nv_bfloat16*>(p.dO_eff) + ro;
+        __half* er = reinterpret_cast<__half*>(p.dO_eff) + ro;
+        __nv_bfloat16* erb = reinterpret_cast<__nv_bfloat16*>(p.dO_effb) + ro;
         __nv_bfloat16* dzr = reinterpret_cast<__nv_bfloat16*>(p.dzo) + ro;
 #pragma unroll 2
         for (int i = 0; i < 8; ++i) {
@@ -284,11 +285,15 @@ __global__ void __launch_bounds__(256) k2_bprep(const __grid_constant__ BprepPar
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
                 const float sg = sigmoid_f(zv[u]);
-                // the bf16 value the later kernels read
-                dov[u] = __bfloat162float(__float2bfloat16_rn(dy[u] * sg));
+                // the fp16 value the later kernels read
+                dov[u] = __half2float(__float2half_rn(dy[u] * sg));
                 dzv[u] = dy[u] * ov[u] * sg * (1.f - sg);
             }
-            st8_bf16(er + 8 * i, dov);
+            uint4 hv;
+            hv.x = pack_f16(dov[0], dov[1]); hv.y = pack_f16(dov[2], dov[3]);
+            hv.z = pack_f16(dov[4], dov[5]); hv.w = pack_f16(dov[6], dov[7]);
+            *reinterpret_cast<uint4*>(er + 8 * i) = hv;
+            st8_bf16(erb + 8 * i, dov);
             st8_bf16(dzr + 8 * i, dzv);
             st_chunk16<false>(Dt, t, 8 * h + i, dov);
         }
@@ -552,7 +557,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             row_st32<false>(S[3], t, h, v);
         }
         waitb(B1D, ph);
-        {  // dO bf16 -> fp16 in place (own chunks)
+        if (!p.dO_f16) {  // dO bf16 -> fp16 in place (own chunks)
             float v[32];
             row_ld32<true>(S[1], t, h, v);
             row_st32<false>(S[1], t, h, v);
@@ -879,11 +884,13 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             s.dgb[tid] = acc;
         }
         if (!cta_wait(&s.bar[B2IN], ph) && tid == 0) atomicOr(&s.bad, 1 << 25);
+        if (!p.dO_f16) {
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {  // dO bf16 -> fp16 in place (row t, columns 32 g4 ..)
-            float v[8];
-            ld_chunk16<true>(tdO, t, 4 * g4 + i, v);
-            st_chunk16<false>(tdO, t, 4 * g4 + i, v);
+            for (int i = 0; i < 4; ++i) {  // dO bf16 -> fp16 in place (row t, columns 32 g4 ..)
+                float v[8];
+                ld_chunk16<true>(tdO, t, 4 * g4 + i, v);
+                st_chunk16<false>(tdO, t, 4 * g4 + i, v);
+            }
         }
         fence_async_smem();
         sync_all();
@@ -1164,7 +1171,9 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
 
     BprepParams bp;
     bp.tdO = tdO_in; bp.T = a.T; bp.H = a.H; bp.Qp = a.Qp; bp.Bp = Bp;
-    bp.zo = a.zo; bp.o_pre = a.o_pre; bp.o_pre_f32 = a.o_pre_f32; bp.dO_eff = a.dO_eff; bp.dzo = a.dzo;
+    bp.zo = a.zo; bp.o_pre = a.o_pre; bp.o_pre_f32 = a.o_pre_f32; bp.dO_eff = a.dO_eff;
+    bp.dO_effb = a.dO_effb; bp.dzo = a.dzo;
+    if (a.zo && !a.dO_effb) return cudaErrorInvalidValue;
     if ((e = cudaFuncSetAttribute(k2_bprep, cudaFuncAttributeMaxDynamicSharedMemorySize, kBprepSmem)) != cudaSuccess) return e;
     MUIR_TIMED("k2_bprep", st, k2_bprep<<<nch, 256, kBprepSmem, st>>>(bp));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1191,6 +1200,7 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     p1.sq = Psc[0]; p1.sk = Psc[1]; p1.sa = Psc[2]; p1.sd = Psc[3];
     p1.Y16 = Y16; p1.dYR16 = dYR16;
     p1.dv = a.dv; p1.dw = a.dw;
+    p1.dO_f16 = a.zo != nullptr;
     if ((e = cudaFuncSetAttribute(k2_bwd1, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwd1Smem)) != cudaSuccess) return e;
     MUIR_TIMED("k2_bwd1", st, k2_bwd1<<<grid, 512, kBwd1Smem, st>>>(p1));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -1206,6 +1216,7 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     p2.dq = a.dq; p2.dk = a.dk; p2.dg = a.dg; p2.de = a.de; p2.dgamma = a.dgamma;
     p2.rnorm = a.rnorm;
     p2.flags = a.flags;
+    p2.dO_f16 = a.zo != nullptr;
     if (!a.flags) return cudaErrorInvalidValue;
     auto k2 = a.rnorm ? k2_bwd2<true> : k2_bwd2<false>;
     if ((e = cudaFuncSetAttribute(k2, cudaFuncAttributeMaxDynamicSharedMemorySize, kBwd2Smem)) != cudaSuccess) return e;

@@ -16,12 +16,14 @@ struct BprepParams {
     const float* Qp;  // [nch][128][128]
     float* Bp;        // Q'^T dO per chunk
     // fused output gate (zo non-null): tdO holds the gradient of the gated
-    // output; dO = dO' sigmoid(zo) is written to dO_eff (bf16, read by the
-    // later kernels) and dzo = dO' o_pre sigmoid'(zo) to dzo (bf16)
+    // output; dO = dO' sigmoid(zo) is written to dO_eff as fp16 (read by the
+    // later kernels) and as bf16 to dO_effb (for the boundary-pivot path), and
+    // dzo = dO' o_pre sigmoid'(zo) to dzo (bf16)
     const void* zo;
     const void* o_pre;
     bool o_pre_f32;
     void* dO_eff;
+    void* dO_effb;
     void* dzo;
 };
 
@@ -50,6 +52,7 @@ struct Bwd1Params {
     float *sq, *sk, *sa, *sd;
     unsigned char *Y16, *dYR16;
     void *dv, *dw;
+    bool dO_f16;                          // tdO holds fp16 (the fused gate's dO), else bf16
 };
 
 struct Bwd2Params {
@@ -66,6 +69,7 @@ struct Bwd2Params {
     void *dq, *dk, *dg, *de, *dgamma;
     const float* rnorm;                   // fused prologue: [nch][2][128] inverse row norms
     int* flags;                           // flags[0] |= 1 when a chunk's decay span exceeds the single pivot
+    bool dO_f16;                          // tdO holds fp16 (the fused gate's dO), else bf16
 };
 
 struct Bwd2Args {
@@ -74,7 +78,8 @@ struct Bwd2Args {
     const void* zo;                         // fused output gate: pre-activation, or null
     const void* o_pre;                      // with zo: the forward's pre-gate output
     bool o_pre_f32;                         // its dtype (fp32, else bf16)
-    void* dO_eff;                           // with zo: B*T*H*128 bf16 of workspace
+    void* dO_eff;                           // with zo: B*T*H*128 fp16 of workspace
+    void* dO_effb;                          // with zo: the same as bf16 (boundary-pivot path)
     void* dzo;                              // with zo: gradient of zo (bf16)
     const float* rnorm;                     // fused q/k prologue: the forward's inverse row norms, or null
     const float* dS_final;                  // or null

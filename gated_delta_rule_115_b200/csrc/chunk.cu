@@ -116,14 +116,26 @@ cudaError_t run_chunk_fwd(const ChunkProblem& P, const float* S0, void* o, float
         if (e != cudaSuccess) return e;
         ChunkProblem G = P;
         G.gate = flags;  // boundary-pivot path only when a chunk's span exceeds the single pivot
-        if (P.qk_raw) {  // that path reads q^ and k^ as tensors
-            char* qh = fw + 256 + nch * 2 * 128 * 4;
-            char* kh = qh + rows * 128 * 2;
-            if ((e = qk_materialise_gated(flags, P.q, qh, rows, st)) != cudaSuccess) return e;
-            if ((e = qk_materialise_gated(flags, P.k, kh, rows, st)) != cudaSuccess) return e;
-            G.q = qh; G.k = kh;
+        if (P.qk_raw) {
+            // that path reads q^ and k^ as tensors: it runs in fp32 on fp32 copies
+            // of every input (q^, k^ from the prologue, the others exact), so that
+            // the normalised rows keep their full precision
+            float* x32 = reinterpret_cast<float*>(fw + fused_f32_offset(P.B, P.T, P.H, P.D, P.C));
+            const long long n = rows * 128;
+            const void* src[7] = {P.q, P.k, P.v, P.g, P.e, P.w, P.gamma};
+            for (int i = 0; i < 7; ++i) {
+                e = i < 2 ? qk_materialise_gated(flags, src[i], x32 + i * n, rows, true, st)
+                          : upcast_gated(flags, src[i], x32 + i * n, n, false, st);
+                if (e != cudaSuccess) return e;
+            }
+            G.q = x32; G.k = x32 + n; G.v = x32 + 2 * n; G.g = x32 + 3 * n; G.e = x32 + 4 * n;
+            G.w = x32 + 5 * n; G.gamma = x32 + 6 * n;
+            G.in_bf16 = false;
+            e = fwd_f32_d128(G, S0, o, S_final, S_chunks, M_chunks, shared, st);
+        } else {
+            e = fwd_bf16_d128(G, S0, o, S_final, S_chunks, M_chunks, shared, st);
         }
-        if ((e = fwd_bf16_d128(G, S0, o, S_final, S_chunks, M_chunks, shared, st)) != cudaSuccess) return e;
+        if (e != cudaSuccess) return e;
         if (P.zo && o) return out_gate_fix_gated(flags, o, P.o_pre, P.zo, rows * 128, P.out_bf16, st);
         return cudaSuccess;
     }
@@ -163,7 +175,8 @@ cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S
         if (P.zo) {  // fused output gate: k2_bprep forms the mixer's dO and dzo
             if (!P.o_pre || !P.dzo) return cudaErrorInvalidValue;
             b.zo = P.zo; b.o_pre = P.o_pre; b.o_pre_f32 = P.o_pre_f32; b.dzo = P.dzo;
-            b.dO_eff = kh + rows * 128 * 2;
+            b.dO_eff = kh + rows * 128 * 2;  // fp16
+            b.dO_effb = qh;                  // bf16 (the q^ region is not used here)
         }
         char* rest = shared;
         if (P.aux && S_chunks) {  // intermediates saved by the forward
@@ -199,18 +212,35 @@ cudaError_t run_chunk_bwd(const ChunkProblem& P, const float* S0, const float* S
         if ((e = v2::run_bwd2(b, st)) != cudaSuccess) return e;
         ChunkProblem G = P;
         G.gate = flags;
-        if (P.qk_raw) {  // the boundary-pivot path reads q^, k^ and returns dq^, dk^
-            if ((e = qk_materialise_gated(flags, P.q, qh, rows, st)) != cudaSuccess) return e;
-            if ((e = qk_materialise_gated(flags, P.k, kh, rows, st)) != cudaSuccess) return e;
-            G.q = qh; G.k = kh;
-        }
-        const void* dO_mix = P.zo ? static_cast<const void*>(b.dO_eff) : dO;
-        if ((e = bwd_bf16_d128(G, S0, S_chunks, M_chunks, dO_mix, dS_final, dq, dk, dv, dg, de, dw,
-                               dgamma, dS0, shared, st)) != cudaSuccess)
-            return e;
+        const void* dO_mix = P.zo ? static_cast<const void*>(b.dO_effb) : dO;
         if (P.qk_raw) {
-            if ((e = qk_jacobian_gated(flags, P.q, dq, rows, st)) != cudaSuccess) return e;
-            if ((e = qk_jacobian_gated(flags, P.k, dk, rows, st)) != cudaSuccess) return e;
+            // the boundary-pivot path in fp32 on fp32 copies (as in the forward);
+            // its dq^, dk^ go through the prologue's Jacobian, the rest to bf16
+            float* x32 = reinterpret_cast<float*>(fw + fused_f32_offset(P.B, P.T, P.H, P.D, P.C));
+            const long long n = rows * 128;
+            // (the fused gate's dO from its fp16 copy)
+            const void* src[8] = {P.q, P.k, P.v, P.g, P.e, P.w, P.gamma, P.zo ? b.dO_eff : dO};
+            for (int i = 0; i < 8; ++i) {
+                e = i < 2 ? qk_materialise_gated(flags, src[i], x32 + i * n, rows, true, st)
+                          : upcast_gated(flags, src[i], x32 + i * n, n, i == 7 && P.zo, st);
+                if (e != cudaSuccess) return e;
+            }
+            G.q = x32; G.k = x32 + n; G.v = x32 + 2 * n; G.g = x32 + 3 * n; G.e = x32 + 4 * n;
+            G.w = x32 + 5 * n; G.gamma = x32 + 6 * n;
+            G.in_bf16 = false;
+            float* g32 = x32 + 8 * n;  // dq^, dk^, dv, dg, de, dw, dgamma
+            if ((e = bwd_f32_d128(G, S0, S_chunks, M_chunks, x32 + 7 * n, dS_final, g32, g32 + n,
+                                  g32 + 2 * n, g32 + 3 * n, g32 + 4 * n, g32 + 5 * n, g32 + 6 * n,
+                                  dS0, shared, st)) != cudaSuccess)
+                return e;
+            if ((e = qk_jacobian_gated(flags, P.q, g32, true, dq, rows, st)) != cudaSuccess) return e;
+            if ((e = qk_jacobian_gated(flags, P.k, g32 + n, true, dk, rows, st)) != cudaSuccess) return e;
+            void* outs[5] = {dv, dg, de, dw, dgamma};
+            for (int i = 0; i < 5; ++i)
+                if ((e = downcast_gated(flags, g32 + (2 + i) * n, outs[i], n, st)) != cudaSuccess) return e;
+        } else if ((e = bwd_bf16_d128(G, S0, S_chunks, M_chunks, dO_mix, dS_final, dq, dk, dv, dg, de,
+                                      dw, dgamma, dS0, shared, st)) != cudaSuccess) {
+            return e;
         }
         if (P.gate_proj)  // the projected gates' gradients -> latent, U, bias
             return v2::run_gates_bwd(*static_cast<const v2::GatesArgs*>(P.gate_proj), st);

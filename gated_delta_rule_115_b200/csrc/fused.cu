@@ -3,11 +3,13 @@
 // o * sigmoid(z); "Muir", wolonglab.org page, "Methodology" and fig. 3(b))
 // for the large-span fallback.  The on-chip kernels apply both stages
 // themselves; when a chunk's decay span sends the work to the boundary-pivot
-// path, that path needs q^ and k^ as tensors, its dq^ and dk^ mapped back
-// through the prologue, and its o gated.  Each kernel here reads the span flag
+// path, that path needs q^ and k^ as tensors (with raw q/k it runs in fp32 on
+// fp32 copies of every input, so that q^ and k^ keep full precision), its
+// dq^ and dk^ mapped back through the prologue, and its o gated.  Each kernel here reads the span flag
 // first and returns at once when it is clear, so in the common case they cost
 // one launch each and no memory traffic.
 #include <cuda_bf16.h>
+#include <cuda_fp16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 
@@ -47,9 +49,19 @@ __device__ __forceinline__ void store4(__nv_bfloat16* p, const float* v) {
     *reinterpret_cast<uint2*>(p) = u;
 }
 
+__device__ __forceinline__ void store4(float* p, const float* v) {
+    *reinterpret_cast<float4*>(p) = make_float4(v[0], v[1], v[2], v[3]);
+}
+
+__device__ __forceinline__ void load4(const float* p, float* v) {
+    const float4 u = *reinterpret_cast<const float4*>(p);
+    v[0] = u.x; v[1] = u.y; v[2] = u.z; v[3] = u.w;
+}
+
 // y = SiLU(x) r, r = 1 / ||SiLU(x)|| (the guard maps a zero row to zero).
+template <typename Ty>
 __global__ void __launch_bounds__(256) k_qk_mat(const int* flag, const __nv_bfloat16* x,
-                                                __nv_bfloat16* y, long long rows) {
+                                                Ty* y, long long rows) {
     if (*flag == 0) return;
     const int lane = threadIdx.x & 31;
     for (long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += (long long)gridDim.x * 8) {
@@ -68,9 +80,10 @@ __global__ void __launch_bounds__(256) k_qk_mat(const int* flag, const __nv_bflo
     }
 }
 
-// dy (gradient of y^) -> dx = SiLU'(x) r (dy - y^ (y^ . dy)), in place.
+// dy (gradient of y^) -> dx = SiLU'(x) r (dy - y^ (y^ . dy)) (bf16, may be dy).
+template <typename Td>
 __global__ void __launch_bounds__(256) k_qk_jac(const int* flag, const __nv_bfloat16* x,
-                                                __nv_bfloat16* dy, long long rows) {
+                                                const Td* dy, __nv_bfloat16* dx, long long rows) {
     if (*flag == 0) return;
     const int lane = threadIdx.x & 31;
     for (long long r = (long long)blockIdx.x * 8 + (threadIdx.x >> 5); r < rows; r += (long long)gridDim.x * 8) {
@@ -93,7 +106,39 @@ __global__ void __launch_bounds__(256) k_qk_jac(const int* flag, const __nv_bflo
 #pragma unroll
         for (int u = 0; u < 4; ++u)
             o[u] = (d[u] - sv[u] * rn * dot) * rn * sg[u] * (1.f + xv[u] * (1.f - sg[u]));
-        store4(dy + r * kD + 4 * lane, o);
+        store4(dx + r * kD + 4 * lane, o);
+    }
+}
+
+__device__ __forceinline__ void load4(const __half* p, float* v) {
+    const uint2 u = *reinterpret_cast<const uint2*>(p);
+    const __half2 a = *reinterpret_cast<const __half2*>(&u.x);
+    const __half2 b = *reinterpret_cast<const __half2*>(&u.y);
+    v[0] = __low2float(a); v[1] = __high2float(a); v[2] = __low2float(b); v[3] = __high2float(b);
+}
+
+// Exact bf16 (or fp16) -> fp32 copy (n a multiple of 4).
+template <typename Ts>
+__global__ void __launch_bounds__(256) k_upcast(const int* flag, const Ts* src, float* dst,
+                                                long long n4) {
+    if (*flag == 0) return;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (long long)gridDim.x * blockDim.x) {
+        float v[4];
+        load4(src + 4 * i, v);
+        store4(dst + 4 * i, v);
+    }
+}
+
+// fp32 -> bf16 (round to nearest even; n a multiple of 4).
+__global__ void __launch_bounds__(256) k_downcast(const int* flag, const float* src,
+                                                  __nv_bfloat16* dst, long long n4) {
+    if (*flag == 0) return;
+    for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n4;
+         i += (long long)gridDim.x * blockDim.x) {
+        float v[4];
+        load4(src + 4 * i, v);
+        store4(dst + 4 * i, v);
     }
 }
 
@@ -131,18 +176,53 @@ int grid_for(long long work, int per_block) {
 }  // namespace
 
 cudaError_t qk_materialise_gated(const int* flag, const void* x, void* y, long long rows,
-                                 cudaStream_t st) {
+                                 bool f32_out, cudaStream_t st) {
     if (rows <= 0) return cudaSuccess;
-    MUIR_TIMED("k_qk_mat", st, k_qk_mat<<<grid_for(rows, 8), 256, 0, st>>>(
-        flag, static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(y), rows));
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    if (f32_out) {
+        MUIR_TIMED("k_qk_mat", st, k_qk_mat<float><<<grid_for(rows, 8), 256, 0, st>>>(
+            flag, xb, static_cast<float*>(y), rows));
+    } else {
+        MUIR_TIMED("k_qk_mat", st, k_qk_mat<__nv_bfloat16><<<grid_for(rows, 8), 256, 0, st>>>(
+            flag, xb, static_cast<__nv_bfloat16*>(y), rows));
+    }
     return cudaGetLastError();
 }
 
-cudaError_t qk_jacobian_gated(const int* flag, const void* x, void* dy, long long rows,
-                              cudaStream_t st) {
+cudaError_t qk_jacobian_gated(const int* flag, const void* x, const void* dy, bool dy_f32,
+                              void* dx, long long rows, cudaStream_t st) {
     if (rows <= 0) return cudaSuccess;
-    MUIR_TIMED("k_qk_jac", st, k_qk_jac<<<grid_for(rows, 8), 256, 0, st>>>(
-        flag, static_cast<const __nv_bfloat16*>(x), static_cast<__nv_bfloat16*>(dy), rows));
+    const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+    __nv_bfloat16* out = static_cast<__nv_bfloat16*>(dx);
+    if (dy_f32) {
+        MUIR_TIMED("k_qk_jac", st, k_qk_jac<float><<<grid_for(rows, 8), 256, 0, st>>>(
+            flag, xb, static_cast<const float*>(dy), out, rows));
+    } else {
+        MUIR_TIMED("k_qk_jac", st, k_qk_jac<__nv_bfloat16><<<grid_for(rows, 8), 256, 0, st>>>(
+            flag, xb, static_cast<const __nv_bfloat16*>(dy), out, rows));
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t upcast_gated(const int* flag, const void* src, float* dst, long long n, bool src_f16,
+                         cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    if (n % 4) return cudaErrorInvalidValue;
+    if (src_f16) {
+        MUIR_TIMED("k_upcast", st, k_upcast<__half><<<grid_for(n / 4, 256), 256, 0, st>>>(
+            flag, static_cast<const __half*>(src), dst, n / 4));
+    } else {
+        MUIR_TIMED("k_upcast", st, k_upcast<__nv_bfloat16><<<grid_for(n / 4, 256), 256, 0, st>>>(
+            flag, static_cast<const __nv_bfloat16*>(src), dst, n / 4));
+    }
+    return cudaGetLastError();
+}
+
+cudaError_t downcast_gated(const int* flag, const float* src, void* dst, long long n, cudaStream_t st) {
+    if (n <= 0) return cudaSuccess;
+    if (n % 4) return cudaErrorInvalidValue;
+    MUIR_TIMED("k_downcast", st, k_downcast<<<grid_for(n / 4, 256), 256, 0, st>>>(
+        flag, src, static_cast<__nv_bfloat16*>(dst), n / 4));
     return cudaGetLastError();
 }
 

@@ -34,11 +34,16 @@ struct ChunkProblem {
 };
 
 // Workspace the fused stages add (inverse row norms, materialised q^ / k^ and
-// the mixer's dO for the large-span fallback).
-inline size_t fused_ws_bytes(int B, int T, int H, int D, int C) {
+// the mixer's dO for the large-span fallback; with raw q/k, fp32 copies of the
+// fallback's eight inputs and seven gradients).
+inline size_t fused_ws_bytes(int B, int T, int H, int D, int C, bool qk_raw) {
     const size_t nch = (size_t)B * H * ((T + C - 1) / C);
     const size_t rows = (size_t)B * T * H;
-    return 256 + nch * 2 * C * 4 + 3 * rows * D * 2;
+    return 256 + nch * 2 * C * 4 + 3 * rows * D * 2 + (qk_raw ? 15 * rows * D * 4 : 0);
+}
+// Offset of the fp32 region inside the fused workspace.
+inline size_t fused_f32_offset(int B, int T, int H, int D, int C) {
+    return fused_ws_bytes(B, T, H, D, C, false);
 }
 
 // Self-test of the bounded device waits (selftest.cu): one block waits
@@ -49,9 +54,12 @@ unsigned int timeouts_selftest();
 // Flag-gated helpers of the fused stages (fused.cu): each returns at once
 // unless *flag != 0 (the large-span fallback ran and needs them).
 cudaError_t qk_materialise_gated(const int* flag, const void* x, void* y, long long rows,
-                                 cudaStream_t st);
-cudaError_t qk_jacobian_gated(const int* flag, const void* x, void* dy, long long rows,
-                              cudaStream_t st);
+                                 bool f32_out, cudaStream_t st);
+cudaError_t qk_jacobian_gated(const int* flag, const void* x, const void* dy, bool dy_f32,
+                              void* dx, long long rows, cudaStream_t st);
+cudaError_t upcast_gated(const int* flag, const void* src, float* dst, long long n, bool src_f16,
+                         cudaStream_t st);
+cudaError_t downcast_gated(const int* flag, const float* src, void* dst, long long n, cudaStream_t st);
 cudaError_t out_gate_fix_gated(const int* flag, void* o, void* o_pre, const void* z, long long n,
                                bool out_bf16, cudaStream_t st);
 

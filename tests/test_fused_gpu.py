@@ -7,11 +7,9 @@ gradient in the backward's first kernel ("Muir", wolonglab.org page,
 
 Metric: max |gpu - oracle| / max |oracle| per tensor.  Bounds: 2e-3 on the
 forward outputs and the final state, 5e-3 on gradients (bf16 inputs, bf16
-gradients), as for the unfused path.  One branch is looser: with raw q/k, a
-chunk whose decay span exceeds the single pivot runs the boundary-pivot path
-on q^ and k^ rounded to bf16 (that path reads them as tensors), which adds up
-to one bf16 rounding (2^-9 relative) to every key and query entry; its bounds
-are 5e-3 and 1e-2.
+gradients), as for the unfused path, in every branch: with raw q/k, a chunk
+whose decay span exceeds the single pivot runs the boundary-pivot path in fp32
+on fp32 copies of q^, k^ and the other inputs.
 """
 import numpy as np
 import pytest
@@ -95,13 +93,11 @@ def test_fused_parity(muir, oracle_mod, wid, over, gate, raw, saved):
     errs.update({n: nmax(gr[n], gr_r[n]) for n in names})
     print(f"fused wid={wid} {over} gate={gate} raw={raw} saved={saved}: " +
           " ".join(f"{n} {v:.2e}" for n, v in errs.items()))
-    fallback_raw = wid == 3 and raw  # large spans with raw q/k: bf16-rounded q^, k^
-    tf, tb = (5e-3, 1e-2) if fallback_raw else (TOL_FWD, TOL_BWD)
     for n in ("o", "S", "o_pre"):
         if n in errs:
-            assert errs[n] < tf, (n, errs)
+            assert errs[n] < TOL_FWD, (n, errs)
     for n in names:
-        assert errs[n] < tb, (n, errs)
+        assert errs[n] < TOL_BWD, (n, errs)
 
 
 def test_fused_off_equals_plain_path(muir):
