@@ -388,6 +388,7 @@ def gpu_arm(args, rank, world, local):
         out["decode"] = decode_measure(muir, I, dev, peaks)
         out["qk_prologue"] = qk_measure(muir, dev, peaks)
         out["other_workloads"] = configs_measure(muir, I, dev, peaks)
+        out["fused_stages"] = fused_measure(muir, I, dev, peaks)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         threads = len(os.sched_getaffinity(0))
         v, desc, dt = oracle_sample(args.cpu_seconds, threads)
@@ -670,6 +671,47 @@ def configs_measure(muir, I, dev, peaks, steps=5, warmup=3):
             "ms": ms, "tokens_per_s": W3.B * W3.T / (ms / 1e3)}
         del wf, wb
     return out
+
+
+def fused_measure(muir, I, dev, peaks, steps=5, warmup=3):
+    """The long-context step with every fused stage on: raw q and k (the
+    SiLU + L2-norm prologue inside the chunk kernels) and the five gate
+    families projected from one latent row per token (R = 512, ranks 64, 64,
+    128, 128, 128; the output gate applied in the output epilogue).  Gate
+    inputs per token-head: the latent shared by the 16 heads (1,024 B / 16)
+    instead of four gate tensors (4 x 256 B)."""
+    import torch
+    W = I.WORKLOADS[WID]
+    x = I.fused_inputs(WID, with_dO=True)
+    lat, proj = I.gate_latent_inputs(W.B, W.T, W.H)
+    d = {k: (v.to(dev) if v is not None else None) for k, v in x.items()}
+    latd = lat.to(dev)
+    projd = {f: (off, U.to(dev), b.to(dev)) for f, (off, U, b) in proj.items()}
+    del x, lat
+    st = torch.cuda.current_stream(dev)
+
+    def step():
+        o, S, sv = muir.chunk_fwd_fused(d["xq"], d["xk"], d["v"], None, None, None, None, d["S0"],
+                                        qk_raw=True, latent=latd, proj=projd)
+        return muir.chunk_bwd_fused(d["xq"], d["xk"], d["v"], None, None, None, None, d["S0"],
+                                    d["dO"], qk_raw=True, saved=sv, latent=latd, proj=projd)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(st)
+    for _ in range(steps):
+        step()
+    b.record(st)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / steps
+    R = sum(I.GATE_RANKS.values())
+    return {"workload": f"long-context fwd+bwd B={W.B} H={W.H} T={W.T} d=128 chunk 128, raw q/k, "
+                        f"gates projected from a latent of R={R}",
+            "ms": ms, "tokens_per_s": W.B * W.T / (ms / 1e3),
+            "gate_input_bytes_per_token_head": R * 2 / W.H,
+            "gate_input_bytes_per_token_head_unfused": 4 * 128 * 2}
 
 
 def qk_measure(muir, dev, peaks, steps=20):

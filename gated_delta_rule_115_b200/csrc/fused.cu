@@ -24,7 +24,7 @@ constexpr int kD = 128;
 __device__ __forceinline__ float sig(float z) {
     float e;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-1.4426950408889634f * z));
-    return 1.f / (1.f + e);
+    return __fdividef(1.f, 1.f + e);
 }
 
 __device__ __forceinline__ float warp_sum(float v) {

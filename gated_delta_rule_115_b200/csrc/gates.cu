@@ -78,8 +78,9 @@ __device__ __forceinline__ void sync_all() {
     tc_fence_after();
 }
 
+// (fast intrinsics: the gates are stored in bf16)
 __device__ __forceinline__ float act_f(int act, float x) {
-    if (act == kActNegSoftplus) return -(fmaxf(x, 0.f) + log1pf(__expf(-fabsf(x))));
+    if (act == kActNegSoftplus) return -(fmaxf(x, 0.f) + __logf(1.f + __expf(-fabsf(x))));
     if (act == kActSigmoid) return sigmoid_f(x);
     return x;
 }
@@ -128,9 +129,9 @@ __device__ __forceinline__ unsigned char* align1024(unsigned char* p) {
 
 // ------------------------------------------------------------------ forward
 
-// 256 threads: warp w reads TMEM lanes 32 (w % 4) .. (rows t) and columns
-// 64 (w / 4) .. +64 (channels); thread 0 issues the copies and the products.
-__global__ void __launch_bounds__(256, 1) k2_gates(const __grid_constant__ GatesFwdParams p) {
+// 512 threads: warp w reads TMEM lanes 32 (w % 4) .. (rows t) and columns
+// 32 (w / 4) .. +32 (channels); thread 0 issues the copies and the products.
+__global__ void __launch_bounds__(512, 1) k2_gates(const __grid_constant__ GatesFwdParams p) {
     extern __shared__ unsigned char smraw[];
     unsigned char* sm = align1024(smraw);
     __shared__ uint64_t barA, barU[2], barM[2];
@@ -187,13 +188,14 @@ __global__ void __launch_bounds__(256, 1) k2_gates(const __grid_constant__ Gates
         if (tid == 0 && idx + 1 < n) issue(idx + 1);  // into the other accumulator
         if (!cta_wait(&barM[s], (uint32_t)((idx >> 1) & 1)) && tid == 0) bad = 1;
         if (tid == 0 && idx + 2 < n) load_U(idx + 2, s);  // product idx has read stage s
-        float v[64];
-        tm_ld64(tm + 128 * s + 64 * half, q, 0, v);
-        const float* bias = p.bias[X] + 128 * h + 64 * half;
-        __nv_bfloat16* dst = p.out[X] + ((row0 + t) * p.H + h) * 128 + 64 * half;
+        float v[32];
+        tmem_ld32(taddr(tm, 32 * q, 128 * s + 32 * half), v);
+        tmem_wait_ld();
+        const float* bias = p.bias[X] + 128 * h + 32 * half;
+        __nv_bfloat16* dst = p.out[X] + ((row0 + t) * p.H + h) * 128 + 32 * half;
         const int act = p.act[X];
 #pragma unroll
-        for (int j = 0; j < 64; j += 8) {
+        for (int j = 0; j < 32; j += 8) {
             float o[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) o[u] = act_f(act, v[j + u] + __ldg(bias + j + u));
@@ -208,8 +210,9 @@ __global__ void __launch_bounds__(256, 1) k2_gates(const __grid_constant__ Gates
 
 // ------------------------------------------------------------------ backward
 
-// dpre = dgate act'(pre) and dlatent, one 128-token tile per CTA.
-__global__ void __launch_bounds__(256, 1) k2_gates_dpre(const __grid_constant__ GatesDpreParams p) {
+// dpre = dgate act'(pre) and dlatent, one 128-token tile per CTA; 512
+// threads (warp w: TMEM lanes 32 (w % 4) .., channels 32 (w / 4) ..).
+__global__ void __launch_bounds__(512, 1) k2_gates_dpre(const __grid_constant__ GatesDpreParams p) {
     extern __shared__ unsigned char smraw[];
     unsigned char* sm = align1024(smraw);
     unsigned char* A = sm;                 // the family's latent slice (2 blocks)
@@ -259,13 +262,14 @@ __global__ void __launch_bounds__(256, 1) k2_gates_dpre(const __grid_constant__ 
             }
             if (!cta_wait(&barM, pm) && tid == 0) bad = 1;
             pm ^= 1u;
-            {  // dpre of row t, channels 64 half .. +64 -> global and the Dp tile
-                float v[64];
-                tm_ld64(tm + 64 * half, q, 0, v);
-                const size_t ro = ((size_t)(row0 + t) * p.H + h) * 128 + 64 * half;
-                const float* bias = p.bias[X] + 128 * h + 64 * half;
+            {  // dpre of row t, channels 32 half .. +32 -> global and the Dp tile
+                float v[32];
+                tmem_ld32(taddr(tm, 32 * q, 32 * half), v);
+                tmem_wait_ld();
+                const size_t ro = ((size_t)(row0 + t) * p.H + h) * 128 + 32 * half;
+                const float* bias = p.bias[X] + 128 * h + 32 * half;
 #pragma unroll
-                for (int j = 0; j < 64; j += 8) {
+                for (int j = 0; j < 32; j += 8) {
                     float dg[8], hi[8], lo[8];
                     ld8_bf16g(p.dout[X] + ro + j, dg);
 #pragma unroll
@@ -276,8 +280,8 @@ __global__ void __launch_bounds__(256, 1) k2_gates_dpre(const __grid_constant__ 
                     }
                     st8_bf16g(p.dpre[X] + ro + j, hi);
                     st8_bf16g(p.dpre_lo[X] + ro + j, lo);
-                    st_chunk16<true>(Dp, t, 8 * half + j / 8, hi);
-                    st_chunk16<true>(Dp + 2 * kBlk, t, 8 * half + j / 8, lo);
+                    st_chunk16<true>(Dp, t, 4 * half + j / 8, hi);
+                    st_chunk16<true>(Dp + 2 * kBlk, t, 4 * half + j / 8, lo);
                 }
             }
             fence_async_smem();
@@ -291,12 +295,18 @@ __global__ void __launch_bounds__(256, 1) k2_gates_dpre(const __grid_constant__ 
             pm ^= 1u;
             if (tid == 0 && h + 2 < p.H) load_U(idx + 2);  // both products of head h read stage s
         }
-        {  // dlatent of row t: columns off .. off + r (half of them per thread)
-            const int w = r / 2;
-            float v[64];
-            tm_ld64(tm + 128 + w * half, q, 0, v);  // w <= 64 columns used
+        {  // dlatent of row t: columns off .. off + r (a quarter of them per thread)
+            const int w = r / 4;  // 16 or 32
+            float v[32];
+            tmem_ld32(taddr(tm, 32 * q, 128 + w * half), v);  // w <= 32 columns used
+            tmem_wait_ld();
             __nv_bfloat16* dst = p.dlat + (size_t)(row0 + t) * p.R + p.off[X] + w * half;
-            for (int j = 0; j < w; j += 8) st8_bf16g(dst + j, v + j);
+            st8_bf16g(dst, v);
+            st8_bf16g(dst + 8, v + 8);
+            if (w == 32) {
+                st8_bf16g(dst + 16, v + 16);
+                st8_bf16g(dst + 24, v + 24);
+            }
         }
         sync_all();
     }
@@ -408,7 +418,7 @@ cudaError_t run_gates_fwd(const GatesArgs& a, cudaStream_t st) {
     const int smem = (nblk + 4) * (int)kBlk + 1024;
     cudaError_t e = cudaFuncSetAttribute(k2_gates, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
-    MUIR_TIMED("k2_gates", st, k2_gates<<<(int)(a.rows / 128), 256, smem, st>>>(p));
+    MUIR_TIMED("k2_gates", st, k2_gates<<<(int)(a.rows / 128), 512, smem, st>>>(p));
     return cudaGetLastError();
 }
 
@@ -439,7 +449,7 @@ cudaError_t run_gates_bwd(const GatesArgs& a, cudaStream_t st) {
     if (e != cudaSuccess) return e;
     const int smem1 = 10 * (int)kBlk + 1024;
     if ((e = cudaFuncSetAttribute(k2_gates_dpre, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1)) != cudaSuccess) return e;
-    MUIR_TIMED("k2_gates_dpre", st, k2_gates_dpre<<<(int)(a.rows / 128), 256, smem1, st>>>(p));
+    MUIR_TIMED("k2_gates_dpre", st, k2_gates_dpre<<<(int)(a.rows / 128), 512, smem1, st>>>(p));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
     const int smem2 = 12 * (int)kBlk + 1024;
     if ((e = cudaFuncSetAttribute(k2_gates_dw, cudaFuncAttributeMaxDynamicSharedMemorySize, smem2)) != cudaSuccess) return e;

@@ -137,11 +137,12 @@ __device__ __forceinline__ void bulk_wait_all() {
 }
 
 // Logistic sigmoid 1 / (1 + e^-z) through the base-2 exponential
-// (e^-z = 2^(-z log2 e)); saturates to 0 and 1 without NaN.
+// (e^-z = 2^(-z log2 e)) and a fast division (a few ulp; its results feed
+// 16-bit operands or bf16 gates); saturates to 0 and 1 without NaN.
 __device__ __forceinline__ float sigmoid_f(float z) {
     float e;
     asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-1.4426950408889634f * z));
-    return 1.f / (1.f + e);
+    return __fdividef(1.f, 1.f + e);
 }
 
 // Fetch the 128-byte line holding `ptr` into L2 (no register result).

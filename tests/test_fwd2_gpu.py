@@ -19,6 +19,16 @@ def nmax(a, r):
     return float(np.abs(a - r).max() / max(np.abs(r).max(), 1e-300))
 
 
+def elem_rel(a, r):
+    """Elementwise relative error with a floor of 1e-3 max|r| (the second
+    metric of the parity reading: logged, and below 1, i.e. no element is off
+    by as much as its own magnitude where that is above the floor)."""
+    a = a.double().cpu().numpy() if hasattr(a, "cpu") else np.asarray(a)
+    r = np.asarray(r)
+    floor = 1e-3 * max(np.abs(r).max(), 1e-300)
+    return float((np.abs(a - r) / np.maximum(np.abs(r), floor)).max())
+
+
 @pytest.fixture(scope="module")
 def muir():
     import gated_delta_rule_115_b200 as m
@@ -56,8 +66,11 @@ def test_fwd2_parity(muir, oracle_mod, wid, over):
     ro, rS, rSc = oracle_mod.chunk_fwd(*[x[n] for n in NAMES], S0=x["S0"], chunk=128)
     torch.cuda.synchronize()
     eo, eS, eC = nmax(o, ro), nmax(S, rS), nmax(Sc, rSc)
-    print(f"fwd2 wid={wid} {over}: o {eo:.2e} S {eS:.2e} chunk states {eC:.2e}")
+    lo, lS = elem_rel(o, ro), elem_rel(S, rS)
+    print(f"fwd2 wid={wid} {over}: o {eo:.2e} S {eS:.2e} chunk states {eC:.2e}; "
+          f"elementwise (floor 1e-3 max): o {lo:.2e} S {lS:.2e}")
     assert eo < TOL and eS < TOL and eC < TOL
+    assert lo < 1.0 and lS < 1.0
 
 
 def test_fwd2_many_chunks_per_cta(muir, oracle_mod):
