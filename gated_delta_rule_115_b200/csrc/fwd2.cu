@@ -85,7 +85,7 @@ struct IntraSmem {
     int bad;
 };
 
-enum { BA = 0, BB, BC, BD, BE, BF, BM1, BM2, BM3, BM4, BM5, BM6, BG };
+enum { BA = 0, BB, BC, BD, BE, BF, BM1, BM2, BM3, BM4, BM5, BM6, BG, BL };
 
 // All threads call: warp 0 polls, the block barrier releases the rest.
 __device__ __forceinline__ bool waitb(IntraSmem& s, int i, uint32_t parity) {
@@ -255,43 +255,51 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         const size_t rbase = (size_t)c * kC * kD + (size_t)t * kD + c0;  // row t, column c0
 
         // ---- 1. log-decay prefix (warp scan over tokens), pivots
+        // L = Tril(1) g: the inclusive prefix over the chunk's tokens as one
+        // tensor-core product (clamped g and the ones are exact in bf16; fp32
+        // accumulation), the ones tile in S5 (free until phase 2)
         waitb(s, BA, ph);
-        float L[32];
-        ld32(S[0], L);
+        {
+            float v[8];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) L[j] = fmaxf(L[j], kLogDecayMin) * kLog2e;
+            for (int i = 0; i < 4; ++i) {
+                ld_chunk16<true>(S[0], t, 4 * h + i, v);
 #pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
+                for (int u = 0; u < 8; ++u) v[u] = fmaxf(v[u], kLogDecayMin);
+                st_chunk16<true>(S[0], t, 4 * h + i, v);
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                const float o = __shfl_up_sync(0xffffffffu, L[j], off);
-                if (lane >= off) L[j] += o;
+                for (int u = 0; u < 8; ++u) v[u] = (c0 + 8 * i + u <= t) ? 1.f : 0.f;
+                st_chunk16<true>(S[5], t, 4 * h + i, v);
             }
         }
-        if (lane == 31) {
-#pragma unroll
-            for (int j = 0; j < 32; ++j) s.tot[q][c0 + j] = L[j];
-        }
         if (QKRAW) s.nrm[h][t] = silu_sq32(S[1], t, h);
-        __syncthreads();
+        fence_async_smem();
+        sync_all();
+        if (tid == 0) {
+            gemm_km16(tm + 0, a5, 0, a0, 0, 0, 128, 128, kBF16, false);
+            mma_commit(&s.bar[BL]);
+        }
         const float rk = QKRAW ? row_rnorm(s.nrm, t) : 1.f;
         if (QKRAW && h == 0) p.rnorm[(size_t)c * 2 * kC + kC + t] = rk;
+        waitb(s, BL, ph);
+        float L[32];
+        tm_ld32w(tm, q, c0, L);
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-            float pre = 0.f;
-            for (int qq = 0; qq < q; ++qq) pre += s.tot[qq][c0 + j];
-            L[j] += pre;
-        }
-        if (q == 0) {
-            const int col = c0 + lane;
-            const float lb = s.tot[0][col] + s.tot[1][col] + s.tot[2][col] + s.tot[3][col];
-            s.Lb[col] = lb;
-            s.P2[col] = 0.5f * lb;
-            s.eP2[col] = ex2(0.5f * lb);
+        for (int j = 0; j < 32; ++j) L[j] *= kLog2e;
+        if (t == kC - 1) {  // the chunk totals: the last row
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+                s.Lb[c0 + j] = L[j];
+                s.P2[c0 + j] = 0.5f * L[j];
+                s.eP2[c0 + j] = ex2(0.5f * L[j]);
+            }
+            bool far = false;
+#pragma unroll
+            for (int j = 0; j < 32; ++j) far |= L[j] < -kSpanMax * kLog2e;
             // a span beyond the single pivot sends the call to the boundary-pivot path
-            if (__any_sync(0xffffffffu, lb < -kSpanMax * kLog2e) && lane == 0) atomicOr(p.flags, 1);
+            if (far) atomicOr(p.flags, 1);
         }
-        __syncthreads();
+        sync_all();
 
         // ---- 2. pivoted key operands: Kp -> S0, Km (hi) -> S1, Km (lo) -> S2, Am -> S5
 #pragma unroll 1
