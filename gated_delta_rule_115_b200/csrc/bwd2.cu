@@ -182,42 +182,6 @@ __device__ __forceinline__ void tm_ld32w(uint32_t tm, int q, int col, float (&v)
     tmem_wait_ld();
 }
 
-// Chunk-local cumulative log decay (log2 units) of this thread's row t and W
-// channels j0..j0+W-1, by a warp scan over tokens plus the totals of the
-// earlier 32-token quarters (tot: [4][128] floats in shared memory, written
-// here).  Ends after a block barrier; tot then holds the quarter totals.
-template <int W>
-__device__ __forceinline__ void log_decay(const __nv_bfloat16* g, int lane, int q, int j0,
-                                          float (*tot)[kD], float (&L)[W]) {
-#pragma unroll
-    for (int i = 0; i < W / 8; ++i) ld8_bf16(g + j0 + 8 * i, L + 8 * i);
-#pragma unroll
-    for (int j = 0; j < W; ++j) L[j] = fmaxf(L[j], kLogDecayMin) * kLog2e;
-#pragma unroll
-    for (int off = 1; off < 32; off <<= 1) {
-#pragma unroll
-        for (int j = 0; j < W; ++j) {
-            const float o = __shfl_up_sync(0xffffffffu, L[j], off);
-            if (lane >= off) L[j] += o;
-        }
-    }
-    if (lane == 31) {
-#pragma unroll
-        for (int j = 0; j < W; ++j) tot[q][j0 + j] = L[j];
-    }
-    __syncthreads();
-#pragma unroll
-    for (int j = 0; j < W; ++j) {
-        float pre = 0.f;
-        for (int qq = 0; qq < q; ++qq) pre += tot[qq][j0 + j];
-        L[j] += pre;
-    }
-}
-
-__device__ __forceinline__ float chunk_total(float (*tot)[kD], int j) {
-    return tot[0][j] + tot[1][j] + tot[2][j] + tot[3][j];
-}
-
 }  // namespace
 
 // ------------------------------------------------------------------ k2_bprep
@@ -439,14 +403,13 @@ __global__ void __launch_bounds__(128, 1) k2_chain_rev(const __grid_constant__ R
 
 namespace {
 struct Bwd1Smem {
-    float tot[4][kD];
     float Lb[kD];
     float red[16];
-    uint64_t bar[16];
+    uint64_t bar[20];
     uint32_t tslot;
     int bad;
 };
-enum { B1D = 0, B1W, B1U, B1Q, B1A, B1T, B1K, B1L, B1KB, B1M1, B1M2, B1M3, B1M4, B1M5, B1M6 };
+enum { B1D = 0, B1W, B1U, B1Q, B1A, B1T, B1K, B1L, B1KB, B1M1, B1M2, B1M3, B1M4, B1M5, B1M6, B1G, B1LM };
 
 // Largest |x| over the block (512 threads, 32 values each); ends with a barrier.
 __device__ __forceinline__ float block_absmax(const float (&v)[32], float* red, int warp, int lane) {
@@ -485,7 +448,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
     const int q = warp & 3, h = warp >> 2, t = 32 * q + lane, c0 = 32 * h;
     const int N = p.T / kC, nch = p.B * p.H * N;
     if (tid == 0) {
-        for (int i = 0; i < 16; ++i) mbar_init(&s.bar[i], 1);
+        for (int i = 0; i < 20; ++i) mbar_init(&s.bar[i], 1);
         s.bad = 0;
         fence_barrier_init();
         prefetch_tmap(&p.tdO);
@@ -524,11 +487,45 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             bulk(S[2], ax + AuxLayout::kW16, B1W);
             bulk(S[4], ax + AuxLayout::kU16, B1U);
             bulk(S[5], ax + AuxLayout::kMQA16, B1Q);
+            mbar_arrive_expect_tx(&s.bar[B1G], kT16Bytes);  // g -> S0 (free until the state tile)
+            tma_load_3d(S[0], &p.tg, 0, hd, z, &s.bar[B1G]);
+            tma_load_3d(S[0] + kT16Block, &p.tg, 64, hd, z, &s.bar[B1G]);
         }
-        // log decay of row t, columns c0..; E = 2^L, Eb = 2^(Lbar - L)
+        // log decay of row t, columns c0..: L = Tril(1) clamp(g) as one product
+        // (ones tile in S3, free until the gradient-state tile); E = 2^L,
+        // Eb = 2^(Lbar - L), Lbar = the product's last row
         float L[32];
-        log_decay<32>(reinterpret_cast<const __nv_bfloat16*>(p.g) + tok * kD, lane, q, c0, s.tot, L);
-        if (q == 0) s.Lb[c0 + lane] = chunk_total(s.tot, c0 + lane);
+        {
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = (c0 + 8 * i + u <= t) ? 1.f : 0.f;
+                st_chunk16<true>(S[3], t, 4 * h + i, v);
+            }
+            waitb(B1G, ph);
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                ld_chunk16<true>(S[0], t, 4 * h + i, v);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) v[u] = fmaxf(v[u], kLogDecayMin);
+                st_chunk16<true>(S[0], t, 4 * h + i, v);
+            }
+            fence_async_smem();
+            sync_all();
+            if (tid == 0) {
+                gemm_km16(tm + 0, a[3], 0, a[0], 0, 0, 128, 128, kBF16, false);
+                mma_commit(&s.bar[B1LM]);
+            }
+            waitb(B1LM, ph);
+            tm_ld32w(tm, q, c0, L);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) L[j] *= kLog2e;
+            if (t == kC - 1) {
+#pragma unroll
+                for (int j = 0; j < 32; ++j) s.Lb[c0 + j] = L[j];
+            }
+        }
         // S_n / sS -> fp16 tile S0, G / sG -> fp16 tile S3 (row j = t)
         float sS, sG;
         {
@@ -719,7 +716,6 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
 
 namespace {
 struct Bwd2Smem {
-    float tot[4][kD];
     float P2[kD];
     float sfx[4][kD];  // per-quarter totals of the reverse scan
     float dgb[kD];     // dLbar of the chunk (value slabs summed in a fixed order)
@@ -728,7 +724,7 @@ struct Bwd2Smem {
     uint32_t tslot;
     int bad;
 };
-enum { B2IN = 0, B2M };
+enum { B2IN = 0, B2M, B2G };
 // which part of a dL product survives, for row r and column col:
 // col < r, col <= r, col > r, col >= r
 enum { kStrictLow = 0, kInclLow, kStrictUp, kInclUp };
@@ -899,14 +895,55 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
         for (int hj = 0; hj < 2; ++hj) {
             const int j0 = 64 * hj + 16 * g4;  // this thread's channels
             const int r0 = 16 * g4;            // their rows in the half tiles
+            // log decay of the half's 64 channels: L = Tril(1) clamp(g) as one
+            // product (g block in Bt1, ones tile in Bt0: both free until the
+            // pivoted operands; TMEM columns 0..63 free until the first round)
+            if (tid == 0) {
+                mbar_arrive_expect_tx(&s.bar[B2G], kT16Block);
+                tma_load_3d(Bt1, &p.tg, 64 * hj, hd, b * p.T + n * kC, &s.bar[B2G]);
+            }
+            {
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) v[u] = (32 * g4 + 8 * i + u <= t) ? 1.f : 0.f;
+                    st_chunk16<true>(Bt0, t, 4 * g4 + i, v);
+                }
+            }
+            if (!cta_wait(&s.bar[B2G], (uint32_t)((2 * it + hj) & 1)) && tid == 0) atomicOr(&s.bad, 1 << 26);
+            {
+                float v[8];
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {  // row t, channels 16 g4 .. +16 of the block
+                    ld_chunk16<true>(Bt1, t, 2 * g4 + i, v);
+#pragma unroll
+                    for (int u = 0; u < 8; ++u) v[u] = fmaxf(v[u], kLogDecayMin);
+                    st_chunk16<true>(Bt1, t, 2 * g4 + i, v);
+                }
+            }
+            fence_async_smem();
+            sync_all();
+            if (tid == 0) {
+                gemm_km16(tm + 0, aB0, 0, aB1, 0, 0, 64, 128, kBF16, false);
+                mma_commit(&s.bar[B2M]);
+            }
+            mma_wait();
             float L[16];
-            log_decay<16>(reinterpret_cast<const __nv_bfloat16*>(p.g) + tok * kD, lane, q, j0, s.tot, L);
-            if (q == 0 && lane < 16) {
-                const float lb = chunk_total(s.tot, j0 + lane);
-                s.P2[j0 + lane] = 0.5f * lb;
-                // (the forward's test, on the same sums: the call then also runs the
-                // boundary-pivot path, which overwrites this kernel's results)
-                if (lb < -kSpanMax * kLog2e) atomicOr(p.flags, 1);
+            tmem_ld16(taddr(tm, 32 * q, 16 * g4), L);
+            tmem_wait_ld();
+#pragma unroll
+            for (int u = 0; u < 16; ++u) L[u] *= kLog2e;
+            if (t == kC - 1) {  // the chunk totals: the last row
+                bool far = false;
+#pragma unroll
+                for (int u = 0; u < 16; ++u) {
+                    s.P2[j0 + u] = 0.5f * L[u];
+                    far |= L[u] < -kSpanMax * kLog2e;
+                }
+                // (the forward's test: the call then also runs the boundary-pivot
+                // path, which overwrites this kernel's results)
+                if (far) atomicOr(p.flags, 1);
             }
             __syncthreads();
             const __nv_bfloat16* kin = reinterpret_cast<const __nv_bfloat16*>(p.k) + tok * kD + j0;
@@ -1194,6 +1231,7 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     const int grid = nch < nsm ? nch : nsm;
     Bwd1Params p1;
     p1.tdO = tdO; p1.B = a.B; p1.T = a.T; p1.H = a.H;
+    if (!map_tokens16(&p1.tg, a.g, a.B, a.T, a.H)) return cudaErrorInvalidValue;
     p1.q = a.q; p1.k = a.k; p1.v = a.v; p1.g = a.g; p1.e = a.e; p1.w = a.w; p1.gamma = a.gamma;
     p1.aux = a.aux; p1.S_chunks = a.S_chunks; p1.dSc = dSc;
     p1.Pq = P16[0]; p1.Pk = P16[1]; p1.Pa = P16[2]; p1.Pd = P16[3];
@@ -1207,6 +1245,7 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
 
     Bwd2Params p2;
     p2.tdO = tdO; p2.B = a.B; p2.T = a.T; p2.H = a.H;
+    if (!map_tokens16(&p2.tg, a.g, a.B, a.T, a.H)) return cudaErrorInvalidValue;
     p2.q = a.q; p2.k = a.k; p2.g = a.g; p2.e = a.e; p2.gamma = a.gamma;
     p2.aux = a.aux; p2.Y16 = Y16; p2.dYR16 = dYR16;
     p2.Pq = P16[0]; p2.Pk = P16[1]; p2.Pa = P16[2]; p2.Pd = P16[3];

@@ -40,7 +40,7 @@ struct RevParams {
 };
 
 struct Bwd1Params {
-    CUtensorMap tdO;
+    CUtensorMap tdO, tg;                  // dO, and g (the log decay) as token-major bf16 tiles
     int B, T, H;
     const void *q, *k, *v, *g, *e, *w, *gamma;
     const unsigned char* aux;
@@ -56,7 +56,7 @@ struct Bwd1Params {
 };
 
 struct Bwd2Params {
-    CUtensorMap tdO;
+    CUtensorMap tdO, tg;
     int B, T, H;
     const void *q, *k, *g, *e, *gamma;
     const unsigned char* aux;
