@@ -94,11 +94,22 @@ __device__ __forceinline__ void prologue8(float* v, float r) {
     for (int u = 0; u < 8; ++u) v[u] = v[u] * sigmoid_f(v[u]) * r;
 }
 
+// The scaled fp16 partials are kept channel-group-major within a chunk:
+// element (t, ch) of chunk c is half 8 (c kD/8 kC + (ch/8) kC + t) + ch % 8,
+// so that one 8-channel group of 32 consecutive rows is one contiguous
+// 512-byte run (each warp's access, on both sides, is coalesced); the scale
+// of (t, 32-channel group ch/32) sits at c 4 kC + (ch/32) kC + t.
+__device__ __forceinline__ size_t pgrp(int c, int t, int ch) {  // in 16-byte words
+    return (size_t)c * (kC * kD / 8) + (size_t)(ch >> 3) * kC + t;
+}
+__device__ __forceinline__ size_t psc(int c, int t, int ch) { return (size_t)c * 4 * kC + (size_t)(ch >> 5) * kC + t; }
+
 // 32 values as fp16 times a power of two: the scale puts the largest
 // magnitude just below 2^15 (fp16 keeps 11 significant bits of every value
 // within 2^-14 of it; the sums these partials join are dominated by larger
-// terms).  dst: 32 halves (64 bytes, 16-byte aligned); *scale: the factor.
-__device__ __forceinline__ void st_scaled32(__half* dst, float* scale, const float* v) {
+// terms).  dst: the first of 4 groups of 8 halves, kC words apart; *scale:
+// the factor.
+__device__ __forceinline__ void st_scaled32(uint4* dst, float* scale, const float* v) {
     float m = 0.f;
 #pragma unroll
     for (int j = 0; j < 32; ++j) m = fmaxf(m, fabsf(v[j]));
@@ -114,13 +125,13 @@ __device__ __forceinline__ void st_scaled32(__half* dst, float* scale, const flo
         u.y = pack_f16(v[8 * i + 2] * inv, v[8 * i + 3] * inv);
         u.z = pack_f16(v[8 * i + 4] * inv, v[8 * i + 5] * inv);
         u.w = pack_f16(v[8 * i + 6] * inv, v[8 * i + 7] * inv);
-        reinterpret_cast<uint4*>(dst)[i] = u;
+        dst[i * kC] = u;
     }
 }
 
 // The same for the two groups a + b and a - b (each with its own scale),
 // without forming them in registers first.
-__device__ __forceinline__ void st_scaled32_pm(__half* dp, float* sp, __half* dm, float* sm_,
+__device__ __forceinline__ void st_scaled32_pm(uint4* dp, float* sp, uint4* dm, float* sm_,
                                                const float* a, const float* b) {
     float mp = 0.f, mm = 0.f;
 #pragma unroll
@@ -148,14 +159,14 @@ __device__ __forceinline__ void st_scaled32_pm(__half* dp, float* sp, __half* dm
         w.y = pack_f16((a[j + 2] - b[j + 2]) * im, (a[j + 3] - b[j + 3]) * im);
         w.z = pack_f16((a[j + 4] - b[j + 4]) * im, (a[j + 5] - b[j + 5]) * im);
         w.w = pack_f16((a[j + 6] - b[j + 6]) * im, (a[j + 7] - b[j + 7]) * im);
-        reinterpret_cast<uint4*>(dp)[i] = u;
-        reinterpret_cast<uint4*>(dm)[i] = w;
+        dp[i * kC] = u;
+        dm[i * kC] = w;
     }
 }
 
 // 8 scaled fp16 values -> floats.
-__device__ __forceinline__ void ld8_scaled(const __half* p, float sc, float* v) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
+__device__ __forceinline__ void ld8_scaled(const uint4* p, float sc, float* v) {
+    const uint4 u = __ldg(p);
     unpack16<false>(u.x, v[0], v[1]);
     unpack16<false>(u.y, v[2], v[3]);
     unpack16<false>(u.z, v[4], v[5]);
@@ -473,7 +484,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
         const size_t tok = ((size_t)b * p.T + (size_t)n * kC + t) * p.H + hd;  // token-major row
         const size_t ro = tok * kD + c0;                                      // this thread's 32 elements
         const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + c0;          // per-chunk arrays
-        const size_t scb = ((size_t)c * kC + t) * 4 + h;                      // their group scales
+        const size_t pb = pgrp(c, t, c0), scb = psc(c, t, c0);               // partials, their scales
         const unsigned char* ax = p.aux + (size_t)c * AuxLayout::kBytes;
         unsigned char* y16 = p.Y16 + (size_t)c * kT16Bytes;
         unsigned char* r16 = p.dYR16 + (size_t)c * kT16Bytes;
@@ -577,7 +588,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             tm_ld32w(tm, q, c0, d);
 #pragma unroll
             for (int j = 0; j < 32; ++j) d[j] *= sS * ex2(L[j]);
-            st_scaled32(p.Pq + cb, p.sq + scb, d);
+            st_scaled32(reinterpret_cast<uint4*>(p.Pq) + pb, p.sq + scb, d);
             tm_ld32w(tm, q, 128 + c0, d);
             const float* up = reinterpret_cast<const float*>(ax + AuxLayout::kUp) + (size_t)t * kD + c0;
 #pragma unroll
@@ -611,7 +622,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             tm_ld32w(tm, q, 128 + c0, d);  // dAbar / sG
 #pragma unroll
             for (int j = 0; j < 32; ++j) d[j] *= sG * ex2(s.Lb[c0 + j] - L[j]);
-            st_scaled32(p.Pa + cb, p.sa + scb, d);
+            st_scaled32(reinterpret_cast<uint4*>(p.Pa) + pb, p.sa + scb, d);
         }
         waitb(B1A, ph);  // (its block barrier also orders the reads of B1 above)
         // ---- phase 4: Abar G / sG (B0); dY = -M_QA^T dO - Abar G
@@ -670,7 +681,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
                 d[j] *= sS * ex2(L[j]);                    // dK~ 2^L
                 e2[j] *= sG * ex2(s.Lb[c0 + j] - L[j]);  // dKbar 2^(Lbar-L)
             }
-            st_scaled32_pm(p.Pk + cb, p.sk + scb, p.Pd + cb, p.sd + scb, d, e2);  // Pk, Pd
+            st_scaled32_pm(reinterpret_cast<uint4*>(p.Pk) + pb, p.sk + scb, reinterpret_cast<uint4*>(p.Pd) + pb, p.sd + scb, d, e2);  // Pk, Pd
         }
         waitb(B1L, ph);
         waitb(B1KB, ph);
@@ -707,6 +718,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
         sync_all();
     }
     if (tid == 0) bulk_wait_all();
+    if (tid == 0) bulk_wait_all();
     if (tid == 0 && s.bad) atomicOr(&g_bwd2_timeouts, (unsigned)s.bad);
     sync_all();
     if (warp == 0) tmem_dealloc(tm, 512);
@@ -724,7 +736,7 @@ struct Bwd2Smem {
     uint32_t tslot;
     int bad;
 };
-enum { B2IN = 0, B2M, B2G };
+enum { B2IN = 0, B2M, B2G, B2X };
 // which part of a dL product survives, for row r and column col:
 // col < r, col <= r, col > r, col >= r
 enum { kStrictLow = 0, kInclLow, kStrictUp, kInclUp };
@@ -1001,35 +1013,47 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             }
             // the second half's rounds were the tiles' last readers
             if (hj == 1 && tid == 0 && c + (int)gridDim.x < nch) load_tiles(c + gridDim.x);
-            // ---- readout: final gradients of channels j0 .. j0 + 15 of row t
+            // ---- readout: final gradients of channels j0 .. j0 + 15 of row t.
+            // k, e (Bt0) and q, gamma (Bt1) of the half come by TMA into the
+            // operand tiles, free now; each thread forms its gradients in the
+            // places of its own inputs and the tiles leave by TMA store.
+            if (tid == 0) {
+                const int z = b * p.T + n * kC;
+                mbar_arrive_expect_tx(&s.bar[B2X], 4 * kT16Block);
+                tma_load_3d(Bt0, &p.tk, 64 * hj, hd, z, &s.bar[B2X]);
+                tma_load_3d(Bt0 + kT16Block, &p.te, 64 * hj, hd, z, &s.bar[B2X]);
+                tma_load_3d(Bt1, &p.tq, 64 * hj, hd, z, &s.bar[B2X]);
+                tma_load_3d(Bt1 + kT16Block, &p.tgam, 64 * hj, hd, z, &s.bar[B2X]);
+            }
             {
                 const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + j0;
                 const size_t ro = tok * kD + j0;
-                const size_t scb = ((size_t)c * kC + t) * 4 + (j0 >> 5);  // channels j0 .. +16 share a group
+                const size_t scb = psc(c, t, j0);  // channels j0 .. +16 share a group
                 const float s_q = __ldg(p.sq + scb), s_k = __ldg(p.sk + scb);
                 const float s_a = __ldg(p.sa + scb), s_d = __ldg(p.sd + scb);
                 float dL[16];
                 float dotq = 0.f, dotk = 0.f;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {  // 8 channels at a time
-                    const int u0 = 8 * hh;
+                    const int u0 = 8 * hh, ci = 2 * g4 + hh;  // ci: the 8-channel chunk in the half's tiles
                     float a_kp[8], a_q[8], a_a[8], a_km[8];
                     tmem_ld8(taddr(tm, 32 * q, 256 + 16 * g4 + u0), a_kp);
                     tmem_ld8(taddr(tm, 32 * q, 320 + 16 * g4 + u0), a_q);
                     tmem_ld8(taddr(tm, 32 * q, 384 + 16 * g4 + u0), a_a);
                     tmem_ld8(taddr(tm, 32 * q, 448 + 16 * g4 + u0), a_km);
-                    tmem_wait_ld();
-                    float kv[8], ev[8], qv[8], gv[8];
-                    ld8_bf16(kin + u0, kv);
-                    ld8_bf16(ein + u0, ev);
-                    ld8_bf16(qin + u0, qv);
-                    ld8_bf16(gin_ + u0, gv);
-                    if (QKRAW) { prologue8(kv, rk); prologue8(qv, rq); }
                     float pq[8], pk[8], pa[8], pl[8];
-                    ld8_scaled(p.Pq + cb + u0, s_q, pq);
-                    ld8_scaled(p.Pk + cb + u0, s_k, pk);
-                    ld8_scaled(p.Pa + cb + u0, s_a, pa);
-                    ld8_scaled(p.Pd + cb + u0, s_d, pl);
+                    ld8_scaled(reinterpret_cast<const uint4*>(p.Pq) + pgrp(c, t, j0 + u0), s_q, pq);
+                    ld8_scaled(reinterpret_cast<const uint4*>(p.Pk) + pgrp(c, t, j0 + u0), s_k, pk);
+                    ld8_scaled(reinterpret_cast<const uint4*>(p.Pa) + pgrp(c, t, j0 + u0), s_a, pa);
+                    ld8_scaled(reinterpret_cast<const uint4*>(p.Pd) + pgrp(c, t, j0 + u0), s_d, pl);
+                    tmem_wait_ld();
+                    if (hh == 0 && !cta_wait(&s.bar[B2X], (uint32_t)hj) && tid == 0) atomicOr(&s.bad, 1 << 27);
+                    float kv[8], ev[8], qv[8], gv[8];
+                    ld_chunk16<true>(Bt0, t, ci, kv);
+                    ld_chunk16<true>(Bt0, t, 8 + ci, ev);
+                    ld_chunk16<true>(Bt1, t, ci, qv);
+                    ld_chunk16<true>(Bt1, t, 8 + ci, gv);
+                    if (QKRAW) { prologue8(kv, rk); prologue8(qv, rq); }
                     float oq[8], og[8], ok[8], oe[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
@@ -1062,12 +1086,13 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                         *reinterpret_cast<float4*>(pk_) = make_float4(ok[0], ok[1], ok[2], ok[3]);
                         *reinterpret_cast<float4*>(pk_ + 4) = make_float4(ok[4], ok[5], ok[6], ok[7]);
                     } else {
-                        st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dq) + ro + u0, oq);
-                        st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dk) + ro + u0, ok);
+                        st_chunk16<true>(Bt1, t, ci, oq);  // dq over q
+                        st_chunk16<true>(Bt0, t, ci, ok);  // dk over k
                     }
-                    st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dgamma) + ro + u0, og);
-                    st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.de) + ro + u0, oe);
+                    st_chunk16<true>(Bt1, t, 8 + ci, og);  // dgamma over gamma
+                    st_chunk16<true>(Bt0, t, 8 + ci, oe);  // de over e
                 }
+                fence_async_smem();  // (the barrier below publishes the tiles to the stores)
                 if (QKRAW) {
                     s.dot[0][4 * hj + g4][t] = dotq;
                     s.dot[1][4 * hj + g4][t] = dotk;
@@ -1086,6 +1111,16 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                     for (int j = 0; j < 16; ++j) s.sfx[q][j0 + j] = dL[j];
                 }
                 __syncthreads();
+                if (tid == 0) {
+                    const int z = b * p.T + n * kC;
+                    if (!QKRAW) {
+                        tma_store_3d(&p.tdq, Bt1, 64 * hj, hd, z);
+                        tma_store_3d(&p.tdk, Bt0, 64 * hj, hd, z);
+                    }
+                    tma_store_3d(&p.tdgam, Bt1 + kT16Block, 64 * hj, hd, z);
+                    tma_store_3d(&p.tde, Bt0 + kT16Block, 64 * hj, hd, z);
+                    bulk_commit();
+                }
                 const __nv_bfloat16* graw = reinterpret_cast<const __nv_bfloat16*>(p.g) + ro;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
@@ -1102,6 +1137,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                     st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dg) + ro + 8 * hh, o);
                 }
             }
+            if (tid == 0) bulk_wait_read();  // the stores have left Bt0, Bt1
             sync_all();
         }
         if (QKRAW) {
@@ -1141,6 +1177,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             sync_all();
         }
     }
+    if (tid == 0) bulk_wait_all();
     if (tid == 0 && s.bad) atomicOr(&g_bwd2_timeouts, (unsigned)s.bad);
     sync_all();
     if (warp == 0) tmem_dealloc(tm, 512);
@@ -1254,6 +1291,12 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     p2.dgb = dgb; p2.nslab = kD / SLAB;
     p2.dq = a.dq; p2.dk = a.dk; p2.dg = a.dg; p2.de = a.de; p2.dgamma = a.dgamma;
     p2.rnorm = a.rnorm;
+    if (!map_tokens16(&p2.tk, a.k, a.B, a.T, a.H) || !map_tokens16(&p2.te, a.e, a.B, a.T, a.H) ||
+        !map_tokens16(&p2.tq, a.q, a.B, a.T, a.H) || !map_tokens16(&p2.tgam, a.gamma, a.B, a.T, a.H) ||
+        !map_tokens16(&p2.tdgam, a.dgamma, a.B, a.T, a.H) || !map_tokens16(&p2.tde, a.de, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
+    if (!a.rnorm && (!map_tokens16(&p2.tdq, a.dq, a.B, a.T, a.H) || !map_tokens16(&p2.tdk, a.dk, a.B, a.T, a.H)))
+        return cudaErrorInvalidValue;
     p2.flags = a.flags;
     p2.dO_f16 = a.zo != nullptr;
     if (!a.flags) return cudaErrorInvalidValue;

@@ -46,8 +46,8 @@ struct Bwd1Params {
     const unsigned char* aux;
     const float* S_chunks;
     const float* dSc;
-    // state-side partials as fp16 [nch][128][128] with one power-of-two scale
-    // per row and 32-column group ([nch][128][4] fp32)
+    // state-side partials as fp16, per chunk [16 channel groups of 8][128 rows][8],
+    // with one power-of-two scale per row and 32-channel group ([nch][4][128] fp32)
     __half *Pq, *Pk, *Pa, *Pd;
     float *sq, *sk, *sa, *sd;
     unsigned char *Y16, *dYR16;
@@ -57,6 +57,8 @@ struct Bwd1Params {
 
 struct Bwd2Params {
     CUtensorMap tdO, tg;
+    CUtensorMap tk, te, tq, tgam;         // the readout's inputs (token-major bf16 tiles)
+    CUtensorMap tdq, tdk, tdgam, tde;     // its outputs, stored as tiles (tdq, tdk unused with raw q/k)
     int B, T, H;
     const void *q, *k, *g, *e, *gamma;
     const unsigned char* aux;

@@ -126,6 +126,15 @@ __device__ __forceinline__ void bulk_store(void* dst, const void* src, uint32_t 
                  "r"(saddr(src)), "r"(bytes)
                  : "memory");
 }
+// 3-D tiled store of one box from shared memory (the tile's layout as the
+// map's swizzle gives it) in this thread's bulk group; the same rules as
+// bulk_store.  Coordinates must be in range (no negative start).
+__device__ __forceinline__ void tma_store_3d(const CUtensorMap* map, const void* src, int x, int y, int z) {
+    asm volatile("cp.async.bulk.tensor.3d.global.shared::cta.tile.bulk_group [%0, {%1, %2, %3}], [%4];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(z), "r"(saddr(src))
+                 : "memory");
+}
 __device__ __forceinline__ void bulk_commit() {
     asm volatile("cp.async.bulk.commit_group;" ::: "memory");
 }
