@@ -590,10 +590,10 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             for (int j = 0; j < 32; ++j) d[j] *= sS * ex2(L[j]);
             st_scaled32(reinterpret_cast<uint4*>(p.Pq) + pb, p.sq + scb, d);
             tm_ld32w(tm, q, 128 + c0, d);
-            const float* up = reinterpret_cast<const float*>(ax + AuxLayout::kUp) + (size_t)t * kD + c0;
+            const float* ub = reinterpret_cast<const float*>(ax + AuxLayout::kUp);
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
-                const float4 x = __ldg(reinterpret_cast<const float4*>(up + j));
+                const float4 x = __ldg(grp4(ub, t, c0 + j));
                 d[j] = d[j] * sS + x.x; d[j + 1] = d[j + 1] * sS + x.y;
                 d[j + 2] = d[j + 2] * sS + x.z; d[j + 3] = d[j + 3] * sS + x.w;
             }
@@ -924,13 +924,17 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 }
             }
             if (!cta_wait(&s.bar[B2G], (uint32_t)((2 * it + hj) & 1)) && tid == 0) atomicOr(&s.bad, 1 << 26);
+            uint32_t gkeep = 0;  // bit u: g of channel j0 + u is at or above the clamp
             {
                 float v[8];
 #pragma unroll
                 for (int i = 0; i < 2; ++i) {  // row t, channels 16 g4 .. +16 of the block
                     ld_chunk16<true>(Bt1, t, 2 * g4 + i, v);
 #pragma unroll
-                    for (int u = 0; u < 8; ++u) v[u] = fmaxf(v[u], kLogDecayMin);
+                    for (int u = 0; u < 8; ++u) {
+                        gkeep |= (v[u] >= kLogDecayMin ? 1u : 0u) << (8 * i + u);
+                        v[u] = fmaxf(v[u], kLogDecayMin);
+                    }
                     st_chunk16<true>(Bt1, t, 2 * g4 + i, v);
                 }
             }
@@ -1027,7 +1031,6 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             }
             {
                 const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + j0;
-                const size_t ro = tok * kD + j0;
                 const size_t scb = psc(c, t, j0);  // channels j0 .. +16 share a group
                 const float s_q = __ldg(p.sq + scb), s_k = __ldg(p.sk + scb);
                 const float s_a = __ldg(p.sa + scb), s_d = __ldg(p.sd + scb);
@@ -1121,20 +1124,18 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                     tma_store_3d(&p.tde, Bt0 + kT16Block, 64 * hj, hd, z);
                     bulk_commit();
                 }
-                const __nv_bfloat16* graw = reinterpret_cast<const __nv_bfloat16*>(p.g) + ro;
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    float o[8], gv[8];
-                    ld8_bf16(graw + 8 * hh, gv);
+                    float o[8];
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const int j = 8 * hh + u;
                         float post = s.dgb[j0 + j];
                         for (int qq = q + 1; qq < 4; ++qq) post += s.sfx[qq][j0 + j];
                         // the clamp g >= -20 passes no gradient below it
-                        o[u] = gv[u] >= kLogDecayMin ? dL[j] + post : 0.f;
+                        o[u] = ((gkeep >> j) & 1u) ? dL[j] + post : 0.f;
                     }
-                    st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dg) + ro + 8 * hh, o);
+                    st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dg) + tok * kD + j0 + 8 * hh, o);
                 }
             }
             if (tid == 0) bulk_wait_read();  // the stores have left Bt0, Bt1
@@ -1201,6 +1202,7 @@ int sm_count() {
 constexpr int kBprepSmem = 2 * kT16Bytes + 1024;
 constexpr int kBwd1Smem = 6 * kT16Bytes + sizeof(Bwd1Smem) + 1024;
 constexpr int kBwd2Smem = 4 * kT16Bytes + 2 * kT32Half + sizeof(Bwd2Smem) + 1024;
+static_assert(kBwd2Smem <= 232448, "k2_bwd2 shared memory");
 template <int SLAB>
 constexpr int rev_smem() { return 3 * 128 * 128 * 4 + SLAB * 512 + 1024; }
 

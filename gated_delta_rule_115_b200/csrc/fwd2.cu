@@ -516,10 +516,9 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             tm_ld32w(tm, q, 128 + c0, v);  // U'
             row_st32<false>(S[1], t, h, v);
             if (ax) {
-                float* up = reinterpret_cast<float*>(ax + AuxLayout::kUp) + (size_t)t * kD + c0;
+                float* ub = reinterpret_cast<float*>(ax + AuxLayout::kUp);
 #pragma unroll
-                for (int j = 0; j < 32; j += 4)
-                    *reinterpret_cast<float4*>(up + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                for (int j = 0; j < 32; j += 4) *grp4(ub, t, c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
             }
         }
         fence_async_smem();
@@ -638,10 +637,9 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
                 for (int j = 0; j < 32; ++j) mt[(size_t)(c0 + j) * kD] = v[j];
             }
             tm_ld32w(tm + 128, q, c0, v);
-            float* bd = p.Bn + rbase;
+            float* bb = p.Bn + (size_t)c * kC * kD;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(bd + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            for (int j = 0; j < 32; j += 4) *grp4(bb, t, c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         }
         sync_all();  // TMEM read out before the next chunk's products
     }
@@ -707,10 +705,10 @@ __global__ void __launch_bounds__(128, 1) k2_chain(const __grid_constant__ Chain
     put_state();
     float Bnext[SLAB];
     auto load_B = [&](int n, float* dst) {
-        const float* src = p.Bn + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
+        const float* blk = p.Bn + ((size_t)bh * N + n) * kD * kD;
 #pragma unroll
         for (int c = 0; c < SLAB; c += 4) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(src + c));
+            const float4 v = __ldg(grp4(blk, j, c0 + c));
             dst[c] = v.x; dst[c + 1] = v.y; dst[c + 2] = v.z; dst[c + 3] = v.w;
         }
     };

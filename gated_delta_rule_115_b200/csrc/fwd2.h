@@ -15,7 +15,8 @@ namespace v2 {
 // Per-chunk intermediates the forward saves for the backward ("aux"), byte
 // offsets inside one chunk's record.  16-bit tiles are stored byte for byte in
 // the 128B-swizzled shared-memory tile layout (tc2.cuh, T16) so the backward
-// reloads them with plain bulk copies; fp32 blocks are row-major 128 x 128.
+// reloads them with plain bulk copies; the fp32 block is 4-column-group-major
+// (tc2.cuh, grp4).
 struct AuxLayout {
     static constexpr size_t kT16 = 0;                 // T = (I + L_A)^-1, fp16 tile
     static constexpr size_t kLK16 = 1 * 32768;        // strict(L_K), fp16 tile
@@ -25,7 +26,7 @@ struct AuxLayout {
     static constexpr size_t kW16 = 5 * 32768;         // W = T K~, fp16 tile
     static constexpr size_t kAbar16 = 6 * 32768;      // Abar, fp16 tile
     static constexpr size_t kKbar16 = 7 * 32768;      // Kbar, fp16 tile
-    static constexpr size_t kUp = 8 * 32768;          // U' = T L_K U, fp32 [t][c]
+    static constexpr size_t kUp = 8 * 32768;          // U' = T L_K U, fp32 (grp4 layout)
     static constexpr size_t kBytes = 8 * 32768 + 65536;
 };
 // The aux buffer: nch records, then Q' [nch][128][128] fp32, then M^T
@@ -54,7 +55,7 @@ struct IntraParams {
     int B, T, H;
     float* M;      // chunk transitions M_n [j][i]: S_{n+1} = M_n S_n + B_n
     float* Mt;     // M_n transposed (optional)
-    float* Bn;     // B_n [j][c]
+    float* Bn;     // B_n [j][c] (grp4 layout)
     float* Qp;     // Q'_n [t][i]: O_n = Q'_n S_n + O_intra_n
     float* Oi;     // O_intra_n [t][c]
     unsigned char* aux;  // per-chunk AuxLayout records, or null (nothing saved)

@@ -93,6 +93,18 @@ __device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
+// Per-chunk fp32 128 x 128 blocks read only by this library's kernels (B_n,
+// U') are kept 4-column-group-major: element
+// (t, col) is component col % 4 of float4 number (col / 4) 128 + t.  A warp
+// whose lanes own consecutive rows then moves one contiguous 512-byte run
+// per 4-column group, where the row-major form costs a transaction per lane.
+__device__ __forceinline__ float4* grp4(float* blk, int t, int col) {
+    return reinterpret_cast<float4*>(blk) + (size_t)(col >> 2) * 128 + t;
+}
+__device__ __forceinline__ const float4* grp4(const float* blk, int t, int col) {
+    return reinterpret_cast<const float4*>(blk) + (size_t)(col >> 2) * 128 + t;
+}
+
 // ------------------------------------------------------------------ TMA
 
 // 3-D tiled load of one box into shared memory, completion counted in bytes
