@@ -354,40 +354,50 @@ __global__ void __launch_bounds__(128, 1) k2_chain_rev(const __grid_constant__ R
             *reinterpret_cast<float*>(Gt + t32_off<SLAB>(c, j >> 2) + (j & 3) * 4) = Gr[c];
     };
     put();
+    // B'_n and S_{n+1} of a step, loaded one step ahead (both come from DRAM)
+    float Bn1[SLAB], Sn1[SLAB];
+    auto load_step = [&](int n, float* Bd, float* Sd) {
+        const float* src = p.Bp + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
+        const float* sn1 = (n + 1 < N) ? p.S_chunks + ((size_t)bh * N + n + 1) * kD * kD + (size_t)j * kD + c0
+                                       : p.S_last + gbase;
+#pragma unroll
+        for (int c = 0; c < SLAB; c += 4) {
+            const float4 v = __ldg(reinterpret_cast<const float4*>(src + c));
+            const float4 w = __ldg(reinterpret_cast<const float4*>(sn1 + c));
+            Bd[c] = v.x; Bd[c + 1] = v.y; Bd[c + 2] = v.z; Bd[c + 3] = v.w;
+            Sd[c] = w.x; Sd[c + 1] = w.y; Sd[c + 2] = w.z; Sd[c + 3] = w.w;
+        }
+    };
+    if (N > 0) load_step(N - 1, Bn1, Sn1);
     fence_async_smem();
     sync_all();
     for (int s = 0; s < N; ++s) {
         const int st = s % STAGES, n = N - 1 - s;
-        // record G_{n+1} and this slab's share of dLbar_n
-        {
-            float* d = p.dSc + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
-            const float* sn1 = (n + 1 < N) ? p.S_chunks + ((size_t)bh * N + n + 1) * kD * kD + (size_t)j * kD + c0
-                                           : p.S_last + gbase;
-            float acc = 0.f;
-#pragma unroll
-            for (int c = 0; c < SLAB; c += 4) {
-                *reinterpret_cast<float4*>(d + c) = make_float4(Gr[c], Gr[c + 1], Gr[c + 2], Gr[c + 3]);
-                const float4 sv = __ldg(reinterpret_cast<const float4*>(sn1 + c));
-                acc += Gr[c] * sv.x + Gr[c + 1] * sv.y + Gr[c + 2] * sv.z + Gr[c + 3] * sv.w;
-            }
-            // one partial per value slab, summed in a fixed order by k2_bwd2
-            p.dgb[((size_t)(c0 / SLAB) * p.nch + (size_t)bh * N + n) * kD + j] = acc;
-        }
-        // only the issuing thread waits for M_n^T (see k2_chain)
+        // the product first: only the issuing thread waits for M_n^T (see k2_chain)
         if (tid == 0) {
             if (!mbar_wait(&bar[st], (uint32_t)((s / STAGES) & 1))) atomicOr(&bad, 4);
             tc_fence_after();
             gemm_kk32<128, SLAB>(tm, saddr(Mst + st * MT), saddr(Gt), 0, SLAB, 128, false);
             mma_commit(&bar[STAGES]);
         }
-        float Bc[SLAB];
+        float Bc[SLAB], Sc[SLAB];
+#pragma unroll
+        for (int c = 0; c < SLAB; ++c) {
+            Bc[c] = Bn1[c];
+            Sc[c] = Sn1[c];
+        }
+        if (s + 1 < N) load_step(n - 1, Bn1, Sn1);
+        // while it runs: record G_{n+1} and this slab's share of dLbar_n
         {
-            const float* src = p.Bp + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
+            float* d = p.dSc + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
+            float acc = 0.f;
 #pragma unroll
             for (int c = 0; c < SLAB; c += 4) {
-                const float4 v = __ldg(reinterpret_cast<const float4*>(src + c));
-                Bc[c] = v.x; Bc[c + 1] = v.y; Bc[c + 2] = v.z; Bc[c + 3] = v.w;
+                *reinterpret_cast<float4*>(d + c) = make_float4(Gr[c], Gr[c + 1], Gr[c + 2], Gr[c + 3]);
+                acc += Gr[c] * Sc[c] + Gr[c + 1] * Sc[c + 1] + Gr[c + 2] * Sc[c + 2] + Gr[c + 3] * Sc[c + 3];
             }
+            // one partial per value slab, summed in a fixed order by k2_bwd2
+            p.dgb[((size_t)(c0 / SLAB) * p.nch + (size_t)bh * N + n) * kD + j] = acc;
         }
         if (!cta_wait(&bar[STAGES], (uint32_t)(s & 1)) && tid == 0) atomicOr(&bad, 8);
         if (tid == 0 && s + STAGES < N) issue(s + STAGES);

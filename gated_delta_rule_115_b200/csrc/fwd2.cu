@@ -794,6 +794,14 @@ __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutPara
     if (tid == 0 && (int)blockIdx.x < nch) issue(blockIdx.x);
     int it = 0;
     for (int c = blockIdx.x; c < nch; c += gridDim.x, ++it) {
+        if (tid == 32) {  // this chunk's O_intra (first chunk) and the next chunk's blocks -> L2
+            const int cn = c + gridDim.x;
+            if (it == 0) bulk_prefetch_l2(p.Oi + (size_t)c * kC * kD, kC * kD * 4);
+            if (cn < nch) {
+                bulk_prefetch_l2(p.S_chunks + (size_t)cn * kD * kD, kD * kD * 4);
+                bulk_prefetch_l2(p.Oi + (size_t)cn * kC * kD, kC * kD * 4);
+            }
+        }
         // S_n^T into St: thread (row r = tid / 2, half) reads 64 values of S_n row r
         {
             const int r = tid >> 1, hf = tid & 1;
