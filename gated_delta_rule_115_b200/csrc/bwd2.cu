@@ -430,7 +430,7 @@ struct Bwd1Smem {
     uint32_t tslot;
     int bad;
 };
-enum { B1D = 0, B1W, B1U, B1Q, B1A, B1T, B1K, B1L, B1KB, B1M1, B1M2, B1M3, B1M4, B1M5, B1M6, B1G, B1LM };
+enum { B1D = 0, B1W, B1U, B1Q, B1A, B1T, B1K, B1L, B1KB, B1M1, B1M2, B1M3, B1M4, B1M5, B1M6, B1G, B1LM, B1V };
 
 // Largest |x| over the block (512 threads, 32 values each); ends with a barrier.
 __device__ __forceinline__ float block_absmax(const float (&v)[32], float* red, int warp, int lane) {
@@ -491,8 +491,6 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
     for (int c = blockIdx.x; c < nch; c += gridDim.x, ++it) {
         const uint32_t ph = (uint32_t)(it & 1);
         const int n = c % N, bh = c / N, hd = bh % p.H, b = bh / p.H;
-        const size_t tok = ((size_t)b * p.T + (size_t)n * kC + t) * p.H + hd;  // token-major row
-        const size_t ro = tok * kD + c0;                                      // this thread's 32 elements
         const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + c0;          // per-chunk arrays
         const size_t pb = pgrp(c, t, c0), scb = psc(c, t, c0);               // partials, their scales
         const unsigned char* ax = p.aux + (size_t)c * AuxLayout::kBytes;
@@ -681,7 +679,16 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             mma_commit(&s.bar[B1M5]);
         }
         waitb(B1M5, ph);
-        if (tid == 0) bulk(S[0], ax + AuxLayout::kKbar16, B1KB);  // S consumed
+        if (tid == 0) {
+            bulk(S[0], ax + AuxLayout::kKbar16, B1KB);  // S consumed
+            // v -> S1, w -> S4 (dO, M_QK consumed) for the last phase
+            const int z = b * p.T + n * kC;
+            mbar_arrive_expect_tx(&s.bar[B1V], 2 * kT16Bytes);
+            tma_load_3d(S[1], &p.tv, 0, hd, z, &s.bar[B1V]);
+            tma_load_3d(S[1] + kT16Block, &p.tv, 64, hd, z, &s.bar[B1V]);
+            tma_load_3d(S[4], &p.tw, 0, hd, z, &s.bar[B1V]);
+            tma_load_3d(S[4] + kT16Block, &p.tw, 64, hd, z, &s.bar[B1V]);
+        }
         {
             float d[32], e2[32];
             tm_ld32w(tm, q, c0, d);         // dK~ / sS
@@ -706,14 +713,11 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             float d[32], e2[32], vv[8], wv[8];
             tm_ld32w(tm, q, 256 + c0, d);
             tm_ld32w(tm, q, 128 + c0, e2);
-            const __nv_bfloat16* vp = reinterpret_cast<const __nv_bfloat16*>(p.v) + ro;
-            const __nv_bfloat16* wp = reinterpret_cast<const __nv_bfloat16*>(p.w) + ro;
-            __nv_bfloat16* dvp = reinterpret_cast<__nv_bfloat16*>(p.dv) + ro;
-            __nv_bfloat16* dwp = reinterpret_cast<__nv_bfloat16*>(p.dw) + ro;
+            waitb(B1V, ph);
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                ld8_bf16(vp + 8 * i, vv);
-                ld8_bf16(wp + 8 * i, wv);
+            for (int i = 0; i < 4; ++i) {  // dv over v (S1), dw over w (S4), stored as tiles
+                ld_chunk16<true>(S[1], t, 4 * h + i, vv);
+                ld_chunk16<true>(S[4], t, 4 * h + i, wv);
                 float o1[8], o2[8];
 #pragma unroll
                 for (int u = 0; u < 8; ++u) {
@@ -721,13 +725,21 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
                     o1[u] = du * wv[u];
                     o2[u] = du * vv[u];
                 }
-                st8_bf16(dvp + 8 * i, o1);
-                st8_bf16(dwp + 8 * i, o2);
+                st_chunk16<true>(S[1], t, 4 * h + i, o1);
+                st_chunk16<true>(S[4], t, 4 * h + i, o2);
             }
         }
+        fence_async_smem();
         sync_all();
+        if (tid == 0) {  // (the next chunk's loads into S1, S4 wait for these reads)
+            const int z = b * p.T + n * kC;
+            tma_store_3d(&p.tdv, S[1], 0, hd, z);
+            tma_store_3d(&p.tdv, S[1] + kT16Block, 64, hd, z);
+            tma_store_3d(&p.tdw, S[4], 0, hd, z);
+            tma_store_3d(&p.tdw, S[4] + kT16Block, 64, hd, z);
+            bulk_commit();
+        }
     }
-    if (tid == 0) bulk_wait_all();
     if (tid == 0) bulk_wait_all();
     if (tid == 0 && s.bad) atomicOr(&g_bwd2_timeouts, (unsigned)s.bad);
     sync_all();
@@ -1280,7 +1292,10 @@ cudaError_t run_bwd2(const Bwd2Args& a, cudaStream_t st) {
     const int grid = nch < nsm ? nch : nsm;
     Bwd1Params p1;
     p1.tdO = tdO; p1.B = a.B; p1.T = a.T; p1.H = a.H;
-    if (!map_tokens16(&p1.tg, a.g, a.B, a.T, a.H)) return cudaErrorInvalidValue;
+    if (!map_tokens16(&p1.tg, a.g, a.B, a.T, a.H) || !map_tokens16(&p1.tv, a.v, a.B, a.T, a.H) ||
+        !map_tokens16(&p1.tw, a.w, a.B, a.T, a.H) || !map_tokens16(&p1.tdv, a.dv, a.B, a.T, a.H) ||
+        !map_tokens16(&p1.tdw, a.dw, a.B, a.T, a.H))
+        return cudaErrorInvalidValue;
     p1.q = a.q; p1.k = a.k; p1.v = a.v; p1.g = a.g; p1.e = a.e; p1.w = a.w; p1.gamma = a.gamma;
     p1.aux = a.aux; p1.S_chunks = a.S_chunks; p1.dSc = dSc;
     p1.Pq = P16[0]; p1.Pk = P16[1]; p1.Pa = P16[2]; p1.Pd = P16[3];

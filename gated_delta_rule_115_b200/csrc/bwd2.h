@@ -41,6 +41,7 @@ struct RevParams {
 
 struct Bwd1Params {
     CUtensorMap tdO, tg;                  // dO, and g (the log decay) as token-major bf16 tiles
+    CUtensorMap tv, tw, tdv, tdw;         // v, w in and dv, dw out, as token-major bf16 tiles
     int B, T, H;
     const void *q, *k, *v, *g, *e, *w, *gamma;
     const unsigned char* aux;
