@@ -226,12 +226,12 @@ __global__ void __launch_bounds__(256) k2_bprep(const __grid_constant__ BprepPar
         tma_load_3d(Dt + kT16Block, &p.tdO, 64, y, z, &bar[0]);
     }
     {  // Q' row t, columns 64h .. +64 -> fp16
-        const float* src = p.Qp + (size_t)c * kC * kD + (size_t)t * kD + 64 * h;
+        const float* qb = p.Qp + (size_t)c * kC * kD;
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             float v[8];
-            const float4 a = __ldg(reinterpret_cast<const float4*>(src + 8 * i));
-            const float4 b = __ldg(reinterpret_cast<const float4*>(src + 8 * i + 4));
+            const float4 a = __ldg(grp4(qb, t, 64 * h + 8 * i));
+            const float4 b = __ldg(grp4(qb, t, 64 * h + 8 * i + 4));
             v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
             st_chunk16<false>(Qt, t, 8 * h + i, v);
         }

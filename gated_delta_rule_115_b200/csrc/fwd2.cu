@@ -549,7 +549,7 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             // Q' = Q~ - M_QA W with Q~ = gamma q 2^L from the bf16 inputs
             float v[32];
             tm_ld32w(tm + 256, q, c0, v);
-            float* qd = p.Qp + rbase;
+            float* qb = p.Qp + (size_t)c * kC * kD;
             const size_t ri = (((size_t)(c / N / p.H) * p.T + (size_t)(c % N) * kC + t) * p.H + y) * kD + c0;
             const __nv_bfloat16* qsrc = reinterpret_cast<const __nv_bfloat16*>(p.q) + ri;
             const __nv_bfloat16* gsrc = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + ri;
@@ -571,14 +571,13 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
                     r[2 * u] = v[j + 2 * u] + q0 * g0 * ex2(L[j + 2 * u]);
                     r[2 * u + 1] = v[j + 2 * u + 1] + q1 * g1 * ex2(L[j + 2 * u + 1]);
                 }
-                *reinterpret_cast<float4*>(qd + j) = make_float4(r[0], r[1], r[2], r[3]);
-                *reinterpret_cast<float4*>(qd + j + 4) = make_float4(r[4], r[5], r[6], r[7]);
+                *grp4(qb, t, c0 + j) = make_float4(r[0], r[1], r[2], r[3]);
+                *grp4(qb, t, c0 + j + 4) = make_float4(r[4], r[5], r[6], r[7]);
             }
             tm_ld32w(tm + 384, q, c0, v);
-            float* od = p.Oi + rbase;
+            float* ob = p.Oi + (size_t)c * kC * kD;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(od + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+            for (int j = 0; j < 32; j += 4) *grp4(ob, t, c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         }
         waitb(s, BE, ph);
         waitb(s, BF, ph);
@@ -761,8 +760,8 @@ __global__ void __launch_bounds__(128, 1) k2_chain(const __grid_constant__ Chain
 // ------------------------------------------------------------------ k2_out
 
 // O_n = Q'_n S_n + O_intra_n per chunk (TF32 products, fp32 accumulation).
-// Persistent, 256 threads; Q'_n by TMA (K-major TF32 tile), S_n^T written by
-// the threads into a K-major TF32 tile.
+// Persistent, 256 threads; the threads write Q'_n (from its group-major
+// block) and S_n^T into K-major TF32 tiles.
 template <typename Tout>
 __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutParams p) {
     constexpr uint32_t MT = 128 * 128 * 4;
@@ -770,6 +769,7 @@ __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutPara
     unsigned char* sm = (unsigned char*)(((uintptr_t)smraw + 1023) & ~(uintptr_t)1023);
     unsigned char* Qt = sm;
     unsigned char* St = sm + MT;
+    unsigned char* Ot = sm + 2 * MT;  // bf16 output tile (T16 layout)
     __shared__ uint64_t bar[2];
     __shared__ uint32_t tslot;
     __shared__ int bad;
@@ -777,63 +777,72 @@ __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutPara
     const int q = warp & 3, h = warp >> 2, t = 32 * q + lane;
     const int N = p.T / kC, nch = p.B * p.H * N;
     if (tid == 0) {
-        mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
         bad = 0;
         fence_barrier_init();
-        prefetch_tmap(&p.tQ);
     }
     if (warp == 0) tmem_alloc(&tslot, 128);
     sync_all();
     const uint32_t tm = tslot;
-    auto issue = [&](int c) {
-        mbar_arrive_expect_tx(&bar[0], MT);
-        for (int kb = 0; kb < 4; ++kb)
-            tma_load_3d(Qt + kb * 128 * 128, &p.tQ, 32 * kb, c * kC, 0, &bar[0]);
-    };
-    if (tid == 0 && (int)blockIdx.x < nch) issue(blockIdx.x);
     int it = 0;
     for (int c = blockIdx.x; c < nch; c += gridDim.x, ++it) {
-        if (tid == 32) {  // this chunk's O_intra (first chunk) and the next chunk's blocks -> L2
+        if (tid == 32) {  // the next chunk's blocks -> L2
             const int cn = c + gridDim.x;
-            if (it == 0) bulk_prefetch_l2(p.Oi + (size_t)c * kC * kD, kC * kD * 4);
             if (cn < nch) {
+                bulk_prefetch_l2(p.Qp + (size_t)cn * kC * kD, kC * kD * 4);
                 bulk_prefetch_l2(p.S_chunks + (size_t)cn * kD * kD, kD * kD * 4);
                 bulk_prefetch_l2(p.Oi + (size_t)cn * kC * kD, kC * kD * 4);
             }
         }
-        // S_n^T into St: thread (row r = tid / 2, half) reads 64 values of S_n row r
+        // Q'_n into Qt: thread (row tid % 128, every other 4-column group) from
+        // the group-major block; S_n^T into St: thread (row r = tid / 2, half)
+        // reads 64 values of S_n row r.  All 32 loads are issued before the
+        // first store, so that their latencies overlap.
         {
+            const float* qb = p.Qp + (size_t)c * kC * kD;
+            const int rq = tid & 127, g0 = tid >> 7;
             const int r = tid >> 1, hf = tid & 1;
             const float* src = p.S_chunks + (size_t)c * kD * kD + (size_t)r * kD + 64 * hf;
-#pragma unroll 4
-            for (int cc = 0; cc < 64; cc += 4) {
-                const float4 v = __ldg(reinterpret_cast<const float4*>(src + cc));
-                const float vv[4] = {v.x, v.y, v.z, v.w};
+            float4 qv[16], sv[16];
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                qv[k] = __ldg(grp4(qb, rq, 4 * (g0 + 2 * k)));
+                sv[k] = __ldg(reinterpret_cast<const float4*>(src + 4 * k));
+            }
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const int g = g0 + 2 * k;
+                *reinterpret_cast<float4*>(Qt + (g >> 3) * 128 * 128 + rq * 128 + (((g & 7) ^ (rq & 7)) << 4)) = qv[k];
+            }
+#pragma unroll
+            for (int k = 0; k < 16; ++k) {
+                const float vv[4] = {sv[k].x, sv[k].y, sv[k].z, sv[k].w};
 #pragma unroll
                 for (int u = 0; u < 4; ++u) {
-                    const int col = 64 * hf + cc + u;  // B row (value column), K index r
+                    const int col = 64 * hf + 4 * k + u;  // B row (value column), K index r
                     *reinterpret_cast<float*>(St + t32_off<128>(col, r >> 2) + (r & 3) * 4) = vv[u];
                 }
             }
         }
         fence_async_smem();
         sync_all();
-        if (tid == 0) {  // Q' is read by the MMA only; its issuer alone waits for it
-            if (!mbar_wait(&bar[0], (uint32_t)(it & 1))) bad = 1;
-            tc_fence_after();
+        if (tid == 0) {
             gemm_kk32<128, 128>(tm, saddr(Qt), saddr(St), 0, 128, 128, false);
             mma_commit(&bar[1]);
+            bulk_wait_read();  // the previous chunk's o tile has left Ot (the barrier below tells the rest)
+        }
+        float4 oa[16];  // O_intra row t, columns 64 h .. +64, loaded while the product runs
+        {
+            const float* oib = p.Oi + (size_t)c * kC * kD;
+#pragma unroll
+            for (int k = 0; k < 16; ++k) oa[k] = __ldg(grp4(oib, t, 64 * h + 4 * k));
         }
         if (!cta_wait(&bar[1], (uint32_t)(it & 1)) && tid == 0) bad = 1;
-        const int cn = c + gridDim.x;
-        if (tid == 0 && cn < nch) issue(cn);
         // epilogue: o[b][n*C + t][h][64 hh ..] = D + O_intra, times sigmoid(zo)
         // when the output gate is fused (the pre-gate value then also to o_pre)
         const int n = c % N, bh = c / N, hd = bh % p.H, b = bh / p.H;
         float v[64];
         tm_ld64(tm + 64 * h, q, 0, v);
-        const float* oi = p.Oi + (size_t)c * kC * kD + (size_t)t * kD + 64 * h;
         const size_t ro = (((size_t)b * p.T + (size_t)n * kC + t) * p.H + hd) * kD + 64 * h;
         Tout* od = reinterpret_cast<Tout*>(p.o) + ro;
         Tout* pd = p.o_pre ? reinterpret_cast<Tout*>(p.o_pre) + ro : nullptr;
@@ -850,7 +859,7 @@ __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutPara
         };
 #pragma unroll
         for (int jj = 0; jj < 64; jj += 4) {
-            const float4 a = __ldg(reinterpret_cast<const float4*>(oi + jj));
+            const float4 a = oa[jj >> 2];
             float r0 = v[jj] + a.x, r1 = v[jj + 1] + a.y, r2 = v[jj + 2] + a.z, r3 = v[jj + 3] + a.w;
             if (zr) {
                 if (pd) put4(pd, jj, r0, r1, r2, r3);
@@ -860,10 +869,26 @@ __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutPara
                 unpack16<true>(zw.y, z2, z3);
                 r0 *= sigmoid_f(z0); r1 *= sigmoid_f(z1); r2 *= sigmoid_f(z2); r3 *= sigmoid_f(z3);
             }
-            put4(od, jj, r0, r1, r2, r3);
+            if constexpr (sizeof(Tout) == 4) {
+                put4(od, jj, r0, r1, r2, r3);
+            } else {
+                v[jj] = r0; v[jj + 1] = r1; v[jj + 2] = r2; v[jj + 3] = r3;
+            }
+        }
+        if constexpr (sizeof(Tout) == 2) {  // bf16 o leaves as a row tile by TMA store
+#pragma unroll
+            for (int i = 0; i < 8; ++i) st_chunk16<true>(Ot, t, 8 * h + i, v + 8 * i);
+            fence_async_smem();
         }
         sync_all();
+        if (sizeof(Tout) == 2 && tid == 0) {
+            const int z = b * p.T + n * kC;
+            tma_store_3d(&p.to, Ot, 0, hd, z);
+            tma_store_3d(&p.to, Ot + kT16Block, 64, hd, z);
+            bulk_commit();
+        }
     }
+    if (tid == 0) bulk_wait_all();
     if (tid == 0 && bad) atomicAdd(&g_v2_timeouts, 1u);
     sync_all();
     if (warp == 0) tmem_dealloc(tm, 128);
@@ -936,7 +961,7 @@ static int sm_count() {
 }
 
 constexpr int kIntraSmem = 6 * kT16Bytes + sizeof(IntraSmem) + 1024;
-constexpr int kOutSmem = 2 * 128 * 128 * 4 + 1024;
+constexpr int kOutSmem = 2 * 128 * 128 * 4 + kT16Bytes + 1024;
 template <int SLAB>
 constexpr int chain_smem() { return 3 * 128 * 128 * 4 + SLAB * 512 + 1024; }
 
@@ -994,11 +1019,11 @@ cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st) {
 
     if (a.o) {
         OutParams op;
-        if (!map_rows32f(&op.tQ, a.Qp, (long long)nch * kC)) return cudaErrorInvalidValue;
         op.B = a.B; op.T = a.T; op.H = a.H;
-        op.S_chunks = a.S_chunks; op.Oi = a.Oi; op.o = a.o;
+        op.Qp = a.Qp; op.S_chunks = a.S_chunks; op.Oi = a.Oi; op.o = a.o;
         op.zo = a.zo; op.o_pre = a.zo ? a.o_pre : nullptr;
         if (a.out_bf16) {
+            if (!map_tokens16(&op.to, a.o, a.B, a.T, a.H)) return cudaErrorInvalidValue;
             e = cudaFuncSetAttribute(k2_out<__nv_bfloat16>, cudaFuncAttributeMaxDynamicSharedMemorySize, kOutSmem);
             if (e != cudaSuccess) return e;
             MUIR_TIMED("k2_out", st, k2_out<__nv_bfloat16><<<grid, 256, kOutSmem, st>>>(op));

@@ -29,7 +29,7 @@ struct AuxLayout {
     static constexpr size_t kUp = 8 * 32768;          // U' = T L_K U, fp32 (grp4 layout)
     static constexpr size_t kBytes = 8 * 32768 + 65536;
 };
-// The aux buffer: nch records, then Q' [nch][128][128] fp32, then M^T
+// The aux buffer: nch records, then Q' [nch][128][128] fp32 (grp4 layout), then M^T
 // [nch][128][128] fp32 (the reverse state pass reads M_n^T), then the final
 // states S_N [B*H][128][128] fp32.
 inline size_t aux_bytes(size_t nch, size_t bh) {
@@ -56,8 +56,8 @@ struct IntraParams {
     float* M;      // chunk transitions M_n [j][i]: S_{n+1} = M_n S_n + B_n
     float* Mt;     // M_n transposed (optional)
     float* Bn;     // B_n [j][c] (grp4 layout)
-    float* Qp;     // Q'_n [t][i]: O_n = Q'_n S_n + O_intra_n
-    float* Oi;     // O_intra_n [t][c]
+    float* Qp;     // Q'_n [t][i] (grp4 layout): O_n = Q'_n S_n + O_intra_n
+    float* Oi;     // O_intra_n [t][c] (grp4 layout)
     unsigned char* aux;  // per-chunk AuxLayout records, or null (nothing saved)
     int* flags;          // flags[0] |= 1 when a chunk's decay span exceeds the single pivot
     // fused q/k prologue: q and k hold raw x; every read applies
@@ -78,8 +78,9 @@ struct ChainParams {
 };
 
 struct OutParams {
-    CUtensorMap tQ;      // Q' rows of 128 fp32
+    CUtensorMap to;      // o as token-major bf16 tiles (bf16 output only)
     int B, T, H;
+    const float* Qp;     // Q' (grp4 layout)
     const float* S_chunks;
     const float* Oi;
     void* o;             // token-major [B][T][H][128], fp32 or bf16

@@ -93,8 +93,8 @@ __device__ __forceinline__ bool cta_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 
-// Per-chunk fp32 128 x 128 blocks read only by this library's kernels (B_n,
-// U') are kept 4-column-group-major: element
+// Per-chunk fp32 128 x 128 blocks read only by this library's kernels (Q',
+// the intra-chunk output, B_n, U') are kept 4-column-group-major: element
 // (t, col) is component col % 4 of float4 number (col / 4) 128 + t.  A warp
 // whose lanes own consecutive rows then moves one contiguous 512-byte run
 // per 4-column group, where the row-major form costs a transaction per lane.
