@@ -288,14 +288,14 @@ __global__ void __launch_bounds__(256) k2_bprep(const __grid_constant__ BprepPar
     }
     if (!cta_wait(&bar[1], 0) && tid == 0) atomicOr(&bad, 2);
     {
-        float* dst = p.Bp + (size_t)c * kD * kD + (size_t)t * kD + 64 * h;
+        float* bb = p.Bp + (size_t)c * kD * kD;
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
             float v[32];
             tm_ld32w(tm, q, 64 * h + 32 * hh, v);
 #pragma unroll
             for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(dst + 32 * hh + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                *grp4(bb, t, 64 * h + 32 * hh + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         }
     }
     if (tid == 0 && bad) atomicOr(&g_bwd2_timeouts, (unsigned)bad);
@@ -357,12 +357,12 @@ __global__ void __launch_bounds__(128, 1) k2_chain_rev(const __grid_constant__ R
     // B'_n and S_{n+1} of a step, loaded one step ahead (both come from DRAM)
     float Bn1[SLAB], Sn1[SLAB];
     auto load_step = [&](int n, float* Bd, float* Sd) {
-        const float* src = p.Bp + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
+        const float* bb = p.Bp + ((size_t)bh * N + n) * kD * kD;
         const float* sn1 = (n + 1 < N) ? p.S_chunks + ((size_t)bh * N + n + 1) * kD * kD + (size_t)j * kD + c0
                                        : p.S_last + gbase;
 #pragma unroll
         for (int c = 0; c < SLAB; c += 4) {
-            const float4 v = __ldg(reinterpret_cast<const float4*>(src + c));
+            const float4 v = __ldg(grp4(bb, j, c0 + c));
             const float4 w = __ldg(reinterpret_cast<const float4*>(sn1 + c));
             Bd[c] = v.x; Bd[c + 1] = v.y; Bd[c + 2] = v.z; Bd[c + 3] = v.w;
             Sd[c] = w.x; Sd[c + 1] = w.y; Sd[c + 2] = w.z; Sd[c + 3] = w.w;
@@ -389,11 +389,11 @@ __global__ void __launch_bounds__(128, 1) k2_chain_rev(const __grid_constant__ R
         if (s + 1 < N) load_step(n - 1, Bn1, Sn1);
         // while it runs: record G_{n+1} and this slab's share of dLbar_n
         {
-            float* d = p.dSc + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
+            float* gb = p.dSc + ((size_t)bh * N + n) * kD * kD;
             float acc = 0.f;
 #pragma unroll
             for (int c = 0; c < SLAB; c += 4) {
-                *reinterpret_cast<float4*>(d + c) = make_float4(Gr[c], Gr[c + 1], Gr[c + 2], Gr[c + 3]);
+                *grp4(gb, j, c0 + c) = make_float4(Gr[c], Gr[c + 1], Gr[c + 2], Gr[c + 3]);
                 acc += Gr[c] * Sc[c] + Gr[c + 1] * Sc[c + 1] + Gr[c + 2] * Sc[c + 2] + Gr[c + 3] * Sc[c + 3];
             }
             // one partial per value slab, summed in a fixed order by k2_bwd2
@@ -560,10 +560,10 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
 #pragma unroll
             for (int j = 0; j < 32; ++j) v[j] *= is;
             row_st32<false>(S[0], t, h, v);
-            src = p.dSc + cb;
+            const float* gb = p.dSc + (size_t)c * kC * kD;
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
-                const float4 x = __ldg(reinterpret_cast<const float4*>(src + j));
+                const float4 x = __ldg(grp4(gb, t, c0 + j));
                 v[j] = x.x; v[j + 1] = x.y; v[j + 2] = x.z; v[j + 3] = x.w;
             }
             sG = pow2_scale(block_absmax(v, s.red, warp, lane));
@@ -780,7 +780,8 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
     unsigned char* tR = sm + 3 * kT16Bytes;
     unsigned char* Bt0 = sm + 4 * kT16Bytes;
     unsigned char* Bt1 = Bt0 + kT32Half;
-    Bwd2Smem& s = *reinterpret_cast<Bwd2Smem*>(Bt1 + kT32Half);
+    unsigned char* Kt = Bt1 + kT32Half;  // k of the current half (T16 block), by TMA
+    Bwd2Smem& s = *reinterpret_cast<Bwd2Smem*>(Kt + kT16Block);
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int q = warp & 3, g4 = warp >> 2, t = 32 * q + lane;
     const int N = p.T / kC, nch = p.B * p.H * N;
@@ -933,8 +934,9 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             // product (g block in Bt1, ones tile in Bt0: both free until the
             // pivoted operands; TMEM columns 0..63 free until the first round)
             if (tid == 0) {
-                mbar_arrive_expect_tx(&s.bar[B2G], kT16Block);
+                mbar_arrive_expect_tx(&s.bar[B2G], 2 * kT16Block);
                 tma_load_3d(Bt1, &p.tg, 64 * hj, hd, b * p.T + n * kC, &s.bar[B2G]);
+                tma_load_3d(Kt, &p.tk, 64 * hj, hd, b * p.T + n * kC, &s.bar[B2G]);  // k of the half
             }
             {
                 float v[8];
@@ -984,13 +986,12 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 if (far) atomicOr(p.flags, 1);
             }
             __syncthreads();
-            const __nv_bfloat16* kin = reinterpret_cast<const __nv_bfloat16*>(p.k) + tok * kD + j0;
             const __nv_bfloat16* ein = reinterpret_cast<const __nv_bfloat16*>(p.e) + tok * kD + j0;
             const __nv_bfloat16* qin = reinterpret_cast<const __nv_bfloat16*>(p.q) + tok * kD + j0;
             const __nv_bfloat16* gin_ = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + tok * kD + j0;
             {  // Am -> Bt0, Km -> Bt1
                 float kv[16], ev[16], am[16], km[16];
-                ld8_bf16(kin, kv); ld8_bf16(kin + 8, kv + 8);
+                ld_chunk16<true>(Kt, t, 2 * g4, kv); ld_chunk16<true>(Kt, t, 2 * g4 + 1, kv + 8);
                 if (QKRAW) { prologue8(kv, rk); prologue8(kv + 8, rk); }
                 ld8_bf16(ein, ev); ld8_bf16(ein + 8, ev + 8);
 #pragma unroll
@@ -1013,7 +1014,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             for (int r = 0; r < 4; ++r) {
                 if (r == 2) {  // Kp -> Bt0, Qp -> Bt1
                     float kv[16], qv[16], gv[16], kp[16], qp[16];
-                    ld8_bf16(kin, kv); ld8_bf16(kin + 8, kv + 8);
+                    ld_chunk16<true>(Kt, t, 2 * g4, kv); ld_chunk16<true>(Kt, t, 2 * g4 + 1, kv + 8);
                     ld8_bf16(qin, qv); ld8_bf16(qin + 8, qv + 8);
                     if (QKRAW) {
                         prologue8(kv, rk); prologue8(kv + 8, rk);
@@ -1040,19 +1041,18 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             // the second half's rounds were the tiles' last readers
             if (hj == 1 && tid == 0 && c + (int)gridDim.x < nch) load_tiles(c + gridDim.x);
             // ---- readout: final gradients of channels j0 .. j0 + 15 of row t.
-            // k, e (Bt0) and q, gamma (Bt1) of the half come by TMA into the
-            // operand tiles, free now; each thread forms its gradients in the
-            // places of its own inputs and the tiles leave by TMA store.
+            // e (Bt0) and q, gamma (Bt1) of the half come by TMA into the
+            // operand tiles, free now (k has its own tile); each thread forms
+            // its gradients in its own inputs' places (dk in the free block of
+            // Bt0) and the tiles leave by TMA store.
             if (tid == 0) {
                 const int z = b * p.T + n * kC;
-                mbar_arrive_expect_tx(&s.bar[B2X], 4 * kT16Block);
-                tma_load_3d(Bt0, &p.tk, 64 * hj, hd, z, &s.bar[B2X]);
+                mbar_arrive_expect_tx(&s.bar[B2X], 3 * kT16Block);
                 tma_load_3d(Bt0 + kT16Block, &p.te, 64 * hj, hd, z, &s.bar[B2X]);
                 tma_load_3d(Bt1, &p.tq, 64 * hj, hd, z, &s.bar[B2X]);
                 tma_load_3d(Bt1 + kT16Block, &p.tgam, 64 * hj, hd, z, &s.bar[B2X]);
             }
             {
-                const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + j0;
                 const size_t scb = psc(c, t, j0);  // channels j0 .. +16 share a group
                 const float s_q = __ldg(p.sq + scb), s_k = __ldg(p.sk + scb);
                 const float s_a = __ldg(p.sa + scb), s_d = __ldg(p.sd + scb);
@@ -1074,7 +1074,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                     tmem_wait_ld();
                     if (hh == 0 && !cta_wait(&s.bar[B2X], (uint32_t)hj) && tid == 0) atomicOr(&s.bad, 1 << 27);
                     float kv[8], ev[8], qv[8], gv[8];
-                    ld_chunk16<true>(Bt0, t, ci, kv);
+                    ld_chunk16<true>(Kt, t, ci, kv);
                     ld_chunk16<true>(Bt0, t, 8 + ci, ev);
                     ld_chunk16<true>(Bt1, t, ci, qv);
                     ld_chunk16<true>(Bt1, t, 8 + ci, gv);
@@ -1104,12 +1104,12 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                             dotq = fmaf(oq[u], qv[u], dotq);
                             dotk = fmaf(ok[u], kv[u], dotk);
                         }
-                        float* pq_ = p.dqh + cb + u0;
-                        float* pk_ = p.dkh + cb + u0;
-                        *reinterpret_cast<float4*>(pq_) = make_float4(oq[0], oq[1], oq[2], oq[3]);
-                        *reinterpret_cast<float4*>(pq_ + 4) = make_float4(oq[4], oq[5], oq[6], oq[7]);
-                        *reinterpret_cast<float4*>(pk_) = make_float4(ok[0], ok[1], ok[2], ok[3]);
-                        *reinterpret_cast<float4*>(pk_ + 4) = make_float4(ok[4], ok[5], ok[6], ok[7]);
+                        float* qhb = p.dqh + (size_t)c * kC * kD;
+                        float* khb = p.dkh + (size_t)c * kC * kD;
+                        *grp4(qhb, t, j0 + u0) = make_float4(oq[0], oq[1], oq[2], oq[3]);
+                        *grp4(qhb, t, j0 + u0 + 4) = make_float4(oq[4], oq[5], oq[6], oq[7]);
+                        *grp4(khb, t, j0 + u0) = make_float4(ok[0], ok[1], ok[2], ok[3]);
+                        *grp4(khb, t, j0 + u0 + 4) = make_float4(ok[4], ok[5], ok[6], ok[7]);
                     } else {
                         st_chunk16<true>(Bt1, t, ci, oq);  // dq over q
                         st_chunk16<true>(Bt0, t, ci, ok);  // dk over k
@@ -1173,11 +1173,10 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 dq_dot += s.dot[0][i][t];
                 dk_dot += s.dot[1][i][t];
             }
-            const size_t cb = (size_t)c * kC * kD + (size_t)t * kD + 32 * g4;
             const size_t ro = tok * kD + 32 * g4;
 #pragma unroll 1
             for (int which = 0; which < 2; ++which) {
-                const float* dy = (which ? p.dkh : p.dqh) + cb;
+                const float* dyb = (which ? p.dkh : p.dqh) + (size_t)c * kC * kD;
                 const __nv_bfloat16* xr = reinterpret_cast<const __nv_bfloat16*>(which ? p.k : p.q) + ro;
                 __nv_bfloat16* dx = reinterpret_cast<__nv_bfloat16*>(which ? p.dk : p.dq) + ro;
                 const float r = which ? rk : rq, dot = which ? dk_dot : dq_dot;
@@ -1185,8 +1184,8 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 for (int i = 0; i < 4; ++i) {
                     float xv[8], o[8];
                     ld8_bf16(xr + 8 * i, xv);
-                    const float4 a0 = *reinterpret_cast<const float4*>(dy + 8 * i);
-                    const float4 a1 = *reinterpret_cast<const float4*>(dy + 8 * i + 4);
+                    const float4 a0 = *grp4(dyb, t, 32 * g4 + 8 * i);
+                    const float4 a1 = *grp4(dyb, t, 32 * g4 + 8 * i + 4);
                     const float dv8[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
@@ -1223,7 +1222,7 @@ int sm_count() {
 
 constexpr int kBprepSmem = 2 * kT16Bytes + 1024;
 constexpr int kBwd1Smem = 6 * kT16Bytes + sizeof(Bwd1Smem) + 1024;
-constexpr int kBwd2Smem = 4 * kT16Bytes + 2 * kT32Half + sizeof(Bwd2Smem) + 1024;
+constexpr int kBwd2Smem = 4 * kT16Bytes + 2 * kT32Half + kT16Block + sizeof(Bwd2Smem) + 1024;
 static_assert(kBwd2Smem <= 232448, "k2_bwd2 shared memory");
 template <int SLAB>
 constexpr int rev_smem() { return 3 * 128 * 128 * 4 + SLAB * 512 + 1024; }

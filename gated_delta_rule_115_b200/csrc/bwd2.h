@@ -14,7 +14,7 @@ struct BprepParams {
     CUtensorMap tdO;
     int T, H;
     const float* Qp;  // [nch][128][128]
-    float* Bp;        // Q'^T dO per chunk
+    float* Bp;        // Q'^T dO per chunk (grp4 layout)
     // fused output gate (zo non-null): tdO holds the gradient of the gated
     // output; dO = dO' sigmoid(zo) is written to dO_eff as fp16 (read by the
     // later kernels) and as bf16 to dO_effb (for the boundary-pivot path), and
@@ -33,7 +33,7 @@ struct RevParams {
     const float* S_chunks;  // chunk-start states
     const float* S_last;    // [B*H][128][128] final states (S_N)
     const float* dS_final;  // or null
-    float* dSc;             // G_{n+1} per chunk
+    float* dSc;             // G_{n+1} per chunk (grp4 layout)
     float* dS0;             // or null
     float* dgb;             // dLbar partials [128 / SLAB][nch][128]
     int N, nch;
@@ -66,7 +66,7 @@ struct Bwd2Params {
     const unsigned char *Y16, *dYR16;
     const __half *Pq, *Pk, *Pa, *Pd;      // k2_bwd1's partials (scaled fp16, see Bwd1Params)
     const float *sq, *sk, *sa, *sd;
-    float *dqh, *dkh;                     // fused prologue: dq^, dk^ before its Jacobian (fp32)
+    float *dqh, *dkh;                     // fused prologue: dq^, dk^ before its Jacobian (fp32, grp4 layout)
     const float* dgb;                     // [nslab][nch][128] partials of dLbar
     int nslab;
     void *dq, *dk, *dg, *de, *dgamma;
