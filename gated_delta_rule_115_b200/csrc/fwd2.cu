@@ -219,7 +219,9 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         tma_load_3d(dst, map, 0, y, z, &s.bar[bar]);
         tma_load_3d(dst + kT16Block, map, 64, y, z, &s.bar[bar]);
     };
-    auto issue_first = [&](int c) {  // g, k, e on BA; q, gamma on BB
+    // g, k, e on BA; q, gamma on BB.  Past the first chunk gamma is issued by
+    // the chunk itself, once the previous chunk's M tile has left S4.
+    auto issue_first = [&](int c, bool with_gamma) {
         int y, z;
         coords(c, y, z);
         mbar_arrive_expect_tx(&s.bar[BA], 3 * kT16Bytes);
@@ -228,7 +230,7 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         load_tile(S[2], &p.te, y, z, BA);
         mbar_arrive_expect_tx(&s.bar[BB], 2 * kT16Bytes);
         load_tile(S[3], &p.tq, y, z, BB);
-        load_tile(S[4], &p.tgam, y, z, BB);
+        if (with_gamma) load_tile(S[4], &p.tgam, y, z, BB);
     };
     // this thread's 4 chunks of 8 columns: chunk index 4h + i
     auto ld32 = [&](const unsigned char* tile, float* v) {
@@ -244,7 +246,7 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             if (!keep(c0 + j)) v[j] = 0.f;
         row_st32<false>(tile, t, h, v);
     };
-    if (tid == 0 && (int)blockIdx.x < nch) issue_first(blockIdx.x);
+    if (tid == 0 && (int)blockIdx.x < nch) issue_first(blockIdx.x, true);
 
     int it = 0;
     for (int c = blockIdx.x; c < nch; c += gridDim.x, ++it) {
@@ -252,8 +254,11 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         uint32_t pg = 0;  // parity of the merge barrier within this chunk
         int y, z;
         coords(c, y, z);
-        const size_t rbase = (size_t)c * kC * kD + (size_t)t * kD + c0;  // row t, column c0
 
+        if (tid == 0 && it > 0) {  // the previous chunk's M tile has left S4 and S5 (the wait below tells the rest)
+            bulk_wait_read();
+            load_tile(S[4], &p.tgam, y, z, BB);
+        }
         // ---- 1. log-decay prefix (warp scan over tokens), pivots
         // L = Tril(1) g: the inclusive prefix over the chunk's tokens as one
         // tensor-core product (clamped g and the ones are exact in bf16; fp32
@@ -616,7 +621,7 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         tc_fence_after();
         const int cn = c + gridDim.x;
         if (tid == 0 && ax) bulk_wait_read();  // M_QA (S5) stored before S5 is reused
-        if (tid == 0 && cn < nch) issue_first(cn);
+        if (tid == 0 && cn < nch) issue_first(cn, false);
         {
             float v[32];
             tm_ld32w(tm, q, c0, v);
@@ -626,10 +631,13 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
                 for (int j = 0; j < 32; ++j)
                     if (c0 + j == t) v[j] += dg;
             }
-            float* md = p.M + rbase;
+            {  // M row t, columns c0 ..: 128B-swizzled fp32 box h of the tile in S4 | S5
+                unsigned char* mb = (h < 2 ? S[4] : S[5]) + (h & 1) * 16384 + t * 128;
 #pragma unroll
-            for (int j = 0; j < 32; j += 4)
-                *reinterpret_cast<float4*>(md + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
+                for (int i = 0; i < 8; ++i)
+                    *reinterpret_cast<float4*>(mb + ((i ^ (t & 7)) << 4)) =
+                        make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+            }
             if (p.Mt) {
                 float* mt = p.Mt + (size_t)c * kC * kD + t;
 #pragma unroll 8
@@ -640,7 +648,14 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
 #pragma unroll
             for (int j = 0; j < 32; j += 4) *grp4(bb, t, c0 + j) = make_float4(v[j], v[j + 1], v[j + 2], v[j + 3]);
         }
-        sync_all();  // TMEM read out before the next chunk's products
+        fence_async_smem();
+        sync_all();  // TMEM read out before the next chunk's products; M tile complete
+        if (tid == 0) {
+#pragma unroll
+            for (int kb = 0; kb < 4; ++kb)
+                tma_store_3d(&p.tM, (kb < 2 ? S[4] : S[5]) + (kb & 1) * 16384, 32 * kb, c * kC, 0);
+            bulk_commit();
+        }
     }
     if (tid == 0) bulk_wait_all();
     if (tid == 0 && s.bad) atomicAdd(&g_v2_timeouts, 1u);
@@ -716,11 +731,6 @@ __global__ void __launch_bounds__(128, 1) k2_chain(const __grid_constant__ Chain
     sync_all();
     for (int n = 0; n < N; ++n) {
         const int st = n % STAGES;
-        if (p.S_chunks) {
-            float* d = p.S_chunks + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
-#pragma unroll
-            for (int c = 0; c < SLAB; c += 4) *reinterpret_cast<float4*>(d + c) = make_float4(Sr[c], Sr[c + 1], Sr[c + 2], Sr[c + 3]);
-        }
         // only the issuing thread waits for the transition tile: it alone reads it
         // (through the MMA), and it reloads the stage later in this step, so a
         // second waiter could see the barrier two phases on and miss its phase
@@ -729,6 +739,11 @@ __global__ void __launch_bounds__(128, 1) k2_chain(const __grid_constant__ Chain
             tc_fence_after();
             gemm_kk32<128, SLAB>(tm, saddr(Mst + st * MT), saddr(St), 0, SLAB, 128, false);
             mma_commit(&bar[STAGES]);
+        }
+        if (p.S_chunks) {  // record S_n while the product runs
+            float* d = p.S_chunks + ((size_t)bh * N + n) * kD * kD + (size_t)j * kD + c0;
+#pragma unroll
+            for (int c = 0; c < SLAB; c += 4) *reinterpret_cast<float4*>(d + c) = make_float4(Sr[c], Sr[c + 1], Sr[c + 2], Sr[c + 3]);
         }
         float Bc[SLAB];
 #pragma unroll
@@ -988,6 +1003,7 @@ cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st) {
         return cudaErrorInvalidValue;
     ip.B = a.B; ip.T = a.T; ip.H = a.H;
     ip.q = a.q; ip.gamma = a.gamma;
+    if (!map_rows32f(&ip.tM, a.M, (long long)nch * kD)) return cudaErrorInvalidValue;
     ip.M = a.M; ip.Mt = a.Mt; ip.Bn = a.Bn; ip.Qp = a.Qp; ip.Oi = a.Oi; ip.flags = a.flags;
     ip.aux = a.aux;
     ip.qk_raw = a.qk_raw; ip.rnorm = a.rnorm;

@@ -51,6 +51,7 @@ inline float* aux_Mt(unsigned char* aux, size_t nch) {
 
 struct IntraParams {
     CUtensorMap tq, tk, tv, tg, te, tw, tgam;  // token-major [B*T][H][128] bf16
+    CUtensorMap tM;                            // M_n as rows of 128 fp32 (stored as tiles)
     const void *q, *gamma;                     // the same tensors (plain loads)
     int B, T, H;
     float* M;      // chunk transitions M_n [j][i]: S_{n+1} = M_n S_n + B_n
