@@ -461,6 +461,10 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             fence_async_smem();
             sync_all();
         }
+        if (tid == 0) {  // k -> S0 (L_A consumed by the merges) for K~ in phase 6
+            mbar_arrive_expect_tx(&s.bar[BD], kT16Bytes);
+            load_tile(S[0], &p.tk, y, z, BD);
+        }
 
         if (ax && tid == 0) {  // T (S2) is final
             bulk_store(ax + AuxLayout::kT16, S[2], kT16Bytes);
@@ -487,8 +491,6 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         if (tid == 0) {
             gemm_km16(tm + 0, a1, 0, a4, 0, 0, 128, 128, kF16, false);  // L_K U
             mma_commit(&s.bar[BM3]);
-            mbar_arrive_expect_tx(&s.bar[BD], kT16Bytes);                // k -> S0
-            load_tile(S[0], &p.tk, y, z, BD);
         }
         waitb(s, BD, ph);
 #pragma unroll 1
@@ -514,6 +516,11 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         tm_to_row(384, S[5], [&](int col) { return col <= t; });
         waitb(s, BM4, ph);
         tc_fence_after();
+        if (tid == 0) {  // k -> S2 (T consumed by X; its record stored) for Kbar in phase 7
+            if (ax) bulk_wait_read();
+            mbar_arrive_expect_tx(&s.bar[BE], kT16Bytes);
+            load_tile(S[2], &p.tk, y, z, BE);
+        }
         {
             float v[32];
             tm_ld32w(tm, q, c0, v);  // W
@@ -540,9 +547,7 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             gemm_km16(tm + 256, a5, 0, a0, 0, 0, 256, 128, kF16, false, true);
             gemm_km16(tm + 384, a3, 0, a4, 0, 0, 128, 128, kF16, true);
             mma_commit(&s.bar[BM5]);
-            if (ax) bulk_wait_read();                       // T (S2), M_QK (S3) stored
-            mbar_arrive_expect_tx(&s.bar[BE], kT16Bytes);  // k -> S2
-            load_tile(S[2], &p.tk, y, z, BE);
+            if (ax) bulk_wait_read();  // M_QK (S3), M_QA (S5) stored
         }
         waitb(s, BM5, ph);
         tc_fence_after();
