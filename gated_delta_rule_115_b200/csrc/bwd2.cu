@@ -69,6 +69,14 @@ __device__ __forceinline__ void sync_all() {
     tc_fence_after();
 }
 
+// 8 bf16 packed in 16 bytes -> floats.
+__device__ __forceinline__ void unpack8_bf16(const uint4 u, float* v) {
+    unpack16<true>(u.x, v[0], v[1]);
+    unpack16<true>(u.y, v[2], v[3]);
+    unpack16<true>(u.z, v[4], v[5]);
+    unpack16<true>(u.w, v[6], v[7]);
+}
+
 // 8 consecutive bf16 of a token-major row -> floats.
 __device__ __forceinline__ void ld8_bf16(const __nv_bfloat16* p, float* v) {
     const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
@@ -930,6 +938,10 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
         for (int hj = 0; hj < 2; ++hj) {
             const int j0 = 64 * hj + 16 * g4;  // this thread's channels
             const int r0 = 16 * g4;            // their rows in the half tiles
+            // e of the row for Am, requested before the log-decay product
+            const __nv_bfloat16* ein = reinterpret_cast<const __nv_bfloat16*>(p.e) + tok * kD + j0;
+            const uint4 eraw0 = __ldg(reinterpret_cast<const uint4*>(ein));
+            const uint4 eraw1 = __ldg(reinterpret_cast<const uint4*>(ein + 8));
             // log decay of the half's 64 channels: L = Tril(1) clamp(g) as one
             // product (g block in Bt1, ones tile in Bt0: both free until the
             // pivoted operands; TMEM columns 0..63 free until the first round)
@@ -986,14 +998,13 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 if (far) atomicOr(p.flags, 1);
             }
             __syncthreads();
-            const __nv_bfloat16* ein = reinterpret_cast<const __nv_bfloat16*>(p.e) + tok * kD + j0;
             const __nv_bfloat16* qin = reinterpret_cast<const __nv_bfloat16*>(p.q) + tok * kD + j0;
             const __nv_bfloat16* gin_ = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + tok * kD + j0;
             {  // Am -> Bt0, Km -> Bt1
                 float kv[16], ev[16], am[16], km[16];
                 ld_chunk16<true>(Kt, t, 2 * g4, kv); ld_chunk16<true>(Kt, t, 2 * g4 + 1, kv + 8);
                 if (QKRAW) { prologue8(kv, rk); prologue8(kv + 8, rk); }
-                ld8_bf16(ein, ev); ld8_bf16(ein + 8, ev + 8);
+                unpack8_bf16(eraw0, ev); unpack8_bf16(eraw1, ev + 8);
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
                     km[u] = kv[u] * ex2(s.P2[j0 + u] - L[u]);
@@ -1010,17 +1021,23 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             //  R3: dL_A^T = -Y dYR^T (strict upper), dM_QA^T = -Y dO^T (inclusive upper) -> dAm
             //  R4: dL_K^T = U dYR^T (strict upper), dM_QK^T = U dO^T (inclusive upper) -> dKm
             // with Am, Km in Bt0, Bt1 for R1, R2 and Kp, Qp for R3, R4.
+            // q and gamma of the row for R3's operands, requested two rounds ahead
+            uint4 qg[4];
+            qg[0] = __ldg(reinterpret_cast<const uint4*>(qin));
+            qg[1] = __ldg(reinterpret_cast<const uint4*>(qin + 8));
+            qg[2] = __ldg(reinterpret_cast<const uint4*>(gin_));
+            qg[3] = __ldg(reinterpret_cast<const uint4*>(gin_ + 8));
 #pragma unroll 1
             for (int r = 0; r < 4; ++r) {
                 if (r == 2) {  // Kp -> Bt0, Qp -> Bt1
                     float kv[16], qv[16], gv[16], kp[16], qp[16];
                     ld_chunk16<true>(Kt, t, 2 * g4, kv); ld_chunk16<true>(Kt, t, 2 * g4 + 1, kv + 8);
-                    ld8_bf16(qin, qv); ld8_bf16(qin + 8, qv + 8);
+                    unpack8_bf16(qg[0], qv); unpack8_bf16(qg[1], qv + 8);
                     if (QKRAW) {
                         prologue8(kv, rk); prologue8(kv + 8, rk);
                         prologue8(qv, rq); prologue8(qv + 8, rq);
                     }
-                    ld8_bf16(gin_, gv); ld8_bf16(gin_ + 8, gv + 8);
+                    unpack8_bf16(qg[2], gv); unpack8_bf16(qg[3], gv + 8);
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
                         const float ep = ex2(L[u] - s.P2[j0 + u]);
