@@ -518,6 +518,13 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             tma_load_3d(S[0], &p.tg, 0, hd, z, &s.bar[B1G]);
             tma_load_3d(S[0] + kT16Block, &p.tg, 64, hd, z, &s.bar[B1G]);
         }
+        // S_n row t (row-major, from DRAM), requested before the log-decay product
+        float4 srow[8];
+        {
+            const float* src = p.S_chunks + cb;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) srow[j] = __ldg(reinterpret_cast<const float4*>(src + 4 * j));
+        }
         // log decay of row t, columns c0..: L = Tril(1) clamp(g) as one product
         // (ones tile in S3, free until the gradient-state tile); E = 2^L,
         // Eb = 2^(Lbar - L), Lbar = the product's last row
@@ -557,10 +564,9 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
         float sS, sG;
         {
             float v[32];
-            const float* src = p.S_chunks + cb;
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
-                const float4 x = __ldg(reinterpret_cast<const float4*>(src + j));
+                const float4 x = srow[j >> 2];
                 v[j] = x.x; v[j + 1] = x.y; v[j + 2] = x.z; v[j + 3] = x.w;
             }
             sS = pow2_scale(block_absmax(v, s.red, warp, lane));
@@ -596,6 +602,12 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             gemm_km16(tm + 128, a[2], 0, a[0], 0, 0, 128, 128, kF16, false);
             mma_commit(&s.bar[B1M1]);
         }
+        float4 urow[8];  // U' row t, requested while the products run
+        {
+            const float* ub = reinterpret_cast<const float*>(ax + AuxLayout::kUp);
+#pragma unroll
+            for (int j = 0; j < 8; ++j) urow[j] = __ldg(grp4(ub, t, c0 + 4 * j));
+        }
         waitb(B1M1, ph);
         tc_fence_after();
         // ---- phase 2: Pq; Y = W S + U' -> fp16 tile S2 (also saved for k2_bwd2)
@@ -606,10 +618,9 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             for (int j = 0; j < 32; ++j) d[j] *= sS * ex2(L[j]);
             st_scaled32(reinterpret_cast<uint4*>(p.Pq) + pb, p.sq + scb, d);
             tm_ld32w(tm, q, 128 + c0, d);
-            const float* ub = reinterpret_cast<const float*>(ax + AuxLayout::kUp);
 #pragma unroll
             for (int j = 0; j < 32; j += 4) {
-                const float4 x = __ldg(grp4(ub, t, c0 + j));
+                const float4 x = urow[j >> 2];
                 d[j] = d[j] * sS + x.x; d[j + 1] = d[j + 1] * sS + x.y;
                 d[j + 2] = d[j + 2] * sS + x.z; d[j + 3] = d[j + 3] * sS + x.w;
             }

@@ -549,6 +549,18 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             mma_commit(&s.bar[BM5]);
             if (ax) bulk_wait_read();  // M_QK (S3), M_QA (S5) stored
         }
+        // q and gamma of row t for Q~, requested while the products run
+        uint4 qraw[4], graw[4];
+        {
+            const size_t ri = (((size_t)(c / N / p.H) * p.T + (size_t)(c % N) * kC + t) * p.H + y) * kD + c0;
+            const __nv_bfloat16* qsrc = reinterpret_cast<const __nv_bfloat16*>(p.q) + ri;
+            const __nv_bfloat16* gsrc = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + ri;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                qraw[i] = __ldg(reinterpret_cast<const uint4*>(qsrc + 8 * i));
+                graw[i] = __ldg(reinterpret_cast<const uint4*>(gsrc + 8 * i));
+            }
+        }
         waitb(s, BM5, ph);
         tc_fence_after();
         if (tid == 0) {
@@ -560,13 +572,10 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             float v[32];
             tm_ld32w(tm + 256, q, c0, v);
             float* qb = p.Qp + (size_t)c * kC * kD;
-            const size_t ri = (((size_t)(c / N / p.H) * p.T + (size_t)(c % N) * kC + t) * p.H + y) * kD + c0;
-            const __nv_bfloat16* qsrc = reinterpret_cast<const __nv_bfloat16*>(p.q) + ri;
-            const __nv_bfloat16* gsrc = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + ri;
 #pragma unroll
             for (int j = 0; j < 32; j += 8) {
-                const uint4 qw = __ldg(reinterpret_cast<const uint4*>(qsrc + j));
-                const uint4 gw = __ldg(reinterpret_cast<const uint4*>(gsrc + j));
+                const uint4 qw = qraw[j >> 3];
+                const uint4 gw = graw[j >> 3];
                 const uint32_t qa[4] = {qw.x, qw.y, qw.z, qw.w}, ga[4] = {gw.x, gw.y, gw.z, gw.w};
                 float r[8];
 #pragma unroll
