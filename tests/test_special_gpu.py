@@ -1,6 +1,6 @@
-"""GPU parity of the special cases the recurrence reduces to (the benchmark spec;
-"Muir", wolonglab.org page, "Methodology": decay, erase and write gates of the
-gated delta rule), run through the on-chip path (bf16, dk = dv = 128, chunk
+"""GPU parity of the special cases the recurrence reduces to ("Muir",
+wolonglab.org page, "Methodology": decay, erase and write gates of the gated
+delta rule), run through the on-chip path (bf16, dk = dv = 128, chunk
 128), forward and backward, against the fp64 oracle, whose own pins fix these
 cases to closed forms:
 
