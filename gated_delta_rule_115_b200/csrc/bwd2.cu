@@ -944,6 +944,7 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 st_chunk16<false>(tdO, t, 4 * g4 + i, v);
             }
         }
+        if (tid == 0) bulk_wait_read();  // the previous chunk's gradient tiles have left Bt0, Bt1
         fence_async_smem();
         sync_all();
 
@@ -1070,6 +1071,8 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
             }
             // the second half's rounds were the tiles' last readers
             if (hj == 1 && tid == 0 && c + (int)gridDim.x < nch) load_tiles(c + gridDim.x);
+            if (hj == 1 && tid < 4 * p.nslab && c + (int)gridDim.x < nch)  // the next chunk's dLbar partials -> L2
+                prefetch_l2(p.dgb + ((size_t)(tid >> 2) * nch + c + gridDim.x) * kD + 32 * (tid & 3));
             // ---- readout: final gradients of channels j0 .. j0 + 15 of row t.
             // e (Bt0) and q, gamma (Bt1) of the half come by TMA into the
             // operand tiles, free now (k has its own tile); each thread forms
@@ -1191,7 +1194,9 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                     st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dg) + tok * kD + j0 + 8 * hh, o);
                 }
             }
-            if (tid == 0) bulk_wait_read();  // the stores have left Bt0, Bt1
+            // the stores have left Bt0, Bt1 before the next half writes them (after
+            // the second half, before the next chunk's first half)
+            if (hj == 0 && tid == 0) bulk_wait_read();
             sync_all();
         }
         if (QKRAW) {
