@@ -45,6 +45,8 @@ constexpr uint32_t kBlk = 16384;  // one 64-column block of a 128-row T16 tile
 struct GatesFwdParams {
     CUtensorMap tlat;
     CUtensorMap tU[kMaxFam];
+    CUtensorMap tout[kMaxFam];  // with stage: the gates as token-major bf16 tiles
+    int stage;                  // 1: the epilogue stages each head's tile and stores it by TMA
     int nfam, H;
     int off[kMaxFam], r[kMaxFam], act[kMaxFam];
     const float* bias[kMaxFam];
@@ -54,6 +56,8 @@ struct GatesFwdParams {
 struct GatesDpreParams {
     CUtensorMap tlat;
     CUtensorMap tU[kMaxFam];
+    CUtensorMap tdo[kMaxFam];            // dgate as token-major bf16 tiles (loaded)
+    CUtensorMap tdh[kMaxFam], tdlo[kMaxFam];  // dpre hi, lo (stored)
     int nfam, H, R;
     int off[kMaxFam], r[kMaxFam], act[kMaxFam];
     const float* bias[kMaxFam];
@@ -94,24 +98,6 @@ __device__ __forceinline__ float act_grad(int act, float x) {
     return 1.f;
 }
 
-// 64 TMEM columns [col, col + 64) of this thread's lane.
-__device__ __forceinline__ void tm_ld64(uint32_t tm, int q, int col, float* v) {
-    float a[32], b[32];
-    tmem_ld32(taddr(tm, 32 * q, col), a);
-    tmem_ld32(taddr(tm, 32 * q, col + 32), b);
-    tmem_wait_ld();
-#pragma unroll
-    for (int i = 0; i < 32; ++i) { v[i] = a[i]; v[32 + i] = b[i]; }
-}
-
-__device__ __forceinline__ void ld8_bf16g(const __nv_bfloat16* p, float* v) {
-    const uint4 u = __ldg(reinterpret_cast<const uint4*>(p));
-    unpack16<true>(u.x, v[0], v[1]);
-    unpack16<true>(u.y, v[2], v[3]);
-    unpack16<true>(u.z, v[4], v[5]);
-    unpack16<true>(u.w, v[6], v[7]);
-}
-
 __device__ __forceinline__ void st8_bf16g(__nv_bfloat16* p, const float* v) {
     uint4 u;
     u.x = pack_bf16(v[0], v[1]);
@@ -147,6 +133,7 @@ __global__ void __launch_bounds__(512, 1) k2_gates(const __grid_constant__ Gates
     }
     unsigned char* A = sm;
     unsigned char* U = sm + nA * kBlk;  // two stages of two blocks
+    unsigned char* O = U + 4 * kBlk;    // with stage: one head's output tile (T16)
     if (tid == 0) {
         mbar_init(&barA, 1);
         for (int s = 0; s < 2; ++s) { mbar_init(&barU[s], 1); mbar_init(&barM[s], 1); }
@@ -186,6 +173,7 @@ __global__ void __launch_bounds__(512, 1) k2_gates(const __grid_constant__ Gates
     for (int idx = 0; idx < n; ++idx) {
         const int s = idx & 1, X = idx / p.H, h = idx % p.H;
         if (tid == 0 && idx + 1 < n) issue(idx + 1);  // into the other accumulator
+        if (p.stage && tid == 0) bulk_wait_read();   // the previous tile has left O (the wait below tells the rest)
         if (!cta_wait(&barM[s], (uint32_t)((idx >> 1) & 1)) && tid == 0) bad = 1;
         if (tid == 0 && idx + 2 < n) load_U(idx + 2, s);  // product idx has read stage s
         float v[32];
@@ -199,10 +187,20 @@ __global__ void __launch_bounds__(512, 1) k2_gates(const __grid_constant__ Gates
             float o[8];
 #pragma unroll
             for (int u = 0; u < 8; ++u) o[u] = act_f(act, v[j + u] + __ldg(bias + j + u));
-            st8_bf16g(dst + j, o);
+            if (p.stage)
+                st_chunk16<true>(O, t, 4 * half + j / 8, o);
+            else
+                st8_bf16g(dst + j, o);
         }
-        sync_all();  // accumulator s read out before product idx + 2 overwrites it
+        if (p.stage) fence_async_smem();
+        sync_all();  // accumulator s read out before product idx + 2 overwrites it; tile complete
+        if (p.stage && tid == 0) {
+            tma_store_3d(&p.tout[X], O, 0, h, (int)row0);
+            tma_store_3d(&p.tout[X], O + kBlk, 64, h, (int)row0);
+            bulk_commit();
+        }
     }
+    if (tid == 0) bulk_wait_all();
     if (tid == 0 && bad) atomicOr(&g_gates_timeouts, 1u);
     sync_all();
     if (warp == 0) tmem_dealloc(tm, 256);
@@ -217,8 +215,9 @@ __global__ void __launch_bounds__(512, 1) k2_gates_dpre(const __grid_constant__ 
     unsigned char* sm = align1024(smraw);
     unsigned char* A = sm;                 // the family's latent slice (2 blocks)
     unsigned char* U = sm + 2 * kBlk;      // two stages of two blocks
-    unsigned char* Dp = sm + 6 * kBlk;     // dpre of one head, bf16 T16: hi, then lo
-    __shared__ uint64_t barA, barU[2], barM;
+    unsigned char* Dp = sm + 6 * kBlk;     // dpre of one head, bf16 T16: hi, then lo (stored by TMA)
+    unsigned char* Do = sm + 10 * kBlk;    // dgate of a head, two stages of a T16 tile
+    __shared__ uint64_t barA, barU[2], barM, barD[2];
     __shared__ uint32_t tslot;
     __shared__ int bad;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -229,6 +228,8 @@ __global__ void __launch_bounds__(512, 1) k2_gates_dpre(const __grid_constant__ 
         mbar_init(&barU[0], 1);
         mbar_init(&barU[1], 1);
         mbar_init(&barM, 1);
+        mbar_init(&barD[0], 1);
+        mbar_init(&barD[1], 1);
         bad = 0;
         fence_barrier_init();
     }
@@ -236,6 +237,17 @@ __global__ void __launch_bounds__(512, 1) k2_gates_dpre(const __grid_constant__ 
     sync_all();
     const uint32_t tm = tslot;  // columns 0..127: pre; 128..255: dlatent of the family
     uint32_t pm = 0;
+    const int n = p.nfam * p.H;
+    auto load_D = [&](int idx) {  // dgate of (family, head) idx -> stage idx & 1
+        const int s = idx & 1, X = idx / p.H, h = idx % p.H;
+        mbar_arrive_expect_tx(&barD[s], 2 * kBlk);
+        tma_load_3d(Do + s * 2 * kBlk, &p.tdo[X], 0, h, (int)row0, &barD[s]);
+        tma_load_3d(Do + s * 2 * kBlk + kBlk, &p.tdo[X], 64, h, (int)row0, &barD[s]);
+    };
+    if (tid == 0) {
+        load_D(0);
+        if (n > 1) load_D(1);
+    }
     auto load_U = [&](int idx) {
         const int s = idx & 1, X = idx / p.H, h = idx % p.H;
         mbar_arrive_expect_tx(&barU[s], 2u * p.r[X] * 128u);
@@ -260,32 +272,44 @@ __global__ void __launch_bounds__(512, 1) k2_gates_dpre(const __grid_constant__ 
                 gemm_km16(tm, saddr(A), 0, saddr(U + s * 2 * kBlk), 0, 0, 128, r, kBF16, false);
                 mma_commit(&barM);
             }
-            if (!cta_wait(&barM, pm) && tid == 0) bad = 1;
+            if (tid == 0) bulk_wait_read();  // the previous head's dpre tiles have left Dp
+            {  // the product and this head's dgate tile; one block barrier releases all
+                int ok = 1;
+                if (tid < 32) ok = (mbar_wait(&barM, pm) && mbar_wait(&barD[s], (uint32_t)((idx >> 1) & 1))) ? 1 : 0;
+                ok = __syncthreads_and(ok);
+                tc_fence_after();
+                if (!ok && tid == 0) bad = 1;
+            }
             pm ^= 1u;
-            {  // dpre of row t, channels 32 half .. +32 -> global and the Dp tile
+            {  // dpre of row t, channels 32 half .. +32 -> the Dp tiles
                 float v[32];
                 tmem_ld32(taddr(tm, 32 * q, 32 * half), v);
                 tmem_wait_ld();
-                const size_t ro = ((size_t)(row0 + t) * p.H + h) * 128 + 32 * half;
                 const float* bias = p.bias[X] + 128 * h + 32 * half;
 #pragma unroll
                 for (int j = 0; j < 32; j += 8) {
                     float dg[8], hi[8], lo[8];
-                    ld8_bf16g(p.dout[X] + ro + j, dg);
+                    ld_chunk16<true>(Do + s * 2 * kBlk, t, 4 * half + j / 8, dg);
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const float o = dg[u] * act_grad(act, v[j + u] + __ldg(bias + j + u));
                         hi[u] = __bfloat162float(__float2bfloat16_rn(o));
                         lo[u] = o - hi[u];
                     }
-                    st8_bf16g(p.dpre[X] + ro + j, hi);
-                    st8_bf16g(p.dpre_lo[X] + ro + j, lo);
                     st_chunk16<true>(Dp, t, 4 * half + j / 8, hi);
                     st_chunk16<true>(Dp + 2 * kBlk, t, 4 * half + j / 8, lo);
                 }
             }
             fence_async_smem();
             sync_all();
+            if (tid == 0) {  // dpre hi, lo leave by TMA store; the next-but-one dgate tile into stage s
+                tma_store_3d(&p.tdh[X], Dp, 0, h, (int)row0);
+                tma_store_3d(&p.tdh[X], Dp + kBlk, 64, h, (int)row0);
+                tma_store_3d(&p.tdlo[X], Dp + 2 * kBlk, 0, h, (int)row0);
+                tma_store_3d(&p.tdlo[X], Dp + 3 * kBlk, 64, h, (int)row0);
+                bulk_commit();
+                if (idx + 2 < n) load_D(idx + 2);
+            }
             if (tid == 0) {  // dlatent (+)= dpre U_h^T: A = Dp (K = channels), B = U (rows i, K = channels)
                 gemm_kk16(tm + 128, saddr(Dp), 0, saddr(U + s * 2 * kBlk), 0, 0, r, 128, kBF16, h > 0);
                 gemm_kk16(tm + 128, saddr(Dp + 2 * kBlk), 0, saddr(U + s * 2 * kBlk), 0, 0, r, 128, kBF16, true);
@@ -310,6 +334,7 @@ __global__ void __launch_bounds__(512, 1) k2_gates_dpre(const __grid_constant__ 
         }
         sync_all();
     }
+    if (tid == 0) bulk_wait_all();
     if (tid == 0 && bad) atomicOr(&g_gates_timeouts, 2u);
     sync_all();
     if (warp == 0) tmem_dealloc(tm, 256);
@@ -415,7 +440,12 @@ cudaError_t run_gates_fwd(const GatesArgs& a, cudaStream_t st) {
         p.bias[X] = f.bias; p.out[X] = static_cast<__nv_bfloat16*>(f.out);
         nblk += f.r / 64;
     }
-    const int smem = (nblk + 4) * (int)kBlk + 1024;
+    // with room for a staged output tile, each head's gates leave by TMA store
+    p.stage = (nblk + 6) * (int)kBlk + 1024 <= 232448;
+    if (p.stage)
+        for (int X = 0; X < a.nfam; ++X)
+            if (!map_tokens16(&p.tout[X], a.fam[X].out, 1, (int)a.rows, a.H)) return cudaErrorInvalidValue;
+    const int smem = (nblk + (p.stage ? 6 : 4)) * (int)kBlk + 1024;
     cudaError_t e = cudaFuncSetAttribute(k2_gates, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
     if (e != cudaSuccess) return e;
     MUIR_TIMED("k2_gates", st, k2_gates<<<(int)(a.rows / 128), 512, smem, st>>>(p));
@@ -436,8 +466,11 @@ cudaError_t run_gates_bwd(const GatesArgs& a, cudaStream_t st) {
         if ((f.r != 64 && f.r != 128) || f.off % 8 || f.off + f.r > a.R) return cudaErrorInvalidValue;
         if (!map_2d16(&p.tU[X], f.U, a.H * 128, f.r, f.r)) return cudaErrorInvalidValue;
         if (!map_tokens16(&q.tdp[X], f.dpre, 1, (int)a.rows, a.H) ||
-            !map_tokens16(&q.tdl[X], f.dpre_lo, 1, (int)a.rows, a.H))
+            !map_tokens16(&q.tdl[X], f.dpre_lo, 1, (int)a.rows, a.H) ||
+            !map_tokens16(&p.tdo[X], f.dout, 1, (int)a.rows, a.H))
             return cudaErrorInvalidValue;
+        p.tdh[X] = q.tdp[X];
+        p.tdlo[X] = q.tdl[X];
         p.off[X] = q.off[X] = f.off; p.r[X] = q.r[X] = f.r; p.act[X] = f.act;
         p.bias[X] = f.bias;
         p.dout[X] = static_cast<const __nv_bfloat16*>(f.dout);
@@ -447,7 +480,7 @@ cudaError_t run_gates_bwd(const GatesArgs& a, cudaStream_t st) {
     }
     cudaError_t e = cudaMemsetAsync(a.dlatent, 0, (size_t)a.rows * a.R * 2, st);
     if (e != cudaSuccess) return e;
-    const int smem1 = 10 * (int)kBlk + 1024;
+    const int smem1 = 14 * (int)kBlk + 1024;
     if ((e = cudaFuncSetAttribute(k2_gates_dpre, cudaFuncAttributeMaxDynamicSharedMemorySize, smem1)) != cudaSuccess) return e;
     MUIR_TIMED("k2_gates_dpre", st, k2_gates_dpre<<<(int)(a.rows / 128), 512, smem1, st>>>(p));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
