@@ -185,8 +185,11 @@ __global__ void __launch_bounds__(512, 1) k2_gates(const __grid_constant__ Gates
 #pragma unroll
         for (int j = 0; j < 32; j += 8) {
             float o[8];
+            const float4 b0 = __ldg(reinterpret_cast<const float4*>(bias + j));  // (bias 16-byte aligned)
+            const float4 b1 = __ldg(reinterpret_cast<const float4*>(bias + j + 4));
+            const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
-            for (int u = 0; u < 8; ++u) o[u] = act_f(act, v[j + u] + __ldg(bias + j + u));
+            for (int u = 0; u < 8; ++u) o[u] = act_f(act, v[j + u] + bb[u]);
             if (p.stage)
                 st_chunk16<true>(O, t, 4 * half + j / 8, o);
             else
@@ -290,9 +293,12 @@ __global__ void __launch_bounds__(512, 1) k2_gates_dpre(const __grid_constant__ 
                 for (int j = 0; j < 32; j += 8) {
                     float dg[8], hi[8], lo[8];
                     ld_chunk16<true>(Do + s * 2 * kBlk, t, 4 * half + j / 8, dg);
+                    const float4 b0 = __ldg(reinterpret_cast<const float4*>(bias + j));
+                    const float4 b1 = __ldg(reinterpret_cast<const float4*>(bias + j + 4));
+                    const float bb[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
-                        const float o = dg[u] * act_grad(act, v[j + u] + __ldg(bias + j + u));
+                        const float o = dg[u] * act_grad(act, v[j + u] + bb[u]);
                         hi[u] = __bfloat162float(__float2bfloat16_rn(o));
                         lo[u] = o - hi[u];
                     }
