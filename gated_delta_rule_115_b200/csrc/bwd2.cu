@@ -69,6 +69,13 @@ __device__ __forceinline__ void sync_all() {
     tc_fence_after();
 }
 
+// 8 consecutive floats of a shared-memory table (32-byte aligned) in two 16-byte loads.
+__device__ __forceinline__ void lds8(const float* p, float* v) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
+
 // 8 bf16 packed in 16 bytes -> floats.
 __device__ __forceinline__ void unpack8_bf16(const uint4 u, float* v) {
     unpack16<true>(u.x, v[0], v[1]);
@@ -431,7 +438,7 @@ __global__ void __launch_bounds__(128, 1) k2_chain_rev(const __grid_constant__ R
 
 namespace {
 struct Bwd1Smem {
-    float Lb[kD];
+    alignas(16) float Lb[kD];
     float red[16];
     uint64_t bar[20];
     uint32_t tslot;
@@ -650,7 +657,12 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             float d[32];
             tm_ld32w(tm, q, 128 + c0, d);  // dAbar / sG
 #pragma unroll
-            for (int j = 0; j < 32; ++j) d[j] *= sG * ex2(s.Lb[c0 + j] - L[j]);
+            for (int jj = 0; jj < 32; jj += 8) {
+                float lb[8];
+                lds8(&s.Lb[c0 + jj], lb);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) d[jj + u] *= sG * ex2(lb[u] - L[jj + u]);
+            }
             st_scaled32(reinterpret_cast<uint4*>(p.Pa) + pb, p.sa + scb, d);
         }
         waitb(B1A, ph);  // (its block barrier also orders the reads of B1 above)
@@ -715,9 +727,14 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
             tm_ld32w(tm, q, c0, d);         // dK~ / sS
             tm_ld32w(tm, q, 384 + c0, e2);  // dKbar / sG
 #pragma unroll
-            for (int j = 0; j < 32; ++j) {
-                d[j] *= sS * ex2(L[j]);                    // dK~ 2^L
-                e2[j] *= sG * ex2(s.Lb[c0 + j] - L[j]);  // dKbar 2^(Lbar-L)
+            for (int jj = 0; jj < 32; jj += 8) {
+                float lb[8];
+                lds8(&s.Lb[c0 + jj], lb);
+#pragma unroll
+                for (int u = 0; u < 8; ++u) {
+                    d[jj + u] *= sS * ex2(L[jj + u]);                 // dK~ 2^L
+                    e2[jj + u] *= sG * ex2(lb[u] - L[jj + u]);       // dKbar 2^(Lbar-L)
+                }
             }
             st_scaled32_pm(reinterpret_cast<uint4*>(p.Pk) + pb, p.sk + scb, reinterpret_cast<uint4*>(p.Pd) + pb, p.sd + scb, d, e2);  // Pk, Pd
         }
@@ -771,9 +788,9 @@ __global__ void __launch_bounds__(512, 1) k2_bwd1(const __grid_constant__ Bwd1Pa
 
 namespace {
 struct Bwd2Smem {
-    float P2[kD];
-    float sfx[4][kD];  // per-quarter totals of the reverse scan
-    float dgb[kD];     // dLbar of the chunk (value slabs summed in a fixed order)
+    alignas(16) float P2[kD];
+    alignas(16) float sfx[4][kD];  // per-quarter totals of the reverse scan
+    alignas(16) float dgb[kD];     // dLbar of the chunk (value slabs summed in a fixed order)
     float dot[2][8][kC];  // fused prologue: row dots dq^.q^ and dk^.k^ per (half, warp group)
     uint64_t bar[8];
     uint32_t tslot;
@@ -1019,9 +1036,11 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 ld_chunk16<true>(Kt, t, 2 * g4, kv); ld_chunk16<true>(Kt, t, 2 * g4 + 1, kv + 8);
                 if (QKRAW) { prologue8(kv, rk); prologue8(kv + 8, rk); }
                 unpack8_bf16(eraw0, ev); unpack8_bf16(eraw1, ev + 8);
+float p16[16];
+                lds8(&s.P2[j0], p16); lds8(&s.P2[j0 + 8], p16 + 8);
 #pragma unroll
                 for (int u = 0; u < 16; ++u) {
-                    km[u] = kv[u] * ex2(s.P2[j0 + u] - L[u]);
+                    km[u] = kv[u] * ex2(p16[u] - L[u]);
                     am[u] = ev[u] * km[u];
                 }
                 put_t(Bt0, r0, am);
@@ -1052,9 +1071,11 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                         prologue8(qv, rq); prologue8(qv + 8, rq);
                     }
                     unpack8_bf16(qg[2], gv); unpack8_bf16(qg[3], gv + 8);
+                    float p16[16];
+                    lds8(&s.P2[j0], p16); lds8(&s.P2[j0 + 8], p16 + 8);
 #pragma unroll
                     for (int u = 0; u < 16; ++u) {
-                        const float ep = ex2(L[u] - s.P2[j0 + u]);
+                        const float ep = ex2(L[u] - p16[u]);
                         kp[u] = kv[u] * ep;
                         qp[u] = qv[u] * gv[u] * ep;
                     }
@@ -1114,11 +1135,13 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                     ld_chunk16<true>(Bt1, t, 8 + ci, gv);
                     if (QKRAW) { prologue8(kv, rk); prologue8(qv, rq); }
                     float oq[8], og[8], ok[8], oe[8];
+                    float p8[8];
+                    lds8(&s.P2[j0 + u0], p8);
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const int j = u0 + u;
-                        const float ep = ex2(L[j] - s.P2[j0 + j]);
-                        const float em = ex2(s.P2[j0 + j] - L[j]);
+                        const float ep = ex2(L[j] - p8[u]);
+                        const float em = ex2(p8[u] - L[j]);
                         const float qh = qv[u] * gv[u];
                         const float dqh = a_q[u] * ep + pq[u];
                         oq[u] = dqh * gv[u];
@@ -1182,14 +1205,19 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 }
 #pragma unroll
                 for (int hh = 0; hh < 2; ++hh) {
-                    float o[8];
+                    float o[8], post[8];
+                    lds8(&s.dgb[j0 + 8 * hh], post);
+                    for (int qq = q + 1; qq < 4; ++qq) {
+                        float f8[8];
+                        lds8(&s.sfx[qq][j0 + 8 * hh], f8);
+#pragma unroll
+                        for (int u = 0; u < 8; ++u) post[u] += f8[u];
+                    }
 #pragma unroll
                     for (int u = 0; u < 8; ++u) {
                         const int j = 8 * hh + u;
-                        float post = s.dgb[j0 + j];
-                        for (int qq = q + 1; qq < 4; ++qq) post += s.sfx[qq][j0 + j];
                         // the clamp g >= -20 passes no gradient below it
-                        o[u] = ((gkeep >> j) & 1u) ? dL[j] + post : 0.f;
+                        o[u] = ((gkeep >> j) & 1u) ? dL[j] + post[u] : 0.f;
                     }
                     st8_bf16(reinterpret_cast<__nv_bfloat16*>(p.dg) + tok * kD + j0 + 8 * hh, o);
                 }

@@ -74,10 +74,9 @@ __device__ __forceinline__ void bf16_split(float x, float& hi, float& lo) {
 // ------------------------------------------------------------------ k2_intra
 
 struct IntraSmem {
-    float tot[4][kC];   // per-quarter totals of the log-decay scan
-    float P2[kD];       // pivot (log2 units)
-    float eP2[kD];      // 2^P2
-    float Lb[kD];       // chunk total (log2 units)
+    alignas(16) float P2[kD];   // pivot (log2 units)
+    alignas(16) float eP2[kD];  // 2^P2
+    alignas(16) float Lb[kD];   // chunk total (log2 units)
     float lblk[4][32][33];  // strictly lower 32x32 diagonal blocks of L_A (leaf inverses)
     float nrm[4][kC];   // fused prologue: per-quarter sums of SiLU(x)^2 of each row
     uint64_t bar[16];
@@ -86,6 +85,13 @@ struct IntraSmem {
 };
 
 enum { BA = 0, BB, BC, BD, BE, BF, BM1, BM2, BM3, BM4, BM5, BM6, BG, BL };
+
+// 8 consecutive floats of a shared-memory table (32-byte aligned) in two 16-byte loads.
+__device__ __forceinline__ void lds8(const float* p, float* v) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0], b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w;
+    v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+}
 
 // All threads call: warp 0 polls, the block barrier releases the rest.
 __device__ __forceinline__ bool waitb(IntraSmem& s, int i, uint32_t parity) {
@@ -313,9 +319,11 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             ld_chunk16<true>(S[1], t, 4 * h + i, kv);
             if (QKRAW) prologue8(kv, rk);
             ld_chunk16<true>(S[2], t, 4 * h + i, ev);
+            float pv8[8];
+            lds8(&s.P2[c0 + 8 * i], pv8);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const float pv = s.P2[c0 + 8 * i + u];
+                const float pv = pv8[u];
                 const float ep = ex2(L[u] - pv), em = ex2(pv - L[u]);
                 kp[u] = kv[u] * ep;
                 bf16_split(kv[u] * em, kmh[u], kml[u]);
@@ -349,9 +357,11 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             ld_chunk16<true>(S[3], t, 4 * h + i, qv);
             if (QKRAW) prologue8(qv, rq);
             ld_chunk16<true>(S[4], t, 4 * h + i, gv);
+            float pv8[8];
+            lds8(&s.P2[c0 + 8 * i], pv8);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const float pv = s.P2[c0 + 8 * i + u];
+                const float pv = pv8[u];
                 bf16_split(qv[u] * gv[u] * ex2(L[u] - pv), qh[u], ql[u]);
             }
             st_chunk16<true>(S[3], t, 4 * h + i, qh);
@@ -606,10 +616,12 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             ld_chunk16<true>(S[2], t, 4 * h + i, kv);
             if (QKRAW) prologue8(kv, rk);
             ld_chunk16<true>(S[3], t, 4 * h + i, ev);
+            float p8[8], e8[8];
+            lds8(&s.P2[c0 + 8 * i], p8);
+            lds8(&s.eP2[c0 + 8 * i], e8);
 #pragma unroll
             for (int u = 0; u < 8; ++u) {
-                const int j = 8 * i + u;
-                const float f = ex2(s.P2[c0 + j] - L[u]) * s.eP2[c0 + j];  // 2^(Lbar - L)
+                const float f = ex2(p8[u] - L[u]) * e8[u];  // 2^(Lbar - L)
                 kv[u] *= f;
                 ev[u] *= kv[u];
             }
