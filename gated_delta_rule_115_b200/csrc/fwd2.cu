@@ -77,7 +77,7 @@ struct IntraSmem {
     alignas(16) float P2[kD];   // pivot (log2 units)
     alignas(16) float eP2[kD];  // 2^P2
     alignas(16) float Lb[kD];   // chunk total (log2 units)
-    float lblk[4][32][33];  // strictly lower 32x32 diagonal blocks of L_A (leaf inverses)
+    alignas(16) float lblk[4][32][36];  // strictly lower 32x32 diagonal blocks of L_A (leaf inverses)
     float nrm[4][kC];   // fused prologue: per-quarter sums of SiLU(x)^2 of each row
     uint64_t bar[16];
     uint32_t tslot;
@@ -385,9 +385,12 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         {
             float la[32];
             tm_ld32w(tm, q, c0, la);
-            if (leaf) {
+            if (leaf) {  // row lane of the block (rows 144 bytes apart: 16-byte stores without conflicts)
 #pragma unroll
-                for (int k = 0; k < 32; ++k) s.lblk[q][lane][k] = (k < lane) ? la[k] : 0.f;
+                for (int k = 0; k < 32; k += 4)
+                    *reinterpret_cast<float4*>(&s.lblk[q][lane][k]) =
+                        make_float4(k < lane ? la[k] : 0.f, k + 1 < lane ? la[k + 1] : 0.f,
+                                    k + 2 < lane ? la[k + 2] : 0.f, k + 3 < lane ? la[k + 3] : 0.f);
             }
 #pragma unroll
             for (int j = 0; j < 32; ++j)
@@ -409,7 +412,13 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             for (int r = 0; r < 32; ++r) {
                 float acc = (r == lane) ? 1.f : 0.f;
 #pragma unroll
-                for (int k = 0; k < r; ++k) acc -= s.lblk[q][r][k] * tcol[k];
+                for (int k4 = 0; k4 < r; k4 += 4) {  // row r of L, four entries per (broadcast) load
+                    const float4 l4 = *reinterpret_cast<const float4*>(&s.lblk[q][r][k4]);
+                    const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        if (k4 + u < r) acc -= lv[u] * tcol[k4 + u];
+                }
                 tcol[r] = acc;
             }
             const int col = c0 + lane;
