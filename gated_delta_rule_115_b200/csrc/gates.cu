@@ -355,6 +355,7 @@ __global__ void __launch_bounds__(128, 1) k2_gates_dw(const __grid_constant__ Ga
     __shared__ uint64_t barL[2], barM;
     __shared__ uint32_t tslot;
     __shared__ int bad;
+    __shared__ __align__(16) float red[8][128];  // dbias partials of the eight row groups
     const int tid = threadIdx.x, warp = tid >> 5;
     const int X = blockIdx.x / p.H, h = blockIdx.x % p.H, r = p.r[X];
     if (tid == 0) {
@@ -382,7 +383,9 @@ __global__ void __launch_bounds__(128, 1) k2_gates_dw(const __grid_constant__ Ga
         load(0);
         if (p.ntile > 1) load(1);
     }
-    float colsum = 0.f;
+    // dbias: thread (8-channel chunk ch, row group rg) sums its 16 rows of every tile
+    const int ch = tid & 15, rg = tid >> 4;
+    float acc8[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     for (int j = 0; j < p.ntile; ++j) {
         const int s = j & 1;
         unsigned char* base = sm + 6 * s * kBlk;
@@ -392,19 +395,23 @@ __global__ void __launch_bounds__(128, 1) k2_gates_dw(const __grid_constant__ Ga
             gemm_mm16(tm, saddr(base + 2 * kBlk), 0, 0, saddr(base + 4 * kBlk), 0, 0, r, 128, kBF16, true);
             mma_commit(&barM);
         }
-        {  // column c of the dpre tile (hi + lo)
-            const int c = tid;
-            float acc = 0.f;
-            for (int row = 0; row < 128; ++row) {
-                const uint32_t o = t16_off(row, c >> 3) + (c & 7) * 2;
-                acc += __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + o)) +
-                       __bfloat162float(*reinterpret_cast<const __nv_bfloat16*>(base + 2 * kBlk + o));
-            }
-            colsum += acc;
+#pragma unroll 4
+        for (int i = 0; i < 16; ++i) {  // rows 16 rg .. +16, channels 8 ch .. +8 (hi + lo)
+            float a[8], b[8];
+            ld_chunk16<true>(base, 16 * rg + i, ch, a);
+            ld_chunk16<true>(base + 2 * kBlk, 16 * rg + i, ch, b);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) acc8[u] += a[u] + b[u];
         }
         if (!cta_wait(&barM, (uint32_t)(j & 1)) && tid == 0) bad = 1;
         if (tid == 0 && j + 2 < p.ntile) load(j + 2);  // stage s consumed by the product and the sums
     }
+    *reinterpret_cast<float4*>(&red[rg][8 * ch]) = make_float4(acc8[0], acc8[1], acc8[2], acc8[3]);
+    *reinterpret_cast<float4*>(&red[rg][8 * ch + 4]) = make_float4(acc8[4], acc8[5], acc8[6], acc8[7]);
+    __syncthreads();
+    float colsum = 0.f;
+#pragma unroll
+    for (int g = 0; g < 8; ++g) colsum += red[g][tid];  // fixed order
     {
         const int c = tid;
         float* dU = p.dU[X] + 128 * h + c;  // dU[i][128 h + c]
