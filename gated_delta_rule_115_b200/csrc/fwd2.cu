@@ -502,10 +502,10 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         }
         fence_async_smem();
         sync_all();
-        if (ax && tid == 0) {  // U (S4) is final; L_K (S1) is overwritten below
+        if (ax && tid == 0) {  // U (S4) is final; L_K's record has left S1 (overwritten below)
+            bulk_wait_read();
             bulk_store(ax + AuxLayout::kU16, S[4], kT16Bytes);
             bulk_commit();
-            bulk_wait_read();
         }
         if (tid == 0) {
             gemm_km16(tm + 0, a1, 0, a4, 0, 0, 128, 128, kF16, false);  // L_K U
@@ -566,7 +566,6 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             gemm_km16(tm + 256, a5, 0, a0, 0, 0, 256, 128, kF16, false, true);
             gemm_km16(tm + 384, a3, 0, a4, 0, 0, 128, 128, kF16, true);
             mma_commit(&s.bar[BM5]);
-            if (ax) bulk_wait_read();  // M_QK (S3), M_QA (S5) stored
         }
         // q and gamma of row t for Q~, requested while the products run
         uint4 qraw[4], graw[4];
@@ -583,6 +582,7 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
         waitb(s, BM5, ph);
         tc_fence_after();
         if (tid == 0) {
+            if (ax) bulk_wait_read();                      // M_QK's record has left S3
             mbar_arrive_expect_tx(&s.bar[BF], kT16Bytes);  // e -> S3
             load_tile(S[3], &p.te, y, z, BF);
         }
