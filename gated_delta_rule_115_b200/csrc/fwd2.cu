@@ -820,6 +820,7 @@ __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutPara
     unsigned char* Qt = sm;
     unsigned char* St = sm + MT;
     unsigned char* Ot = sm + 2 * MT;  // bf16 output tile (T16 layout)
+    unsigned char* Ss = Ot + kT16Bytes;  // S_n by TMA: four 128-byte-swizzled boxes of 32 columns
     __shared__ uint64_t bar[2];
     __shared__ uint32_t tslot;
     __shared__ int bad;
@@ -827,38 +828,46 @@ __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutPara
     const int q = warp & 3, h = warp >> 2, t = 32 * q + lane;
     const int N = p.T / kC, nch = p.B * p.H * N;
     if (tid == 0) {
+        mbar_init(&bar[0], 1);
         mbar_init(&bar[1], 1);
         bad = 0;
         fence_barrier_init();
+        prefetch_tmap(&p.tS);
     }
     if (warp == 0) tmem_alloc(&tslot, 128);
     sync_all();
     const uint32_t tm = tslot;
+    auto issue_S = [&](int cc) {
+        mbar_arrive_expect_tx(&bar[0], MT);
+        for (int kb = 0; kb < 4; ++kb)
+            tma_load_3d(Ss + kb * 128 * 128, &p.tS, 32 * kb, cc * kD, 0, &bar[0]);
+    };
+    if (tid == 0 && (int)blockIdx.x < nch) issue_S(blockIdx.x);
     int it = 0;
     for (int c = blockIdx.x; c < nch; c += gridDim.x, ++it) {
         if (tid == 32) {  // the next chunk's blocks -> L2
             const int cn = c + gridDim.x;
             if (cn < nch) {
                 bulk_prefetch_l2(p.Qp + (size_t)cn * kC * kD, kC * kD * 4);
-                bulk_prefetch_l2(p.S_chunks + (size_t)cn * kD * kD, kD * kD * 4);
                 bulk_prefetch_l2(p.Oi + (size_t)cn * kC * kD, kC * kD * 4);
             }
         }
         // Q'_n into Qt: thread (row tid % 128, every other 4-column group) from
-        // the group-major block; S_n^T into St: thread (row r = tid / 2, half)
-        // reads 64 values of S_n row r.  All 32 loads are issued before the
-        // first store, so that their latencies overlap.
+        // the group-major block, its loads issued before the wait for S_n;
+        // S_n^T into St: thread (row r = tid / 2, half) reads 64 values of S_n
+        // row r from the TMA boxes.
         {
             const float* qb = p.Qp + (size_t)c * kC * kD;
             const int rq = tid & 127, g0 = tid >> 7;
             const int r = tid >> 1, hf = tid & 1;
-            const float* src = p.S_chunks + (size_t)c * kD * kD + (size_t)r * kD + 64 * hf;
             float4 qv[16], sv[16];
 #pragma unroll
-            for (int k = 0; k < 16; ++k) {
-                qv[k] = __ldg(grp4(qb, rq, 4 * (g0 + 2 * k)));
-                sv[k] = __ldg(reinterpret_cast<const float4*>(src + 4 * k));
-            }
+            for (int k = 0; k < 16; ++k) qv[k] = __ldg(grp4(qb, rq, 4 * (g0 + 2 * k)));
+            if (!cta_wait(&bar[0], (uint32_t)(it & 1)) && tid == 0) bad = 1;
+#pragma unroll
+            for (int k = 0; k < 16; ++k)  // columns 64 hf + 4k .. +4: box 2 hf + k / 8, chunk k % 8
+                sv[k] = *reinterpret_cast<const float4*>(Ss + (2 * hf + (k >> 3)) * 128 * 128 + r * 128 +
+                                                         (((k & 7) ^ (r & 7)) << 4));
 #pragma unroll
             for (int k = 0; k < 16; ++k) {
                 const int g = g0 + 2 * k;
@@ -879,6 +888,7 @@ __global__ void __launch_bounds__(256, 1) k2_out(const __grid_constant__ OutPara
         if (tid == 0) {
             gemm_kk32<128, 128>(tm, saddr(Qt), saddr(St), 0, 128, 128, false);
             mma_commit(&bar[1]);
+            if (c + (int)gridDim.x < nch) issue_S(c + gridDim.x);  // Ss read out above
             bulk_wait_read();  // the previous chunk's o tile has left Ot (the barrier below tells the rest)
         }
         float4 oa[16];  // O_intra row t, columns 64 h .. +64, loaded while the product runs
@@ -1011,7 +1021,7 @@ static int sm_count() {
 }
 
 constexpr int kIntraSmem = 6 * kT16Bytes + sizeof(IntraSmem) + 1024;
-constexpr int kOutSmem = 2 * 128 * 128 * 4 + kT16Bytes + 1024;
+constexpr int kOutSmem = 3 * 128 * 128 * 4 + kT16Bytes + 1024;
 template <int SLAB>
 constexpr int chain_smem() { return 3 * 128 * 128 * 4 + SLAB * 512 + 1024; }
 
@@ -1072,6 +1082,7 @@ cudaError_t run_fwd2(const Fwd2Args& a, cudaStream_t st) {
         OutParams op;
         op.B = a.B; op.T = a.T; op.H = a.H;
         op.Qp = a.Qp; op.S_chunks = a.S_chunks; op.Oi = a.Oi; op.o = a.o;
+        if (!map_rows32f(&op.tS, a.S_chunks, (long long)nch * kD)) return cudaErrorInvalidValue;
         op.zo = a.zo; op.o_pre = a.zo ? a.o_pre : nullptr;
         if (a.out_bf16) {
             if (!map_tokens16(&op.to, a.o, a.B, a.T, a.H)) return cudaErrorInvalidValue;

@@ -80,6 +80,7 @@ struct ChainParams {
 
 struct OutParams {
     CUtensorMap to;      // o as token-major bf16 tiles (bf16 output only)
+    CUtensorMap tS;      // S_n rows of 128 fp32
     int B, T, H;
     const float* Qp;     // Q' (grp4 layout)
     const float* S_chunks;
