@@ -796,7 +796,7 @@ struct Bwd2Smem {
     uint32_t tslot;
     int bad;
 };
-enum { B2IN = 0, B2M, B2G, B2X };
+enum { B2IN = 0, B2M, B2G, B2X, B2Q };
 // which part of a dL product survives, for row r and column col:
 // col < r, col <= r, col > r, col >= r
 enum { kStrictLow = 0, kInclLow, kStrictUp, kInclUp };
@@ -1029,8 +1029,6 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 if (far) atomicOr(p.flags, 1);
             }
             __syncthreads();
-            const __nv_bfloat16* qin = reinterpret_cast<const __nv_bfloat16*>(p.q) + tok * kD + j0;
-            const __nv_bfloat16* gin_ = reinterpret_cast<const __nv_bfloat16*>(p.gamma) + tok * kD + j0;
             {  // Am -> Bt0, Km -> Bt1
                 float kv[16], ev[16], am[16], km[16];
                 ld_chunk16<true>(Kt, t, 2 * g4, kv); ld_chunk16<true>(Kt, t, 2 * g4 + 1, kv + 8);
@@ -1054,23 +1052,25 @@ float p16[16];
             //  R3: dL_A^T = -Y dYR^T (strict upper), dM_QA^T = -Y dO^T (inclusive upper) -> dAm
             //  R4: dL_K^T = U dYR^T (strict upper), dM_QK^T = U dO^T (inclusive upper) -> dKm
             // with Am, Km in Bt0, Bt1 for R1, R2 and Kp, Qp for R3, R4.
-            // q and gamma of the row for R3's operands, requested two rounds ahead
-            uint4 qg[4];
-            qg[0] = __ldg(reinterpret_cast<const uint4*>(qin));
-            qg[1] = __ldg(reinterpret_cast<const uint4*>(qin + 8));
-            qg[2] = __ldg(reinterpret_cast<const uint4*>(gin_));
-            qg[3] = __ldg(reinterpret_cast<const uint4*>(gin_ + 8));
 #pragma unroll 1
             for (int r = 0; r < 4; ++r) {
-                if (r == 2) {  // Kp -> Bt0, Qp -> Bt1
+                if (r == 2) {  // Kp -> Bt0, Qp -> Bt1; q and gamma of the half come by TMA into Bt1 first
+                    if (tid == 0) {
+                        const int z = b * p.T + n * kC;
+                        mbar_arrive_expect_tx(&s.bar[B2Q], 2 * kT16Block);
+                        tma_load_3d(Bt1, &p.tq, 64 * hj, hd, z, &s.bar[B2Q]);
+                        tma_load_3d(Bt1 + kT16Block, &p.tgam, 64 * hj, hd, z, &s.bar[B2Q]);
+                    }
                     float kv[16], qv[16], gv[16], kp[16], qp[16];
                     ld_chunk16<true>(Kt, t, 2 * g4, kv); ld_chunk16<true>(Kt, t, 2 * g4 + 1, kv + 8);
-                    unpack8_bf16(qg[0], qv); unpack8_bf16(qg[1], qv + 8);
+                    if (!cta_wait(&s.bar[B2Q], (uint32_t)hj) && tid == 0) atomicOr(&s.bad, 1 << 29);
+                    ld_chunk16<true>(Bt1, t, 2 * g4, qv); ld_chunk16<true>(Bt1, t, 2 * g4 + 1, qv + 8);
+                    ld_chunk16<true>(Bt1, t, 8 + 2 * g4, gv); ld_chunk16<true>(Bt1, t, 9 + 2 * g4, gv + 8);
+                    __syncthreads();  // every thread has its q, gamma before Qp overwrites Bt1
                     if (QKRAW) {
                         prologue8(kv, rk); prologue8(kv + 8, rk);
                         prologue8(qv, rq); prologue8(qv + 8, rq);
                     }
-                    unpack8_bf16(qg[2], gv); unpack8_bf16(qg[3], gv + 8);
                     float p16[16];
                     lds8(&s.P2[j0], p16); lds8(&s.P2[j0 + 8], p16 + 8);
 #pragma unroll
