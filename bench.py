@@ -58,9 +58,9 @@ DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 6 * 128 * 2 + 128 * 2  # S read+writ
 # keyed by kernel; valid only while the chunk-kernel source hash matches.
 NCU_TRAFFIC = {
     # ncu --set full of one k2_bwd2 launch at B=1 H=16 T=8192 (131,072 token-heads):
-    # 474.3 MB read + 153.5 MB written; traffic scales with the chunks processed
-    "k2_bwd2": {"bytes_per_token_head": (474.266624e6 + 153.491968e6) / 131072,
-                "source": "105eaf8bd03d04f8"},
+    # 473.5 MB read + 152.7 MB written; traffic scales with the chunks processed
+    "k2_bwd2": {"bytes_per_token_head": (473.458944e6 + 152.689152e6) / 131072,
+                "source": "1bdfd05c90e4a404"},
 }
 
 
