@@ -28,9 +28,9 @@
 // (dY, dYR, dU -> dv, dw; the state-side terms; Y and dYR for k2_bwd2),
 // k2_bwd2 (the decay-masked gradients in TF32 with the dL matrices as
 // tensor-memory operands, one 64-channel half at a time; final dq, dk, dg, de,
-// dgamma).  Precision: products with a state (S, G) use bf16 operands, the
-// bounded-range products fp16, the decay-masked gradients TF32; fp32
-// accumulation throughout.
+// dgamma).  Precision: products with a state (S, G) use fp16 operands with a
+// power-of-two scale per chunk, the bounded-range products fp16, the
+// decay-masked gradients TF32; fp32 accumulation throughout.
 #include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>

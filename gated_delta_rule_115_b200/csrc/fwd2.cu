@@ -265,7 +265,7 @@ __global__ void __launch_bounds__(512, 1) k2_intra(const __grid_constant__ Intra
             bulk_wait_read();
             load_tile(S[4], &p.tgam, y, z, BB);
         }
-        // ---- 1. log-decay prefix (warp scan over tokens), pivots
+        // ---- 1. log-decay prefix, pivots
         // L = Tril(1) g: the inclusive prefix over the chunk's tokens as one
         // tensor-core product (clamped g and the ones are exact in bf16; fp32
         // accumulation), the ones tile in S5 (free until phase 2)

@@ -10,7 +10,8 @@ namespace muir {
 namespace v2 {
 
 // Per-chunk fp32 arrays are indexed by chunk c = (b * H + h) * N + n, each
-// chunk a row-major 128 x 128 block.
+// chunk a 128 x 128 block: row-major, or 4-column-group-major where a field
+// says grp4 (tc2.cuh).
 
 // Per-chunk intermediates the forward saves for the backward ("aux"), byte
 // offsets inside one chunk's record.  16-bit tiles are stored byte for byte in
