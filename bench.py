@@ -58,9 +58,9 @@ DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 6 * 128 * 2 + 128 * 2  # S read+writ
 # keyed by kernel; valid only while the chunk-kernel source hash matches.
 NCU_TRAFFIC = {
     # ncu --set full of one k2_bwd2 launch at B=1 H=16 T=8192 (131,072 token-heads):
-    # 473.5 MB read + 152.7 MB written; traffic scales with the chunks processed
-    "k2_bwd2": {"bytes_per_token_head": (473.458944e6 + 152.689152e6) / 131072,
-                "source": "1bdfd05c90e4a404"},
+    # 475.2 MB read + 153.4 MB written; traffic scales with the chunks processed
+    "k2_bwd2": {"bytes_per_token_head": (475.151616e6 + 153.384704e6) / 131072,
+                "source": "74c642fe6d855d43"},
 }
 
 
