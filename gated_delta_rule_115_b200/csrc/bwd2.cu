@@ -888,18 +888,24 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
         for (int u = 0; u < 16; ++u)
             *reinterpret_cast<float*>(tile + t32_off<64>(r0 + u, t >> 2) + (t & 3) * 4) = tf32_round(v[u]);
     };
-    auto round_ = [&](uint32_t ax0, uint32_t bx0, bool negx, uint32_t ax1, uint32_t bx1, bool negy,
-                      int mode0, int mode1, int acc_col) {
-        if (tid == 0) {
-            gemm_kk16(tm + 0, ax0, 0, bx0, 0, 0, 128, 128, kF16, false, negx);
-            gemm_kk16(tm + 128, ax1, 0, bx1, 0, 0, 128, 128, kF16, false, negy);
-            mma_commit(&s.bar[B2M]);
-        }
+    // Round r in two parts.  The first (thread 0) issues its two dL products
+    // into TMEM columns 0..255; they read only the four chunk tiles, so they
+    // run while the threads form the round's pivoted operand tiles.  The
+    // second masks them and accumulates the TF32 pair.
+    auto round_issue = [&](int r) {
+        const uint32_t ax = r == 0 ? aR : r == 1 ? aO : r == 2 ? aY : aU;
+        const uint32_t bx0 = r < 2 ? aY : aR, bx1 = r < 2 ? aU : aO;
+        gemm_kk16(tm + 0, ax, 0, bx0, 0, 0, 128, 128, kF16, false, r != 3);
+        gemm_kk16(tm + 128, ax, 0, bx1, 0, 0, 128, 128, kF16, false, r == 2);
+        mma_commit(&s.bar[B2M]);
+    };
+    auto round_finish = [&](int r) {
         mma_wait();
-        mask_rows(mode0, mode1);
-        sync_all();
+        mask_rows(r == 0 ? kStrictLow : r == 1 ? kInclLow : kStrictUp,
+                  r == 0 ? kStrictLow : r == 1 ? kInclLow : kInclUp);
+        sync_all();  // the masks, and the operand tiles' generic writes (fenced by their writers)
         if (tid == 0) {
-            acc_pair(acc_col);
+            acc_pair(256 + 64 * r);
             mma_commit(&s.bar[B2M]);
         }
         mma_wait();
@@ -1028,7 +1034,8 @@ __global__ void __launch_bounds__(512, 1) k2_bwd2(const __grid_constant__ Bwd2Pa
                 // path, which overwrites this kernel's results)
                 if (far) atomicOr(p.flags, 1);
             }
-            __syncthreads();
+            sync_all();  // every row's L has left TMEM columns 0..63
+            if (tid == 0) round_issue(0);
             {  // Am -> Bt0, Km -> Bt1
                 float kv[16], ev[16], am[16], km[16];
                 ld_chunk16<true>(Kt, t, 2 * g4, kv); ld_chunk16<true>(Kt, t, 2 * g4 + 1, kv + 8);
@@ -1045,7 +1052,6 @@ float p16[16];
                 put_t(Bt1, r0, km);
             }
             fence_async_smem();
-            sync_all();
             // Four rounds (one loop, so that their code is issued once):
             //  R1: dL_A = -dYR Y^T, dL_K = dYR U^T (strict) -> dKp = dL_A Am + dL_K Km
             //  R2: dM_QA = -dO Y^T, dM_QK = dO U^T (inclusive) -> dQp = dM_QA Am + dM_QK Km
@@ -1060,6 +1066,7 @@ float p16[16];
                         mbar_arrive_expect_tx(&s.bar[B2Q], 2 * kT16Block);
                         tma_load_3d(Bt1, &p.tq, 64 * hj, hd, z, &s.bar[B2Q]);
                         tma_load_3d(Bt1 + kT16Block, &p.tgam, 64 * hj, hd, z, &s.bar[B2Q]);
+                        round_issue(2);
                     }
                     float kv[16], qv[16], gv[16], kp[16], qp[16];
                     ld_chunk16<true>(Kt, t, 2 * g4, kv); ld_chunk16<true>(Kt, t, 2 * g4 + 1, kv + 8);
@@ -1082,13 +1089,10 @@ float p16[16];
                     put_t(Bt0, r0, kp);
                     put_t(Bt1, r0, qp);
                     fence_async_smem();
-                    sync_all();
+                } else if (r != 0 && tid == 0) {
+                    round_issue(r);
                 }
-                const uint32_t ax = r == 0 ? aR : r == 1 ? aO : r == 2 ? aY : aU;
-                const uint32_t bx0 = r < 2 ? aY : aR, bx1 = r < 2 ? aU : aO;
-                const int mode0 = r == 0 ? kStrictLow : r == 1 ? kInclLow : kStrictUp;
-                const int mode1 = r == 0 ? kStrictLow : r == 1 ? kInclLow : kInclUp;
-                round_(ax, bx0, r != 3, ax, bx1, r == 2, mode0, mode1, 256 + 64 * r);
+                round_finish(r);
             }
             // the second half's rounds were the tiles' last readers
             if (hj == 1 && tid == 0 && c + (int)gridDim.x < nch) load_tiles(c + gridDim.x);
