@@ -1094,10 +1094,6 @@ float p16[16];
                 }
                 round_finish(r);
             }
-            // the second half's rounds were the tiles' last readers
-            if (hj == 1 && tid == 0 && c + (int)gridDim.x < nch) load_tiles(c + gridDim.x);
-            if (hj == 1 && tid < 4 * p.nslab && c + (int)gridDim.x < nch)  // the next chunk's dLbar partials -> L2
-                prefetch_l2(p.dgb + ((size_t)(tid >> 2) * nch + c + gridDim.x) * kD + 32 * (tid & 3));
             // ---- readout: final gradients of channels j0 .. j0 + 15 of row t.
             // e (Bt0) and q, gamma (Bt1) of the half come by TMA into the
             // operand tiles, free now (k has its own tile); each thread forms
@@ -1109,7 +1105,12 @@ float p16[16];
                 tma_load_3d(Bt0 + kT16Block, &p.te, 64 * hj, hd, z, &s.bar[B2X]);
                 tma_load_3d(Bt1, &p.tq, 64 * hj, hd, z, &s.bar[B2X]);
                 tma_load_3d(Bt1 + kT16Block, &p.tgam, 64 * hj, hd, z, &s.bar[B2X]);
+                // the second half's rounds were the tiles' last readers; the next
+                // chunk's tiles queue behind the readout's inputs
+                if (hj == 1 && c + (int)gridDim.x < nch) load_tiles(c + gridDim.x);
             }
+            if (hj == 1 && tid < 4 * p.nslab && c + (int)gridDim.x < nch)  // the next chunk's dLbar partials -> L2
+                prefetch_l2(p.dgb + ((size_t)(tid >> 2) * nch + c + gridDim.x) * kD + 32 * (tid & 3));
             {
                 const size_t scb = psc(c, t, j0);  // channels j0 .. +16 share a group
                 const float s_q = __ldg(p.sq + scb), s_k = __ldg(p.sk + scb);
