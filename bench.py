@@ -58,9 +58,9 @@ DECODE_BYTES_PER_HEAD = 2 * 128 * 128 * 4 + 6 * 128 * 2 + 128 * 2  # S read+writ
 # keyed by kernel; valid only while the chunk-kernel source hash matches.
 NCU_TRAFFIC = {
     # ncu --set full of one k2_bwd2 launch at B=1 H=16 T=8192 (131,072 token-heads):
-    # 475.2 MB read + 153.4 MB written; traffic scales with the chunks processed
-    "k2_bwd2": {"bytes_per_token_head": (475.151616e6 + 153.384704e6) / 131072,
-                "source": "74c642fe6d855d43"},
+    # 476.6 MB read + 154.5 MB written; traffic scales with the chunks processed
+    "k2_bwd2": {"bytes_per_token_head": (476.6144e6 + 154.4576e6) / 131072,
+                "source": "3028ae8d4b2a9580"},
 }
 
 
