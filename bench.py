@@ -29,6 +29,7 @@ import statistics
 import subprocess
 import sys
 import tempfile
+import threading
 import time
 
 ROOT = os.path.dirname(os.path.abspath(__file__))
@@ -200,7 +201,76 @@ class ClockSampler:
         rows = [r.strip().split(",") for r in self.f.read().strip().splitlines() if r.strip()]
         self.f.close()
         os.unlink(self.f.name)
-        return summarize_clocks(rows)
+        out = summarize_clocks(rows)
+        out["sampler"] = "nvidia-smi, 200 ms"
+        return out
+
+
+class NvmlClockSampler:
+    """In-process NVML reads every ``period`` seconds on a background thread
+    while the timed region runs, so that a region of a few hundred
+    milliseconds still gets several samples.  Only queries: no clock, limit or
+    mode of the GPU is changed.  Rows take the nvidia-smi sampler's form."""
+
+    # NVML clock-event reason bits, in the order summarize_clocks reads them
+    REASONS = (("hw_slowdown", 0x8), ("hw_thermal_slowdown", 0x40),
+               ("sw_thermal_slowdown", 0x20), ("sw_power_cap", 0x4))
+
+    def __init__(self, gpu_id: str, nvml=None, period: float = 0.01):
+        if nvml is None:
+            import pynvml as nvml
+        self.nvml = nvml
+        nvml.nvmlInit()
+        try:
+            self.h = (nvml.nvmlDeviceGetHandleByUUID(gpu_id) if gpu_id
+                      else nvml.nvmlDeviceGetHandleByIndex(0))
+            self.max_mhz = nvml.nvmlDeviceGetMaxClockInfo(self.h, nvml.NVML_CLOCK_SM)
+            self.reasons = (getattr(nvml, "nvmlDeviceGetCurrentClocksEventReasons", None)
+                            or nvml.nvmlDeviceGetCurrentClocksThrottleReasons)
+            self.rows = []
+            self._sample()  # a query that fails, fails here rather than in the thread
+        except Exception:
+            nvml.nvmlShutdown()
+            raise
+        self.rows = []  # (that sample precedes the region)
+        self.period = period
+        self.done = threading.Event()
+        self.thread = threading.Thread(target=self._run, daemon=True)
+        self.thread.start()
+
+    def _sample(self):
+        n = self.nvml
+        sm = n.nvmlDeviceGetClockInfo(self.h, n.NVML_CLOCK_SM)
+        watts = n.nvmlDeviceGetPowerUsage(self.h) / 1000.0
+        mask = int(self.reasons(self.h))
+        flags = ["Active" if mask & bit else "Not Active" for _, bit in self.REASONS]
+        self.rows.append([str(sm), str(self.max_mhz), "%.1f" % watts, hex(mask)] + flags)
+
+    def _run(self):
+        while not self.done.wait(self.period):
+            try:
+                self._sample()
+            except Exception:
+                return
+
+    def stop(self) -> dict:
+        self.done.set()
+        self.thread.join(timeout=5)
+        try:
+            self.nvml.nvmlShutdown()
+        except Exception:
+            pass
+        out = summarize_clocks(list(self.rows))
+        out["sampler"] = "nvml, %d ms" % round(self.period * 1e3)
+        return out
+
+
+def clock_sampler(gpu_id: str):
+    """The NVML sampler, or nvidia-smi's where NVML cannot be read."""
+    try:
+        return NvmlClockSampler(gpu_id)
+    except Exception:
+        return ClockSampler(gpu_id)
 
 
 def summarize_clocks(rows) -> dict:
@@ -338,7 +408,7 @@ def gpu_arm(args, rank, world, local):
 
         def start():
             nonlocal sampler
-            sampler = ClockSampler(gpu_id)
+            sampler = clock_sampler(gpu_id)
             L.muir_profile_reset()
             L.muir_profile_enable(1)
             e0.record(st)

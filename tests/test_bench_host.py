@@ -38,6 +38,52 @@ def test_summarize_clocks():
     assert bench.summarize_clocks([])["samples"] == 0
 
 
+class _FakeNvml:
+    """Stands in for pynvml: answers the read-only queries the sampler makes."""
+    NVML_CLOCK_SM = 1
+
+    def __init__(self, clocks, mask):
+        self.clocks, self.mask, self.calls, self.shut = list(clocks), mask, 0, False
+
+    def nvmlInit(self):
+        pass
+
+    def nvmlShutdown(self):
+        self.shut = True
+
+    def nvmlDeviceGetHandleByUUID(self, uuid):
+        assert uuid.startswith("GPU-")
+        return "h"
+
+    def nvmlDeviceGetMaxClockInfo(self, h, kind):
+        return 1965
+
+    def nvmlDeviceGetClockInfo(self, h, kind):
+        self.calls += 1
+        return self.clocks[min(self.calls - 1, len(self.clocks) - 1)]
+
+    def nvmlDeviceGetPowerUsage(self, h):
+        return 950000
+
+    def nvmlDeviceGetCurrentClocksEventReasons(self, h):
+        return self.mask
+
+
+def test_nvml_clock_sampler_reads_clocks_and_reasons():
+    import time
+    fake = _FakeNvml([1000, 1965, 1965, 1965, 1965], mask=0x4)
+    s = bench.NvmlClockSampler("GPU-0000", nvml=fake, period=0.002)
+    time.sleep(0.05)
+    c = s.stop()
+    assert fake.shut and c["samples"] >= 3
+    assert c["sm_mhz"] == 1965 and c["sm_max_mhz"] == 1965  # the pre-region sample is dropped
+    assert c["reasons"] == ["sw_power_cap"] and c["sampler"].startswith("nvml")
+    fake = _FakeNvml([1965], mask=0x8 | 0x40)
+    s = bench.NvmlClockSampler("GPU-0000", nvml=fake, period=0.002)
+    time.sleep(0.02)
+    assert s.stop()["reasons"] == ["hw_slowdown", "hw_thermal_slowdown"]
+
+
 def test_roofline_picks_the_binding_bound():
     peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1600.0, "bf16_tflops_sustained": 1400.0,
              "source": "measured"}
